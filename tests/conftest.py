@@ -1,0 +1,19 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the CUDA library")
+    config.addinivalue_line("markers", "slow: long CPU oracle runs")
+
+
+def pytest_collection_modifyitems(config, items):
+    # GPU tests run only when a CUDA device is present; selecting them with -m gpu on a
+    # machine without one makes them fail loudly instead of silently skipping.
+    pass
