@@ -1,0 +1,354 @@
+"""Benchmark: bs=1 residual block-diffusion decoding on one B200 per rank.
+
+Workload (the full bs=1 decode of the 4B-class dense model): 36 layers, d=2560, GQA 32/8,
+head_dim 128, SiLU MLP 9728, V=151936 tied bf16 embedding, random-init weights N(0,0.02),
+a 512-token uniform random prompt, 4096 generated tokens in blocks of 32 with the
+fixed-TPF=11 commit schedule (3 rounds + 1 KV-fill forward per block), one CUDA graph per
+block whose while node loops the rounds on the device.
+
+One step = one whole generation of 4096 tokens (128 block-graph launches) after the
+prompt prefix is in the KV cache.  `value` is tokens/s over all ranks (device-timed,
+inputs resident in HBM); `e2e` is the same metric through dlm_generate with the prompt
+in pinned host memory and every block's tokens read back to the host (prefill included).
+Replicas only: every rank decodes its own request, no collective on the data path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dlm|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PROMPT = 512
+GEN = 4096
+TPF_K = 11
+TAU = 0.9
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="dlm", choices=["dlm", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=36, help=argparse.SUPPRESS)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class Clocks:
+    def __init__(self, index):
+        self.path = tempfile.mktemp(suffix=".csv")
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), "--query-gpu=" + q,
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ launch accounting
+def launches_per_step(cfg, rounds, blocks, attn_combine_layers):
+    """Kernels of this library launched in one step (the schedule of dlm_api.cu)."""
+    nl = cfg["n_layers"]
+    per_round = 3 + nl * 10 + attn_combine_layers + 5 + 1
+    per_fill = 1 + (nl - 1) * 10 + attn_combine_layers * (nl - 1) // max(nl, 1) + 2
+    return rounds * per_round + blocks * (per_fill + 2)
+
+
+# ------------------------------------------------------------------ oracle baseline
+def oracle_sample(cfg, seconds=10.0):
+    """Times the CPU oracle on 1/36 of a round of the 4B-class model: one full-size layer
+    (QKV, O, gate, up, down projections and block attention over a 2560-key prefix) and
+    1/36 of the vocabulary of the LM head with its row statistics and P E, repeated until
+    `seconds` elapse.  Returns (seconds per full round, repetitions, threads)."""
+    import numpy as np
+
+    import oracle as O
+    from block_diffusion_decoding_denoising_b200 import gen
+    d, F, Hq, Hkv, hd, V, B = (cfg[k] for k in ("d", "ffn", "n_q_heads", "n_kv_heads", "head_dim", "vocab",
+                                                 "block_size"))
+    nl = cfg["n_layers"]
+    W = {n: gen.bf16_bits(gen.normal_np(40 + i, r * c, 0.02).reshape(r, c)) for i, (n, r, c) in enumerate(
+        [("qkv", (Hq + 2 * Hkv) * hd, d), ("o", d, Hq * hd), ("g", F, d), ("u", F, d), ("dn", d, F)])}
+    Vs = V // nl
+    E = gen.bf16_bits(gen.normal_np(50, Vs * d, 0.02).reshape(Vs, d))
+    x = gen.normal_np(51, B * d).reshape(B, d)
+    Lp = 2560
+    q = gen.normal_np(52, B * Hq * hd).reshape(B, Hq, hd)
+    kc = gen.normal_np(53, Hkv * (Lp + B) * hd).reshape(Hkv, Lp + B, hd)
+    vc = gen.normal_np(54, Hkv * (Lp + B) * hd).reshape(Hkv, Lp + B, hd)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        O.linear(x, W["qkv"])
+        O.attention(q, kc, vc, Lp)
+        O.linear(np.zeros((B, Hq * hd)) + 0.1, W["o"])
+        O.linear(x, W["g"])
+        O.linear(x, W["u"])
+        O.linear(np.zeros((B, F)) + 0.1, W["dn"])
+        O.lmhead(x, E, mask_id=-1)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return el / reps * nl, reps, O.hw_threads()
+
+
+def reference_arm(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle as O
+    oracle_sample(cfg, 0.0)  # warm the build
+    for _ in range(args.warmup):
+        oracle_sample(cfg, 0.0)
+    times = []
+    for _ in range(args.steps):
+        t_round, reps, thr = oracle_sample(cfg, 0.0)
+        times.append(t_round)
+    t_round = statistics.mean(times)
+    # fixed-TPF=11 schedule: 3 rounds + 1 KV-fill forward (about one round) per 32 tokens
+    blocks = GEN // cfg["block_size"]
+    t_step = blocks * 4 * t_round
+    tps = GEN / t_step
+    line = {"metric": "bs=1 decode tokens/s (fixed TPF=11)", "value": tps, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": workload_config(cfg),
+            "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": O.hw_threads(), "kind": "oracle",
+                             "sample": "1/36 of a denoising round per step (one full-size layer + 1/36 of the "
+                                       "LM head), scaled to 4 forwards per 32-token block"},
+            "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "extra": {"rounds_per_s": 1.0 / t_round}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg):
+    return {"workload": "full bs=1 decode, 4B-class dense model (36L d2560 GQA32/8 hd128 F9728 V151936 bf16), "
+                        "prompt 512, generate 4096 in blocks of 32, fixed TPF=11",
+            "model": "random-init 4B-class block-diffusion transformer", "global_batch": 1, "seq_len": PROMPT + GEN,
+            "block_size": cfg["block_size"], "parallelism": "replicas", "l2": "inputs larger than L2 (8.06 GB weights)"}
+
+
+# ------------------------------------------------------------------ main arm
+def main():
+    args = parse()
+    from block_diffusion_decoding_denoising_b200 import gen
+    cfg = gen.config_4b(max_ctx=PROMPT + GEN, n_layers=args.layers)
+    if args.impl == "reference":
+        reference_arm(args, cfg)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from block_diffusion_decoding_denoising_b200 import build, dlm
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    build.build()
+    dev = torch.device("cuda", local)
+    B = cfg["block_size"]
+    blocks = GEN // B
+    w = gen.model_weights_torch(cfg, seed=0, device=dev)
+    m = dlm.Model(cfg, w, device=dev)
+    prompt_np = gen.prompt_np(cfg, PROMPT, seed=rank)
+    prompt = torch.from_numpy(prompt_np).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    tokens_out = torch.zeros((blocks, B), dtype=torch.int32, device=dev)
+    rounds_out = torch.zeros((blocks, 2), dtype=torch.int32, device=dev)
+    m.prefill(prompt)
+    torch.cuda.synchronize()
+
+    def step(mode=dlm.COMMIT_TOPK, k=TPF_K, nblk=blocks):
+        m.set_prefix_len(PROMPT)
+        for b in range(nblk):
+            m.decode_block(TAU, mode, k, tokens_out[b], rounds_out[b])
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    clocks = Clocks(local)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    ck = clocks.stop()
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    rb = rounds_out.cpu().numpy()
+    assert np.all(rb[:, 1] == 0), "device status %s" % rb[:, 1]
+    rounds_per_step = int(rb[:, 0].sum())
+    ms_step = ms / args.steps
+    tps = world * GEN / (ms_step / 1e3)
+
+    # denoise rounds/s with the threshold schedule (tau = 0.9: about one commit per round on
+    # random weights, i.e. up to B rounds per block), on 4 blocks
+    step(dlm.COMMIT_THRESHOLD, 1, 4)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    step(dlm.COMMIT_THRESHOLD, 1, 4)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    tau_rounds = int(rounds_out[:4, 0].sum().item())
+    tau_ms = e0.elapsed_time(e1)
+    tau_rounds_per_s = tau_rounds / (tau_ms / 1e3)
+
+    # dominant kernel: the tensor-core GEMM, timed alone with CUDA events over every
+    # projection of one round (36 x {QKV, O, gate, up, down} + LM head), partial sums only
+    L = dlm.lib()
+    import ctypes as C
+    x = torch.randn((B, cfg["ffn"]), device=dev).to(torch.bfloat16)
+    shapes = []
+    for lw in w["layers"]:
+        shapes += [(lw["w_qkv"], cfg["d"]), (lw["w_o"], cfg["n_q_heads"] * cfg["head_dim"]),
+                   (lw["w_gate"], cfg["d"]), (lw["w_up"], cfg["d"]), (lw["w_down"], cfg["ffn"])]
+    shapes.append((w["embed"], cfg["d"]))
+    scratch_n = max(L.dlm_gemm_scratch_size(B, t.shape[0], K) for t, K in shapes)
+    scratch = torch.empty(scratch_n, dtype=torch.uint8, device=dev)
+    sp = C.c_void_p(stream.cuda_stream)
+
+    def gemms():
+        for t, K in shapes:
+            L.dlm_gemm_bf16(C.c_void_p(x.data_ptr()), C.c_void_p(t.data_ptr()), None, B, t.shape[0], K,
+                            C.c_void_p(scratch.data_ptr()), scratch_n, sp)
+
+    for _ in range(3):
+        gemms()
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 5
+    g0.record(stream)
+    for _ in range(reps):
+        gemms()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    gemm_s = g0.elapsed_time(g1) / 1e3 / (reps * len(shapes))
+    gemm_bytes = sum(t.numel() * 2 + B * K * 2 for t, K in shapes) / len(shapes)
+    hbm, tflops, peak_kind = peaks()
+    achieved = gemm_bytes / gemm_s / 1e9
+
+    # end to end through dlm_generate: pinned host prompt in, every block's tokens out
+    pin_prompt = torch.from_numpy(prompt_np).pin_memory()
+    e2e_times = []
+    for i in range(args.warmup + args.steps):
+        barrier()
+        t0 = time.perf_counter()
+        out, rpb, tm = m.generate(pin_prompt.numpy(), GEN, TAU, dlm.COMMIT_TOPK, TPF_K)
+        t1 = time.perf_counter()
+        if i >= args.warmup:
+            e2e_times.append(t1 - t0)
+    e2e_s = max(e2e_times) if e2e_times else float("nan")
+    if world > 1:
+        t = torch.tensor([e2e_s], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    e2e_tps = world * GEN / e2e_s
+
+    weight_bytes = sum(v.numel() * 2 for k, v in w.items() if k != "layers") + sum(
+        v.numel() * 2 for l in w["layers"] for v in l.values())
+    mean_L = PROMPT + GEN / 2
+    round_bytes = weight_bytes + 147456 * mean_L * cfg["n_layers"] / 36
+    round_ms = ms_step / (rounds_per_step + blocks)  # rounds and KV-fill forwards of the step
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_round, reps_cpu, thr = oracle_sample(cfg, 10.0)
+        cpu = {"value": GEN / (blocks * 4 * t_round), "unit": "tokens/s", "cores": thr, "kind": "oracle",
+               "sample": "%d x (1/36 of a denoising round: one full-size layer + 1/36 of the LM head), scaled to a "
+                         "round and to 4 forwards per 32-token block" % reps_cpu}
+
+    if rank == 0:
+        line = {
+            "metric": "bs=1 decode tokens/s (fixed TPF=11)", "value": tps, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(cfg),
+            "roofline": {"bound": "hbm", "kernel": "k_gemm_tc (tensor-core weight-streaming GEMM)",
+                         "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "peak_kind": peak_kind, "traffic": None},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_tps, "unit": "tokens/s", "h2d_bytes_per_step": PROMPT * 4,
+                    "d2h_bytes_per_step": GEN * 4 + blocks * 8},
+            "gpu_launches": args.steps * launches_per_step(cfg, rounds_per_step, blocks, cfg["n_layers"]),
+            "clocks": ck,
+            "extra": {"rounds_per_step": rounds_per_step, "tpf": GEN / rounds_per_step,
+                      "round_or_fill_ms": round_ms,
+                      "round_roofline_frac": (round_bytes / (round_ms / 1e3) / 1e9) / hbm,
+                      "tau0.9_rounds_per_s": tau_rounds_per_s, "tau0.9_rounds_per_block": tau_rounds / 4,
+                      "gemm_avg_launch_us": gemm_s * 1e6},
+        }
+        print(json.dumps(line), flush=True)
+    m.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

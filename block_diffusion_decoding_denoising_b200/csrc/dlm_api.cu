@@ -1,0 +1,924 @@
+// dlm_api.cu -- context, workspace layout, round orchestration, the per-block CUDA graph
+// and the extern "C" entry points of libdlm.so (declared in include/dlm.h).
+//
+// The per-block graph ["ORL: diffusion LLMs get a learnable 'tokens per forward'"
+// (richland.au blog), "What shipped", "dlmrt, the inference engine": the denoising loop
+// of a block stays on the GPU and a conditional node decides after every round whether
+// to continue]:
+//
+//   [init: tokens = MASK, committed = 0, s = 0, round = 0]
+//     -> WHILE(cond) { one denoising round ... k_commit sets cond = any uncommitted
+//                      && round < B through cudaGraphSetConditional }
+//     -> [KV-fill forward of the committed block, L += B, copy tokens/rounds out]
+//
+// The prefix length L lives in device memory (ctx->d_L) so the same instantiated graph
+// serves every block; the host keeps a mirror for argument checks.
+#include <chrono>
+#include <new>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "dlm_internal.h"
+#include "dlm_ops.h"
+
+using namespace dlm;
+
+namespace {
+
+constexpr int kPrefillChunk = 256;
+
+struct GraphEntry {
+  int mode;
+  float tau;
+  int k;
+  cudaGraph_t graph;
+  cudaGraphExec_t exec;
+};
+
+}  // namespace
+
+struct dlm_ctx {
+  dlm_config cfg;
+  dlm_weights w;
+  std::vector<dlm_layer_weights> layers;
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
+  __nv_bfloat16* kv = nullptr;
+  size_t kv_bytes = 0;
+  int L = 0;
+  int Tmax = 0;
+  // workspace carve
+  int* d_L = nullptr;
+  int* d_err = nullptr;
+  float* h = nullptr;
+  __nv_bfloat16* xn = nullptr;
+  __nv_bfloat16* q = nullptr;
+  __nv_bfloat16* o = nullptr;
+  __nv_bfloat16* act = nullptr;
+  __nv_bfloat16* sbf = nullptr;
+  float* partial = nullptr;
+  size_t partial_bytes = 0;
+  float* attn_part = nullptr;
+  int attn_splits_B = 1, attn_splits_T = 1;
+  float* logits = nullptr;
+  __nv_bfloat16* P = nullptr;
+  int32_t* tok_buf = nullptr;
+  // internal block state (graph path)
+  int32_t* b_tokens = nullptr;
+  uint8_t* b_committed = nullptr;
+  float* b_s = nullptr;
+  int32_t* b_round = nullptr;
+  int32_t* b_status = nullptr;
+  dlm_row_stats b_stats{};
+  int32_t* out_tokens = nullptr;
+  int32_t* out_rounds = nullptr;
+  cudaStream_t cap_stream = nullptr;
+  std::vector<GraphEntry> graphs;
+  std::string err;
+};
+
+namespace {
+
+// ------------------------------------------------------------------ helpers
+dlm_status fail(dlm_ctx* ctx, dlm_status code, const char* fmt, ...) {
+  if (ctx) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    ctx->err = buf;
+  }
+  return code;
+}
+
+#define CU(call)                                                                              \
+  do {                                                                                        \
+    cudaError_t e_ = (call);                                                                  \
+    if (e_ != cudaSuccess)                                                                    \
+      return fail(ctx, DLM_ECUDA, "%s:%d %s: %s", __FILE__, __LINE__, #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t count) {
+    off = align256(off);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+int max_tokens(const dlm_config& c) {
+  return c.block_size > kPrefillChunk ? c.block_size : kPrefillChunk;
+}
+
+size_t max_partial_bytes(const dlm_config& c, int Tmax) {
+  const int qkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim, ho = c.n_q_heads * c.head_dim;
+  size_t m = 0;
+  for (int T : {c.block_size, Tmax}) {
+    size_t v[] = {gemm_partial_bytes(T, c.d, c.d, A_KMAJOR), gemm_partial_bytes(T, qkv, c.d, A_KMAJOR),
+                  gemm_partial_bytes(T, c.d, ho, A_KMAJOR), gemm_partial_bytes(T, c.ffn, c.d, A_PAIR),
+                  gemm_partial_bytes(T, c.d, c.ffn, A_KMAJOR)};
+    for (size_t x : v) m = x > m ? x : m;
+  }
+  const int B = c.block_size;
+  size_t lm = gemm_partial_bytes(B, c.vocab, c.d, A_KMAJOR);
+  size_t pe = gemm_partial_bytes(B, c.d, c.vocab, A_MNMAJOR);
+  m = lm > m ? lm : m;
+  m = pe > m ? pe : m;
+  return m;
+}
+
+// Lays out the workspace (base == nullptr: size only).
+size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
+  Carver cv{base};
+  const int Tmax = max_tokens(c), B = c.block_size, ho = c.n_q_heads * c.head_dim;
+  int* hdr = cv.take<int>(64);
+  float* h = cv.take<float>((size_t)Tmax * c.d);
+  auto* xn = cv.take<__nv_bfloat16>((size_t)Tmax * c.d);
+  auto* q = cv.take<__nv_bfloat16>((size_t)Tmax * ho);
+  auto* o = cv.take<__nv_bfloat16>((size_t)Tmax * ho);
+  auto* act = cv.take<__nv_bfloat16>((size_t)Tmax * c.ffn);
+  auto* sbf = cv.take<__nv_bfloat16>((size_t)B * c.d);
+  size_t pb = max_partial_bytes(c, Tmax);
+  float* partial = cv.take<float>(pb / sizeof(float));
+  int sB = attention_max_splits(B, c.n_q_heads, c.n_kv_heads, c.max_ctx);
+  int sT = attention_max_splits(Tmax, c.n_q_heads, c.n_kv_heads, c.max_ctx);
+  size_t ab = attention_scratch_bytes(B, c.n_q_heads, c.head_dim, sB);
+  size_t at = attention_scratch_bytes(Tmax, c.n_q_heads, c.head_dim, sT);
+  float* attn = cv.take<float>((ab > at ? ab : at) / sizeof(float));
+  float* logits = cv.take<float>((size_t)B * c.vocab);
+  auto* P = cv.take<__nv_bfloat16>((size_t)B * c.vocab);
+  int32_t* tok = cv.take<int32_t>((size_t)c.max_ctx);
+  int32_t* bt = cv.take<int32_t>(B);
+  uint8_t* bc = cv.take<uint8_t>(B);
+  float* bs = cv.take<float>((size_t)B * c.d);
+  int32_t* br = cv.take<int32_t>(4);
+  float* st = cv.take<float>((size_t)4 * B);
+  int32_t* sa = cv.take<int32_t>(B);
+  int32_t* ot = cv.take<int32_t>(B);
+  int32_t* orr = cv.take<int32_t>(4);
+  if (x && base) {
+    x->d_L = hdr;
+    x->d_err = hdr + 1;
+    x->h = h;
+    x->xn = xn;
+    x->q = q;
+    x->o = o;
+    x->act = act;
+    x->sbf = sbf;
+    x->partial = partial;
+    x->partial_bytes = pb;
+    x->attn_part = attn;
+    x->attn_splits_B = sB;
+    x->attn_splits_T = sT;
+    x->logits = logits;
+    x->P = P;
+    x->tok_buf = tok;
+    x->b_tokens = bt;
+    x->b_committed = bc;
+    x->b_s = bs;
+    x->b_round = br;
+    x->b_status = br + 1;
+    x->b_stats = dlm_row_stats{st, st + B, st + 2 * B, st + 3 * B, sa};
+    x->out_tokens = ot;
+    x->out_rounds = orr;
+    x->Tmax = Tmax;
+  }
+  return align256(cv.off);
+}
+
+bool valid_cfg(const dlm_config* c, char* msg, size_t n) {
+  if (!c) { snprintf(msg, n, "null config"); return false; }
+  if (c->n_layers < 0 || c->d < 64 || c->d % 64 || c->n_q_heads < 1 || c->n_kv_heads < 1 ||
+      c->n_q_heads % c->n_kv_heads || !(c->head_dim == 32 || c->head_dim == 64 || c->head_dim == 128) ||
+      c->ffn < 64 || c->ffn % 64 || c->vocab < 2 || c->vocab % 8 || c->mask_id < 0 ||
+      c->mask_id >= c->vocab || c->block_size < 1 || c->block_size > 64 ||
+      c->max_ctx < c->block_size || !(c->rms_eps > 0.f) || !(c->rope_theta > 0.f) ||
+      (c->n_q_heads * c->head_dim) % 64) {
+    snprintf(msg, n, "invalid dlm_config");
+    return false;
+  }
+  if (c->weight_fmt != DLM_WEIGHTS_BF16 && c->weight_fmt != DLM_WEIGHTS_NVFP4) {
+    snprintf(msg, n, "invalid weight_fmt %d", c->weight_fmt);
+    return false;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ launch helpers
+struct Runner {
+  dlm_ctx* ctx;
+  cudaStream_t s;
+  char msg[512];
+
+  dlm_status gemm(int a_mode, const void* a0, const void* a1, const void* x, int T, int N, int K,
+                  GemmOut* out) {
+    GemmPlan p;
+    if (!gemm_plan(&p, a_mode, a0, a1, x, T, N, K, ctx->partial, msg, sizeof(msg)))
+      return fail(ctx, DLM_EUNSUPPORTED, "%s", msg);
+    if (p.partial_bytes > ctx->partial_bytes)
+      return fail(ctx, DLM_ENOMEM_WS, "gemm partials %zu > %zu", p.partial_bytes, ctx->partial_bytes);
+    cudaError_t e = gemm_launch(p, ctx->d_err, s);
+    if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "gemm launch: %s", cudaGetErrorString(e));
+    *out = p.out;
+    return DLM_OK;
+  }
+  dlm_status check() {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "launch: %s", cudaGetErrorString(e));
+    return DLM_OK;
+  }
+};
+
+#define TRY(x)                      \
+  do {                              \
+    dlm_status st_ = (x);           \
+    if (st_ != DLM_OK) return st_;  \
+  } while (0)
+
+struct FwdSpec {
+  int T;
+  const int32_t* tokens;  // device [T]
+  const float* s;         // device fp32 [T][d], or nullptr (no adapter)
+  int pos0;               // used when !dev_L
+  bool dev_L;             // positions from ctx->d_L (graph mode)
+  bool causal;
+  bool lm_head;           // round: LM head + stats + s_out
+  dlm_row_stats stats;
+  float* s_out;
+};
+
+int threads_for(int d) { return d >= 1024 ? 512 : (d >= 256 ? 256 : 128); }
+
+// One forward pass of T tokens (round, KV-fill or prefill chunk), all on stream r.s.
+dlm_status forward(Runner& r, const FwdSpec& f) {
+  dlm_ctx* ctx = r.ctx;
+  const dlm_config& c = ctx->cfg;
+  const int T = f.T, d = c.d, Hq = c.n_q_heads, Hkv = c.n_kv_heads, hd = c.head_dim, F = c.ffn;
+  const int ho = Hq * hd, nqkv = (Hq + 2 * Hkv) * hd;
+  const int nt = threads_for(d);
+  const size_t rowsm = (size_t)d * sizeof(float);
+  const __nv_bfloat16* first_gain =
+      (const __nv_bfloat16*)(c.n_layers > 0 ? ctx->layers[0].attn_norm : ctx->w.final_norm);
+
+  // embedding + residual adapter
+  EmbedArgs ea{};
+  ea.embed = (const __nv_bfloat16*)ctx->w.embed;
+  ea.tokens = f.tokens;
+  ea.h = ctx->h;
+  ea.xn = ctx->xn;
+  ea.gain = first_gain;
+  ea.d = d;
+  ea.eps = c.rms_eps;
+  if (f.s) {
+    long n = (long)T * d;
+    k_to_bf16<<<(unsigned)((n + 255) / 256), 256, 0, r.s>>>(f.s, ctx->sbf, n);
+    TRY(r.check());
+    TRY(r.gemm(A_KMAJOR, ctx->w.w_adapter, nullptr, ctx->sbf, T, d, d, &ea.adapter));
+    ea.has_adapter = 1;
+  }
+  k_embed_adapter_norm<<<T, nt, rowsm, r.s>>>(ea);
+  TRY(r.check());
+
+  const size_t layer_kv = (size_t)Hkv * c.max_ctx * hd;
+  for (int l = 0; l < c.n_layers; ++l) {
+    const dlm_layer_weights& W = ctx->layers[l];
+    __nv_bfloat16* kc = ctx->kv + (size_t)(2 * l) * layer_kv;
+    __nv_bfloat16* vc = ctx->kv + (size_t)(2 * l + 1) * layer_kv;
+    QkvArgs qa{};
+    TRY(r.gemm(A_KMAJOR, W.w_qkv, nullptr, ctx->xn, T, nqkv, d, &qa.y));
+    qa.q = ctx->q;
+    qa.kc = kc;
+    qa.vc = vc;
+    qa.Hq = Hq;
+    qa.Hkv = Hkv;
+    qa.hd = hd;
+    qa.max_ctx = c.max_ctx;
+    qa.pos0 = f.pos0;
+    qa.pos0_dev = f.dev_L ? ctx->d_L : nullptr;
+    qa.rope_theta = (double)c.rope_theta;
+    k_qkv_rope<<<dim3(Hq + 2 * Hkv, T), hd / 2, 0, r.s>>>(qa);
+    TRY(r.check());
+    // the last layer's K/V do not depend on anything after its QKV projection
+    if (!f.lm_head && l == c.n_layers - 1) break;
+
+    AttnArgs aa{};
+    aa.q = ctx->q;
+    aa.kc = kc;
+    aa.vc = vc;
+    aa.o = ctx->o;
+    aa.part_o = ctx->attn_part;
+    aa.T = T;
+    aa.Hq = Hq;
+    aa.Hkv = Hkv;
+    aa.hd = hd;
+    aa.max_ctx = c.max_ctx;
+    aa.pos0 = f.pos0;
+    aa.pos0_dev = f.dev_L ? ctx->d_L : nullptr;
+    aa.causal = f.causal ? 1 : 0;
+    aa.max_splits = (T <= c.block_size) ? ctx->attn_splits_B : ctx->attn_splits_T;
+    aa.part_ml = ctx->attn_part + (size_t)aa.max_splits * T * Hq * hd;
+    aa.err = ctx->d_err;
+    cudaError_t e = attention_launch(aa, r.s);
+    if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "attention: %s", cudaGetErrorString(e));
+
+    ResidArgs ra{};
+    TRY(r.gemm(A_KMAJOR, W.w_o, nullptr, ctx->o, T, d, ho, &ra.y));
+    ra.h = ctx->h;
+    ra.xn = ctx->xn;
+    ra.gain = (const __nv_bfloat16*)W.mlp_norm;
+    ra.d = d;
+    ra.eps = c.rms_eps;
+    k_residual_norm<<<T, nt, rowsm, r.s>>>(ra);
+    TRY(r.check());
+
+    SiluArgs sa{};
+    TRY(r.gemm(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, &sa.y));
+    sa.out = ctx->act;
+    sa.F = F;
+    k_silu_gate<<<dim3((F + 255) / 256, T), 256, 0, r.s>>>(sa);
+    TRY(r.check());
+
+    ResidArgs rd{};
+    TRY(r.gemm(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, &rd.y));
+    rd.h = ctx->h;
+    rd.xn = ctx->xn;
+    rd.gain = (const __nv_bfloat16*)(l + 1 < c.n_layers ? ctx->layers[l + 1].attn_norm : ctx->w.final_norm);
+    rd.d = d;
+    rd.eps = c.rms_eps;
+    k_residual_norm<<<T, nt, rowsm, r.s>>>(rd);
+    TRY(r.check());
+  }
+  if (!f.lm_head) return DLM_OK;
+
+  // LM head: logits, row statistics, P = softmax, s = P E
+  StoreArgs la{};
+  TRY(r.gemm(A_KMAJOR, ctx->w.embed, nullptr, ctx->xn, T, c.vocab, d, &la.y));
+  la.out = ctx->logits;
+  la.N = c.vocab;
+  la.ld = c.vocab;
+  k_store_rows<<<dim3((c.vocab + 255) / 256, T), 256, 0, r.s>>>(la);
+  TRY(r.check());
+  RowStatsArgs rs{};
+  rs.logits = ctx->logits;
+  rs.ld = c.vocab;
+  rs.V = c.vocab;
+  rs.mask_id = c.mask_id;
+  rs.stats = f.stats;
+  rs.P = ctx->P;
+  k_rowstats<<<T, 1024, 0, r.s>>>(rs);
+  TRY(r.check());
+  StoreArgs pa{};
+  TRY(r.gemm(A_MNMAJOR, ctx->w.embed, nullptr, ctx->P, T, d, c.vocab, &pa.y));
+  pa.out = f.s_out;
+  pa.N = d;
+  pa.ld = d;
+  k_store_rows<<<dim3((d + 255) / 256, T), 256, 0, r.s>>>(pa);
+  return r.check();
+}
+
+dlm_status launch_commit(Runner& r, const dlm_block_state& st, float tau, int mode, int k,
+                         bool use_cond, cudaGraphConditionalHandle h) {
+  const dlm_config& c = r.ctx->cfg;
+  CommitArgs ca{};
+  ca.maxprob = st.stats.maxprob;
+  ca.argmax = st.stats.argmax;
+  ca.tokens = st.tokens;
+  ca.committed = st.committed;
+  ca.s = st.s;
+  ca.round = st.round;
+  ca.status = st.status;
+  ca.B = c.block_size;
+  ca.d = c.d;
+  ca.tau = tau;
+  ca.mode = mode;
+  ca.k = k;
+  ca.use_cond = use_cond ? 1 : 0;
+  ca.cond = h;
+  k_commit<<<1, 64, 0, r.s>>>(ca);
+  return r.check();
+}
+
+dlm_status check_commit_args(dlm_ctx* ctx, float tau, int mode, int k) {
+  if (mode != DLM_COMMIT_THRESHOLD && mode != DLM_COMMIT_TOPK)
+    return fail(ctx, DLM_EINVAL, "commit mode %d", mode);
+  if (mode == DLM_COMMIT_THRESHOLD && std::isnan(tau)) return fail(ctx, DLM_EINVAL, "tau is NaN");
+  if (mode == DLM_COMMIT_TOPK && k < 1) return fail(ctx, DLM_EINVAL, "tpf_k < 1");
+  return DLM_OK;
+}
+
+dlm_block_state internal_state(dlm_ctx* ctx) {
+  dlm_block_state st{};
+  st.tokens = ctx->b_tokens;
+  st.committed = ctx->b_committed;
+  st.s = ctx->b_s;
+  st.round = ctx->b_round;
+  st.status = ctx->b_status;
+  st.stats = ctx->b_stats;
+  return st;
+}
+
+dlm_status launch_block_init(Runner& r, const dlm_block_state& st) {
+  const dlm_config& c = r.ctx->cfg;
+  BlockInitArgs ba{st.tokens, st.committed, st.s, st.round, st.status, c.block_size, c.d, c.mask_id};
+  k_block_init<<<64, 256, 0, r.s>>>(ba);
+  return r.check();
+}
+
+dlm_status build_block_graph(dlm_ctx* ctx, int mode, float tau, int k, GraphEntry* out) {
+  cudaGraph_t g = nullptr, g_init = nullptr, g_fill = nullptr;
+  CU(cudaGraphCreate(&g, 0));
+  cudaGraphConditionalHandle h;
+  CU(cudaGraphConditionalHandleCreate(&h, g, 1, cudaGraphCondAssignDefault));
+  cudaStream_t cs = ctx->cap_stream;
+  Runner r{ctx, cs, {}};
+  dlm_block_state st = internal_state(ctx);
+  const dlm_config& c = ctx->cfg;
+
+  // init
+  CU(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
+  dlm_status s1 = launch_block_init(r, st);
+  cudaError_t e = cudaStreamEndCapture(cs, &g_init);
+  if (s1 != DLM_OK) return s1;
+  CU(e);
+  cudaGraphNode_t n_init, n_while, n_fill;
+  CU(cudaGraphAddChildGraphNode(&n_init, g, nullptr, 0, g_init));
+
+  // while node with the round as its body
+  cudaGraphNodeParams cp = {};
+  cp.type = cudaGraphNodeTypeConditional;
+  cp.conditional.handle = h;
+  cp.conditional.type = cudaGraphCondTypeWhile;
+  cp.conditional.size = 1;
+  CU(cudaGraphAddNode(&n_while, g, &n_init, 1, &cp));
+  cudaGraph_t body = cp.conditional.phGraph_out[0];
+  CU(cudaStreamBeginCaptureToGraph(cs, body, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal));
+  FwdSpec f{};
+  f.T = c.block_size;
+  f.tokens = st.tokens;
+  f.s = st.s;
+  f.dev_L = true;
+  f.lm_head = true;
+  f.stats = st.stats;
+  f.s_out = st.s;
+  dlm_status s2 = forward(r, f);
+  if (s2 == DLM_OK) s2 = launch_commit(r, st, tau, mode, k, true, h);
+  e = cudaStreamEndCapture(cs, nullptr);
+  if (s2 != DLM_OK) return s2;
+  CU(e);
+
+  // KV-fill of the committed block, then the block outputs and L += B
+  CU(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
+  FwdSpec kf{};
+  kf.T = c.block_size;
+  kf.tokens = st.tokens;
+  kf.dev_L = true;
+  dlm_status s3 = forward(r, kf);
+  if (s3 == DLM_OK) {
+    BlockFinishArgs fa{st.tokens, st.round, st.status, ctx->d_err, ctx->out_tokens, ctx->out_rounds,
+                       ctx->d_L, c.block_size};
+    k_block_finish<<<1, 64, 0, cs>>>(fa);
+    s3 = r.check();
+  }
+  e = cudaStreamEndCapture(cs, &g_fill);
+  if (s3 != DLM_OK) return s3;
+  CU(e);
+  CU(cudaGraphAddChildGraphNode(&n_fill, g, &n_while, 1, g_fill));
+  cudaGraphExec_t ex;
+  CU(cudaGraphInstantiate(&ex, g, 0));
+  cudaGraphDestroy(g_init);
+  cudaGraphDestroy(g_fill);
+  *out = GraphEntry{mode, tau, k, g, ex};
+  return DLM_OK;
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+extern "C" {
+
+const char* dlm_version(void) { return "dlm-b200 0.1 (sm_100a)"; }
+
+void dlm_debug_set_gemm_impl(int impl) { g_gemm_impl = impl; }
+
+size_t dlm_workspace_size(const dlm_config* cfg) {
+  char msg[128];
+  if (!valid_cfg(cfg, msg, sizeof(msg))) return 0;
+  return carve(nullptr, *cfg, nullptr);
+}
+
+size_t dlm_kv_cache_size(const dlm_config* c) {
+  char msg[128];
+  if (!valid_cfg(c, msg, sizeof(msg))) return 0;
+  return (size_t)2 * c->n_layers * c->n_kv_heads * c->max_ctx * c->head_dim * 2;
+}
+
+dlm_status dlm_ctx_create(const dlm_config* cfg, const dlm_weights* w, void* d_workspace,
+                          size_t ws_bytes, void* d_kv_cache, size_t kv_bytes, dlm_ctx** out) {
+  char msg[256];
+  if (!out) return DLM_EINVAL;
+  *out = nullptr;
+  if (!valid_cfg(cfg, msg, sizeof(msg)) || !w || !d_workspace || (!d_kv_cache && cfg->n_layers > 0))
+    return DLM_EINVAL;
+  if (!w->embed || !w->w_adapter || !w->final_norm || (cfg->n_layers > 0 && !w->layers)) return DLM_EINVAL;
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    const dlm_layer_weights& L = w->layers[l];
+    if (!L.attn_norm || !L.w_qkv || !L.w_o || !L.mlp_norm || !L.w_gate || !L.w_up || !L.w_down)
+      return DLM_EINVAL;
+  }
+  if (cfg->weight_fmt != DLM_WEIGHTS_BF16) return DLM_EUNSUPPORTED;
+  if ((uintptr_t)d_workspace % 256) return DLM_EINVAL;
+  if (ws_bytes < dlm_workspace_size(cfg)) return DLM_ENOMEM_WS;
+  if (kv_bytes < dlm_kv_cache_size(cfg)) return DLM_ENOMEM_WS;
+  dlm_ctx* ctx = new (std::nothrow) dlm_ctx();
+  if (!ctx) return DLM_EINVAL;
+  ctx->cfg = *cfg;
+  ctx->w = *w;
+  ctx->layers.assign(w->layers, w->layers + cfg->n_layers);
+  ctx->w.layers = ctx->layers.data();
+  ctx->ws = (uint8_t*)d_workspace;
+  ctx->ws_bytes = ws_bytes;
+  ctx->kv = (__nv_bfloat16*)d_kv_cache;
+  ctx->kv_bytes = kv_bytes;
+  carve(ctx, *cfg, ctx->ws);
+  cudaError_t e = cudaStreamCreateWithFlags(&ctx->cap_stream, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->ws, 0, 256, ctx->cap_stream);
+  if (e == cudaSuccess) e = (cudaError_t)gemm_init_attributes();
+  if (e == cudaSuccess) e = (cudaError_t)attention_init_attributes();
+  if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->cap_stream);
+  if (e != cudaSuccess) {
+    if (ctx->cap_stream) cudaStreamDestroy(ctx->cap_stream);
+    delete ctx;
+    return DLM_ECUDA;
+  }
+  *out = ctx;
+  return DLM_OK;
+}
+
+dlm_status dlm_ctx_destroy(dlm_ctx* ctx) {
+  if (!ctx) return DLM_EINVAL;
+  for (auto& g : ctx->graphs) {
+    cudaGraphExecDestroy(g.exec);
+    cudaGraphDestroy(g.graph);
+  }
+  if (ctx->cap_stream) cudaStreamDestroy(ctx->cap_stream);
+  delete ctx;
+  return DLM_OK;
+}
+
+const char* dlm_last_error(const dlm_ctx* ctx) { return ctx ? ctx->err.c_str() : "null context"; }
+
+int dlm_prefix_len(const dlm_ctx* ctx) { return ctx ? ctx->L : -1; }
+
+dlm_status dlm_set_prefix_len(dlm_ctx* ctx, int L, void* stream) {
+  if (!ctx) return DLM_EINVAL;
+  if (L < 0 || L > ctx->cfg.max_ctx) return fail(ctx, DLM_EINVAL, "L=%d", L);
+  k_set_int<<<1, 1, 0, (cudaStream_t)stream>>>(ctx->d_L, L);
+  CU(cudaGetLastError());
+  ctx->L = L;
+  return DLM_OK;
+}
+
+dlm_status dlm_prefill(dlm_ctx* ctx, const int32_t* d_tokens, int n, void* stream) {
+  if (!ctx) return DLM_EINVAL;
+  if (!d_tokens || n < 0) return fail(ctx, DLM_EINVAL, "prefill args");
+  if (ctx->L + n > ctx->cfg.max_ctx) return fail(ctx, DLM_EKVCAP, "prefill: %d + %d > %d", ctx->L, n, ctx->cfg.max_ctx);
+  Runner r{ctx, (cudaStream_t)stream, {}};
+  for (int off = 0; off < n; off += kPrefillChunk) {
+    int T = n - off < kPrefillChunk ? n - off : kPrefillChunk;
+    FwdSpec f{};
+    f.T = T;
+    f.tokens = d_tokens + off;
+    f.pos0 = ctx->L + off;
+    f.causal = true;
+    TRY(forward(r, f));
+  }
+  return dlm_set_prefix_len(ctx, ctx->L + n, stream);
+}
+
+dlm_status dlm_block_init(dlm_ctx* ctx, const dlm_block_state* st, void* stream) {
+  if (!ctx) return DLM_EINVAL;
+  if (!st || !st->tokens || !st->committed || !st->s || !st->round) return fail(ctx, DLM_EINVAL, "block state");
+  Runner r{ctx, (cudaStream_t)stream, {}};
+  return launch_block_init(r, *st);
+}
+
+dlm_status dlm_round(dlm_ctx* ctx, const dlm_block_state* st, float tau, int commit_mode, int tpf_k,
+                     void* stream) {
+  if (!ctx) return DLM_EINVAL;
+  if (!st || !st->tokens || !st->committed || !st->s || !st->round || !st->stats.m || !st->stats.lse ||
+      !st->stats.maxprob || !st->stats.entropy || !st->stats.argmax)
+    return fail(ctx, DLM_EINVAL, "block state");
+  TRY(check_commit_args(ctx, tau, commit_mode, tpf_k));
+  const dlm_config& c = ctx->cfg;
+  if (ctx->L + c.block_size > c.max_ctx)
+    return fail(ctx, DLM_EKVCAP, "round: L %d + B %d > %d", ctx->L, c.block_size, c.max_ctx);
+  Runner r{ctx, (cudaStream_t)stream, {}};
+  FwdSpec f{};
+  f.T = c.block_size;
+  f.tokens = st->tokens;
+  f.s = st->s;
+  f.pos0 = ctx->L;
+  f.lm_head = true;
+  f.stats = st->stats;
+  f.s_out = st->s;
+  TRY(forward(r, f));
+  return launch_commit(r, *st, tau, commit_mode, tpf_k, false, 0);
+}
+
+dlm_status dlm_kv_fill(dlm_ctx* ctx, const int32_t* d_tokens, void* stream) {
+  if (!ctx) return DLM_EINVAL;
+  if (!d_tokens) return fail(ctx, DLM_EINVAL, "kv_fill tokens");
+  const dlm_config& c = ctx->cfg;
+  if (ctx->L + c.block_size > c.max_ctx) return fail(ctx, DLM_EKVCAP, "kv_fill: capacity");
+  Runner r{ctx, (cudaStream_t)stream, {}};
+  FwdSpec f{};
+  f.T = c.block_size;
+  f.tokens = d_tokens;
+  f.pos0 = ctx->L;
+  TRY(forward(r, f));
+  return dlm_set_prefix_len(ctx, ctx->L + c.block_size, stream);
+}
+
+dlm_status dlm_decode_block(dlm_ctx* ctx, float tau, int commit_mode, int tpf_k, int32_t* d_tokens_out,
+                            int32_t* d_rounds_out, void* stream) {
+  if (!ctx) return DLM_EINVAL;
+  TRY(check_commit_args(ctx, tau, commit_mode, tpf_k));
+  const dlm_config& c = ctx->cfg;
+  if (ctx->L + c.block_size > c.max_ctx)
+    return fail(ctx, DLM_EKVCAP, "decode_block: L %d + B %d > %d", ctx->L, c.block_size, c.max_ctx);
+  GraphEntry* ge = nullptr;
+  for (auto& g : ctx->graphs)
+    if (g.mode == commit_mode && (commit_mode == DLM_COMMIT_TOPK ? g.k == tpf_k : g.tau == tau)) ge = &g;
+  if (!ge) {
+    GraphEntry ne{};
+    TRY(build_block_graph(ctx, commit_mode, tau, tpf_k, &ne));
+    ctx->graphs.push_back(ne);
+    ge = &ctx->graphs.back();
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  CU(cudaGraphLaunch(ge->exec, s));
+  if (d_tokens_out) CU(cudaMemcpyAsync(d_tokens_out, ctx->out_tokens, c.block_size * 4, cudaMemcpyDeviceToDevice, s));
+  if (d_rounds_out) CU(cudaMemcpyAsync(d_rounds_out, ctx->out_rounds, 2 * 4, cudaMemcpyDeviceToDevice, s));
+  ctx->L += c.block_size;
+  return DLM_OK;
+}
+
+dlm_status dlm_generate(dlm_ctx* ctx, const int32_t* h_prompt, int prompt_len, int max_new, float tau,
+                        int commit_mode, int tpf_k, int32_t* h_tokens_out, int32_t* h_rounds_per_block,
+                        dlm_timing* h_timing, void* stream) {
+  if (!ctx) return DLM_EINVAL;
+  if ((!h_prompt && prompt_len > 0) || prompt_len < 0 || max_new < 0 || (!h_tokens_out && max_new > 0))
+    return fail(ctx, DLM_EINVAL, "generate args");
+  TRY(check_commit_args(ctx, tau, commit_mode, tpf_k));
+  const dlm_config& c = ctx->cfg;
+  const int B = c.block_size;
+  const int nblk = (max_new + B - 1) / B;
+  if ((long)prompt_len + (long)nblk * B > c.max_ctx)
+    return fail(ctx, DLM_EKVCAP, "generate: %d + %d blocks of %d > %d", prompt_len, nblk, B, c.max_ctx);
+  cudaStream_t s = (cudaStream_t)stream;
+  auto t0 = std::chrono::steady_clock::now();
+  TRY(dlm_set_prefix_len(ctx, 0, stream));
+  if (prompt_len > 0) {
+    CU(cudaMemcpyAsync(ctx->tok_buf, h_prompt, (size_t)prompt_len * 4, cudaMemcpyHostToDevice, s));
+    TRY(dlm_prefill(ctx, ctx->tok_buf, prompt_len, stream));
+  }
+  CU(cudaStreamSynchronize(s));
+  auto t1 = std::chrono::steady_clock::now();
+  int total_rounds = 0;
+  int32_t rb[2];
+  for (int b = 0; b < nblk; ++b) {
+    TRY(dlm_decode_block(ctx, tau, commit_mode, tpf_k, nullptr, nullptr, stream));
+    const int keep = (max_new - b * B) < B ? (max_new - b * B) : B;
+    CU(cudaMemcpyAsync(h_tokens_out + (size_t)b * B, ctx->out_tokens, (size_t)keep * 4, cudaMemcpyDeviceToHost, s));
+    CU(cudaMemcpyAsync(rb, ctx->out_rounds, 8, cudaMemcpyDeviceToHost, s));
+    CU(cudaStreamSynchronize(s));
+    if (rb[1] != 0) return fail(ctx, rb[1], "block %d: device status %d", b, rb[1]);
+    if (h_rounds_per_block) h_rounds_per_block[b] = rb[0];
+    total_rounds += rb[0];
+  }
+  auto t2 = std::chrono::steady_clock::now();
+  if (h_timing) {
+    h_timing->prefill_ms = std::chrono::duration<double, std::milli>(t1 - t0).count();
+    h_timing->decode_ms = std::chrono::duration<double, std::milli>(t2 - t1).count();
+    h_timing->n_blocks = nblk;
+    h_timing->n_rounds = total_rounds;
+  }
+  return DLM_OK;
+}
+
+// ------------------------------------------------------------------ single operations
+static size_t op_header() { return 256; }
+
+size_t dlm_gemm_scratch_size(int T, int N, int K) {
+  return op_header() + align256(gemm_partial_bytes(T, N, K, A_KMAJOR));
+}
+
+dlm_status dlm_gemm_bf16(const void* d_x, const void* d_w, float* d_y, int T, int N, int K, void* d_scratch,
+                         size_t scratch_bytes, void* stream) {
+  dlm_ctx* ctx = nullptr;
+  if (!d_x || !d_w || !d_scratch || T < 1 || T > kMaxTokens || N < 1 || K < 64 || K % 8) return DLM_EINVAL;
+  if (scratch_bytes < dlm_gemm_scratch_size(T, N, K)) return DLM_ENOMEM_WS;
+  CU((cudaError_t)gemm_init_attributes());
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* sc = (uint8_t*)d_scratch;
+  int* err = (int*)sc;
+  float* partial = (float*)(sc + op_header());
+  char msg[256];
+  GemmPlan p;
+  if (!gemm_plan(&p, A_KMAJOR, d_w, nullptr, d_x, T, N, K, partial, msg, sizeof(msg))) return DLM_EUNSUPPORTED;
+  CU(cudaMemsetAsync(err, 0, 4, s));
+  CU(gemm_launch(p, err, s));
+  if (!d_y) return DLM_OK;  // partial sums only (the tensor-core kernel alone)
+  StoreArgs a{};
+  a.y = p.out;
+  a.out = d_y;
+  a.N = N;
+  a.ld = N;
+  k_store_rows<<<dim3((N + 255) / 256, T), 256, 0, s>>>(a);
+  CU(cudaGetLastError());
+  return DLM_OK;
+}
+
+size_t dlm_lmhead_scratch_size(int B, int V, int d) {
+  size_t lm = gemm_partial_bytes(B, V, d, A_KMAJOR), pe = gemm_partial_bytes(B, d, V, A_MNMAJOR);
+  return op_header() + align256(lm > pe ? lm : pe) + align256((size_t)B * V * 4) + align256((size_t)B * V * 2);
+}
+
+dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int V, int d, int mask_id,
+                               const void* d_p_given, dlm_row_stats stats, float* d_s, void* d_scratch,
+                               size_t scratch_bytes, void* stream) {
+  dlm_ctx* ctx = nullptr;
+  if (!d_x || !d_embed || !d_s || !d_scratch || B < 1 || B > kMaxTokens || V < 2 || V % 8 || d < 64 ||
+      d % 64 || !stats.m || !stats.lse || !stats.maxprob || !stats.entropy || !stats.argmax)
+    return DLM_EINVAL;
+  if (scratch_bytes < dlm_lmhead_scratch_size(B, V, d)) return DLM_ENOMEM_WS;
+  CU((cudaError_t)gemm_init_attributes());
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* sc = (uint8_t*)d_scratch;
+  int* err = (int*)sc;
+  size_t lm = gemm_partial_bytes(B, V, d, A_KMAJOR), pe = gemm_partial_bytes(B, d, V, A_MNMAJOR);
+  float* partial = (float*)(sc + op_header());
+  float* logits = (float*)(sc + op_header() + align256(lm > pe ? lm : pe));
+  __nv_bfloat16* P = (__nv_bfloat16*)((uint8_t*)logits + align256((size_t)B * V * 4));
+  char msg[256];
+  CU(cudaMemsetAsync(err, 0, 4, s));
+  GemmPlan p;
+  if (!gemm_plan(&p, A_KMAJOR, d_embed, nullptr, d_x, B, V, d, partial, msg, sizeof(msg))) return DLM_EUNSUPPORTED;
+  CU(gemm_launch(p, err, s));
+  StoreArgs la{};
+  la.y = p.out;
+  la.out = logits;
+  la.N = V;
+  la.ld = V;
+  k_store_rows<<<dim3((V + 255) / 256, B), 256, 0, s>>>(la);
+  CU(cudaGetLastError());
+  RowStatsArgs rs{};
+  rs.logits = logits;
+  rs.ld = V;
+  rs.V = V;
+  rs.mask_id = mask_id;
+  rs.stats = stats;
+  rs.P = d_p_given ? nullptr : P;
+  k_rowstats<<<B, 1024, 0, s>>>(rs);
+  CU(cudaGetLastError());
+  GemmPlan q;
+  if (!gemm_plan(&q, A_MNMAJOR, d_embed, nullptr, d_p_given ? d_p_given : P, B, d, V, partial, msg, sizeof(msg)))
+    return DLM_EUNSUPPORTED;
+  CU(gemm_launch(q, err, s));
+  StoreArgs pa{};
+  pa.y = q.out;
+  pa.out = d_s;
+  pa.N = d;
+  pa.ld = d;
+  k_store_rows<<<dim3((d + 255) / 256, B), 256, 0, s>>>(pa);
+  CU(cudaGetLastError());
+  return DLM_OK;
+}
+
+size_t dlm_adapter_scratch_size(int B, int d) {
+  return op_header() + align256(gemm_partial_bytes(B, d, d, A_KMAJOR)) + align256((size_t)B * d * 2);
+}
+
+dlm_status dlm_adapter_embed(const void* d_embed, const void* d_w_adapter, const int32_t* d_tokens,
+                             const float* d_s, float* d_h0, int B, int d, void* d_scratch, size_t scratch_bytes,
+                             void* stream) {
+  dlm_ctx* ctx = nullptr;
+  if (!d_embed || !d_w_adapter || !d_tokens || !d_s || !d_h0 || !d_scratch || B < 1 || B > kMaxTokens ||
+      d < 64 || d % 64)
+    return DLM_EINVAL;
+  if (scratch_bytes < dlm_adapter_scratch_size(B, d)) return DLM_ENOMEM_WS;
+  CU((cudaError_t)gemm_init_attributes());
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* sc = (uint8_t*)d_scratch;
+  int* err = (int*)sc;
+  float* partial = (float*)(sc + op_header());
+  __nv_bfloat16* sbf = (__nv_bfloat16*)(sc + op_header() + align256(gemm_partial_bytes(B, d, d, A_KMAJOR)));
+  CU(cudaMemsetAsync(err, 0, 4, s));
+  long n = (long)B * d;
+  k_to_bf16<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(d_s, sbf, n);
+  CU(cudaGetLastError());
+  char msg[256];
+  GemmPlan p;
+  if (!gemm_plan(&p, A_KMAJOR, d_w_adapter, nullptr, sbf, B, d, d, partial, msg, sizeof(msg))) return DLM_EUNSUPPORTED;
+  CU(gemm_launch(p, err, s));
+  EmbedArgs ea{};
+  ea.embed = (const __nv_bfloat16*)d_embed;
+  ea.tokens = d_tokens;
+  ea.adapter = p.out;
+  ea.has_adapter = 1;
+  ea.h = d_h0;
+  ea.d = d;
+  k_embed_adapter_norm<<<B, threads_for(d), (size_t)d * 4, s>>>(ea);
+  CU(cudaGetLastError());
+  return DLM_OK;
+}
+
+size_t dlm_attention_scratch_size(int T, int Hq, int hd, int max_ctx) {
+  int sp = attention_split_cap(T, max_ctx);  // upper bound of the split count
+  return op_header() + align256(attention_scratch_bytes(T, Hq, hd, sp));
+}
+
+dlm_status dlm_bd_attention(const void* d_q, const void* d_k_cache, const void* d_v_cache, void* d_o, int T,
+                            int L, int Hq, int Hkv, int hd, int max_ctx, int causal, void* d_scratch,
+                            size_t scratch_bytes, void* stream) {
+  dlm_ctx* ctx = nullptr;
+  if (!d_q || !d_k_cache || !d_v_cache || !d_o || !d_scratch || T < 1 || L < 0 || Hq < 1 || Hkv < 1 ||
+      Hq % Hkv || !(hd == 32 || hd == 64 || hd == 128) || L + T > max_ctx)
+    return DLM_EINVAL;
+  if (scratch_bytes < dlm_attention_scratch_size(T, Hq, hd, max_ctx)) return DLM_ENOMEM_WS;
+  CU((cudaError_t)attention_init_attributes());
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* sc = (uint8_t*)d_scratch;
+  AttnArgs a{};
+  a.q = (const __nv_bfloat16*)d_q;
+  a.kc = (const __nv_bfloat16*)d_k_cache;
+  a.vc = (const __nv_bfloat16*)d_v_cache;
+  a.o = (__nv_bfloat16*)d_o;
+  a.T = T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.hd = hd;
+  a.max_ctx = max_ctx;
+  a.pos0 = L;
+  a.causal = causal ? 1 : 0;
+  a.max_splits = attention_max_splits(T, Hq, Hkv, max_ctx);
+  a.part_o = (float*)(sc + op_header());
+  a.part_ml = a.part_o + (size_t)a.max_splits * T * Hq * hd;
+  a.err = (int*)sc;
+  CU(cudaMemsetAsync(sc, 0, 4, s));
+  CU(attention_launch(a, s));
+  return DLM_OK;
+}
+
+dlm_status dlm_commit(const float* d_maxprob, const int32_t* d_argmax, int32_t* d_tokens, uint8_t* d_committed,
+                      float* d_s, int32_t* d_round, int32_t* d_status, int B, int d, float tau, int commit_mode,
+                      int tpf_k, void* stream) {
+  if (!d_maxprob || !d_argmax || !d_tokens || !d_committed || !d_s || !d_round || B < 1 || B > 64 || d < 1)
+    return DLM_EINVAL;
+  if (commit_mode != DLM_COMMIT_THRESHOLD && commit_mode != DLM_COMMIT_TOPK) return DLM_EINVAL;
+  if (commit_mode == DLM_COMMIT_THRESHOLD && std::isnan(tau)) return DLM_EINVAL;
+  if (commit_mode == DLM_COMMIT_TOPK && tpf_k < 1) return DLM_EINVAL;
+  CommitArgs ca{};
+  ca.maxprob = d_maxprob;
+  ca.argmax = d_argmax;
+  ca.tokens = d_tokens;
+  ca.committed = d_committed;
+  ca.s = d_s;
+  ca.round = d_round;
+  ca.status = d_status;
+  ca.B = B;
+  ca.d = d;
+  ca.tau = tau;
+  ca.mode = commit_mode;
+  ca.k = tpf_k;
+  k_commit<<<1, 64, 0, (cudaStream_t)stream>>>(ca);
+  return cudaGetLastError() == cudaSuccess ? DLM_OK : DLM_ECUDA;
+}
+
+dlm_status dlm_nvfp4_quantize(const void* d_w, int rows, int cols, void* d_codes, void* d_scales,
+                              float* d_tensor_scale, void* stream) {
+  if (!d_w || !d_codes || !d_scales || !d_tensor_scale || rows < 1 || cols < 16 || cols % 16) return DLM_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(d_tensor_scale, 0, 4, s) != cudaSuccess) return DLM_ECUDA;
+  long n = (long)rows * cols;
+  k_amax_bf16<<<1024, 256, 0, s>>>((const __nv_bfloat16*)d_w, n, (unsigned*)d_tensor_scale);
+  long nblk = (long)rows * (cols / 16);
+  k_nvfp4_quantize<<<(unsigned)((nblk + 255) / 256), 256, 0, s>>>((const __nv_bfloat16*)d_w, rows, cols,
+                                                                  (uint8_t*)d_codes, (uint8_t*)d_scales,
+                                                                  (const unsigned*)d_tensor_scale, nullptr);
+  k_amax_to_scale<<<1, 1, 0, s>>>(d_tensor_scale);
+  return cudaGetLastError() == cudaSuccess ? DLM_OK : DLM_ECUDA;
+}
+
+}  // extern "C"

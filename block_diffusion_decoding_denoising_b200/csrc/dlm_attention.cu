@@ -1,0 +1,384 @@
+// dlm_attention.cu -- block-diffusion attention of one layer.
+//
+// The T queries of a block (positions L .. L+T-1) attend to every key of the prefix KV
+// cache [0, L) and bidirectionally to all T keys of the block itself [L, L+T) (the block
+// K/V are written to the cache before this kernel runs).  With `causal` set the query at
+// position p sees keys [0, p] instead (prompt prefill).  [model card "QwenDLM-4B-ORL",
+// "The paper's evaluation pipeline": the SDARPrefixKV block decoder]
+//
+// GQA packing: the G = Hq / Hkv query heads that share a KV head are stacked with the
+// block's tokens into one set of T*G query rows, so one K/V tile read from HBM serves
+// all of them.  A CTA owns 64 query rows (4 warps x 16) of one KV head and one split of
+// the key range; the key range is split across CTAs (flash-decoding) so that short
+// blocks still spread the KV stream over the SMs, and a combine kernel merges the splits
+// with their (max, sum) statistics.  S = Q K^T and O = P V run on the tensor cores
+// (mma.sync m16n8k16 bf16, fp32 accumulate); softmax is online in fp32 (base-2 exponent).
+#include <cstdio>
+
+#include "dlm_device.cuh"
+#include "dlm_internal.h"
+
+namespace dlm {
+
+constexpr int kAttnRows = 64;   // query rows per CTA
+constexpr int kAttnKeys = 64;   // keys per tile
+constexpr int kMinKeysPerSplit = 256;
+
+template <int HD>
+struct AttnSmem {
+  static constexpr int kTileBytes = 64 * HD * 2;
+  static constexpr int kBytes = kTileBytes /*Q*/ + 4 * kTileBytes /*K,V double-buffered*/;
+};
+
+// 16-byte chunk swizzle inside a [64][HD] bf16 tile (row stride HD*2 bytes) that keeps
+// ldmatrix reads of 8 consecutive rows free of bank conflicts.
+template <int HD>
+__device__ __forceinline__ int swz(int row, int chunk) {
+  if constexpr (HD >= 64) return chunk ^ (row & 7);
+  else return chunk ^ ((row >> 1) & 3);
+}
+template <int HD>
+__device__ __forceinline__ uint32_t tile_addr(uint32_t base, int row, int col) {
+  // col in elements, multiple of 8 for chunk-aligned accesses
+  return base + row * (HD * 2) + swz<HD>(row, col >> 3) * 16 + (col & 7) * 2;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Number of key splits used for nkeys keys (the same rule on host and device).
+__host__ __device__ __forceinline__ int attn_splits(int nkeys, int max_splits) {
+  int s = (nkeys + kMinKeysPerSplit - 1) / kMinKeysPerSplit;
+  if (s > max_splits) s = max_splits;
+  if (s < 1) s = 1;
+  return s;
+}
+
+template <int HD>
+__global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const int G = a.Hq / a.Hkv;
+  const int rows_total = a.T * G;
+  const int g = blockIdx.y, qt = blockIdx.x, split = blockIdx.z;
+  const int L = a.pos0_dev ? *a.pos0_dev : a.pos0;
+  const int nkeys = L + a.T;
+  const int nsplit = attn_splits(nkeys, a.max_splits);
+  if (split >= nsplit) return;
+  int chunk = (nkeys + nsplit - 1) / nsplit;
+  chunk = (chunk + kAttnKeys - 1) / kAttnKeys * kAttnKeys;
+  const int k0 = split * chunk;
+  int k1 = min(nkeys, k0 + chunk);
+  const int row0 = qt * kAttnRows;
+  if (a.causal) {
+    // the last valid row of this CTA sees keys up to L + t_max
+    int rlast = min(rows_total, row0 + kAttnRows) - 1;
+    k1 = min(k1, L + rlast / G + 1);
+  }
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int gid = lane / 4, tig = lane % 4;
+  const uint32_t sQ = smem_u32(sm);
+  const uint32_t sK[2] = {sQ + AttnSmem<HD>::kTileBytes, sQ + 3 * AttnSmem<HD>::kTileBytes};
+  const uint32_t sV[2] = {sQ + 2 * AttnSmem<HD>::kTileBytes, sQ + 4 * AttnSmem<HD>::kTileBytes};
+  constexpr int CH = HD / 8;  // 16-byte chunks per row
+
+  // ---- Q tile: row r <-> (token t = r / G, head g*G + r % G)
+  for (int i = threadIdx.x; i < kAttnRows * CH; i += 128) {
+    int r = i / CH, ch = i % CH;
+    int R = row0 + r;
+    bool v = R < rows_total;
+    int t = v ? R / G : 0, h = g * G + (v ? R % G : 0);
+    const __nv_bfloat16* src = a.q + ((size_t)t * a.Hq + h) * HD + ch * 8;
+    cp_async16(sQ + r * (HD * 2) + swz<HD>(r, ch) * 16, src, v);
+  }
+  cp_commit();
+
+  const __nv_bfloat16* kbase = a.kc + (size_t)g * a.max_ctx * HD;
+  const __nv_bfloat16* vbase = a.vc + (size_t)g * a.max_ctx * HD;
+  auto load_kv = [&](int buf, int kt0) {
+    for (int i = threadIdx.x; i < kAttnKeys * CH; i += 128) {
+      int r = i / CH, ch = i % CH;
+      int key = kt0 + r;
+      bool v = key < k1;
+      size_t off = (size_t)(v ? key : 0) * HD + ch * 8;
+      cp_async16(sK[buf] + r * (HD * 2) + swz<HD>(r, ch) * 16, kbase + off, v);
+      cp_async16(sV[buf] + r * (HD * 2) + swz<HD>(r, ch) * 16, vbase + off, v);
+    }
+    cp_commit();
+  };
+
+  const int ntiles = (k1 > k0) ? (k1 - k0 + kAttnKeys - 1) / kAttnKeys : 0;
+  if (ntiles > 0) load_kv(0, k0);
+
+  // Q fragments for this warp's 16 rows
+  cp_wait<1>();
+  if (ntiles == 0) cp_wait<0>();
+  __syncthreads();
+  uint32_t qf[HD / 16][4];
+#pragma unroll
+  for (int ks = 0; ks < HD / 16; ++ks) {
+    int r = warp * 16 + (lane % 16);
+    int col = ks * 16 + (lane / 16) * 8;
+    ldsm_x4(tile_addr<HD>(sQ, r, col), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+  }
+
+  // per-thread rows: gid and gid + 8 of the warp's 16
+  const int rA = row0 + warp * 16 + gid, rB = rA + 8;
+  const int lim_A = a.causal ? (L + min(rA, rows_total - 1) / G) : (nkeys - 1);
+  const int lim_B = a.causal ? (L + min(rB, rows_total - 1) / G) : (nkeys - 1);
+  const float sl2 = 1.4426950408889634f / sqrtf((float)HD);  // log2(e) / sqrt(hd)
+  float m_A = -INFINITY, m_B = -INFINITY, l_A = 0.f, l_B = 0.f;
+  float acc[HD / 8][4];
+#pragma unroll
+  for (int i = 0; i < HD / 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+  for (int it = 0; it < ntiles; ++it) {
+    const int buf = it & 1;
+    const int kt0 = k0 + it * kAttnKeys;
+    if (it + 1 < ntiles) {
+      load_kv(buf ^ 1, kt0 + kAttnKeys);
+      cp_wait<1>();
+    } else {
+      cp_wait<0>();
+    }
+    __syncthreads();
+
+    // S = Q K^T for 16 rows x 64 keys
+    float s[8][4];
+#pragma unroll
+    for (int nb = 0; nb < 8; ++nb) s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < HD / 16; ++ks) {
+#pragma unroll
+      for (int nb2 = 0; nb2 < 4; ++nb2) {
+        // matrices: [keys nb2*16 + 0..7, hd ks*16 + 0..7], [.., +8], [keys +8.., hd 0..7], [.., +8]
+        int m = lane / 8;
+        int key = nb2 * 16 + (m / 2) * 8 + (lane % 8);
+        int col = ks * 16 + (m % 2) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(tile_addr<HD>(sK[buf], key, col), b0, b1, b2, b3);
+        mma16816(s[nb2 * 2], qf[ks], b0, b1);
+        mma16816(s[nb2 * 2 + 1], qf[ks], b2, b3);
+      }
+    }
+    // mask, running max
+    float mx_A = -INFINITY, mx_B = -INFINITY;
+#pragma unroll
+    for (int nb = 0; nb < 8; ++nb) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        int key = kt0 + nb * 8 + tig * 2 + j;
+        float vA = (key <= lim_A && key < k1) ? s[nb][j] * sl2 : -INFINITY;
+        float vB = (key <= lim_B && key < k1) ? s[nb][2 + j] * sl2 : -INFINITY;
+        s[nb][j] = vA;
+        s[nb][2 + j] = vB;
+        mx_A = fmaxf(mx_A, vA);
+        mx_B = fmaxf(mx_B, vB);
+      }
+    }
+    mx_A = fmaxf(mx_A, __shfl_xor_sync(0xffffffffu, mx_A, 1));
+    mx_A = fmaxf(mx_A, __shfl_xor_sync(0xffffffffu, mx_A, 2));
+    mx_B = fmaxf(mx_B, __shfl_xor_sync(0xffffffffu, mx_B, 1));
+    mx_B = fmaxf(mx_B, __shfl_xor_sync(0xffffffffu, mx_B, 2));
+    const float mn_A = fmaxf(m_A, mx_A), mn_B = fmaxf(m_B, mx_B);
+    const float base_A = (mn_A == -INFINITY) ? 0.f : mn_A;
+    const float base_B = (mn_B == -INFINITY) ? 0.f : mn_B;
+    const float al_A = exp2f(m_A - base_A), al_B = exp2f(m_B - base_B);
+    m_A = mn_A;
+    m_B = mn_B;
+    float rs_A = 0.f, rs_B = 0.f;
+#pragma unroll
+    for (int nb = 0; nb < 8; ++nb) {
+      s[nb][0] = exp2f(s[nb][0] - base_A);
+      s[nb][1] = exp2f(s[nb][1] - base_A);
+      s[nb][2] = exp2f(s[nb][2] - base_B);
+      s[nb][3] = exp2f(s[nb][3] - base_B);
+      rs_A += s[nb][0] + s[nb][1];
+      rs_B += s[nb][2] + s[nb][3];
+    }
+    l_A = l_A * al_A + rs_A;
+    l_B = l_B * al_B + rs_B;
+#pragma unroll
+    for (int i = 0; i < HD / 8; ++i) {
+      acc[i][0] *= al_A;
+      acc[i][1] *= al_A;
+      acc[i][2] *= al_B;
+      acc[i][3] *= al_B;
+    }
+    // O += P V
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {  // 16 keys per k-step
+      uint32_t pa[4];
+      pa[0] = pack_bf16(s[2 * ks][0], s[2 * ks][1]);
+      pa[1] = pack_bf16(s[2 * ks][2], s[2 * ks][3]);
+      pa[2] = pack_bf16(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+      pa[3] = pack_bf16(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+#pragma unroll
+      for (int nb2 = 0; nb2 < HD / 16; ++nb2) {
+        // matrices: [keys ks*16+0..7, hd nb2*16+0..7], [keys +8, ..], [keys 0..7, hd +8], [keys +8, hd +8]
+        int m = lane / 8;
+        int key = ks * 16 + (m % 2) * 8 + (lane % 8);
+        int col = nb2 * 16 + (m / 2) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(tile_addr<HD>(sV[buf], key, col), b0, b1, b2, b3);
+        mma16816(acc[nb2 * 2], pa, b0, b1);
+        mma16816(acc[nb2 * 2 + 1], pa, b2, b3);
+      }
+    }
+    __syncthreads();  // buffer `buf` is refilled two iterations later
+  }
+
+  // row sums across the quad
+  l_A += __shfl_xor_sync(0xffffffffu, l_A, 1);
+  l_A += __shfl_xor_sync(0xffffffffu, l_A, 2);
+  l_B += __shfl_xor_sync(0xffffffffu, l_B, 1);
+  l_B += __shfl_xor_sync(0xffffffffu, l_B, 2);
+
+  const int Rows = a.Hkv * rows_total;
+  for (int half = 0; half < 2; ++half) {
+    const int R = half ? rB : rA;
+    if (R >= rows_total) continue;
+    const float mrow = half ? m_B : m_A, lrow = half ? l_B : l_A;
+    const int t = R / G, h = g * G + R % G;
+    if (nsplit == 1) {
+      const float inv = lrow > 0.f ? 1.f / lrow : 0.f;
+      __nv_bfloat16* dst = a.o + ((size_t)t * a.Hq + h) * HD;
+#pragma unroll
+      for (int nb = 0; nb < HD / 8; ++nb) {
+        int col = nb * 8 + tig * 2;
+        *reinterpret_cast<__nv_bfloat162*>(dst + col) =
+            __floats2bfloat162_rn(acc[nb][half * 2] * inv, acc[nb][half * 2 + 1] * inv);
+      }
+    } else {
+      const size_t prow = (size_t)split * Rows + (size_t)g * rows_total + R;
+      float* dst = a.part_o + prow * HD;
+#pragma unroll
+      for (int nb = 0; nb < HD / 8; ++nb) {
+        int col = nb * 8 + tig * 2;
+        *reinterpret_cast<float2*>(dst + col) = make_float2(acc[nb][half * 2], acc[nb][half * 2 + 1]);
+      }
+      if (tig == 0) {
+        a.part_ml[prow * 2 + 0] = mrow;
+        a.part_ml[prow * 2 + 1] = lrow;
+      }
+    }
+  }
+}
+
+// Merges the key splits: o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
+__global__ void k_attn_combine(AttnArgs a) {
+  const int G = a.Hq / a.Hkv;
+  const int rows_total = a.T * G;
+  const int Rows = a.Hkv * rows_total;
+  const int L = a.pos0_dev ? *a.pos0_dev : a.pos0;
+  const int nsplit = attn_splits(L + a.T, a.max_splits);
+  if (nsplit == 1) return;
+  const int row = blockIdx.x;  // over Rows
+  if (row >= Rows) return;
+  const int g = row / rows_total, R = row % rows_total;
+  const int t = R / G, h = g * G + R % G;
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) {
+    float ms = a.part_ml[((size_t)s * Rows + row) * 2];
+    float ls = a.part_ml[((size_t)s * Rows + row) * 2 + 1];
+    if (ls > 0.f) M = fmaxf(M, ms);
+  }
+  for (int e = threadIdx.x; e < a.hd; e += blockDim.x) {
+    float num = 0.f, den = 0.f;
+    for (int s = 0; s < nsplit; ++s) {
+      float ms = a.part_ml[((size_t)s * Rows + row) * 2];
+      float ls = a.part_ml[((size_t)s * Rows + row) * 2 + 1];
+      if (!(ls > 0.f)) continue;
+      float w = exp2f(ms - M);
+      num += w * a.part_o[((size_t)s * Rows + row) * a.hd + e];
+      den += w * ls;
+    }
+    a.o[((size_t)t * a.Hq + h) * a.hd + e] = f2bf(den > 0.f ? num / den : 0.f);
+  }
+}
+
+int attention_max_splits(int T, int Hq, int Hkv, int max_ctx) {
+  const int G = Hq / Hkv;
+  const int qtiles = (T * G + kAttnRows - 1) / kAttnRows;
+  int ctas = qtiles * Hkv;
+  int s = (kSMs + ctas - 1) / ctas;  // enough splits to cover the SMs once
+  int by_len = (max_ctx + T + kMinKeysPerSplit - 1) / kMinKeysPerSplit;
+  if (s > by_len) s = by_len;
+  if (s < 1) s = 1;
+  if (s > 64) s = 64;
+  return s;
+}
+
+size_t attention_scratch_bytes(int T, int Hq, int hd, int max_splits) {
+  size_t rows = (size_t)T * Hq;
+  return (size_t)max_splits * rows * (hd + 2) * sizeof(float);
+}
+
+int attention_init_attributes() {
+  static bool done = false;
+  if (done) return 0;
+  cudaError_t e = cudaFuncSetAttribute(k_bd_attention<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       AttnSmem<32>::kBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_bd_attention<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem<64>::kBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_bd_attention<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnSmem<128>::kBytes);
+  if (e == cudaSuccess) done = true;
+  return (int)e;
+}
+
+int attention_split_cap(int T, int max_ctx) {
+  int by_len = (max_ctx + T + kMinKeysPerSplit - 1) / kMinKeysPerSplit;
+  return by_len < 64 ? (by_len < 1 ? 1 : by_len) : 64;
+}
+
+template <int HD>
+static cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
+  const int G = a.Hq / a.Hkv;
+  dim3 grid((a.T * G + kAttnRows - 1) / kAttnRows, a.Hkv, a.max_splits);
+  k_bd_attention<HD><<<grid, 128, AttnSmem<HD>::kBytes, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (a.max_splits > 1) {
+    k_attn_combine<<<a.Hkv * a.T * G, 128, 0, s>>>(a);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+cudaError_t attention_launch(const AttnArgs& a, cudaStream_t s) {
+  switch (a.hd) {
+    case 32: return launch_hd<32>(a, s);
+    case 64: return launch_hd<64>(a, s);
+    case 128: return launch_hd<128>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace dlm

@@ -1,0 +1,401 @@
+// dlm_gemm.cu -- weight-streaming GEMM y[T][N] = x[T][K] W[N][K]^T for the dense
+// projections of a denoising round (M = block size), on the sm_100a tensor cores.
+//
+// bs=1 rounds are bound by the HBM stream of the weights, so the kernel is shaped around
+// that stream ("swap AB"): the weights are the 128-row A operand of tcgen05.mma, the
+// block's tokens are the N = T operand, and the fp32 accumulator lives in TMEM.
+//   * One warp issues TMA (cp.async.bulk.tensor, 128-byte swizzle) loads of the weight
+//     tile and the activation tile of each k-block into an S-stage ring in shared memory.
+//   * One thread issues the MMAs (4 x K=16 per k-block) and commits each stage back to
+//     the producer; at the end of a tile it commits the accumulator to the epilogue.
+//   * Four epilogue warps read the accumulator out of TMEM (tcgen05.ld) and store fp32
+//     partial sums; two TMEM accumulators let the next tile's MMAs overlap the epilogue.
+//   * Work is split stream-K: the (tile, k-block) units of the whole GEMM are cut into
+//     `grid` equal contiguous ranges, one per SM, so every SM streams the same number of
+//     weight bytes whatever the tile count.  A tile covered by several CTAs leaves one
+//     partial per CTA ("slot"); the consumer sums the slots in a fixed order.
+// No TMA multicast is used anywhere.
+#include <cstdio>
+#include <cstring>
+
+#include "dlm_device.cuh"
+#include "dlm_internal.h"
+
+namespace dlm {
+
+int g_gemm_impl = 0;
+
+template <int NT>
+struct GemmCfg {
+  static constexpr int kABytes = kTileM * kTileK * 2;          // 16 KB
+  static constexpr int kBBytes = NT * kTileK * 2;              // NT rows of 128 B
+  static constexpr int kStageBytes = kABytes + kBBytes;        // multiple of 1024
+  static constexpr int kStages = NT <= 64 ? 8 : (NT <= 128 ? 6 : 4);
+  static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kTmemCols = (2 * NT < 32) ? 32 : 2 * NT;  // power of two for NT >= 16
+};
+
+struct GemmKArgs {
+  int a_mode;
+  int T;
+  GemmOut out;
+  int* err;
+};
+
+// 192 threads: warp 0 = TMA producer (and TMEM allocator), warp 1 = MMA issuer,
+// warps 2..5 = epilogue (TMEM lane quarter = warp % 4).
+template <int NT>
+__global__ void __launch_bounds__(192, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap ta1,
+          const __grid_constant__ CUtensorMap tb, GemmKArgs args) {
+  using Cfg = GemmCfg<NT>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = (uint64_t*)(smem + S * Cfg::kStageBytes);
+  uint64_t* full = bars;            // [S]
+  uint64_t* empty = bars + S;       // [S]
+  uint64_t* acc_full = bars + 2 * S;   // [2]
+  uint64_t* acc_empty = bars + 2 * S + 2;  // [2]
+  uint64_t* mma_done = bars + 2 * S + 4;   // [1]
+  uint32_t* tmem_holder = (uint32_t*)(bars + 2 * S + 5);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const GemmOut& o = args.out;
+  const int c = blockIdx.x;
+  const long u_begin = unit_begin(c, o.units, o.grid), u_end = unit_begin(c + 1, o.units, o.grid);
+
+  if (warp == 1 && lane == 0) {
+    for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 128); }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&ta0);
+    if (args.a_mode == A_PAIR || args.a_mode == A_MNMAJOR) prefetch_tmap(&ta1);
+    prefetch_tmap(&tb);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed_parity[8];
+    bool armed[8];
+    for (int i = 0; i < S; ++i) armed[i] = false;
+    bool ok = true;
+    for (long u = u_begin; u < u_end && ok; ++u) {
+      const int tile = (int)(u / o.n_kb), kb = (int)(u % o.n_kb);
+      if (!mbar_wait(&empty[stage], phase ^ 1, args.err)) { ok = false; break; }
+      uint8_t* sa = smem + stage * Cfg::kStageBytes;
+      uint8_t* sb = sa + Cfg::kABytes;
+      mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
+      armed[stage] = true;
+      armed_parity[stage] = phase;
+      if (args.a_mode == A_KMAJOR) {
+        tma_load_2d(sa, &ta0, &full[stage], kb * kTileK, tile * kTileM);
+      } else if (args.a_mode == A_PAIR) {
+        tma_load_2d(sa, &ta0, &full[stage], kb * kTileK, tile * 64);
+        tma_load_2d(sa + Cfg::kABytes / 2, &ta1, &full[stage], kb * kTileK, tile * 64);
+      } else {  // A^T stored [K][N]: two 64-wide column boxes of 64 K-rows
+        tma_load_2d(sa, &ta0, &full[stage], tile * kTileM, kb * kTileK);
+        tma_load_2d(sa + Cfg::kABytes / 2, &ta0, &full[stage], tile * kTileM + 64, kb * kTileK);
+      }
+      tma_load_2d(sb, &tb, &full[stage], kb * kTileK, 0);
+      if (++stage == S) { stage = 0; phase ^= 1; }
+    }
+    // never leave the CTA with copies in flight: wait (bounded) for every armed stage
+    for (int i = 0; i < S; ++i)
+      if (armed[i]) mbar_wait(&full[i], armed_parity[i], args.err);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    const uint32_t idesc = idesc_bf16(128, NT, args.a_mode == A_MNMAJOR, false);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    long u = u_begin;
+    while (u < u_end && ok) {
+      const int tile = (int)(u / o.n_kb);
+      const long seg_end = ((long)tile + 1) * o.n_kb < u_end ? ((long)tile + 1) * o.n_kb : u_end;
+      if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, args.err)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * NT;
+      for (long uu = u; uu < seg_end; ++uu) {
+        if (!mbar_wait(&full[stage], phase, args.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
+        const uint32_t sb = sa + Cfg::kABytes;
+#pragma unroll
+        for (int k = 0; k < kTileK / 16; ++k) {
+          uint64_t adesc = (args.a_mode == A_MNMAJOR)
+                               ? sw128_desc(sa + k * 2048, Cfg::kABytes / 2, 1024)
+                               : sw128_desc(sa + k * 32, 16, 1024);
+          uint64_t bdesc = sw128_desc(sb + k * 32, 16, 1024);
+          mma_bf16(d_tmem, adesc, bdesc, idesc, (uu > u || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[stage]);
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      mma_commit(&acc_full[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      u = seg_end;
+    }
+    // all MMAs of this thread complete before TMEM is released
+    mma_commit(mma_done);
+    mbar_wait(mma_done, 0, args.err);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: TMEM -> fp32 partials
+    const int quarter = warp % 4;
+    const int row = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    long u = u_begin;
+    float v[32];
+    while (u < u_end) {
+      const int tile = (int)(u / o.n_kb);
+      const long seg_end = ((long)tile + 1) * o.n_kb < u_end ? ((long)tile + 1) * o.n_kb : u_end;
+      if (!mbar_wait(&acc_full[acc], acc_phase, args.err)) break;
+      tc_fence_after();
+      const int slot = c - cta_of_unit((long)tile * o.n_kb, o.units, o.grid);
+      float* dst = o.partial + (((size_t)tile * o.max_slots + slot) * o.T) * kTileM + row;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * NT;
+      static_assert(NT % 32 == 0, "token tile is a multiple of 32");
+#pragma unroll 1
+      for (int cb = 0; cb < NT / 32; ++cb) {
+        if (cb * 32 >= o.T) break;
+        tmem_ld32(taddr + cb * 32, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int t = cb * 32 + j;
+          if (t < o.T) dst[(size_t)t * kTileM] = v[j];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      u = seg_end;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem_base, Cfg::kTmemCols);
+}
+
+// ------------------------------------------------------------------ CUDA-core kernel
+// Same output contract with a single slot; a plain reference-grade kernel kept as a
+// debugging aid (selected with dlm_debug_set_gemm_impl(1)).
+struct SimtArgs {
+  const __nv_bfloat16* a0;
+  const __nv_bfloat16* a1;
+  const __nv_bfloat16* x;
+  int a_mode, N, K, T;
+  GemmOut out;
+};
+
+__global__ void k_gemm_simt(SimtArgs a) {
+  const int tile = blockIdx.x, row = threadIdx.x, t = blockIdx.y;
+  if (t >= a.T) return;
+  const __nv_bfloat16* xr = a.x + (size_t)t * a.K;
+  const __nv_bfloat16* wr = nullptr;
+  bool valid = true;
+  if (a.a_mode == A_KMAJOR) {
+    int n = tile * kTileM + row;
+    valid = n < a.N;
+    wr = a.a0 + (size_t)n * a.K;
+  } else if (a.a_mode == A_PAIR) {
+    int f = tile * 64 + (row % 64);
+    valid = f < a.N;
+    wr = (row < 64 ? a.a0 : a.a1) + (size_t)f * a.K;
+  }
+  float acc = 0.f;
+  if (valid) {
+    if (a.a_mode == A_MNMAJOR) {
+      int n = tile * kTileM + row;
+      if (n < a.N)
+        for (int k = 0; k < a.K; ++k) acc += bf2f(xr[k]) * bf2f(a.a0[(size_t)k * a.N + n]);
+    } else {
+      for (int k = 0; k < a.K; ++k) acc += bf2f(xr[k]) * bf2f(wr[k]);
+    }
+  }
+  a.out.partial[((size_t)tile * a.out.max_slots) * a.out.T * kTileM + (size_t)t * kTileM + row] = acc;
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode() {
+  static PFN_encodeTiled fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_encodeTiled)p;
+  }
+  return fn;
+}
+
+bool encode_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, char* err,
+                    size_t errlen) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) {
+    snprintf(err, errlen, "cuTensorMapEncodeTiled entry point unavailable");
+    return false;
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(err, errlen, "cuTensorMapEncodeTiled failed (%d): dims %llu x %llu box %u x %u", (int)r,
+             (unsigned long long)inner, (unsigned long long)outer, box_inner, box_outer);
+    return false;
+  }
+  return true;
+}
+
+static int pad_nt(int T) {
+  if (T <= 32) return 32;
+  if (T <= 64) return 64;
+  if (T <= 128) return 128;
+  return 256;
+}
+
+static void partition(int T, int N, int K, int a_mode, GemmOut* o) {
+  const int rows_per_tile = (a_mode == A_PAIR) ? 64 : kTileM;
+  o->T = T;
+  o->n_tiles = (N + rows_per_tile - 1) / rows_per_tile;
+  o->n_kb = (K + kTileK - 1) / kTileK;
+  o->units = (long)o->n_tiles * o->n_kb;
+  int grid = kSMs;
+  if (g_gemm_impl == 1) grid = o->n_tiles;
+  if (o->units < grid) grid = (int)o->units;
+  o->grid = grid;
+  int ms = 1;
+  if (g_gemm_impl != 1) {
+    for (int t = 0; t < o->n_tiles; ++t) {
+      int lo = cta_of_unit((long)t * o->n_kb, o->units, grid);
+      int hi = cta_of_unit((long)(t + 1) * o->n_kb - 1, o->units, grid);
+      if (hi - lo + 1 > ms) ms = hi - lo + 1;
+    }
+  }
+  o->max_slots = ms;
+}
+
+size_t gemm_partial_bytes(int T, int N, int K, int a_mode) {
+  GemmOut o;
+  partition(T, N, K, a_mode, &o);
+  return (size_t)o.n_tiles * o.max_slots * T * kTileM * sizeof(float);
+}
+
+bool gemm_plan(GemmPlan* p, int a_mode, const void* a0, const void* a1, const void* x, int T, int N,
+               int K, float* partial, char* err, size_t errlen) {
+  memset(p, 0, sizeof(*p));
+  if (T < 1 || T > kMaxTokens || N < 1 || K < kTileK || K % 8 != 0) {
+    snprintf(err, errlen, "gemm: unsupported shape T=%d N=%d K=%d", T, N, K);
+    return false;
+  }
+  p->a_mode = a_mode;
+  p->a0 = a0;
+  p->a1 = a1;
+  p->x = x;
+  p->N = N;
+  p->K = K;
+  p->T = T;
+  p->nt = pad_nt(T);
+  partition(T, N, K, a_mode, &p->out);
+  p->out.partial = partial;
+  p->partial_bytes = (size_t)p->out.n_tiles * p->out.max_slots * T * kTileM * sizeof(float);
+  bool ok = true;
+  if (a_mode == A_KMAJOR) {
+    ok = encode_tmap_2d(&p->ta0, a0, K, N, (uint64_t)K * 2, kTileK, kTileM, err, errlen);
+    p->ta1 = p->ta0;
+  } else if (a_mode == A_PAIR) {
+    ok = encode_tmap_2d(&p->ta0, a0, K, N, (uint64_t)K * 2, kTileK, 64, err, errlen) &&
+         encode_tmap_2d(&p->ta1, a1, K, N, (uint64_t)K * 2, kTileK, 64, err, errlen);
+  } else {
+    // A^T stored [K][N] row-major: inner dimension N, boxes of 64 (N) x 64 (K rows)
+    ok = encode_tmap_2d(&p->ta0, a0, N, K, (uint64_t)N * 2, 64, kTileK, err, errlen);
+    p->ta1 = p->ta0;
+  }
+  ok = ok && encode_tmap_2d(&p->tb, x, K, T, (uint64_t)K * 2, kTileK, p->nt, err, errlen);
+  return ok;
+}
+
+template <int NT>
+static cudaError_t launch_nt(const GemmPlan& p, int* d_err, cudaStream_t s) {
+  GemmKArgs a;
+  a.a_mode = p.a_mode;
+  a.T = p.T;
+  a.out = p.out;
+  a.err = d_err;
+  k_gemm_tc<NT><<<p.out.grid, 192, GemmCfg<NT>::kSmem, s>>>(p.ta0, p.ta1, p.tb, a);
+  return cudaGetLastError();
+}
+
+template <int NT>
+static cudaError_t set_smem_attr() {
+  return cudaFuncSetAttribute(k_gemm_tc<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<NT>::kSmem);
+}
+
+// Sets the dynamic shared-memory limits of every GEMM instantiation once per process
+// (must happen outside stream capture).
+int gemm_init_attributes() {
+  static bool done = false;
+  if (done) return 0;
+  cudaError_t e = set_smem_attr<32>();
+  if (e == cudaSuccess) e = set_smem_attr<64>();
+  if (e == cudaSuccess) e = set_smem_attr<128>();
+  if (e == cudaSuccess) e = set_smem_attr<256>();
+  if (e == cudaSuccess) done = true;
+  return (int)e;
+}
+
+static cudaError_t gemm_launch_simt(const GemmPlan& p, cudaStream_t s);
+
+cudaError_t gemm_launch(const GemmPlan& p, int* d_err, cudaStream_t s) {
+  if (g_gemm_impl == 1) return gemm_launch_simt(p, s);
+  switch (p.nt) {
+    case 32: return launch_nt<32>(p, d_err, s);
+    case 64: return launch_nt<64>(p, d_err, s);
+    case 128: return launch_nt<128>(p, d_err, s);
+    default: return launch_nt<256>(p, d_err, s);
+  }
+}
+
+static cudaError_t gemm_launch_simt(const GemmPlan& p, cudaStream_t s) {
+  SimtArgs a;
+  a.a0 = (const __nv_bfloat16*)p.a0;
+  a.a1 = (const __nv_bfloat16*)p.a1;
+  a.x = (const __nv_bfloat16*)p.x;
+  a.a_mode = p.a_mode;
+  a.N = p.N;
+  a.K = p.K;
+  a.T = p.T;
+  a.out = p.out;
+  dim3 grid(p.out.n_tiles, p.T);
+  k_gemm_simt<<<grid, kTileM, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace dlm

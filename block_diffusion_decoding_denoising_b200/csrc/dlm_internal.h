@@ -1,0 +1,80 @@
+// dlm_internal.h -- declarations shared by the translation units of libdlm (host side).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/dlm.h"
+
+namespace dlm {
+
+constexpr int kSMs = 148;        // B200 streaming multiprocessors
+constexpr int kTileM = 128;      // output features per GEMM tile (tcgen05 M)
+constexpr int kTileK = 64;       // reduction elements per k-block (one 128-byte swizzle atom)
+constexpr int kMaxTokens = 256;  // tokens per forward pass (tcgen05 N <= 256)
+
+// Partial-sum layout written by the GEMM: [tile][slot][T][128] fp32.  Tile tau covers
+// output features [128 tau, 128 tau + 128) (for the gate/up pair: gate features
+// [64 tau, 64 tau + 64) in rows 0..63 and up features in rows 64..127).  The slots of a
+// tile are the CTAs whose stream-K range intersects it, summed in slot order.
+struct GemmOut {
+  float* partial;
+  int T;          // tokens
+  int n_tiles;
+  int n_kb;
+  int grid;       // CTAs of the stream-K partition
+  long units;     // n_tiles * n_kb
+  int max_slots;
+};
+
+enum AMode : int {
+  A_KMAJOR = 0,   // W [N][K]: one 128-row box per k-block
+  A_PAIR = 1,     // two matrices [F][K] interleaved 64 + 64 rows per tile (gate/up)
+  A_MNMAJOR = 2,  // A^T stored [K][N] (e.g. E [V][d] for s = P E): two 64-column boxes
+};
+
+struct GemmPlan {
+  CUtensorMap ta0, ta1, tb;
+  int a_mode;
+  int nt;            // MMA N (tokens padded to 16/32/64/128/256)
+  int N, K, T;
+  const void *a0, *a1, *x;
+  GemmOut out;
+  size_t partial_bytes;
+};
+
+// host helpers (dlm_gemm.cu)
+bool encode_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, char* err, size_t errlen);
+size_t gemm_partial_bytes(int T, int N, int K, int a_mode);
+// Plans y = x W^T.  `a0` is W (or Wg for A_PAIR, E for A_MNMAJOR), `a1` Wu for A_PAIR.
+bool gemm_plan(GemmPlan* p, int a_mode, const void* a0, const void* a1, const void* x, int T,
+               int N, int K, float* partial, char* err, size_t errlen);
+cudaError_t gemm_launch(const GemmPlan& p, int* d_err, cudaStream_t s);
+int gemm_init_attributes();
+extern int g_gemm_impl;  // 0 = tcgen05 (default), 1 = plain CUDA-core kernel (debug aid)
+
+// attention (dlm_attention.cu)
+struct AttnArgs {
+  const __nv_bfloat16* q;    // [T][Hq][hd]
+  const __nv_bfloat16* kc;   // [Hkv][max_ctx][hd] (one layer)
+  const __nv_bfloat16* vc;
+  __nv_bfloat16* o;          // [T][Hq][hd]
+  float* part_o;             // [max_splits][Hkv * T * G][hd]
+  float* part_ml;            // [max_splits][Hkv * T * G][2]
+  int T, Hq, Hkv, hd, max_ctx;
+  int pos0;                  // prefix length L when pos0_dev == nullptr
+  const int* pos0_dev;       // device L (graph mode)
+  int causal;
+  int max_splits;
+  int* err;
+};
+size_t attention_scratch_bytes(int T, int Hq, int hd, int max_splits);
+int attention_max_splits(int T, int Hq, int Hkv, int max_ctx);
+cudaError_t attention_launch(const AttnArgs& a, cudaStream_t s);
+int attention_init_attributes();
+int attention_split_cap(int T, int max_ctx);
+
+}  // namespace dlm

@@ -1,0 +1,371 @@
+// dlm_ops.cu -- the light kernels of a denoising round: they consume the GEMM partial
+// sums and apply what follows each projection, plus the LM-head statistics and the
+// commit rule.
+//
+// Round data flow (one block of T = B tokens at positions L .. L+B-1):
+//   s (fp32) --bf16--> W_a GEMM --k_embed_adapter_norm--> h = E[x] + W_a s, xn = RMSNorm(h)
+//   per layer: QKV GEMM --k_qkv_rope--> q, K/V cache rows [L, L+B) (RoPE, bf16)
+//              attention --> o (bf16)
+//              O GEMM --k_residual_norm--> h += o W_o^T, xn = RMSNorm(h)
+//              gate/up GEMM --k_silu_gate--> a = silu(g) * u (bf16)
+//              down GEMM --k_residual_norm--> h += a W_d^T, xn = RMSNorm(h) (next norm)
+//   LM head: E GEMM --> logits --k_rowstats--> stats, P = softmax (bf16)
+//            P E (MN-major GEMM) --k_store_rows--> s
+//   k_commit: commit rule, loop condition.
+#include <cfloat>
+#include <cstdio>
+
+#include "dlm_device.cuh"
+#include "dlm_internal.h"
+#include "dlm_ops.h"
+
+namespace dlm {
+
+// ------------------------------------------------------------------ block reductions
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nw = blockDim.x / 32;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = 0.f;
+  for (int i = 0; i < nw; ++i) r += red[i];  // fixed order: deterministic
+  return r;
+}
+
+// RMSNorm of one row held in `row` (shared, fp32), written as bf16: x * r * g, with
+// r = 1 / sqrt(mean(x^2) + eps).
+__device__ void norm_row_to_bf16(const float* row, int d, const __nv_bfloat16* g, float eps,
+                                 __nv_bfloat16* out, float* red) {
+  float ss = 0.f;
+  for (int n = threadIdx.x; n < d; n += blockDim.x) ss += row[n] * row[n];
+  ss = block_sum(ss, red);
+  const float r = 1.0f / sqrtf(ss / (float)d + eps);
+  for (int n = threadIdx.x; n < d; n += blockDim.x) out[n] = f2bf(row[n] * r * bf2f(g[n]));
+}
+
+// h[t] = E[tok_t] (+ W_a s_t from the GEMM partials when `has_adapter`), then
+// xn[t] = RMSNorm(h[t]) with gain g.  One CTA per token.
+__global__ void k_embed_adapter_norm(EmbedArgs a) {
+  extern __shared__ float rowbuf[];
+  __shared__ float red[32];
+  const int t = blockIdx.x;
+  const int tok = a.tokens[t];
+  const __nv_bfloat16* e = a.embed + (size_t)tok * a.d;
+  for (int n = threadIdx.x; n < a.d; n += blockDim.x) {
+    float v = bf2f(e[n]);
+    if (a.has_adapter) v += gemm_out(a.adapter, n, t);
+    rowbuf[n] = v;
+    a.h[(size_t)t * a.d + n] = v;
+  }
+  __syncthreads();
+  if (a.gain) norm_row_to_bf16(rowbuf, a.d, a.gain, a.eps, a.xn + (size_t)t * a.d, red);
+}
+
+// h[t] += y[t] (GEMM output of W_o or W_d); xn[t] = RMSNorm(h[t]) with the next gain.
+__global__ void k_residual_norm(ResidArgs a) {
+  extern __shared__ float rowbuf[];
+  __shared__ float red[32];
+  const int t = blockIdx.x;
+  for (int n = threadIdx.x; n < a.d; n += blockDim.x) {
+    float v = a.h[(size_t)t * a.d + n] + gemm_out(a.y, n, t);
+    rowbuf[n] = v;
+    a.h[(size_t)t * a.d + n] = v;
+  }
+  __syncthreads();
+  if (a.gain) norm_row_to_bf16(rowbuf, a.d, a.gain, a.eps, a.xn + (size_t)t * a.d, red);
+}
+
+// QKV projection output -> RoPE (NeoX pairing (j, j + hd/2), theta_j = base^(-2j/hd),
+// absolute position L + t; angles in double precision) -> bf16 q and the K/V cache rows.
+// grid (Hq + 2 Hkv, T), hd/2 threads.
+__global__ void k_qkv_rope(QkvArgs a) {
+  const int hh = blockIdx.x, t = blockIdx.y, j = threadIdx.x;
+  const int hd = a.hd, half = hd / 2;
+  if (j >= half) return;
+  const int L = a.pos0_dev ? *a.pos0_dev : a.pos0;
+  const long pos = (long)L + t;
+  float x0 = gemm_out(a.y, hh * hd + j, t);
+  float x1 = gemm_out(a.y, hh * hd + j + half, t);
+  if (hh < a.Hq + a.Hkv) {
+    double theta = pow(a.rope_theta, -2.0 * (double)j / (double)hd);
+    double s, c;
+    sincos((double)pos * theta, &s, &c);
+    float cf = (float)c, sf = (float)s;
+    float r0 = x0 * cf - x1 * sf;
+    float r1 = x0 * sf + x1 * cf;
+    x0 = r0;
+    x1 = r1;
+  }
+  __nv_bfloat16* dst;
+  if (hh < a.Hq) {
+    dst = a.q + ((size_t)t * a.Hq + hh) * hd;
+  } else if (hh < a.Hq + a.Hkv) {
+    dst = a.kc + ((size_t)(hh - a.Hq) * a.max_ctx + pos) * hd;
+  } else {
+    dst = a.vc + ((size_t)(hh - a.Hq - a.Hkv) * a.max_ctx + pos) * hd;
+  }
+  dst[j] = f2bf(x0);
+  dst[j + half] = f2bf(x1);
+}
+
+// a[t][f] = bf16(silu(g) * u), g and u from the paired gate/up GEMM (tile = 64 + 64 rows).
+__global__ void k_silu_gate(SiluArgs a) {
+  const int t = blockIdx.y;
+  const int f = blockIdx.x * blockDim.x + threadIdx.x;
+  if (f >= a.F) return;
+  const int tile = f / 64, r = f % 64;
+  const float g = gemm_sum(a.y, tile, r, t);
+  const float u = gemm_sum(a.y, tile, 64 + r, t);
+  const float silu = g / (1.0f + expf(-g));
+  a.out[(size_t)t * a.F + f] = f2bf(silu * u);
+}
+
+// out[t][n] = y[t][n] (fp32), n < N.
+__global__ void k_store_rows(StoreArgs a) {
+  const int t = blockIdx.y;
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= a.N) return;
+  a.out[(size_t)t * a.ld + n] = gemm_out(a.y, n, t);
+}
+
+// bf16 copy of s (the W_a GEMM input).
+__global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n) {
+  long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = f2bf(x[i]);
+}
+
+// Row statistics of logits[b][:] (mask id excluded) and P = softmax as bf16.
+// m = max, argmax = lowest id of the max, Z = sum e^(l-m), lse = m + ln Z,
+// maxprob = 1/Z, entropy = ln Z - sum e^(l-m)(l-m) / Z.  One CTA per row.
+__global__ void k_rowstats(RowStatsArgs a) {
+  __shared__ float red_v[32];
+  __shared__ int red_i[32];
+  __shared__ float bcast[2];
+  const int b = blockIdx.x;
+  const float* l = a.logits + (size_t)b * a.ld;
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nw = blockDim.x / 32;
+  float m = -INFINITY;
+  int am = 0x7fffffff;
+  for (int v = threadIdx.x; v < a.V; v += blockDim.x) {
+    if (v == a.mask_id) continue;
+    float x = l[v];
+    if (x > m || (x == m && v < am)) { m = x; am = v; }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    int a2 = __shfl_xor_sync(0xffffffffu, am, o);
+    if (m2 > m || (m2 == m && a2 < am)) { m = m2; am = a2; }
+  }
+  if (lane == 0) { red_v[warp] = m; red_i[warp] = am; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float mm = red_v[0];
+    int aa = red_i[0];
+    for (int i = 1; i < nw; ++i)
+      if (red_v[i] > mm || (red_v[i] == mm && red_i[i] < aa)) { mm = red_v[i]; aa = red_i[i]; }
+    bcast[0] = mm;
+    red_i[0] = aa;
+  }
+  __syncthreads();
+  m = bcast[0];
+  am = red_i[0];
+  __syncthreads();
+  float z = 0.f, A = 0.f;
+  for (int v = threadIdx.x; v < a.V; v += blockDim.x) {
+    if (v == a.mask_id) continue;
+    float x = l[v] - m;
+    float e = expf(x);
+    z += e;
+    A += e * x;
+  }
+  z = block_sum(z, red_v);
+  A = block_sum(A, red_v);
+  const float lnz = logf(z);
+  const float lse = m + lnz;
+  if (threadIdx.x == 0) {
+    a.stats.m[b] = m;
+    a.stats.lse[b] = lse;
+    a.stats.maxprob[b] = 1.0f / z;
+    a.stats.entropy[b] = lnz - A / z;
+    a.stats.argmax[b] = am;
+  }
+  if (a.P) {
+    __nv_bfloat16* p = a.P + (size_t)b * a.V;
+    for (int v = threadIdx.x; v < a.V; v += blockDim.x)
+      p[v] = f2bf(v == a.mask_id ? 0.f : expf(l[v] - lse));
+  }
+}
+
+// Commit rule for one block (one CTA, blockDim >= B).  Threshold mode: every uncommitted
+// position with maxprob >= tau, or if none qualifies the single uncommitted position with
+// the largest maxprob (ties -> lowest position).  Top-k mode: the min(k, remaining)
+// uncommitted positions of largest maxprob (ties -> lowest position).  Newly committed
+// positions take their argmax token and get a zero residual row.
+__global__ void k_commit(CommitArgs a) {
+  __shared__ float mp[64];
+  __shared__ int unc[64];
+  __shared__ int sel[64];
+  __shared__ int best;
+  const int i = threadIdx.x;
+  const int B = a.B;
+  if (i < B) {
+    mp[i] = a.maxprob[i];
+    unc[i] = a.committed[i] ? 0 : 1;
+    sel[i] = 0;
+  }
+  __syncthreads();
+  if (a.mode == DLM_COMMIT_THRESHOLD) {
+    int q = (i < B && unc[i] && mp[i] >= a.tau) ? 1 : 0;
+    if (i < B) sel[i] = q;
+    int nq = __syncthreads_count(q);
+    if (nq == 0 && i == 0) {
+      int bi = -1;
+      for (int j = 0; j < B; ++j)
+        if (unc[j] && (bi < 0 || mp[j] > mp[bi])) bi = j;
+      best = bi;
+    }
+    __syncthreads();
+    if (nq == 0 && i < B) sel[i] = (i == best) ? 1 : 0;
+  } else {
+    if (i < B && unc[i]) {
+      int rank = 0;
+      for (int j = 0; j < B; ++j)
+        if (unc[j] && (mp[j] > mp[i] || (mp[j] == mp[i] && j < i))) ++rank;
+      sel[i] = rank < a.k ? 1 : 0;
+    }
+  }
+  __syncthreads();
+  if (i < B && sel[i]) {
+    a.tokens[i] = a.argmax[i];
+    a.committed[i] = 1;
+  }
+  __syncthreads();
+  // committed positions (old and new) carry no residual into the next round
+  for (int r = 0; r < B; ++r) {
+    if (unc[r] && !sel[r]) continue;
+    for (int n = threadIdx.x; n < a.d; n += blockDim.x) a.s[(size_t)r * a.d + n] = 0.f;
+  }
+  int left = (i < B && unc[i] && !sel[i]) ? 1 : 0;
+  int nleft = __syncthreads_count(left);
+  if (i == 0) {
+    int rnd = *a.round + 1;
+    *a.round = rnd;
+    unsigned cond = (nleft > 0 && rnd < B) ? 1u : 0u;
+    if (nleft > 0 && rnd >= B && a.status) atomicCAS(a.status, 0, DLM_EROUNDCAP);
+    if (a.use_cond) cudaGraphSetConditional(a.cond, cond);
+  }
+}
+
+// tokens = mask_id, committed = 0, s = 0, round = 0, status = 0.
+__global__ void k_block_init(BlockInitArgs a) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < a.B) {
+    a.tokens[i] = a.mask_id;
+    a.committed[i] = 0;
+  }
+  if (i == 0) {
+    *a.round = 0;
+    if (a.status) *a.status = 0;
+  }
+  for (long n = i; n < (long)a.B * a.d; n += (long)gridDim.x * blockDim.x) a.s[n] = 0.f;
+}
+
+// End of a block: copy tokens and {round, status} out, merge the kernel error flag into
+// the status, and advance the device prefix length by B.
+__global__ void k_block_finish(BlockFinishArgs a) {
+  const int i = threadIdx.x;
+  if (i < a.B) a.tokens_out[i] = a.tokens[i];
+  if (i == 0) {
+    a.rounds_out[0] = *a.round;
+    int st = *a.status;
+    if (st == 0 && a.err) st = *a.err;
+    a.rounds_out[1] = st;
+    if (a.L_dev) *a.L_dev += a.B;
+  }
+}
+
+__global__ void k_set_int(int* p, int v) { *p = v; }
+
+// amax bits -> tensor scale amax / (6 * 448), in place.
+__global__ void k_amax_to_scale(float* p) {
+  *p = __uint_as_float(*reinterpret_cast<unsigned*>(p)) / (6.0f * 448.0f);
+}
+
+// ------------------------------------------------------------------ NVFP4 quantizer
+// Per-tensor scale S = amax / (6 * 448) (fp32 division), per 16-element block e4m3 scale
+// sigma = RN_e4m3(amax_blk / (6 S)) (saturating), codes = RNE e2m1 of w / (sigma S).
+__global__ void k_amax_bf16(const __nv_bfloat16* w, long n, unsigned* amax_bits) {
+  float m = 0.f;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
+    m = fmaxf(m, fabsf(bf2f(w[i])));
+  m = warp_max(m);
+  if (threadIdx.x % 32 == 0) atomicMax(amax_bits, __float_as_uint(m));  // m >= 0: bit order = value order
+}
+
+__device__ __forceinline__ uint8_t e2m1_rne(float r) {
+  // magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6; ties to the even code
+  const float a = fabsf(r);
+  uint8_t c;
+  if (a <= 0.25f) c = 0;
+  else if (a < 0.75f) c = 1;
+  else if (a <= 1.25f) c = 2;
+  else if (a < 1.75f) c = 3;
+  else if (a <= 2.5f) c = 4;
+  else if (a < 3.5f) c = 5;
+  else if (a <= 5.0f) c = 6;
+  else c = 7;
+  return (uint8_t)(c | ((r < 0.f) ? 8 : 0));
+}
+
+__device__ __forceinline__ float e4m3_value_dev(uint8_t b) {
+  int E = (b >> 3) & 15, m = b & 7;
+  if (E == 0) return ldexpf((float)m, -9);
+  return ldexpf(1.0f + m / 8.0f, E - 7);
+}
+
+// Rounds a non-negative fp32 value to e4m3 (RNE, saturating at 448); returns the bits.
+__device__ __forceinline__ uint8_t e4m3_rne_bits(float x) {
+  if (!(x > 0.f)) return 0;
+  if (x >= 448.f) return 0x7E;
+  int e;
+  frexpf(x, &e);  // x = f 2^e, f in [0.5, 1)
+  int qexp = e - 4;
+  if (qexp < -9) qexp = -9;
+  float q = ldexpf(1.0f, qexp);
+  float r = rintf(x / q) * q;  // x / q exact (power of two), rintf: ties to even
+  if (r > 448.f) r = 448.f;
+  // encode r
+  int e2;
+  float f2 = frexpf(r, &e2);
+  int E = e2 - 1 + 7;
+  if (E <= 0) return (uint8_t)((int)rintf(r / ldexpf(1.0f, -9)) & 7);
+  int mm = (int)rintf((f2 * 2.0f - 1.0f) * 8.0f);
+  return (uint8_t)((E << 3) | mm);
+}
+
+__global__ void k_nvfp4_quantize(const __nv_bfloat16* w, int rows, int cols, uint8_t* codes,
+                                 uint8_t* scales, const unsigned* amax_bits, float* tscale) {
+  const float amax = __uint_as_float(*amax_bits);
+  const float S = amax / (6.0f * 448.0f);
+  const long nblk = (long)rows * (cols / 16);
+  const long b = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (b == 0 && tscale) *tscale = S;
+  if (b >= nblk) return;
+  const __nv_bfloat16* src = w + b * 16;
+  float v[16];
+  float bm = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) { v[j] = bf2f(src[j]); bm = fmaxf(bm, fabsf(v[j])); }
+  uint8_t sb = (S > 0.f) ? e4m3_rne_bits(bm / (6.0f * S)) : 0;
+  scales[b] = sb;
+  const float denom = e4m3_value_dev(sb) * S;
+#pragma unroll
+  for (int j = 0; j < 16; j += 2) {
+    uint8_t c0 = denom > 0.f ? e2m1_rne(v[j] / denom) : 0;
+    uint8_t c1 = denom > 0.f ? e2m1_rne(v[j + 1] / denom) : 0;
+    codes[b * 8 + j / 2] = (uint8_t)(c0 | (c1 << 4));
+  }
+}
+
+}  // namespace dlm

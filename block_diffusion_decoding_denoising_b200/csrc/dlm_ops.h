@@ -1,0 +1,115 @@
+// dlm_ops.h -- argument structs and declarations of the light kernels (dlm_ops.cu).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "dlm_internal.h"
+
+namespace dlm {
+
+struct EmbedArgs {
+  const __nv_bfloat16* embed;  // [V][d]
+  const int32_t* tokens;       // [T]
+  GemmOut adapter;             // W_a s partials (when has_adapter)
+  int has_adapter;
+  float* h;                    // [T][d]
+  __nv_bfloat16* xn;           // [T][d]
+  const __nv_bfloat16* gain;   // [d]
+  int d;
+  float eps;
+};
+
+struct ResidArgs {
+  GemmOut y;
+  float* h;
+  __nv_bfloat16* xn;
+  const __nv_bfloat16* gain;  // nullptr: skip the norm
+  int d;
+  float eps;
+};
+
+struct QkvArgs {
+  GemmOut y;
+  __nv_bfloat16* q;   // [T][Hq][hd]
+  __nv_bfloat16* kc;  // [Hkv][max_ctx][hd] of this layer
+  __nv_bfloat16* vc;
+  int Hq, Hkv, hd, max_ctx;
+  int pos0;
+  const int* pos0_dev;
+  double rope_theta;
+};
+
+struct SiluArgs {
+  GemmOut y;
+  __nv_bfloat16* out;  // [T][F]
+  int F;
+};
+
+struct StoreArgs {
+  GemmOut y;
+  float* out;
+  int N;
+  int ld;
+};
+
+struct RowStatsArgs {
+  const float* logits;  // [B][ld]
+  int ld;
+  int V;
+  int mask_id;
+  dlm_row_stats stats;
+  __nv_bfloat16* P;     // [B][V] or nullptr
+};
+
+struct CommitArgs {
+  const float* maxprob;
+  const int32_t* argmax;
+  int32_t* tokens;
+  uint8_t* committed;
+  float* s;
+  int32_t* round;
+  int32_t* status;
+  int B, d;
+  float tau;
+  int mode, k;
+  int use_cond;
+  cudaGraphConditionalHandle cond;
+};
+
+struct BlockInitArgs {
+  int32_t* tokens;
+  uint8_t* committed;
+  float* s;
+  int32_t* round;
+  int32_t* status;
+  int B, d, mask_id;
+};
+
+struct BlockFinishArgs {
+  const int32_t* tokens;
+  const int32_t* round;
+  const int32_t* status;
+  const int* err;
+  int32_t* tokens_out;
+  int32_t* rounds_out;
+  int* L_dev;
+  int B;
+};
+
+__global__ void k_embed_adapter_norm(EmbedArgs a);
+__global__ void k_residual_norm(ResidArgs a);
+__global__ void k_qkv_rope(QkvArgs a);
+__global__ void k_silu_gate(SiluArgs a);
+__global__ void k_store_rows(StoreArgs a);
+__global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n);
+__global__ void k_rowstats(RowStatsArgs a);
+__global__ void k_commit(CommitArgs a);
+__global__ void k_block_init(BlockInitArgs a);
+__global__ void k_block_finish(BlockFinishArgs a);
+__global__ void k_set_int(int* p, int v);
+__global__ void k_amax_to_scale(float* p);
+__global__ void k_amax_bf16(const __nv_bfloat16* w, long n, unsigned* amax_bits);
+__global__ void k_nvfp4_quantize(const __nv_bfloat16* w, int rows, int cols, uint8_t* codes,
+                                 uint8_t* scales, const unsigned* amax_bits, float* tscale);
+
+}  // namespace dlm

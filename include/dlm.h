@@ -1,0 +1,246 @@
+/* dlm.h -- C ABI of libdlm.so: residual block-diffusion decoding at batch size 1 on one
+ * B200 (sm_100a).
+ *
+ * What the library computes (sources cited by page title and section):
+ *   - Block-wise diffusion decoding: a block of B masked positions is refined by denoising
+ *     rounds; each round yields a distribution over the still-unresolved positions and the
+ *     block commits after enough rounds.  ["ORL: diffusion LLMs get a learnable 'tokens per
+ *     forward'" (richland.au blog), "What shipped", opening paragraph]
+ *   - Residual self-conditioning: the previous round's distribution P_prev is fed back
+ *     through an adapter on the tied embedding E.  This library fixes the adapter as
+ *     h0_i = E[x_i] + W_a (P_prev,i E), W_a of size d x d.  [same page, "What shipped",
+ *     "On-policy residual learning"]
+ *   - Block-diffusion attention: block queries attend causally to a prefix KV cache and
+ *     bidirectionally within the block (GQA, bf16 KV).  [model card "QwenDLM-4B-ORL"
+ *     (shadowgraph.io), "The paper's evaluation pipeline": --dllm-algorithm SDARPrefixKV]
+ *   - LM head fused with per-row statistics (max, argmax, logsumexp, max-prob, entropy)
+ *     so that logits are not a kernel output.  [same card and section:
+ *     SDAR_FUSED_ROW_STATS=1]
+ *   - Confidence-threshold commit: positions whose max-prob >= tau commit, at least the
+ *     single most confident one per round; a fixed top-k schedule is also offered.
+ *     [blog, "What shipped", "Adjacent entropy contraction": "more positions clear the
+ *     commit bar"; card: SDAR_COMMIT_GRAPH=1]
+ *   - One CUDA graph per block whose conditional (while) node decides after every round
+ *     whether to continue, so the host only launches the block and reads tokens back.
+ *     [blog, "What shipped", "dlmrt, the inference engine"]
+ *
+ * Conventions
+ *   - Every function returns a dlm_status (0 = DLM_OK), throws nothing and never exits.
+ *   - Device pointers are marked d_, host pointers h_.  The caller owns all memory:
+ *     weights, workspace, KV cache and block state.  The library keeps pointers only and
+ *     never allocates device memory.
+ *   - All device work is ordered on the stream passed in (cudaStream_t, passed as void*
+ *     so this header needs no CUDA include).  Only dlm_generate synchronizes.
+ *   - A context is not thread-safe.  Weights are read-only.
+ *   - Matrices are row-major bf16 "out x in" (PyTorch nn.Linear layout) unless stated.
+ */
+#ifndef DLM_H_
+#define DLM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int dlm_status;
+#define DLM_OK 0
+#define DLM_EINVAL 1        /* null pointer, bad dims, tau NaN, B outside [1,64], k < 1 */
+#define DLM_ENOMEM_WS 2     /* workspace or scratch too small */
+#define DLM_EKVCAP 3        /* L + B exceeds the KV capacity (max_ctx) */
+#define DLM_ECUDA 4         /* a CUDA runtime/driver error; see dlm_last_error */
+#define DLM_EROUNDCAP 5     /* a block reached B rounds with positions uncommitted */
+#define DLM_ETIMEOUT 6      /* a device-side bounded wait gave up (kernel returned early) */
+#define DLM_EUNSUPPORTED 7  /* shape or format this build does not handle */
+
+#define DLM_COMMIT_THRESHOLD 0 /* commit max-prob >= tau, at least one per round */
+#define DLM_COMMIT_TOPK 1      /* commit the top min(k, remaining) by max-prob */
+
+#define DLM_WEIGHTS_BF16 0
+#define DLM_WEIGHTS_NVFP4 1 /* MLP and LM head in NVFP4, attention projections bf16 */
+
+typedef struct dlm_config {
+  int n_layers;    /* transformer layers */
+  int d;           /* model width; multiple of 64 */
+  int n_q_heads;   /* query heads */
+  int n_kv_heads;  /* key/value heads; divides n_q_heads */
+  int head_dim;    /* 32, 64 or 128 */
+  int ffn;         /* SiLU-gated MLP width; multiple of 64 */
+  int vocab;       /* V; rows of the tied embedding */
+  int mask_id;     /* id of the mask token (embedded by its row of E, never predicted) */
+  int max_ctx;     /* KV capacity in positions */
+  int block_size;  /* B, in [1, 64] */
+  float rope_theta;/* RoPE base (NeoX rotate-half pairing (j, j + hd/2)) */
+  float rms_eps;   /* RMSNorm epsilon */
+  int weight_fmt;  /* DLM_WEIGHTS_BF16 or DLM_WEIGHTS_NVFP4 */
+} dlm_config;
+
+/* One NVFP4 matrix [rows][cols]: e2m1 codes (2 per byte, element 2j in the low nibble),
+ * one e4m3 scale per 16 consecutive elements of a row, and one fp32 tensor scale.
+ * Produced by dlm_nvfp4_quantize. */
+typedef struct dlm_nvfp4_matrix {
+  const void* codes;   /* device, uint8 [rows][cols/2] */
+  const void* scales;  /* device, uint8 [rows][cols/16] */
+  float tensor_scale;
+} dlm_nvfp4_matrix;
+
+typedef struct dlm_layer_weights {
+  const void* attn_norm; /* bf16 [d] */
+  const void* w_qkv;     /* bf16 [(Hq + 2 Hkv) hd][d]; rows: q heads, k heads, v heads */
+  const void* w_o;       /* bf16 [d][Hq hd] */
+  const void* mlp_norm;  /* bf16 [d] */
+  const void* w_gate;    /* bf16 [F][d] */
+  const void* w_up;      /* bf16 [F][d] */
+  const void* w_down;    /* bf16 [d][F] */
+  dlm_nvfp4_matrix q_gate, q_up, q_down; /* used when weight_fmt == DLM_WEIGHTS_NVFP4 */
+} dlm_layer_weights;
+
+typedef struct dlm_weights {
+  const void* embed;      /* E, bf16 [V][d]: token embedding and tied LM head */
+  const void* w_adapter;  /* W_a, bf16 [d][d] */
+  const void* final_norm; /* bf16 [d] */
+  const dlm_layer_weights* layers; /* host array [n_layers]; copied by dlm_ctx_create */
+  dlm_nvfp4_matrix q_embed; /* NVFP4 E for the LM head when weight_fmt == NVFP4 */
+} dlm_weights;
+
+/* Per-row statistics of one round, device arrays of length B. */
+typedef struct dlm_row_stats {
+  float* m;        /* max logit */
+  float* lse;      /* log-sum-exp */
+  float* maxprob;  /* exp(m - lse) */
+  float* entropy;  /* nats */
+  int32_t* argmax; /* lowest id among the maxima; the mask id is excluded */
+} dlm_row_stats;
+
+/* Caller-owned device state of one block (resumable: everything lives here). */
+typedef struct dlm_block_state {
+  int32_t* tokens;     /* [B]: mask_id or the committed id */
+  uint8_t* committed;  /* [B]: 0/1 */
+  float* s;            /* [B][d]: residual input P_prev E (zero rows where there is none) */
+  int32_t* round;      /* [1]: rounds done in this block */
+  int32_t* status;     /* [1]: 0 or a DLM_E* code raised on the device */
+  dlm_row_stats stats; /* written by every round */
+} dlm_block_state;
+
+typedef struct dlm_timing {
+  double prefill_ms;   /* prompt prefill */
+  double decode_ms;    /* all blocks, including KV-fill and per-block read-back */
+  int n_blocks;
+  int n_rounds;        /* denoising rounds in total */
+} dlm_timing;
+
+typedef struct dlm_ctx dlm_ctx;
+
+/* ---------------------------------------------------------------- context */
+/* Bytes of device workspace a context needs (256-byte aligned base). */
+size_t dlm_workspace_size(const dlm_config* cfg);
+/* Bytes of the bf16 KV cache: 2 * n_layers * n_kv_heads * max_ctx * head_dim * 2. */
+size_t dlm_kv_cache_size(const dlm_config* cfg);
+/* Validates cfg, copies the weight pointer table, carves the workspace.  The KV cache
+ * layout is [layer][K|V][kv_head][max_ctx][head_dim] bf16.  Sets the prefix length L = 0. */
+dlm_status dlm_ctx_create(const dlm_config* cfg, const dlm_weights* w, void* d_workspace,
+                          size_t ws_bytes, void* d_kv_cache, size_t kv_bytes, dlm_ctx** out);
+dlm_status dlm_ctx_destroy(dlm_ctx* ctx);
+/* Message of the last error on this context ("" if none); valid until the next call. */
+const char* dlm_last_error(const dlm_ctx* ctx);
+/* Current prefix length L (positions of the KV cache holding committed context). */
+int dlm_prefix_len(const dlm_ctx* ctx);
+/* Sets L (0 <= L <= max_ctx - B).  Rows >= L of the KV cache are treated as free. */
+dlm_status dlm_set_prefix_len(dlm_ctx* ctx, int L, void* stream);
+
+/* ---------------------------------------------------------------- decoding */
+/* Causal prefill of n prompt tokens at positions [L, L + n); L += n.  d_tokens int32 [n]. */
+dlm_status dlm_prefill(dlm_ctx* ctx, const int32_t* d_tokens, int n, void* stream);
+
+/* Initialises a block state: tokens = mask_id, committed = 0, s = 0, round = 0, status = 0. */
+dlm_status dlm_block_init(dlm_ctx* ctx, const dlm_block_state* st, void* stream);
+
+/* One denoising round over the block at prefix length L (L unchanged), updating the
+ * caller's state in place: embedding + residual adapter, the transformer layers with
+ * block-diffusion attention (block K/V written to cache rows [L, L+B)), fused LM head
+ * with row statistics and s = softmax(logits) E, then the commit rule.  tau is used by
+ * DLM_COMMIT_THRESHOLD, tpf_k by DLM_COMMIT_TOPK. */
+dlm_status dlm_round(dlm_ctx* ctx, const dlm_block_state* st, float tau, int commit_mode,
+                     int tpf_k, void* stream);
+
+/* Clean forward of a committed block (s = 0, no LM head) writing its K/V to rows
+ * [L, L+B); then L += B.  d_tokens int32 [B]. */
+dlm_status dlm_kv_fill(dlm_ctx* ctx, const int32_t* d_tokens, void* stream);
+
+/* Decodes one whole block on the device: one launch of a CUDA graph that initialises
+ * the block, loops rounds in a while-conditional node until every position is committed
+ * (or B rounds), then runs the KV-fill forward.  Writes d_tokens_out int32 [B] and
+ * d_rounds_out int32 [2] = {rounds, device status}.  L += B (host and device).  The graph
+ * is instantiated on first use per (commit mode, tau, k) and reused. */
+dlm_status dlm_decode_block(dlm_ctx* ctx, float tau, int commit_mode, int tpf_k,
+                            int32_t* d_tokens_out, int32_t* d_rounds_out, void* stream);
+
+/* Host-level generation: copies the prompt to the device, prefills it at L = 0, decodes
+ * ceil(max_new / B) blocks with dlm_decode_block, reading each block's tokens back, and
+ * returns max_new tokens (the last block truncated) and the rounds of every block.
+ * Synchronizes.  h_prompt int32 [prompt_len]; h_tokens_out int32 [max_new];
+ * h_rounds_per_block int32 [ceil(max_new/B)] (may be NULL); h_timing may be NULL. */
+dlm_status dlm_generate(dlm_ctx* ctx, const int32_t* h_prompt, int prompt_len, int max_new,
+                        float tau, int commit_mode, int tpf_k, int32_t* h_tokens_out,
+                        int32_t* h_rounds_per_block, dlm_timing* h_timing, void* stream);
+
+/* ---------------------------------------------------------------- single operations
+ * Stand-alone entry points of the kernels one round is made of, used by the parity tests
+ * and the per-kernel benchmarks.  `scratch` is caller-owned device memory of at least
+ * the size the matching *_scratch_size function returns. */
+
+/* y[T][N] (fp32) = x[T][K] (bf16) W[N][K]^T (bf16) on the tensor cores.  T <= 256,
+ * K % 8 == 0, K >= 64.  d_y may be NULL: then only the tensor-core kernel runs and its
+ * fp32 partial sums stay in the scratch (used to time that kernel alone). */
+size_t dlm_gemm_scratch_size(int T, int N, int K);
+dlm_status dlm_gemm_bf16(const void* d_x, const void* d_w, float* d_y, int T, int N, int K,
+                         void* d_scratch, size_t scratch_bytes, void* stream);
+
+/* LM head fused with row statistics and the residual contraction:
+ *   logits = x E^T (x: bf16 [B][d], already normalised), stats of every row with the
+ *   mask id excluded (mask_id < 0: none excluded), and s = P E with P = softmax(logits)
+ *   (d_p_given == NULL) or P = d_p_given (bf16 [B][V]).  s: fp32 [B][d]. */
+size_t dlm_lmhead_scratch_size(int B, int V, int d);
+dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int V, int d,
+                               int mask_id, const void* d_p_given, dlm_row_stats stats,
+                               float* d_s, void* d_scratch, size_t scratch_bytes, void* stream);
+
+/* Adapter step: h0[B][d] (fp32) = E[tokens] + W_a bf16(s), s fp32 [B][d]. */
+size_t dlm_adapter_scratch_size(int B, int d);
+dlm_status dlm_adapter_embed(const void* d_embed, const void* d_w_adapter, const int32_t* d_tokens,
+                             const float* d_s, float* d_h0, int B, int d, void* d_scratch,
+                             size_t scratch_bytes, void* stream);
+
+/* Block-diffusion attention of one layer: T queries at positions [L, L+T) against the
+ * cache rows [0, L+T) of one layer (causal != 0: query at position p sees keys [0, p]).
+ * q bf16 [T][Hq][hd]; k_cache, v_cache bf16 [Hkv][max_ctx][hd]; o bf16 [T][Hq][hd]. */
+size_t dlm_attention_scratch_size(int T, int Hq, int hd, int max_ctx);
+dlm_status dlm_bd_attention(const void* d_q, const void* d_k_cache, const void* d_v_cache,
+                            void* d_o, int T, int L, int Hq, int Hkv, int hd, int max_ctx,
+                            int causal, void* d_scratch, size_t scratch_bytes, void* stream);
+
+/* Commit rule on device arrays (one block of B positions).  Updates tokens, committed,
+ * zeroes the s rows of newly committed positions, increments *d_round. */
+dlm_status dlm_commit(const float* d_maxprob, const int32_t* d_argmax, int32_t* d_tokens,
+                      uint8_t* d_committed, float* d_s, int32_t* d_round, int32_t* d_status,
+                      int B, int d, float tau, int commit_mode, int tpf_k, void* stream);
+
+/* NVFP4 quantizer (per-tensor fp32 scale amax / (6 * 448), e4m3 scale per 16 elements,
+ * round-to-nearest-even e2m1 codes) of a bf16 [rows][cols] matrix, cols % 16 == 0.
+ * Writes codes uint8 [rows][cols/2], scales uint8 [rows][cols/16], *d_tensor_scale. */
+dlm_status dlm_nvfp4_quantize(const void* d_w, int rows, int cols, void* d_codes, void* d_scales,
+                              float* d_tensor_scale, void* stream);
+
+/* Version string of the build. */
+const char* dlm_version(void);
+
+/* Debugging aid: 0 (default) runs the dense projections on the tcgen05 tensor-core GEMM,
+ * 1 on a plain CUDA-core kernel with the same output contract (slow; for cross-checks). */
+void dlm_debug_set_gemm_impl(int impl);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DLM_H_ */

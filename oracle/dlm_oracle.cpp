@@ -216,6 +216,7 @@ typedef struct orc_kv {
 typedef struct orc_stats {
   double m, lse, maxprob, entropy;
   int argmax;
+  double gap2;  // largest minus second-largest logit (ambiguity of the argmax)
 } orc_stats;
 
 void orc_set_threads(int n) { g_threads = n; }
@@ -313,15 +314,20 @@ void linear(const double* x, int T, const orc_mat& W, double* y, bool act_fp4) {
     for (int t = 0; t < T; ++t) quantize_act_row(x + size_t(t) * K, K, xq.data() + size_t(t) * K);
     xin = xq.data();
   }
+  // x transposed to [K][T] so that the T sums of one weight row advance together; every
+  // output is still the plain sum over k = 0 .. K-1 in ascending order.
+  std::vector<double> xt(size_t(K) * T);
+  for (int t = 0; t < T; ++t)
+    for (int k = 0; k < K; ++k) xt[size_t(k) * T + t] = xin[size_t(t) * K + k];
   parallel_for(N, [&](long n) {
-    std::vector<double> w(K);
+    std::vector<double> w(K), acc(T, 0.0);
     mat_row(W, n, w.data());
-    for (int t = 0; t < T; ++t) {
-      double acc = 0.0;
-      const double* xr = xin + size_t(t) * K;
-      for (int k = 0; k < K; ++k) acc += xr[k] * w[k];
-      y[size_t(t) * N + n] = acc;
+    for (int k = 0; k < K; ++k) {
+      const double wk = w[k];
+      const double* xk = xt.data() + size_t(k) * T;
+      for (int t = 0; t < T; ++t) acc[t] += xk[t] * wk;
     }
+    for (int t = 0; t < T; ++t) y[size_t(t) * N + n] = acc[t];
   });
 }
 
@@ -417,6 +423,10 @@ void orc_rowstats(const double* logits, int B, int V, int mask_id, orc_stats* st
       double p = std::exp(lp);
       if (p > 0.0) H -= p * lp;
     }
+    double second = -std::numeric_limits<double>::infinity();
+    for (int v = 0; v < V; ++v)
+      if (v != mask_id && v != am) second = std::max(second, l[v]);
+    st[b].gap2 = m - second;
     st[b].m = m;
     st[b].lse = lse;
     st[b].maxprob = std::exp(m - lse);

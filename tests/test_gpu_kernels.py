@@ -1,0 +1,222 @@
+"""Per-kernel parity of the CUDA path (through the C ABI) against the CPU oracle, on
+seeded inputs: the tensor-core GEMM, block-diffusion attention (the attention sweep
+shapes), the fused LM head with row statistics and P E (the single-round LM-head
+workload), the residual adapter, the commit rule and the NVFP4 quantizer."""
+import numpy as np
+import pytest
+
+import oracle as O
+from block_diffusion_decoding_denoising_b200 import gen
+from helpers import (RTOL_BF16, assert_close, bf16_f64, from_torch_bf16, rel_err, to_torch_bf16,
+                     unambiguous_argmax)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from block_diffusion_decoding_denoising_b200 import build, dlm
+    build.build()
+    dlm.lib()
+    return dlm
+
+
+def _bits(seed, shape, std=1.0):
+    return gen.bf16_bits(gen.normal_np(seed, int(np.prod(shape)), std).reshape(shape))
+
+
+# ------------------------------------------------------------------ GEMM
+GEMM_SHAPES = [(32, 6144, 2560), (32, 2560, 9728), (8, 200, 320), (5, 64, 64), (33, 300, 1000),
+               (100, 384, 192), (200, 256, 512), (256, 130, 128), (1, 128, 64), (64, 19456, 256)]
+
+
+@pytest.mark.parametrize("T,N,K", GEMM_SHAPES)
+def test_gemm_tcgen05_parity(lib, T, N, K):
+    xb = _bits(100 + T, (T, K))
+    wb = _bits(200 + N, (N, K), 0.02)
+    y = lib.gemm_bf16(to_torch_bf16(xb), to_torch_bf16(wb)).cpu().numpy().astype(np.float64)
+    ref = O.linear(bf16_f64(xb), wb)
+    # identical bf16 operands: only the fp32 accumulation order differs
+    assert_close(y, ref, 1e-3, "gemm %dx%dx%d" % (T, N, K))
+
+
+def test_gemm_cuda_core_debug_path_matches(lib):
+    T, N, K = 16, 300, 256
+    xb = _bits(7, (T, K))
+    wb = _bits(8, (N, K), 0.02)
+    lib.set_gemm_impl(1)
+    try:
+        y = lib.gemm_bf16(to_torch_bf16(xb), to_torch_bf16(wb)).cpu().numpy()
+    finally:
+        lib.set_gemm_impl(0)
+    assert_close(y, O.linear(bf16_f64(xb), wb), 1e-3, "simt gemm")
+
+
+# ------------------------------------------------------------------ attention
+def _attn_case(lib, B, L, Hq=32, Hkv=8, hd=128, causal=False, rows=None, seed=0):
+    import torch
+    q, k, v = gen.attention_inputs_torch(B, L, Hq, Hkv, hd, seed=seed)
+    o = lib.bd_attention(q, k, v, L, causal=causal)
+    torch.cuda.synchronize()
+    qf = bf16_f64(from_torch_bf16(q))
+    kf = bf16_f64(from_torch_bf16(k))
+    vf = bf16_f64(from_torch_bf16(v))
+    of = bf16_f64(from_torch_bf16(o))
+    if rows is None:
+        ref = O.attention(qf, kf, vf, L, causal)
+        return of, ref
+    # sampled query rows: non-causal queries all see keys [0, L + B), so a subset of
+    # rows is evaluated at pos0 = L + B - len(rows) with the same key range
+    sel = np.array(rows)
+    ref = O.attention(qf[sel], kf, vf, L + B - len(sel), False)
+    return of[sel], ref
+
+
+@pytest.mark.parametrize("B", [4, 16, 32, 64])
+@pytest.mark.parametrize("L", [1024, 4096])
+def test_attention_sweep_full(lib, B, L):
+    got, ref = _attn_case(lib, B, L)
+    assert_close(got, ref, RTOL_BF16, "attention B=%d L=%d" % (B, L))
+
+
+@pytest.mark.parametrize("B", [4, 16, 32, 64])
+@pytest.mark.parametrize("L", [16384, 65536])
+def test_attention_sweep_sampled_rows(lib, B, L):
+    rows = sorted({0, B // 2, B - 1})
+    got, ref = _attn_case(lib, B, L, rows=rows)
+    assert_close(got, ref, RTOL_BF16, "attention B=%d L=%d rows %s" % (B, L, rows))
+
+
+def test_attention_empty_prefix_and_tiny_heads(lib):
+    got, ref = _attn_case(lib, 8, 0, Hq=2, Hkv=1, hd=32)
+    assert_close(got, ref, RTOL_BF16, "L=0 tiny heads")
+    got, ref = _attn_case(lib, 1, 0, Hq=4, Hkv=4, hd=64)
+    assert_close(got, ref, RTOL_BF16, "one query, MHA")
+
+
+@pytest.mark.parametrize("T,L", [(100, 37), (256, 0), (64, 300)])
+def test_attention_causal_prefill(lib, T, L):
+    got, ref = _attn_case(lib, T, L, Hq=8, Hkv=2, hd=128, causal=True)
+    assert_close(got, ref, RTOL_BF16, "causal T=%d L=%d" % (T, L))
+
+
+# ------------------------------------------------------------------ LM head + row stats + P E
+def _check_stats(st, ref, what, logits=None):
+    for k in ("m", "lse", "maxprob", "entropy"):
+        assert_close(st[k].cpu().numpy(), ref[k], RTOL_BF16, "%s %s" % (what, k))
+    am = st["argmax"].cpu().numpy()
+    ok = np.ones(len(am), bool) if logits is None else unambiguous_argmax(logits)
+    assert np.array_equal(am[ok], ref["argmax"][ok]), what + " argmax"
+
+
+@pytest.mark.parametrize("B,V,d,mask", [(8, 1000, 192, 999), (3, 520, 64, -1), (32, 4096, 256, 4095)])
+def test_lmhead_small(lib, B, V, d, mask):
+    xb = _bits(11, (B, d))
+    Eb = _bits(12, (V, d), 0.1)
+    st = lib.lmhead_rowstats(to_torch_bf16(xb), to_torch_bf16(Eb), mask_id=mask)
+    ref = O.lmhead(bf16_f64(xb), Eb, mask_id=mask, want_logits=True)
+    _check_stats(st, ref, "lmhead", ref["logits"])
+    assert_close(st["s"].cpu().numpy(), ref["s"], RTOL_BF16, "s")
+
+
+def test_lmhead_given_p(lib):
+    import torch
+    B, V, d = 4, 640, 128
+    xb = _bits(13, (B, d))
+    Eb = _bits(14, (V, d), 0.1)
+    z = np.exp(gen.normal_np(15, B * V, 3.0).reshape(B, V))
+    Pb = gen.bf16_bits(z / z.sum(1, keepdims=True))
+    st = lib.lmhead_rowstats(to_torch_bf16(xb), to_torch_bf16(Eb), p_given=to_torch_bf16(Pb))
+    ref = O.lmhead(bf16_f64(xb), Eb, p_given=bf16_f64(Pb), want_logits=True)
+    _check_stats(st, ref, "lmhead given P", ref["logits"])
+    assert_close(st["s"].cpu().numpy(), ref["s"], RTOL_BF16, "s = P E")
+
+
+def test_lmhead_one_hot_p_reproduces_rows_exactly(lib):
+    B, V, d = 2, 1024, 256
+    xb = _bits(16, (B, d))
+    Eb = _bits(17, (V, d), 0.1)
+    P = np.zeros((B, V))
+    P[0, 5] = 1.0
+    P[1, 1000] = 1.0
+    st = lib.lmhead_rowstats(to_torch_bf16(xb), to_torch_bf16(Eb), p_given=to_torch_bf16(gen.bf16_bits(P)))
+    s = st["s"].cpu().numpy().astype(np.float64)
+    np.testing.assert_array_equal(s[0], bf16_f64(Eb)[5])
+    np.testing.assert_array_equal(s[1], bf16_f64(Eb)[1000])
+
+
+def test_lmhead_single_round_4b_shapes(lib):
+    """Single round at 4B-class shapes: B=32, d=2560, V=151936, P_prev given."""
+    import torch
+    B, d, V = 32, 2560, 151936
+    H, E, Wa, P = gen.lmhead_inputs_torch(B, d, V)
+    x = H.to(torch.bfloat16)
+    st = lib.lmhead_rowstats(x, E, mask_id=V - 1, p_given=P)
+    st2 = lib.lmhead_rowstats(x, E, mask_id=V - 1)
+    torch.cuda.synchronize()
+    xb, Eb, Pb = from_torch_bf16(x), from_torch_bf16(E), from_torch_bf16(P)
+    ref = O.lmhead(bf16_f64(xb), Eb, mask_id=V - 1, p_given=bf16_f64(Pb), want_logits=True)
+    _check_stats(st, ref, "4b lmhead", ref["logits"])
+    assert_close(st["s"].cpu().numpy(), ref["s"], RTOL_BF16, "4b s = P_prev E")
+    ref2 = O.lmhead(bf16_f64(xb), Eb, mask_id=V - 1)
+    assert_close(st2["s"].cpu().numpy(), ref2["s"], RTOL_BF16, "4b s = softmax E")
+
+
+# ------------------------------------------------------------------ adapter
+@pytest.mark.parametrize("B,d,V", [(32, 2560, 1000), (8, 64, 512)])
+def test_adapter_embed(lib, B, d, V):
+    import torch
+    Eb = _bits(20, (V, d), 0.02)
+    Wab = _bits(21, (d, d), 0.02)
+    s = gen.normal_np(22, B * d, 0.05).reshape(B, d)
+    tok = gen.uniform_tokens_np(23, B, 0, V)
+    h0 = lib.adapter_embed(to_torch_bf16(Eb), to_torch_bf16(Wab), torch.from_numpy(tok).cuda(),
+                           torch.from_numpy(s.astype(np.float32)).cuda()).cpu().numpy()
+    s32 = s.astype(np.float32).astype(np.float64)
+    s_bf = np.array([O.round_bf16(v) for v in s32.reshape(-1)]).reshape(B, d)
+    ref = bf16_f64(Eb)[tok] + O.linear(s_bf, Wab)
+    assert_close(h0, ref, 1e-3, "adapter")
+
+
+# ------------------------------------------------------------------ commit
+@pytest.mark.parametrize("case", range(12))
+def test_commit_matches_oracle(lib, case):
+    import torch
+    B, d = [8, 32, 64, 1][case % 4], 16
+    rng = np.random.default_rng(case)
+    mp = rng.random(B).astype(np.float32)
+    if case % 3 == 0:
+        mp[: B // 2] = mp[0]  # ties
+    am = rng.integers(0, 500, B).astype(np.int32)
+    com = (rng.random(B) < 0.3).astype(np.uint8)
+    if com.all():
+        com[0] = 0
+    tok = np.where(com == 1, rng.integers(0, 500, B), 511).astype(np.int32)
+    mode = case % 2
+    tau = [0.5, 0.95, 1.5, 0.0][case % 4]
+    k = [1, 3, 11][case % 3]
+    s = np.ones((B, d), np.float32)
+    t = {n: torch.from_numpy(v).cuda() for n, v in dict(mp=mp, am=am, tok=tok.copy(), com=com.copy(), s=s).items()}
+    rnd = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lib.commit(t["mp"], t["am"], t["tok"], t["com"], t["s"], rnd, tau, mode, k)
+    n, rtok, rcom = O.commit(mp.astype(np.float64), am, tau, mode, k, tok, com)
+    np.testing.assert_array_equal(t["com"].cpu().numpy(), rcom)
+    np.testing.assert_array_equal(t["tok"].cpu().numpy(), rtok)
+    srow = t["s"].cpu().numpy()
+    assert np.all(srow[rcom == 1] == 0) and np.all(srow[rcom == 0] == 1)
+    assert int(rnd.item()) == 1
+
+
+# ------------------------------------------------------------------ NVFP4 quantizer
+@pytest.mark.parametrize("rows,cols,std", [(64, 256, 0.02), (9728, 2560, 0.02), (5, 48, 3.0)])
+def test_nvfp4_quantizer_bit_exact(lib, rows, cols, std):
+    import torch
+    wb = _bits(30 + rows, (rows, cols), std)
+    codes, scales, ts = lib.nvfp4_quantize(to_torch_bf16(wb))
+    torch.cuda.synchronize()
+    rc, rs, rS = O.nvfp4_quantize(bf16_f64(wb).astype(np.float32))
+    assert np.float32(ts.item()) == np.float32(rS)
+    np.testing.assert_array_equal(scales.cpu().numpy(), rs)
+    np.testing.assert_array_equal(codes.cpu().numpy(), rc)

@@ -1,0 +1,297 @@
+"""Model-level parity of the CUDA path against the CPU oracle: prefill KV, denoising
+rounds in lock-step (the oracle's state injected every round), free-running decoding
+until the first ambiguous event, the per-block CUDA graph against eager rounds, and
+dlm_generate.  Integer decisions (argmax ids, commit masks, round counts) must be
+bit-exact except where the oracle's own numbers make them ambiguous: top-2 logit gap
+below 1e-3, max-prob within 1e-3 of tau, or a ranking boundary (min-1 / top-k) between
+max-probs within a relative 1e-3."""
+import numpy as np
+import pytest
+
+import oracle as O
+from block_diffusion_decoding_denoising_b200 import gen
+from helpers import RTOL_BF16, assert_close, bf16_f64, from_torch_bf16, rel_err, to_torch_bf16
+
+pytestmark = pytest.mark.gpu
+
+GAP = 1e-3
+
+
+@pytest.fixture(scope="module")
+def dlm():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from block_diffusion_decoding_denoising_b200 import build, dlm as D
+    build.build()
+    D.lib()
+    return D
+
+
+def torch_weights(w_np):
+    out = {k: to_torch_bf16(w_np[k]) for k in ("embed", "w_adapter", "final_norm")}
+    out["layers"] = [{k: to_torch_bf16(v) for k, v in l.items()} for l in w_np["layers"]]
+    return out
+
+
+def small_model(std=0.02, n_layers=1, d=64, Hq=2, Hkv=1, hd=32, F=256, V=512, B=8, seed=0, max_ctx=256):
+    cfg = dict(n_layers=n_layers, d=d, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=hd, ffn=F, vocab=V,
+               mask_id=V - 1, max_ctx=max_ctx, block_size=B, rope_theta=10000.0, rms_eps=1e-6, weight_fmt=0)
+    w = gen.model_weights_np(cfg, seed, std=std, embed_std=8.0 / np.sqrt(d))
+    return cfg, w
+
+
+MODELS = {
+    "tiny": lambda: small_model(0.02),                      # the tiny oracle-scale model as specified
+    "tiny_distinct": lambda: small_model(0.125),            # larger layer weights: distinct positions
+    "two_layer_gqa": lambda: small_model(0.06, n_layers=2, d=256, Hq=4, Hkv=2, hd=64, F=512, V=1024, B=16),
+}
+
+
+def inject_kv(m, orc, upto):
+    import torch
+    kv = m.kv_view()
+    kv[:, 0, :, :upto] = torch.from_numpy(orc.kc[:, :, :upto]).to(torch.bfloat16).cuda()
+    kv[:, 1, :, :upto] = torch.from_numpy(orc.vc[:, :, :upto]).to(torch.bfloat16).cuda()
+
+
+def set_state(st, tokens, committed, s, rnd):
+    import torch
+    st["tokens"].copy_(torch.from_numpy(np.ascontiguousarray(tokens, np.int32)))
+    st["committed"].copy_(torch.from_numpy(np.ascontiguousarray(committed, np.uint8)))
+    st["s"].copy_(torch.from_numpy(np.ascontiguousarray(s, np.float32)))
+    st["round"].fill_(int(rnd))
+    st["status"].zero_()
+
+
+def ambiguous(stats, committed, tau, mode, k):
+    """Per-position ambiguity mask of one round's decisions, from the oracle's numbers,
+    and whether the round's selection as a whole is ambiguous."""
+    mp = stats["maxprob"]
+    amb = stats["gap2"] < GAP
+    unc = np.where(committed == 0)[0]
+    whole = False
+    if len(unc) == 0:
+        return amb, whole
+    if mode == 0:
+        near = np.abs(mp - tau) < GAP
+        amb = amb | near
+        clear_q = [i for i in unc if mp[i] >= tau and not near[i]]
+        maybe_q = [i for i in unc if near[i]]
+        if not clear_q:
+            if maybe_q:
+                whole = True  # the min-1 fallback may or may not trigger
+            else:
+                top = np.sort(mp[unc])[::-1]
+                if len(top) > 1 and top[0] - top[1] <= GAP * top[0]:
+                    whole = True
+    else:
+        top = np.sort(mp[unc])[::-1]
+        kk = min(k, len(unc))
+        if kk < len(unc) and top[kk - 1] - top[kk] <= GAP * top[kk - 1]:
+            whole = True
+    return amb, whole
+
+
+def lockstep(D, name, mode, tau, k, prompt_len=32, n_blocks=2):
+    import torch
+    cfg, w = MODELS[name]()
+    B, d = cfg["block_size"], cfg["d"]
+    orc = O.OracleModel(cfg, w, act_round=True)
+    prompt = gen.prompt_np(cfg, prompt_len)
+    orc.prefill(prompt)
+    m = D.Model(cfg, torch_weights(w))
+    m.set_prefix_len(prompt_len)
+    st = m.new_block_state()
+    report = dict(rounds=0, whole_ambiguous=0, compared=0)
+    L = prompt_len
+    for blk in range(n_blocks):
+        inject_kv(m, orc, L)
+        tok = np.full(B, cfg["mask_id"], np.int32)
+        com = np.zeros(B, np.uint8)
+        s = np.zeros((B, d))
+        rnd = 0
+        while not com.all() and rnd < B:
+            set_state(st, tok, com, s, rnd)
+            m.round(st, tau, mode, k)
+            n, new, ost = orc.round(tok, com, s, rnd, L, tau, mode, k)
+            torch.cuda.synchronize()
+            gst = {key: st["stats"][key].cpu().numpy() for key in st["stats"]}
+            for key in ("m", "lse", "maxprob", "entropy"):
+                assert_close(gst[key], ost[key], RTOL_BF16, "%s round %d %s" % (name, rnd, key))
+            amb, whole = ambiguous(ost, com, tau, mode, k)
+            ok = ~amb
+            assert np.array_equal(gst["argmax"][ok], ost["argmax"][ok]), "argmax round %d" % rnd
+            gcom = st["committed"].cpu().numpy()
+            gtok = st["tokens"].cpu().numpy()
+            report["rounds"] += 1
+            if whole:
+                report["whole_ambiguous"] += 1
+            else:
+                sel = ok | (com == 1)
+                assert np.array_equal(gcom[sel], new["committed"][sel]), "commit mask round %d" % rnd
+                both = sel & (new["committed"] == 1)
+                assert np.array_equal(gtok[both], new["tokens"][both]), "tokens round %d" % rnd
+                report["compared"] += 1
+                assert int(st["round"].item()) == rnd + 1
+            unc_rows = new["committed"] == 0
+            gs = st["s"].cpu().numpy()
+            if unc_rows.any() and not whole:
+                assert_close(gs[unc_rows & (gcom == 0)], new["s"][unc_rows & (gcom == 0)], RTOL_BF16, "s")
+            tok, com, s, rnd = new["tokens"], new["committed"], new["s"], new["round"]
+        assert com.all()
+        # both sides write the committed block's K/V with a clean forward
+        orc.forward(tok, None, L, want_xf=False)
+        m.set_prefix_len(L)
+        m.kv_fill(torch.from_numpy(tok).cuda())
+        torch.cuda.synchronize()
+        kv = m.kv_view()
+        gk = kv[:, 0, :, L:L + B].float().cpu().numpy()
+        assert_close(gk, orc.kc[:, :, L:L + B], RTOL_BF16, "kv fill K")
+        L += B
+    assert report["compared"] >= report["rounds"] // 2, report
+    return report
+
+
+@pytest.mark.parametrize("name", list(MODELS))
+def test_prefill_kv_parity(dlm, name):
+    import torch
+    cfg, w = MODELS[name]()
+    P = 40
+    prompt = gen.prompt_np(cfg, P)
+    orc = O.OracleModel(cfg, w, act_round=True)
+    orc.prefill(prompt)
+    m = dlm.Model(cfg, torch_weights(w))
+    m.prefill(torch.from_numpy(prompt).cuda())
+    torch.cuda.synchronize()
+    assert m.prefix_len == P
+    kv = m.kv_view()
+    assert_close(kv[:, 0, :, :P].float().cpu().numpy(), orc.kc[:, :, :P], RTOL_BF16, "prefill K")
+    assert_close(kv[:, 1, :, :P].float().cpu().numpy(), orc.vc[:, :, :P], RTOL_BF16, "prefill V")
+
+
+@pytest.mark.parametrize("name", list(MODELS))
+@pytest.mark.parametrize("mode,tau,k", [(0, 0.9, 1), (1, 0.0, 3)])
+def test_round_lockstep(dlm, name, mode, tau, k):
+    lockstep(dlm, name, mode, tau, k)
+
+
+def test_graph_decode_matches_eager_rounds(dlm):
+    """The per-block CUDA graph (while node) and eager dlm_round calls run the same
+    kernels on the same inputs: tokens, round counts and the KV cache must be identical."""
+    import torch
+    cfg, w = MODELS["tiny_distinct"]()
+    B = cfg["block_size"]
+    prompt = torch.from_numpy(gen.prompt_np(cfg, 32)).cuda()
+    tw = torch_weights(w)
+    a = dlm.Model(cfg, tw)
+    a.prefill(prompt)
+    b = dlm.Model(cfg, tw)
+    b.prefill(prompt)
+    st = b.new_block_state()
+    for blk in range(3):
+        tok_a = torch.zeros(B, dtype=torch.int32, device="cuda")
+        rr = torch.zeros(2, dtype=torch.int32, device="cuda")
+        a.decode_block(0.9, 0, 1, tok_a, rr)
+        b.block_init(st)
+        rounds = 0
+        while True:
+            b.round(st, 0.9, 0, 1)
+            rounds += 1
+            if bool(st["committed"].all().item()) or rounds >= B:
+                break
+        b.kv_fill(st["tokens"])
+        torch.cuda.synchronize()
+        assert np.array_equal(tok_a.cpu().numpy(), st["tokens"].cpu().numpy())
+        assert int(rr[0].item()) == rounds and int(rr[1].item()) == 0
+        assert a.prefix_len == b.prefix_len == 32 + (blk + 1) * B
+    assert torch.equal(a.kv_view(), b.kv_view())
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_distinct"])
+def test_generate_free_running_vs_oracle(dlm, name):
+    """dlm_generate against the oracle's block loop, round by round; the comparison
+    stops at the first ambiguous event (after it the trajectories may legitimately part)."""
+    import torch
+    cfg, w = MODELS[name]()
+    B, d = cfg["block_size"], cfg["d"]
+    P, n_blocks, tau = 32, 4, 0.9
+    prompt = gen.prompt_np(cfg, P)
+    m = dlm.Model(cfg, torch_weights(w))
+    out, rpb, tm = m.generate(prompt, n_blocks * B, tau)
+    assert tm.n_blocks == n_blocks and tm.n_rounds == int(rpb.sum())
+    assert np.all((out >= 0) & (out < cfg["vocab"] - 1))
+    orc = O.OracleModel(cfg, w, act_round=True)
+    orc.prefill(prompt)
+    L = P
+    for blk in range(n_blocks):
+        tok = np.full(B, cfg["mask_id"], np.int32)
+        com = np.zeros(B, np.uint8)
+        s = np.zeros((B, d))
+        rnd = 0
+        while not com.all():
+            n, new, ost = orc.round(tok, com, s, rnd, L, tau, 0, 1)
+            amb, whole = ambiguous(ost, com, tau, 0, 1)
+            newly = (new["committed"] == 1) & (com == 0)
+            if whole or amb[newly].any() or amb[com == 0].any():
+                return  # ambiguous event: parity is only claimed up to here
+            tok, com, s, rnd = new["tokens"], new["committed"], new["s"], new["round"]
+        assert rpb[blk] == rnd, "block %d rounds" % blk
+        assert np.array_equal(out[blk * B:(blk + 1) * B], tok), "block %d tokens" % blk
+        orc.forward(tok, None, L, want_xf=False)
+        L += B
+
+
+def test_generate_truncates_and_reports_status(dlm):
+    import torch
+    cfg, w = MODELS["tiny_distinct"]()
+    m = dlm.Model(cfg, torch_weights(w))
+    prompt = gen.prompt_np(cfg, 16)
+    out, rpb, tm = m.generate(prompt, 13, 0.9, mode=1, k=3)
+    assert out.shape == (13,) and len(rpb) == 2 and np.all(rpb == 3)
+    # capacity check: prompt + blocks beyond max_ctx
+    with pytest.raises(dlm.DlmError) as e:
+        m.generate(np.zeros(cfg["max_ctx"] - 4, np.int32), 8, 0.9)
+    assert e.value.status == dlm.DLM_EKVCAP
+    with pytest.raises(dlm.DlmError) as e:
+        m.generate(prompt, 8, float("nan"))
+    assert e.value.status == dlm.DLM_EINVAL
+
+
+def test_round_4b_lockstep_sampled(dlm):
+    """One lock-step round of the 4B-class model (36 layers, d=2560, V=151936) at prefix
+    length 512.  The prefix K/V is a seeded synthetic input shared by both sides."""
+    import torch
+    cfg = gen.config_4b(max_ctx=512 + 32)
+    B, d, L = cfg["block_size"], cfg["d"], 512
+    tw = gen.model_weights_torch(cfg, seed=0, device="cuda")
+    m = dlm.Model(cfg, tw)
+    kv = m.kv_view()
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1234)
+    kv[:, :, :, :L] = torch.randn(kv[:, :, :, :L].shape, generator=g, device="cuda").to(torch.bfloat16)
+    m.set_prefix_len(L)
+    st = m.new_block_state()
+    # round 1 state: a few committed positions, a residual s on the others
+    rng = np.random.default_rng(0)
+    com = (rng.random(B) < 0.25).astype(np.uint8)
+    tok = np.where(com == 1, rng.integers(0, cfg["vocab"] - 1, B), cfg["mask_id"]).astype(np.int32)
+    s = np.where(com[:, None] == 1, 0.0, rng.normal(0, 0.02, (B, d))).astype(np.float32)
+    set_state(st, tok, com, s, 1)
+    m.round(st, 0.9, 0, 1)
+    torch.cuda.synchronize()
+    w_np = {k: from_torch_bf16(tw[k]) for k in ("embed", "w_adapter", "final_norm")}
+    w_np["layers"] = [{k: from_torch_bf16(v) for k, v in l.items()} for l in tw["layers"]]
+    orc = O.OracleModel(cfg, w_np, act_round=True, max_ctx=L + B)
+    kvh = kv[:, :, :, :L].float().cpu().numpy()
+    orc.kc[:, :, :L] = kvh[:, 0]
+    orc.vc[:, :, :L] = kvh[:, 1]
+    n, new, ost = orc.round(tok, com, s.astype(np.float64), 1, L, 0.9, 0, 1)
+    gst = {key: st["stats"][key].cpu().numpy() for key in st["stats"]}
+    for key in ("m", "lse", "maxprob", "entropy"):
+        assert_close(gst[key], ost[key], RTOL_BF16, "4b " + key)
+    amb, whole = ambiguous(ost, com, 0.9, 0, 1)
+    assert np.array_equal(gst["argmax"][~amb], ost["argmax"][~amb])
+    if not whole:
+        assert np.array_equal(st["committed"].cpu().numpy(), new["committed"])
+    unc = (new["committed"] == 0) & (st["committed"].cpu().numpy() == 0)
+    assert_close(st["s"].cpu().numpy()[unc], new["s"][unc], RTOL_BF16, "4b s")
