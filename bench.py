@@ -42,6 +42,10 @@ def parse():
     ap.add_argument("--impl", default="dlm", choices=["dlm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=36, help=argparse.SUPPRESS)
+    # profiling cases (small, for ncu): "quick" = the decode loop on 256 generated tokens
+    # without the extra measurements; "gemm" = every projection GEMM of two layers plus
+    # the LM-head GEMM, `--steps` launches each
+    ap.add_argument("--case", default="full", choices=["full", "quick", "gemm"])
     return ap.parse_args()
 
 
@@ -180,9 +184,47 @@ def workload_config(cfg):
 
 
 # ------------------------------------------------------------------ main arm
+def gemm_case(args):
+    """Every projection GEMM of two 4B-class layers and the LM-head GEMM, with the split
+    activations a round uses (T = 32), `--steps` launches each: a small ncu target."""
+    import ctypes as C
+
+    import torch
+
+    from block_diffusion_decoding_denoising_b200 import build, dlm, gen
+    build.build()
+    cfg = gen.config_4b(n_layers=2)
+    w = gen.model_weights_torch(cfg, seed=0, device="cuda")
+    L = dlm.lib()
+    B = cfg["block_size"]
+    pad = L.dlm_split_pad(B)
+    x2 = torch.randn((2 * pad, cfg["ffn"]), device="cuda").to(torch.bfloat16)
+    shapes = []
+    for lw in w["layers"]:
+        shapes += [(lw["w_qkv"], cfg["d"]), (lw["w_o"], cfg["n_q_heads"] * cfg["head_dim"]),
+                   (lw["w_gate"], cfg["d"]), (lw["w_up"], cfg["d"]), (lw["w_down"], cfg["ffn"])]
+    shapes.append((w["embed"], cfg["d"]))
+    n = max(L.dlm_gemm_scratch_size(B, t.shape[0], K) for t, K in shapes)
+    sc = torch.empty(n, dtype=torch.uint8, device="cuda")
+    s = C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for _ in range(args.steps):
+        for t, K in shapes:
+            st = L.dlm_gemm_bf16x2(C.c_void_p(x2.data_ptr()), C.c_void_p(t.data_ptr()), None, B, t.shape[0], K,
+                                   C.c_void_p(sc.data_ptr()), n, s)
+            assert st == 0, st
+    torch.cuda.synchronize()
+    print("gemm case done: %d launches" % (args.steps * len(shapes)))
+
+
 def main():
+    global GEN
     args = parse()
     from block_diffusion_decoding_denoising_b200 import gen
+    if args.case == "gemm":
+        gemm_case(args)
+        return
+    if args.case == "quick":
+        GEN = 256
     cfg = gen.config_4b(max_ctx=PROMPT + GEN, n_layers=args.layers)
     if args.impl == "reference":
         reference_arm(args, cfg)
@@ -246,6 +288,14 @@ def main():
     rounds_per_step = int(rb[:, 0].sum())
     ms_step = ms / args.steps
     tps = world * GEN / (ms_step / 1e3)
+    if args.case == "quick":
+        if rank == 0:
+            print(json.dumps({"case": "quick", "tokens_per_s": tps, "ms_per_step": ms_step,
+                              "rounds_per_step": rounds_per_step}), flush=True)
+        m.close()
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     # denoise rounds/s with the threshold schedule (tau = 0.9: about one commit per round on
     # random weights, i.e. up to B rounds per block), on 4 blocks
@@ -264,7 +314,7 @@ def main():
     # projection of one round (36 x {QKV, O, gate, up, down} + LM head), partial sums only
     L = dlm.lib()
     import ctypes as C
-    x = torch.randn((B, cfg["ffn"]), device=dev).to(torch.bfloat16)
+    x = torch.randn((2 * L.dlm_split_pad(B), cfg["ffn"]), device=dev).to(torch.bfloat16)
     shapes = []
     for lw in w["layers"]:
         shapes += [(lw["w_qkv"], cfg["d"]), (lw["w_o"], cfg["n_q_heads"] * cfg["head_dim"]),
@@ -276,8 +326,8 @@ def main():
 
     def gemms():
         for t, K in shapes:
-            L.dlm_gemm_bf16(C.c_void_p(x.data_ptr()), C.c_void_p(t.data_ptr()), None, B, t.shape[0], K,
-                            C.c_void_p(scratch.data_ptr()), scratch_n, sp)
+            L.dlm_gemm_bf16x2(C.c_void_p(x.data_ptr()), C.c_void_p(t.data_ptr()), None, B, t.shape[0], K,
+                              C.c_void_p(scratch.data_ptr()), scratch_n, sp)
 
     for _ in range(3):
         gemms()
@@ -290,7 +340,7 @@ def main():
     g1.record(stream)
     torch.cuda.synchronize()
     gemm_s = g0.elapsed_time(g1) / 1e3 / (reps * len(shapes))
-    gemm_bytes = sum(t.numel() * 2 + B * K * 2 for t, K in shapes) / len(shapes)
+    gemm_bytes = sum(t.numel() * 2 + 2 * B * K * 2 for t, K in shapes) / len(shapes)
     hbm, tflops, peak_kind = peaks()
     achieved = gemm_bytes / gemm_s / 1e9
 

@@ -29,7 +29,7 @@ using namespace dlm;
 
 namespace {
 
-constexpr int kPrefillChunk = 256;
+constexpr int kPrefillChunk = kMaxSplitTokens;  // prefill tokens per forward pass
 
 struct GraphEntry {
   int mode;
@@ -142,13 +142,15 @@ size_t max_partial_bytes(const dlm_config& c, int Tmax) {
 size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   Carver cv{base};
   const int Tmax = max_tokens(c), B = c.block_size, ho = c.n_q_heads * c.head_dim;
+  // GEMM inputs are split bf16 pairs: 2 * pad rows (high halves, then low halves)
+  const size_t R2 = 2 * (size_t)split_pad(Tmax), B2 = 2 * (size_t)split_pad(B);
   int* hdr = cv.take<int>(64);
   float* h = cv.take<float>((size_t)Tmax * c.d);
-  auto* xn = cv.take<__nv_bfloat16>((size_t)Tmax * c.d);
+  auto* xn = cv.take<__nv_bfloat16>(R2 * c.d);
   auto* q = cv.take<__nv_bfloat16>((size_t)Tmax * ho);
-  auto* o = cv.take<__nv_bfloat16>((size_t)Tmax * ho);
-  auto* act = cv.take<__nv_bfloat16>((size_t)Tmax * c.ffn);
-  auto* sbf = cv.take<__nv_bfloat16>((size_t)B * c.d);
+  auto* o = cv.take<__nv_bfloat16>(R2 * ho);
+  auto* act = cv.take<__nv_bfloat16>(R2 * c.ffn);
+  auto* sbf = cv.take<__nv_bfloat16>(B2 * c.d);
   size_t pb = max_partial_bytes(c, Tmax);
   float* partial = cv.take<float>(pb / sizeof(float));
   int sB = attention_max_splits(B, c.n_q_heads, c.n_kv_heads, c.max_ctx);
@@ -157,7 +159,7 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   size_t at = attention_scratch_bytes(Tmax, c.n_q_heads, c.head_dim, sT);
   float* attn = cv.take<float>((ab > at ? ab : at) / sizeof(float));
   float* logits = cv.take<float>((size_t)B * c.vocab);
-  auto* P = cv.take<__nv_bfloat16>((size_t)B * c.vocab);
+  auto* P = cv.take<__nv_bfloat16>(B2 * c.vocab);
   int32_t* tok = cv.take<int32_t>((size_t)c.max_ctx);
   int32_t* bt = cv.take<int32_t>(B);
   uint8_t* bc = cv.take<uint8_t>(B);
@@ -224,7 +226,7 @@ struct Runner {
   dlm_status gemm(int a_mode, const void* a0, const void* a1, const void* x, int T, int N, int K,
                   GemmOut* out) {
     GemmPlan p;
-    if (!gemm_plan(&p, a_mode, a0, a1, x, T, N, K, ctx->partial, msg, sizeof(msg)))
+    if (!gemm_plan(&p, a_mode, a0, a1, x, T, N, K, ctx->partial, msg, sizeof(msg), true))
       return fail(ctx, DLM_EUNSUPPORTED, "%s", msg);
     if (p.partial_bytes > ctx->partial_bytes)
       return fail(ctx, DLM_ENOMEM_WS, "gemm partials %zu > %zu", p.partial_bytes, ctx->partial_bytes);
@@ -268,6 +270,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   const int ho = Hq * hd, nqkv = (Hq + 2 * Hkv) * hd;
   const int nt = threads_for(d);
   const size_t rowsm = (size_t)d * sizeof(float);
+  const long pad = split_pad(T);  // low halves of split activations start `pad` rows down
   const __nv_bfloat16* first_gain =
       (const __nv_bfloat16*)(c.n_layers > 0 ? ctx->layers[0].attn_norm : ctx->w.final_norm);
 
@@ -277,12 +280,13 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   ea.tokens = f.tokens;
   ea.h = ctx->h;
   ea.xn = ctx->xn;
+  ea.xn_lo = pad * d;
   ea.gain = first_gain;
   ea.d = d;
   ea.eps = c.rms_eps;
   if (f.s) {
     long n = (long)T * d;
-    k_to_bf16<<<(unsigned)((n + 255) / 256), 256, 0, r.s>>>(f.s, ctx->sbf, n);
+    k_to_bf16<<<(unsigned)((n + 255) / 256), 256, 0, r.s>>>(f.s, ctx->sbf, n, pad * d);
     TRY(r.check());
     TRY(r.gemm(A_KMAJOR, ctx->w.w_adapter, nullptr, ctx->sbf, T, d, d, &ea.adapter));
     ea.has_adapter = 1;
@@ -317,6 +321,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     aa.kc = kc;
     aa.vc = vc;
     aa.o = ctx->o;
+    aa.o_lo = pad * ho;
     aa.part_o = ctx->attn_part;
     aa.T = T;
     aa.Hq = Hq;
@@ -336,6 +341,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     TRY(r.gemm(A_KMAJOR, W.w_o, nullptr, ctx->o, T, d, ho, &ra.y));
     ra.h = ctx->h;
     ra.xn = ctx->xn;
+    ra.xn_lo = pad * d;
     ra.gain = (const __nv_bfloat16*)W.mlp_norm;
     ra.d = d;
     ra.eps = c.rms_eps;
@@ -345,6 +351,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     SiluArgs sa{};
     TRY(r.gemm(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, &sa.y));
     sa.out = ctx->act;
+    sa.lo = pad * F;
     sa.F = F;
     k_silu_gate<<<dim3((F + 255) / 256, T), 256, 0, r.s>>>(sa);
     TRY(r.check());
@@ -353,6 +360,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     TRY(r.gemm(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, &rd.y));
     rd.h = ctx->h;
     rd.xn = ctx->xn;
+    rd.xn_lo = pad * d;
     rd.gain = (const __nv_bfloat16*)(l + 1 < c.n_layers ? ctx->layers[l + 1].attn_norm : ctx->w.final_norm);
     rd.d = d;
     rd.eps = c.rms_eps;
@@ -376,6 +384,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   rs.mask_id = c.mask_id;
   rs.stats = f.stats;
   rs.P = ctx->P;
+  rs.P_lo = pad * c.vocab;
   k_rowstats<<<T, 1024, 0, r.s>>>(rs);
   TRY(r.check());
   StoreArgs pa{};
@@ -724,10 +733,12 @@ size_t dlm_gemm_scratch_size(int T, int N, int K) {
   return op_header() + align256(gemm_partial_bytes(T, N, K, A_KMAJOR));
 }
 
-dlm_status dlm_gemm_bf16(const void* d_x, const void* d_w, float* d_y, int T, int N, int K, void* d_scratch,
-                         size_t scratch_bytes, void* stream) {
+static dlm_status gemm_op(const void* d_x, const void* d_w, float* d_y, int T, int N, int K, void* d_scratch,
+                          size_t scratch_bytes, void* stream, bool split) {
   dlm_ctx* ctx = nullptr;
-  if (!d_x || !d_w || !d_scratch || T < 1 || T > kMaxTokens || N < 1 || K < 64 || K % 8) return DLM_EINVAL;
+  if (!d_x || !d_w || !d_scratch || T < 1 || T > (split ? kMaxSplitTokens : kMaxTokens) || N < 1 || K < 64 ||
+      K % 8)
+    return DLM_EINVAL;
   if (scratch_bytes < dlm_gemm_scratch_size(T, N, K)) return DLM_ENOMEM_WS;
   CU((cudaError_t)gemm_init_attributes());
   cudaStream_t s = (cudaStream_t)stream;
@@ -736,7 +747,8 @@ dlm_status dlm_gemm_bf16(const void* d_x, const void* d_w, float* d_y, int T, in
   float* partial = (float*)(sc + op_header());
   char msg[256];
   GemmPlan p;
-  if (!gemm_plan(&p, A_KMAJOR, d_w, nullptr, d_x, T, N, K, partial, msg, sizeof(msg))) return DLM_EUNSUPPORTED;
+  if (!gemm_plan(&p, A_KMAJOR, d_w, nullptr, d_x, T, N, K, partial, msg, sizeof(msg), split))
+    return DLM_EUNSUPPORTED;
   CU(cudaMemsetAsync(err, 0, 4, s));
   CU(gemm_launch(p, err, s));
   if (!d_y) return DLM_OK;  // partial sums only (the tensor-core kernel alone)
@@ -750,16 +762,29 @@ dlm_status dlm_gemm_bf16(const void* d_x, const void* d_w, float* d_y, int T, in
   return DLM_OK;
 }
 
+dlm_status dlm_gemm_bf16(const void* d_x, const void* d_w, float* d_y, int T, int N, int K, void* d_scratch,
+                         size_t scratch_bytes, void* stream) {
+  return gemm_op(d_x, d_w, d_y, T, N, K, d_scratch, scratch_bytes, stream, false);
+}
+
+int dlm_split_pad(int T) { return split_pad(T); }
+
+dlm_status dlm_gemm_bf16x2(const void* d_x2, const void* d_w, float* d_y, int T, int N, int K, void* d_scratch,
+                           size_t scratch_bytes, void* stream) {
+  return gemm_op(d_x2, d_w, d_y, T, N, K, d_scratch, scratch_bytes, stream, true);
+}
+
 size_t dlm_lmhead_scratch_size(int B, int V, int d) {
   size_t lm = gemm_partial_bytes(B, V, d, A_KMAJOR), pe = gemm_partial_bytes(B, d, V, A_MNMAJOR);
-  return op_header() + align256(lm > pe ? lm : pe) + align256((size_t)B * V * 4) + align256((size_t)B * V * 2);
+  return op_header() + align256(lm > pe ? lm : pe) + align256((size_t)B * V * 4) +
+         align256((size_t)2 * split_pad(B) * V * 2);
 }
 
 dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int V, int d, int mask_id,
                                const void* d_p_given, dlm_row_stats stats, float* d_s, void* d_scratch,
                                size_t scratch_bytes, void* stream) {
   dlm_ctx* ctx = nullptr;
-  if (!d_x || !d_embed || !d_s || !d_scratch || B < 1 || B > kMaxTokens || V < 2 || V % 8 || d < 64 ||
+  if (!d_x || !d_embed || !d_s || !d_scratch || B < 1 || B > kMaxSplitTokens || V < 2 || V % 8 || d < 64 ||
       d % 64 || !stats.m || !stats.lse || !stats.maxprob || !stats.entropy || !stats.argmax)
     return DLM_EINVAL;
   if (scratch_bytes < dlm_lmhead_scratch_size(B, V, d)) return DLM_ENOMEM_WS;
@@ -790,10 +815,12 @@ dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int 
   rs.mask_id = mask_id;
   rs.stats = stats;
   rs.P = d_p_given ? nullptr : P;
+  rs.P_lo = (long)split_pad(B) * V;  // own softmax: split bf16 pair; a given P is plain bf16
   k_rowstats<<<B, 1024, 0, s>>>(rs);
   CU(cudaGetLastError());
   GemmPlan q;
-  if (!gemm_plan(&q, A_MNMAJOR, d_embed, nullptr, d_p_given ? d_p_given : P, B, d, V, partial, msg, sizeof(msg)))
+  if (!gemm_plan(&q, A_MNMAJOR, d_embed, nullptr, d_p_given ? d_p_given : P, B, d, V, partial, msg, sizeof(msg),
+                 d_p_given == nullptr))
     return DLM_EUNSUPPORTED;
   CU(gemm_launch(q, err, s));
   StoreArgs pa{};
@@ -807,14 +834,14 @@ dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int 
 }
 
 size_t dlm_adapter_scratch_size(int B, int d) {
-  return op_header() + align256(gemm_partial_bytes(B, d, d, A_KMAJOR)) + align256((size_t)B * d * 2);
+  return op_header() + align256(gemm_partial_bytes(B, d, d, A_KMAJOR)) + align256((size_t)2 * split_pad(B) * d * 2);
 }
 
 dlm_status dlm_adapter_embed(const void* d_embed, const void* d_w_adapter, const int32_t* d_tokens,
                              const float* d_s, float* d_h0, int B, int d, void* d_scratch, size_t scratch_bytes,
                              void* stream) {
   dlm_ctx* ctx = nullptr;
-  if (!d_embed || !d_w_adapter || !d_tokens || !d_s || !d_h0 || !d_scratch || B < 1 || B > kMaxTokens ||
+  if (!d_embed || !d_w_adapter || !d_tokens || !d_s || !d_h0 || !d_scratch || B < 1 || B > kMaxSplitTokens ||
       d < 64 || d % 64)
     return DLM_EINVAL;
   if (scratch_bytes < dlm_adapter_scratch_size(B, d)) return DLM_ENOMEM_WS;
@@ -826,11 +853,12 @@ dlm_status dlm_adapter_embed(const void* d_embed, const void* d_w_adapter, const
   __nv_bfloat16* sbf = (__nv_bfloat16*)(sc + op_header() + align256(gemm_partial_bytes(B, d, d, A_KMAJOR)));
   CU(cudaMemsetAsync(err, 0, 4, s));
   long n = (long)B * d;
-  k_to_bf16<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(d_s, sbf, n);
+  k_to_bf16<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(d_s, sbf, n, (long)split_pad(B) * d);
   CU(cudaGetLastError());
   char msg[256];
   GemmPlan p;
-  if (!gemm_plan(&p, A_KMAJOR, d_w_adapter, nullptr, sbf, B, d, d, partial, msg, sizeof(msg))) return DLM_EUNSUPPORTED;
+  if (!gemm_plan(&p, A_KMAJOR, d_w_adapter, nullptr, sbf, B, d, d, partial, msg, sizeof(msg), true))
+    return DLM_EUNSUPPORTED;
   CU(gemm_launch(p, err, s));
   EmbedArgs ea{};
   ea.embed = (const __nv_bfloat16*)d_embed;

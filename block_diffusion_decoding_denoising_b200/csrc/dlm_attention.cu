@@ -271,8 +271,8 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
 #pragma unroll
       for (int nb = 0; nb < HD / 8; ++nb) {
         int col = nb * 8 + tig * 2;
-        *reinterpret_cast<__nv_bfloat162*>(dst + col) =
-            __floats2bfloat162_rn(acc[nb][half * 2] * inv, acc[nb][half * 2 + 1] * inv);
+        store_split(dst + col, a.o_lo, acc[nb][half * 2] * inv);
+        store_split(dst + col + 1, a.o_lo, acc[nb][half * 2 + 1] * inv);
       }
     } else {
       const size_t prow = (size_t)split * Rows + (size_t)g * rows_total + R;
@@ -318,7 +318,7 @@ __global__ void k_attn_combine(AttnArgs a) {
       num += w * a.part_o[((size_t)s * Rows + row) * a.hd + e];
       den += w * ls;
     }
-    a.o[((size_t)t * a.Hq + h) * a.hd + e] = f2bf(den > 0.f ? num / den : 0.f);
+    store_split(a.o + ((size_t)t * a.Hq + h) * a.hd + e, a.o_lo, den > 0.f ? num / den : 0.f);
   }
 }
 

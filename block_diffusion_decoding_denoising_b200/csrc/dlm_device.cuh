@@ -20,6 +20,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ __nv_bfloat16 f2bf(float x) { return __float2bfloat16_rn(x); }
 
+// Stores v as a split bf16 pair: the high half at p[0] and, when lo_off != 0, the
+// rounding remainder at p[lo_off] (hi + lo carries about 16 significant bits).
+__device__ __forceinline__ void store_split(__nv_bfloat16* p, long lo_off, float v) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  p[0] = h;
+  if (lo_off) p[lo_off] = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
 // Records the first error code seen by any thread (0 = no error).
 __device__ __forceinline__ void set_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);

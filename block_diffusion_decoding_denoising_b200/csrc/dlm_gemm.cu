@@ -38,6 +38,7 @@ struct GemmCfg {
 struct GemmKArgs {
   int a_mode;
   int T;
+  int lo_col;  // 0, or the MMA column where the low halves of split activations start
   GemmOut out;
   int* err;
 };
@@ -172,10 +173,18 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
       float* dst = o.partial + (((size_t)tile * o.max_slots + slot) * o.T) * kTileM + row;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * NT;
       static_assert(NT % 32 == 0, "token tile is a multiple of 32");
+      const int ncb = (args.lo_col ? args.lo_col : NT) / 32;
 #pragma unroll 1
-      for (int cb = 0; cb < NT / 32; ++cb) {
+      for (int cb = 0; cb < ncb; ++cb) {
         if (cb * 32 >= o.T) break;
         tmem_ld32(taddr + cb * 32, v);
+        if (args.lo_col) {
+          // split activation x = hi + lo: the two column sets add up
+          float w[32];
+          tmem_ld32(taddr + args.lo_col + cb * 32, w);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] += w[j];
+        }
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int t = cb * 32 + j;
@@ -201,6 +210,7 @@ struct SimtArgs {
   const __nv_bfloat16* a0;
   const __nv_bfloat16* a1;
   const __nv_bfloat16* x;
+  long lo_off;  // elements from a high row to its low row (split activations), or 0
   int a_mode, N, K, T;
   GemmOut out;
 };
@@ -225,9 +235,15 @@ __global__ void k_gemm_simt(SimtArgs a) {
     if (a.a_mode == A_MNMAJOR) {
       int n = tile * kTileM + row;
       if (n < a.N)
-        for (int k = 0; k < a.K; ++k) acc += bf2f(xr[k]) * bf2f(a.a0[(size_t)k * a.N + n]);
+        for (int k = 0; k < a.K; ++k) {
+          float xv = bf2f(xr[k]) + (a.lo_off ? bf2f(xr[k + a.lo_off]) : 0.f);
+          acc += xv * bf2f(a.a0[(size_t)k * a.N + n]);
+        }
     } else {
-      for (int k = 0; k < a.K; ++k) acc += bf2f(xr[k]) * bf2f(wr[k]);
+      for (int k = 0; k < a.K; ++k) {
+        float xv = bf2f(xr[k]) + (a.lo_off ? bf2f(xr[k + a.lo_off]) : 0.f);
+        acc += xv * bf2f(wr[k]);
+      }
     }
   }
   a.out.partial[((size_t)tile * a.out.max_slots) * a.out.T * kTileM + (size_t)t * kTileM + row] = acc;
@@ -308,11 +324,13 @@ size_t gemm_partial_bytes(int T, int N, int K, int a_mode) {
   return (size_t)o.n_tiles * o.max_slots * T * kTileM * sizeof(float);
 }
 
+int split_pad(int T) { return T <= 32 ? 32 : (T <= 64 ? 64 : 128); }
+
 bool gemm_plan(GemmPlan* p, int a_mode, const void* a0, const void* a1, const void* x, int T, int N,
-               int K, float* partial, char* err, size_t errlen) {
+               int K, float* partial, char* err, size_t errlen, bool split) {
   memset(p, 0, sizeof(*p));
-  if (T < 1 || T > kMaxTokens || N < 1 || K < kTileK || K % 8 != 0) {
-    snprintf(err, errlen, "gemm: unsupported shape T=%d N=%d K=%d", T, N, K);
+  if (T < 1 || T > (split ? kMaxSplitTokens : kMaxTokens) || N < 1 || K < kTileK || K % 8 != 0) {
+    snprintf(err, errlen, "gemm: unsupported shape T=%d N=%d K=%d split=%d", T, N, K, (int)split);
     return false;
   }
   p->a_mode = a_mode;
@@ -322,7 +340,8 @@ bool gemm_plan(GemmPlan* p, int a_mode, const void* a0, const void* a1, const vo
   p->N = N;
   p->K = K;
   p->T = T;
-  p->nt = pad_nt(T);
+  p->nt = split ? 2 * split_pad(T) : pad_nt(T);
+  p->lo_col = split ? split_pad(T) : 0;
   partition(T, N, K, a_mode, &p->out);
   p->out.partial = partial;
   p->partial_bytes = (size_t)p->out.n_tiles * p->out.max_slots * T * kTileM * sizeof(float);
@@ -338,7 +357,8 @@ bool gemm_plan(GemmPlan* p, int a_mode, const void* a0, const void* a1, const vo
     ok = encode_tmap_2d(&p->ta0, a0, N, K, (uint64_t)N * 2, 64, kTileK, err, errlen);
     p->ta1 = p->ta0;
   }
-  ok = ok && encode_tmap_2d(&p->tb, x, K, T, (uint64_t)K * 2, kTileK, p->nt, err, errlen);
+  // split activations: rows [0, T) high halves, rows [pad, pad + T) low halves
+  ok = ok && encode_tmap_2d(&p->tb, x, K, split ? p->nt : T, (uint64_t)K * 2, kTileK, p->nt, err, errlen);
   return ok;
 }
 
@@ -347,6 +367,7 @@ static cudaError_t launch_nt(const GemmPlan& p, int* d_err, cudaStream_t s) {
   GemmKArgs a;
   a.a_mode = p.a_mode;
   a.T = p.T;
+  a.lo_col = p.lo_col;
   a.out = p.out;
   a.err = d_err;
   k_gemm_tc<NT><<<p.out.grid, 192, GemmCfg<NT>::kSmem, s>>>(p.ta0, p.ta1, p.tb, a);
@@ -388,6 +409,7 @@ static cudaError_t gemm_launch_simt(const GemmPlan& p, cudaStream_t s) {
   a.a0 = (const __nv_bfloat16*)p.a0;
   a.a1 = (const __nv_bfloat16*)p.a1;
   a.x = (const __nv_bfloat16*)p.x;
+  a.lo_off = (long)p.lo_col * p.K;
   a.a_mode = p.a_mode;
   a.N = p.N;
   a.K = p.K;

@@ -13,7 +13,8 @@ namespace dlm {
 constexpr int kSMs = 148;        // B200 streaming multiprocessors
 constexpr int kTileM = 128;      // output features per GEMM tile (tcgen05 M)
 constexpr int kTileK = 64;       // reduction elements per k-block (one 128-byte swizzle atom)
-constexpr int kMaxTokens = 256;  // tokens per forward pass (tcgen05 N <= 256)
+constexpr int kMaxTokens = 256;  // tokens per GEMM with plain bf16 activations (tcgen05 N <= 256)
+constexpr int kMaxSplitTokens = 128;  // tokens per GEMM with split (hi + lo) activations
 
 // Partial-sum layout written by the GEMM: [tile][slot][T][128] fp32.  Tile tau covers
 // output features [128 tau, 128 tau + 128) (for the gate/up pair: gate features
@@ -38,7 +39,8 @@ enum AMode : int {
 struct GemmPlan {
   CUtensorMap ta0, ta1, tb;
   int a_mode;
-  int nt;            // MMA N (tokens padded to 16/32/64/128/256)
+  int nt;            // MMA N (tokens padded to 32/64/128/256; twice the pad when split)
+  int lo_col;        // split activations: MMA column of the low halves (= pad), else 0
   int N, K, T;
   const void *a0, *a1, *x;
   GemmOut out;
@@ -50,8 +52,11 @@ bool encode_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, char* err, size_t errlen);
 size_t gemm_partial_bytes(int T, int N, int K, int a_mode);
 // Plans y = x W^T.  `a0` is W (or Wg for A_PAIR, E for A_MNMAJOR), `a1` Wu for A_PAIR.
+// split: x holds high halves in rows [0, T) and low halves in rows [pad, pad + T),
+// pad = split_pad(T); the GEMM computes (hi + lo) W^T with the weight tile read once.
+int split_pad(int T);
 bool gemm_plan(GemmPlan* p, int a_mode, const void* a0, const void* a1, const void* x, int T,
-               int N, int K, float* partial, char* err, size_t errlen);
+               int N, int K, float* partial, char* err, size_t errlen, bool split = false);
 cudaError_t gemm_launch(const GemmPlan& p, int* d_err, cudaStream_t s);
 int gemm_init_attributes();
 extern int g_gemm_impl;  // 0 = tcgen05 (default), 1 = plain CUDA-core kernel (debug aid)
@@ -61,7 +66,8 @@ struct AttnArgs {
   const __nv_bfloat16* q;    // [T][Hq][hd]
   const __nv_bfloat16* kc;   // [Hkv][max_ctx][hd] (one layer)
   const __nv_bfloat16* vc;
-  __nv_bfloat16* o;          // [T][Hq][hd]
+  __nv_bfloat16* o;          // [T][Hq][hd] (high halves when o_lo != 0)
+  long o_lo;                 // elements to the low halves of a split output, 0 = plain bf16
   float* part_o;             // [max_splits][Hkv * T * G][hd]
   float* part_ml;            // [max_splits][Hkv * T * G][2]
   int T, Hq, Hkv, hd, max_ctx;

@@ -36,12 +36,12 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 // RMSNorm of one row held in `row` (shared, fp32), written as bf16: x * r * g, with
 // r = 1 / sqrt(mean(x^2) + eps).
 __device__ void norm_row_to_bf16(const float* row, int d, const __nv_bfloat16* g, float eps,
-                                 __nv_bfloat16* out, float* red) {
+                                 __nv_bfloat16* out, long lo_off, float* red) {
   float ss = 0.f;
   for (int n = threadIdx.x; n < d; n += blockDim.x) ss += row[n] * row[n];
   ss = block_sum(ss, red);
   const float r = 1.0f / sqrtf(ss / (float)d + eps);
-  for (int n = threadIdx.x; n < d; n += blockDim.x) out[n] = f2bf(row[n] * r * bf2f(g[n]));
+  for (int n = threadIdx.x; n < d; n += blockDim.x) store_split(out + n, lo_off, row[n] * r * bf2f(g[n]));
 }
 
 // h[t] = E[tok_t] (+ W_a s_t from the GEMM partials when `has_adapter`), then
@@ -59,7 +59,7 @@ __global__ void k_embed_adapter_norm(EmbedArgs a) {
     a.h[(size_t)t * a.d + n] = v;
   }
   __syncthreads();
-  if (a.gain) norm_row_to_bf16(rowbuf, a.d, a.gain, a.eps, a.xn + (size_t)t * a.d, red);
+  if (a.gain) norm_row_to_bf16(rowbuf, a.d, a.gain, a.eps, a.xn + (size_t)t * a.d, a.xn_lo, red);
 }
 
 // h[t] += y[t] (GEMM output of W_o or W_d); xn[t] = RMSNorm(h[t]) with the next gain.
@@ -73,7 +73,7 @@ __global__ void k_residual_norm(ResidArgs a) {
     a.h[(size_t)t * a.d + n] = v;
   }
   __syncthreads();
-  if (a.gain) norm_row_to_bf16(rowbuf, a.d, a.gain, a.eps, a.xn + (size_t)t * a.d, red);
+  if (a.gain) norm_row_to_bf16(rowbuf, a.d, a.gain, a.eps, a.xn + (size_t)t * a.d, a.xn_lo, red);
 }
 
 // QKV projection output -> RoPE (NeoX pairing (j, j + hd/2), theta_j = base^(-2j/hd),
@@ -118,7 +118,7 @@ __global__ void k_silu_gate(SiluArgs a) {
   const float g = gemm_sum(a.y, tile, r, t);
   const float u = gemm_sum(a.y, tile, 64 + r, t);
   const float silu = g / (1.0f + expf(-g));
-  a.out[(size_t)t * a.F + f] = f2bf(silu * u);
+  store_split(a.out + (size_t)t * a.F + f, a.lo, silu * u);
 }
 
 // out[t][n] = y[t][n] (fp32), n < N.
@@ -129,10 +129,10 @@ __global__ void k_store_rows(StoreArgs a) {
   a.out[(size_t)t * a.ld + n] = gemm_out(a.y, n, t);
 }
 
-// bf16 copy of s (the W_a GEMM input).
-__global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n) {
+// Split bf16 copy of s (the W_a GEMM input): high halves at y[i], low halves at y[i + lo].
+__global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo) {
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = f2bf(x[i]);
+  if (i < n) store_split(y + i, lo, x[i]);
 }
 
 // Row statistics of logits[b][:] (mask id excluded) and P = softmax as bf16.
@@ -193,7 +193,7 @@ __global__ void k_rowstats(RowStatsArgs a) {
   if (a.P) {
     __nv_bfloat16* p = a.P + (size_t)b * a.V;
     for (int v = threadIdx.x; v < a.V; v += blockDim.x)
-      p[v] = f2bf(v == a.mask_id ? 0.f : expf(l[v] - lse));
+      store_split(p + v, a.P_lo, v == a.mask_id ? 0.f : expf(l[v] - lse));
   }
 }
 

@@ -13,7 +13,8 @@ struct EmbedArgs {
   GemmOut adapter;             // W_a s partials (when has_adapter)
   int has_adapter;
   float* h;                    // [T][d]
-  __nv_bfloat16* xn;           // [T][d]
+  __nv_bfloat16* xn;           // [T][d] high halves
+  long xn_lo;                  // elements to the low halves (split activations), 0 = none
   const __nv_bfloat16* gain;   // [d]
   int d;
   float eps;
@@ -23,6 +24,7 @@ struct ResidArgs {
   GemmOut y;
   float* h;
   __nv_bfloat16* xn;
+  long xn_lo;
   const __nv_bfloat16* gain;  // nullptr: skip the norm
   int d;
   float eps;
@@ -41,7 +43,8 @@ struct QkvArgs {
 
 struct SiluArgs {
   GemmOut y;
-  __nv_bfloat16* out;  // [T][F]
+  __nv_bfloat16* out;  // [T][F] high halves
+  long lo;             // elements to the low halves
   int F;
 };
 
@@ -58,7 +61,8 @@ struct RowStatsArgs {
   int V;
   int mask_id;
   dlm_row_stats stats;
-  __nv_bfloat16* P;     // [B][V] or nullptr
+  __nv_bfloat16* P;     // [B][V] high halves, or nullptr
+  long P_lo;            // elements to the low halves, 0 = none
 };
 
 struct CommitArgs {
@@ -101,7 +105,7 @@ __global__ void k_residual_norm(ResidArgs a);
 __global__ void k_qkv_rope(QkvArgs a);
 __global__ void k_silu_gate(SiluArgs a);
 __global__ void k_store_rows(StoreArgs a);
-__global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n);
+__global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo);
 __global__ void k_rowstats(RowStatsArgs a);
 __global__ void k_commit(CommitArgs a);
 __global__ void k_block_init(BlockInitArgs a);

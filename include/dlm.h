@@ -197,16 +197,26 @@ size_t dlm_gemm_scratch_size(int T, int N, int K);
 dlm_status dlm_gemm_bf16(const void* d_x, const void* d_w, float* d_y, int T, int N, int K,
                          void* d_scratch, size_t scratch_bytes, void* stream);
 
+/* The same GEMM with split activations, the form every projection of a round uses:
+ * x = hi + lo, both bf16, so the activations carry about 16 significant bits while the
+ * weight tile is still streamed from HBM once.  d_x2 holds 2 * dlm_split_pad(T) rows of K:
+ * high halves in rows [0, T), low halves in rows [pad, pad + T).  T <= 128. */
+int dlm_split_pad(int T);
+dlm_status dlm_gemm_bf16x2(const void* d_x2, const void* d_w, float* d_y, int T, int N, int K,
+                           void* d_scratch, size_t scratch_bytes, void* stream);
+
 /* LM head fused with row statistics and the residual contraction:
  *   logits = x E^T (x: bf16 [B][d], already normalised), stats of every row with the
  *   mask id excluded (mask_id < 0: none excluded), and s = P E with P = softmax(logits)
- *   (d_p_given == NULL) or P = d_p_given (bf16 [B][V]).  s: fp32 [B][d]. */
+ *   (d_p_given == NULL; P carried as a split bf16 pair) or P = d_p_given (bf16 [B][V]).
+ *   s: fp32 [B][d].  B <= 128. */
 size_t dlm_lmhead_scratch_size(int B, int V, int d);
 dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int V, int d,
                                int mask_id, const void* d_p_given, dlm_row_stats stats,
                                float* d_s, void* d_scratch, size_t scratch_bytes, void* stream);
 
-/* Adapter step: h0[B][d] (fp32) = E[tokens] + W_a bf16(s), s fp32 [B][d]. */
+/* Adapter step: h0[B][d] (fp32) = E[tokens] + W_a s, s fp32 [B][d] (carried into the GEMM
+ * as a split bf16 pair).  B <= 128. */
 size_t dlm_adapter_scratch_size(int B, int d);
 dlm_status dlm_adapter_embed(const void* d_embed, const void* d_w_adapter, const int32_t* d_tokens,
                              const float* d_s, float* d_h0, int B, int d, void* d_scratch,

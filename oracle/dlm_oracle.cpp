@@ -47,11 +47,10 @@
 //      scale sigma = RNE_e4m3(amax_blk / (6 S)); code q = RNE onto the e2m1 grid of
 //      w / (sigma S), saturating at +-6; dequant = q * sigma * S.  Activations use the
 //      same quantizer with one fp32 scale per row.
-//   R9 storage precision (option act_round): where the CUDA path stores a tensor in bf16
-//      the oracle rounds the same tensor to bf16 (round-to-nearest-even), so integer
-//      decisions are taken on the same operand precision.  The points are: s before W_a,
-//      every normalised GEMM input, q/k/v after RoPE (the KV cache), the attention output
-//      before W_o, silu(g)*u before W_d.  Arithmetic itself stays fp64.
+//   R9 attention operand precision (option act_round): the KV cache holds bf16 values and
+//      the attention takes bf16 queries, so with act_round set the oracle rounds q, k and v
+//      to bf16 (round-to-nearest-even) after RoPE, as they are stored; integer decisions
+//      are then taken on the same attention operands.  Every other value stays fp64.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -524,9 +523,7 @@ void forward(const orc_model& M, const orc_cfg& C, const int* tokens, const doub
   // embedding + residual self-conditioning (R1, R2)
   for (int i = 0; i < n; ++i) mat_row(M.embed, tokens[i], h.data() + size_t(i) * d);
   if (s) {
-    std::vector<double> sr(size_t(n) * d);
-    for (size_t i = 0; i < sr.size(); ++i) sr[i] = maybe_round(s[i], rnd);
-    linear(sr.data(), n, M.w_adapter, tmp.data(), false);
+    linear(s, n, M.w_adapter, tmp.data(), false);
     for (size_t i = 0; i < h.size(); ++i) h[i] += tmp[i];
   }
   std::vector<double> qkv(size_t(n) * nqkv), q(size_t(n) * Hq * hd), o(size_t(n) * Hq * hd);
@@ -537,7 +534,6 @@ void forward(const orc_model& M, const orc_cfg& C, const int* tokens, const doub
     double* vl = kv.v + size_t(l) * Hkv * kv.max_ctx * hd;
     // attention sub-block
     for (int i = 0; i < n; ++i) rmsnorm(h.data() + size_t(i) * d, d, L.attn_norm, C.rms_eps, xn.data() + size_t(i) * d);
-    for (auto& x : xn) x = maybe_round(x, rnd);
     linear(xn.data(), n, L.w_qkv, qkv.data(), fp4);
     for (int i = 0; i < n; ++i) {
       double* row = qkv.data() + size_t(i) * nqkv;
@@ -552,24 +548,21 @@ void forward(const orc_model& M, const orc_cfg& C, const int* tokens, const doub
       }
     }
     orc_attention(q.data(), n, Hq, Hkv, hd, kl, vl, kv.max_ctx, pos0, causal ? 1 : 0, o.data());
-    for (auto& x : o) x = maybe_round(x, rnd);
     linear(o.data(), n, L.w_o, tmp.data(), fp4);
     for (size_t i = 0; i < h.size(); ++i) h[i] += tmp[i];
     // MLP sub-block
     for (int i = 0; i < n; ++i) rmsnorm(h.data() + size_t(i) * d, d, L.mlp_norm, C.rms_eps, xn.data() + size_t(i) * d);
-    for (auto& x : xn) x = maybe_round(x, rnd);
     linear(xn.data(), n, L.w_gate, g.data(), fp4);
     linear(xn.data(), n, L.w_up, u.data(), fp4);
     for (size_t i = 0; i < a.size(); ++i) {
       double silu = g[i] / (1.0 + std::exp(-g[i]));
-      a[i] = maybe_round(silu * u[i], rnd);
+      a[i] = silu * u[i];
     }
     linear(a.data(), n, L.w_down, tmp.data(), fp4);
     for (size_t i = 0; i < h.size(); ++i) h[i] += tmp[i];
   }
   if (xf) {
     for (int i = 0; i < n; ++i) rmsnorm(h.data() + size_t(i) * d, d, M.final_norm, C.rms_eps, xf + size_t(i) * d);
-    for (size_t i = 0; i < size_t(n) * d; ++i) xf[i] = maybe_round(xf[i], rnd);
   }
 }
 

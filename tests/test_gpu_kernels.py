@@ -42,6 +42,21 @@ def test_gemm_tcgen05_parity(lib, T, N, K):
     assert_close(y, ref, 1e-3, "gemm %dx%dx%d" % (T, N, K))
 
 
+@pytest.mark.parametrize("T,N,K", [(32, 6144, 2560), (8, 200, 320), (100, 384, 192), (128, 512, 1024)])
+def test_gemm_split_activation_parity(lib, T, N, K):
+    """x carried as a bf16 pair hi + lo: the GEMM must match the fp64 product with x
+    exact to about 16 significant bits, far tighter than a single bf16 rounding."""
+    import torch
+    x = gen.normal_np(300 + T, T * K).reshape(T, K).astype(np.float32)
+    wb = _bits(400 + N, (N, K), 0.02)
+    y = lib.gemm_bf16x2(torch.from_numpy(x).cuda(), to_torch_bf16(wb)).cpu().numpy()
+    ref = O.linear(x.astype(np.float64), wb)
+    e = assert_close(y, ref, 5e-5, "split gemm %dx%dx%d" % (T, N, K))
+    # a single bf16 rounding of x would be two orders of magnitude worse
+    xb = gen.bf16_bits(x.astype(np.float64))
+    assert rel_err(O.linear(bf16_f64(xb), wb), ref) > 20 * e
+
+
 def test_gemm_cuda_core_debug_path_matches(lib):
     T, N, K = 16, 300, 256
     xb = _bits(7, (T, K))
@@ -175,9 +190,8 @@ def test_adapter_embed(lib, B, d, V):
     h0 = lib.adapter_embed(to_torch_bf16(Eb), to_torch_bf16(Wab), torch.from_numpy(tok).cuda(),
                            torch.from_numpy(s.astype(np.float32)).cuda()).cpu().numpy()
     s32 = s.astype(np.float32).astype(np.float64)
-    s_bf = np.array([O.round_bf16(v) for v in s32.reshape(-1)]).reshape(B, d)
-    ref = bf16_f64(Eb)[tok] + O.linear(s_bf, Wab)
-    assert_close(h0, ref, 1e-3, "adapter")
+    ref = bf16_f64(Eb)[tok] + O.linear(s32, Wab)
+    assert_close(h0, ref, 1e-4, "adapter")
 
 
 # ------------------------------------------------------------------ commit
