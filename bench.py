@@ -46,6 +46,9 @@ def parse():
     # without the extra measurements; "gemm" = every projection GEMM of two layers plus
     # the LM-head GEMM, `--steps` launches each
     ap.add_argument("--case", default="full", choices=["full", "quick", "gemm"])
+    # the quick case with eager dlm_round / dlm_kv_fill calls instead of the block graph
+    # (same kernels; ncu cannot profile kernel nodes of graphs with conditional nodes)
+    ap.add_argument("--eager", action="store_true")
     return ap.parse_args()
 
 
@@ -256,10 +259,19 @@ def main():
     m.prefill(prompt)
     torch.cuda.synchronize()
 
+    est = m.new_block_state()
+
     def step(mode=dlm.COMMIT_TOPK, k=TPF_K, nblk=blocks):
         m.set_prefix_len(PROMPT)
         for b in range(nblk):
-            m.decode_block(TAU, mode, k, tokens_out[b], rounds_out[b])
+            if args.eager and mode == dlm.COMMIT_TOPK:
+                m.block_init(est)
+                for _ in range((B + k - 1) // k):
+                    m.round(est, TAU, mode, k)
+                m.kv_fill(est["tokens"])
+                rounds_out[b, 0] = (B + k - 1) // k
+            else:
+                m.decode_block(TAU, mode, k, tokens_out[b], rounds_out[b])
 
     def barrier():
         if world > 1:

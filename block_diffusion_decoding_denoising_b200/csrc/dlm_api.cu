@@ -103,6 +103,8 @@ dlm_status fail(dlm_ctx* ctx, dlm_status code, const char* fmt, ...) {
       return fail(ctx, DLM_ECUDA, "%s:%d %s: %s", __FILE__, __LINE__, #call, cudaGetErrorString(e_)); \
   } while (0)
 
+#define CU_LAUNCH(call) CU(call)
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Carver {
@@ -286,12 +288,12 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   ea.eps = c.rms_eps;
   if (f.s) {
     long n = (long)T * d;
-    k_to_bf16<<<(unsigned)((n + 255) / 256), 256, 0, r.s>>>(f.s, ctx->sbf, n, pad * d);
+    CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, r.s, f.s, ctx->sbf, n, pad * d));
     TRY(r.check());
     TRY(r.gemm(A_KMAJOR, ctx->w.w_adapter, nullptr, ctx->sbf, T, d, d, &ea.adapter));
     ea.has_adapter = 1;
   }
-  k_embed_adapter_norm<<<T, nt, rowsm, r.s>>>(ea);
+  CU_LAUNCH(launch_k(k_embed_adapter_norm, dim3(T), dim3(nt), rowsm, r.s, ea));
   TRY(r.check());
 
   const size_t layer_kv = (size_t)Hkv * c.max_ctx * hd;
@@ -311,7 +313,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     qa.pos0 = f.pos0;
     qa.pos0_dev = f.dev_L ? ctx->d_L : nullptr;
     qa.rope_theta = (double)c.rope_theta;
-    k_qkv_rope<<<dim3(Hq + 2 * Hkv, T), hd / 2, 0, r.s>>>(qa);
+    CU_LAUNCH(launch_k(k_qkv_rope, dim3(dim3(Hq + 2 * Hkv, T)), dim3(hd / 2), 0, r.s, qa));
     TRY(r.check());
     // the last layer's K/V do not depend on anything after its QKV projection
     if (!f.lm_head && l == c.n_layers - 1) break;
@@ -345,7 +347,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     ra.gain = (const __nv_bfloat16*)W.mlp_norm;
     ra.d = d;
     ra.eps = c.rms_eps;
-    k_residual_norm<<<T, nt, rowsm, r.s>>>(ra);
+    CU_LAUNCH(launch_k(k_residual_norm, dim3(T), dim3(nt), rowsm, r.s, ra));
     TRY(r.check());
 
     SiluArgs sa{};
@@ -353,7 +355,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     sa.out = ctx->act;
     sa.lo = pad * F;
     sa.F = F;
-    k_silu_gate<<<dim3((F + 255) / 256, T), 256, 0, r.s>>>(sa);
+    CU_LAUNCH(launch_k(k_silu_gate, dim3(dim3((F + 255) / 256, T)), dim3(256), 0, r.s, sa));
     TRY(r.check());
 
     ResidArgs rd{};
@@ -364,7 +366,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     rd.gain = (const __nv_bfloat16*)(l + 1 < c.n_layers ? ctx->layers[l + 1].attn_norm : ctx->w.final_norm);
     rd.d = d;
     rd.eps = c.rms_eps;
-    k_residual_norm<<<T, nt, rowsm, r.s>>>(rd);
+    CU_LAUNCH(launch_k(k_residual_norm, dim3(T), dim3(nt), rowsm, r.s, rd));
     TRY(r.check());
   }
   if (!f.lm_head) return DLM_OK;
@@ -375,7 +377,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   la.out = ctx->logits;
   la.N = c.vocab;
   la.ld = c.vocab;
-  k_store_rows<<<dim3((c.vocab + 255) / 256, T), 256, 0, r.s>>>(la);
+  CU_LAUNCH(launch_k(k_store_rows, dim3(dim3((c.vocab + 255) / 256, T)), dim3(256), 0, r.s, la));
   TRY(r.check());
   RowStatsArgs rs{};
   rs.logits = ctx->logits;
@@ -385,19 +387,20 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   rs.stats = f.stats;
   rs.P = ctx->P;
   rs.P_lo = pad * c.vocab;
-  k_rowstats<<<T, 1024, 0, r.s>>>(rs);
+  CU_LAUNCH(launch_k(k_rowstats, dim3(T), dim3(1024), 0, r.s, rs));
   TRY(r.check());
   StoreArgs pa{};
   TRY(r.gemm(A_MNMAJOR, ctx->w.embed, nullptr, ctx->P, T, d, c.vocab, &pa.y));
   pa.out = f.s_out;
   pa.N = d;
   pa.ld = d;
-  k_store_rows<<<dim3((d + 255) / 256, T), 256, 0, r.s>>>(pa);
+  CU_LAUNCH(launch_k(k_store_rows, dim3(dim3((d + 255) / 256, T)), dim3(256), 0, r.s, pa));
   return r.check();
 }
 
 dlm_status launch_commit(Runner& r, const dlm_block_state& st, float tau, int mode, int k,
                          bool use_cond, cudaGraphConditionalHandle h) {
+  dlm_ctx* ctx = r.ctx;
   const dlm_config& c = r.ctx->cfg;
   CommitArgs ca{};
   ca.maxprob = st.stats.maxprob;
@@ -414,7 +417,7 @@ dlm_status launch_commit(Runner& r, const dlm_block_state& st, float tau, int mo
   ca.k = k;
   ca.use_cond = use_cond ? 1 : 0;
   ca.cond = h;
-  k_commit<<<1, 64, 0, r.s>>>(ca);
+  CU_LAUNCH(launch_k(k_commit, dim3(1), dim3(64), 0, r.s, ca));
   return r.check();
 }
 
@@ -438,9 +441,10 @@ dlm_block_state internal_state(dlm_ctx* ctx) {
 }
 
 dlm_status launch_block_init(Runner& r, const dlm_block_state& st) {
+  dlm_ctx* ctx = r.ctx;
   const dlm_config& c = r.ctx->cfg;
   BlockInitArgs ba{st.tokens, st.committed, st.s, st.round, st.status, c.block_size, c.d, c.mask_id};
-  k_block_init<<<64, 256, 0, r.s>>>(ba);
+  CU_LAUNCH(launch_k(k_block_init, dim3(64), dim3(256), 0, r.s, ba));
   return r.check();
 }
 
@@ -496,7 +500,7 @@ dlm_status build_block_graph(dlm_ctx* ctx, int mode, float tau, int k, GraphEntr
   if (s3 == DLM_OK) {
     BlockFinishArgs fa{st.tokens, st.round, st.status, ctx->d_err, ctx->out_tokens, ctx->out_rounds,
                        ctx->d_L, c.block_size};
-    k_block_finish<<<1, 64, 0, cs>>>(fa);
+    CU_LAUNCH(launch_k(k_block_finish, dim3(1), dim3(64), 0, cs, fa));
     s3 = r.check();
   }
   e = cudaStreamEndCapture(cs, &g_fill);
@@ -519,6 +523,8 @@ extern "C" {
 const char* dlm_version(void) { return "dlm-b200 0.1 (sm_100a)"; }
 
 void dlm_debug_set_gemm_impl(int impl) { g_gemm_impl = impl; }
+
+void dlm_debug_set_pdl(int on) { g_pdl = on != 0; }
 
 size_t dlm_workspace_size(const dlm_config* cfg) {
   char msg[128];
@@ -592,7 +598,7 @@ int dlm_prefix_len(const dlm_ctx* ctx) { return ctx ? ctx->L : -1; }
 dlm_status dlm_set_prefix_len(dlm_ctx* ctx, int L, void* stream) {
   if (!ctx) return DLM_EINVAL;
   if (L < 0 || L > ctx->cfg.max_ctx) return fail(ctx, DLM_EINVAL, "L=%d", L);
-  k_set_int<<<1, 1, 0, (cudaStream_t)stream>>>(ctx->d_L, L);
+  CU_LAUNCH(launch_k(k_set_int, dim3(1), dim3(1), 0, (cudaStream_t)stream, ctx->d_L, L));
   CU(cudaGetLastError());
   ctx->L = L;
   return DLM_OK;
@@ -757,7 +763,7 @@ static dlm_status gemm_op(const void* d_x, const void* d_w, float* d_y, int T, i
   a.out = d_y;
   a.N = N;
   a.ld = N;
-  k_store_rows<<<dim3((N + 255) / 256, T), 256, 0, s>>>(a);
+  CU_LAUNCH(launch_k(k_store_rows, dim3(dim3((N + 255) / 256, T)), dim3(256), 0, s, a));
   CU(cudaGetLastError());
   return DLM_OK;
 }
@@ -806,7 +812,7 @@ dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int 
   la.out = logits;
   la.N = V;
   la.ld = V;
-  k_store_rows<<<dim3((V + 255) / 256, B), 256, 0, s>>>(la);
+  CU_LAUNCH(launch_k(k_store_rows, dim3(dim3((V + 255) / 256, B)), dim3(256), 0, s, la));
   CU(cudaGetLastError());
   RowStatsArgs rs{};
   rs.logits = logits;
@@ -816,7 +822,7 @@ dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int 
   rs.stats = stats;
   rs.P = d_p_given ? nullptr : P;
   rs.P_lo = (long)split_pad(B) * V;  // own softmax: split bf16 pair; a given P is plain bf16
-  k_rowstats<<<B, 1024, 0, s>>>(rs);
+  CU_LAUNCH(launch_k(k_rowstats, dim3(B), dim3(1024), 0, s, rs));
   CU(cudaGetLastError());
   GemmPlan q;
   if (!gemm_plan(&q, A_MNMAJOR, d_embed, nullptr, d_p_given ? d_p_given : P, B, d, V, partial, msg, sizeof(msg),
@@ -828,7 +834,7 @@ dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int 
   pa.out = d_s;
   pa.N = d;
   pa.ld = d;
-  k_store_rows<<<dim3((d + 255) / 256, B), 256, 0, s>>>(pa);
+  CU_LAUNCH(launch_k(k_store_rows, dim3(dim3((d + 255) / 256, B)), dim3(256), 0, s, pa));
   CU(cudaGetLastError());
   return DLM_OK;
 }
@@ -853,7 +859,7 @@ dlm_status dlm_adapter_embed(const void* d_embed, const void* d_w_adapter, const
   __nv_bfloat16* sbf = (__nv_bfloat16*)(sc + op_header() + align256(gemm_partial_bytes(B, d, d, A_KMAJOR)));
   CU(cudaMemsetAsync(err, 0, 4, s));
   long n = (long)B * d;
-  k_to_bf16<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(d_s, sbf, n, (long)split_pad(B) * d);
+  CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, d_s, sbf, n, (long)split_pad(B) * d));
   CU(cudaGetLastError());
   char msg[256];
   GemmPlan p;
@@ -867,7 +873,7 @@ dlm_status dlm_adapter_embed(const void* d_embed, const void* d_w_adapter, const
   ea.has_adapter = 1;
   ea.h = d_h0;
   ea.d = d;
-  k_embed_adapter_norm<<<B, threads_for(d), (size_t)d * 4, s>>>(ea);
+  CU_LAUNCH(launch_k(k_embed_adapter_norm, dim3(B), dim3(threads_for(d)), (size_t)d * 4, s, ea));
   CU(cudaGetLastError());
   return DLM_OK;
 }
@@ -912,6 +918,7 @@ dlm_status dlm_bd_attention(const void* d_q, const void* d_k_cache, const void* 
 dlm_status dlm_commit(const float* d_maxprob, const int32_t* d_argmax, int32_t* d_tokens, uint8_t* d_committed,
                       float* d_s, int32_t* d_round, int32_t* d_status, int B, int d, float tau, int commit_mode,
                       int tpf_k, void* stream) {
+  dlm_ctx* ctx = nullptr;
   if (!d_maxprob || !d_argmax || !d_tokens || !d_committed || !d_s || !d_round || B < 1 || B > 64 || d < 1)
     return DLM_EINVAL;
   if (commit_mode != DLM_COMMIT_THRESHOLD && commit_mode != DLM_COMMIT_TOPK) return DLM_EINVAL;
@@ -930,22 +937,23 @@ dlm_status dlm_commit(const float* d_maxprob, const int32_t* d_argmax, int32_t* 
   ca.tau = tau;
   ca.mode = commit_mode;
   ca.k = tpf_k;
-  k_commit<<<1, 64, 0, (cudaStream_t)stream>>>(ca);
+  CU_LAUNCH(launch_k(k_commit, dim3(1), dim3(64), 0, (cudaStream_t)stream, ca));
   return cudaGetLastError() == cudaSuccess ? DLM_OK : DLM_ECUDA;
 }
 
 dlm_status dlm_nvfp4_quantize(const void* d_w, int rows, int cols, void* d_codes, void* d_scales,
                               float* d_tensor_scale, void* stream) {
+  dlm_ctx* ctx = nullptr;
   if (!d_w || !d_codes || !d_scales || !d_tensor_scale || rows < 1 || cols < 16 || cols % 16) return DLM_EINVAL;
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(d_tensor_scale, 0, 4, s) != cudaSuccess) return DLM_ECUDA;
   long n = (long)rows * cols;
-  k_amax_bf16<<<1024, 256, 0, s>>>((const __nv_bfloat16*)d_w, n, (unsigned*)d_tensor_scale);
+  CU_LAUNCH(launch_k(k_amax_bf16, dim3(1024), dim3(256), 0, s, (const __nv_bfloat16*)d_w, n, (unsigned*)d_tensor_scale));
   long nblk = (long)rows * (cols / 16);
-  k_nvfp4_quantize<<<(unsigned)((nblk + 255) / 256), 256, 0, s>>>((const __nv_bfloat16*)d_w, rows, cols,
+  CU_LAUNCH(launch_k(k_nvfp4_quantize, dim3((unsigned)((nblk + 255) / 256)), dim3(256), 0, s, (const __nv_bfloat16*)d_w, rows, cols,
                                                                   (uint8_t*)d_codes, (uint8_t*)d_scales,
-                                                                  (const unsigned*)d_tensor_scale, nullptr);
-  k_amax_to_scale<<<1, 1, 0, s>>>(d_tensor_scale);
+                                                                  (const unsigned*)d_tensor_scale, nullptr));
+  CU_LAUNCH(launch_k(k_amax_to_scale, dim3(1), dim3(1), 0, s, d_tensor_scale));
   return cudaGetLastError() == cudaSuccess ? DLM_OK : DLM_ECUDA;
 }
 

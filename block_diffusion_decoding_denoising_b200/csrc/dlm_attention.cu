@@ -81,6 +81,8 @@ __host__ __device__ __forceinline__ int attn_splits(int nkeys, int max_splits) {
 
 template <int HD>
 __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ __align__(128) uint8_t sm[];
   const int G = a.Hq / a.Hkv;
   const int rows_total = a.T * G;
@@ -230,14 +232,18 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
       acc[i][2] *= al_B;
       acc[i][3] *= al_B;
     }
-    // O += P V
+    // O += P V, with P carried as a bf16 pair (hi + lo) so the weights keep ~16 bits
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {  // 16 keys per k-step
-      uint32_t pa[4];
-      pa[0] = pack_bf16(s[2 * ks][0], s[2 * ks][1]);
-      pa[1] = pack_bf16(s[2 * ks][2], s[2 * ks][3]);
-      pa[2] = pack_bf16(s[2 * ks + 1][0], s[2 * ks + 1][1]);
-      pa[3] = pack_bf16(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+      uint32_t pa[4], pl[4];
+      const float* p4[4] = {&s[2 * ks][0], &s[2 * ks][2], &s[2 * ks + 1][0], &s[2 * ks + 1][2]};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(p4[r][0], p4[r][1]);
+        const float2 hf = __bfloat1622float2(hi);
+        pa[r] = *reinterpret_cast<const uint32_t*>(&hi);
+        pl[r] = pack_bf16(p4[r][0] - hf.x, p4[r][1] - hf.y);
+      }
 #pragma unroll
       for (int nb2 = 0; nb2 < HD / 16; ++nb2) {
         // matrices: [keys ks*16+0..7, hd nb2*16+0..7], [keys +8, ..], [keys 0..7, hd +8], [keys +8, hd +8]
@@ -248,6 +254,8 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
         ldsm_x4_t(tile_addr<HD>(sV[buf], key, col), b0, b1, b2, b3);
         mma16816(acc[nb2 * 2], pa, b0, b1);
         mma16816(acc[nb2 * 2 + 1], pa, b2, b3);
+        mma16816(acc[nb2 * 2], pl, b0, b1);
+        mma16816(acc[nb2 * 2 + 1], pl, b2, b3);
       }
     }
     __syncthreads();  // buffer `buf` is refilled two iterations later
@@ -292,6 +300,8 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
 
 // Merges the key splits: o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
 __global__ void k_attn_combine(AttnArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int G = a.Hq / a.Hkv;
   const int rows_total = a.T * G;
   const int Rows = a.Hkv * rows_total;
@@ -362,13 +372,9 @@ template <int HD>
 static cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   const int G = a.Hq / a.Hkv;
   dim3 grid((a.T * G + kAttnRows - 1) / kAttnRows, a.Hkv, a.max_splits);
-  k_bd_attention<HD><<<grid, 128, AttnSmem<HD>::kBytes, s>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_k(k_bd_attention<HD>, grid, dim3(128), AttnSmem<HD>::kBytes, s, a);
   if (e != cudaSuccess) return e;
-  if (a.max_splits > 1) {
-    k_attn_combine<<<a.Hkv * a.T * G, 128, 0, s>>>(a);
-    e = cudaGetLastError();
-  }
+  if (a.max_splits > 1) e = launch_k(k_attn_combine, dim3(a.Hkv * a.T * G), dim3(128), 0, s, a);
   return e;
 }
 

@@ -28,6 +28,17 @@ __device__ __forceinline__ void store_split(__nv_bfloat16* p, long lo_off, float
   if (lo_off) p[lo_off] = __float2bfloat16_rn(v - __bfloat162float(h));
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Every kernel of a round lets the next kernel in the stream launch as soon as all of its
+// own CTAs are running (pdl_trigger at entry), and waits for the previous kernel to
+// complete and flush (pdl_wait) before it reads or writes any mutable global memory.
+// Only constant data (weights) may be touched before pdl_wait.  Both are no-ops for a
+// kernel launched without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Records the first error code seen by any thread (0 = no error).
 __device__ __forceinline__ void set_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);

@@ -24,6 +24,7 @@
 namespace dlm {
 
 int g_gemm_impl = 0;
+bool g_pdl = true;
 
 template <int NT>
 struct GemmCfg {
@@ -85,33 +86,52 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  pdl_trigger();
+  if (warp != 0) pdl_wait();  // the producer waits after requesting its first weight tiles
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
-    int stage = 0;
-    uint32_t phase = 0;
     uint32_t armed_parity[8];
     bool armed[8];
     for (int i = 0; i < S; ++i) armed[i] = false;
-    bool ok = true;
-    for (long u = u_begin; u < u_end && ok; ++u) {
+    auto load_a = [&](long u, int st) {
       const int tile = (int)(u / o.n_kb), kb = (int)(u % o.n_kb);
+      uint8_t* sa = smem + st * Cfg::kStageBytes;
+      if (args.a_mode == A_KMAJOR) {
+        tma_load_2d(sa, &ta0, &full[st], kb * kTileK, tile * kTileM);
+      } else if (args.a_mode == A_PAIR) {
+        tma_load_2d(sa, &ta0, &full[st], kb * kTileK, tile * 64);
+        tma_load_2d(sa + Cfg::kABytes / 2, &ta1, &full[st], kb * kTileK, tile * 64);
+      } else {  // A^T stored [K][N]: two 64-wide column boxes of 64 K-rows
+        tma_load_2d(sa, &ta0, &full[st], tile * kTileM, kb * kTileK);
+        tma_load_2d(sa + Cfg::kABytes / 2, &ta0, &full[st], tile * kTileM + 64, kb * kTileK);
+      }
+    };
+    auto load_b = [&](long u, int st) {
+      const int kb = (int)(u % o.n_kb);
+      tma_load_2d(smem + st * Cfg::kStageBytes + Cfg::kABytes, &tb, &full[st], kb * kTileK, 0);
+    };
+    // The weights do not depend on the previous kernel: the first S stages of them are
+    // requested before waiting for it, the activations only after.
+    const long n_pre = (u_end - u_begin) < S ? (u_end - u_begin) : S;
+    for (long i = 0; i < n_pre; ++i) {
+      mbar_arrive_expect_tx(&full[i], Cfg::kStageBytes);
+      armed[i] = true;
+      armed_parity[i] = 0;
+      load_a(u_begin + i, (int)i);
+    }
+    pdl_wait();
+    for (long i = 0; i < n_pre; ++i) load_b(u_begin + i, (int)i);
+    int stage = (int)(n_pre % S);
+    uint32_t phase = (n_pre == S) ? 1u : 0u;
+    bool ok = true;
+    for (long u = u_begin + n_pre; u < u_end && ok; ++u) {
       if (!mbar_wait(&empty[stage], phase ^ 1, args.err)) { ok = false; break; }
-      uint8_t* sa = smem + stage * Cfg::kStageBytes;
-      uint8_t* sb = sa + Cfg::kABytes;
       mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
       armed[stage] = true;
       armed_parity[stage] = phase;
-      if (args.a_mode == A_KMAJOR) {
-        tma_load_2d(sa, &ta0, &full[stage], kb * kTileK, tile * kTileM);
-      } else if (args.a_mode == A_PAIR) {
-        tma_load_2d(sa, &ta0, &full[stage], kb * kTileK, tile * 64);
-        tma_load_2d(sa + Cfg::kABytes / 2, &ta1, &full[stage], kb * kTileK, tile * 64);
-      } else {  // A^T stored [K][N]: two 64-wide column boxes of 64 K-rows
-        tma_load_2d(sa, &ta0, &full[stage], tile * kTileM, kb * kTileK);
-        tma_load_2d(sa + Cfg::kABytes / 2, &ta0, &full[stage], tile * kTileM + 64, kb * kTileK);
-      }
-      tma_load_2d(sb, &tb, &full[stage], kb * kTileK, 0);
+      load_a(u, stage);
+      load_b(u, stage);
       if (++stage == S) { stage = 0; phase ^= 1; }
     }
     // never leave the CTA with copies in flight: wait (bounded) for every armed stage
@@ -370,8 +390,7 @@ static cudaError_t launch_nt(const GemmPlan& p, int* d_err, cudaStream_t s) {
   a.lo_col = p.lo_col;
   a.out = p.out;
   a.err = d_err;
-  k_gemm_tc<NT><<<p.out.grid, 192, GemmCfg<NT>::kSmem, s>>>(p.ta0, p.ta1, p.tb, a);
-  return cudaGetLastError();
+  return launch_k(k_gemm_tc<NT>, dim3(p.out.grid), dim3(192), GemmCfg<NT>::kSmem, s, p.ta0, p.ta1, p.tb, a);
 }
 
 template <int NT>

@@ -10,6 +10,26 @@
 
 namespace dlm {
 
+// Programmatic dependent launch for every kernel of a round (default on; a debugging
+// switch turns it off).  See pdl_trigger / pdl_wait in dlm_device.cuh.
+extern bool g_pdl;
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                            Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 constexpr int kSMs = 148;        // B200 streaming multiprocessors
 constexpr int kTileM = 128;      // output features per GEMM tile (tcgen05 M)
 constexpr int kTileK = 64;       // reduction elements per k-block (one 128-byte swizzle atom)

@@ -47,6 +47,8 @@ __device__ void norm_row_to_bf16(const float* row, int d, const __nv_bfloat16* g
 // h[t] = E[tok_t] (+ W_a s_t from the GEMM partials when `has_adapter`), then
 // xn[t] = RMSNorm(h[t]) with gain g.  One CTA per token.
 __global__ void k_embed_adapter_norm(EmbedArgs a) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float rowbuf[];
   __shared__ float red[32];
   const int t = blockIdx.x;
@@ -64,6 +66,8 @@ __global__ void k_embed_adapter_norm(EmbedArgs a) {
 
 // h[t] += y[t] (GEMM output of W_o or W_d); xn[t] = RMSNorm(h[t]) with the next gain.
 __global__ void k_residual_norm(ResidArgs a) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float rowbuf[];
   __shared__ float red[32];
   const int t = blockIdx.x;
@@ -80,6 +84,8 @@ __global__ void k_residual_norm(ResidArgs a) {
 // absolute position L + t; angles in double precision) -> bf16 q and the K/V cache rows.
 // grid (Hq + 2 Hkv, T), hd/2 threads.
 __global__ void k_qkv_rope(QkvArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int hh = blockIdx.x, t = blockIdx.y, j = threadIdx.x;
   const int hd = a.hd, half = hd / 2;
   if (j >= half) return;
@@ -111,6 +117,8 @@ __global__ void k_qkv_rope(QkvArgs a) {
 
 // a[t][f] = bf16(silu(g) * u), g and u from the paired gate/up GEMM (tile = 64 + 64 rows).
 __global__ void k_silu_gate(SiluArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.y;
   const int f = blockIdx.x * blockDim.x + threadIdx.x;
   if (f >= a.F) return;
@@ -123,6 +131,8 @@ __global__ void k_silu_gate(SiluArgs a) {
 
 // out[t][n] = y[t][n] (fp32), n < N.
 __global__ void k_store_rows(StoreArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.y;
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= a.N) return;
@@ -131,6 +141,8 @@ __global__ void k_store_rows(StoreArgs a) {
 
 // Split bf16 copy of s (the W_a GEMM input): high halves at y[i], low halves at y[i + lo].
 __global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo) {
+  pdl_trigger();
+  pdl_wait();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) store_split(y + i, lo, x[i]);
 }
@@ -139,6 +151,8 @@ __global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo) {
 // m = max, argmax = lowest id of the max, Z = sum e^(l-m), lse = m + ln Z,
 // maxprob = 1/Z, entropy = ln Z - sum e^(l-m)(l-m) / Z.  One CTA per row.
 __global__ void k_rowstats(RowStatsArgs a) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red_v[32];
   __shared__ int red_i[32];
   __shared__ float bcast[2];
@@ -203,6 +217,8 @@ __global__ void k_rowstats(RowStatsArgs a) {
 // uncommitted positions of largest maxprob (ties -> lowest position).  Newly committed
 // positions take their argmax token and get a zero residual row.
 __global__ void k_commit(CommitArgs a) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float mp[64];
   __shared__ int unc[64];
   __shared__ int sel[64];
@@ -259,6 +275,8 @@ __global__ void k_commit(CommitArgs a) {
 
 // tokens = mask_id, committed = 0, s = 0, round = 0, status = 0.
 __global__ void k_block_init(BlockInitArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < a.B) {
     a.tokens[i] = a.mask_id;
@@ -274,6 +292,8 @@ __global__ void k_block_init(BlockInitArgs a) {
 // End of a block: copy tokens and {round, status} out, merge the kernel error flag into
 // the status, and advance the device prefix length by B.
 __global__ void k_block_finish(BlockFinishArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int i = threadIdx.x;
   if (i < a.B) a.tokens_out[i] = a.tokens[i];
   if (i == 0) {
@@ -285,10 +305,16 @@ __global__ void k_block_finish(BlockFinishArgs a) {
   }
 }
 
-__global__ void k_set_int(int* p, int v) { *p = v; }
+__global__ void k_set_int(int* p, int v) {
+  pdl_trigger();
+  pdl_wait();
+  *p = v;
+}
 
 // amax bits -> tensor scale amax / (6 * 448), in place.
 __global__ void k_amax_to_scale(float* p) {
+  pdl_trigger();
+  pdl_wait();
   *p = __uint_as_float(*reinterpret_cast<unsigned*>(p)) / (6.0f * 448.0f);
 }
 
@@ -296,6 +322,8 @@ __global__ void k_amax_to_scale(float* p) {
 // Per-tensor scale S = amax / (6 * 448) (fp32 division), per 16-element block e4m3 scale
 // sigma = RN_e4m3(amax_blk / (6 S)) (saturating), codes = RNE e2m1 of w / (sigma S).
 __global__ void k_amax_bf16(const __nv_bfloat16* w, long n, unsigned* amax_bits) {
+  pdl_trigger();
+  pdl_wait();
   float m = 0.f;
   for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
     m = fmaxf(m, fabsf(bf2f(w[i])));
@@ -346,6 +374,8 @@ __device__ __forceinline__ uint8_t e4m3_rne_bits(float x) {
 
 __global__ void k_nvfp4_quantize(const __nv_bfloat16* w, int rows, int cols, uint8_t* codes,
                                  uint8_t* scales, const unsigned* amax_bits, float* tscale) {
+  pdl_trigger();
+  pdl_wait();
   const float amax = __uint_as_float(*amax_bits);
   const float S = amax / (6.0f * 448.0f);
   const long nblk = (long)rows * (cols / 16);

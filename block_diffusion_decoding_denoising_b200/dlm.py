@@ -113,6 +113,7 @@ def lib():
         L.dlm_commit.argtypes = [p, p, p, p, p, p, p, i, i, f, i, i, p]
         L.dlm_nvfp4_quantize.argtypes = [p, i, i, p, p, p, p]
         L.dlm_debug_set_gemm_impl.argtypes = [i]
+        L.dlm_debug_set_pdl.argtypes = [i]
         _lib = L
     return _lib
 
@@ -138,6 +139,10 @@ def _check(st, ctx=None):
 
 def set_gemm_impl(impl: int) -> None:
     lib().dlm_debug_set_gemm_impl(int(impl))
+
+
+def set_pdl(on: bool) -> None:
+    lib().dlm_debug_set_pdl(int(bool(on)))
 
 
 # ------------------------------------------------------------------ single operations

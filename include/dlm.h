@@ -249,6 +249,11 @@ const char* dlm_version(void);
  * 1 on a plain CUDA-core kernel with the same output contract (slow; for cross-checks). */
 void dlm_debug_set_gemm_impl(int impl);
 
+/* Debugging aid: 1 (default) launches the kernels of a round with programmatic dependent
+ * launch (each kernel starts while its predecessor drains; weight tiles are prefetched
+ * before the dependency resolves), 0 launches them plainly stream-ordered. */
+void dlm_debug_set_pdl(int on);
+
 #ifdef __cplusplus
 }
 #endif
