@@ -30,6 +30,7 @@ using namespace dlm;
 namespace {
 
 constexpr int kPrefillChunk = kMaxSplitTokens;  // prefill tokens per forward pass
+constexpr int kRowChunk = 4096;                  // vocabulary entries per row-statistics CTA
 
 struct GraphEntry {
   int mode;
@@ -62,6 +63,9 @@ struct dlm_ctx {
   __nv_bfloat16* sbf = nullptr;
   float* partial = nullptr;
   size_t partial_bytes = 0;
+  int* tile_cnt = nullptr;   // per-tile arrival counters of the GEMM epilogue
+  float* ss = nullptr;       // per-tile sums of squares [ceil(d/128)][Tmax]
+  float* rs_part = nullptr;  // row-statistics chunk partials
   float* attn_part = nullptr;
   int attn_splits_B = 1, attn_splits_T = 1;
   float* logits = nullptr;
@@ -155,6 +159,9 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   auto* sbf = cv.take<__nv_bfloat16>(B2 * c.d);
   size_t pb = max_partial_bytes(c, Tmax);
   float* partial = cv.take<float>(pb / sizeof(float));
+  int* cnt = cv.take<int>((size_t)(c.vocab + 63) / 64 + (c.ffn + 63) / 64 + 64);
+  float* ssb = cv.take<float>((size_t)((c.d + 127) / 128) * Tmax);
+  float* rsp = cv.take<float>((size_t)4 * B * ((c.vocab + kRowChunk - 1) / kRowChunk));
   int sB = attention_max_splits(B, c.n_q_heads, c.n_kv_heads, c.max_ctx);
   int sT = attention_max_splits(Tmax, c.n_q_heads, c.n_kv_heads, c.max_ctx);
   size_t ab = attention_scratch_bytes(B, c.n_q_heads, c.head_dim, sB);
@@ -182,6 +189,9 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
     x->sbf = sbf;
     x->partial = partial;
     x->partial_bytes = pb;
+    x->tile_cnt = cnt;
+    x->ss = ssb;
+    x->rs_part = rsp;
     x->attn_part = attn;
     x->attn_splits_B = sB;
     x->attn_splits_T = sT;
@@ -225,16 +235,18 @@ struct Runner {
   cudaStream_t s;
   char msg[512];
 
+  // One projection with split activations and the fused epilogue `epi`.
   dlm_status gemm(int a_mode, const void* a0, const void* a1, const void* x, int T, int N, int K,
-                  GemmOut* out) {
+                  EpiArgs epi) {
     GemmPlan p;
     if (!gemm_plan(&p, a_mode, a0, a1, x, T, N, K, ctx->partial, msg, sizeof(msg), true))
       return fail(ctx, DLM_EUNSUPPORTED, "%s", msg);
     if (p.partial_bytes > ctx->partial_bytes)
       return fail(ctx, DLM_ENOMEM_WS, "gemm partials %zu > %zu", p.partial_bytes, ctx->partial_bytes);
+    epi.tile_cnt = ctx->tile_cnt;
+    p.epi = epi;
     cudaError_t e = gemm_launch(p, ctx->d_err, s);
     if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "gemm launch: %s", cudaGetErrorString(e));
-    *out = p.out;
     return DLM_OK;
   }
   dlm_status check() {
@@ -262,59 +274,64 @@ struct FwdSpec {
   float* s_out;
 };
 
-int threads_for(int d) { return d >= 1024 ? 512 : (d >= 256 ? 256 : 128); }
+// RMSNorm of h into the split GEMM input buffer xn, from the per-tile sums of squares.
+dlm_status norm_apply(Runner& r, int T, const void* gain) {
+  dlm_ctx* ctx = r.ctx;
+  const dlm_config& c = ctx->cfg;
+  NormArgs na{ctx->h, ctx->ss, (const __nv_bfloat16*)gain, ctx->xn, (long)split_pad(T) * c.d,
+              c.d, T, (c.d + 127) / 128, c.rms_eps};
+  CU_LAUNCH(launch_k(k_norm_apply, dim3((c.d + 255) / 256, T), dim3(256), 0, r.s, na));
+  return DLM_OK;
+}
 
-// One forward pass of T tokens (round, KV-fill or prefill chunk), all on stream r.s.
+// One forward pass of T tokens (round, KV-fill or prefill chunk), all on stream r.s:
+//   [s -> split bf16 -> W_a GEMM (+E[x])] or E[x]; RMSNorm
+//   per layer: QKV GEMM (+RoPE, K/V cache) ; attention ; O GEMM (+residual) ; RMSNorm ;
+//              gate/up GEMM (+SiLU gate) ; down GEMM (+residual) ; RMSNorm (next gain)
+//   round only: LM head GEMM -> logits ; row statistics + P ; P E GEMM -> s_out
 dlm_status forward(Runner& r, const FwdSpec& f) {
   dlm_ctx* ctx = r.ctx;
   const dlm_config& c = ctx->cfg;
   const int T = f.T, d = c.d, Hq = c.n_q_heads, Hkv = c.n_kv_heads, hd = c.head_dim, F = c.ffn;
   const int ho = Hq * hd, nqkv = (Hq + 2 * Hkv) * hd;
-  const int nt = threads_for(d);
-  const size_t rowsm = (size_t)d * sizeof(float);
   const long pad = split_pad(T);  // low halves of split activations start `pad` rows down
-  const __nv_bfloat16* first_gain =
-      (const __nv_bfloat16*)(c.n_layers > 0 ? ctx->layers[0].attn_norm : ctx->w.final_norm);
+  const void* first_gain = c.n_layers > 0 ? ctx->layers[0].attn_norm : ctx->w.final_norm;
 
   // embedding + residual adapter
-  EmbedArgs ea{};
-  ea.embed = (const __nv_bfloat16*)ctx->w.embed;
-  ea.tokens = f.tokens;
-  ea.h = ctx->h;
-  ea.xn = ctx->xn;
-  ea.xn_lo = pad * d;
-  ea.gain = first_gain;
-  ea.d = d;
-  ea.eps = c.rms_eps;
   if (f.s) {
     long n = (long)T * d;
     CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, r.s, f.s, ctx->sbf, n, pad * d));
-    TRY(r.check());
-    TRY(r.gemm(A_KMAJOR, ctx->w.w_adapter, nullptr, ctx->sbf, T, d, d, &ea.adapter));
-    ea.has_adapter = 1;
+    EpiArgs e{};
+    e.op = EPI_EMBED;
+    e.h = ctx->h;
+    e.ss = ctx->ss;
+    e.embed = (const __nv_bfloat16*)ctx->w.embed;
+    e.tokens = f.tokens;
+    TRY(r.gemm(A_KMAJOR, ctx->w.w_adapter, nullptr, ctx->sbf, T, d, d, e));
+  } else {
+    EmbedRowsArgs ea{(const __nv_bfloat16*)ctx->w.embed, f.tokens, ctx->h, ctx->ss, d, T};
+    CU_LAUNCH(launch_k(k_embed_rows, dim3((d + 127) / 128, T), dim3(128), 0, r.s, ea));
   }
-  CU_LAUNCH(launch_k(k_embed_adapter_norm, dim3(T), dim3(nt), rowsm, r.s, ea));
-  TRY(r.check());
+  TRY(norm_apply(r, T, first_gain));
 
   const size_t layer_kv = (size_t)Hkv * c.max_ctx * hd;
   for (int l = 0; l < c.n_layers; ++l) {
     const dlm_layer_weights& W = ctx->layers[l];
     __nv_bfloat16* kc = ctx->kv + (size_t)(2 * l) * layer_kv;
     __nv_bfloat16* vc = ctx->kv + (size_t)(2 * l + 1) * layer_kv;
-    QkvArgs qa{};
-    TRY(r.gemm(A_KMAJOR, W.w_qkv, nullptr, ctx->xn, T, nqkv, d, &qa.y));
-    qa.q = ctx->q;
-    qa.kc = kc;
-    qa.vc = vc;
-    qa.Hq = Hq;
-    qa.Hkv = Hkv;
-    qa.hd = hd;
-    qa.max_ctx = c.max_ctx;
-    qa.pos0 = f.pos0;
-    qa.pos0_dev = f.dev_L ? ctx->d_L : nullptr;
-    qa.rope_theta = (double)c.rope_theta;
-    CU_LAUNCH(launch_k(k_qkv_rope, dim3(dim3(Hq + 2 * Hkv, T)), dim3(hd / 2), 0, r.s, qa));
-    TRY(r.check());
+    EpiArgs eq{};
+    eq.op = EPI_QKV;
+    eq.q = ctx->q;
+    eq.kc = kc;
+    eq.vc = vc;
+    eq.Hq = Hq;
+    eq.Hkv = Hkv;
+    eq.hd = hd;
+    eq.max_ctx = c.max_ctx;
+    eq.pos0 = f.pos0;
+    eq.pos0_dev = f.dev_L ? ctx->d_L : nullptr;
+    eq.rope_theta = c.rope_theta;
+    TRY(r.gemm(A_KMAJOR, W.w_qkv, nullptr, ctx->xn, T, nqkv, d, eq));
     // the last layer's K/V do not depend on anything after its QKV projection
     if (!f.lm_head && l == c.n_layers - 1) break;
 
@@ -339,63 +356,48 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     cudaError_t e = attention_launch(aa, r.s);
     if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "attention: %s", cudaGetErrorString(e));
 
-    ResidArgs ra{};
-    TRY(r.gemm(A_KMAJOR, W.w_o, nullptr, ctx->o, T, d, ho, &ra.y));
-    ra.h = ctx->h;
-    ra.xn = ctx->xn;
-    ra.xn_lo = pad * d;
-    ra.gain = (const __nv_bfloat16*)W.mlp_norm;
-    ra.d = d;
-    ra.eps = c.rms_eps;
-    CU_LAUNCH(launch_k(k_residual_norm, dim3(T), dim3(nt), rowsm, r.s, ra));
-    TRY(r.check());
+    EpiArgs er{};
+    er.op = EPI_RESID;
+    er.h = ctx->h;
+    er.ss = ctx->ss;
+    TRY(r.gemm(A_KMAJOR, W.w_o, nullptr, ctx->o, T, d, ho, er));
+    TRY(norm_apply(r, T, W.mlp_norm));
 
-    SiluArgs sa{};
-    TRY(r.gemm(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, &sa.y));
-    sa.out = ctx->act;
-    sa.lo = pad * F;
-    sa.F = F;
-    CU_LAUNCH(launch_k(k_silu_gate, dim3(dim3((F + 255) / 256, T)), dim3(256), 0, r.s, sa));
-    TRY(r.check());
+    EpiArgs es{};
+    es.op = EPI_SILU;
+    es.act = ctx->act;
+    es.act_lo = pad * F;
+    TRY(r.gemm(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, es));
 
-    ResidArgs rd{};
-    TRY(r.gemm(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, &rd.y));
-    rd.h = ctx->h;
-    rd.xn = ctx->xn;
-    rd.xn_lo = pad * d;
-    rd.gain = (const __nv_bfloat16*)(l + 1 < c.n_layers ? ctx->layers[l + 1].attn_norm : ctx->w.final_norm);
-    rd.d = d;
-    rd.eps = c.rms_eps;
-    CU_LAUNCH(launch_k(k_residual_norm, dim3(T), dim3(nt), rowsm, r.s, rd));
-    TRY(r.check());
+    TRY(r.gemm(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, er));
+    TRY(norm_apply(r, T, l + 1 < c.n_layers ? ctx->layers[l + 1].attn_norm : ctx->w.final_norm));
   }
   if (!f.lm_head) return DLM_OK;
 
-  // LM head: logits, row statistics, P = softmax, s = P E
-  StoreArgs la{};
-  TRY(r.gemm(A_KMAJOR, ctx->w.embed, nullptr, ctx->xn, T, c.vocab, d, &la.y));
-  la.out = ctx->logits;
-  la.N = c.vocab;
-  la.ld = c.vocab;
-  CU_LAUNCH(launch_k(k_store_rows, dim3(dim3((c.vocab + 255) / 256, T)), dim3(256), 0, r.s, la));
-  TRY(r.check());
+  // LM head: logits, row statistics, P = softmax (split bf16), s = P E
+  EpiArgs el{};
+  el.op = EPI_STORE;
+  el.out = ctx->logits;
+  el.ld = c.vocab;
+  TRY(r.gemm(A_KMAJOR, ctx->w.embed, nullptr, ctx->xn, T, c.vocab, d, el));
   RowStatsArgs rs{};
   rs.logits = ctx->logits;
   rs.ld = c.vocab;
   rs.V = c.vocab;
   rs.mask_id = c.mask_id;
+  rs.chunk = kRowChunk;
+  rs.part = ctx->rs_part;
   rs.stats = f.stats;
   rs.P = ctx->P;
   rs.P_lo = pad * c.vocab;
-  CU_LAUNCH(launch_k(k_rowstats, dim3(T), dim3(1024), 0, r.s, rs));
-  TRY(r.check());
-  StoreArgs pa{};
-  TRY(r.gemm(A_MNMAJOR, ctx->w.embed, nullptr, ctx->P, T, d, c.vocab, &pa.y));
-  pa.out = f.s_out;
-  pa.N = d;
-  pa.ld = d;
-  CU_LAUNCH(launch_k(k_store_rows, dim3(dim3((d + 255) / 256, T)), dim3(256), 0, r.s, pa));
-  return r.check();
+  const int nch = (c.vocab + kRowChunk - 1) / kRowChunk;
+  CU_LAUNCH(launch_k(k_rowstats_part, dim3(nch, T), dim3(256), 0, r.s, rs));
+  CU_LAUNCH(launch_k(k_rowstats_final, dim3(nch, T), dim3(256), 0, r.s, rs));
+  EpiArgs ep{};
+  ep.op = EPI_STORE;
+  ep.out = f.s_out;
+  ep.ld = d;
+  return r.gemm(A_MNMAJOR, ctx->w.embed, nullptr, ctx->P, T, d, c.vocab, ep);
 }
 
 dlm_status launch_commit(Runner& r, const dlm_block_state& st, float tau, int mode, int k,
@@ -522,8 +524,6 @@ extern "C" {
 
 const char* dlm_version(void) { return "dlm-b200 0.1 (sm_100a)"; }
 
-void dlm_debug_set_gemm_impl(int impl) { g_gemm_impl = impl; }
-
 void dlm_debug_set_pdl(int on) { g_pdl = on != 0; }
 
 size_t dlm_workspace_size(const dlm_config* cfg) {
@@ -567,7 +567,7 @@ dlm_status dlm_ctx_create(const dlm_config* cfg, const dlm_weights* w, void* d_w
   ctx->kv_bytes = kv_bytes;
   carve(ctx, *cfg, ctx->ws);
   cudaError_t e = cudaStreamCreateWithFlags(&ctx->cap_stream, cudaStreamNonBlocking);
-  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->ws, 0, 256, ctx->cap_stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->ws, 0, ws_bytes, ctx->cap_stream);
   if (e == cudaSuccess) e = (cudaError_t)gemm_init_attributes();
   if (e == cudaSuccess) e = (cudaError_t)attention_init_attributes();
   if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->cap_stream);
@@ -733,10 +733,51 @@ dlm_status dlm_generate(dlm_ctx* ctx, const int32_t* h_prompt, int prompt_len, i
 }
 
 // ------------------------------------------------------------------ single operations
+}  // extern "C"
+
+// ------------------------------------------------------------------ single operations
+// Scratch of a single-operation call: [256 B status][tile counters][GEMM partials][extras].
 static size_t op_header() { return 256; }
+static size_t op_counters(int N) { return align256((size_t)((N + 63) / 64 + 2) * 4); }
+
+struct OpScratch {
+  uint8_t* base;
+  size_t off;
+  int* err;
+  int* cnt;
+  float* partial;
+  OpScratch(void* p, int n_cnt, size_t partial_bytes) : base((uint8_t*)p) {
+    err = (int*)base;
+    cnt = (int*)(base + op_header());
+    partial = (float*)(base + op_header() + op_counters(n_cnt));
+    off = op_header() + op_counters(n_cnt) + align256(partial_bytes);
+  }
+  template <class T>
+  T* take(size_t count) {
+    T* q = (T*)(base + off);
+    off += align256(count * sizeof(T));
+    return q;
+  }
+};
+
+static dlm_status op_gemm(const GemmPlan& plan0, EpiArgs epi, const OpScratch& sc, cudaStream_t s) {
+  dlm_ctx* ctx = nullptr;
+  GemmPlan p = plan0;
+  epi.tile_cnt = sc.cnt;
+  p.epi = epi;
+  CU(gemm_launch(p, sc.err, s));
+  return DLM_OK;
+}
+
+static size_t lmhead_partial(int B, int V, int d) {
+  size_t lm = gemm_partial_bytes(B, V, d, A_KMAJOR), pe = gemm_partial_bytes(B, d, V, A_MNMAJOR);
+  return lm > pe ? lm : pe;
+}
+
+extern "C" {
 
 size_t dlm_gemm_scratch_size(int T, int N, int K) {
-  return op_header() + align256(gemm_partial_bytes(T, N, K, A_KMAJOR));
+  return op_header() + op_counters(N) + align256(gemm_partial_bytes(T, N, K, A_KMAJOR));
 }
 
 static dlm_status gemm_op(const void* d_x, const void* d_w, float* d_y, int T, int N, int K, void* d_scratch,
@@ -748,24 +789,17 @@ static dlm_status gemm_op(const void* d_x, const void* d_w, float* d_y, int T, i
   if (scratch_bytes < dlm_gemm_scratch_size(T, N, K)) return DLM_ENOMEM_WS;
   CU((cudaError_t)gemm_init_attributes());
   cudaStream_t s = (cudaStream_t)stream;
-  uint8_t* sc = (uint8_t*)d_scratch;
-  int* err = (int*)sc;
-  float* partial = (float*)(sc + op_header());
+  OpScratch sc(d_scratch, N, gemm_partial_bytes(T, N, K, A_KMAJOR));
   char msg[256];
   GemmPlan p;
-  if (!gemm_plan(&p, A_KMAJOR, d_w, nullptr, d_x, T, N, K, partial, msg, sizeof(msg), split))
+  if (!gemm_plan(&p, A_KMAJOR, d_w, nullptr, d_x, T, N, K, sc.partial, msg, sizeof(msg), split))
     return DLM_EUNSUPPORTED;
-  CU(cudaMemsetAsync(err, 0, 4, s));
-  CU(gemm_launch(p, err, s));
-  if (!d_y) return DLM_OK;  // partial sums only (the tensor-core kernel alone)
-  StoreArgs a{};
-  a.y = p.out;
-  a.out = d_y;
-  a.N = N;
-  a.ld = N;
-  CU_LAUNCH(launch_k(k_store_rows, dim3(dim3((N + 255) / 256, T)), dim3(256), 0, s, a));
-  CU(cudaGetLastError());
-  return DLM_OK;
+  CU(cudaMemsetAsync(d_scratch, 0, op_header() + op_counters(N), s));
+  EpiArgs e{};
+  e.op = d_y ? EPI_STORE : EPI_PARTIAL;  // no output: the tensor-core kernel alone
+  e.out = d_y;
+  e.ld = N;
+  return op_gemm(p, e, sc, s);
 }
 
 dlm_status dlm_gemm_bf16(const void* d_x, const void* d_w, float* d_y, int T, int N, int K, void* d_scratch,
@@ -781,9 +815,9 @@ dlm_status dlm_gemm_bf16x2(const void* d_x2, const void* d_w, float* d_y, int T,
 }
 
 size_t dlm_lmhead_scratch_size(int B, int V, int d) {
-  size_t lm = gemm_partial_bytes(B, V, d, A_KMAJOR), pe = gemm_partial_bytes(B, d, V, A_MNMAJOR);
-  return op_header() + align256(lm > pe ? lm : pe) + align256((size_t)B * V * 4) +
-         align256((size_t)2 * split_pad(B) * V * 2);
+  const int nch = (V + kRowChunk - 1) / kRowChunk;
+  return op_header() + op_counters(V > d ? V : d) + align256(lmhead_partial(B, V, d)) +
+         align256((size_t)B * V * 4) + align256((size_t)2 * split_pad(B) * V * 2) + align256((size_t)16 * B * nch);
 }
 
 dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int V, int d, int mask_id,
@@ -796,51 +830,46 @@ dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int 
   if (scratch_bytes < dlm_lmhead_scratch_size(B, V, d)) return DLM_ENOMEM_WS;
   CU((cudaError_t)gemm_init_attributes());
   cudaStream_t s = (cudaStream_t)stream;
-  uint8_t* sc = (uint8_t*)d_scratch;
-  int* err = (int*)sc;
-  size_t lm = gemm_partial_bytes(B, V, d, A_KMAJOR), pe = gemm_partial_bytes(B, d, V, A_MNMAJOR);
-  float* partial = (float*)(sc + op_header());
-  float* logits = (float*)(sc + op_header() + align256(lm > pe ? lm : pe));
-  __nv_bfloat16* P = (__nv_bfloat16*)((uint8_t*)logits + align256((size_t)B * V * 4));
+  const int nch = (V + kRowChunk - 1) / kRowChunk;
+  OpScratch sc(d_scratch, V > d ? V : d, lmhead_partial(B, V, d));
+  float* logits = sc.take<float>((size_t)B * V);
+  __nv_bfloat16* P = sc.take<__nv_bfloat16>((size_t)2 * split_pad(B) * V);
+  float* part = sc.take<float>((size_t)4 * B * nch);
+  CU(cudaMemsetAsync(d_scratch, 0, op_header() + op_counters(V > d ? V : d), s));
   char msg[256];
-  CU(cudaMemsetAsync(err, 0, 4, s));
   GemmPlan p;
-  if (!gemm_plan(&p, A_KMAJOR, d_embed, nullptr, d_x, B, V, d, partial, msg, sizeof(msg))) return DLM_EUNSUPPORTED;
-  CU(gemm_launch(p, err, s));
-  StoreArgs la{};
-  la.y = p.out;
-  la.out = logits;
-  la.N = V;
-  la.ld = V;
-  CU_LAUNCH(launch_k(k_store_rows, dim3(dim3((V + 255) / 256, B)), dim3(256), 0, s, la));
-  CU(cudaGetLastError());
+  if (!gemm_plan(&p, A_KMAJOR, d_embed, nullptr, d_x, B, V, d, sc.partial, msg, sizeof(msg))) return DLM_EUNSUPPORTED;
+  EpiArgs el{};
+  el.op = EPI_STORE;
+  el.out = logits;
+  el.ld = V;
+  TRY(op_gemm(p, el, sc, s));
   RowStatsArgs rs{};
   rs.logits = logits;
   rs.ld = V;
   rs.V = V;
   rs.mask_id = mask_id;
+  rs.chunk = kRowChunk;
+  rs.part = part;
   rs.stats = stats;
   rs.P = d_p_given ? nullptr : P;
   rs.P_lo = (long)split_pad(B) * V;  // own softmax: split bf16 pair; a given P is plain bf16
-  CU_LAUNCH(launch_k(k_rowstats, dim3(B), dim3(1024), 0, s, rs));
-  CU(cudaGetLastError());
+  CU_LAUNCH(launch_k(k_rowstats_part, dim3(nch, B), dim3(256), 0, s, rs));
+  CU_LAUNCH(launch_k(k_rowstats_final, dim3(nch, B), dim3(256), 0, s, rs));
   GemmPlan q;
-  if (!gemm_plan(&q, A_MNMAJOR, d_embed, nullptr, d_p_given ? d_p_given : P, B, d, V, partial, msg, sizeof(msg),
+  if (!gemm_plan(&q, A_MNMAJOR, d_embed, nullptr, d_p_given ? d_p_given : P, B, d, V, sc.partial, msg, sizeof(msg),
                  d_p_given == nullptr))
     return DLM_EUNSUPPORTED;
-  CU(gemm_launch(q, err, s));
-  StoreArgs pa{};
-  pa.y = q.out;
-  pa.out = d_s;
-  pa.N = d;
-  pa.ld = d;
-  CU_LAUNCH(launch_k(k_store_rows, dim3(dim3((d + 255) / 256, B)), dim3(256), 0, s, pa));
-  CU(cudaGetLastError());
-  return DLM_OK;
+  EpiArgs ep{};
+  ep.op = EPI_STORE;
+  ep.out = d_s;
+  ep.ld = d;
+  return op_gemm(q, ep, sc, s);
 }
 
 size_t dlm_adapter_scratch_size(int B, int d) {
-  return op_header() + align256(gemm_partial_bytes(B, d, d, A_KMAJOR)) + align256((size_t)2 * split_pad(B) * d * 2);
+  return op_header() + op_counters(d) + align256(gemm_partial_bytes(B, d, d, A_KMAJOR)) +
+         align256((size_t)2 * split_pad(B) * d * 2) + align256((size_t)((d + 127) / 128) * B * 4);
 }
 
 dlm_status dlm_adapter_embed(const void* d_embed, const void* d_w_adapter, const int32_t* d_tokens,
@@ -853,29 +882,24 @@ dlm_status dlm_adapter_embed(const void* d_embed, const void* d_w_adapter, const
   if (scratch_bytes < dlm_adapter_scratch_size(B, d)) return DLM_ENOMEM_WS;
   CU((cudaError_t)gemm_init_attributes());
   cudaStream_t s = (cudaStream_t)stream;
-  uint8_t* sc = (uint8_t*)d_scratch;
-  int* err = (int*)sc;
-  float* partial = (float*)(sc + op_header());
-  __nv_bfloat16* sbf = (__nv_bfloat16*)(sc + op_header() + align256(gemm_partial_bytes(B, d, d, A_KMAJOR)));
-  CU(cudaMemsetAsync(err, 0, 4, s));
+  OpScratch sc(d_scratch, d, gemm_partial_bytes(B, d, d, A_KMAJOR));
+  __nv_bfloat16* sbf = sc.take<__nv_bfloat16>((size_t)2 * split_pad(B) * d);
+  float* ss = sc.take<float>((size_t)((d + 127) / 128) * B);
+  CU(cudaMemsetAsync(d_scratch, 0, op_header() + op_counters(d), s));
   long n = (long)B * d;
-  CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, d_s, sbf, n, (long)split_pad(B) * d));
-  CU(cudaGetLastError());
+  CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, d_s, sbf, n,
+                     (long)split_pad(B) * d));
   char msg[256];
   GemmPlan p;
-  if (!gemm_plan(&p, A_KMAJOR, d_w_adapter, nullptr, sbf, B, d, d, partial, msg, sizeof(msg), true))
+  if (!gemm_plan(&p, A_KMAJOR, d_w_adapter, nullptr, sbf, B, d, d, sc.partial, msg, sizeof(msg), true))
     return DLM_EUNSUPPORTED;
-  CU(gemm_launch(p, err, s));
-  EmbedArgs ea{};
-  ea.embed = (const __nv_bfloat16*)d_embed;
-  ea.tokens = d_tokens;
-  ea.adapter = p.out;
-  ea.has_adapter = 1;
-  ea.h = d_h0;
-  ea.d = d;
-  CU_LAUNCH(launch_k(k_embed_adapter_norm, dim3(B), dim3(threads_for(d)), (size_t)d * 4, s, ea));
-  CU(cudaGetLastError());
-  return DLM_OK;
+  EpiArgs e{};
+  e.op = EPI_EMBED;
+  e.h = d_h0;
+  e.ss = ss;
+  e.embed = (const __nv_bfloat16*)d_embed;
+  e.tokens = d_tokens;
+  return op_gemm(p, e, sc, s);
 }
 
 size_t dlm_attention_scratch_size(int T, int Hq, int hd, int max_ctx) {

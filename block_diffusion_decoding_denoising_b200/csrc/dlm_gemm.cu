@@ -23,7 +23,6 @@
 
 namespace dlm {
 
-int g_gemm_impl = 0;
 bool g_pdl = true;
 
 template <int NT>
@@ -32,17 +31,104 @@ struct GemmCfg {
   static constexpr int kBBytes = NT * kTileK * 2;              // NT rows of 128 B
   static constexpr int kStageBytes = kABytes + kBBytes;        // multiple of 1024
   static constexpr int kStages = NT <= 64 ? 8 : (NT <= 128 ? 6 : 4);
-  static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kXchBytes = 128 * 33 * 4;                // epilogue row exchange
+  static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + kXchBytes;
   static constexpr int kTmemCols = (2 * NT < 32) ? 32 : 2 * NT;  // power of two for NT >= 16
 };
 
 struct GemmKArgs {
   int a_mode;
   int T;
+  int N;       // valid output rows (features)
   int lo_col;  // 0, or the MMA column where the low halves of split activations start
   GemmOut out;
+  EpiArgs epi;
   int* err;
 };
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Applies the epilogue op to one block of (up to) 32 tokens of a finished tile.  Runs on the
+// 128 epilogue threads; `row` is this thread's tile row, v[j] its value for token t0 + j.
+__device__ __forceinline__ void finish_block(const GemmKArgs& a, int tile, int row, int t0, const float* v,
+                                             float (*xch)[33], int L) {
+  const EpiArgs& e = a.epi;
+  const int T = a.T;
+  const int nt = (T - t0) < 32 ? (T - t0) : 32;
+  if (e.op == EPI_STORE) {
+    const int n = tile * kTileM + row;
+    if (n < a.N)
+      for (int j = 0; j < nt; ++j) e.out[(size_t)(t0 + j) * e.ld + n] = v[j];
+  } else if (e.op == EPI_RESID || e.op == EPI_EMBED) {
+    const int n = tile * kTileM + row;
+    const bool ok = n < a.N;
+    for (int j = 0; j < 32; ++j) {
+      float hn = 0.f;
+      if (ok && j < nt) {
+        const int t = t0 + j;
+        const float base = (e.op == EPI_RESID) ? e.h[(size_t)t * a.N + n]
+                                               : bf2f(e.embed[(size_t)e.tokens[t] * a.N + n]);
+        hn = base + v[j];
+        e.h[(size_t)t * a.N + n] = hn;
+      }
+      xch[row][j] = hn * hn;
+    }
+    epi_sync();
+    if (row < nt) {
+      float ss = 0.f;
+      for (int r = 0; r < kTileM; ++r) ss += xch[r][row];
+      e.ss[(size_t)tile * T + t0 + row] = ss;
+    }
+    epi_sync();
+  } else if (e.op == EPI_SILU) {
+    for (int j = 0; j < 32; ++j) xch[row][j] = v[j];
+    epi_sync();
+    const int f = tile * 64 + row;
+    if (row < 64 && f < a.N) {
+      for (int j = 0; j < nt; ++j) {
+        const float g = xch[row][j], u = xch[row + 64][j];
+        const float silu = g / (1.0f + expf(-g));
+        store_split(e.act + (size_t)(t0 + j) * a.N + f, e.act_lo, silu * u);
+      }
+    }
+    epi_sync();
+  } else if (e.op == EPI_QKV) {
+    for (int j = 0; j < 32; ++j) xch[row][j] = v[j];
+    epi_sync();
+    const int n = tile * kTileM + row;
+    const int hd = e.hd, half = hd / 2;
+    const int hh = n / hd, jj = n % hd;
+    if (n < a.N) {
+      const int partner = (jj < half) ? row + half : row - half;
+      const bool rope = hh < e.Hq + e.Hkv;
+      const double theta = pow((double)e.rope_theta, -2.0 * (double)(jj % half) / (double)hd);
+      __nv_bfloat16* dst;
+      size_t stride_t;
+      if (hh < e.Hq) {
+        dst = e.q + (size_t)hh * hd + jj;
+        stride_t = (size_t)e.Hq * hd;
+      } else if (hh < e.Hq + e.Hkv) {
+        dst = e.kc + ((size_t)(hh - e.Hq) * e.max_ctx + L) * hd + jj;
+        stride_t = hd;
+      } else {
+        dst = e.vc + ((size_t)(hh - e.Hq - e.Hkv) * e.max_ctx + L) * hd + jj;
+        stride_t = hd;
+      }
+      for (int j = 0; j < nt; ++j) {
+        const int t = t0 + j;
+        float out = xch[row][j];
+        if (rope) {
+          double sn, cs;
+          sincos((double)(L + t) * theta, &sn, &cs);
+          const float c = (float)cs, s = (float)sn, pv = xch[partner][j];
+          out = (jj < half) ? out * c - pv * s : pv * s + out * c;
+        }
+        dst[(size_t)t * stride_t] = f2bf(out);
+      }
+    }
+    epi_sync();
+  }
+}
 
 // 192 threads: warp 0 = TMA producer (and TMEM allocator), warp 1 = MMA issuer,
 // warps 2..5 = epilogue (TMEM lane quarter = warp % 4).
@@ -61,6 +147,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
   uint64_t* acc_empty = bars + 2 * S + 2;  // [2]
   uint64_t* mma_done = bars + 2 * S + 4;   // [1]
   uint32_t* tmem_holder = (uint32_t*)(bars + 2 * S + 5);
+  int* last_flag = (int*)(bars + 2 * S + 6);
+  float(*xch)[33] = reinterpret_cast<float(*)[33]>(smem + S * Cfg::kStageBytes + 256);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const GemmOut& o = args.out;
@@ -86,7 +174,6 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  pdl_trigger();
   if (warp != 0) pdl_wait();  // the producer waits after requesting its first weight tiles
 
   if (warp == 0 && lane == 0) {
@@ -134,6 +221,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
       load_b(u, stage);
       if (++stage == S) { stage = 0; phase ^= 1; }
     }
+    pdl_trigger();  // all loads issued: the next kernel may start its prologue
     // never leave the CTA with copies in flight: wait (bounded) for every armed stage
     for (int i = 0; i < S; ++i)
       if (armed[i]) mbar_wait(&full[i], armed_parity[i], args.err);
@@ -177,42 +265,86 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
     mma_commit(mma_done);
     mbar_wait(mma_done, 0, args.err);
   } else if (warp >= 2) {
-    // ---------------- epilogue: TMEM -> fp32 partials
+    // ---------------- epilogue: TMEM -> partial sums / finished tiles
     const int quarter = warp % 4;
-    const int row = quarter * 32 + lane;
+    const int row = quarter * 32 + lane;  // tile row = TMEM lane
+    const int et = threadIdx.x - 64;      // 0 .. 127
+    const EpiArgs& e = args.epi;
+    const int L = (e.op == EPI_QKV) ? (e.pos0_dev ? *e.pos0_dev : e.pos0) : 0;
+    const int ncb = (args.T + 31) / 32;
     int acc = 0;
     uint32_t acc_phase = 0;
     long u = u_begin;
     float v[32];
+    auto load_block = [&](uint32_t taddr, int cb) {
+      tmem_ld32(taddr + cb * 32, v);
+      if (args.lo_col) {
+        // split activation x = hi + lo: the two column sets add up
+        float w[32];
+        tmem_ld32(taddr + args.lo_col + cb * 32, w);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] += w[j];
+      }
+    };
     while (u < u_end) {
       const int tile = (int)(u / o.n_kb);
       const long seg_end = ((long)tile + 1) * o.n_kb < u_end ? ((long)tile + 1) * o.n_kb : u_end;
       if (!mbar_wait(&acc_full[acc], acc_phase, args.err)) break;
       tc_fence_after();
-      const int slot = c - cta_of_unit((long)tile * o.n_kb, o.units, o.grid);
-      float* dst = o.partial + (((size_t)tile * o.max_slots + slot) * o.T) * kTileM + row;
+      const int lo_c = cta_of_unit((long)tile * o.n_kb, o.units, o.grid);
+      const int hi_c = cta_of_unit((long)(tile + 1) * o.n_kb - 1, o.units, o.grid);
+      const int nslots = hi_c - lo_c + 1, slot = c - lo_c;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * NT;
-      static_assert(NT % 32 == 0, "token tile is a multiple of 32");
-      const int ncb = (args.lo_col ? args.lo_col : NT) / 32;
+      bool finisher = true;
+      if (nslots > 1 || e.op == EPI_PARTIAL) {
+        float* dst = o.partial + (((size_t)tile * o.max_slots + slot) * o.T) * kTileM + row;
 #pragma unroll 1
-      for (int cb = 0; cb < ncb; ++cb) {
-        if (cb * 32 >= o.T) break;
-        tmem_ld32(taddr + cb * 32, v);
-        if (args.lo_col) {
-          // split activation x = hi + lo: the two column sets add up
-          float w[32];
-          tmem_ld32(taddr + args.lo_col + cb * 32, w);
+        for (int cb = 0; cb < ncb; ++cb) {
+          load_block(taddr, cb);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] += w[j];
+          for (int j = 0; j < 32; ++j) {
+            const int t = cb * 32 + j;
+            if (t < o.T) dst[(size_t)t * kTileM] = v[j];
+          }
         }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int t = cb * 32 + j;
-          if (t < o.T) dst[(size_t)t * kTileM] = v[j];
+        tc_fence_before();
+        mbar_arrive(&acc_empty[acc]);  // the accumulator can take the next tile now
+        if (e.op == EPI_PARTIAL) {
+          finisher = false;
+        } else {
+          __threadfence();
+          epi_sync();
+          if (et == 0) *last_flag = (atomicAdd(&e.tile_cnt[tile], 1) == nslots - 1) ? 1 : 0;
+          epi_sync();
+          finisher = *last_flag != 0;
+          if (finisher) __threadfence();
         }
       }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[acc]);
+      if (finisher) {
+#pragma unroll 1
+        for (int cb = 0; cb < ncb; ++cb) {
+          if (nslots == 1) {
+            load_block(taddr, cb);
+          } else {
+            const float* src = o.partial + ((size_t)tile * o.max_slots * o.T) * kTileM + row;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int t = cb * 32 + j;
+              float sum = 0.f;
+              if (t < o.T)
+                for (int sl = 0; sl < nslots; ++sl) sum += __ldcg(src + ((size_t)sl * o.T + t) * kTileM);
+              v[j] = sum;
+            }
+          }
+          finish_block(args, tile, row, cb * 32, v, xch, L);
+        }
+        if (nslots == 1) {
+          tc_fence_before();
+          mbar_arrive(&acc_empty[acc]);
+        } else if (et == 0) {
+          e.tile_cnt[tile] = 0;  // ready for the next GEMM
+        }
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       u = seg_end;
     }
@@ -221,52 +353,6 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem_base, Cfg::kTmemCols);
-}
-
-// ------------------------------------------------------------------ CUDA-core kernel
-// Same output contract with a single slot; a plain reference-grade kernel kept as a
-// debugging aid (selected with dlm_debug_set_gemm_impl(1)).
-struct SimtArgs {
-  const __nv_bfloat16* a0;
-  const __nv_bfloat16* a1;
-  const __nv_bfloat16* x;
-  long lo_off;  // elements from a high row to its low row (split activations), or 0
-  int a_mode, N, K, T;
-  GemmOut out;
-};
-
-__global__ void k_gemm_simt(SimtArgs a) {
-  const int tile = blockIdx.x, row = threadIdx.x, t = blockIdx.y;
-  if (t >= a.T) return;
-  const __nv_bfloat16* xr = a.x + (size_t)t * a.K;
-  const __nv_bfloat16* wr = nullptr;
-  bool valid = true;
-  if (a.a_mode == A_KMAJOR) {
-    int n = tile * kTileM + row;
-    valid = n < a.N;
-    wr = a.a0 + (size_t)n * a.K;
-  } else if (a.a_mode == A_PAIR) {
-    int f = tile * 64 + (row % 64);
-    valid = f < a.N;
-    wr = (row < 64 ? a.a0 : a.a1) + (size_t)f * a.K;
-  }
-  float acc = 0.f;
-  if (valid) {
-    if (a.a_mode == A_MNMAJOR) {
-      int n = tile * kTileM + row;
-      if (n < a.N)
-        for (int k = 0; k < a.K; ++k) {
-          float xv = bf2f(xr[k]) + (a.lo_off ? bf2f(xr[k + a.lo_off]) : 0.f);
-          acc += xv * bf2f(a.a0[(size_t)k * a.N + n]);
-        }
-    } else {
-      for (int k = 0; k < a.K; ++k) {
-        float xv = bf2f(xr[k]) + (a.lo_off ? bf2f(xr[k + a.lo_off]) : 0.f);
-        acc += xv * bf2f(wr[k]);
-      }
-    }
-  }
-  a.out.partial[((size_t)tile * a.out.max_slots) * a.out.T * kTileM + (size_t)t * kTileM + row] = acc;
 }
 
 // ------------------------------------------------------------------ host side
@@ -324,16 +410,13 @@ static void partition(int T, int N, int K, int a_mode, GemmOut* o) {
   o->n_kb = (K + kTileK - 1) / kTileK;
   o->units = (long)o->n_tiles * o->n_kb;
   int grid = kSMs;
-  if (g_gemm_impl == 1) grid = o->n_tiles;
   if (o->units < grid) grid = (int)o->units;
   o->grid = grid;
   int ms = 1;
-  if (g_gemm_impl != 1) {
-    for (int t = 0; t < o->n_tiles; ++t) {
-      int lo = cta_of_unit((long)t * o->n_kb, o->units, grid);
-      int hi = cta_of_unit((long)(t + 1) * o->n_kb - 1, o->units, grid);
-      if (hi - lo + 1 > ms) ms = hi - lo + 1;
-    }
+  for (int t = 0; t < o->n_tiles; ++t) {
+    int lo = cta_of_unit((long)t * o->n_kb, o->units, grid);
+    int hi = cta_of_unit((long)(t + 1) * o->n_kb - 1, o->units, grid);
+    if (hi - lo + 1 > ms) ms = hi - lo + 1;
   }
   o->max_slots = ms;
 }
@@ -387,8 +470,10 @@ static cudaError_t launch_nt(const GemmPlan& p, int* d_err, cudaStream_t s) {
   GemmKArgs a;
   a.a_mode = p.a_mode;
   a.T = p.T;
+  a.N = p.N;
   a.lo_col = p.lo_col;
   a.out = p.out;
+  a.epi = p.epi;
   a.err = d_err;
   return launch_k(k_gemm_tc<NT>, dim3(p.out.grid), dim3(192), GemmCfg<NT>::kSmem, s, p.ta0, p.ta1, p.tb, a);
 }
@@ -411,32 +496,13 @@ int gemm_init_attributes() {
   return (int)e;
 }
 
-static cudaError_t gemm_launch_simt(const GemmPlan& p, cudaStream_t s);
-
 cudaError_t gemm_launch(const GemmPlan& p, int* d_err, cudaStream_t s) {
-  if (g_gemm_impl == 1) return gemm_launch_simt(p, s);
   switch (p.nt) {
     case 32: return launch_nt<32>(p, d_err, s);
     case 64: return launch_nt<64>(p, d_err, s);
     case 128: return launch_nt<128>(p, d_err, s);
     default: return launch_nt<256>(p, d_err, s);
   }
-}
-
-static cudaError_t gemm_launch_simt(const GemmPlan& p, cudaStream_t s) {
-  SimtArgs a;
-  a.a0 = (const __nv_bfloat16*)p.a0;
-  a.a1 = (const __nv_bfloat16*)p.a1;
-  a.x = (const __nv_bfloat16*)p.x;
-  a.lo_off = (long)p.lo_col * p.K;
-  a.a_mode = p.a_mode;
-  a.N = p.N;
-  a.K = p.K;
-  a.T = p.T;
-  a.out = p.out;
-  dim3 grid(p.out.n_tiles, p.T);
-  k_gemm_simt<<<grid, kTileM, 0, s>>>(a);
-  return cudaGetLastError();
 }
 
 }  // namespace dlm

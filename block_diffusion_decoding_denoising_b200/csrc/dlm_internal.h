@@ -56,8 +56,40 @@ enum AMode : int {
   A_MNMAJOR = 2,  // A^T stored [K][N] (e.g. E [V][d] for s = P E): two 64-column boxes
 };
 
+// What the GEMM does with a finished output tile.  The CTA that completes a tile (the only
+// CTA of a single-slot tile, else the last of its slots to arrive, found with a per-tile
+// counter) sums the slots in slot order and applies the op; the counter is reset to zero
+// for the next GEMM.
+enum EpiOp : int {
+  EPI_PARTIAL = 0,  // leave the per-slot partial sums only (kernel timing)
+  EPI_STORE = 1,    // out[t][n] = y (fp32)
+  EPI_QKV = 2,      // RoPE on q/k heads, bf16 q and K/V cache rows at position L + t
+  EPI_RESID = 3,    // h[t][n] += y; ss[tile][t] = sum of h^2 over the tile's rows
+  EPI_SILU = 4,     // gate/up pair: act[t][f] = silu(g) * u as a split bf16 pair
+  EPI_EMBED = 5,    // h[t][n] = E[token_t][n] + y; ss[tile][t] as EPI_RESID
+};
+
+struct EpiArgs {
+  int op;
+  int* tile_cnt;                // [n_tiles] arrival counters, zero between GEMMs
+  float* out;                   // EPI_STORE
+  int ld;
+  __nv_bfloat16 *q, *kc, *vc;   // EPI_QKV
+  int Hq, Hkv, hd, max_ctx;
+  int pos0;
+  const int* pos0_dev;
+  float rope_theta;
+  float* h;                     // EPI_RESID / EPI_EMBED: [T][d]
+  float* ss;                    // [n_tiles][T]
+  const __nv_bfloat16* embed;   // EPI_EMBED
+  const int32_t* tokens;
+  __nv_bfloat16* act;           // EPI_SILU: [T][F] high halves
+  long act_lo;
+};
+
 struct GemmPlan {
   CUtensorMap ta0, ta1, tb;
+  EpiArgs epi;
   int a_mode;
   int nt;            // MMA N (tokens padded to 32/64/128/256; twice the pad when split)
   int lo_col;        // split activations: MMA column of the low halves (= pad), else 0
@@ -79,7 +111,6 @@ bool gemm_plan(GemmPlan* p, int a_mode, const void* a0, const void* a1, const vo
                int N, int K, float* partial, char* err, size_t errlen, bool split = false);
 cudaError_t gemm_launch(const GemmPlan& p, int* d_err, cudaStream_t s);
 int gemm_init_attributes();
-extern int g_gemm_impl;  // 0 = tcgen05 (default), 1 = plain CUDA-core kernel (debug aid)
 
 // attention (dlm_attention.cu)
 struct AttnArgs {

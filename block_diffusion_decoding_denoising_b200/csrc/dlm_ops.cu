@@ -44,99 +44,40 @@ __device__ void norm_row_to_bf16(const float* row, int d, const __nv_bfloat16* g
   for (int n = threadIdx.x; n < d; n += blockDim.x) store_split(out + n, lo_off, row[n] * r * bf2f(g[n]));
 }
 
-// h[t] = E[tok_t] (+ W_a s_t from the GEMM partials when `has_adapter`), then
-// xn[t] = RMSNorm(h[t]) with gain g.  One CTA per token.
-__global__ void k_embed_adapter_norm(EmbedArgs a) {
+// h[t][n] = E[tok_t][n] and ss[tile][t] = sum over the tile's 128 features of h^2 (the
+// same per-tile layout the GEMM's residual epilogue writes).  grid (ceil(d/128), T), 128 thr.
+__global__ void k_embed_rows(EmbedRowsArgs a) {
   pdl_trigger();
   pdl_wait();
-  extern __shared__ float rowbuf[];
-  __shared__ float red[32];
-  const int t = blockIdx.x;
-  const int tok = a.tokens[t];
-  const __nv_bfloat16* e = a.embed + (size_t)tok * a.d;
-  for (int n = threadIdx.x; n < a.d; n += blockDim.x) {
-    float v = bf2f(e[n]);
-    if (a.has_adapter) v += gemm_out(a.adapter, n, t);
-    rowbuf[n] = v;
+  __shared__ float red[128];
+  const int tile = blockIdx.x, t = blockIdx.y, r = threadIdx.x;
+  const int n = tile * 128 + r;
+  float v = 0.f;
+  if (n < a.d) {
+    v = bf2f(a.embed[(size_t)a.tokens[t] * a.d + n]);
     a.h[(size_t)t * a.d + n] = v;
   }
+  red[r] = v * v;
   __syncthreads();
-  if (a.gain) norm_row_to_bf16(rowbuf, a.d, a.gain, a.eps, a.xn + (size_t)t * a.d, a.xn_lo, red);
-}
-
-// h[t] += y[t] (GEMM output of W_o or W_d); xn[t] = RMSNorm(h[t]) with the next gain.
-__global__ void k_residual_norm(ResidArgs a) {
-  pdl_trigger();
-  pdl_wait();
-  extern __shared__ float rowbuf[];
-  __shared__ float red[32];
-  const int t = blockIdx.x;
-  for (int n = threadIdx.x; n < a.d; n += blockDim.x) {
-    float v = a.h[(size_t)t * a.d + n] + gemm_out(a.y, n, t);
-    rowbuf[n] = v;
-    a.h[(size_t)t * a.d + n] = v;
+  if (r == 0) {
+    float ss = 0.f;
+    for (int i = 0; i < 128; ++i) ss += red[i];
+    a.ss[(size_t)tile * a.T + t] = ss;
   }
-  __syncthreads();
-  if (a.gain) norm_row_to_bf16(rowbuf, a.d, a.gain, a.eps, a.xn + (size_t)t * a.d, a.xn_lo, red);
 }
 
-// QKV projection output -> RoPE (NeoX pairing (j, j + hd/2), theta_j = base^(-2j/hd),
-// absolute position L + t; angles in double precision) -> bf16 q and the K/V cache rows.
-// grid (Hq + 2 Hkv, T), hd/2 threads.
-__global__ void k_qkv_rope(QkvArgs a) {
-  pdl_trigger();
-  pdl_wait();
-  const int hh = blockIdx.x, t = blockIdx.y, j = threadIdx.x;
-  const int hd = a.hd, half = hd / 2;
-  if (j >= half) return;
-  const int L = a.pos0_dev ? *a.pos0_dev : a.pos0;
-  const long pos = (long)L + t;
-  float x0 = gemm_out(a.y, hh * hd + j, t);
-  float x1 = gemm_out(a.y, hh * hd + j + half, t);
-  if (hh < a.Hq + a.Hkv) {
-    double theta = pow(a.rope_theta, -2.0 * (double)j / (double)hd);
-    double s, c;
-    sincos((double)pos * theta, &s, &c);
-    float cf = (float)c, sf = (float)s;
-    float r0 = x0 * cf - x1 * sf;
-    float r1 = x0 * sf + x1 * cf;
-    x0 = r0;
-    x1 = r1;
-  }
-  __nv_bfloat16* dst;
-  if (hh < a.Hq) {
-    dst = a.q + ((size_t)t * a.Hq + hh) * hd;
-  } else if (hh < a.Hq + a.Hkv) {
-    dst = a.kc + ((size_t)(hh - a.Hq) * a.max_ctx + pos) * hd;
-  } else {
-    dst = a.vc + ((size_t)(hh - a.Hq - a.Hkv) * a.max_ctx + pos) * hd;
-  }
-  dst[j] = f2bf(x0);
-  dst[j + half] = f2bf(x1);
-}
-
-// a[t][f] = bf16(silu(g) * u), g and u from the paired gate/up GEMM (tile = 64 + 64 rows).
-__global__ void k_silu_gate(SiluArgs a) {
-  pdl_trigger();
-  pdl_wait();
-  const int t = blockIdx.y;
-  const int f = blockIdx.x * blockDim.x + threadIdx.x;
-  if (f >= a.F) return;
-  const int tile = f / 64, r = f % 64;
-  const float g = gemm_sum(a.y, tile, r, t);
-  const float u = gemm_sum(a.y, tile, 64 + r, t);
-  const float silu = g / (1.0f + expf(-g));
-  store_split(a.out + (size_t)t * a.F + f, a.lo, silu * u);
-}
-
-// out[t][n] = y[t][n] (fp32), n < N.
-__global__ void k_store_rows(StoreArgs a) {
+// xn[t][n] = split bf16 of h[t][n] * r_t * g[n], r_t = 1 / sqrt(sum_tiles ss[tile][t] / d + eps)
+// (RMSNorm; the sums of squares come per 128-feature tile from the producing kernel).
+// grid (ceil(d/256), T), 256 threads.
+__global__ void k_norm_apply(NormArgs a) {
   pdl_trigger();
   pdl_wait();
   const int t = blockIdx.y;
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= a.N) return;
-  a.out[(size_t)t * a.ld + n] = gemm_out(a.y, n, t);
+  float ss = 0.f;
+  for (int i = 0; i < a.n_tiles; ++i) ss += a.ss[(size_t)i * a.T + t];
+  const float r = 1.0f / sqrtf(ss / (float)a.d + a.eps);
+  if (n < a.d) store_split(a.xn + (size_t)t * a.d + n, a.xn_lo, a.h[(size_t)t * a.d + n] * r * bf2f(a.gain[n]));
 }
 
 // Split bf16 copy of s (the W_a GEMM input): high halves at y[i], low halves at y[i + lo].
@@ -147,28 +88,29 @@ __global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo) {
   if (i < n) store_split(y + i, lo, x[i]);
 }
 
-// Row statistics of logits[b][:] (mask id excluded) and P = softmax as bf16.
-// m = max, argmax = lowest id of the max, Z = sum e^(l-m), lse = m + ln Z,
-// maxprob = 1/Z, entropy = ln Z - sum e^(l-m)(l-m) / Z.  One CTA per row.
-__global__ void k_rowstats(RowStatsArgs a) {
+// Row statistics, phase 1: for logits[b][chunk] (mask id excluded) the chunk's max m_c,
+// its lowest argmax, Z_c = sum e^(l - m_c) and A_c = sum e^(l - m_c) (l - m_c).
+// grid (n_chunks, B), 256 threads.
+__global__ void k_rowstats_part(RowStatsArgs a) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red_v[32];
   __shared__ int red_i[32];
-  __shared__ float bcast[2];
-  const int b = blockIdx.x;
+  __shared__ float bc;
+  const int ch = blockIdx.x, b = blockIdx.y;
+  const int v0 = ch * a.chunk, v1 = min(a.V, v0 + a.chunk);
   const float* l = a.logits + (size_t)b * a.ld;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nw = blockDim.x / 32;
   float m = -INFINITY;
   int am = 0x7fffffff;
-  for (int v = threadIdx.x; v < a.V; v += blockDim.x) {
+  for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
     if (v == a.mask_id) continue;
-    float x = l[v];
+    const float x = l[v];
     if (x > m || (x == m && v < am)) { m = x; am = v; }
   }
   for (int o = 16; o > 0; o >>= 1) {
-    float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-    int a2 = __shfl_xor_sync(0xffffffffu, am, o);
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const int a2 = __shfl_xor_sync(0xffffffffu, am, o);
     if (m2 > m || (m2 == m && a2 < am)) { m = m2; am = a2; }
   }
   if (lane == 0) { red_v[warp] = m; red_i[warp] = am; }
@@ -178,35 +120,70 @@ __global__ void k_rowstats(RowStatsArgs a) {
     int aa = red_i[0];
     for (int i = 1; i < nw; ++i)
       if (red_v[i] > mm || (red_v[i] == mm && red_i[i] < aa)) { mm = red_v[i]; aa = red_i[i]; }
-    bcast[0] = mm;
+    bc = mm;
     red_i[0] = aa;
   }
   __syncthreads();
-  m = bcast[0];
+  m = bc;
   am = red_i[0];
   __syncthreads();
   float z = 0.f, A = 0.f;
-  for (int v = threadIdx.x; v < a.V; v += blockDim.x) {
-    if (v == a.mask_id) continue;
-    float x = l[v] - m;
-    float e = expf(x);
-    z += e;
-    A += e * x;
+  if (m > -INFINITY) {
+    for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
+      if (v == a.mask_id) continue;
+      const float x = l[v] - m;
+      const float ex = expf(x);
+      z += ex;
+      A += ex * x;
+    }
   }
   z = block_sum(z, red_v);
   A = block_sum(A, red_v);
-  const float lnz = logf(z);
-  const float lse = m + lnz;
   if (threadIdx.x == 0) {
-    a.stats.m[b] = m;
+    float4* p = reinterpret_cast<float4*>(a.part) + (size_t)b * gridDim.x + ch;
+    *p = make_float4(m, __int_as_float(am), z, A);
+  }
+}
+
+// Row statistics, phase 2: merges the chunk partials of row b (every CTA redundantly, in
+// chunk order), chunk 0 writes the statistics, and every CTA writes its chunk of
+// P = softmax as a split bf16 pair.  Merge: M = max m_c, Z = sum_c e^(m_c - M) Z_c,
+// A = sum_c e^(m_c - M) (A_c + (m_c - M) Z_c); lse = M + ln Z, maxprob = 1/Z,
+// entropy = ln Z - A / Z.  grid (n_chunks, B), 256 threads.
+__global__ void k_rowstats_final(RowStatsArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const int ch = blockIdx.x, b = blockIdx.y, nch = gridDim.x;
+  const float4* part = reinterpret_cast<const float4*>(a.part) + (size_t)b * nch;
+  float M = -INFINITY;
+  int am = 0x7fffffff;
+  for (int i = 0; i < nch; ++i) {
+    const float4 q = part[i];
+    const int ai = __float_as_int(q.y);
+    if (q.x > M) { M = q.x; am = ai; }  // chunks in id order: the first maximal chunk wins
+  }
+  float Z = 0.f, A = 0.f;
+  for (int i = 0; i < nch; ++i) {
+    const float4 q = part[i];
+    if (q.x == -INFINITY) continue;
+    const float w = expf(q.x - M);
+    Z += w * q.z;
+    A += w * (q.w + (q.x - M) * q.z);
+  }
+  const float lnz = logf(Z);
+  const float lse = M + lnz;
+  if (ch == 0 && threadIdx.x == 0) {
+    a.stats.m[b] = M;
     a.stats.lse[b] = lse;
-    a.stats.maxprob[b] = 1.0f / z;
-    a.stats.entropy[b] = lnz - A / z;
+    a.stats.maxprob[b] = 1.0f / Z;
+    a.stats.entropy[b] = lnz - A / Z;
     a.stats.argmax[b] = am;
   }
   if (a.P) {
+    const int v0 = ch * a.chunk, v1 = min(a.V, v0 + a.chunk);
+    const float* l = a.logits + (size_t)b * a.ld;
     __nv_bfloat16* p = a.P + (size_t)b * a.V;
-    for (int v = threadIdx.x; v < a.V; v += blockDim.x)
+    for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x)
       store_split(p + v, a.P_lo, v == a.mask_id ? 0.f : expf(l[v] - lse));
   }
 }

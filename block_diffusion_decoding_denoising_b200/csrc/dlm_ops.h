@@ -7,52 +7,22 @@
 
 namespace dlm {
 
-struct EmbedArgs {
+struct EmbedRowsArgs {
   const __nv_bfloat16* embed;  // [V][d]
   const int32_t* tokens;       // [T]
-  GemmOut adapter;             // W_a s partials (when has_adapter)
-  int has_adapter;
   float* h;                    // [T][d]
-  __nv_bfloat16* xn;           // [T][d] high halves
-  long xn_lo;                  // elements to the low halves (split activations), 0 = none
+  float* ss;                   // [ceil(d/128)][T]
+  int d, T;
+};
+
+struct NormArgs {
+  const float* h;              // [T][d]
+  const float* ss;             // [n_tiles][T]
   const __nv_bfloat16* gain;   // [d]
-  int d;
+  __nv_bfloat16* xn;           // [T][d] high halves
+  long xn_lo;                  // elements to the low halves
+  int d, T, n_tiles;
   float eps;
-};
-
-struct ResidArgs {
-  GemmOut y;
-  float* h;
-  __nv_bfloat16* xn;
-  long xn_lo;
-  const __nv_bfloat16* gain;  // nullptr: skip the norm
-  int d;
-  float eps;
-};
-
-struct QkvArgs {
-  GemmOut y;
-  __nv_bfloat16* q;   // [T][Hq][hd]
-  __nv_bfloat16* kc;  // [Hkv][max_ctx][hd] of this layer
-  __nv_bfloat16* vc;
-  int Hq, Hkv, hd, max_ctx;
-  int pos0;
-  const int* pos0_dev;
-  double rope_theta;
-};
-
-struct SiluArgs {
-  GemmOut y;
-  __nv_bfloat16* out;  // [T][F] high halves
-  long lo;             // elements to the low halves
-  int F;
-};
-
-struct StoreArgs {
-  GemmOut y;
-  float* out;
-  int N;
-  int ld;
 };
 
 struct RowStatsArgs {
@@ -60,6 +30,8 @@ struct RowStatsArgs {
   int ld;
   int V;
   int mask_id;
+  int chunk;            // vocabulary entries per CTA
+  float* part;          // [B][n_chunks] float4 (m, argmax bits, Z, A)
   dlm_row_stats stats;
   __nv_bfloat16* P;     // [B][V] high halves, or nullptr
   long P_lo;            // elements to the low halves, 0 = none
@@ -100,13 +72,11 @@ struct BlockFinishArgs {
   int B;
 };
 
-__global__ void k_embed_adapter_norm(EmbedArgs a);
-__global__ void k_residual_norm(ResidArgs a);
-__global__ void k_qkv_rope(QkvArgs a);
-__global__ void k_silu_gate(SiluArgs a);
-__global__ void k_store_rows(StoreArgs a);
+__global__ void k_embed_rows(EmbedRowsArgs a);
+__global__ void k_norm_apply(NormArgs a);
 __global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo);
-__global__ void k_rowstats(RowStatsArgs a);
+__global__ void k_rowstats_part(RowStatsArgs a);
+__global__ void k_rowstats_final(RowStatsArgs a);
 __global__ void k_commit(CommitArgs a);
 __global__ void k_block_init(BlockInitArgs a);
 __global__ void k_block_finish(BlockFinishArgs a);

@@ -112,7 +112,6 @@ def lib():
         L.dlm_bd_attention.argtypes = [p, p, p, p, i, i, i, i, i, i, i, p, z, p]
         L.dlm_commit.argtypes = [p, p, p, p, p, p, p, i, i, f, i, i, p]
         L.dlm_nvfp4_quantize.argtypes = [p, i, i, p, p, p, p]
-        L.dlm_debug_set_gemm_impl.argtypes = [i]
         L.dlm_debug_set_pdl.argtypes = [i]
         _lib = L
     return _lib
@@ -135,10 +134,6 @@ def _check(st, ctx=None):
             m = lib().dlm_last_error(ctx)
             msg = m.decode() if m else ""
         raise DlmError(st, msg)
-
-
-def set_gemm_impl(impl: int) -> None:
-    lib().dlm_debug_set_gemm_impl(int(impl))
 
 
 def set_pdl(on: bool) -> None:

@@ -245,10 +245,6 @@ dlm_status dlm_nvfp4_quantize(const void* d_w, int rows, int cols, void* d_codes
 /* Version string of the build. */
 const char* dlm_version(void);
 
-/* Debugging aid: 0 (default) runs the dense projections on the tcgen05 tensor-core GEMM,
- * 1 on a plain CUDA-core kernel with the same output contract (slow; for cross-checks). */
-void dlm_debug_set_gemm_impl(int impl);
-
 /* Debugging aid: 1 (default) launches the kernels of a round with programmatic dependent
  * launch (each kernel starts while its predecessor drains; weight tiles are prefetched
  * before the dependency resolves), 0 launches them plainly stream-ordered. */

@@ -57,18 +57,6 @@ def test_gemm_split_activation_parity(lib, T, N, K):
     assert rel_err(O.linear(bf16_f64(xb), wb), ref) > 20 * e
 
 
-def test_gemm_cuda_core_debug_path_matches(lib):
-    T, N, K = 16, 300, 256
-    xb = _bits(7, (T, K))
-    wb = _bits(8, (N, K), 0.02)
-    lib.set_gemm_impl(1)
-    try:
-        y = lib.gemm_bf16(to_torch_bf16(xb), to_torch_bf16(wb)).cpu().numpy()
-    finally:
-        lib.set_gemm_impl(0)
-    assert_close(y, O.linear(bf16_f64(xb), wb), 1e-3, "simt gemm")
-
-
 # ------------------------------------------------------------------ attention
 def _attn_case(lib, B, L, Hq=32, Hkv=8, hd=128, causal=False, rows=None, seed=0):
     import torch
