@@ -289,7 +289,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
     while (u < u_end) {
       const int tile = (int)(u / o.n_kb);
       const long seg_end = ((long)tile + 1) * o.n_kb < u_end ? ((long)tile + 1) * o.n_kb : u_end;
-      if (!mbar_wait(&acc_full[acc], acc_phase, args.err)) break;
+      // one thread polls the accumulator barrier; the named barrier hands the outcome to
+      // all 128 epilogue threads so they leave (on a timeout) or go on together
+      if (et == 0) *last_flag = mbar_wait(&acc_full[acc], acc_phase, args.err) ? 1 : 0;
+      epi_sync();
+      const bool got = *last_flag != 0;
+      epi_sync();
+      if (!got) break;
       tc_fence_after();
       const int lo_c = cta_of_unit((long)tile * o.n_kb, o.units, o.grid);
       const int hi_c = cta_of_unit((long)(tile + 1) * o.n_kb - 1, o.units, o.grid);
