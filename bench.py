@@ -49,6 +49,7 @@ def parse():
     # the quick case with eager dlm_round / dlm_kv_fill calls instead of the block graph
     # (same kernels; ncu cannot profile kernel nodes of graphs with conditional nodes)
     ap.add_argument("--eager", action="store_true")
+    ap.add_argument("--pdl", type=int, default=1, help=argparse.SUPPRESS)
     return ap.parse_args()
 
 
@@ -246,6 +247,7 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     build.build()
+    dlm.set_pdl(bool(args.pdl))
     dev = torch.device("cuda", local)
     B = cfg["block_size"]
     blocks = GEN // B

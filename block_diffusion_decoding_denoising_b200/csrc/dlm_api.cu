@@ -66,6 +66,7 @@ struct dlm_ctx {
   int* tile_cnt = nullptr;   // per-tile arrival counters of the GEMM epilogue
   float* ss = nullptr;       // per-tile sums of squares [ceil(d/128)][Tmax]
   float* rs_part = nullptr;  // row-statistics chunk partials
+  float2* rope_tab = nullptr;  // [max_ctx][hd/2] (cos, sin)
   float* attn_part = nullptr;
   int attn_splits_B = 1, attn_splits_T = 1;
   float* logits = nullptr;
@@ -162,6 +163,7 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   int* cnt = cv.take<int>((size_t)(c.vocab + 63) / 64 + (c.ffn + 63) / 64 + 64);
   float* ssb = cv.take<float>((size_t)((c.d + 127) / 128) * Tmax);
   float* rsp = cv.take<float>((size_t)4 * B * ((c.vocab + kRowChunk - 1) / kRowChunk));
+  float2* rtab = cv.take<float2>((size_t)c.max_ctx * (c.head_dim / 2));
   int sB = attention_max_splits(B, c.n_q_heads, c.n_kv_heads, c.max_ctx);
   int sT = attention_max_splits(Tmax, c.n_q_heads, c.n_kv_heads, c.max_ctx);
   size_t ab = attention_scratch_bytes(B, c.n_q_heads, c.head_dim, sB);
@@ -192,6 +194,7 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
     x->tile_cnt = cnt;
     x->ss = ssb;
     x->rs_part = rsp;
+    x->rope_tab = rtab;
     x->attn_part = attn;
     x->attn_splits_B = sB;
     x->attn_splits_T = sT;
@@ -330,7 +333,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     eq.max_ctx = c.max_ctx;
     eq.pos0 = f.pos0;
     eq.pos0_dev = f.dev_L ? ctx->d_L : nullptr;
-    eq.rope_theta = c.rope_theta;
+    eq.rope_tab = ctx->rope_tab;
     TRY(r.gemm(A_KMAJOR, W.w_qkv, nullptr, ctx->xn, T, nqkv, d, eq));
     // the last layer's K/V do not depend on anything after its QKV projection
     if (!f.lm_head && l == c.n_layers - 1) break;
@@ -568,6 +571,12 @@ dlm_status dlm_ctx_create(const dlm_config* cfg, const dlm_weights* w, void* d_w
   carve(ctx, *cfg, ctx->ws);
   cudaError_t e = cudaStreamCreateWithFlags(&ctx->cap_stream, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaMemsetAsync(ctx->ws, 0, ws_bytes, ctx->cap_stream);
+  if (e == cudaSuccess) {
+    const long nrt = (long)cfg->max_ctx * (cfg->head_dim / 2);
+    k_rope_table<<<(unsigned)((nrt + 255) / 256), 256, 0, ctx->cap_stream>>>(ctx->rope_tab, cfg->max_ctx,
+                                                                          cfg->head_dim, (double)cfg->rope_theta);
+    e = cudaGetLastError();
+  }
   if (e == cudaSuccess) e = (cudaError_t)gemm_init_attributes();
   if (e == cudaSuccess) e = (cudaError_t)attention_init_attributes();
   if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->cap_stream);
@@ -794,7 +803,8 @@ static dlm_status gemm_op(const void* d_x, const void* d_w, float* d_y, int T, i
   GemmPlan p;
   if (!gemm_plan(&p, A_KMAJOR, d_w, nullptr, d_x, T, N, K, sc.partial, msg, sizeof(msg), split))
     return DLM_EUNSUPPORTED;
-  CU(cudaMemsetAsync(d_scratch, 0, op_header() + op_counters(N), s));
+  // the status word and tile counters start at zero (a partial-sums-only call uses neither)
+  if (d_y) CU(cudaMemsetAsync(d_scratch, 0, op_header() + op_counters(N), s));
   EpiArgs e{};
   e.op = d_y ? EPI_STORE : EPI_PARTIAL;  // no output: the tensor-core kernel alone
   e.out = d_y;

@@ -50,18 +50,23 @@ __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" :::
 
 // Applies the epilogue op to one block of (up to) 32 tokens of a finished tile.  Runs on the
 // 128 epilogue threads; `row` is this thread's tile row, v[j] its value for token t0 + j.
-__device__ __forceinline__ void finish_block(const GemmKArgs& a, int tile, int row, int t0, const float* v,
+__device__ __forceinline__ void finish_block(const GemmKArgs& a, int tile, int row, int t0, const float (&v)[32],
                                              float (*xch)[33], int L) {
   const EpiArgs& e = a.epi;
   const int T = a.T;
   const int nt = (T - t0) < 32 ? (T - t0) : 32;
   if (e.op == EPI_STORE) {
     const int n = tile * kTileM + row;
-    if (n < a.N)
-      for (int j = 0; j < nt; ++j) e.out[(size_t)(t0 + j) * e.ld + n] = v[j];
+    if (n < a.N) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < nt) e.out[(size_t)(t0 + j) * e.ld + n] = v[j];
+    }
   } else if (e.op == EPI_RESID || e.op == EPI_EMBED) {
     const int n = tile * kTileM + row;
     const bool ok = n < a.N;
+    const __nv_bfloat16* erow = nullptr;
+#pragma unroll
     for (int j = 0; j < 32; ++j) {
       float hn = 0.f;
       if (ok && j < nt) {
@@ -73,6 +78,7 @@ __device__ __forceinline__ void finish_block(const GemmKArgs& a, int tile, int r
       }
       xch[row][j] = hn * hn;
     }
+    (void)erow;
     epi_sync();
     if (row < nt) {
       float ss = 0.f;
@@ -81,18 +87,23 @@ __device__ __forceinline__ void finish_block(const GemmKArgs& a, int tile, int r
     }
     epi_sync();
   } else if (e.op == EPI_SILU) {
+#pragma unroll
     for (int j = 0; j < 32; ++j) xch[row][j] = v[j];
     epi_sync();
     const int f = tile * 64 + row;
     if (row < 64 && f < a.N) {
-      for (int j = 0; j < nt; ++j) {
-        const float g = xch[row][j], u = xch[row + 64][j];
-        const float silu = g / (1.0f + expf(-g));
-        store_split(e.act + (size_t)(t0 + j) * a.N + f, e.act_lo, silu * u);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j < nt) {
+          const float g = xch[row][j], u = xch[row + 64][j];
+          const float silu = g / (1.0f + expf(-g));
+          store_split(e.act + (size_t)(t0 + j) * a.N + f, e.act_lo, silu * u);
+        }
       }
     }
     epi_sync();
   } else if (e.op == EPI_QKV) {
+#pragma unroll
     for (int j = 0; j < 32; ++j) xch[row][j] = v[j];
     epi_sync();
     const int n = tile * kTileM + row;
@@ -101,7 +112,7 @@ __device__ __forceinline__ void finish_block(const GemmKArgs& a, int tile, int r
     if (n < a.N) {
       const int partner = (jj < half) ? row + half : row - half;
       const bool rope = hh < e.Hq + e.Hkv;
-      const double theta = pow((double)e.rope_theta, -2.0 * (double)(jj % half) / (double)hd);
+      const float2* tab = e.rope_tab + (jj % half);  // (cos, sin) at [position][jj % half]
       __nv_bfloat16* dst;
       size_t stride_t;
       if (hh < e.Hq) {
@@ -114,16 +125,18 @@ __device__ __forceinline__ void finish_block(const GemmKArgs& a, int tile, int r
         dst = e.vc + ((size_t)(hh - e.Hq - e.Hkv) * e.max_ctx + L) * hd + jj;
         stride_t = hd;
       }
-      for (int j = 0; j < nt; ++j) {
-        const int t = t0 + j;
-        float out = xch[row][j];
-        if (rope) {
-          double sn, cs;
-          sincos((double)(L + t) * theta, &sn, &cs);
-          const float c = (float)cs, s = (float)sn, pv = xch[partner][j];
-          out = (jj < half) ? out * c - pv * s : pv * s + out * c;
+#pragma unroll 4
+      for (int j = 0; j < 32; ++j) {
+        if (j < nt) {
+          const int t = t0 + j;
+          float out = xch[row][j];
+          if (rope) {
+            const float2 cs = tab[(size_t)(L + t) * half];
+            const float pv = xch[partner][j];
+            out = (jj < half) ? out * cs.x - pv * cs.y : pv * cs.y + out * cs.x;
+          }
+          dst[(size_t)t * stride_t] = f2bf(out);
         }
-        dst[(size_t)t * stride_t] = f2bf(out);
       }
     }
     epi_sync();
@@ -275,6 +288,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
     int acc = 0;
     uint32_t acc_phase = 0;
     long u = u_begin;
+    const int TP = ncb * 32;  // tokens padded to 32 in the partial layout
     float v[32];
     auto load_block = [&](uint32_t taddr, int cb) {
       tmem_ld32(taddr + cb * 32, v);
@@ -301,17 +315,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
       const int hi_c = cta_of_unit((long)(tile + 1) * o.n_kb - 1, o.units, o.grid);
       const int nslots = hi_c - lo_c + 1, slot = c - lo_c;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * NT;
+      // partials: [tile][slot][row][TP] fp32, each thread's tokens contiguous
+      float* const tile_part = o.partial + (size_t)tile * o.max_slots * kTileM * TP + (size_t)row * TP;
       bool finisher = true;
       if (nslots > 1 || e.op == EPI_PARTIAL) {
-        float* dst = o.partial + (((size_t)tile * o.max_slots + slot) * o.T) * kTileM + row;
+        float4* dst = reinterpret_cast<float4*>(tile_part + (size_t)slot * kTileM * TP);
 #pragma unroll 1
         for (int cb = 0; cb < ncb; ++cb) {
           load_block(taddr, cb);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int t = cb * 32 + j;
-            if (t < o.T) dst[(size_t)t * kTileM] = v[j];
-          }
+          for (int q = 0; q < 8; ++q) dst[cb * 8 + q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[acc]);  // the accumulator can take the next tile now
@@ -323,6 +336,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
           if (et == 0) *last_flag = (atomicAdd(&e.tile_cnt[tile], 1) == nslots - 1) ? 1 : 0;
           epi_sync();
           finisher = *last_flag != 0;
+          epi_sync();  // the flag is rewritten by the next segment's wait
           if (finisher) __threadfence();
         }
       }
@@ -332,14 +346,36 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
           if (nslots == 1) {
             load_block(taddr, cb);
           } else {
-            const float* src = o.partial + ((size_t)tile * o.max_slots * o.T) * kTileM + row;
+            // sum the slots in slot order, two slots of loads in flight at a time
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int t = cb * 32 + j;
-              float sum = 0.f;
-              if (t < o.T)
-                for (int sl = 0; sl < nslots; ++sl) sum += __ldcg(src + ((size_t)sl * o.T + t) * kTileM);
-              v[j] = sum;
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+            for (int sl = 0; sl < nslots; sl += 2) {
+              const float4* a0 = reinterpret_cast<const float4*>(tile_part + (size_t)sl * kTileM * TP) + cb * 8;
+              const float4* a1 = reinterpret_cast<const float4*>(tile_part + (size_t)(sl + 1) * kTileM * TP) + cb * 8;
+              const bool two = sl + 1 < nslots;
+              float4 x0[8], x1[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q) x0[q] = __ldcg(a0 + q);
+              if (two) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) x1[q] = __ldcg(a1 + q);
+              }
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                v[4 * q] += x0[q].x;
+                v[4 * q + 1] += x0[q].y;
+                v[4 * q + 2] += x0[q].z;
+                v[4 * q + 3] += x0[q].w;
+              }
+              if (two) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                  v[4 * q] += x1[q].x;
+                  v[4 * q + 1] += x1[q].y;
+                  v[4 * q + 2] += x1[q].z;
+                  v[4 * q + 3] += x1[q].w;
+                }
+              }
             }
           }
           finish_block(args, tile, row, cb * 32, v, xch, L);
@@ -430,7 +466,7 @@ static void partition(int T, int N, int K, int a_mode, GemmOut* o) {
 size_t gemm_partial_bytes(int T, int N, int K, int a_mode) {
   GemmOut o;
   partition(T, N, K, a_mode, &o);
-  return (size_t)o.n_tiles * o.max_slots * T * kTileM * sizeof(float);
+  return (size_t)o.n_tiles * o.max_slots * ((T + 31) / 32 * 32) * kTileM * sizeof(float);
 }
 
 int split_pad(int T) { return T <= 32 ? 32 : (T <= 64 ? 64 : 128); }
@@ -453,7 +489,7 @@ bool gemm_plan(GemmPlan* p, int a_mode, const void* a0, const void* a1, const vo
   p->lo_col = split ? split_pad(T) : 0;
   partition(T, N, K, a_mode, &p->out);
   p->out.partial = partial;
-  p->partial_bytes = (size_t)p->out.n_tiles * p->out.max_slots * T * kTileM * sizeof(float);
+  p->partial_bytes = gemm_partial_bytes(T, N, K, a_mode);
   bool ok = true;
   if (a_mode == A_KMAJOR) {
     ok = encode_tmap_2d(&p->ta0, a0, K, N, (uint64_t)K * 2, kTileK, kTileM, err, errlen);

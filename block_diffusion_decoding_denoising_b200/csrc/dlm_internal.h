@@ -78,7 +78,7 @@ struct EpiArgs {
   int Hq, Hkv, hd, max_ctx;
   int pos0;
   const int* pos0_dev;
-  float rope_theta;
+  const float2* rope_tab;       // (cos, sin) of position p, pair j at [p][j], j < hd/2
   float* h;                     // EPI_RESID / EPI_EMBED: [T][d]
   float* ss;                    // [n_tiles][T]
   const __nv_bfloat16* embed;   // EPI_EMBED

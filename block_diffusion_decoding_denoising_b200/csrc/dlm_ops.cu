@@ -288,6 +288,19 @@ __global__ void k_set_int(int* p, int v) {
   *p = v;
 }
 
+// RoPE table: tab[p][j] = (cos, sin) of p * theta_j, theta_j = base^(-2j/hd), computed in
+// double precision once per context (NeoX rotate-half pairing (j, j + hd/2)).
+__global__ void k_rope_table(float2* tab, int max_ctx, int hd, double base) {
+  const int half = hd / 2;
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long)max_ctx * half) return;
+  const int p = (int)(i / half), j = (int)(i % half);
+  const double theta = pow(base, -2.0 * (double)j / (double)hd);
+  double s, c;
+  sincos((double)p * theta, &s, &c);
+  tab[i] = make_float2((float)c, (float)s);
+}
+
 // amax bits -> tensor scale amax / (6 * 448), in place.
 __global__ void k_amax_to_scale(float* p) {
   pdl_trigger();

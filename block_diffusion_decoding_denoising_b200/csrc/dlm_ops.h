@@ -81,6 +81,7 @@ __global__ void k_commit(CommitArgs a);
 __global__ void k_block_init(BlockInitArgs a);
 __global__ void k_block_finish(BlockFinishArgs a);
 __global__ void k_set_int(int* p, int v);
+__global__ void k_rope_table(float2* tab, int max_ctx, int hd, double base);
 __global__ void k_amax_to_scale(float* p);
 __global__ void k_amax_bf16(const __nv_bfloat16* w, long n, unsigned* amax_bits);
 __global__ void k_nvfp4_quantize(const __nv_bfloat16* w, int rows, int cols, uint8_t* codes,
