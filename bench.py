@@ -210,14 +210,23 @@ def gemm_case(args):
     shapes.append((w["embed"], cfg["d"]))
     n = max(L.dlm_gemm_scratch_size(B, t.shape[0], K) for t, K in shapes)
     sc = torch.empty(n, dtype=torch.uint8, device="cuda")
+    y = torch.empty((B, max(t.shape[0] for t, K in shapes)), dtype=torch.float32, device="cuda")
     s = C.c_void_p(torch.cuda.current_stream().cuda_stream)
-    for _ in range(args.steps):
+    times = {}
+    for mode in ("partial", "store"):
+        yp = C.c_void_p(y.data_ptr()) if mode == "store" else None
         for t, K in shapes:
-            st = L.dlm_gemm_bf16x2(C.c_void_p(x2.data_ptr()), C.c_void_p(t.data_ptr()), None, B, t.shape[0], K,
-                                   C.c_void_p(sc.data_ptr()), n, s)
-            assert st == 0, st
-    torch.cuda.synchronize()
-    print("gemm case done: %d launches" % (args.steps * len(shapes)))
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ev[0].record()
+            for _ in range(args.steps):
+                st = L.dlm_gemm_bf16x2(C.c_void_p(x2.data_ptr()), C.c_void_p(t.data_ptr()), yp, B, t.shape[0], K,
+                                       C.c_void_p(sc.data_ptr()), n, s)
+                assert st == 0, st
+            ev[1].record()
+            torch.cuda.synchronize()
+            key = "%s %dx%d" % (mode, t.shape[0], K)
+            times[key] = round(ev[0].elapsed_time(ev[1]) * 1e3 / args.steps, 2)
+    print(json.dumps({"case": "gemm", "us_per_launch": times}))
 
 
 def main():

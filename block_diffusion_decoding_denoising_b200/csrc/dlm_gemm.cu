@@ -65,20 +65,27 @@ __device__ __forceinline__ void finish_block(const GemmKArgs& a, int tile, int r
   } else if (e.op == EPI_RESID || e.op == EPI_EMBED) {
     const int n = tile * kTileM + row;
     const bool ok = n < a.N;
-    const __nv_bfloat16* erow = nullptr;
+    // all loads first (independent, in flight together), then the stores
+    float base[32];
+    if (e.op == EPI_RESID) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) base[j] = (ok && j < nt) ? e.h[(size_t)(t0 + j) * a.N + n] : 0.f;
+    } else {
+      int tok[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) tok[j] = (j < nt) ? e.tokens[t0 + j] : 0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) base[j] = (ok && j < nt) ? bf2f(e.embed[(size_t)tok[j] * a.N + n]) : 0.f;
+    }
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       float hn = 0.f;
       if (ok && j < nt) {
-        const int t = t0 + j;
-        const float base = (e.op == EPI_RESID) ? e.h[(size_t)t * a.N + n]
-                                               : bf2f(e.embed[(size_t)e.tokens[t] * a.N + n]);
-        hn = base + v[j];
-        e.h[(size_t)t * a.N + n] = hn;
+        hn = base[j] + v[j];
+        e.h[(size_t)(t0 + j) * a.N + n] = hn;
       }
       xch[row][j] = hn * hn;
     }
-    (void)erow;
     epi_sync();
     if (row < nt) {
       float ss = 0.f;
@@ -125,17 +132,18 @@ __device__ __forceinline__ void finish_block(const GemmKArgs& a, int tile, int r
         dst = e.vc + ((size_t)(hh - e.Hq - e.Hkv) * e.max_ctx + L) * hd + jj;
         stride_t = hd;
       }
-#pragma unroll 4
+      float2 cs[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) cs[j] = (rope && j < nt) ? tab[(size_t)(L + t0 + j) * half] : make_float2(1.f, 0.f);
+#pragma unroll
       for (int j = 0; j < 32; ++j) {
         if (j < nt) {
-          const int t = t0 + j;
           float out = xch[row][j];
           if (rope) {
-            const float2 cs = tab[(size_t)(L + t) * half];
             const float pv = xch[partner][j];
-            out = (jj < half) ? out * cs.x - pv * cs.y : pv * cs.y + out * cs.x;
+            out = (jj < half) ? out * cs[j].x - pv * cs[j].y : pv * cs[j].y + out * cs[j].x;
           }
-          dst[(size_t)t * stride_t] = f2bf(out);
+          dst[(size_t)(t0 + j) * stride_t] = f2bf(out);
         }
       }
     }
@@ -356,10 +364,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
               float4 x0[8], x1[8];
 #pragma unroll
               for (int q = 0; q < 8; ++q) x0[q] = __ldcg(a0 + q);
-              if (two) {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) x1[q] = __ldcg(a1 + q);
-              }
+              for (int q = 0; q < 8; ++q) x1[q] = two ? __ldcg(a1 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+              // slot order: all of slot sl, then all of slot sl + 1
 #pragma unroll
               for (int q = 0; q < 8; ++q) {
                 v[4 * q] += x0[q].x;
@@ -367,14 +374,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
                 v[4 * q + 2] += x0[q].z;
                 v[4 * q + 3] += x0[q].w;
               }
-              if (two) {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  v[4 * q] += x1[q].x;
-                  v[4 * q + 1] += x1[q].y;
-                  v[4 * q + 2] += x1[q].z;
-                  v[4 * q + 3] += x1[q].w;
-                }
+              for (int q = 0; q < 8; ++q) {
+                v[4 * q] += x1[q].x;
+                v[4 * q + 1] += x1[q].y;
+                v[4 * q + 2] += x1[q].z;
+                v[4 * q + 3] += x1[q].w;
               }
             }
           }
