@@ -216,7 +216,7 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
 
 bool valid_cfg(const dlm_config* c, char* msg, size_t n) {
   if (!c) { snprintf(msg, n, "null config"); return false; }
-  if (c->n_layers < 0 || c->d < 64 || c->d % 64 || c->n_q_heads < 1 || c->n_kv_heads < 1 ||
+  if (c->n_layers < 0 || c->d < 64 || c->d % 64 || c->d > 8192 || c->n_q_heads < 1 || c->n_kv_heads < 1 ||
       c->n_q_heads % c->n_kv_heads || !(c->head_dim == 32 || c->head_dim == 64 || c->head_dim == 128) ||
       c->ffn < 64 || c->ffn % 64 || c->vocab < 2 || c->vocab % 8 || c->mask_id < 0 ||
       c->mask_id >= c->vocab || c->block_size < 1 || c->block_size > 64 ||
@@ -240,7 +240,7 @@ struct Runner {
 
   // One projection with split activations and the fused epilogue `epi`.
   dlm_status gemm(int a_mode, const void* a0, const void* a1, const void* x, int T, int N, int K,
-                  EpiArgs epi) {
+                  EpiArgs epi, GemmOut* out = nullptr) {
     GemmPlan p;
     if (!gemm_plan(&p, a_mode, a0, a1, x, T, N, K, ctx->partial, msg, sizeof(msg), true))
       return fail(ctx, DLM_EUNSUPPORTED, "%s", msg);
@@ -250,7 +250,15 @@ struct Runner {
     p.epi = epi;
     cudaError_t e = gemm_launch(p, ctx->d_err, s);
     if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "gemm launch: %s", cudaGetErrorString(e));
+    if (out) *out = p.out;
     return DLM_OK;
+  }
+  // A projection that leaves per-slot partial sums (finished by the next kernel).
+  dlm_status gemm_partial(int a_mode, const void* a0, const void* a1, const void* x, int T, int N, int K,
+                          GemmOut* out) {
+    EpiArgs e{};
+    e.op = EPI_PARTIAL;
+    return gemm(a_mode, a0, a1, x, T, N, K, e, out);
   }
   dlm_status check() {
     cudaError_t e = cudaGetLastError();
@@ -277,21 +285,40 @@ struct FwdSpec {
   float* s_out;
 };
 
-// RMSNorm of h into the split GEMM input buffer xn, from the per-tile sums of squares.
-dlm_status norm_apply(Runner& r, int T, const void* gain) {
+// h update + RMSNorm into the split GEMM input xn, one CTA per token (see k_resid_norm).
+dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_tokens, const void* gain) {
   dlm_ctx* ctx = r.ctx;
   const dlm_config& c = ctx->cfg;
-  NormArgs na{ctx->h, ctx->ss, (const __nv_bfloat16*)gain, ctx->xn, (long)split_pad(T) * c.d,
-              c.d, T, (c.d + 127) / 128, c.rms_eps};
-  CU_LAUNCH(launch_k(k_norm_apply, dim3((c.d + 255) / 256, T), dim3(256), 0, r.s, na));
+  ResNormArgs a{};
+  if (y) a.out = *y;
+  a.out.T = T;
+  a.h = ctx->h;
+  a.embed = embed_tokens ? (const __nv_bfloat16*)ctx->w.embed : nullptr;
+  a.tokens = embed_tokens;
+  a.gain = (const __nv_bfloat16*)gain;
+  a.xn = ctx->xn;
+  a.xn_lo = (long)split_pad(T) * c.d;
+  a.d = c.d;
+  a.eps = c.rms_eps;
+  const int threads = c.d >= 4096 ? 1024 : (c.d >= 1024 ? 512 : 128);
+  CU_LAUNCH(launch_k(k_resid_norm, dim3(T), dim3(threads), 0, r.s, a));
+  return DLM_OK;
+}
+
+// Finishes the tiles of a partial-sums GEMM with `epi` (one CTA per tile and 32 tokens).
+dlm_status finish_tiles(Runner& r, const GemmOut& y, int N, const EpiArgs& epi) {
+  dlm_ctx* ctx = r.ctx;
+  FinishArgs a{y, epi, N};
+  CU_LAUNCH(launch_k(k_finish_tiles, dim3(y.n_tiles, (y.T + 31) / 32), dim3(128), 0, r.s, a));
   return DLM_OK;
 }
 
 // One forward pass of T tokens (round, KV-fill or prefill chunk), all on stream r.s:
-//   [s -> split bf16 -> W_a GEMM (+E[x])] or E[x]; RMSNorm
-//   per layer: QKV GEMM (+RoPE, K/V cache) ; attention ; O GEMM (+residual) ; RMSNorm ;
-//              gate/up GEMM (+SiLU gate) ; down GEMM (+residual) ; RMSNorm (next gain)
+//   [s -> split bf16 -> W_a GEMM] ; h = E[x] (+ W_a s) ; RMSNorm
+//   per layer: QKV GEMM ; RoPE + K/V cache ; attention ; O GEMM ; residual + RMSNorm ;
+//              gate/up GEMM ; SiLU gate ; down GEMM ; residual + RMSNorm (next gain)
 //   round only: LM head GEMM -> logits ; row statistics + P ; P E GEMM -> s_out
+// The projections leave per-slot partial sums; the kernel after each one finishes them.
 dlm_status forward(Runner& r, const FwdSpec& f) {
   dlm_ctx* ctx = r.ctx;
   const dlm_config& c = ctx->cfg;
@@ -299,29 +326,24 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   const int ho = Hq * hd, nqkv = (Hq + 2 * Hkv) * hd;
   const long pad = split_pad(T);  // low halves of split activations start `pad` rows down
   const void* first_gain = c.n_layers > 0 ? ctx->layers[0].attn_norm : ctx->w.final_norm;
+  GemmOut y;
 
   // embedding + residual adapter
   if (f.s) {
     long n = (long)T * d;
     CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, r.s, f.s, ctx->sbf, n, pad * d));
-    EpiArgs e{};
-    e.op = EPI_EMBED;
-    e.h = ctx->h;
-    e.ss = ctx->ss;
-    e.embed = (const __nv_bfloat16*)ctx->w.embed;
-    e.tokens = f.tokens;
-    TRY(r.gemm(A_KMAJOR, ctx->w.w_adapter, nullptr, ctx->sbf, T, d, d, e));
+    TRY(r.gemm_partial(A_KMAJOR, ctx->w.w_adapter, nullptr, ctx->sbf, T, d, d, &y));
+    TRY(resid_norm(r, T, &y, f.tokens, first_gain));
   } else {
-    EmbedRowsArgs ea{(const __nv_bfloat16*)ctx->w.embed, f.tokens, ctx->h, ctx->ss, d, T};
-    CU_LAUNCH(launch_k(k_embed_rows, dim3((d + 127) / 128, T), dim3(128), 0, r.s, ea));
+    TRY(resid_norm(r, T, nullptr, f.tokens, first_gain));
   }
-  TRY(norm_apply(r, T, first_gain));
 
   const size_t layer_kv = (size_t)Hkv * c.max_ctx * hd;
   for (int l = 0; l < c.n_layers; ++l) {
     const dlm_layer_weights& W = ctx->layers[l];
     __nv_bfloat16* kc = ctx->kv + (size_t)(2 * l) * layer_kv;
     __nv_bfloat16* vc = ctx->kv + (size_t)(2 * l + 1) * layer_kv;
+    TRY(r.gemm_partial(A_KMAJOR, W.w_qkv, nullptr, ctx->xn, T, nqkv, d, &y));
     EpiArgs eq{};
     eq.op = EPI_QKV;
     eq.q = ctx->q;
@@ -334,7 +356,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     eq.pos0 = f.pos0;
     eq.pos0_dev = f.dev_L ? ctx->d_L : nullptr;
     eq.rope_tab = ctx->rope_tab;
-    TRY(r.gemm(A_KMAJOR, W.w_qkv, nullptr, ctx->xn, T, nqkv, d, eq));
+    TRY(finish_tiles(r, y, nqkv, eq));
     // the last layer's K/V do not depend on anything after its QKV projection
     if (!f.lm_head && l == c.n_layers - 1) break;
 
@@ -359,25 +381,23 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     cudaError_t e = attention_launch(aa, r.s);
     if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "attention: %s", cudaGetErrorString(e));
 
-    EpiArgs er{};
-    er.op = EPI_RESID;
-    er.h = ctx->h;
-    er.ss = ctx->ss;
-    TRY(r.gemm(A_KMAJOR, W.w_o, nullptr, ctx->o, T, d, ho, er));
-    TRY(norm_apply(r, T, W.mlp_norm));
+    TRY(r.gemm_partial(A_KMAJOR, W.w_o, nullptr, ctx->o, T, d, ho, &y));
+    TRY(resid_norm(r, T, &y, nullptr, W.mlp_norm));
 
+    TRY(r.gemm_partial(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, &y));
     EpiArgs es{};
     es.op = EPI_SILU;
     es.act = ctx->act;
     es.act_lo = pad * F;
-    TRY(r.gemm(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, es));
+    TRY(finish_tiles(r, y, F, es));
 
-    TRY(r.gemm(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, er));
-    TRY(norm_apply(r, T, l + 1 < c.n_layers ? ctx->layers[l + 1].attn_norm : ctx->w.final_norm));
+    TRY(r.gemm_partial(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, &y));
+    TRY(resid_norm(r, T, &y, nullptr, l + 1 < c.n_layers ? ctx->layers[l + 1].attn_norm : ctx->w.final_norm));
   }
   if (!f.lm_head) return DLM_OK;
 
-  // LM head: logits, row statistics, P = softmax (split bf16), s = P E
+  // LM head: logits (finished inside the GEMM: its tiles are mostly single-slot), row
+  // statistics, P = softmax (split bf16), s = P E
   EpiArgs el{};
   el.op = EPI_STORE;
   el.out = ctx->logits;
@@ -396,11 +416,12 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   const int nch = (c.vocab + kRowChunk - 1) / kRowChunk;
   CU_LAUNCH(launch_k(k_rowstats_part, dim3(nch, T), dim3(256), 0, r.s, rs));
   CU_LAUNCH(launch_k(k_rowstats_final, dim3(nch, T), dim3(256), 0, r.s, rs));
+  TRY(r.gemm_partial(A_MNMAJOR, ctx->w.embed, nullptr, ctx->P, T, d, c.vocab, &y));
   EpiArgs ep{};
   ep.op = EPI_STORE;
   ep.out = f.s_out;
   ep.ld = d;
-  return r.gemm(A_MNMAJOR, ctx->w.embed, nullptr, ctx->P, T, d, c.vocab, ep);
+  return finish_tiles(r, y, d, ep);
 }
 
 dlm_status launch_commit(Runner& r, const dlm_block_state& st, float tau, int mode, int k,

@@ -195,18 +195,134 @@ __host__ __device__ __forceinline__ int cta_of_unit(long u, long units, int grid
   return c;
 }
 
-// Sum of the partials of output (token t, tile row `row`) of tile `tile`, in slot order.
-__device__ __forceinline__ float gemm_sum(const GemmOut& o, int tile, int row, int t) {
-  const int lo = cta_of_unit((long)tile * o.n_kb, o.units, o.grid);
-  const int hi = cta_of_unit((long)(tile + 1) * o.n_kb - 1, o.units, o.grid);
-  const float* p = o.partial + ((size_t)tile * o.max_slots * o.T + t) * kTileM + row;
-  float acc = 0.f;
-  for (int s = 0; s <= hi - lo; ++s) acc += p[(size_t)s * o.T * kTileM];
-  return acc;
+// Partial sums: [tile][slot][TP][128] fp32 with TP = T rounded up to 32.  sum_slots32 adds
+// the slots of (tile, row) for tokens t0 .. t0+31 in slot order, two slots of 32
+// independent loads in flight at a time (L2 reads: the partials were written by other SMs).
+__device__ __forceinline__ void sum_slots32(const GemmOut& o, int tile, int row, int t0, int TP, int nslots,
+                                            float (&v)[32]) {
+  const float* base = o.partial + (size_t)tile * o.max_slots * kTileM * TP + (size_t)t0 * kTileM + row;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = 0.f;
+  for (int sl = 0; sl < nslots; sl += 2) {
+    const float* a0 = base + (size_t)sl * kTileM * TP;
+    const float* a1 = a0 + (size_t)kTileM * TP;
+    const bool two = sl + 1 < nslots;
+    float x0[32], x1[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x0[j] = (t0 + j < o.T) ? __ldcg(a0 + (size_t)j * kTileM) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x1[j] = (two && t0 + j < o.T) ? __ldcg(a1 + (size_t)j * kTileM) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = (v[j] + x0[j]) + x1[j];
+  }
 }
-// Output feature n of a plain (A_KMAJOR / A_MNMAJOR) GEMM.
-__device__ __forceinline__ float gemm_out(const GemmOut& o, int n, int t) {
-  return gemm_sum(o, n / kTileM, n % kTileM, t);
+
+__device__ __forceinline__ int tile_slots(const GemmOut& o, int tile) {
+  return cta_of_unit((long)(tile + 1) * o.n_kb - 1, o.units, o.grid) - cta_of_unit((long)tile * o.n_kb, o.units, o.grid) + 1;
+}
+
+// Applies the epilogue op to one block of (up to) 32 tokens of a finished tile.  Runs on the
+// 128 threads of which `row` is this thread's tile row and v[j] its value for token t0 + j;
+// `sync` synchronizes those 128 threads.  N = valid output features, T = tokens, L = the
+// position of token 0.
+template <class Sync>
+__device__ __forceinline__ void apply_epi(const EpiArgs& e, int N, int T, int tile, int row, int t0,
+                                          const float (&v)[32], float (*xch)[33], int L, Sync sync) {
+  const int nt = (T - t0) < 32 ? (T - t0) : 32;
+  if (e.op == EPI_STORE) {
+    const int n = tile * kTileM + row;
+    if (n < N) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < nt) e.out[(size_t)(t0 + j) * e.ld + n] = v[j];
+    }
+  } else if (e.op == EPI_RESID || e.op == EPI_EMBED) {
+    const int n = tile * kTileM + row;
+    const bool ok = n < N;
+    // all loads first (independent, in flight together), then the stores
+    float base[32];
+    if (e.op == EPI_RESID) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) base[j] = (ok && j < nt) ? e.h[(size_t)(t0 + j) * N + n] : 0.f;
+    } else {
+      int tok[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) tok[j] = (j < nt) ? e.tokens[t0 + j] : 0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) base[j] = (ok && j < nt) ? bf2f(e.embed[(size_t)tok[j] * N + n]) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float hn = 0.f;
+      if (ok && j < nt) {
+        hn = base[j] + v[j];
+        e.h[(size_t)(t0 + j) * N + n] = hn;
+      }
+      xch[row][j] = hn * hn;
+    }
+    sync();
+    if (row < nt) {
+      float ss = 0.f;
+      for (int r = 0; r < kTileM; ++r) ss += xch[r][row];
+      e.ss[(size_t)tile * T + t0 + row] = ss;
+    }
+    sync();
+  } else if (e.op == EPI_SILU) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) xch[row][j] = v[j];
+    sync();
+    const int f = tile * 64 + row;
+    if (row < 64 && f < N) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j < nt) {
+          const float g = xch[row][j], u = xch[row + 64][j];
+          const float silu = g / (1.0f + expf(-g));
+          store_split(e.act + (size_t)(t0 + j) * N + f, e.act_lo, silu * u);
+        }
+      }
+    }
+    sync();
+  } else if (e.op == EPI_QKV) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) xch[row][j] = v[j];
+    sync();
+    const int n = tile * kTileM + row;
+    const int hd = e.hd, half = hd / 2;
+    const int hh = n / hd, jj = n % hd;
+    if (n < N) {
+      const int partner = (jj < half) ? row + half : row - half;
+      const bool rope = hh < e.Hq + e.Hkv;
+      const float2* tab = e.rope_tab + (jj % half);  // (cos, sin) at [position][jj % half]
+      __nv_bfloat16* dst;
+      size_t stride_t;
+      if (hh < e.Hq) {
+        dst = e.q + (size_t)hh * hd + jj;
+        stride_t = (size_t)e.Hq * hd;
+      } else if (hh < e.Hq + e.Hkv) {
+        dst = e.kc + ((size_t)(hh - e.Hq) * e.max_ctx + L) * hd + jj;
+        stride_t = hd;
+      } else {
+        dst = e.vc + ((size_t)(hh - e.Hq - e.Hkv) * e.max_ctx + L) * hd + jj;
+        stride_t = hd;
+      }
+      float2 cs[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) cs[j] = (rope && j < nt) ? tab[(size_t)(L + t0 + j) * half] : make_float2(1.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j < nt) {
+          float out = xch[row][j];
+          if (rope) {
+            const float pv = xch[partner][j];
+            out = (jj < half) ? out * cs[j].x - pv * cs[j].y : pv * cs[j].y + out * cs[j].x;
+          }
+          dst[(size_t)(t0 + j) * stride_t] = f2bf(out);
+        }
+      }
+    }
+    sync();
+  }
 }
 
 // ---------------------------------------------------------------- warp reductions

@@ -48,108 +48,9 @@ struct GemmKArgs {
 
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-// Applies the epilogue op to one block of (up to) 32 tokens of a finished tile.  Runs on the
-// 128 epilogue threads; `row` is this thread's tile row, v[j] its value for token t0 + j.
-__device__ __forceinline__ void finish_block(const GemmKArgs& a, int tile, int row, int t0, const float (&v)[32],
-                                             float (*xch)[33], int L) {
-  const EpiArgs& e = a.epi;
-  const int T = a.T;
-  const int nt = (T - t0) < 32 ? (T - t0) : 32;
-  if (e.op == EPI_STORE) {
-    const int n = tile * kTileM + row;
-    if (n < a.N) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (j < nt) e.out[(size_t)(t0 + j) * e.ld + n] = v[j];
-    }
-  } else if (e.op == EPI_RESID || e.op == EPI_EMBED) {
-    const int n = tile * kTileM + row;
-    const bool ok = n < a.N;
-    // all loads first (independent, in flight together), then the stores
-    float base[32];
-    if (e.op == EPI_RESID) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) base[j] = (ok && j < nt) ? e.h[(size_t)(t0 + j) * a.N + n] : 0.f;
-    } else {
-      int tok[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) tok[j] = (j < nt) ? e.tokens[t0 + j] : 0;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) base[j] = (ok && j < nt) ? bf2f(e.embed[(size_t)tok[j] * a.N + n]) : 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      float hn = 0.f;
-      if (ok && j < nt) {
-        hn = base[j] + v[j];
-        e.h[(size_t)(t0 + j) * a.N + n] = hn;
-      }
-      xch[row][j] = hn * hn;
-    }
-    epi_sync();
-    if (row < nt) {
-      float ss = 0.f;
-      for (int r = 0; r < kTileM; ++r) ss += xch[r][row];
-      e.ss[(size_t)tile * T + t0 + row] = ss;
-    }
-    epi_sync();
-  } else if (e.op == EPI_SILU) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) xch[row][j] = v[j];
-    epi_sync();
-    const int f = tile * 64 + row;
-    if (row < 64 && f < a.N) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (j < nt) {
-          const float g = xch[row][j], u = xch[row + 64][j];
-          const float silu = g / (1.0f + expf(-g));
-          store_split(e.act + (size_t)(t0 + j) * a.N + f, e.act_lo, silu * u);
-        }
-      }
-    }
-    epi_sync();
-  } else if (e.op == EPI_QKV) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) xch[row][j] = v[j];
-    epi_sync();
-    const int n = tile * kTileM + row;
-    const int hd = e.hd, half = hd / 2;
-    const int hh = n / hd, jj = n % hd;
-    if (n < a.N) {
-      const int partner = (jj < half) ? row + half : row - half;
-      const bool rope = hh < e.Hq + e.Hkv;
-      const float2* tab = e.rope_tab + (jj % half);  // (cos, sin) at [position][jj % half]
-      __nv_bfloat16* dst;
-      size_t stride_t;
-      if (hh < e.Hq) {
-        dst = e.q + (size_t)hh * hd + jj;
-        stride_t = (size_t)e.Hq * hd;
-      } else if (hh < e.Hq + e.Hkv) {
-        dst = e.kc + ((size_t)(hh - e.Hq) * e.max_ctx + L) * hd + jj;
-        stride_t = hd;
-      } else {
-        dst = e.vc + ((size_t)(hh - e.Hq - e.Hkv) * e.max_ctx + L) * hd + jj;
-        stride_t = hd;
-      }
-      float2 cs[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) cs[j] = (rope && j < nt) ? tab[(size_t)(L + t0 + j) * half] : make_float2(1.f, 0.f);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (j < nt) {
-          float out = xch[row][j];
-          if (rope) {
-            const float pv = xch[partner][j];
-            out = (jj < half) ? out * cs[j].x - pv * cs[j].y : pv * cs[j].y + out * cs[j].x;
-          }
-          dst[(size_t)(t0 + j) * stride_t] = f2bf(out);
-        }
-      }
-    }
-    epi_sync();
-  }
-}
+struct EpiSync {
+  __device__ __forceinline__ void operator()() const { epi_sync(); }
+};
 
 // 192 threads: warp 0 = TMA producer (and TMEM allocator), warp 1 = MMA issuer,
 // warps 2..5 = epilogue (TMEM lane quarter = warp % 4).
@@ -323,16 +224,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
       const int hi_c = cta_of_unit((long)(tile + 1) * o.n_kb - 1, o.units, o.grid);
       const int nslots = hi_c - lo_c + 1, slot = c - lo_c;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * NT;
-      // partials: [tile][slot][row][TP] fp32, each thread's tokens contiguous
-      float* const tile_part = o.partial + (size_t)tile * o.max_slots * kTileM * TP + (size_t)row * TP;
+      // partials: [tile][slot][TP][128] fp32 (token-major; a warp's rows are contiguous)
+      float* const tile_part = o.partial + (size_t)tile * o.max_slots * kTileM * TP + row;
       bool finisher = true;
       if (nslots > 1 || e.op == EPI_PARTIAL) {
-        float4* dst = reinterpret_cast<float4*>(tile_part + (size_t)slot * kTileM * TP);
+        float* dst = tile_part + (size_t)slot * kTileM * TP;
 #pragma unroll 1
         for (int cb = 0; cb < ncb; ++cb) {
           load_block(taddr, cb);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) dst[cb * 8 + q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * kTileM] = v[j];
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[acc]);  // the accumulator can take the next tile now
@@ -354,36 +255,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
           if (nslots == 1) {
             load_block(taddr, cb);
           } else {
-            // sum the slots in slot order, two slots of loads in flight at a time
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.f;
-            for (int sl = 0; sl < nslots; sl += 2) {
-              const float4* a0 = reinterpret_cast<const float4*>(tile_part + (size_t)sl * kTileM * TP) + cb * 8;
-              const float4* a1 = reinterpret_cast<const float4*>(tile_part + (size_t)(sl + 1) * kTileM * TP) + cb * 8;
-              const bool two = sl + 1 < nslots;
-              float4 x0[8], x1[8];
-#pragma unroll
-              for (int q = 0; q < 8; ++q) x0[q] = __ldcg(a0 + q);
-#pragma unroll
-              for (int q = 0; q < 8; ++q) x1[q] = two ? __ldcg(a1 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-              // slot order: all of slot sl, then all of slot sl + 1
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                v[4 * q] += x0[q].x;
-                v[4 * q + 1] += x0[q].y;
-                v[4 * q + 2] += x0[q].z;
-                v[4 * q + 3] += x0[q].w;
-              }
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                v[4 * q] += x1[q].x;
-                v[4 * q + 1] += x1[q].y;
-                v[4 * q + 2] += x1[q].z;
-                v[4 * q + 3] += x1[q].w;
-              }
-            }
+            sum_slots32(o, tile, row, cb * 32, TP, nslots, v);
           }
-          finish_block(args, tile, row, cb * 32, v, xch, L);
+          apply_epi(args.epi, args.N, args.T, tile, row, cb * 32, v, xch, L, EpiSync());
         }
         if (nslots == 1) {
           tc_fence_before();

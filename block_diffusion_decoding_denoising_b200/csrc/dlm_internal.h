@@ -36,7 +36,8 @@ constexpr int kTileK = 64;       // reduction elements per k-block (one 128-byte
 constexpr int kMaxTokens = 256;  // tokens per GEMM with plain bf16 activations (tcgen05 N <= 256)
 constexpr int kMaxSplitTokens = 128;  // tokens per GEMM with split (hi + lo) activations
 
-// Partial-sum layout written by the GEMM: [tile][slot][T][128] fp32.  Tile tau covers
+// Partial-sum layout written by the GEMM: [tile][slot][TP][128] fp32, TP = T rounded up to
+// 32 (token-major: the 128 rows of one token are contiguous).  Tile tau covers
 // output features [128 tau, 128 tau + 128) (for the gate/up pair: gate features
 // [64 tau, 64 tau + 64) in rows 0..63 and up features in rows 64..127).  The slots of a
 // tile are the CTAs whose stream-K range intersects it, summed in slot order.

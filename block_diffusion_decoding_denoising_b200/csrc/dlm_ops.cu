@@ -33,51 +33,83 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return r;
 }
 
-// RMSNorm of one row held in `row` (shared, fp32), written as bf16: x * r * g, with
-// r = 1 / sqrt(mean(x^2) + eps).
-__device__ void norm_row_to_bf16(const float* row, int d, const __nv_bfloat16* g, float eps,
-                                 __nv_bfloat16* out, long lo_off, float* red) {
-  float ss = 0.f;
-  for (int n = threadIdx.x; n < d; n += blockDim.x) ss += row[n] * row[n];
-  ss = block_sum(ss, red);
-  const float r = 1.0f / sqrtf(ss / (float)d + eps);
-  for (int n = threadIdx.x; n < d; n += blockDim.x) store_split(out + n, lo_off, row[n] * r * bf2f(g[n]));
-}
+struct SyncAll {
+  __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
 
-// h[t][n] = E[tok_t][n] and ss[tile][t] = sum over the tile's 128 features of h^2 (the
-// same per-tile layout the GEMM's residual epilogue writes).  grid (ceil(d/128), T), 128 thr.
-__global__ void k_embed_rows(EmbedRowsArgs a) {
+// Finishes the tiles of a GEMM that left per-slot partial sums: sums the slots of (tile,
+// 32 tokens) in slot order and applies the op (RoPE + KV cache, SiLU gate, or a store).
+// grid (n_tiles, ceil(T/32)), 128 threads (thread = tile row).
+__global__ void k_finish_tiles(FinishArgs a) {
   pdl_trigger();
   pdl_wait();
-  __shared__ float red[128];
-  const int tile = blockIdx.x, t = blockIdx.y, r = threadIdx.x;
-  const int n = tile * 128 + r;
-  float v = 0.f;
-  if (n < a.d) {
-    v = bf2f(a.embed[(size_t)a.tokens[t] * a.d + n]);
-    a.h[(size_t)t * a.d + n] = v;
-  }
-  red[r] = v * v;
+  __shared__ float xch[128][33];
+  const int tile = blockIdx.x, t0 = blockIdx.y * 32, row = threadIdx.x;
+  const int TP = (a.out.T + 31) / 32 * 32;
+  float v[32];
+  sum_slots32(a.out, tile, row, t0, TP, tile_slots(a.out, tile), v);
+  const int L = (a.epi.op == EPI_QKV) ? (a.epi.pos0_dev ? *a.epi.pos0_dev : a.epi.pos0) : 0;
+  apply_epi(a.epi, a.N, a.out.T, tile, row, t0, v, xch, L, SyncAll());
+}
+
+// Residual update and RMSNorm of one token row (one CTA per token):
+//   h[t] = h[t] + y[t]        (residual of a projection whose partial sums are in `out`)
+//   h[t] = E[tok_t] + y[t]    (embedding, with y = W_a s, or y = 0 when out.partial is null)
+//   xn[t] = h[t] / sqrt(mean(h[t]^2) + eps) * g   as a split bf16 pair.
+// Each thread owns features threadIdx.x + k * blockDim.x, k < kFeat, so all their slot
+// loads are issued together.
+constexpr int kFeat = 8;
+__global__ void __launch_bounds__(1024) k_resid_norm(ResNormArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float red[32];
+  __shared__ int nsl[64];
+  const int t = blockIdx.x;
+  const GemmOut& o = a.out;
+  const bool has_y = o.partial != nullptr;
+  const int TP = (o.T + 31) / 32 * 32;
+  if (has_y)
+    for (int i = threadIdx.x; i < o.n_tiles; i += blockDim.x) nsl[i] = tile_slots(o, i);
   __syncthreads();
-  if (r == 0) {
-    float ss = 0.f;
-    for (int i = 0; i < 128; ++i) ss += red[i];
-    a.ss[(size_t)tile * a.T + t] = ss;
+  const int tok = a.embed ? a.tokens[t] : 0;
+  float hv[kFeat];
+#pragma unroll
+  for (int k = 0; k < kFeat; ++k) {
+    const int n = threadIdx.x + k * blockDim.x;
+    hv[k] = 0.f;
+    if (n >= a.d) continue;
+    float y = 0.f;
+    if (has_y) {
+      const int tile = n >> 7, row = n & 127, ns = nsl[tile];
+      const float* p = o.partial + ((size_t)tile * o.max_slots * TP + t) * kTileM + row;
+      const size_t st = (size_t)TP * kTileM;
+      for (int sl = 0; sl < ns; sl += 4) {
+        const float x0 = __ldcg(p + sl * st);
+        const float x1 = sl + 1 < ns ? __ldcg(p + (sl + 1) * st) : 0.f;
+        const float x2 = sl + 2 < ns ? __ldcg(p + (sl + 2) * st) : 0.f;
+        const float x3 = sl + 3 < ns ? __ldcg(p + (sl + 3) * st) : 0.f;
+        y = (((y + x0) + x1) + x2) + x3;  // slot order
+      }
+    }
+    const float base = a.embed ? bf2f(a.embed[(size_t)tok * a.d + n]) : a.h[(size_t)t * a.d + n];
+    hv[k] = base + y;
   }
-}
-
-// xn[t][n] = split bf16 of h[t][n] * r_t * g[n], r_t = 1 / sqrt(sum_tiles ss[tile][t] / d + eps)
-// (RMSNorm; the sums of squares come per 128-feature tile from the producing kernel).
-// grid (ceil(d/256), T), 256 threads.
-__global__ void k_norm_apply(NormArgs a) {
-  pdl_trigger();
-  pdl_wait();
-  const int t = blockIdx.y;
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
   float ss = 0.f;
-  for (int i = 0; i < a.n_tiles; ++i) ss += a.ss[(size_t)i * a.T + t];
+#pragma unroll
+  for (int k = 0; k < kFeat; ++k) {
+    const int n = threadIdx.x + k * blockDim.x;
+    if (n < a.d) {
+      a.h[(size_t)t * a.d + n] = hv[k];
+      ss += hv[k] * hv[k];
+    }
+  }
+  ss = block_sum(ss, red);
   const float r = 1.0f / sqrtf(ss / (float)a.d + a.eps);
-  if (n < a.d) store_split(a.xn + (size_t)t * a.d + n, a.xn_lo, a.h[(size_t)t * a.d + n] * r * bf2f(a.gain[n]));
+#pragma unroll
+  for (int k = 0; k < kFeat; ++k) {
+    const int n = threadIdx.x + k * blockDim.x;
+    if (n < a.d) store_split(a.xn + (size_t)t * a.d + n, a.xn_lo, hv[k] * r * bf2f(a.gain[n]));
+  }
 }
 
 // Split bf16 copy of s (the W_a GEMM input): high halves at y[i], low halves at y[i + lo].

@@ -7,21 +7,21 @@
 
 namespace dlm {
 
-struct EmbedRowsArgs {
-  const __nv_bfloat16* embed;  // [V][d]
-  const int32_t* tokens;       // [T]
-  float* h;                    // [T][d]
-  float* ss;                   // [ceil(d/128)][T]
-  int d, T;
+struct FinishArgs {
+  GemmOut out;   // partial sums of the GEMM
+  EpiArgs epi;   // op applied to each finished tile
+  int N;         // valid output features
 };
 
-struct NormArgs {
-  const float* h;              // [T][d]
-  const float* ss;             // [n_tiles][T]
+struct ResNormArgs {
+  GemmOut out;                 // partial sums of a GEMM with N = d (partial == nullptr: y = 0)
+  float* h;                    // [T][d] residual stream
+  const __nv_bfloat16* embed;  // non-null: h = E[tokens] + y instead of h += y
+  const int32_t* tokens;
   const __nv_bfloat16* gain;   // [d]
   __nv_bfloat16* xn;           // [T][d] high halves
   long xn_lo;                  // elements to the low halves
-  int d, T, n_tiles;
+  int d;
   float eps;
 };
 
@@ -72,8 +72,8 @@ struct BlockFinishArgs {
   int B;
 };
 
-__global__ void k_embed_rows(EmbedRowsArgs a);
-__global__ void k_norm_apply(NormArgs a);
+__global__ void k_finish_tiles(FinishArgs a);
+__global__ void k_resid_norm(ResNormArgs a);
 __global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo);
 __global__ void k_rowstats_part(RowStatsArgs a);
 __global__ void k_rowstats_final(RowStatsArgs a);
