@@ -216,7 +216,7 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
 
 bool valid_cfg(const dlm_config* c, char* msg, size_t n) {
   if (!c) { snprintf(msg, n, "null config"); return false; }
-  if (c->n_layers < 0 || c->d < 64 || c->d % 64 || c->d > 8192 || c->n_q_heads < 1 || c->n_kv_heads < 1 ||
+  if (c->n_layers < 0 || c->d < 64 || c->d % 64 || c->d > 4096 || c->n_q_heads < 1 || c->n_kv_heads < 1 ||
       c->n_q_heads % c->n_kv_heads || !(c->head_dim == 32 || c->head_dim == 64 || c->head_dim == 128) ||
       c->ffn < 64 || c->ffn % 64 || c->vocab < 2 || c->vocab % 8 || c->mask_id < 0 ||
       c->mask_id >= c->vocab || c->block_size < 1 || c->block_size > 64 ||
@@ -300,7 +300,7 @@ dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_t
   a.xn_lo = (long)split_pad(T) * c.d;
   a.d = c.d;
   a.eps = c.rms_eps;
-  const int threads = c.d >= 4096 ? 1024 : (c.d >= 1024 ? 512 : 128);
+  const int threads = c.d > 1024 ? 1024 : (c.d > 256 ? 256 : 64);  // d <= 4 * threads
   CU_LAUNCH(launch_k(k_resid_norm, dim3(T), dim3(threads), 0, r.s, a));
   return DLM_OK;
 }

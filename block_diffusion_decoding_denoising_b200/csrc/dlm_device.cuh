@@ -196,24 +196,28 @@ __host__ __device__ __forceinline__ int cta_of_unit(long u, long units, int grid
 }
 
 // Partial sums: [tile][slot][TP][128] fp32 with TP = T rounded up to 32.  sum_slots32 adds
-// the slots of (tile, row) for tokens t0 .. t0+31 in slot order, two slots of 32
-// independent loads in flight at a time (L2 reads: the partials were written by other SMs).
+// the slots of (tile, row) for tokens t0 .. t0+31 in slot order, NB slots of 32 independent
+// loads in flight at a time (L2 reads: the partials were written by other SMs).
+template <int NB = 2>
 __device__ __forceinline__ void sum_slots32(const GemmOut& o, int tile, int row, int t0, int TP, int nslots,
                                             float (&v)[32]) {
   const float* base = o.partial + (size_t)tile * o.max_slots * kTileM * TP + (size_t)t0 * kTileM + row;
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = 0.f;
-  for (int sl = 0; sl < nslots; sl += 2) {
-    const float* a0 = base + (size_t)sl * kTileM * TP;
-    const float* a1 = a0 + (size_t)kTileM * TP;
-    const bool two = sl + 1 < nslots;
-    float x0[32], x1[32];
+  for (int sl = 0; sl < nslots; sl += NB) {
+    float x[NB][32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) x0[j] = (t0 + j < o.T) ? __ldcg(a0 + (size_t)j * kTileM) : 0.f;
+    for (int b = 0; b < NB; ++b) {
+      const float* a = base + (size_t)(sl + b) * kTileM * TP;
+      const bool ok = sl + b < nslots;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) x1[j] = (two && t0 + j < o.T) ? __ldcg(a1 + (size_t)j * kTileM) : 0.f;
+      for (int j = 0; j < 32; ++j) x[b][j] = (ok && t0 + j < o.T) ? __ldcg(a + (size_t)j * kTileM) : 0.f;
+    }
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = (v[j] + x0[j]) + x1[j];
+    for (int b = 0; b < NB; ++b) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += x[b][j];  // slot order
+    }
   }
 }
 

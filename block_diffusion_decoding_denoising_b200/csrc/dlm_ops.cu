@@ -47,7 +47,7 @@ __global__ void k_finish_tiles(FinishArgs a) {
   const int tile = blockIdx.x, t0 = blockIdx.y * 32, row = threadIdx.x;
   const int TP = (a.out.T + 31) / 32 * 32;
   float v[32];
-  sum_slots32(a.out, tile, row, t0, TP, tile_slots(a.out, tile), v);
+  sum_slots32<4>(a.out, tile, row, t0, TP, tile_slots(a.out, tile), v);
   const int L = (a.epi.op == EPI_QKV) ? (a.epi.pos0_dev ? *a.epi.pos0_dev : a.epi.pos0) : 0;
   apply_epi(a.epi, a.N, a.out.T, tile, row, t0, v, xch, L, SyncAll());
 }
@@ -56,9 +56,10 @@ __global__ void k_finish_tiles(FinishArgs a) {
 //   h[t] = h[t] + y[t]        (residual of a projection whose partial sums are in `out`)
 //   h[t] = E[tok_t] + y[t]    (embedding, with y = W_a s, or y = 0 when out.partial is null)
 //   xn[t] = h[t] / sqrt(mean(h[t]^2) + eps) * g   as a split bf16 pair.
-// Each thread owns features threadIdx.x + k * blockDim.x, k < kFeat, so all their slot
-// loads are issued together.
-constexpr int kFeat = 8;
+// Each thread owns features threadIdx.x + k * blockDim.x, k < kFeat, and issues the loads
+// of all their slots (up to kSlotsReg each) before summing them in slot order.
+constexpr int kFeat = 4;
+constexpr int kSlotsReg = 12;
 __global__ void __launch_bounds__(1024) k_resid_norm(ResNormArgs a) {
   pdl_trigger();
   pdl_wait();
@@ -68,35 +69,33 @@ __global__ void __launch_bounds__(1024) k_resid_norm(ResNormArgs a) {
   const GemmOut& o = a.out;
   const bool has_y = o.partial != nullptr;
   const int TP = (o.T + 31) / 32 * 32;
+  const size_t st = (size_t)TP * kTileM;
   if (has_y)
     for (int i = threadIdx.x; i < o.n_tiles; i += blockDim.x) nsl[i] = tile_slots(o, i);
   __syncthreads();
   const int tok = a.embed ? a.tokens[t] : 0;
-  float hv[kFeat];
+  float base[kFeat], x[kFeat][kSlotsReg];
+  int ns[kFeat];
+  const float* pp[kFeat];
 #pragma unroll
   for (int k = 0; k < kFeat; ++k) {
     const int n = threadIdx.x + k * blockDim.x;
-    hv[k] = 0.f;
-    if (n >= a.d) continue;
-    float y = 0.f;
-    if (has_y) {
-      const int tile = n >> 7, row = n & 127, ns = nsl[tile];
-      const float* p = o.partial + ((size_t)tile * o.max_slots * TP + t) * kTileM + row;
-      const size_t st = (size_t)TP * kTileM;
-      for (int sl = 0; sl < ns; sl += 4) {
-        const float x0 = __ldcg(p + sl * st);
-        const float x1 = sl + 1 < ns ? __ldcg(p + (sl + 1) * st) : 0.f;
-        const float x2 = sl + 2 < ns ? __ldcg(p + (sl + 2) * st) : 0.f;
-        const float x3 = sl + 3 < ns ? __ldcg(p + (sl + 3) * st) : 0.f;
-        y = (((y + x0) + x1) + x2) + x3;  // slot order
-      }
-    }
-    const float base = a.embed ? bf2f(a.embed[(size_t)tok * a.d + n]) : a.h[(size_t)t * a.d + n];
-    hv[k] = base + y;
+    const bool ok = n < a.d;
+    ns[k] = (ok && has_y) ? nsl[n >> 7] : 0;
+    pp[k] = has_y ? o.partial + ((size_t)(n >> 7) * o.max_slots * TP + t) * kTileM + (n & 127) : nullptr;
+    base[k] = !ok ? 0.f : (a.embed ? bf2f(a.embed[(size_t)tok * a.d + n]) : a.h[(size_t)t * a.d + n]);
+#pragma unroll
+    for (int sl = 0; sl < kSlotsReg; ++sl) x[k][sl] = sl < ns[k] ? __ldcg(pp[k] + sl * st) : 0.f;
   }
+  float hv[kFeat];
   float ss = 0.f;
 #pragma unroll
   for (int k = 0; k < kFeat; ++k) {
+    float y = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < kSlotsReg; ++sl) y += x[k][sl];  // slot order
+    for (int sl = kSlotsReg; sl < ns[k]; ++sl) y += __ldcg(pp[k] + sl * st);
+    hv[k] = base[k] + y;
     const int n = threadIdx.x + k * blockDim.x;
     if (n < a.d) {
       a.h[(size_t)t * a.d + n] = hv[k];
