@@ -60,7 +60,7 @@ class KV(C.Structure):
 
 class Stats(C.Structure):
     _fields_ = [("m", C.c_double), ("lse", C.c_double), ("maxprob", C.c_double),
-                ("entropy", C.c_double), ("argmax", C.c_int), ("gap2", C.c_double)]
+                ("entropy", C.c_double), ("argmax", C.c_int), ("gap2", C.c_double), ("qmargin", C.c_double)]
 
 
 class Block(C.Structure):
@@ -244,7 +244,8 @@ def attention(q, kc, vc, pos0, causal=False):
 
 
 def _stats_to_dict(st):
-    return {k: np.array([getattr(s, k) for s in st]) for k in ("m", "lse", "maxprob", "entropy", "argmax", "gap2")}
+    return {k: np.array([getattr(s, k) for s in st])
+            for k in ("m", "lse", "maxprob", "entropy", "argmax", "gap2", "qmargin")}
 
 
 def rowstats(logits, mask_id=-1):

@@ -137,6 +137,40 @@ uint8_t e2m1_encode(float rf) {
   return uint8_t(sign | best);
 }
 
+// Margin of a rounding decision: the distance of the rounded quantity from its nearest
+// decision boundary, relative to the boundary.  Quantization codes are integer decisions
+// taken from floats; two computations whose inputs differ by a relative epsilon can round
+// differently only where this margin is below about epsilon (like a top-2 logit gap for
+// an argmax).
+double e2m1_margin(float rf) {
+  const double a = std::fabs(double(rf));
+  const double bounds[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};  // midpoints of kE2M1
+  double m = std::numeric_limits<double>::infinity();
+  for (double b : bounds) m = std::min(m, std::fabs(a - b) / b);
+  return m;
+}
+
+// Margin of round_e4m3_nonneg(x): the midpoints between neighbouring e4m3 values inside
+// x's binade are (k + 1/2) q (q = the binade's spacing), and the one just below the binade
+// lies a quarter spacing under its lower edge; values from 448 up saturate to 448.
+double e4m3_margin(float xf) {
+  const double x = double(xf);
+  if (!(x > 0.0)) return std::numeric_limits<double>::infinity();
+  if (x >= 448.0) return (x - 432.0) / 432.0;  // saturated: 432 is the midpoint below 448
+  int e;
+  std::frexp(x, &e);
+  int qexp = e - 4;
+  if (qexp < -9) qexp = -9;
+  const double q = std::ldexp(1.0, qexp);
+  const double mid = (std::floor(x / q) + 0.5) * q;
+  double m = std::fabs(x - mid) / mid;
+  if (e - 4 >= -9) {
+    const double below = std::ldexp(1.0, e - 1) - q / 4;
+    m = std::min(m, std::fabs(x - below) / below);
+  }
+  return m;
+}
+
 double e2m1_value(uint8_t c) {
   double v = kE2M1[c & 7];
   return (c & 8) ? -v : v;
@@ -162,6 +196,32 @@ void parallel_for(long n, F f) {
     th.emplace_back([=, &f] { for (long i = a; i < b; ++i) f(i); });
   }
   for (auto& x : th) x.join();
+}
+
+// Quantize one row of `cols` values (cols % 16 == 0) with tensor scale S; `margin`
+// (optional) is lowered to the smallest margin of the row's rounding decisions.
+void quantize_row(const float* w, int cols, float S, uint8_t* codes, uint8_t* scales, double* margin) {
+  for (int b = 0; b < cols / 16; ++b) {
+    float amax = 0.0f;
+    for (int j = 0; j < 16; ++j) amax = std::max(amax, std::fabs(w[b * 16 + j]));
+    double sig = 0.0;
+    if (S > 0.0f) {
+      sig = round_e4m3_nonneg(amax / (6.0f * S));
+      if (margin) *margin = std::min(*margin, e4m3_margin(amax / (6.0f * S)));
+    }
+    scales[b] = e4m3_bits(sig);
+    float denom = float(sig) * S;
+    for (int j = 0; j < 16; ++j) {
+      uint8_t c = 0;
+      if (denom > 0.0f) {
+        c = e2m1_encode(w[b * 16 + j] / denom);
+        if (margin) *margin = std::min(*margin, e2m1_margin(w[b * 16 + j] / denom));
+      }
+      int idx = b * 16 + j;
+      if (idx % 2 == 0) codes[idx / 2] = c;
+      else codes[idx / 2] = uint8_t(codes[idx / 2] | (c << 4));
+    }
+  }
 }
 
 }  // namespace
@@ -215,7 +275,9 @@ typedef struct orc_kv {
 typedef struct orc_stats {
   double m, lse, maxprob, entropy;
   int argmax;
-  double gap2;  // largest minus second-largest logit (ambiguity of the argmax)
+  double gap2;     // largest minus second-largest logit (ambiguity of the argmax)
+  double qmargin;  // smallest margin of the row's NVFP4 activation rounding decisions
+                   // (e2m1_margin / e4m3_margin) in the forward pass; +inf without any
 } orc_stats;
 
 void orc_set_threads(int n) { g_threads = n; }
@@ -232,21 +294,7 @@ float orc_nvfp4_tensor_scale(const float* w, long n) {
 
 // Quantize one row of `cols` values (cols % 16 == 0) with tensor scale S.
 void orc_nvfp4_quantize_row(const float* w, int cols, float S, uint8_t* codes, uint8_t* scales) {
-  for (int b = 0; b < cols / 16; ++b) {
-    float amax = 0.0f;
-    for (int j = 0; j < 16; ++j) amax = std::max(amax, std::fabs(w[b * 16 + j]));
-    double sig = 0.0;
-    if (S > 0.0f) sig = round_e4m3_nonneg(amax / (6.0f * S));
-    scales[b] = e4m3_bits(sig);
-    float denom = float(sig) * S;
-    for (int j = 0; j < 16; ++j) {
-      uint8_t c = 0;
-      if (denom > 0.0f) c = e2m1_encode(w[b * 16 + j] / denom);
-      int idx = b * 16 + j;
-      if (idx % 2 == 0) codes[idx / 2] = c;
-      else codes[idx / 2] = uint8_t(codes[idx / 2] | (c << 4));
-    }
-  }
+  quantize_row(w, cols, S, codes, scales, nullptr);
 }
 
 void orc_nvfp4_quantize(const float* w, int rows, int cols, uint8_t* codes, uint8_t* scales,
@@ -293,24 +341,27 @@ void mat_row(const orc_mat& W, long r, double* out) {
   }
 }
 
-// NVFP4 input quantization of one activation row (R8): per-row fp32 scale.
-void quantize_act_row(const double* x, int cols, double* out) {
+// NVFP4 input quantization of one activation row (R8): per-row fp32 scale.  `margin`
+// (optional) is lowered to the smallest margin of the row's rounding decisions.
+void quantize_act_row(const double* x, int cols, double* out, double* margin) {
   std::vector<float> xf(cols);
   for (int i = 0; i < cols; ++i) xf[i] = float(x[i]);
   float S = orc_nvfp4_tensor_scale(xf.data(), cols);
   std::vector<uint8_t> codes(cols / 2), scales(cols / 16);
-  orc_nvfp4_quantize_row(xf.data(), cols, S, codes.data(), scales.data());
+  quantize_row(xf.data(), cols, S, codes.data(), scales.data(), margin);
   for (int c = 0; c < cols; ++c) out[c] = orc_nvfp4_value(codes.data(), scales.data(), S, cols, 0, c);
 }
 
-// y[t][n] = sum_k x[t][k] W[n][k]  (plain triple loop, fp64)
-void linear(const double* x, int T, const orc_mat& W, double* y, bool act_fp4) {
+// y[t][n] = sum_k x[t][k] W[n][k]  (plain triple loop, fp64).  qm[t] (optional) collects
+// the rounding margins of row t's input quantization.
+void linear(const double* x, int T, const orc_mat& W, double* y, bool act_fp4, double* qm = nullptr) {
   const int K = W.cols, N = W.rows;
   std::vector<double> xq;
   const double* xin = x;
   if (act_fp4 && W.fmt == 1) {
     xq.resize(size_t(T) * K);
-    for (int t = 0; t < T; ++t) quantize_act_row(x + size_t(t) * K, K, xq.data() + size_t(t) * K);
+    for (int t = 0; t < T; ++t)
+      quantize_act_row(x + size_t(t) * K, K, xq.data() + size_t(t) * K, qm ? qm + t : nullptr);
     xin = xq.data();
   }
   // x transposed to [K][T] so that the T sums of one weight row advance together; every
@@ -426,6 +477,7 @@ void orc_rowstats(const double* logits, int B, int V, int mask_id, orc_stats* st
     for (int v = 0; v < V; ++v)
       if (v != mask_id && v != am) second = std::max(second, l[v]);
     st[b].gap2 = m - second;
+    st[b].qmargin = std::numeric_limits<double>::infinity();
     st[b].m = m;
     st[b].lse = lse;
     st[b].maxprob = std::exp(m - lse);
@@ -440,9 +492,10 @@ void orc_rowstats(const double* logits, int B, int V, int mask_id, orc_stats* st
 void orc_lmhead(const double* x, int B, const orc_mat* E, int mask_id, int act_fp4,
                 const double* p_given, orc_stats* st, double* s, double* logits_out) {
   const int V = E->rows, d = E->cols;
-  std::vector<double> logits(size_t(B) * V);
-  linear(x, B, *E, logits.data(), act_fp4 != 0);
+  std::vector<double> logits(size_t(B) * V), qm(B, std::numeric_limits<double>::infinity());
+  linear(x, B, *E, logits.data(), act_fp4 != 0, qm.data());
   orc_rowstats(logits.data(), B, V, mask_id, st);
+  for (int b = 0; b < B; ++b) st[b].qmargin = qm[b];
   if (logits_out) std::memcpy(logits_out, logits.data(), logits.size() * sizeof(double));
   std::vector<double> P(size_t(B) * V);
   for (int b = 0; b < B; ++b)
@@ -515,7 +568,7 @@ namespace {
 //  Writes K/V rows [pos0, pos0+n) of every layer.  If xf != nullptr it receives the
 //  final normalised hidden state [n][d] (the LM head input).
 void forward(const orc_model& M, const orc_cfg& C, const int* tokens, const double* s, int n,
-             int pos0, bool causal, orc_kv& kv, double* xf) {
+             int pos0, bool causal, orc_kv& kv, double* xf, double* qm = nullptr) {
   const int d = C.d, Hq = C.n_q_heads, Hkv = C.n_kv_heads, hd = C.head_dim, F = C.ffn;
   const bool rnd = C.act_round != 0, fp4 = C.act_fp4 != 0;
   const int nqkv = (Hq + 2 * Hkv) * hd;
@@ -534,7 +587,7 @@ void forward(const orc_model& M, const orc_cfg& C, const int* tokens, const doub
     double* vl = kv.v + size_t(l) * Hkv * kv.max_ctx * hd;
     // attention sub-block
     for (int i = 0; i < n; ++i) rmsnorm(h.data() + size_t(i) * d, d, L.attn_norm, C.rms_eps, xn.data() + size_t(i) * d);
-    linear(xn.data(), n, L.w_qkv, qkv.data(), fp4);
+    linear(xn.data(), n, L.w_qkv, qkv.data(), fp4, qm);
     for (int i = 0; i < n; ++i) {
       double* row = qkv.data() + size_t(i) * nqkv;
       long pos = pos0 + i;
@@ -548,17 +601,17 @@ void forward(const orc_model& M, const orc_cfg& C, const int* tokens, const doub
       }
     }
     orc_attention(q.data(), n, Hq, Hkv, hd, kl, vl, kv.max_ctx, pos0, causal ? 1 : 0, o.data());
-    linear(o.data(), n, L.w_o, tmp.data(), fp4);
+    linear(o.data(), n, L.w_o, tmp.data(), fp4, qm);
     for (size_t i = 0; i < h.size(); ++i) h[i] += tmp[i];
     // MLP sub-block
     for (int i = 0; i < n; ++i) rmsnorm(h.data() + size_t(i) * d, d, L.mlp_norm, C.rms_eps, xn.data() + size_t(i) * d);
-    linear(xn.data(), n, L.w_gate, g.data(), fp4);
-    linear(xn.data(), n, L.w_up, u.data(), fp4);
+    linear(xn.data(), n, L.w_gate, g.data(), fp4, qm);
+    linear(xn.data(), n, L.w_up, u.data(), fp4, qm);
     for (size_t i = 0; i < a.size(); ++i) {
       double silu = g[i] / (1.0 + std::exp(-g[i]));
       a[i] = silu * u[i];
     }
-    linear(a.data(), n, L.w_down, tmp.data(), fp4);
+    linear(a.data(), n, L.w_down, tmp.data(), fp4, qm);
     for (size_t i = 0; i < h.size(); ++i) h[i] += tmp[i];
   }
   if (xf) {
@@ -590,9 +643,10 @@ void orc_forward(const orc_model* M, const orc_cfg* C, const int* tokens, const 
 int orc_round(const orc_model* M, const orc_cfg* C, orc_block* blk, orc_kv* kv, int L, double tau,
               int mode, int k, orc_stats* st) {
   const int B = C->block_size, d = C->d;
-  std::vector<double> xf(size_t(B) * d), snext(size_t(B) * d);
-  forward(*M, *C, blk->tokens, blk->s, B, L, false, *kv, xf.data());
+  std::vector<double> xf(size_t(B) * d), snext(size_t(B) * d), qm(B, std::numeric_limits<double>::infinity());
+  forward(*M, *C, blk->tokens, blk->s, B, L, false, *kv, xf.data(), qm.data());
   orc_lmhead(xf.data(), B, &M->embed, C->mask_id, C->act_fp4, nullptr, st, snext.data(), nullptr);
+  for (int i = 0; i < B; ++i) st[i].qmargin = std::min(st[i].qmargin, qm[i]);
   std::vector<double> mp(B);
   std::vector<int> am(B);
   for (int i = 0; i < B; ++i) { mp[i] = st[i].maxprob; am[i] = st[i].argmax; }

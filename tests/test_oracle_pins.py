@@ -429,3 +429,36 @@ def test_block_attention_is_bidirectional(tiny):
     x1 = m.forward(t1, None, 16)
     x2 = m.forward(t2, None, 16)
     assert np.abs(x1[0] - x2[0]).max() > 1e-6
+
+
+# ---------------------------------------------------------------- NVFP4 rounding margins
+def _lmhead_qmargin(rows):
+    """qmargin of orc_lmhead's activation quantization for the given x rows (d = 32)."""
+    x = np.array(rows, np.float64)
+    B, d = x.shape
+    E = gen.bf16_bits(gen.normal_np(99, 8 * d, 0.1).reshape(8, d))
+    Ef = (E.astype(np.uint32) << np.uint32(16)).view(np.float32)
+    codes, scales, S = O.nvfp4_quantize(Ef)
+    q = {"codes": codes, "scales": scales, "tscale": S, "rows": 8, "cols": d}
+    return O.lmhead(x, q, act_fp4=True)["qmargin"], O.lmhead(x, q, act_fp4=False)["qmargin"]
+
+
+def test_qmargin_pins():
+    """Rows whose quantization decisions sit at known distances from the rounding boundaries
+    (the e2m1 midpoints 0.25 .. 5 and the e4m3 midpoints (k + 1/2) q):
+      row 0: block 0 on the e2m1 grid with amax/(6S) = 448 (saturated, 16/432 above the
+             midpoint 432), block 1 on the grid with block scale 96 (4 below the midpoint
+             100; e2m1 values sit at least 1/7 from a midpoint) -> 16/432;
+      row 1: block 1 scaled to put amax/(6S) on the e4m3 midpoint 100 -> ~0;
+      row 2: one element exactly on the e2m1 midpoint 2.5 -> ~0."""
+    grid = [6, 4, 3, 2, 1.5, 1, 0.5, 0, -6, -4, -3, -2, -1.5, -1, -0.5, 0]
+    b0 = np.array(grid, np.float64)
+    r0 = np.concatenate([b0, b0 * 96.0 / 448.0])
+    r1 = np.concatenate([b0, b0 * 100.0 / 448.0])
+    b2 = b0.copy()
+    b2[1] = 2.5
+    r2 = np.concatenate([b2, b0 * 96.0 / 448.0])
+    qm, qm_off = _lmhead_qmargin([r0, r1, r2])
+    assert abs(qm[0] - 16.0 / 432.0) < 1e-5, qm
+    assert qm[1] < 1e-5 and qm[2] < 1e-5, qm
+    assert np.all(np.isinf(qm_off))
