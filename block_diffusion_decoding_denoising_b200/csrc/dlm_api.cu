@@ -29,7 +29,7 @@ using namespace dlm;
 
 namespace {
 
-constexpr int kPrefillChunk = kMaxSplitTokens;  // prefill tokens per forward pass
+constexpr int kPrefillChunk = kMaxSplitTokens;  // prefill tokens per forward pass (bf16 weights)
 constexpr int kRowChunk = 4096;                  // vocabulary entries per row-statistics CTA
 
 struct GraphEntry {
@@ -72,6 +72,12 @@ struct dlm_ctx {
   float* logits = nullptr;
   __nv_bfloat16* P = nullptr;
   int32_t* tok_buf = nullptr;
+  // NVFP4 weights: quantized GEMM inputs, their row scales, and E dequantised to bf16
+  // (q sigma, exact; the tensor scale is applied where the rows are used)
+  bool fp4 = false;
+  __half* xq = nullptr;
+  float* sx = nullptr;
+  __nv_bfloat16* e_deq = nullptr;
   // internal block state (graph path)
   int32_t* b_tokens = nullptr;
   uint8_t* b_committed = nullptr;
@@ -128,6 +134,11 @@ int max_tokens(const dlm_config& c) {
   return c.block_size > kPrefillChunk ? c.block_size : kPrefillChunk;
 }
 
+// Tokens per prefill forward: the NVFP4 GEMM takes at most kMaxF4Tokens.
+int prefill_chunk(const dlm_config& c) {
+  return c.weight_fmt == DLM_WEIGHTS_NVFP4 ? kMaxF4Tokens : kPrefillChunk;
+}
+
 size_t max_partial_bytes(const dlm_config& c, int Tmax) {
   const int qkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim, ho = c.n_q_heads * c.head_dim;
   size_t m = 0;
@@ -142,6 +153,13 @@ size_t max_partial_bytes(const dlm_config& c, int Tmax) {
   size_t pe = gemm_partial_bytes(B, c.d, c.vocab, A_MNMAJOR);
   m = lm > m ? lm : m;
   m = pe > m ? pe : m;
+  if (c.weight_fmt == DLM_WEIGHTS_NVFP4 && c.d % 256 == 0 && c.ffn % 256 == 0) {
+    for (int T : {c.block_size, kMaxF4Tokens}) {
+      size_t v[] = {gemm_fp4_partial_bytes(T, c.ffn, c.d, A_PAIR), gemm_fp4_partial_bytes(T, c.d, c.ffn, A_KMAJOR),
+                    gemm_fp4_partial_bytes(T, c.vocab, c.d, A_KMAJOR)};
+      for (size_t x : v) m = x > m ? x : m;
+    }
+  }
   return m;
 }
 
@@ -180,7 +198,15 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   int32_t* sa = cv.take<int32_t>(B);
   int32_t* ot = cv.take<int32_t>(B);
   int32_t* orr = cv.take<int32_t>(4);
+  const bool fp4 = c.weight_fmt == DLM_WEIGHTS_NVFP4;
+  __half* xq = fp4 ? cv.take<__half>((size_t)kMaxF4Tokens * (c.d > c.ffn ? c.d : c.ffn)) : nullptr;
+  float* sx = fp4 ? cv.take<float>(kMaxF4Tokens) : nullptr;
+  __nv_bfloat16* edq = fp4 ? cv.take<__nv_bfloat16>((size_t)c.vocab * c.d) : nullptr;
   if (x && base) {
+    x->fp4 = fp4;
+    x->xq = xq;
+    x->sx = sx;
+    x->e_deq = edq;
     x->d_L = hdr;
     x->d_err = hdr + 1;
     x->h = h;
@@ -260,6 +286,19 @@ struct Runner {
     e.op = EPI_PARTIAL;
     return gemm(a_mode, a0, a1, x, T, N, K, e, out);
   }
+  // NVFP4 projection of the quantized activations in ctx->xq (see act_quant).
+  dlm_status gemm_fp4(int a_mode, const dlm_nvfp4_matrix& w0, const dlm_nvfp4_matrix* w1, int T, int N, int K,
+                      GemmOut* out) {
+    GemmF4Plan p;
+    if (!gemm_fp4_plan(&p, a_mode, w0, w1, ctx->xq, kMaxF4Tokens, ctx->sx, T, N, K, ctx->partial, msg, sizeof(msg)))
+      return fail(ctx, DLM_EUNSUPPORTED, "%s", msg);
+    if (p.partial_bytes > ctx->partial_bytes)
+      return fail(ctx, DLM_ENOMEM_WS, "nvfp4 gemm partials %zu > %zu", p.partial_bytes, ctx->partial_bytes);
+    cudaError_t e = gemm_fp4_launch(p, ctx->d_err, s);
+    if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "nvfp4 gemm launch: %s", cudaGetErrorString(e));
+    *out = p.out;
+    return DLM_OK;
+  }
   dlm_status check() {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "launch: %s", cudaGetErrorString(e));
@@ -293,8 +332,9 @@ dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_t
   if (y) a.out = *y;
   a.out.T = T;
   a.h = ctx->h;
-  a.embed = embed_tokens ? (const __nv_bfloat16*)ctx->w.embed : nullptr;
+  a.embed = embed_tokens ? (ctx->fp4 ? ctx->e_deq : (const __nv_bfloat16*)ctx->w.embed) : nullptr;
   a.tokens = embed_tokens;
+  a.embed_scale = ctx->fp4 ? ctx->w.q_embed.tensor_scale : 1.0f;
   a.gain = (const __nv_bfloat16*)gain;
   a.xn = ctx->xn;
   a.xn_lo = (long)split_pad(T) * c.d;
@@ -302,6 +342,20 @@ dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_t
   a.eps = c.rms_eps;
   const int threads = c.d > 1024 ? 1024 : (c.d > 256 ? 256 : 64);  // d <= 4 * threads
   CU_LAUNCH(launch_k(k_resid_norm, dim3(T), dim3(threads), 0, r.s, a));
+  return DLM_OK;
+}
+
+// Quantizes the T rows of a split bf16 GEMM input (hi at x, lo at x + lo) to NVFP4 in
+// ctx->xq / ctx->sx (see k_act_quant).
+dlm_status act_quant(Runner& r, int T, const __nv_bfloat16* x, long lo, int K) {
+  dlm_ctx* ctx = r.ctx;
+  ActQuantArgs a{};
+  a.xb = x;
+  a.xb_lo = lo;
+  a.K = K;
+  a.xq = ctx->xq;
+  a.sx = ctx->sx;
+  CU_LAUNCH(launch_k(k_act_quant, dim3(T), dim3(256), 0, r.s, a));
   return DLM_OK;
 }
 
@@ -384,14 +438,24 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     TRY(r.gemm_partial(A_KMAJOR, W.w_o, nullptr, ctx->o, T, d, ho, &y));
     TRY(resid_norm(r, T, &y, nullptr, W.mlp_norm));
 
-    TRY(r.gemm_partial(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, &y));
+    if (ctx->fp4) {
+      TRY(act_quant(r, T, ctx->xn, pad * d, d));
+      TRY(r.gemm_fp4(A_PAIR, W.q_gate, &W.q_up, T, F, d, &y));
+    } else {
+      TRY(r.gemm_partial(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, &y));
+    }
     EpiArgs es{};
     es.op = EPI_SILU;
     es.act = ctx->act;
     es.act_lo = pad * F;
     TRY(finish_tiles(r, y, F, es));
 
-    TRY(r.gemm_partial(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, &y));
+    if (ctx->fp4) {
+      TRY(act_quant(r, T, ctx->act, pad * F, F));
+      TRY(r.gemm_fp4(A_KMAJOR, W.q_down, nullptr, T, d, F, &y));
+    } else {
+      TRY(r.gemm_partial(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, &y));
+    }
     TRY(resid_norm(r, T, &y, nullptr, l + 1 < c.n_layers ? ctx->layers[l + 1].attn_norm : ctx->w.final_norm));
   }
   if (!f.lm_head) return DLM_OK;
@@ -402,7 +466,13 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   el.op = EPI_STORE;
   el.out = ctx->logits;
   el.ld = c.vocab;
-  TRY(r.gemm(A_KMAJOR, ctx->w.embed, nullptr, ctx->xn, T, c.vocab, d, el));
+  if (ctx->fp4) {
+    TRY(act_quant(r, T, ctx->xn, pad * d, d));
+    TRY(r.gemm_fp4(A_KMAJOR, ctx->w.q_embed, nullptr, T, c.vocab, d, &y));
+    TRY(finish_tiles(r, y, c.vocab, el));
+  } else {
+    TRY(r.gemm(A_KMAJOR, ctx->w.embed, nullptr, ctx->xn, T, c.vocab, d, el));
+  }
   RowStatsArgs rs{};
   rs.logits = ctx->logits;
   rs.ld = c.vocab;
@@ -416,11 +486,13 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   const int nch = (c.vocab + kRowChunk - 1) / kRowChunk;
   CU_LAUNCH(launch_k(k_rowstats_part, dim3(nch, T), dim3(256), 0, r.s, rs));
   CU_LAUNCH(launch_k(k_rowstats_final, dim3(nch, T), dim3(256), 0, r.s, rs));
-  TRY(r.gemm_partial(A_MNMAJOR, ctx->w.embed, nullptr, ctx->P, T, d, c.vocab, &y));
+  // NVFP4: s = P (q sigma) scaled by the tensor scale of E
+  TRY(r.gemm_partial(A_MNMAJOR, ctx->fp4 ? ctx->e_deq : ctx->w.embed, nullptr, ctx->P, T, d, c.vocab, &y));
   EpiArgs ep{};
   ep.op = EPI_STORE;
   ep.out = f.s_out;
   ep.ld = d;
+  ep.scale = ctx->fp4 ? ctx->w.q_embed.tensor_scale : 0.f;
   return finish_tiles(r, y, d, ep);
 }
 
@@ -569,13 +641,19 @@ dlm_status dlm_ctx_create(const dlm_config* cfg, const dlm_weights* w, void* d_w
   *out = nullptr;
   if (!valid_cfg(cfg, msg, sizeof(msg)) || !w || !d_workspace || (!d_kv_cache && cfg->n_layers > 0))
     return DLM_EINVAL;
-  if (!w->embed || !w->w_adapter || !w->final_norm || (cfg->n_layers > 0 && !w->layers)) return DLM_EINVAL;
+  const bool fp4 = cfg->weight_fmt == DLM_WEIGHTS_NVFP4;
+  auto q_ok = [](const dlm_nvfp4_matrix& m) { return m.codes && m.scales && std::isfinite(m.tensor_scale); };
+  if ((!fp4 && !w->embed) || (fp4 && !q_ok(w->q_embed)) || !w->w_adapter || !w->final_norm ||
+      (cfg->n_layers > 0 && !w->layers))
+    return DLM_EINVAL;
   for (int l = 0; l < cfg->n_layers; ++l) {
     const dlm_layer_weights& L = w->layers[l];
-    if (!L.attn_norm || !L.w_qkv || !L.w_o || !L.mlp_norm || !L.w_gate || !L.w_up || !L.w_down)
-      return DLM_EINVAL;
+    if (!L.attn_norm || !L.w_qkv || !L.w_o || !L.mlp_norm) return DLM_EINVAL;
+    if (!fp4 && (!L.w_gate || !L.w_up || !L.w_down)) return DLM_EINVAL;
+    if (fp4 && (!q_ok(L.q_gate) || !q_ok(L.q_up) || !q_ok(L.q_down))) return DLM_EINVAL;
   }
-  if (cfg->weight_fmt != DLM_WEIGHTS_BF16) return DLM_EUNSUPPORTED;
+  // NVFP4 GEMMs stream 256 reduction elements per stage: d and ffn must be multiples of 256
+  if (fp4 && (cfg->d % 256 || cfg->ffn % 256)) return DLM_EUNSUPPORTED;
   if ((uintptr_t)d_workspace % 256) return DLM_EINVAL;
   if (ws_bytes < dlm_workspace_size(cfg)) return DLM_ENOMEM_WS;
   if (kv_bytes < dlm_kv_cache_size(cfg)) return DLM_ENOMEM_WS;
@@ -598,7 +676,16 @@ dlm_status dlm_ctx_create(const dlm_config* cfg, const dlm_weights* w, void* d_w
                                                                           cfg->head_dim, (double)cfg->rope_theta);
     e = cudaGetLastError();
   }
+  if (e == cudaSuccess && fp4) {
+    // E for the embedding rows and P E: q sigma in bf16 (exact); the tensor scale is applied
+    // where they are used
+    const long nb = (long)cfg->vocab * (cfg->d / 16);
+    k_nvfp4_dequant_bf16<<<(unsigned)((nb + 255) / 256), 256, 0, ctx->cap_stream>>>(
+        (const uint8_t*)w->q_embed.codes, (const uint8_t*)w->q_embed.scales, nb, ctx->e_deq);
+    e = cudaGetLastError();
+  }
   if (e == cudaSuccess) e = (cudaError_t)gemm_init_attributes();
+  if (e == cudaSuccess && fp4) e = (cudaError_t)gemm_fp4_init_attributes();
   if (e == cudaSuccess) e = (cudaError_t)attention_init_attributes();
   if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->cap_stream);
   if (e != cudaSuccess) {
@@ -639,8 +726,9 @@ dlm_status dlm_prefill(dlm_ctx* ctx, const int32_t* d_tokens, int n, void* strea
   if (!d_tokens || n < 0) return fail(ctx, DLM_EINVAL, "prefill args");
   if (ctx->L + n > ctx->cfg.max_ctx) return fail(ctx, DLM_EKVCAP, "prefill: %d + %d > %d", ctx->L, n, ctx->cfg.max_ctx);
   Runner r{ctx, (cudaStream_t)stream, {}};
-  for (int off = 0; off < n; off += kPrefillChunk) {
-    int T = n - off < kPrefillChunk ? n - off : kPrefillChunk;
+  const int chunk = prefill_chunk(ctx->cfg);
+  for (int off = 0; off < n; off += chunk) {
+    int T = n - off < chunk ? n - off : chunk;
     FwdSpec f{};
     f.T = T;
     f.tokens = d_tokens + off;
@@ -1010,6 +1098,47 @@ dlm_status dlm_nvfp4_quantize(const void* d_w, int rows, int cols, void* d_codes
                                                                   (const unsigned*)d_tensor_scale, nullptr));
   CU_LAUNCH(launch_k(k_amax_to_scale, dim3(1), dim3(1), 0, s, d_tensor_scale));
   return cudaGetLastError() == cudaSuccess ? DLM_OK : DLM_ECUDA;
+}
+
+size_t dlm_gemm_nvfp4_scratch_size(int T, int N, int K) {
+  if (T < 1 || T > kMaxF4Tokens || N < 1 || K < 256 || K % 256 || K > 16384) return 0;
+  return op_header() + op_counters(N) + align256(gemm_fp4_partial_bytes(T, N, K, A_KMAJOR)) +
+         align256((size_t)kMaxF4Tokens * K * 2) + align256(kMaxF4Tokens * 4);
+}
+
+dlm_status dlm_gemm_nvfp4(const float* d_x, const dlm_nvfp4_matrix* w, float* d_y, int T, int N, int K,
+                          void* d_scratch, size_t scratch_bytes, void* stream) {
+  dlm_ctx* ctx = nullptr;
+  if (!d_x || !w || !w->codes || !w->scales || !d_scratch || T < 1 || T > kMaxF4Tokens || N < 1 || K < 256 ||
+      K % 256 || K > 16384)
+    return DLM_EINVAL;
+  if (scratch_bytes < dlm_gemm_nvfp4_scratch_size(T, N, K)) return DLM_ENOMEM_WS;
+  CU((cudaError_t)gemm_fp4_init_attributes());
+  cudaStream_t s = (cudaStream_t)stream;
+  OpScratch sc(d_scratch, N, gemm_fp4_partial_bytes(T, N, K, A_KMAJOR));
+  __half* xq = sc.take<__half>((size_t)kMaxF4Tokens * K);
+  float* sx = sc.take<float>(kMaxF4Tokens);
+  CU(cudaMemsetAsync(d_scratch, 0, op_header(), s));
+  ActQuantArgs q{};
+  q.xf = d_x;
+  q.K = K;
+  q.xq = xq;
+  q.sx = sx;
+  CU_LAUNCH(launch_k(k_act_quant, dim3(T), dim3(256), 0, s, q));
+  char msg[256];
+  GemmF4Plan p;
+  if (!gemm_fp4_plan(&p, A_KMAJOR, *w, nullptr, xq, kMaxF4Tokens, sx, T, N, K, sc.partial, msg, sizeof(msg)))
+    return DLM_EUNSUPPORTED;
+  CU(gemm_fp4_launch(p, sc.err, s));
+  if (d_y) {
+    EpiArgs e{};
+    e.op = EPI_STORE;
+    e.out = d_y;
+    e.ld = N;
+    FinishArgs fa{p.out, e, N};
+    CU_LAUNCH(launch_k(k_finish_tiles, dim3(p.out.n_tiles, (T + 31) / 32), dim3(128), 0, s, fa));
+  }
+  return DLM_OK;
 }
 
 }  // extern "C"

@@ -238,7 +238,7 @@ __device__ __forceinline__ void apply_epi(const EpiArgs& e, int N, int T, int ti
     if (n < N) {
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (j < nt) e.out[(size_t)(t0 + j) * e.ld + n] = v[j];
+        if (j < nt) e.out[(size_t)(t0 + j) * e.ld + n] = (e.scale != 0.f) ? v[j] * e.scale : v[j];
     }
   } else if (e.op == EPI_RESID || e.op == EPI_EMBED) {
     const int n = tile * kTileM + row;
@@ -327,6 +327,56 @@ __device__ __forceinline__ void apply_epi(const EpiArgs& e, int N, int T, int ti
     }
     sync();
   }
+}
+
+// ---------------------------------------------------------------- NVFP4 number formats
+// e2m1 code of r (magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6; ties to the even code; sign in bit 3).
+__device__ __forceinline__ uint8_t e2m1_rne(float r) {
+  const float a = fabsf(r);
+  uint8_t c;
+  if (a <= 0.25f) c = 0;
+  else if (a < 0.75f) c = 1;
+  else if (a <= 1.25f) c = 2;
+  else if (a < 1.75f) c = 3;
+  else if (a <= 2.5f) c = 4;
+  else if (a < 3.5f) c = 5;
+  else if (a <= 5.0f) c = 6;
+  else c = 7;
+  return (uint8_t)(c | ((r < 0.f) ? 8 : 0));
+}
+
+// Value of an e2m1 code (bit 3 = sign).
+__device__ __forceinline__ float e2m1_value_dev(uint8_t c) {
+  const int m = c & 7;
+  const float mag = (m < 4) ? 0.5f * m : (m < 6 ? (float)(m - 2) : (m == 6 ? 4.0f : 6.0f));
+  return (c & 8) ? -mag : mag;
+}
+
+// Value of an e4m3 byte (sign bit ignored: scales are non-negative).
+__device__ __forceinline__ float e4m3_value_dev(uint8_t b) {
+  int E = (b >> 3) & 15, m = b & 7;
+  if (E == 0) return ldexpf((float)m, -9);
+  return ldexpf(1.0f + m / 8.0f, E - 7);
+}
+
+// Rounds a non-negative fp32 value to e4m3 (RNE, saturating at 448); returns the bits.
+__device__ __forceinline__ uint8_t e4m3_rne_bits(float x) {
+  if (!(x > 0.f)) return 0;
+  if (x >= 448.f) return 0x7E;
+  int e;
+  frexpf(x, &e);  // x = f 2^e, f in [0.5, 1)
+  int qexp = e - 4;
+  if (qexp < -9) qexp = -9;
+  float q = ldexpf(1.0f, qexp);
+  float r = rintf(x / q) * q;  // x / q exact (power of two), rintf: ties to even
+  if (r > 448.f) r = 448.f;
+  // encode r
+  int e2;
+  float f2 = frexpf(r, &e2);
+  int E = e2 - 1 + 7;
+  if (E <= 0) return (uint8_t)((int)rintf(r / ldexpf(1.0f, -9)) & 7);
+  int mm = (int)rintf((f2 * 2.0f - 1.0f) * 8.0f);
+  return (uint8_t)((E << 3) | mm);
 }
 
 // ---------------------------------------------------------------- warp reductions

@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -35,6 +36,7 @@ constexpr int kTileM = 128;      // output features per GEMM tile (tcgen05 M)
 constexpr int kTileK = 64;       // reduction elements per k-block (one 128-byte swizzle atom)
 constexpr int kMaxTokens = 256;  // tokens per GEMM with plain bf16 activations (tcgen05 N <= 256)
 constexpr int kMaxSplitTokens = 128;  // tokens per GEMM with split (hi + lo) activations
+constexpr int kMaxF4Tokens = 64;      // tokens per NVFP4 GEMM
 
 // Partial-sum layout written by the GEMM: [tile][slot][TP][128] fp32, TP = T rounded up to
 // 32 (token-major: the 128 rows of one token are contiguous).  Tile tau covers
@@ -80,6 +82,7 @@ struct EpiArgs {
   int pos0;
   const int* pos0_dev;
   const float2* rope_tab;       // (cos, sin) of position p, pair j at [p][j], j < hd/2
+  float scale;                  // EPI_STORE: out = scale * y (0 means 1)
   float* h;                     // EPI_RESID / EPI_EMBED: [T][d]
   float* ss;                    // [n_tiles][T]
   const __nv_bfloat16* embed;   // EPI_EMBED
@@ -112,6 +115,26 @@ bool gemm_plan(GemmPlan* p, int a_mode, const void* a0, const void* a1, const vo
                int N, int K, float* partial, char* err, size_t errlen, bool split = false);
 cudaError_t gemm_launch(const GemmPlan& p, int* d_err, cudaStream_t s);
 int gemm_init_attributes();
+
+// NVFP4 GEMM (dlm_gemm_fp4.cu): y = (x quantized per row) W^T with W in NVFP4.  x is given
+// as f16 values q sigma of the row quantizer (`xq`, x_rows >= 64 rows of K) with the row
+// scales `sx`; leaves scaled per-slot partial sums like the bf16 GEMM.  K % 256 == 0, T <= 64.
+struct GemmF4Plan {
+  CUtensorMap tc0, tc1, ts0, ts1, tb;
+  int a_mode;        // A_KMAJOR, or A_PAIR (gate/up: w0 = gate, w1 = up)
+  int nt;            // MMA N: 32 or 64
+  int N, K, T;
+  float sw0, sw1;
+  const float* sx;
+  GemmOut out;
+  size_t partial_bytes;
+};
+size_t gemm_fp4_partial_bytes(int T, int N, int K, int a_mode);
+bool gemm_fp4_plan(GemmF4Plan* p, int a_mode, const dlm_nvfp4_matrix& w0, const dlm_nvfp4_matrix* w1,
+                   const __half* xq, int x_rows, const float* sx, int T, int N, int K, float* partial, char* err,
+                   size_t errlen);
+cudaError_t gemm_fp4_launch(const GemmF4Plan& p, int* d_err, cudaStream_t s);
+int gemm_fp4_init_attributes();
 
 // attention (dlm_attention.cu)
 struct AttnArgs {

@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(1024) k_resid_norm(ResNormArgs a) {
     const bool ok = n < a.d;
     ns[k] = (ok && has_y) ? nsl[n >> 7] : 0;
     pp[k] = has_y ? o.partial + ((size_t)(n >> 7) * o.max_slots * TP + t) * kTileM + (n & 127) : nullptr;
-    base[k] = !ok ? 0.f : (a.embed ? bf2f(a.embed[(size_t)tok * a.d + n]) : a.h[(size_t)t * a.d + n]);
+    base[k] = !ok ? 0.f : (a.embed ? bf2f(a.embed[(size_t)tok * a.d + n]) * a.embed_scale : a.h[(size_t)t * a.d + n]);
 #pragma unroll
     for (int sl = 0; sl < kSlotsReg; ++sl) x[k][sl] = sl < ns[k] ? __ldcg(pp[k] + sl * st) : 0.f;
   }
@@ -352,47 +352,6 @@ __global__ void k_amax_bf16(const __nv_bfloat16* w, long n, unsigned* amax_bits)
   if (threadIdx.x % 32 == 0) atomicMax(amax_bits, __float_as_uint(m));  // m >= 0: bit order = value order
 }
 
-__device__ __forceinline__ uint8_t e2m1_rne(float r) {
-  // magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6; ties to the even code
-  const float a = fabsf(r);
-  uint8_t c;
-  if (a <= 0.25f) c = 0;
-  else if (a < 0.75f) c = 1;
-  else if (a <= 1.25f) c = 2;
-  else if (a < 1.75f) c = 3;
-  else if (a <= 2.5f) c = 4;
-  else if (a < 3.5f) c = 5;
-  else if (a <= 5.0f) c = 6;
-  else c = 7;
-  return (uint8_t)(c | ((r < 0.f) ? 8 : 0));
-}
-
-__device__ __forceinline__ float e4m3_value_dev(uint8_t b) {
-  int E = (b >> 3) & 15, m = b & 7;
-  if (E == 0) return ldexpf((float)m, -9);
-  return ldexpf(1.0f + m / 8.0f, E - 7);
-}
-
-// Rounds a non-negative fp32 value to e4m3 (RNE, saturating at 448); returns the bits.
-__device__ __forceinline__ uint8_t e4m3_rne_bits(float x) {
-  if (!(x > 0.f)) return 0;
-  if (x >= 448.f) return 0x7E;
-  int e;
-  frexpf(x, &e);  // x = f 2^e, f in [0.5, 1)
-  int qexp = e - 4;
-  if (qexp < -9) qexp = -9;
-  float q = ldexpf(1.0f, qexp);
-  float r = rintf(x / q) * q;  // x / q exact (power of two), rintf: ties to even
-  if (r > 448.f) r = 448.f;
-  // encode r
-  int e2;
-  float f2 = frexpf(r, &e2);
-  int E = e2 - 1 + 7;
-  if (E <= 0) return (uint8_t)((int)rintf(r / ldexpf(1.0f, -9)) & 7);
-  int mm = (int)rintf((f2 * 2.0f - 1.0f) * 8.0f);
-  return (uint8_t)((E << 3) | mm);
-}
-
 __global__ void k_nvfp4_quantize(const __nv_bfloat16* w, int rows, int cols, uint8_t* codes,
                                  uint8_t* scales, const unsigned* amax_bits, float* tscale) {
   pdl_trigger();
@@ -417,6 +376,82 @@ __global__ void k_nvfp4_quantize(const __nv_bfloat16* w, int rows, int cols, uin
     uint8_t c1 = denom > 0.f ? e2m1_rne(v[j + 1] / denom) : 0;
     codes[b * 8 + j / 2] = (uint8_t)(c0 | (c1 << 4));
   }
+}
+
+// ------------------------------------------------------------------ NVFP4 activations
+// One CTA (256 threads) per row; each thread owns up to kAqBlocks 16-element blocks.
+constexpr int kAqBlocks = 4;
+__global__ void __launch_bounds__(256) k_act_quant(ActQuantArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float red[32];
+  const int t = blockIdx.x, nb = a.K / 16;
+  float v[kAqBlocks][16];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < kAqBlocks; ++i) {
+    const int b = threadIdx.x + i * 256;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[i][j] = 0.f;
+    if (b < nb) {
+      const size_t off = (size_t)t * a.K + (size_t)b * 16;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        v[i][j] = a.xf ? a.xf[off + j] : bf2f(a.xb[off + j]) + bf2f(a.xb[off + j + a.xb_lo]);
+        amax = fmaxf(amax, fabsf(v[i][j]));
+      }
+    }
+  }
+  amax = warp_max(amax);
+  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = amax;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float m = threadIdx.x < 8 ? red[threadIdx.x] : 0.f;
+    m = warp_max(m);
+    if (threadIdx.x == 0) red[8] = m;
+  }
+  __syncthreads();
+  const float S = red[8] / (6.0f * 448.0f);
+  if (threadIdx.x == 0) a.sx[t] = S;
+#pragma unroll
+  for (int i = 0; i < kAqBlocks; ++i) {
+    const int b = threadIdx.x + i * 256;
+    if (b >= nb) continue;
+    float bm = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) bm = fmaxf(bm, fabsf(v[i][j]));
+    const uint8_t sb = (S > 0.f) ? e4m3_rne_bits(bm / (6.0f * S)) : 0;
+    const float sig = e4m3_value_dev(sb);
+    const float denom = sig * S;
+    __align__(16) __half out[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const uint8_t c = denom > 0.f ? e2m1_rne(v[i][j] / denom) : 0;
+      out[j] = __float2half_rn(e2m1_value_dev(c) * sig);  // exact: <= 6 significant bits
+    }
+    uint4* dst = reinterpret_cast<uint4*>(a.xq + (size_t)t * a.K + (size_t)b * 16);
+    dst[0] = reinterpret_cast<const uint4*>(out)[0];
+    dst[1] = reinterpret_cast<const uint4*>(out)[1];
+  }
+}
+
+// NVFP4 matrix -> bf16 values q sigma (without the tensor scale; exact in bf16), one thread
+// per 16-element block.
+__global__ void k_nvfp4_dequant_bf16(const uint8_t* codes, const uint8_t* scales, long n_blocks,
+                                     __nv_bfloat16* out) {
+  const long b = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= n_blocks) return;
+  const float sig = e4m3_value_dev(scales[b]);
+  __align__(16) __nv_bfloat16 o[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint8_t c = codes[b * 8 + j];
+    o[2 * j] = f2bf(e2m1_value_dev(c & 15) * sig);
+    o[2 * j + 1] = f2bf(e2m1_value_dev(c >> 4) * sig);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(out + b * 16);
+  dst[0] = reinterpret_cast<const uint4*>(o)[0];
+  dst[1] = reinterpret_cast<const uint4*>(o)[1];
 }
 
 }  // namespace dlm

@@ -1,6 +1,7 @@
 // dlm_ops.h -- argument structs and declarations of the light kernels (dlm_ops.cu).
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "dlm_internal.h"
@@ -18,6 +19,7 @@ struct ResNormArgs {
   float* h;                    // [T][d] residual stream
   const __nv_bfloat16* embed;  // non-null: h = E[tokens] + y instead of h += y
   const int32_t* tokens;
+  float embed_scale;           // E rows are multiplied by it (1 for bf16 weights)
   const __nv_bfloat16* gain;   // [d]
   __nv_bfloat16* xn;           // [T][d] high halves
   long xn_lo;                  // elements to the low halves
@@ -35,6 +37,18 @@ struct RowStatsArgs {
   dlm_row_stats stats;
   __nv_bfloat16* P;     // [B][V] high halves, or nullptr
   long P_lo;            // elements to the low halves, 0 = none
+};
+
+// Per-row NVFP4 quantizer of GEMM input activations: row t of x (fp32 `xf`, or the split
+// bf16 pair `xb` + `xb_lo`) gets the scale sx[t] = amax / (6 * 448), one e4m3 scale sigma
+// per 16 elements and e2m1 codes q; xq[t][k] = q sigma as f16 (exact).
+struct ActQuantArgs {
+  const float* xf;
+  const __nv_bfloat16* xb;
+  long xb_lo;
+  int K;
+  __half* xq;
+  float* sx;
 };
 
 struct CommitArgs {
@@ -81,6 +95,9 @@ __global__ void k_commit(CommitArgs a);
 __global__ void k_block_init(BlockInitArgs a);
 __global__ void k_block_finish(BlockFinishArgs a);
 __global__ void k_set_int(int* p, int v);
+__global__ void k_act_quant(ActQuantArgs a);
+__global__ void k_nvfp4_dequant_bf16(const uint8_t* codes, const uint8_t* scales, long n_blocks,
+                                     __nv_bfloat16* out);
 __global__ void k_rope_table(float2* tab, int max_ctx, int hd, double base);
 __global__ void k_amax_to_scale(float* p);
 __global__ void k_amax_bf16(const __nv_bfloat16* w, long n, unsigned* amax_bits);

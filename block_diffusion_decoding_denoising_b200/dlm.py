@@ -112,6 +112,9 @@ def lib():
         L.dlm_bd_attention.argtypes = [p, p, p, p, i, i, i, i, i, i, i, p, z, p]
         L.dlm_commit.argtypes = [p, p, p, p, p, p, p, i, i, f, i, i, p]
         L.dlm_nvfp4_quantize.argtypes = [p, i, i, p, p, p, p]
+        L.dlm_gemm_nvfp4_scratch_size.restype = z
+        L.dlm_gemm_nvfp4_scratch_size.argtypes = [i, i, i]
+        L.dlm_gemm_nvfp4.argtypes = [p, C.POINTER(Nvfp4Matrix), p, i, i, i, p, z, p]
         L.dlm_debug_set_pdl.argtypes = [i]
         _lib = L
     return _lib
@@ -119,6 +122,10 @@ def lib():
 
 def _ptr(t):
     return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _addr(t):
+    return None if t is None else t.data_ptr()
 
 
 def _stream(stream=None):
@@ -242,6 +249,46 @@ def nvfp4_quantize(w, stream=None):
     return codes, scales, ts
 
 
+def _q_matrix(q):
+    return Nvfp4Matrix(_ptr(q["codes"]).value, _ptr(q["scales"]).value, float(q["tscale"]))
+
+
+def nvfp4_matrix(w, stream=None):
+    """NVFP4 form of a bf16 [rows][cols] weight as a dict(codes, scales, tscale (float), rows, cols)."""
+    codes, scales, ts = nvfp4_quantize(w, stream)
+    return {"codes": codes, "scales": scales, "tscale": float(ts.item()), "rows": w.shape[0], "cols": w.shape[1]}
+
+
+def quantize_model(weights: dict, stream=None) -> dict:
+    """Adds the NVFP4 matrices an NVFP4 model runs on (q_gate, q_up, q_down per layer and
+    q_embed) to a bf16 weight dict, quantized on the device."""
+    out = dict(weights)
+    out["layers"] = []
+    for lw in weights["layers"]:
+        l2 = dict(lw)
+        for n in ("gate", "up", "down"):
+            l2["q_" + n] = nvfp4_matrix(lw["w_" + n], stream)
+        out["layers"].append(l2)
+    out["q_embed"] = nvfp4_matrix(weights["embed"], stream)
+    return out
+
+
+def gemm_nvfp4(x, q, stream=None):
+    """y[T][N] fp32 = Q(x) W^T with W the NVFP4 matrix q (see nvfp4_matrix) and Q the
+    per-row NVFP4 quantizer of x (fp32 [T][K])."""
+    import torch
+    T, K = x.shape
+    N = q["rows"]
+    y = torch.empty((T, N), dtype=torch.float32, device=x.device)
+    n = lib().dlm_gemm_nvfp4_scratch_size(T, N, K)
+    if n == 0:
+        raise DlmError(DLM_EINVAL, "unsupported nvfp4 gemm shape")
+    sc = _scratch(n, x.device)
+    m = _q_matrix(q)
+    _check(lib().dlm_gemm_nvfp4(_ptr(x), C.byref(m), _ptr(y), T, N, K, _ptr(sc), n, _stream(stream)))
+    return y
+
+
 # ------------------------------------------------------------------ model context
 class Model:
     """Owns (through torch) the workspace and the KV cache of one dlm context."""
@@ -255,13 +302,17 @@ class Model:
         L = lib()
         nl = cfg["n_layers"]
         self._layers = (LayerWeights * max(nl, 1))()
+        fp4 = int(cfg.get("weight_fmt", 0)) == WEIGHTS_NVFP4
+        empty = Nvfp4Matrix(None, None, 0.0)
         for i, lw in enumerate(weights["layers"]):
+            qs = [_q_matrix(lw["q_" + n]) if fp4 else empty for n in ("gate", "up", "down")]
             self._layers[i] = LayerWeights(_ptr(lw["attn_norm"]).value, _ptr(lw["w_qkv"]).value,
                                            _ptr(lw["w_o"]).value, _ptr(lw["mlp_norm"]).value,
-                                           _ptr(lw["w_gate"]).value, _ptr(lw["w_up"]).value,
-                                           _ptr(lw["w_down"]).value)
-        self._w = Weights(_ptr(weights["embed"]).value, _ptr(weights["w_adapter"]).value,
-                          _ptr(weights["final_norm"]).value, self._layers)
+                                           _addr(lw.get("w_gate")), _addr(lw.get("w_up")),
+                                           _addr(lw.get("w_down")), *qs)
+        self._w = Weights(_addr(weights.get("embed")), _ptr(weights["w_adapter"]).value,
+                          _ptr(weights["final_norm"]).value, self._layers,
+                          _q_matrix(weights["q_embed"]) if fp4 else empty)
         ws = L.dlm_workspace_size(C.byref(self.cfg))
         kv = L.dlm_kv_cache_size(C.byref(self.cfg))
         if ws == 0:

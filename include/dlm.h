@@ -97,11 +97,13 @@ typedef struct dlm_layer_weights {
 } dlm_layer_weights;
 
 typedef struct dlm_weights {
-  const void* embed;      /* E, bf16 [V][d]: token embedding and tied LM head */
+  const void* embed;      /* E, bf16 [V][d]: token embedding and tied LM head (bf16 weights;
+                             unused with NVFP4 weights, where E is q_embed throughout) */
   const void* w_adapter;  /* W_a, bf16 [d][d] */
   const void* final_norm; /* bf16 [d] */
   const dlm_layer_weights* layers; /* host array [n_layers]; copied by dlm_ctx_create */
-  dlm_nvfp4_matrix q_embed; /* NVFP4 E for the LM head when weight_fmt == NVFP4 */
+  dlm_nvfp4_matrix q_embed; /* NVFP4 E when weight_fmt == NVFP4: the LM head streams it; the
+                               embedding rows and P E use its dequantised values */
 } dlm_weights;
 
 /* Per-row statistics of one round, device arrays of length B. */
@@ -241,6 +243,16 @@ dlm_status dlm_commit(const float* d_maxprob, const int32_t* d_argmax, int32_t* 
  * Writes codes uint8 [rows][cols/2], scales uint8 [rows][cols/16], *d_tensor_scale. */
 dlm_status dlm_nvfp4_quantize(const void* d_w, int rows, int cols, void* d_codes, void* d_scales,
                               float* d_tensor_scale, void* stream);
+
+/* NVFP4 weight GEMM: y[T][N] (fp32) = Q(x) W^T, where W is an NVFP4 matrix [N][K] (see
+ * dlm_nvfp4_matrix; host struct, device arrays) and Q(x) quantizes each row of x (fp32
+ * [T][K]) to NVFP4 with its own fp32 scale amax_row / (6 * 448), e4m3 scales per 16 elements
+ * and round-to-nearest-even e2m1 codes, the format the pages' B200 numbers use ("ORL:
+ * diffusion LLMs get a learnable 'tokens per forward'", "What shipped").  T <= 64,
+ * K % 256 == 0, K <= 16384.  d_y may be NULL: partial sums only (kernel timing). */
+size_t dlm_gemm_nvfp4_scratch_size(int T, int N, int K);
+dlm_status dlm_gemm_nvfp4(const float* d_x, const dlm_nvfp4_matrix* w, float* d_y, int T, int N, int K,
+                          void* d_scratch, size_t scratch_bytes, void* stream);
 
 /* Version string of the build. */
 const char* dlm_version(void);
