@@ -110,6 +110,7 @@ def lib():
         L.dlm_attention_scratch_size.restype = z
         L.dlm_attention_scratch_size.argtypes = [i, i, i, i]
         L.dlm_bd_attention.argtypes = [p, p, p, p, i, i, i, i, i, i, i, p, z, p]
+        L.dlm_bd_attention_noalloc.argtypes = [p, p, p, p, i, i, i, i, i, i, i, p]
         L.dlm_commit.argtypes = [p, p, p, p, p, p, p, i, i, f, i, i, p]
         L.dlm_nvfp4_quantize.argtypes = [p, i, i, p, p, p, p]
         L.dlm_gemm_nvfp4_scratch_size.restype = z
@@ -229,6 +230,19 @@ def bd_attention(q, k_cache, v_cache, L, causal=False, stream=None):
     sc = _scratch(n, q.device)
     _check(lib().dlm_bd_attention(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), T, int(L), Hq, Hkv, hd,
                                   max_ctx, int(causal), _ptr(sc), n, _stream(stream)))
+    return o
+
+
+def bd_attention_noalloc(q, k_cache, v_cache, L, causal=False, o=None, stream=None):
+    """bd_attention through the entry point that takes no scratch (library-owned static
+    device memory; see dlm_bd_attention_noalloc).  `o` may be given to reuse an output."""
+    import torch
+    T, Hq, hd = q.shape
+    Hkv, max_ctx, _ = k_cache.shape
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib().dlm_bd_attention_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), T, int(L), Hq, Hkv,
+                                          hd, max_ctx, int(causal), _stream(stream)))
     return o
 
 
