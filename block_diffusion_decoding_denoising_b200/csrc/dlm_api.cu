@@ -363,7 +363,8 @@ dlm_status act_quant(Runner& r, int T, const __nv_bfloat16* x, long lo, int K) {
 dlm_status finish_tiles(Runner& r, const GemmOut& y, int N, const EpiArgs& epi) {
   dlm_ctx* ctx = r.ctx;
   FinishArgs a{y, epi, N};
-  CU_LAUNCH(launch_k(k_finish_tiles, dim3(y.n_tiles, (y.T + 31) / 32), dim3(128), 0, r.s, a));
+  void (*k)(FinishArgs) = epi.op == EPI_QKV ? k_finish_qkv : (epi.op == EPI_SILU ? k_finish_silu : k_finish_store);
+  CU_LAUNCH(launch_k(k, dim3(y.n_tiles, (y.T + 31) / 32), dim3(256), 0, r.s, a));
   return DLM_OK;
 }
 
@@ -1136,7 +1137,7 @@ dlm_status dlm_gemm_nvfp4(const float* d_x, const dlm_nvfp4_matrix* w, float* d_
     e.out = d_y;
     e.ld = N;
     FinishArgs fa{p.out, e, N};
-    CU_LAUNCH(launch_k(k_finish_tiles, dim3(p.out.n_tiles, (T + 31) / 32), dim3(128), 0, s, fa));
+    CU_LAUNCH(launch_k(k_finish_store, dim3(p.out.n_tiles, (T + 31) / 32), dim3(256), 0, s, fa));
   }
   return DLM_OK;
 }

@@ -33,23 +33,122 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return r;
 }
 
-struct SyncAll {
-  __device__ __forceinline__ void operator()() const { __syncthreads(); }
-};
+// ------------------------------------------------------------------ tile finishers
+// The finishers sum a GEMM's per-slot partials ([tile][slot][TP][128], slot order) for one
+// tile and 32 tokens (grid: tiles x ceil(T / 32)) and apply the op.  256 threads; a thread
+// owns a pair of tile rows for 8 tokens, so RoPE (rows j, j + hd/2) and SiLU-mul (gate row
+// r, up row r + 64) combine values the same thread loaded: no shared memory, no barrier.
+// All loads of a thread are issued before any sum.
+constexpr int kFinTok = 8;    // tokens per thread
+constexpr int kFinSlots = 4;  // slots loaded per batch
 
-// Finishes the tiles of a GEMM that left per-slot partial sums: sums the slots of (tile,
-// 32 tokens) in slot order and applies the op (RoPE + KV cache, SiLU gate, or a store).
-// grid (n_tiles, ceil(T/32)), 128 threads (thread = tile row).
-__global__ void k_finish_tiles(FinishArgs a) {
+// v[a|b][j] = sum over slots of rows ra / rb, tokens t0 + j (0 where t0 + j >= T)
+__device__ __forceinline__ void finish_load_pair(const GemmOut& o, int tile, int ra, int rb, int t0,
+                                                 float (&va)[kFinTok], float (&vb)[kFinTok]) {
+  const int TP = (o.T + 31) / 32 * 32;
+  const int ns = tile_slots(o, tile);
+  const float* base = o.partial + (size_t)tile * o.max_slots * kTileM * TP + (size_t)t0 * kTileM;
+#pragma unroll
+  for (int j = 0; j < kFinTok; ++j) { va[j] = 0.f; vb[j] = 0.f; }
+  for (int sl = 0; sl < ns; sl += kFinSlots) {
+    float xa[kFinSlots][kFinTok], xb[kFinSlots][kFinTok];
+#pragma unroll
+    for (int b = 0; b < kFinSlots; ++b) {
+      const float* p = base + (size_t)(sl + b) * kTileM * TP;
+      const bool ok = sl + b < ns;
+#pragma unroll
+      for (int j = 0; j < kFinTok; ++j) {
+        const bool in = ok && t0 + j < o.T;
+        xa[b][j] = in ? __ldcg(p + (size_t)j * kTileM + ra) : 0.f;
+        xb[b][j] = in ? __ldcg(p + (size_t)j * kTileM + rb) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kFinSlots; ++b)
+#pragma unroll
+      for (int j = 0; j < kFinTok; ++j) { va[j] += xa[b][j]; vb[j] += xb[b][j]; }
+  }
+}
+
+// QKV: RoPE (NeoX pairs j, j + hd/2, angles from the fp64-built table) on q and k heads;
+// q as bf16 [T][Hq][hd], K and V rows into the cache at positions L + t.
+__global__ void __launch_bounds__(256) k_finish_qkv(FinishArgs a) {
   pdl_trigger();
   pdl_wait();
-  __shared__ float xch[128][33];
-  const int tile = blockIdx.x, t0 = blockIdx.y * 32, row = threadIdx.x;
-  const int TP = (a.out.T + 31) / 32 * 32;
-  float v[32];
-  sum_slots32<4>(a.out, tile, row, t0, TP, tile_slots(a.out, tile), v);
-  const int L = (a.epi.op == EPI_QKV) ? (a.epi.pos0_dev ? *a.epi.pos0_dev : a.epi.pos0) : 0;
-  apply_epi(a.epi, a.N, a.out.T, tile, row, t0, v, xch, L, SyncAll());
+  const EpiArgs& e = a.epi;
+  const int tile = blockIdx.x, p = threadIdx.x % 64, tg = threadIdx.x / 64;
+  const int t0 = blockIdx.y * 32 + tg * kFinTok;
+  const int half = e.hd / 2;
+  const int ra = (p / half) * e.hd + p % half, rb = ra + half;  // rows of the pair in the tile
+  const int n = tile * kTileM + ra;                              // feature of row ra
+  if (n >= a.N || t0 >= a.out.T) return;
+  const int L = e.pos0_dev ? *e.pos0_dev : e.pos0;
+  float va[kFinTok], vb[kFinTok];
+  finish_load_pair(a.out, tile, ra, rb, t0, va, vb);
+  const int hh = n / e.hd, jj = n % e.hd;  // jj < half
+  const bool rope = hh < e.Hq + e.Hkv;
+  float2 cs[kFinTok];
+#pragma unroll
+  for (int j = 0; j < kFinTok; ++j)
+    cs[j] = (rope && t0 + j < a.out.T) ? e.rope_tab[(size_t)(L + t0 + j) * half + jj] : make_float2(1.f, 0.f);
+  __nv_bfloat16* dst;
+  size_t stride_t;
+  if (hh < e.Hq) {
+    dst = e.q + (size_t)t0 * e.Hq * e.hd + (size_t)hh * e.hd + jj;
+    stride_t = (size_t)e.Hq * e.hd;
+  } else if (hh < e.Hq + e.Hkv) {
+    dst = e.kc + ((size_t)(hh - e.Hq) * e.max_ctx + L + t0) * e.hd + jj;
+    stride_t = e.hd;
+  } else {
+    dst = e.vc + ((size_t)(hh - e.Hq - e.Hkv) * e.max_ctx + L + t0) * e.hd + jj;
+    stride_t = e.hd;
+  }
+#pragma unroll
+  for (int j = 0; j < kFinTok; ++j) {
+    if (t0 + j < a.out.T) {
+      const float x0 = va[j], x1 = vb[j];
+      dst[(size_t)j * stride_t] = f2bf(x0 * cs[j].x - x1 * cs[j].y);
+      dst[(size_t)j * stride_t + half] = f2bf(x0 * cs[j].y + x1 * cs[j].x);
+    }
+  }
+}
+
+// gate/up pair tile (gate features in rows 0..63, up in 64..127): act = silu(g) u as a split
+// bf16 pair.
+__global__ void __launch_bounds__(256) k_finish_silu(FinishArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const EpiArgs& e = a.epi;
+  const int tile = blockIdx.x, r = threadIdx.x % 64, tg = threadIdx.x / 64;
+  const int t0 = blockIdx.y * 32 + tg * kFinTok;
+  const int f = tile * 64 + r;
+  if (f >= a.N || t0 >= a.out.T) return;
+  float g[kFinTok], u[kFinTok];
+  finish_load_pair(a.out, tile, r, r + 64, t0, g, u);
+#pragma unroll
+  for (int j = 0; j < kFinTok; ++j)
+    if (t0 + j < a.out.T) store_split(e.act + (size_t)(t0 + j) * a.N + f, e.act_lo, g[j] / (1.0f + expf(-g[j])) * u[j]);
+}
+
+// out[t][n] = scale * y (scale 0 means 1), rows r and r + 64 of the tile per thread.
+__global__ void __launch_bounds__(256) k_finish_store(FinishArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const EpiArgs& e = a.epi;
+  const int tile = blockIdx.x, r = threadIdx.x % 64, tg = threadIdx.x / 64;
+  const int t0 = blockIdx.y * 32 + tg * kFinTok;
+  if (t0 >= a.out.T) return;
+  float va[kFinTok], vb[kFinTok];
+  finish_load_pair(a.out, tile, r, r + 64, t0, va, vb);
+  const float sc = e.scale != 0.f ? e.scale : 1.f;
+  const int na = tile * kTileM + r, nb = na + 64;
+#pragma unroll
+  for (int j = 0; j < kFinTok; ++j) {
+    if (t0 + j < a.out.T) {
+      if (na < a.N) e.out[(size_t)(t0 + j) * e.ld + na] = (e.scale != 0.f) ? va[j] * sc : va[j];
+      if (nb < a.N) e.out[(size_t)(t0 + j) * e.ld + nb] = (e.scale != 0.f) ? vb[j] * sc : vb[j];
+    }
+  }
 }
 
 // Residual update and RMSNorm of one token row (one CTA per token):

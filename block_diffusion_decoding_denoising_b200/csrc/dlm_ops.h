@@ -86,7 +86,9 @@ struct BlockFinishArgs {
   int B;
 };
 
-__global__ void k_finish_tiles(FinishArgs a);
+__global__ void k_finish_qkv(FinishArgs a);
+__global__ void k_finish_silu(FinishArgs a);
+__global__ void k_finish_store(FinishArgs a);
 __global__ void k_resid_norm(ResNormArgs a);
 __global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo);
 __global__ void k_rowstats_part(RowStatsArgs a);
