@@ -45,7 +45,7 @@ def parse():
     # profiling cases (small, for ncu): "quick" = the decode loop on 256 generated tokens
     # without the extra measurements; "gemm" = every projection GEMM of two layers plus
     # the LM-head GEMM, `--steps` launches each
-    ap.add_argument("--case", default="full", choices=["full", "quick", "gemm"])
+    ap.add_argument("--case", default="full", choices=["full", "quick", "gemm", "lmhead"])
     # the quick case with eager dlm_round / dlm_kv_fill calls instead of the block graph
     # (same kernels; ncu cannot profile kernel nodes of graphs with conditional nodes)
     ap.add_argument("--eager", action="store_true")
@@ -229,12 +229,49 @@ def gemm_case(args):
     print(json.dumps({"case": "gemm", "us_per_launch": times}))
 
 
+def lmhead_case(args):
+    """Single round of the LM head at 4B-class shapes (B 32, d 2560, V 151936): the fused
+    pass over E with a given P_prev (the config's own workload) and with P = softmax, then
+    the W_a adapter step; `--steps` timed calls each after `--warmup`."""
+    import torch
+
+    from block_diffusion_decoding_denoising_b200 import build, dlm, gen
+    build.build()
+    B, d, V = 32, 2560, 151936
+    H, E, Wa, P = gen.lmhead_inputs_torch(B, d, V)
+    x = H.to(torch.bfloat16)
+    tokens = torch.full((B,), V - 1, dtype=torch.int32, device="cuda")
+    s = torch.zeros((B, d), dtype=torch.float32, device="cuda")
+    out = {}
+    for name, fn in (("lmhead_given_p", lambda: dlm.lmhead_rowstats(x, E, mask_id=V - 1, p_given=P)),
+                     ("lmhead_softmax", lambda: dlm.lmhead_rowstats(x, E, mask_id=V - 1)),
+                     ("adapter", lambda: dlm.adapter_embed(E, Wa, tokens, s))):
+        for _ in range(max(args.warmup, 1)):
+            fn()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record()
+        for _ in range(args.steps):
+            fn()
+        ev[1].record()
+        torch.cuda.synchronize()
+        out[name] = ev[0].elapsed_time(ev[1]) * 1e3 / args.steps
+    e_bytes = V * d * 2
+    hbm, _, kind = peaks()
+    gbs = (e_bytes + B * V * 2) / (out["lmhead_given_p"] * 1e-6) / 1e9
+    print(json.dumps({"case": "lmhead", "us_per_call": out, "given_p_GBs": gbs, "frac": gbs / hbm,
+                      "peak": hbm, "peak_kind": kind}), flush=True)
+
+
 def main():
     global GEN
     args = parse()
     from block_diffusion_decoding_denoising_b200 import gen
     if args.case == "gemm":
         gemm_case(args)
+        return
+    if args.case == "lmhead":
+        lmhead_case(args)
         return
     if args.case == "quick":
         GEN = 256

@@ -74,6 +74,7 @@ struct dlm_ctx {
   int32_t* tok_buf = nullptr;
   // NVFP4 weights: quantized GEMM inputs, their row scales, and E dequantised to bf16
   // (q sigma, exact; the tensor scale is applied where the rows are used)
+  void* lmf = nullptr;  // scratch of the fused LM head (null: the unfused path is used)
   bool fp4 = false;
   __half* xq = nullptr;
   float* sx = nullptr;
@@ -202,7 +203,10 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   __half* xq = fp4 ? cv.take<__half>((size_t)kMaxF4Tokens * (c.d > c.ffn ? c.d : c.ffn)) : nullptr;
   float* sx = fp4 ? cv.take<float>(kMaxF4Tokens) : nullptr;
   __nv_bfloat16* edq = fp4 ? cv.take<__nv_bfloat16>((size_t)c.vocab * c.d) : nullptr;
+  const bool fused = !fp4 && lmhead_fused_supported(B, c.d);
+  uint8_t* lmf = fused ? cv.take<uint8_t>(lmhead_fused_scratch_bytes(c.vocab, c.d)) : nullptr;
   if (x && base) {
+    x->lmf = lmf;
     x->fp4 = fp4;
     x->xq = xq;
     x->sx = sx;
@@ -463,6 +467,14 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
 
   // LM head: logits (finished inside the GEMM: its tiles are mostly single-slot), row
   // statistics, P = softmax (split bf16), s = P E
+  if (ctx->lmf && T <= 32) {
+    // one pass over E: logits, row statistics and s = P E (split x: pad = 32 for T <= 32)
+    char msg[256];
+    cudaError_t e = lmhead_fused_launch(ctx->xn, ctx->w.embed, nullptr, T, c.vocab, d, c.mask_id, f.stats, f.s_out,
+                                        ctx->lmf, ctx->d_err, r.s, msg, sizeof(msg));
+    if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "fused lm head: %s %s", cudaGetErrorString(e), msg);
+    return DLM_OK;
+  }
   EpiArgs el{};
   el.op = EPI_STORE;
   el.out = ctx->logits;
@@ -936,8 +948,12 @@ dlm_status dlm_gemm_bf16x2(const void* d_x2, const void* d_w, float* d_y, int T,
 
 size_t dlm_lmhead_scratch_size(int B, int V, int d) {
   const int nch = (V + kRowChunk - 1) / kRowChunk;
-  return op_header() + op_counters(V > d ? V : d) + align256(lmhead_partial(B, V, d)) +
-         align256((size_t)B * V * 4) + align256((size_t)2 * split_pad(B) * V * 2) + align256((size_t)16 * B * nch);
+  size_t unfused = op_header() + op_counters(V > d ? V : d) + align256(lmhead_partial(B, V, d)) +
+                   align256((size_t)B * V * 4) + align256((size_t)2 * split_pad(B) * V * 2) +
+                   align256((size_t)16 * B * nch);
+  if (!lmhead_fused_supported(B, d)) return unfused;
+  size_t fused = op_header() + align256((size_t)64 * d * 2) + align256(lmhead_fused_scratch_bytes(V, d));
+  return fused > unfused ? fused : unfused;
 }
 
 dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int V, int d, int mask_id,
@@ -948,8 +964,20 @@ dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int 
       d % 64 || !stats.m || !stats.lse || !stats.maxprob || !stats.entropy || !stats.argmax)
     return DLM_EINVAL;
   if (scratch_bytes < dlm_lmhead_scratch_size(B, V, d)) return DLM_ENOMEM_WS;
-  CU((cudaError_t)gemm_init_attributes());
   cudaStream_t s = (cudaStream_t)stream;
+  if (lmhead_fused_supported(B, d)) {
+    // one pass over E; x as the split pair the kernel reads (high halves = x, low halves 0)
+    uint8_t* base = (uint8_t*)d_scratch;
+    void* x2 = base + op_header();
+    void* lmf = base + op_header() + align256((size_t)64 * d * 2);
+    CU(cudaMemsetAsync(base, 0, op_header() + (size_t)64 * d * 2, s));
+    CU(cudaMemcpyAsync(x2, d_x, (size_t)B * d * 2, cudaMemcpyDeviceToDevice, s));
+    char msg[256];
+    cudaError_t e = lmhead_fused_launch(x2, d_embed, d_p_given, B, V, d, mask_id, stats, d_s, lmf, (int*)base, s,
+                                        msg, sizeof(msg));
+    return e == cudaSuccess ? DLM_OK : DLM_ECUDA;
+  }
+  CU((cudaError_t)gemm_init_attributes());
   const int nch = (V + kRowChunk - 1) / kRowChunk;
   OpScratch sc(d_scratch, V > d ? V : d, lmhead_partial(B, V, d));
   float* logits = sc.take<float>((size_t)B * V);

@@ -93,6 +93,27 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// The same load with an L2 eviction-priority policy (see l2_policy_*).
+__device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                                 int y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+// L2 policies: keep lines that will be read again soon / let lines read for the last time go.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -183,12 +204,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool a_mn_major,
 // ---------------------------------------------------------------- stream-K partition
 // The (tile, k-block) units of a GEMM are cut into `grid` contiguous ranges; CTA c owns
 // units [unit_begin(c), unit_begin(c + 1)).
+// 32-bit arithmetic (the planners keep units * grid below 2^32; a 64-bit division costs
+// about a hundred instructions on the critical path of every finishing thread).
 __host__ __device__ __forceinline__ long unit_begin(int c, long units, int grid) {
-  return (long)c * units / grid;
+  return (long)((uint32_t)c * (uint32_t)units / (uint32_t)grid);
 }
 // Largest CTA index c with unit_begin(c) <= u.
 __host__ __device__ __forceinline__ int cta_of_unit(long u, long units, int grid) {
-  int c = (int)((u * (long)grid) / units);
+  int c = (int)((uint32_t)u * (uint32_t)grid / (uint32_t)units);
   if (c >= grid) c = grid - 1;
   while (c + 1 < grid && unit_begin(c + 1, units, grid) <= u) ++c;
   while (c > 0 && unit_begin(c, units, grid) > u) --c;

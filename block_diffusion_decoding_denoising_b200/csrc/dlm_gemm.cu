@@ -368,6 +368,10 @@ bool gemm_plan(GemmPlan* p, int a_mode, const void* a0, const void* a1, const vo
   p->lo_col = split ? split_pad(T) : 0;
   partition(T, N, K, a_mode, &p->out);
   p->out.partial = partial;
+  if ((unsigned long long)p->out.units * (unsigned long long)p->out.grid >= (1ull << 32)) {
+    snprintf(err, errlen, "gemm: %ld units exceed the 32-bit partition arithmetic", p->out.units);
+    return false;
+  }
   p->partial_bytes = gemm_partial_bytes(T, N, K, a_mode);
   bool ok = true;
   if (a_mode == A_KMAJOR) {

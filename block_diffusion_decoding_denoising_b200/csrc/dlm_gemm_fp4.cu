@@ -441,6 +441,10 @@ bool gemm_fp4_plan(GemmF4Plan* p, int a_mode, const dlm_nvfp4_matrix& w0, const 
   p->sx = sx;
   partition_f4(T, N, K, a_mode, &p->out);
   p->out.partial = partial;
+  if ((unsigned long long)p->out.units * (unsigned long long)p->out.grid >= (1ull << 32)) {
+    snprintf(err, errlen, "gemm: %ld units exceed the 32-bit partition arithmetic", p->out.units);
+    return false;
+  }
   p->partial_bytes = gemm_fp4_partial_bytes(T, N, K, a_mode);
   const uint32_t rows = (a_mode == A_PAIR) ? 64 : kTileM;
   bool ok = encode_2d(&p->tc0, CU_TENSOR_MAP_DATA_TYPE_UINT8, w0.codes, (uint64_t)K / 2, N, (uint64_t)K / 2, 128,

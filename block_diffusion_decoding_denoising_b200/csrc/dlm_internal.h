@@ -136,6 +136,15 @@ bool gemm_fp4_plan(GemmF4Plan* p, int a_mode, const dlm_nvfp4_matrix& w0, const 
 cudaError_t gemm_fp4_launch(const GemmF4Plan& p, int* d_err, cudaStream_t s);
 int gemm_fp4_init_attributes();
 
+// LM head fused with the row statistics and s = P E (dlm_lmhead.cu), one pass over E.
+// x2: split bf16 pair, rows [0, T) high halves, rows [32, 32 + T) low halves; p_given:
+// bf16 [T][V] or nullptr (P = softmax of the logits).  T <= 32, d % 256 == 0, d <= 3584.
+bool lmhead_fused_supported(int T, int d);
+size_t lmhead_fused_scratch_bytes(int V, int d);
+cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_given, int T, int V, int d,
+                                int mask_id, dlm_row_stats stats, float* s, void* scratch, int* d_err,
+                                cudaStream_t st, char* err, size_t errlen);
+
 // attention (dlm_attention.cu)
 struct AttnArgs {
   const __nv_bfloat16* q;    // [T][Hq][hd]

@@ -1,0 +1,610 @@
+// dlm_lmhead.cu -- the LM head fused with the row statistics and the residual contraction,
+// in one pass over the tied embedding E:
+//   logits = x E^T (never stored), per row: max, lowest argmax, Z = sum e^(l - r),
+//   A = sum e^(l - r) l for a reference r, and s = P E with P = softmax(logits) (or a
+//   given P).
+// ("QwenDLM-4B-ORL" model card, "The paper's evaluation pipeline": the LM head runs with
+// fused row statistics; "ORL: diffusion LLMs get a learnable 'tokens per forward'", "What
+// shipped": the previous round's distribution is fed back through the tied embedding.)
+//
+// Work split: vocabulary tiles of 128 rows, a contiguous range of tiles per cluster of two
+// CTAs; CTA rank r owns the model-width half [r d/2, (r + 1) d/2).  Per tile:
+//   L  partial logits over the CTA's half: tcgen05, A = E tile (K-major), B = x (split
+//      bf16 hi + lo accumulated into the same TMEM columns); double-buffered accumulator.
+//   X  the two partial logit tiles are swapped through distributed shared memory (remote
+//      stores + a remote mbarrier arrive with cluster-scope release), so both CTAs hold
+//      the same full logits; they are read transposed ([token][vocab]) for the per-token
+//      reductions.  Running reference r_t: the first tile's max, raised (and the
+//      accumulators rescaled) only when a tile's max exceeds it by more than 8.
+//   PE s^T[d][t] += E_tile^T P_tile: tcgen05 with A = the same E tile re-read (from L2) as
+//      an MN-major operand and B = P written by the epilogue into shared memory as a split
+//      bf16 pair; s stays in TMEM (one 128-row x 32-column accumulator per 128 features).
+// The MMA warp issues L(i + 1) before PE(i) so the statistics of tile i overlap the next
+// tile's weight stream.  A cluster leaves (r, Z, A, max, argmax) per token and its s half;
+// k_lmf_combine merges the clusters in a fixed order.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "dlm_device.cuh"
+#include "dlm_internal.h"
+
+namespace dlm {
+
+namespace {
+
+constexpr int kLmT = 32;                // tokens (MMA N)
+constexpr int kLmStages = 5;
+constexpr int kLmStageBytes = 24576;    // E box 16 KB + x box 8 KB (L) / 2 E boxes + P box (PE)
+constexpr int kLmPBytes = 16384;        // P tile: 64 rows (hi, lo) x 128 vocab, 2 swizzle atoms
+constexpr int kLmXBytes = kLmT * 128 * 4;  // one partial-logit tile [32][128] fp32
+constexpr int kLmMaxChunks = 14;        // d / 2 <= 1792
+constexpr int kLmSCol = 64;             // TMEM column of the first s accumulator
+constexpr float kLmRescale = 8.0f;      // raise the reference when a max exceeds it by this
+constexpr int kLmSmem = kLmStages * kLmStageBytes + 2 * kLmPBytes + 4 * kLmXBytes + 1024 + 1024;
+
+struct LmfArgs {
+  int V, d, T, mask_id;
+  int n_tiles, n_clu;
+  int given;            // 1: P comes from memory (tp), s = P E without normalisation
+  float* part_stats;    // [n_clu][32][4]: reference, Z, A, max
+  int* part_arg;        // [n_clu][32]
+  float* part_s;        // [n_clu][d][32]
+  int* err;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_peer(uint32_t local_addr, uint32_t peer) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(peer));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* err) {
+  for (uint32_t i = 0; i < kWaitPolls; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (i >= 16) __nanosleep(i < 1024 ? 32 : 256);
+  }
+  set_error(err, DLM_ETIMEOUT);
+  return false;
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st32_f(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
+      "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]),
+      "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
+      "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Barrier of the 128 epilogue threads that also returns whether any of them passed true.
+__device__ __forceinline__ bool epi_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+__host__ __device__ __forceinline__ int lm_tile_begin(int c, int n_tiles, int n_clu) {
+  return (int)((long)c * n_tiles / n_clu);
+}
+
+// Offset of element (row, v) of the P tile (K-major B operand, 128-byte swizzle, two 64-wide
+// atoms of 64 rows each).
+__device__ __forceinline__ uint32_t p_offset(int row, int v) {
+  const int atom = v >> 6, c = v & 63;
+  return (uint32_t)(atom * 8192 + row * 128 + ((((c >> 3) ^ (row & 7)) << 4) | ((c & 7) << 1)));
+}
+
+__global__ void __launch_bounds__(192, 1)
+k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ CUtensorMap tem,
+               const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tp, LmfArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* ring = smem;
+  uint8_t* pbuf = smem + kLmStages * kLmStageBytes;                     // [2][16 KB]
+  float* mine = (float*)(pbuf + 2 * kLmPBytes);                         // [2][32][128]
+  float* theirs = mine + 2 * kLmT * 128;                                // [2][32][128]
+  uint64_t* bars = (uint64_t*)(theirs + 2 * kLmT * 128);
+  uint64_t* full = bars;                      // [S]
+  uint64_t* empty = bars + kLmStages;         // [S]
+  uint64_t* accl_full = bars + 2 * kLmStages; // [2]
+  uint64_t* accl_empty = accl_full + 2;       // [2] (128 arrivals)
+  uint64_t* p_ready = accl_empty + 2;         // [2] (4 arrivals)
+  uint64_t* pe_done = p_ready + 2;            // [2]
+  uint64_t* xfull = pe_done + 2;              // [2] (128 remote arrivals from the peer)
+  uint64_t* mma_done = xfull + 2;
+  uint32_t* tmem_holder = (uint32_t*)(mma_done + 1);
+  int* flag = (int*)(mma_done + 2);
+  float* fac = (float*)(mma_done + 3);        // [32] rescale factors of the current tile
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
+  const int clu = blockIdx.x / 2;
+  const int dh = a.d / 2, d0 = (int)rank * dh;
+  const int KB = dh / 64, CH = dh / 128;
+  const int tb = lm_tile_begin(clu, a.n_tiles, a.n_clu), te = lm_tile_begin(clu + 1, a.n_tiles, a.n_clu);
+  const int nt = te - tb;
+
+  if (warp == 1 && lane == 0) {
+    for (int i = 0; i < kLmStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accl_full[i], 1);
+      mbar_init(&accl_empty[i], 128);
+      mbar_init(&p_ready[i], 4);
+      mbar_init(&pe_done[i], 1);
+      mbar_init(&xfull[i], 128);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tek);
+    prefetch_tmap(&tem);
+    prefetch_tmap(&tx);
+    if (a.given) prefetch_tmap(&tp);
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  pdl_trigger();
+  pdl_wait();
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer: L(0), L(1), PE(0), L(2), PE(1), ..., PE(nt - 1)
+    // E tiles are read twice (L from HBM, PE about two tiles later): the first read asks L2
+    // to keep the lines, the second lets them go; x is read for every tile and kept.
+    const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    auto next_stage = [&]() -> uint8_t* {
+      if (!mbar_wait(&empty[stage], phase ^ 1, a.err)) { ok = false; return nullptr; }
+      return ring + stage * kLmStageBytes;
+    };
+    auto advance = [&]() { if (++stage == kLmStages) { stage = 0; phase ^= 1; } };
+    auto load_l = [&](int i) {
+      const int tile = tb + i;
+      for (int kb = 0; kb < KB && ok; ++kb) {
+        uint8_t* st = next_stage();
+        if (!ok) break;
+        mbar_arrive_expect_tx(&full[stage], 16384 + 8192);
+        tma_load_2d_hint(st, &tek, &full[stage], d0 + kb * 64, tile * 128, keep);
+        tma_load_2d_hint(st + 16384, &tx, &full[stage], d0 + kb * 64, 0, keep);
+        advance();
+      }
+    };
+    auto load_pe = [&](int i) {
+      const int tile = tb + i;
+      for (int ch = 0; ch < CH && ok; ++ch)
+        for (int vh = 0; vh < 2 && ok; ++vh) {
+          uint8_t* st = next_stage();
+          if (!ok) break;
+          mbar_arrive_expect_tx(&full[stage], 16384 + (a.given ? 4096 : 0));
+          tma_load_2d_hint(st, &tem, &full[stage], d0 + ch * 128, tile * 128 + vh * 64, drop);
+          tma_load_2d_hint(st + 8192, &tem, &full[stage], d0 + ch * 128 + 64, tile * 128 + vh * 64, drop);
+          if (a.given) tma_load_2d_hint(st + 16384, &tp, &full[stage], tile * 128 + vh * 64, 0, drop);
+          advance();
+        }
+    };
+    for (int i = 0; i < nt && ok; ++i) {
+      load_l(i);
+      if (i >= 1) load_pe(i - 1);
+    }
+    if (ok && nt > 0) load_pe(nt - 1);
+    // no copies left in flight: wait for the stages still owned by the MMA warp
+    for (int i = 0; i < kLmStages && ok; ++i) {
+      if (!mbar_wait(&empty[stage], phase ^ 1, a.err)) break;
+      advance();
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer (same order as the producer)
+    const uint32_t idesc_l = idesc_bf16(128, kLmT, false, false);
+    const uint32_t idesc_pe = idesc_bf16(128, kLmT, true, false);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    auto mma_l = [&](int i) {
+      const int b = i & 1;
+      if (!mbar_wait(&accl_empty[b], ((i >> 1) & 1) ^ 1, a.err)) { ok = false; return; }
+      tc_fence_after();
+      const uint32_t dl = tmem + b * kLmT;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&full[stage], phase, a.err)) { ok = false; return; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(ring + stage * kLmStageBytes), sx = sa + 16384;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)  // x = hi + lo: rows 0..31 and 32..63 of the x box
+            mma_bf16(dl, sw128_desc(sa + k * 32, 16, 1024), sw128_desc(sx + h * 4096 + k * 32, 16, 1024),
+                     idesc_l, (kb | k | h) ? 1u : 0u);
+        mma_commit(&empty[stage]);
+        if (++stage == kLmStages) { stage = 0; phase ^= 1; }
+      }
+      mma_commit(&accl_full[b]);
+    };
+    auto mma_pe = [&](int i) {
+      const int b = i & 1;
+      if (!mbar_wait(&p_ready[b], (i >> 1) & 1, a.err)) { ok = false; return; }
+      tc_fence_after();
+      const uint32_t pb = smem_u32(pbuf + b * kLmPBytes);
+      for (int ch = 0; ch < CH; ++ch) {
+        const uint32_t ds = tmem + kLmSCol + ch * kLmT;
+        for (int vh = 0; vh < 2; ++vh) {
+          if (!mbar_wait(&full[stage], phase, a.err)) { ok = false; return; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(ring + stage * kLmStageBytes);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = sw128_desc(sa + k * 2048, 8192, 1024);  // E^T: 16 vocab rows per step
+            const bool first = (i == 0 && vh == 0 && k == 0);
+            if (a.given) {
+              mma_bf16(ds, ad, sw128_desc(sa + 16384 + k * 32, 16, 1024), idesc_pe, first ? 0u : 1u);
+            } else {
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                mma_bf16(ds, ad, sw128_desc(pb + vh * 8192 + h * 4096 + k * 32, 16, 1024), idesc_pe,
+                         (first && h == 0) ? 0u : 1u);
+            }
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == kLmStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      mma_commit(&pe_done[b]);
+    };
+    for (int i = 0; i < nt && ok; ++i) {
+      mma_l(i);
+      if (ok && i >= 1) mma_pe(i - 1);
+    }
+    if (ok && nt > 0) mma_pe(nt - 1);
+    mma_commit(mma_done);
+    mbar_wait(mma_done, 0, a.err);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: exchange, statistics, P, rescale, outputs
+    const int et = threadIdx.x - 64;        // 0..127
+    const int q = warp % 4, row = q * 32 + lane;   // TMEM lane of this thread
+    const int tw = et / 32;                  // tokens 8 tw .. 8 tw + 7 in the transposed phase
+    float ref[8], Z[8], A[8], mbest[8];
+    int arg[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { ref[j] = -INFINITY; Z[j] = 0.f; A[j] = 0.f; mbest[j] = -INFINITY; arg[j] = 0x7fffffff; }
+    const uint32_t theirs_peer = map_peer(smem_u32(theirs), peer);
+    const uint32_t xfull_peer = map_peer(smem_u32(xfull), peer);
+    bool ok = true;
+    for (int i = 0; i < nt && ok; ++i) {
+      const int b = i & 1, tile = tb + i;
+      // 1. this CTA's partial logits of vocabulary row `row`, 32 tokens
+      if (et == 0) *flag = mbar_wait(&accl_full[b], (i >> 1) & 1, a.err) ? 1 : 0;
+      epi_bar();
+      ok = *flag != 0;
+      epi_bar();
+      if (!ok) break;
+      tc_fence_after();
+      float lp[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * kLmT, lp);
+      tc_fence_before();
+      mbar_arrive(&accl_empty[b]);
+      // 2. swap with the peer: own copy locally, the peer's copy by remote stores
+      float* mb = mine + b * kLmT * 128;
+      const uint32_t tpeer = theirs_peer + (uint32_t)(b * kLmT * 128 * 4);
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        mb[t * 128 + row] = lp[t];
+        st_cluster_f32(tpeer + (uint32_t)((t * 128 + row) * 4), lp[t]);
+      }
+      mbar_arrive_remote(xfull_peer + b * 8);
+      // every thread acquires the peer's tile itself; the barrier also publishes the local
+      // partial writes to the transposed reads
+      if (epi_any(!mbar_wait_cluster(&xfull[b], (i >> 1) & 1, a.err))) { ok = false; break; }
+      // 3. per-token statistics over the tile: warp tw, tokens 8 tw + j, lane: vocab 4 lane .. +3
+      const float* tb_ = theirs + b * kLmT * 128;
+      int need = 0;
+      float pv[8][4];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int t = tw * 8 + j;
+        const float4 x0 = *reinterpret_cast<const float4*>(mb + t * 128 + lane * 4);
+        const float4 x1 = *reinterpret_cast<const float4*>(tb_ + t * 128 + lane * 4);
+        float l[4] = {x0.x + x1.x, x0.y + x1.y, x0.z + x1.z, x0.w + x1.w};
+        float mx = -INFINITY;
+        int ax = 0x7fffffff;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int v = tile * 128 + lane * 4 + u;
+          if (v >= a.V || v == a.mask_id) l[u] = -INFINITY;
+          if (l[u] > mx) { mx = l[u]; ax = v; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float m2 = __shfl_xor_sync(0xffffffffu, mx, o);
+          const int a2 = __shfl_xor_sync(0xffffffffu, ax, o);
+          if (m2 > mx || (m2 == mx && a2 < ax)) { mx = m2; ax = a2; }
+        }
+        if (mx > mbest[j]) { mbest[j] = mx; arg[j] = ax; }
+        float f = 1.f;
+        if (i == 0) {
+          ref[j] = mx;
+        } else if (mx > ref[j] + kLmRescale) {
+          f = expf(ref[j] - mx);
+          ref[j] = mx;
+          Z[j] *= f;
+          A[j] *= f;
+          need = 1;
+        }
+        if (lane == 0) fac[t] = f;
+        float zs = 0.f, as = 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float p = (l[u] == -INFINITY) ? 0.f : expf(l[u] - ref[j]);
+          pv[j][u] = p;
+          zs += p;
+          as += (p > 0.f) ? p * l[u] : 0.f;
+        }
+        Z[j] += warp_sum(zs);
+        A[j] += warp_sum(as);
+      }
+      // 4. P(i) goes into pbuf[b]: PE(i - 2) must be done with it; a rescale also needs
+      //    PE(i - 1) done (s final up to tile i - 1).  With a given P nothing is written or
+      //    rescaled, but PE(i) still waits for this point, which keeps the MMA warp at most
+      //    one PE ahead of these waits.
+      const bool rescale = !a.given && epi_any(need != 0);  // also publishes fac[]
+      bool fail = false;
+      if (rescale && i >= 1) fail = !mbar_wait(&pe_done[(i - 1) & 1], ((i - 1) >> 1) & 1, a.err);
+      else if (i >= 2) fail = !mbar_wait(&pe_done[b], ((i - 2) >> 1) & 1, a.err);
+      if (epi_any(fail)) { ok = false; break; }
+      tc_fence_after();
+      if (rescale) {
+        float fv[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) fv[t] = fac[t];
+        for (int ch = 0; ch < CH; ++ch) {
+          float sv[32];
+          const uint32_t sa = tmem + ((uint32_t)(q * 32) << 16) + kLmSCol + ch * kLmT;
+          tmem_ld32(sa, sv);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) sv[t] *= fv[t];
+          tmem_st32_f(sa, sv);
+        }
+        tc_fence_before();
+      }
+      uint8_t* pt = pbuf + b * kLmPBytes;
+#pragma unroll
+      for (int j = 0; j < 8 && !a.given; ++j) {
+        const int t = tw * 8 + j;
+        const bool live = t < a.T;
+        __align__(8) __nv_bfloat16 hi[4], lo[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float p = live ? pv[j][u] : 0.f;
+          hi[u] = f2bf(p);
+          lo[u] = f2bf(p - bf2f(hi[u]));
+        }
+        *reinterpret_cast<uint2*>(pt + p_offset(t, lane * 4)) = *reinterpret_cast<const uint2*>(hi);
+        *reinterpret_cast<uint2*>(pt + p_offset(32 + t, lane * 4)) = *reinterpret_cast<const uint2*>(lo);
+      }
+      fence_proxy_async_smem();  // generic-proxy writes of P visible to the tensor cores
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready[b]);
+    }
+    // 5. outputs of the cluster: s half (every CTA), statistics (rank 0)
+    if (ok && nt > 0) {
+      const int last = nt - 1;
+      if (et == 0) *flag = mbar_wait(&pe_done[last & 1], (last >> 1) & 1, a.err) ? 1 : 0;
+      epi_bar();
+      ok = *flag != 0;
+      epi_bar();
+      if (ok) {
+        tc_fence_after();
+        for (int ch = 0; ch < CH; ++ch) {
+          float sv[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + kLmSCol + ch * kLmT, sv);
+          float4* dst = reinterpret_cast<float4*>(a.part_s + ((size_t)clu * a.d + d0 + ch * 128 + row) * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) dst[u] = make_float4(sv[4 * u], sv[4 * u + 1], sv[4 * u + 2], sv[4 * u + 3]);
+        }
+        if (rank == 0 && lane == 0) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int t = tw * 8 + j;
+            float* ps = a.part_stats + ((size_t)clu * 32 + t) * 4;
+            ps[0] = ref[j];
+            ps[1] = Z[j];
+            ps[2] = A[j];
+            ps[3] = mbest[j];
+            a.part_arg[(size_t)clu * 32 + t] = arg[j];
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer no longer writes into this CTA's shared memory
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// Merge of the clusters: for token t, M = max_c r_c, Z = sum_c Z_c e^(r_c - M), lse = M + ln Z,
+// maxprob = e^(max - lse), entropy = lse - A / Z, argmax from the first cluster holding the
+// max; s[t][f] = sum_c e^(r_c - M) s_c[f][t] / Z (given P: plain sum).  Clusters in
+// ascending order.  grid: d / 32 CTAs of 256 threads (8 warps x 32 features).
+__global__ void __launch_bounds__(256) k_lmf_combine(LmfArgs a, dlm_row_stats stats, float* s) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float w[64][33];     // per-cluster weights, clusters in chunks of 64
+  __shared__ float red[8][32][33];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int f = blockIdx.x * 32 + lane;
+  float acc[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) acc[t] = 0.f;
+  // token-wise reference and normaliser (thread t < 32 of warp 0 owns token t)
+  __shared__ float Mt[32], iZ[32];
+  if (threadIdx.x < 32) {
+    const int t = threadIdx.x;
+    float M = -INFINITY;
+    for (int c = 0; c < a.n_clu; ++c) M = fmaxf(M, a.part_stats[((size_t)c * 32 + t) * 4]);
+    float Zs = 0.f, As = 0.f, mx = -INFINITY;
+    int am = 0x7fffffff;
+    for (int c = 0; c < a.n_clu; ++c) {
+      const float* ps = a.part_stats + ((size_t)c * 32 + t) * 4;
+      const float e = expf(ps[0] - M);
+      Zs += ps[1] * e;
+      As += ps[2] * e;
+      if (ps[3] > mx) { mx = ps[3]; am = a.part_arg[(size_t)c * 32 + t]; }
+    }
+    Mt[t] = M;
+    iZ[t] = a.given ? 1.f : 1.f / Zs;
+    if (blockIdx.x == 0 && t < a.T) {
+      const float lse = M + logf(Zs);
+      stats.m[t] = mx;
+      stats.lse[t] = lse;
+      stats.maxprob[t] = expf(mx - lse);
+      stats.entropy[t] = lse - As / Zs;
+      stats.argmax[t] = am;
+    }
+  }
+  __syncthreads();
+  for (int c0 = 0; c0 < a.n_clu; c0 += 64) {
+    const int nc = a.n_clu - c0 < 64 ? a.n_clu - c0 : 64;
+    for (int i = threadIdx.x; i < nc * 32; i += blockDim.x) {
+      const int c = i / 32, t = i % 32;
+      w[c][t] = a.given ? 1.f : expf(a.part_stats[((size_t)(c0 + c) * 32 + t) * 4] - Mt[t]);
+    }
+    __syncthreads();
+    for (int c = warp; c < nc; c += 8) {
+      const float4* src = reinterpret_cast<const float4*>(a.part_s + ((size_t)(c0 + c) * a.d + f) * 32);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float4 x = __ldcg(src + u);
+        acc[4 * u] += w[c][4 * u] * x.x;
+        acc[4 * u + 1] += w[c][4 * u + 1] * x.y;
+        acc[4 * u + 2] += w[c][4 * u + 2] * x.z;
+        acc[4 * u + 3] += w[c][4 * u + 3] * x.w;
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int t = 0; t < 32; ++t) red[warp][lane][t] = acc[t];
+  __syncthreads();
+  // thread (warp, lane): token t = warp * 4 + (lane / 8), features lane % 8 .. in steps of 8
+  for (int i = threadIdx.x; i < 32 * 32; i += blockDim.x) {
+    const int t = i / 32, fl = i % 32;
+    if (t >= a.T) continue;
+    float v = 0.f;
+    for (int wv = 0; wv < 8; ++wv) v += red[wv][fl][t];  // warps in order
+    s[(size_t)t * a.d + blockIdx.x * 32 + fl] = v * iZ[t];
+  }
+}
+
+bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                    uint32_t box_outer, char* err, size_t errlen) {
+  return encode_tmap_2d(map, base, inner, outer, inner * 2, box_inner, box_outer, err, errlen);
+}
+
+}  // namespace
+
+size_t lmhead_fused_scratch_bytes(int V, int d) {
+  const int n_tiles = (V + 127) / 128;
+  const int n_clu = n_tiles < kSMs / 2 ? n_tiles : kSMs / 2;
+  return (size_t)n_clu * 32 * 4 * sizeof(float) + (size_t)n_clu * 32 * sizeof(int) +
+         (size_t)n_clu * d * 32 * sizeof(float) + 1024;
+}
+
+bool lmhead_fused_supported(int T, int d) {
+  return T >= 1 && T <= kLmT && d % 256 == 0 && d / 256 <= kLmMaxChunks;
+}
+
+// x2: split bf16 pair, rows [0, T) high halves and [32, 32 + T) low halves (pad = 32).
+cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_given, int T, int V, int d,
+                                int mask_id, dlm_row_stats stats, float* s, void* scratch, int* d_err,
+                                cudaStream_t st, char* err, size_t errlen) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_lmhead_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmSmem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  LmfArgs a{};
+  a.V = V;
+  a.d = d;
+  a.T = T;
+  a.mask_id = mask_id;
+  a.n_tiles = (V + 127) / 128;
+  a.n_clu = a.n_tiles < kSMs / 2 ? a.n_tiles : kSMs / 2;
+  a.given = p_given != nullptr;
+  uint8_t* sc = (uint8_t*)scratch;
+  a.part_stats = (float*)sc;
+  a.part_arg = (int*)(sc + (size_t)a.n_clu * 32 * 4 * sizeof(float));
+  a.part_s = (float*)(sc + (((size_t)a.n_clu * 32 * 5 * 4 + 255) & ~(size_t)255));
+  a.err = d_err;
+  CUtensorMap tek, tem, tx, tp;
+  if (!encode_bf16_2d(&tek, E, d, V, 64, 128, err, errlen) || !encode_bf16_2d(&tem, E, d, V, 64, 64, err, errlen) ||
+      !encode_bf16_2d(&tx, x2, d, 64, 64, 64, err, errlen))
+    return cudaErrorInvalidValue;
+  if (p_given) {
+    if (!encode_bf16_2d(&tp, p_given, V, T, 64, 32, err, errlen)) return cudaErrorInvalidValue;
+  } else {
+    tp = tx;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * a.n_clu);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = kLmSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = g_pdl ? 2 : 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_lmhead_fused, tek, tem, tx, tp, a);
+  if (e != cudaSuccess) return e;
+  return launch_k(k_lmf_combine, dim3(d / 32), dim3(256), 0, st, a, stats, s);
+}
+
+}  // namespace dlm

@@ -150,6 +150,52 @@ def test_lmhead_one_hot_p_reproduces_rows_exactly(lib):
     np.testing.assert_array_equal(s[1], bf16_f64(Eb)[1000])
 
 
+def _rescale_case(B, V, d):
+    """x = token-dependent mix of features 0 and 1 only, so the logits are set by E[:, 0:2]:
+    N(0, 1) plus a +9 bump in the last tile of each multi-tile cluster range, so those
+    clusters raise their reference and rescale (the bump exceeds the first tile's max by
+    more than 8) with about 5 % of the mass from before the bump: a wrong rescale factor
+    is visible at the 2e-2 tolerance."""
+    E = gen.normal_np(31, V * d, 0.1).reshape(V, d)
+    E[:, 0] = gen.normal_np(32, V, 1.0)
+    E[:, 1] = gen.normal_np(33, V, 0.5)
+    # the bump goes into the last vocabulary tile of every multi-tile range of the fused
+    # kernel's schedule (contiguous tile ranges over min(tiles, 74) clusters)
+    n_tiles = (V + 127) // 128
+    n_clu = min(n_tiles, 74)
+    for c in range(n_clu):
+        tb, te = c * n_tiles // n_clu, (c + 1) * n_tiles // n_clu
+        if te - tb >= 2 and (te - 1) * 128 + 5 < V:
+            E[(te - 1) * 128 + 5, 0] += 9.0
+    x = np.zeros((B, d))
+    x[:, 0] = 1.0
+    x[:, 1] = (np.arange(B) + 1) / 8.0
+    return gen.bf16_bits(x), gen.bf16_bits(E)
+
+
+@pytest.mark.parametrize("B,V,d,mask", [(5, 20000, 512, 19999), (32, 20000, 256, -1), (1, 3000, 768, 7)])
+def test_lmhead_fused_rescale_and_ragged(lib, B, V, d, mask):
+    """The fused single-pass LM head (d % 256 == 0, B <= 32): reference raised inside a
+    cluster, a ragged last vocabulary tile, B < 32, mask exclusion."""
+    xb, Eb = _rescale_case(B, V, d)
+    st = lib.lmhead_rowstats(to_torch_bf16(xb), to_torch_bf16(Eb), mask_id=mask)
+    ref = O.lmhead(bf16_f64(xb), Eb, mask_id=mask, want_logits=True)
+    _check_stats(st, ref, "fused lmhead", ref["logits"])
+    assert_close(st["s"].cpu().numpy(), ref["s"], RTOL_BF16, "fused s")
+
+
+def test_lmhead_fused_given_p_multi_tile(lib):
+    B, V, d = 7, 20000, 512
+    xb = _bits(41, (B, d))
+    Eb = _bits(42, (V, d), 0.1)
+    z = np.exp(gen.normal_np(43, B * V, 3.0).reshape(B, V))
+    Pb = gen.bf16_bits(z / z.sum(1, keepdims=True))
+    st = lib.lmhead_rowstats(to_torch_bf16(xb), to_torch_bf16(Eb), mask_id=V - 1, p_given=to_torch_bf16(Pb))
+    ref = O.lmhead(bf16_f64(xb), Eb, mask_id=V - 1, p_given=bf16_f64(Pb), want_logits=True)
+    _check_stats(st, ref, "fused lmhead given P", ref["logits"])
+    assert_close(st["s"].cpu().numpy(), ref["s"], RTOL_BF16, "fused s = P E")
+
+
 def test_lmhead_single_round_4b_shapes(lib):
     """Single round at 4B-class shapes: B=32, d=2560, V=151936, P_prev given."""
     import torch
