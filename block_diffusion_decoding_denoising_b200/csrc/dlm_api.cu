@@ -328,7 +328,7 @@ struct FwdSpec {
   float* s_out;
 };
 
-// h update + RMSNorm into the split GEMM input xn, one CTA per token (see k_resid_norm).
+// h update + RMSNorm into the split GEMM input xn, a 4-CTA cluster per token (see k_resid_norm).
 dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_tokens, const void* gain) {
   dlm_ctx* ctx = r.ctx;
   const dlm_config& c = ctx->cfg;
@@ -344,8 +344,7 @@ dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_t
   a.xn_lo = (long)split_pad(T) * c.d;
   a.d = c.d;
   a.eps = c.rms_eps;
-  const int threads = c.d > 1024 ? 1024 : (c.d > 256 ? 256 : 64);  // d <= 4 * threads
-  CU_LAUNCH(launch_k(k_resid_norm, dim3(T), dim3(threads), 0, r.s, a));
+  CU_LAUNCH(launch_k_cluster(k_resid_norm, dim3(T * kRnCluster), dim3(256), 0, r.s, kRnCluster, a));
   return DLM_OK;
 }
 

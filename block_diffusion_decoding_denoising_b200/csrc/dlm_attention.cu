@@ -22,7 +22,7 @@ namespace dlm {
 
 constexpr int kAttnRows = 64;   // query rows per CTA
 constexpr int kAttnKeys = 64;   // keys per tile
-constexpr int kMinKeysPerSplit = 256;
+constexpr int kMinKeysPerSplit = 128;
 
 template <int HD>
 struct AttnSmem {
@@ -336,7 +336,7 @@ int attention_max_splits(int T, int Hq, int Hkv, int max_ctx) {
   const int G = Hq / Hkv;
   const int qtiles = (T * G + kAttnRows - 1) / kAttnRows;
   int ctas = qtiles * Hkv;
-  int s = (kSMs + ctas - 1) / ctas;  // enough splits to cover the SMs once
+  int s = (2 * kSMs + ctas - 1) / ctas;  // enough splits for two CTAs per SM (each CTA is latency-bound)
   int by_len = (max_ctx + T + kMinKeysPerSplit - 1) / kMinKeysPerSplit;
   if (s > by_len) s = by_len;
   if (s < 1) s = 1;

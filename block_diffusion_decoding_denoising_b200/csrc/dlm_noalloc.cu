@@ -26,7 +26,7 @@
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
 constexpr size_t kNoAllocStatusBytes = 256;                // status word, padded
 constexpr int kNoAllocMaxDevices = 64;
 

@@ -151,26 +151,33 @@ __global__ void __launch_bounds__(256) k_finish_store(FinishArgs a) {
   }
 }
 
-// Residual update and RMSNorm of one token row (one CTA per token):
+// Residual update and RMSNorm of one token row, spread over a cluster of kRnCluster CTAs:
 //   h[t] = h[t] + y[t]        (residual of a projection whose partial sums are in `out`)
 //   h[t] = E[tok_t] + y[t]    (embedding, with y = W_a s, or y = 0 when out.partial is null)
 //   xn[t] = h[t] / sqrt(mean(h[t]^2) + eps) * g   as a split bf16 pair.
-// Each thread owns features threadIdx.x + k * blockDim.x, k < kFeat, and issues the loads
-// of all their slots (up to kSlotsReg each) before summing them in slot order.
+// CTA rank r of token t's cluster owns features [r d/4, (r + 1) d/4); each of its 256
+// threads owns features r d/4 + threadIdx.x + k 256 (k < kFeat) and issues the loads of all
+// their slots (up to kSlotsReg each) before summing them in slot order.  The four partial
+// sums of squares are exchanged through distributed shared memory and added in rank order.
+constexpr int kRnThreads = 256;
 constexpr int kFeat = 4;
 constexpr int kSlotsReg = 12;
-__global__ void __launch_bounds__(1024) k_resid_norm(ResNormArgs a) {
+__global__ void __launch_bounds__(kRnThreads) k_resid_norm(ResNormArgs a) {
   pdl_trigger();
   pdl_wait();
-  __shared__ float red[32];
-  __shared__ int nsl[64];
-  const int t = blockIdx.x;
+  __shared__ float red[kRnThreads / 32];
+  __shared__ float ss_all[kRnCluster];
+  __shared__ int nsl[16];
+  const int t = blockIdx.x / kRnCluster;
+  uint32_t rank;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+  const int dq = a.d / kRnCluster, f0 = (int)rank * dq;
   const GemmOut& o = a.out;
   const bool has_y = o.partial != nullptr;
-  const int TP = (o.T + 31) / 32 * 32;
-  const size_t st = (size_t)TP * kTileM;
-  if (has_y)
-    for (int i = threadIdx.x; i < o.n_tiles; i += blockDim.x) nsl[i] = tile_slots(o, i);
+  const uint32_t TP = (uint32_t)(o.T + 31) / 32 * 32;
+  const uint32_t st = TP * kTileM;
+  const int tile0 = f0 >> 7, ntl = ((f0 + dq - 1) >> 7) - tile0 + 1;  // tiles of this CTA's features
+  if (has_y && (int)threadIdx.x < ntl) nsl[threadIdx.x] = tile_slots(o, tile0 + threadIdx.x);
   __syncthreads();
   const int tok = a.embed ? a.tokens[t] : 0;
   float base[kFeat], x[kFeat][kSlotsReg];
@@ -178,9 +185,9 @@ __global__ void __launch_bounds__(1024) k_resid_norm(ResNormArgs a) {
   const float* pp[kFeat];
 #pragma unroll
   for (int k = 0; k < kFeat; ++k) {
-    const int n = threadIdx.x + k * blockDim.x;
-    const bool ok = n < a.d;
-    ns[k] = (ok && has_y) ? nsl[n >> 7] : 0;
+    const int n = f0 + threadIdx.x + k * kRnThreads;
+    const bool ok = (int)threadIdx.x + k * kRnThreads < dq;
+    ns[k] = (ok && has_y) ? nsl[(n >> 7) - tile0] : 0;
     pp[k] = has_y ? o.partial + ((size_t)(n >> 7) * o.max_slots * TP + t) * kTileM + (n & 127) : nullptr;
     base[k] = !ok ? 0.f : (a.embed ? bf2f(a.embed[(size_t)tok * a.d + n]) * a.embed_scale : a.h[(size_t)t * a.d + n]);
 #pragma unroll
@@ -195,18 +202,28 @@ __global__ void __launch_bounds__(1024) k_resid_norm(ResNormArgs a) {
     for (int sl = 0; sl < kSlotsReg; ++sl) y += x[k][sl];  // slot order
     for (int sl = kSlotsReg; sl < ns[k]; ++sl) y += __ldcg(pp[k] + sl * st);
     hv[k] = base[k] + y;
-    const int n = threadIdx.x + k * blockDim.x;
-    if (n < a.d) {
+    const int n = f0 + threadIdx.x + k * kRnThreads;
+    if ((int)threadIdx.x + k * kRnThreads < dq) {
       a.h[(size_t)t * a.d + n] = hv[k];
       ss += hv[k] * hv[k];
     }
   }
   ss = block_sum(ss, red);
-  const float r = 1.0f / sqrtf(ss / (float)a.d + a.eps);
+  if (threadIdx.x < kRnCluster) {
+    // this CTA's partial into slot `rank` of every CTA of the cluster (itself included)
+    uint32_t dst;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(dst) : "r"(smem_u32(&ss_all[rank])), "r"((uint32_t)threadIdx.x));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dst), "f"(ss) : "memory");
+  }
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  float tot = 0.f;
+#pragma unroll
+  for (int q = 0; q < kRnCluster; ++q) tot += ss_all[q];  // rank order: the same sum everywhere
+  const float r = 1.0f / sqrtf(tot / (float)a.d + a.eps);
 #pragma unroll
   for (int k = 0; k < kFeat; ++k) {
-    const int n = threadIdx.x + k * blockDim.x;
-    if (n < a.d) store_split(a.xn + (size_t)t * a.d + n, a.xn_lo, hv[k] * r * bf2f(a.gain[n]));
+    const int n = f0 + threadIdx.x + k * kRnThreads;
+    if ((int)threadIdx.x + k * kRnThreads < dq) store_split(a.xn + (size_t)t * a.d + n, a.xn_lo, hv[k] * r * bf2f(a.gain[n]));
   }
 }
 

@@ -14,6 +14,8 @@ struct FinishArgs {
   int N;         // valid output features
 };
 
+constexpr int kRnCluster = 4;  // CTAs per token of k_resid_norm (a thread-block cluster)
+
 struct ResNormArgs {
   GemmOut out;                 // partial sums of a GEMM with N = d (partial == nullptr: y = 0)
   float* h;                    // [T][d] residual stream

@@ -235,10 +235,10 @@ dlm_status dlm_bd_attention(const void* d_q, const void* d_k_cache, const void* 
 /* The same attention with no scratch argument, for callers that cannot give the library
  * device memory beyond the operands (nothing is allocated by the call).  The pages have no
  * counterpart: it is an interface variant of dlm_bd_attention.  Its split-KV partials live
- * in a fixed 8 MiB array of static device memory per device; calls whose partials
+ * in a fixed 16 MiB array of static device memory per device; calls whose partials
  * (split count x T x Hq x (hd + 2) x 4 bytes, the split count as dlm_bd_attention picks it
- * from T, Hq, Hkv and max_ctx) exceed 8 MiB - 256 B are rejected with DLM_ENOMEM_WS.  The
- * 4B-class shapes (T <= 64, 32/8 heads, hd 128) need at most 5.6 MB.  The first call on a
+ * from T, Hq, Hkv and max_ctx) exceed 16 MiB - 256 B are rejected with DLM_ENOMEM_WS.  The
+ * 4B-class shapes (T <= 64, 32/8 heads, hd 128) need at most 10.7 MB.  The first call on a
  * device looks the array up and sets kernel attributes: make it before starting any stream
  * capture on that device.  Every call clears the array's status word on `stream`.  The
  * array is shared: calls that may overlap in time race on it and must be serialised by the
