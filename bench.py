@@ -180,6 +180,114 @@ def reference_arm(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+def nvfp4_measure(args, cfg, w, prompt, dev, stream):
+    """Decode tokens/s with the MLP and E in NVFP4 (same schedule as the main line), and
+    the NVFP4 GEMM's bandwidth on the gate (9728 x 2560) and down (2560 x 9728) shapes."""
+    import torch
+
+    from block_diffusion_decoding_denoising_b200 import dlm
+    c5 = dict(cfg)
+    c5["weight_fmt"] = dlm.WEIGHTS_NVFP4
+    wq = dlm.quantize_model(w)
+    m = dlm.Model(c5, wq, device=dev)
+    B = c5["block_size"]
+    blocks = GEN // B
+    tok = torch.zeros((blocks, B), dtype=torch.int32, device=dev)
+    rr = torch.zeros((blocks, 2), dtype=torch.int32, device=dev)
+    m.prefill(prompt)
+
+    def step():
+        m.set_prefix_len(PROMPT)
+        for b in range(blocks):
+            m.decode_block(TAU, dlm.COMMIT_TOPK, TPF_K, tok[b], rr[b])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert int(rr[:, 1].abs().sum().item()) == 0, "device status"
+    ms = e0.elapsed_time(e1) / args.steps
+    rounds = int(rr[:, 0].sum().item())
+    m.close()
+    # the GEMM alone
+    out = {"tokens_per_s": GEN / (ms / 1e3), "ms_per_step": ms, "rounds_per_step": rounds}
+    L = dlm.lib()
+    import ctypes as C
+    sp = C.c_void_p(stream.cuda_stream)
+    gb = []
+    for q, K in ((wq["layers"][0]["q_gate"], cfg["d"]), (wq["layers"][0]["q_down"], cfg["ffn"])):
+        x = torch.randn((B, K), device=dev)
+        n = L.dlm_gemm_nvfp4_scratch_size(B, q["rows"], K)
+        sc = torch.empty(n, dtype=torch.uint8, device=dev)
+        qm = dlm._q_matrix(q)
+        call = lambda: L.dlm_gemm_nvfp4(C.c_void_p(x.data_ptr()), C.byref(qm), None, B, q["rows"], K,
+                                        C.c_void_p(sc.data_ptr()), n, sp)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        g0.record(stream)
+        for _ in range(reps):
+            call()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        us = g0.elapsed_time(g1) * 1e3 / reps
+        nbytes = q["rows"] * K * 0.5625 + B * K * 2
+        gb.append({"shape": "%dx%d" % (q["rows"], K), "us": us, "GBs": nbytes / (us * 1e-6) / 1e9})
+    hbm, _, kind = peaks()
+    out["gemm"] = gb
+    out["gemm_frac"] = max(g["GBs"] for g in gb) / hbm
+    round_bytes = 3.632e9
+    out["round_ms"] = ms / (rounds + blocks)
+    out["round_roofline_frac"] = round_bytes / (out["round_ms"] / 1e3) / 1e9 / hbm
+    return out
+
+
+def lmhead_measure(args, w, dev):
+    """The fused LM head (row statistics and s = P E in one pass over E) on the model's E."""
+    import torch
+
+    from block_diffusion_decoding_denoising_b200 import dlm
+    E = w["embed"]
+    V, d = E.shape
+    B = 32
+    x = torch.randn((B, d), device=dev).to(torch.bfloat16)
+    for _ in range(2):
+        dlm.lmhead_rowstats(x, E, mask_id=V - 1)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 5
+    e0.record()
+    for _ in range(reps):
+        dlm.lmhead_rowstats(x, E, mask_id=V - 1)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    hbm, _, kind = peaks()
+    gbs = V * d * 2 / (us * 1e-6) / 1e9
+    return {"us_per_call": us, "algorithmic_bytes": V * d * 2, "GBs": gbs, "frac": gbs / hbm,
+            "note": "E read once is the algorithmic figure; the kernel re-reads each E tile for P E (L2 or DRAM)"}
+
+
+def profile_traffic(name):
+    """DRAM bytes per launch (read + write) from the committed ncu summary of that kernel
+    (a line 'dram_bytes_per_launch: N'), or None."""
+    p = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", name)
+    try:
+        for line in open(p):
+            if line.startswith("dram_bytes_per_launch:"):
+                return float(line.split(":")[1])
+    except OSError:
+        pass
+    return None
+
+
 def workload_config(cfg):
     return {"workload": "full bs=1 decode, 4B-class dense model (36L d2560 GQA32/8 hd128 F9728 V151936 bf16), "
                         "prompt 512, generate 4096 in blocks of 32, fixed TPF=11",
@@ -226,6 +334,21 @@ def gemm_case(args):
             torch.cuda.synchronize()
             key = "%s %dx%d" % (mode, t.shape[0], K)
             times[key] = round(ev[0].elapsed_time(ev[1]) * 1e3 / args.steps, 2)
+    # the NVFP4 GEMM on the gate shape (layer 0's weight quantized on the device)
+    q = dlm.nvfp4_matrix(w["layers"][0]["w_gate"])
+    xf = torch.randn((B, cfg["d"]), device="cuda")
+    nq = L.dlm_gemm_nvfp4_scratch_size(B, q["rows"], cfg["d"])
+    scq = torch.empty(nq, dtype=torch.uint8, device="cuda")
+    qm = dlm._q_matrix(q)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(args.steps):
+        st = L.dlm_gemm_nvfp4(C.c_void_p(xf.data_ptr()), C.byref(qm), None, B, q["rows"], cfg["d"],
+                              C.c_void_p(scq.data_ptr()), nq, s)
+        assert st == 0, st
+    ev[1].record()
+    torch.cuda.synchronize()
+    times["nvfp4 partial %dx%d" % (q["rows"], cfg["d"])] = round(ev[0].elapsed_time(ev[1]) * 1e3 / args.steps, 2)
     print(json.dumps({"case": "gemm", "us_per_launch": times}))
 
 
@@ -400,9 +523,27 @@ def main():
     g1.record(stream)
     torch.cuda.synchronize()
     gemm_s = g0.elapsed_time(g1) / 1e3 / (reps * len(shapes))
-    gemm_bytes = sum(t.numel() * 2 + 2 * B * K * 2 for t, K in shapes) / len(shapes)
     hbm, tflops, peak_kind = peaks()
-    achieved = gemm_bytes / gemm_s / 1e9
+    # the roofline line: the gate projection (9728 x 2560), each layer's own weight in turn so
+    # that no launch finds its weights in L2, against the ncu capture of the same launch
+    gate = [(lw["w_gate"], cfg["d"]) for lw in w["layers"]]
+
+    def gates():
+        for t, K in gate:
+            L.dlm_gemm_bf16x2(C.c_void_p(x.data_ptr()), C.c_void_p(t.data_ptr()), None, B, t.shape[0], K,
+                              C.c_void_p(scratch.data_ptr()), scratch_n, sp)
+
+    gates()
+    torch.cuda.synchronize()
+    g0.record(stream)
+    for _ in range(reps):
+        gates()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    gate_s = g0.elapsed_time(g1) / 1e3 / (reps * len(gate))
+    gate_bytes = cfg["ffn"] * cfg["d"] * 2 + 2 * B * cfg["d"] * 2
+    achieved = gate_bytes / gate_s / 1e9
+    gemm_avg_gbs = sum(t.numel() * 2 + 2 * B * K * 2 for t, K in shapes) / len(shapes) / gemm_s / 1e9
 
     # end to end through dlm_generate: pinned host prompt in, every block's tokens out
     pin_prompt = torch.from_numpy(prompt_np).pin_memory()
@@ -427,6 +568,13 @@ def main():
     round_bytes = weight_bytes + 147456 * mean_L * cfg["n_layers"] / 36
     round_ms = ms_step / (rounds_per_step + blocks)  # rounds and KV-fill forwards of the step
 
+    # NVFP4 weights (MLP and E; attention bf16): the same decode, and the NVFP4 GEMM alone
+    # on the MLP shapes (partial sums only, inputs quantized per row)
+    m.close()
+    nv = nvfp4_measure(args, cfg, w, prompt, dev, stream)
+    # the fused LM head alone (LM-head configuration shapes: B 32, d 2560, V 151936, P = softmax)
+    lm = lmhead_measure(args, w, dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_round, reps_cpu, thr = oracle_sample(cfg, 10.0)
@@ -440,9 +588,11 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(cfg),
-            "roofline": {"bound": "hbm", "kernel": "k_gemm_tc (tensor-core weight-streaming GEMM)",
+            "roofline": {"bound": "hbm", "kernel": "k_gemm_tc: 9728x2560 bf16 weight GEMM, 32 tokens as a split "
+                                                     "bf16 pair (the gate projection), partial sums",
                          "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                         "peak_kind": peak_kind, "traffic": None},
+                         "peak_kind": peak_kind, "traffic": profile_traffic("k_gemm_tc_9728x2560_t32.md"),
+                         "algorithmic_bytes": gate_bytes, "launch_us": gate_s * 1e6},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_tps, "unit": "tokens/s", "h2d_bytes_per_step": PROMPT * 4,
                     "d2h_bytes_per_step": GEN * 4 + blocks * 8},
@@ -452,10 +602,10 @@ def main():
                       "round_or_fill_ms": round_ms,
                       "round_roofline_frac": (round_bytes / (round_ms / 1e3) / 1e9) / hbm,
                       "tau0.9_rounds_per_s": tau_rounds_per_s, "tau0.9_rounds_per_block": tau_rounds / 4,
-                      "gemm_avg_launch_us": gemm_s * 1e6},
+                      "gemm_avg_launch_us": gemm_s * 1e6, "gemm_all_shapes_GBs": gemm_avg_gbs,
+                      "nvfp4": nv, "lmhead_fused": lm},
         }
         print(json.dumps(line), flush=True)
-    m.close()
     if world > 1:
         dist.destroy_process_group()
 

@@ -32,8 +32,9 @@ namespace {
 
 constexpr int kF4K = 256;            // reduction elements per stage (128 code bytes per row)
 constexpr int kSubs = kF4K / 64;     // 64-element sub-blocks per stage
-constexpr int kASlots = 4;           // decoded A sub-blocks resident in tensor memory
+constexpr int kASlots = 8;           // decoded A sub-blocks resident in tensor memory (two stages)
 constexpr int kACol = 128;           // first TMEM column of the A slots (32 columns each)
+static_assert(kASlots % kSubs == 0, "a stage's sub-blocks take consecutive slots");
 constexpr int kF4Threads = 320;
 
 template <int NT>
@@ -45,7 +46,7 @@ struct F4Cfg {
   static constexpr int kStageBytes = kCodeBytes + kBBytes + kScaleBytes;  // multiple of 1024
   static constexpr int kStages = NT <= 32 ? 6 : 4;
   static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 512 /*barriers*/;
-  static constexpr int kTmemCols = 256;             // 2 accumulators (<= 128) + A slots
+  static constexpr int kTmemCols = 512;             // 2 accumulators (<= 128) + A slots
 };
 
 struct F4KArgs {
@@ -275,6 +276,13 @@ k_gemm_fp4(const __grid_constant__ CUtensorMap tc0, const __grid_constant__ CUte
       for (int q = 0; q < 8; ++q)  // 16-byte chunk q of the row sits at chunk q ^ (row % 8)
         cw[q] = *reinterpret_cast<const uint4*>(base + row * 128 + ((q ^ (row & 7)) << 4));
       const uint4 scw = *reinterpret_cast<const uint4*>(base + Cfg::kCodeBytes + Cfg::kBBytes + row * 16);
+      // the stage's four slots (kASlots is a multiple of kSubs: they are consecutive)
+      const int slot0 = slot;
+      for (int j = 0; j < kSubs && ok; ++j)
+        if (!mbar_wait(&a_empty[slot0 + j], sphase ^ 1, args.err)) ok = false;
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
       for (int j = 0; j < kSubs; ++j) {
         // sub-block j: elements 64 j .. 64 j + 63 = code chunks 2j, 2j+1, scale bytes 4j .. 4j+3
         const uint32_t sw = (j == 0) ? scw.x : (j == 1) ? scw.y : (j == 2) ? scw.z : scw.w;
@@ -288,17 +296,17 @@ k_gemm_fp4(const __grid_constant__ CUtensorMap tc0, const __grid_constant__ CUte
           uint32_t h[4];
           e2m1x8_to_f16x2(words[w], h);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) r[4 * w + i] = hmul2_u32(h[i], sig[w / 2]);  // 8 elements per word pair -> 16 per scale
+          for (int i = 0; i < 4; ++i) r[4 * w + i] = hmul2_u32(h[i], sig[w / 2]);  // 16 elements per scale
         }
-        if (!mbar_wait(&a_empty[slot], sphase ^ 1, args.err)) { ok = false; break; }
-        tc_fence_after();
-        tmem_st32(lane_base + slot * 32, r);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[slot]);
-        if (++slot == kASlots) { slot = 0; sphase ^= 1; }
+        tmem_st32(lane_base + (slot0 + j) * 32, r);
       }
+      tmem_wait_st();  // one wait for the stage's four stores
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0)
+        for (int j = 0; j < kSubs; ++j) mbar_arrive(&a_full[slot0 + j]);
+      slot += kSubs;
+      if (slot == kASlots) { slot = 0; sphase ^= 1; }
       if (++stage == S) { stage = 0; phase ^= 1; }
     }
   } else if (warp >= 2) {

@@ -39,6 +39,7 @@ constexpr int kLmStageBytes = 24576;    // E box 16 KB + x box 8 KB (L) / 2 E bo
 constexpr int kLmPBytes = 16384;        // P tile: 64 rows (hi, lo) x 128 vocab, 2 swizzle atoms
 constexpr int kLmXBytes = kLmT * 128 * 4;  // one partial-logit tile [32][128] fp32
 constexpr int kLmMaxChunks = 14;        // d / 2 <= 1792
+constexpr int kLmMaxClusters = kSMs / 2;  // clusters of two CTAs
 constexpr int kLmSCol = 64;             // TMEM column of the first s accumulator
 constexpr float kLmRescale = 8.0f;      // raise the reference when a max exceeds it by this
 constexpr int kLmSmem = kLmStages * kLmStageBytes + 2 * kLmPBytes + 4 * kLmXBytes + 1024 + 1024;
@@ -465,70 +466,89 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
 }
 
 // Merge of the clusters: for token t, M = max_c r_c, Z = sum_c Z_c e^(r_c - M), lse = M + ln Z,
-// maxprob = e^(max - lse), entropy = lse - A / Z, argmax from the first cluster holding the
-// max; s[t][f] = sum_c e^(r_c - M) s_c[f][t] / Z (given P: plain sum).  Clusters in
-// ascending order.  grid: d / 32 CTAs of 256 threads (8 warps x 32 features).
+// maxprob = e^(max - lse), entropy = lse - A / Z, argmax from the lowest-index cluster holding
+// the max; s[t][f] = sum_c e^(r_c - M) s_c[f][t] / Z (given P: plain sum).  The per-token
+// reductions run over the lanes of a warp (a fixed shuffle tree), the s sums over the warps
+// of a CTA (each warp a fixed set of clusters, then the warps in order).
+// grid: d / 32 CTAs of 256 threads (8 warps x 32 features).
 __global__ void __launch_bounds__(256) k_lmf_combine(LmfArgs a, dlm_row_stats stats, float* s) {
   pdl_trigger();
   pdl_wait();
-  __shared__ float w[64][33];     // per-cluster weights, clusters in chunks of 64
+  __shared__ __align__(16) float w[kLmMaxClusters][32];  // per-cluster weight of each token
   __shared__ float red[8][32][33];
+  __shared__ float iZ[32];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // 1. per token: warp `warp` handles tokens warp, warp + 8, ...; lanes stride the clusters
+  for (int t = warp; t < 32; t += 8) {
+    float M = -INFINITY;
+    for (int c = lane; c < a.n_clu; c += 32) M = fmaxf(M, a.part_stats[((size_t)c * 32 + t) * 4]);
+    M = warp_max(M);
+    float zs = 0.f, as = 0.f, mx = -INFINITY;
+    int mc = 0x7fffffff;
+    for (int c = lane; c < a.n_clu; c += 32) {
+      const float4 ps = *reinterpret_cast<const float4*>(a.part_stats + ((size_t)c * 32 + t) * 4);
+      const float e = expf(ps.x - M);
+      w[c][t] = a.given ? 1.f : e;
+      zs += ps.y * e;
+      as += ps.z * e;
+      if (ps.w > mx) { mx = ps.w; mc = c; }  // clusters visited in increasing order
+    }
+    zs = warp_sum(zs);
+    as = warp_sum(as);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, mx, o);
+      const int c2 = __shfl_xor_sync(0xffffffffu, mc, o);
+      if (m2 > mx || (m2 == mx && c2 < mc)) { mx = m2; mc = c2; }
+    }
+    if (lane == 0) {
+      iZ[t] = a.given ? 1.f : 1.f / zs;
+      if (blockIdx.x == 0 && t < a.T) {
+        const float lse = M + logf(zs);
+        stats.m[t] = mx;
+        stats.lse[t] = lse;
+        stats.maxprob[t] = expf(mx - lse);
+        stats.entropy[t] = lse - as / zs;
+        stats.argmax[t] = a.part_arg[(size_t)mc * 32 + t];
+      }
+    }
+  }
+  __syncthreads();
+  // 2. s: lane = feature blockIdx.x * 32 + lane, warp = clusters warp, warp + 8, ...; the next
+  //    cluster's 128 bytes are loaded while the current one is accumulated
   const int f = blockIdx.x * 32 + lane;
   float acc[32];
 #pragma unroll
   for (int t = 0; t < 32; ++t) acc[t] = 0.f;
-  // token-wise reference and normaliser (thread t < 32 of warp 0 owns token t)
-  __shared__ float Mt[32], iZ[32];
-  if (threadIdx.x < 32) {
-    const int t = threadIdx.x;
-    float M = -INFINITY;
-    for (int c = 0; c < a.n_clu; ++c) M = fmaxf(M, a.part_stats[((size_t)c * 32 + t) * 4]);
-    float Zs = 0.f, As = 0.f, mx = -INFINITY;
-    int am = 0x7fffffff;
-    for (int c = 0; c < a.n_clu; ++c) {
-      const float* ps = a.part_stats + ((size_t)c * 32 + t) * 4;
-      const float e = expf(ps[0] - M);
-      Zs += ps[1] * e;
-      As += ps[2] * e;
-      if (ps[3] > mx) { mx = ps[3]; am = a.part_arg[(size_t)c * 32 + t]; }
-    }
-    Mt[t] = M;
-    iZ[t] = a.given ? 1.f : 1.f / Zs;
-    if (blockIdx.x == 0 && t < a.T) {
-      const float lse = M + logf(Zs);
-      stats.m[t] = mx;
-      stats.lse[t] = lse;
-      stats.maxprob[t] = expf(mx - lse);
-      stats.entropy[t] = lse - As / Zs;
-      stats.argmax[t] = am;
-    }
-  }
-  __syncthreads();
-  for (int c0 = 0; c0 < a.n_clu; c0 += 64) {
-    const int nc = a.n_clu - c0 < 64 ? a.n_clu - c0 : 64;
-    for (int i = threadIdx.x; i < nc * 32; i += blockDim.x) {
-      const int c = i / 32, t = i % 32;
-      w[c][t] = a.given ? 1.f : expf(a.part_stats[((size_t)(c0 + c) * 32 + t) * 4] - Mt[t]);
-    }
-    __syncthreads();
-    for (int c = warp; c < nc; c += 8) {
-      const float4* src = reinterpret_cast<const float4*>(a.part_s + ((size_t)(c0 + c) * a.d + f) * 32);
+  float4 cur[8], nxt[8];
+  int c = warp;
+  if (c < a.n_clu) {
+    const float4* src = reinterpret_cast<const float4*>(a.part_s + ((size_t)c * a.d + f) * 32);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float4 x = __ldcg(src + u);
-        acc[4 * u] += w[c][4 * u] * x.x;
-        acc[4 * u + 1] += w[c][4 * u + 1] * x.y;
-        acc[4 * u + 2] += w[c][4 * u + 2] * x.z;
-        acc[4 * u + 3] += w[c][4 * u + 3] * x.w;
-      }
+    for (int u = 0; u < 8; ++u) cur[u] = __ldcg(src + u);
+  }
+  for (; c < a.n_clu; c += 8) {
+    const int cn = c + 8;
+    if (cn < a.n_clu) {
+      const float4* src = reinterpret_cast<const float4*>(a.part_s + ((size_t)cn * a.d + f) * 32);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) nxt[u] = __ldcg(src + u);
     }
-    __syncthreads();
+    const float4* wc = reinterpret_cast<const float4*>(&w[c][0]);  // broadcast reads
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float4 wv = wc[u];
+      acc[4 * u] += wv.x * cur[u].x;
+      acc[4 * u + 1] += wv.y * cur[u].y;
+      acc[4 * u + 2] += wv.z * cur[u].z;
+      acc[4 * u + 3] += wv.w * cur[u].w;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) cur[u] = nxt[u];
   }
 #pragma unroll
   for (int t = 0; t < 32; ++t) red[warp][lane][t] = acc[t];
   __syncthreads();
-  // thread (warp, lane): token t = warp * 4 + (lane / 8), features lane % 8 .. in steps of 8
   for (int i = threadIdx.x; i < 32 * 32; i += blockDim.x) {
     const int t = i / 32, fl = i % 32;
     if (t >= a.T) continue;
@@ -547,7 +567,7 @@ bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t
 
 size_t lmhead_fused_scratch_bytes(int V, int d) {
   const int n_tiles = (V + 127) / 128;
-  const int n_clu = n_tiles < kSMs / 2 ? n_tiles : kSMs / 2;
+  const int n_clu = n_tiles < kLmMaxClusters ? n_tiles : kLmMaxClusters;
   return (size_t)n_clu * 32 * 4 * sizeof(float) + (size_t)n_clu * 32 * sizeof(int) +
          (size_t)n_clu * d * 32 * sizeof(float) + 1024;
 }
@@ -572,7 +592,7 @@ cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_giv
   a.T = T;
   a.mask_id = mask_id;
   a.n_tiles = (V + 127) / 128;
-  a.n_clu = a.n_tiles < kSMs / 2 ? a.n_tiles : kSMs / 2;
+  a.n_clu = a.n_tiles < kLmMaxClusters ? a.n_tiles : kLmMaxClusters;
   a.given = p_given != nullptr;
   uint8_t* sc = (uint8_t*)scratch;
   a.part_stats = (float*)sc;
