@@ -76,9 +76,12 @@ struct dlm_ctx {
   // (q sigma, exact; the tensor scale is applied where the rows are used)
   void* lmf = nullptr;  // scratch of the fused LM head (null: the unfused path is used)
   bool fp4 = false;
-  __half* xq = nullptr;
+  uint8_t* xcodes = nullptr;   // [32][max(d, F) / 2] e2m1 codes of the GEMM input
+  uint8_t* xscales = nullptr;  // e4m3 scales, tiled [max(d, F) / 64][32][16 B]
   float* sx = nullptr;
   __nv_bfloat16* e_deq = nullptr;
+  uint8_t* sf = nullptr;       // weight scales re-tiled for the FP4 MMA: per layer (gate/up, down), then E
+  size_t sf_pair = 0, sf_down = 0;
   // internal block state (graph path)
   int32_t* b_tokens = nullptr;
   uint8_t* b_committed = nullptr;
@@ -200,16 +203,27 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   int32_t* ot = cv.take<int32_t>(B);
   int32_t* orr = cv.take<int32_t>(4);
   const bool fp4 = c.weight_fmt == DLM_WEIGHTS_NVFP4;
-  __half* xq = fp4 ? cv.take<__half>((size_t)kMaxF4Tokens * (c.d > c.ffn ? c.d : c.ffn)) : nullptr;
+  const size_t kmax = c.d > c.ffn ? c.d : c.ffn;
+  uint8_t* xcodes = fp4 ? cv.take<uint8_t>((size_t)kMaxF4Tokens * kmax / 2) : nullptr;
+  uint8_t* xscales = fp4 ? cv.take<uint8_t>(kmax / 64 * 512) : nullptr;
   float* sx = fp4 ? cv.take<float>(kMaxF4Tokens) : nullptr;
   __nv_bfloat16* edq = fp4 ? cv.take<__nv_bfloat16>((size_t)c.vocab * c.d) : nullptr;
+  const bool fp4_shapes = fp4 && c.d % 256 == 0 && c.ffn % 256 == 0;
+  const size_t sfp = fp4_shapes ? align256(nvf4_sf_tile_bytes(c.ffn, c.d, A_PAIR)) : 0;
+  const size_t sfd = fp4_shapes ? align256(nvf4_sf_tile_bytes(c.d, c.ffn, A_KMAJOR)) : 0;
+  const size_t sfe = fp4_shapes ? align256(nvf4_sf_tile_bytes(c.vocab, c.d, A_KMAJOR)) : 0;
+  uint8_t* sf = fp4_shapes ? cv.take<uint8_t>((size_t)c.n_layers * (sfp + sfd) + sfe) : nullptr;
   const bool fused = !fp4 && lmhead_fused_supported(B, c.d);
   uint8_t* lmf = fused ? cv.take<uint8_t>(lmhead_fused_scratch_bytes(c.vocab, c.d)) : nullptr;
   if (x && base) {
     x->lmf = lmf;
     x->fp4 = fp4;
-    x->xq = xq;
+    x->xcodes = xcodes;
+    x->xscales = xscales;
     x->sx = sx;
+    x->sf = sf;
+    x->sf_pair = sfp;
+    x->sf_down = sfd;
     x->e_deq = edq;
     x->d_L = hdr;
     x->d_err = hdr + 1;
@@ -290,11 +304,13 @@ struct Runner {
     e.op = EPI_PARTIAL;
     return gemm(a_mode, a0, a1, x, T, N, K, e, out);
   }
-  // NVFP4 projection of the quantized activations in ctx->xq (see act_quant).
-  dlm_status gemm_fp4(int a_mode, const dlm_nvfp4_matrix& w0, const dlm_nvfp4_matrix* w1, int T, int N, int K,
-                      GemmOut* out) {
+  // NVFP4 projection of the quantized activations in ctx->xcodes / xscales (see act_quant);
+  // `sfa`: the weight's re-tiled scales.
+  dlm_status gemm_fp4(int a_mode, const dlm_nvfp4_matrix& w0, const dlm_nvfp4_matrix* w1, const uint8_t* sfa, int T,
+                      int N, int K, GemmOut* out) {
     GemmF4Plan p;
-    if (!gemm_fp4_plan(&p, a_mode, w0, w1, ctx->xq, kMaxF4Tokens, ctx->sx, T, N, K, ctx->partial, msg, sizeof(msg)))
+    if (!gemm_fp4_plan(&p, a_mode, w0, w1, sfa, ctx->xcodes, ctx->xscales, kMaxF4Tokens, ctx->sx, T, N, K,
+                       ctx->partial, msg, sizeof(msg)))
       return fail(ctx, DLM_EUNSUPPORTED, "%s", msg);
     if (p.partial_bytes > ctx->partial_bytes)
       return fail(ctx, DLM_ENOMEM_WS, "nvfp4 gemm partials %zu > %zu", p.partial_bytes, ctx->partial_bytes);
@@ -349,14 +365,15 @@ dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_t
 }
 
 // Quantizes the T rows of a split bf16 GEMM input (hi at x, lo at x + lo) to NVFP4 in
-// ctx->xq / ctx->sx (see k_act_quant).
+// ctx->xcodes / xscales / sx (see k_act_quant).
 dlm_status act_quant(Runner& r, int T, const __nv_bfloat16* x, long lo, int K) {
   dlm_ctx* ctx = r.ctx;
   ActQuantArgs a{};
   a.xb = x;
   a.xb_lo = lo;
   a.K = K;
-  a.xq = ctx->xq;
+  a.codes = ctx->xcodes;
+  a.scales = ctx->xscales;
   a.sx = ctx->sx;
   CU_LAUNCH(launch_k(k_act_quant, dim3(T), dim3(256), 0, r.s, a));
   return DLM_OK;
@@ -444,7 +461,7 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
 
     if (ctx->fp4) {
       TRY(act_quant(r, T, ctx->xn, pad * d, d));
-      TRY(r.gemm_fp4(A_PAIR, W.q_gate, &W.q_up, T, F, d, &y));
+      TRY(r.gemm_fp4(A_PAIR, W.q_gate, &W.q_up, ctx->sf + l * (ctx->sf_pair + ctx->sf_down), T, F, d, &y));
     } else {
       TRY(r.gemm_partial(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, &y));
     }
@@ -456,7 +473,8 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
 
     if (ctx->fp4) {
       TRY(act_quant(r, T, ctx->act, pad * F, F));
-      TRY(r.gemm_fp4(A_KMAJOR, W.q_down, nullptr, T, d, F, &y));
+      TRY(r.gemm_fp4(A_KMAJOR, W.q_down, nullptr, ctx->sf + l * (ctx->sf_pair + ctx->sf_down) + ctx->sf_pair, T,
+                     d, F, &y));
     } else {
       TRY(r.gemm_partial(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, &y));
     }
@@ -480,7 +498,8 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   el.ld = c.vocab;
   if (ctx->fp4) {
     TRY(act_quant(r, T, ctx->xn, pad * d, d));
-    TRY(r.gemm_fp4(A_KMAJOR, ctx->w.q_embed, nullptr, T, c.vocab, d, &y));
+    TRY(r.gemm_fp4(A_KMAJOR, ctx->w.q_embed, nullptr, ctx->sf + c.n_layers * (ctx->sf_pair + ctx->sf_down), T,
+                   c.vocab, d, &y));
     TRY(finish_tiles(r, y, c.vocab, el));
   } else {
     TRY(r.gemm(A_KMAJOR, ctx->w.embed, nullptr, ctx->xn, T, c.vocab, d, el));
@@ -696,6 +715,16 @@ dlm_status dlm_ctx_create(const dlm_config* cfg, const dlm_weights* w, void* d_w
         (const uint8_t*)w->q_embed.codes, (const uint8_t*)w->q_embed.scales, nb, ctx->e_deq);
     e = cudaGetLastError();
   }
+  // the weights' e4m3 scales, re-tiled for the FP4 MMA (tensor-memory scale layout)
+  for (int l = 0; l < cfg->n_layers && fp4 && e == cudaSuccess; ++l) {
+    uint8_t* base = ctx->sf + l * (ctx->sf_pair + ctx->sf_down);
+    e = nvf4_sf_tile(w->layers[l].q_gate, &w->layers[l].q_up, cfg->ffn, cfg->d, A_PAIR, base, ctx->cap_stream);
+    if (e == cudaSuccess)
+      e = nvf4_sf_tile(w->layers[l].q_down, nullptr, cfg->d, cfg->ffn, A_KMAJOR, base + ctx->sf_pair, ctx->cap_stream);
+  }
+  if (e == cudaSuccess && fp4)
+    e = nvf4_sf_tile(w->q_embed, nullptr, cfg->vocab, cfg->d, A_KMAJOR,
+                     ctx->sf + cfg->n_layers * (ctx->sf_pair + ctx->sf_down), ctx->cap_stream);
   if (e == cudaSuccess) e = (cudaError_t)gemm_init_attributes();
   if (e == cudaSuccess && fp4) e = (cudaError_t)gemm_fp4_init_attributes();
   if (e == cudaSuccess) e = (cudaError_t)attention_init_attributes();
@@ -1131,7 +1160,8 @@ dlm_status dlm_nvfp4_quantize(const void* d_w, int rows, int cols, void* d_codes
 size_t dlm_gemm_nvfp4_scratch_size(int T, int N, int K) {
   if (T < 1 || T > kMaxF4Tokens || N < 1 || K < 256 || K % 256 || K > 16384) return 0;
   return op_header() + op_counters(N) + align256(gemm_fp4_partial_bytes(T, N, K, A_KMAJOR)) +
-         align256((size_t)kMaxF4Tokens * K * 2) + align256(kMaxF4Tokens * 4);
+         align256((size_t)kMaxF4Tokens * K / 2) + align256((size_t)K / 64 * 512) + align256(kMaxF4Tokens * 4) +
+         align256(nvf4_sf_tile_bytes(N, K, A_KMAJOR));
 }
 
 dlm_status dlm_gemm_nvfp4(const float* d_x, const dlm_nvfp4_matrix* w, float* d_y, int T, int N, int K,
@@ -1144,18 +1174,26 @@ dlm_status dlm_gemm_nvfp4(const float* d_x, const dlm_nvfp4_matrix* w, float* d_
   CU((cudaError_t)gemm_fp4_init_attributes());
   cudaStream_t s = (cudaStream_t)stream;
   OpScratch sc(d_scratch, N, gemm_fp4_partial_bytes(T, N, K, A_KMAJOR));
-  __half* xq = sc.take<__half>((size_t)kMaxF4Tokens * K);
+  uint8_t* xcodes = sc.take<uint8_t>((size_t)kMaxF4Tokens * K / 2);
+  uint8_t* xscales = sc.take<uint8_t>((size_t)K / 64 * 512);
   float* sx = sc.take<float>(kMaxF4Tokens);
+  uint8_t* sfa = sc.take<uint8_t>(nvf4_sf_tile_bytes(N, K, A_KMAJOR));
   CU(cudaMemsetAsync(d_scratch, 0, op_header(), s));
+  // rows T.. of the token codes and scales are read by the MMA (their columns are dropped)
+  CU(cudaMemsetAsync(xcodes, 0, (size_t)kMaxF4Tokens * K / 2, s));
+  CU(cudaMemsetAsync(xscales, 0, (size_t)K / 64 * 512, s));
+  CU(nvf4_sf_tile(*w, nullptr, N, K, A_KMAJOR, sfa, s));
   ActQuantArgs q{};
   q.xf = d_x;
   q.K = K;
-  q.xq = xq;
+  q.codes = xcodes;
+  q.scales = xscales;
   q.sx = sx;
   CU_LAUNCH(launch_k(k_act_quant, dim3(T), dim3(256), 0, s, q));
   char msg[256];
   GemmF4Plan p;
-  if (!gemm_fp4_plan(&p, A_KMAJOR, *w, nullptr, xq, kMaxF4Tokens, sx, T, N, K, sc.partial, msg, sizeof(msg)))
+  if (!gemm_fp4_plan(&p, A_KMAJOR, *w, nullptr, sfa, xcodes, xscales, kMaxF4Tokens, sx, T, N, K, sc.partial, msg,
+                     sizeof(msg)))
     return DLM_EUNSUPPORTED;
   CU(gemm_fp4_launch(p, sc.err, s));
   if (d_y) {

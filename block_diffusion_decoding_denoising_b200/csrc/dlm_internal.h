@@ -57,7 +57,7 @@ constexpr int kTileM = 128;      // output features per GEMM tile (tcgen05 M)
 constexpr int kTileK = 64;       // reduction elements per k-block (one 128-byte swizzle atom)
 constexpr int kMaxTokens = 256;  // tokens per GEMM with plain bf16 activations (tcgen05 N <= 256)
 constexpr int kMaxSplitTokens = 128;  // tokens per GEMM with split (hi + lo) activations
-constexpr int kMaxF4Tokens = 64;      // tokens per NVFP4 GEMM
+constexpr int kMaxF4Tokens = 32;      // tokens per NVFP4 GEMM (MMA N)
 
 // Partial-sum layout written by the GEMM: [tile][slot][TP][128] fp32, TP = T rounded up to
 // 32 (token-major: the 128 rows of one token are contiguous).  Tile tau covers
@@ -137,23 +137,27 @@ bool gemm_plan(GemmPlan* p, int a_mode, const void* a0, const void* a1, const vo
 cudaError_t gemm_launch(const GemmPlan& p, int* d_err, cudaStream_t s);
 int gemm_init_attributes();
 
-// NVFP4 GEMM (dlm_gemm_fp4.cu): y = (x quantized per row) W^T with W in NVFP4.  x is given
-// as f16 values q sigma of the row quantizer (`xq`, x_rows >= 64 rows of K) with the row
-// scales `sx`; leaves scaled per-slot partial sums like the bf16 GEMM.  K % 256 == 0, T <= 64.
+// NVFP4 GEMM (dlm_gemm_fp4.cu): y = Q(x) W^T with W in NVFP4 on the block-scaled FP4
+// tensor cores.  x is given quantized (k_act_quant): e2m1 codes [x_rows][K/2], e4m3 scales
+// tiled [K/64][32][16 B], row scales sx; the weight scales come re-tiled by nvf4_sf_tile.  Leaves
+// scaled per-slot partial sums like the bf16 GEMM.  K % 256 == 0, T <= 32, x_rows >= 32.
 struct GemmF4Plan {
-  CUtensorMap tc0, tc1, ts0, ts1, tb;
+  CUtensorMap tc0, tc1, tbc;
   int a_mode;        // A_KMAJOR, or A_PAIR (gate/up: w0 = gate, w1 = up)
-  int nt;            // MMA N: 32 or 64
   int N, K, T;
   float sw0, sw1;
   const float* sx;
+  const uint8_t* sfa, *sfb;
   GemmOut out;
   size_t partial_bytes;
 };
 size_t gemm_fp4_partial_bytes(int T, int N, int K, int a_mode);
+size_t nvf4_sf_tile_bytes(int N, int K, int a_mode);
+cudaError_t nvf4_sf_tile(const dlm_nvfp4_matrix& w0, const dlm_nvfp4_matrix* w1, int N, int K, int a_mode,
+                         uint8_t* out, cudaStream_t s);
 bool gemm_fp4_plan(GemmF4Plan* p, int a_mode, const dlm_nvfp4_matrix& w0, const dlm_nvfp4_matrix* w1,
-                   const __half* xq, int x_rows, const float* sx, int T, int N, int K, float* partial, char* err,
-                   size_t errlen);
+                   const uint8_t* sfa_tiled, const uint8_t* xcodes, const uint8_t* xscales, int x_rows, const float* sx,
+                   int T, int N, int K, float* partial, char* err, size_t errlen);
 cudaError_t gemm_fp4_launch(const GemmF4Plan& p, int* d_err, cudaStream_t s);
 int gemm_fp4_init_attributes();
 

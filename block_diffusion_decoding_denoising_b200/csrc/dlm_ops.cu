@@ -537,17 +537,15 @@ __global__ void __launch_bounds__(256) k_act_quant(ActQuantArgs a) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) bm = fmaxf(bm, fabsf(v[i][j]));
     const uint8_t sb = (S > 0.f) ? e4m3_rne_bits(bm / (6.0f * S)) : 0;
-    const float sig = e4m3_value_dev(sb);
-    const float denom = sig * S;
-    __align__(16) __half out[16];
+    const float denom = e4m3_value_dev(sb) * S;
+    uint32_t packed[2] = {0u, 0u};
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const uint8_t c = denom > 0.f ? e2m1_rne(v[i][j] / denom) : 0;
-      out[j] = __float2half_rn(e2m1_value_dev(c) * sig);  // exact: <= 6 significant bits
+      const uint32_t c = denom > 0.f ? e2m1_rne(v[i][j] / denom) : 0u;
+      packed[j / 8] |= c << (4 * (j % 8));  // element 2m in the low nibble of byte m
     }
-    uint4* dst = reinterpret_cast<uint4*>(a.xq + (size_t)t * a.K + (size_t)b * 16);
-    dst[0] = reinterpret_cast<const uint4*>(out)[0];
-    dst[1] = reinterpret_cast<const uint4*>(out)[1];
+    a.scales[((size_t)(b / 4) * 32 + t) * 16 + (b % 4)] = sb;  // [64-element block][token][16 B]
+    *reinterpret_cast<uint2*>(a.codes + (size_t)t * (a.K / 2) + (size_t)b * 8) = make_uint2(packed[0], packed[1]);
   }
 }
 

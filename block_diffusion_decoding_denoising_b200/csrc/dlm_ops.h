@@ -43,13 +43,16 @@ struct RowStatsArgs {
 
 // Per-row NVFP4 quantizer of GEMM input activations: row t of x (fp32 `xf`, or the split
 // bf16 pair `xb` + `xb_lo`) gets the scale sx[t] = amax / (6 * 448), one e4m3 scale sigma
-// per 16 elements and e2m1 codes q; xq[t][k] = q sigma as f16 (exact).
+// per 16 elements and e2m1 codes (codes[t][K/2], element 2j in the low nibble).  The
+// scales are written in the FP4 MMA's copy layout: byte (b / 4) * 512 + t * 16 + b % 4 holds
+// the scale of group b (tokens t < 32; the other 12 bytes of each 16 are not used).
 struct ActQuantArgs {
   const float* xf;
   const __nv_bfloat16* xb;
   long xb_lo;
   int K;
-  __half* xq;
+  uint8_t* codes;
+  uint8_t* scales;
   float* sx;
 };
 

@@ -263,8 +263,9 @@ dlm_status dlm_nvfp4_quantize(const void* d_w, int rows, int cols, void* d_codes
  * dlm_nvfp4_matrix; host struct, device arrays) and Q(x) quantizes each row of x (fp32
  * [T][K]) to NVFP4 with its own fp32 scale amax_row / (6 * 448), e4m3 scales per 16 elements
  * and round-to-nearest-even e2m1 codes, the format the pages' B200 numbers use ("ORL:
- * diffusion LLMs get a learnable 'tokens per forward'", "What shipped").  T <= 64,
- * K % 256 == 0, K <= 16384.  d_y may be NULL: partial sums only (kernel timing). */
+ * diffusion LLMs get a learnable 'tokens per forward'", "What shipped"), on the
+ * block-scaled FP4 tensor cores.  T <= 32, K % 256 == 0, K <= 16384.  d_y may be NULL:
+ * partial sums only (kernel timing). */
 size_t dlm_gemm_nvfp4_scratch_size(int T, int N, int K);
 dlm_status dlm_gemm_nvfp4(const float* d_x, const dlm_nvfp4_matrix* w, float* d_y, int T, int N, int K,
                           void* d_scratch, size_t scratch_bytes, void* stream);

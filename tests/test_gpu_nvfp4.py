@@ -1,7 +1,8 @@
-"""NVFP4 weight GEMM (dlm_gemm_nvfp4) against the oracle: weights quantized by the
-oracle's codec, activations quantized per row on both sides from the same fp32 values.
-The products of the quantized operands are exact on both sides, so the results differ
-only by accumulation order (the contract is rel 6e-2; a tighter bound is checked too)."""
+"""NVFP4 weight GEMM (dlm_gemm_nvfp4, block-scaled FP4 tensor cores) against the oracle:
+weights quantized by the oracle's codec, activations quantized per row on both sides from
+the same fp32 values.  The products of the quantized operands are exact on both sides, so
+the results differ only by accumulation order (the contract is rel 6e-2; a tighter bound is
+checked too)."""
 import numpy as np
 import pytest
 
@@ -46,7 +47,7 @@ def run_case(D, T, N, K, seed, std=0.02, x_std=1.0):
     return err
 
 
-@pytest.mark.parametrize("T", [1, 5, 32, 33, 64])
+@pytest.mark.parametrize("T", [1, 5, 17, 32])
 @pytest.mark.parametrize("N,K", [(128, 256), (384, 512), (200, 768), (640, 2560)])
 def test_gemm_nvfp4_small(lib, T, N, K):
     run_case(lib, T, N, K, seed=T * 1000 + N + K)
@@ -82,4 +83,4 @@ def test_gemm_nvfp4_rejects_bad_shapes(lib):
         lib.gemm_nvfp4(torch.zeros((4, 320), device="cuda"), q)  # K % 256 != 0
     q2 = to_device_q(oracle_q(gen.bf16_bits(gen.normal_np(6, 128 * 256, 0.02).reshape(128, 256))))
     with pytest.raises(DlmError):
-        lib.gemm_nvfp4(torch.zeros((65, 256), device="cuda"), q2)  # T > 64
+        lib.gemm_nvfp4(torch.zeros((33, 256), device="cuda"), q2)  # T > 32
