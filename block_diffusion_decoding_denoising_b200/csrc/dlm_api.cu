@@ -345,7 +345,8 @@ struct FwdSpec {
 };
 
 // h update + RMSNorm into the split GEMM input xn, a 4-CTA cluster per token (see k_resid_norm).
-dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_tokens, const void* gain) {
+dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_tokens, const void* gain,
+                      bool quantize = false) {
   dlm_ctx* ctx = r.ctx;
   const dlm_config& c = ctx->cfg;
   ResNormArgs a{};
@@ -360,6 +361,11 @@ dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_t
   a.xn_lo = (long)split_pad(T) * c.d;
   a.d = c.d;
   a.eps = c.rms_eps;
+  if (quantize) {  // the next GEMM is NVFP4: quantize its input here (see k_act_quant)
+    a.qcodes = ctx->xcodes;
+    a.qscales = ctx->xscales;
+    a.qsx = ctx->sx;
+  }
   CU_LAUNCH(launch_k_cluster(k_resid_norm, dim3(T * kRnCluster), dim3(256), 0, r.s, kRnCluster, a));
   return DLM_OK;
 }
@@ -457,10 +463,9 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "attention: %s", cudaGetErrorString(e));
 
     TRY(r.gemm_partial(A_KMAJOR, W.w_o, nullptr, ctx->o, T, d, ho, &y));
-    TRY(resid_norm(r, T, &y, nullptr, W.mlp_norm));
+    TRY(resid_norm(r, T, &y, nullptr, W.mlp_norm, ctx->fp4));
 
-    if (ctx->fp4) {
-      TRY(act_quant(r, T, ctx->xn, pad * d, d));
+    if (ctx->fp4) {  // input quantized by the residual+RMSNorm above
       TRY(r.gemm_fp4(A_PAIR, W.q_gate, &W.q_up, ctx->sf + l * (ctx->sf_pair + ctx->sf_down), T, F, d, &y));
     } else {
       TRY(r.gemm_partial(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, &y));
@@ -478,7 +483,9 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     } else {
       TRY(r.gemm_partial(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, &y));
     }
-    TRY(resid_norm(r, T, &y, nullptr, l + 1 < c.n_layers ? ctx->layers[l + 1].attn_norm : ctx->w.final_norm));
+    const bool last = l + 1 == c.n_layers;
+    TRY(resid_norm(r, T, &y, nullptr, last ? ctx->w.final_norm : ctx->layers[l + 1].attn_norm,
+                   last && ctx->fp4 && f.lm_head));
   }
   if (!f.lm_head) return DLM_OK;
 
@@ -496,8 +503,8 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   el.op = EPI_STORE;
   el.out = ctx->logits;
   el.ld = c.vocab;
-  if (ctx->fp4) {
-    TRY(act_quant(r, T, ctx->xn, pad * d, d));
+  if (ctx->fp4) {  // input quantized by the last residual+RMSNorm
+    if (c.n_layers == 0) TRY(act_quant(r, T, ctx->xn, pad * d, d));
     TRY(r.gemm_fp4(A_KMAJOR, ctx->w.q_embed, nullptr, ctx->sf + c.n_layers * (ctx->sf_pair + ctx->sf_down), T,
                    c.vocab, d, &y));
     TRY(finish_tiles(r, y, c.vocab, el));

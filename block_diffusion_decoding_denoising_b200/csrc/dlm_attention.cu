@@ -298,10 +298,15 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
   }
 }
 
-// Merges the key splits: o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-__global__ void k_attn_combine(AttnArgs a) {
+// Merges the key splits: o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.  One CTA (128
+// threads) per row: the split weights are formed once (thread s loads split s's (m, l)),
+// then thread e loads O_s[e] of every split at once and sums them in split order.
+__global__ void __launch_bounds__(128) k_attn_combine(AttnArgs a) {
   pdl_trigger();
   pdl_wait();
+  __shared__ float wsp[64];
+  __shared__ float red[4];
+  __shared__ float den_s;
   const int G = a.Hq / a.Hkv;
   const int rows_total = a.T * G;
   const int Rows = a.Hkv * rows_total;
@@ -312,22 +317,39 @@ __global__ void k_attn_combine(AttnArgs a) {
   if (row >= Rows) return;
   const int g = row / rows_total, R = row % rows_total;
   const int t = R / G, h = g * G + R % G;
-  float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) {
-    float ms = a.part_ml[((size_t)s * Rows + row) * 2];
-    float ls = a.part_ml[((size_t)s * Rows + row) * 2 + 1];
-    if (ls > 0.f) M = fmaxf(M, ms);
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  float ms = -INFINITY, ls = 0.f;
+  if (tid < nsplit) {
+    ms = a.part_ml[((size_t)tid * Rows + row) * 2];
+    ls = a.part_ml[((size_t)tid * Rows + row) * 2 + 1];
   }
-  for (int e = threadIdx.x; e < a.hd; e += blockDim.x) {
-    float num = 0.f, den = 0.f;
-    for (int s = 0; s < nsplit; ++s) {
-      float ms = a.part_ml[((size_t)s * Rows + row) * 2];
-      float ls = a.part_ml[((size_t)s * Rows + row) * 2 + 1];
-      if (!(ls > 0.f)) continue;
-      float w = exp2f(ms - M);
-      num += w * a.part_o[((size_t)s * Rows + row) * a.hd + e];
-      den += w * ls;
+  float mx = warp_max(ls > 0.f ? ms : -INFINITY);
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  const float w = (tid < nsplit && ls > 0.f) ? exp2f(ms - M) : 0.f;
+  if (tid < 64) wsp[tid] = w;
+  __syncthreads();
+  if (tid == 0) {
+    float den = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) den += wsp[sp] * a.part_ml[((size_t)sp * Rows + row) * 2 + 1];  // split order
+    den_s = den;
+  }
+  __syncthreads();
+  const float den = den_s;
+  for (int e = tid; e < a.hd; e += blockDim.x) {
+    float num = 0.f;
+    const float* po = a.part_o + (size_t)row * a.hd + e;
+    const size_t sstride = (size_t)Rows * a.hd;
+    int sp = 0;
+    for (; sp + 8 <= nsplit; sp += 8) {  // eight independent loads in flight
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = __ldcg(po + (size_t)(sp + u) * sstride);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) num += wsp[sp + u] * x[u];
     }
+    for (; sp < nsplit; ++sp) num += wsp[sp] * __ldcg(po + (size_t)sp * sstride);
     store_split(a.o + ((size_t)t * a.Hq + h) * a.hd + e, a.o_lo, den > 0.f ? num / den : 0.f);
   }
 }

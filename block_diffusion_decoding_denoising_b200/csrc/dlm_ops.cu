@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kRnThreads) k_resid_norm(ResNormArgs a) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red[kRnThreads / 32];
-  __shared__ float ss_all[kRnCluster];
+  __shared__ float ss_all[kRnCluster], amax_all[kRnCluster];
   __shared__ int nsl[16];
   const int t = blockIdx.x / kRnCluster;
   uint32_t rank;
@@ -220,10 +220,57 @@ __global__ void __launch_bounds__(kRnThreads) k_resid_norm(ResNormArgs a) {
 #pragma unroll
   for (int q = 0; q < kRnCluster; ++q) tot += ss_all[q];  // rank order: the same sum everywhere
   const float r = 1.0f / sqrtf(tot / (float)a.d + a.eps);
+  float xv[kFeat];
 #pragma unroll
   for (int k = 0; k < kFeat; ++k) {
     const int n = f0 + threadIdx.x + k * kRnThreads;
-    if ((int)threadIdx.x + k * kRnThreads < dq) store_split(a.xn + (size_t)t * a.d + n, a.xn_lo, hv[k] * r * bf2f(a.gain[n]));
+    xv[k] = 0.f;
+    if ((int)threadIdx.x + k * kRnThreads < dq) {
+      xv[k] = hv[k] * r * bf2f(a.gain[n]);
+      store_split(a.xn + (size_t)t * a.d + n, a.xn_lo, xv[k]);
+    }
+  }
+  if (a.qcodes == nullptr) return;
+  // NVFP4 input of the next GEMM (the quantizer of k_act_quant on the fp32 row): row scale
+  // from the amax over the cluster, then 16-element groups = half-warps (the features of a
+  // warp for one k are 32 consecutive ones; d / 4 is a multiple of 64 here)
+  float am = 0.f;
+#pragma unroll
+  for (int k = 0; k < kFeat; ++k) am = fmaxf(am, fabsf(xv[k]));
+  am = warp_max(am);
+  __syncthreads();  // red[] is reused
+  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = am;
+  __syncthreads();
+  if (threadIdx.x < kRnCluster) {
+    float m = 0.f;
+    for (int i = 0; i < kRnThreads / 32; ++i) m = fmaxf(m, red[i]);
+    uint32_t dst;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(dst) : "r"(smem_u32(&amax_all[rank])), "r"((uint32_t)threadIdx.x));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dst), "f"(m) : "memory");
+  }
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  float amax = 0.f;
+#pragma unroll
+  for (int q = 0; q < kRnCluster; ++q) amax = fmaxf(amax, amax_all[q]);
+  const float S = amax / (6.0f * 448.0f);
+  if (rank == 0 && threadIdx.x == 0) a.qsx[t] = S;
+  const int lane = threadIdx.x % 32;
+#pragma unroll
+  for (int k = 0; k < kFeat; ++k) {
+    if ((int)(threadIdx.x - lane) + k * kRnThreads >= dq) continue;  // whole warp out of range
+    const int n = f0 + threadIdx.x + k * kRnThreads;
+    float bm = fabsf(xv[k]);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));  // within the half-warp
+    const uint8_t sb = (S > 0.f) ? e4m3_rne_bits(bm / (6.0f * S)) : 0;
+    const float denom = e4m3_value_dev(sb) * S;
+    const uint32_t code = denom > 0.f ? e2m1_rne(xv[k] / denom) : 0u;
+    const uint32_t hi = __shfl_down_sync(0xffffffffu, code, 1);
+    if ((lane & 1) == 0) a.qcodes[(size_t)t * (a.d / 2) + n / 2] = (uint8_t)(code | (hi << 4));
+    if ((lane & 15) == 0) {
+      const int gi = n / 16;
+      a.qscales[((size_t)(gi / 4) * 32 + t) * 16 + (gi % 4)] = sb;
+    }
   }
 }
 

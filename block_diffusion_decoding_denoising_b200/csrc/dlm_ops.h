@@ -25,6 +25,9 @@ struct ResNormArgs {
   const __nv_bfloat16* gain;   // [d]
   __nv_bfloat16* xn;           // [T][d] high halves
   long xn_lo;                  // elements to the low halves
+  uint8_t* qcodes;             // non-null: also quantize xn to NVFP4 (see ActQuantArgs)
+  uint8_t* qscales;
+  float* qsx;
   int d;
   float eps;
 };
