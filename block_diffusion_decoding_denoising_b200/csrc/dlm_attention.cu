@@ -358,7 +358,7 @@ int attention_max_splits(int T, int Hq, int Hkv, int max_ctx) {
   const int G = Hq / Hkv;
   const int qtiles = (T * G + kAttnRows - 1) / kAttnRows;
   int ctas = qtiles * Hkv;
-  int s = (2 * kSMs + ctas - 1) / ctas;  // enough splits for two CTAs per SM (each CTA is latency-bound)
+  int s = (2 * kSMs) / ctas;  // two CTAs per SM in a single wave (each CTA is latency-bound)
   int by_len = (max_ctx + T + kMinKeysPerSplit - 1) / kMinKeysPerSplit;
   if (s > by_len) s = by_len;
   if (s < 1) s = 1;

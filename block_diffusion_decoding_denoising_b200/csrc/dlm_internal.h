@@ -163,7 +163,7 @@ int gemm_fp4_init_attributes();
 
 // LM head fused with the row statistics and s = P E (dlm_lmhead.cu), one pass over E.
 // x2: split bf16 pair, rows [0, T) high halves, rows [32, 32 + T) low halves; p_given:
-// bf16 [T][V] or nullptr (P = softmax of the logits).  T <= 32, d % 256 == 0, d <= 3584.
+// bf16 [T][V] or nullptr (P = softmax of the logits).  T <= 32, d % 256 == 0, d <= 3072.
 bool lmhead_fused_supported(int T, int d);
 size_t lmhead_fused_scratch_bytes(int V, int d);
 cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_given, int T, int V, int d,

@@ -9,8 +9,9 @@
 //
 // Work split: vocabulary tiles of 128 rows, a contiguous range of tiles per cluster of two
 // CTAs; CTA rank r owns the model-width half [r d/2, (r + 1) d/2).  Per tile:
-//   L  partial logits over the CTA's half: tcgen05, A = E tile (K-major), B = x (split
-//      bf16 hi + lo accumulated into the same TMEM columns); double-buffered accumulator.
+//   L  partial logits over the CTA's half: tcgen05, A = E tile (K-major), B = x as a split
+//      bf16 pair (N = 64: the high halves in TMEM columns 0..31, the low halves in 32..63,
+//      added by the epilogue), so each E chunk is read once per MMA; double-buffered.
 //   X  the two partial logit tiles are swapped through distributed shared memory (remote
 //      stores + a remote mbarrier arrive with cluster-scope release), so both CTAs hold
 //      the same full logits; they are read transposed ([token][vocab]) for the per-token
@@ -38,9 +39,9 @@ constexpr int kLmStages = 5;
 constexpr int kLmStageBytes = 24576;    // E box 16 KB + x box 8 KB (L) / 2 E boxes + P box (PE)
 constexpr int kLmPBytes = 16384;        // P tile: 64 rows (hi, lo) x 128 vocab, 2 swizzle atoms
 constexpr int kLmXBytes = kLmT * 128 * 4;  // one partial-logit tile [32][128] fp32
-constexpr int kLmMaxChunks = 14;        // d / 2 <= 1792
-constexpr int kLmMaxClusters = kSMs / 2;  // clusters of two CTAs
-constexpr int kLmSCol = 64;             // TMEM column of the first s accumulator
+constexpr int kLmMaxChunks = 12;        // d / 2 <= 1536 (TMEM: 128 + 12 x 32 columns)
+constexpr int kLmMaxClusters = kSMs / 2;  // clusters of two CTAs (<= 80: five per merge chunk)
+constexpr int kLmSCol = 128;            // TMEM column of the first s accumulator
 constexpr float kLmRescale = 8.0f;      // raise the reference when a max exceeds it by this
 constexpr int kLmSmem = kLmStages * kLmStageBytes + 2 * kLmPBytes + 4 * kLmXBytes + 1024 + 1024;
 
@@ -236,70 +237,84 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
       if (!mbar_wait(&empty[stage], phase ^ 1, a.err)) break;
       advance();
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer (same order as the producer)
-    const uint32_t idesc_l = idesc_bf16(128, kLmT, false, false);
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (same order as the producer).  The whole warp runs the loop
+    // and waits; one elected lane issues the MMAs and commits (outcomes made warp-uniform).
+    const uint32_t idesc_l = idesc_bf16(128, 2 * kLmT, false, false);
     const uint32_t idesc_pe = idesc_bf16(128, kLmT, true, false);
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, a.err)) != 0;
+    };
     auto mma_l = [&](int i) {
       const int b = i & 1;
-      if (!mbar_wait(&accl_empty[b], ((i >> 1) & 1) ^ 1, a.err)) { ok = false; return; }
+      if (!wait_all(&accl_empty[b], ((i >> 1) & 1) ^ 1)) { ok = false; return; }
       tc_fence_after();
-      const uint32_t dl = tmem + b * kLmT;
+      const uint32_t dl = tmem + b * 2 * kLmT;
       for (int kb = 0; kb < KB; ++kb) {
-        if (!mbar_wait(&full[stage], phase, a.err)) { ok = false; return; }
+        if (!wait_all(&full[stage], phase)) { ok = false; return; }
         tc_fence_after();
-        const uint32_t sa = smem_u32(ring + stage * kLmStageBytes), sx = sa + 16384;
+        const uint32_t sa = smem_u32(ring + stage * kLmStageBytes);
+        const uint64_t ad = sw128_desc(sa, 16, 1024), xd = sw128_desc(sa + 16384, 16, 1024);
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-#pragma unroll
-          for (int h = 0; h < 2; ++h)  // x = hi + lo: rows 0..31 and 32..63 of the x box
-            mma_bf16(dl, sw128_desc(sa + k * 32, 16, 1024), sw128_desc(sx + h * 4096 + k * 32, 16, 1024),
-                     idesc_l, (kb | k | h) ? 1u : 0u);
-        mma_commit(&empty[stage]);
+          for (int k = 0; k < 4; ++k)  // x box rows 0..31 = hi, 32..63 = lo -> D columns 0..63
+            mma_bf16(dl, ad + 2 * k, xd + 2 * k, idesc_l, (kb | k) ? 1u : 0u);  // +32 B per k step
+          mma_commit(&empty[stage]);
+        }
+        __syncwarp();
         if (++stage == kLmStages) { stage = 0; phase ^= 1; }
       }
-      mma_commit(&accl_full[b]);
+      if (elect_one()) mma_commit(&accl_full[b]);
+      __syncwarp();
     };
     auto mma_pe = [&](int i) {
       const int b = i & 1;
-      if (!mbar_wait(&p_ready[b], (i >> 1) & 1, a.err)) { ok = false; return; }
+      if (!wait_all(&p_ready[b], (i >> 1) & 1)) { ok = false; return; }
       tc_fence_after();
-      const uint32_t pb = smem_u32(pbuf + b * kLmPBytes);
+      const uint64_t pd = sw128_desc(smem_u32(pbuf + b * kLmPBytes), 16, 1024);
       for (int ch = 0; ch < CH; ++ch) {
         const uint32_t ds = tmem + kLmSCol + ch * kLmT;
         for (int vh = 0; vh < 2; ++vh) {
-          if (!mbar_wait(&full[stage], phase, a.err)) { ok = false; return; }
+          if (!wait_all(&full[stage], phase)) { ok = false; return; }
           tc_fence_after();
           const uint32_t sa = smem_u32(ring + stage * kLmStageBytes);
+          const uint64_t ad0 = sw128_desc(sa, 8192, 1024), gd = sw128_desc(sa + 16384, 16, 1024);
+          if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = sw128_desc(sa + k * 2048, 8192, 1024);  // E^T: 16 vocab rows per step
-            const bool first = (i == 0 && vh == 0 && k == 0);
-            if (a.given) {
-              mma_bf16(ds, ad, sw128_desc(sa + 16384 + k * 32, 16, 1024), idesc_pe, first ? 0u : 1u);
-            } else {
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad = ad0 + 128 * k;  // E^T: 16 vocab rows (2048 B) per step
+              const bool first = (i == 0 && vh == 0 && k == 0);
+              if (a.given) {
+                mma_bf16(ds, ad, gd + 2 * k, idesc_pe, first ? 0u : 1u);
+              } else {
 #pragma unroll
-              for (int h = 0; h < 2; ++h)
-                mma_bf16(ds, ad, sw128_desc(pb + vh * 8192 + h * 4096 + k * 32, 16, 1024), idesc_pe,
-                         (first && h == 0) ? 0u : 1u);
+                for (int h = 0; h < 2; ++h)  // P rows 0..31 = hi, 32..63 = lo (+4096 B)
+                  mma_bf16(ds, ad, pd + (vh * 8192 + h * 4096 + k * 32) / 16, idesc_pe,
+                           (first && h == 0) ? 0u : 1u);
+              }
             }
+            mma_commit(&empty[stage]);
           }
-          mma_commit(&empty[stage]);
+          __syncwarp();
           if (++stage == kLmStages) { stage = 0; phase ^= 1; }
         }
       }
-      mma_commit(&pe_done[b]);
+      if (elect_one()) mma_commit(&pe_done[b]);
+      __syncwarp();
     };
     for (int i = 0; i < nt && ok; ++i) {
       mma_l(i);
       if (ok && i >= 1) mma_pe(i - 1);
     }
     if (ok && nt > 0) mma_pe(nt - 1);
-    mma_commit(mma_done);
-    mbar_wait(mma_done, 0, a.err);
+    if (elect_one()) {
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, a.err);
+    }
+    __syncwarp();
   } else if (warp >= 2) {
     // ---------------- epilogue: exchange, statistics, P, rescale, outputs
     const int et = threadIdx.x - 64;        // 0..127
@@ -322,7 +337,14 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
       if (!ok) break;
       tc_fence_after();
       float lp[32];
-      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * kLmT, lp);
+      {
+        float lo_[32];
+        const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + b * 2 * kLmT;
+        tmem_ld32(ta, lp);
+        tmem_ld32(ta + kLmT, lo_);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) lp[t] += lo_[t];
+      }
       tc_fence_before();
       mbar_arrive(&accl_empty[b]);
       // 2. swap with the peer: own copy locally, the peer's copy by remote stores
@@ -467,55 +489,84 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
 
 // Merge of the clusters: for token t, M = max_c r_c, Z = sum_c Z_c e^(r_c - M), lse = M + ln Z,
 // maxprob = e^(max - lse), entropy = lse - A / Z, argmax from the lowest-index cluster holding
-// the max; s[t][f] = sum_c e^(r_c - M) s_c[f][t] / Z (given P: plain sum).  The per-token
-// reductions run over the lanes of a warp (a fixed shuffle tree), the s sums over the warps
-// of a CTA (each warp a fixed set of clusters, then the warps in order).
-// grid: d / 32 CTAs of 256 threads (8 warps x 32 features).
-__global__ void __launch_bounds__(256) k_lmf_combine(LmfArgs a, dlm_row_stats stats, float* s) {
+// the max; s[t][f] = sum_c e^(r_c - M) s_c[f][t] / Z (given P: plain sum).
+// grid: d / 32 CTAs of 512 threads (16 warps x 32 features).  The per-token values are reduced
+// in two steps (16 cluster chunks, then the chunks in order); the s sums over the warps (each
+// a fixed set of clusters, the next cluster's 128 bytes loaded while the current one is
+// accumulated), then the warps in order.
+constexpr int kLmfWarps = 16;
+constexpr int kLmfSmem = (kLmMaxClusters * 32 + kLmfWarps * 32 * 33 + 4 * kLmfWarps * 32) * 4;
+__global__ void __launch_bounds__(kLmfWarps * 32) k_lmf_combine(LmfArgs a, dlm_row_stats stats, float* s) {
   pdl_trigger();
   pdl_wait();
-  __shared__ __align__(16) float w[kLmMaxClusters][32];  // per-cluster weight of each token
-  __shared__ float red[8][32][33];
-  __shared__ float iZ[32];
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // 1. per token: warp `warp` handles tokens warp, warp + 8, ...; lanes stride the clusters
-  for (int t = warp; t < 32; t += 8) {
-    float M = -INFINITY;
-    for (int c = lane; c < a.n_clu; c += 32) M = fmaxf(M, a.part_stats[((size_t)c * 32 + t) * 4]);
-    M = warp_max(M);
-    float zs = 0.f, as = 0.f, mx = -INFINITY;
-    int mc = 0x7fffffff;
-    for (int c = lane; c < a.n_clu; c += 32) {
-      const float4 ps = *reinterpret_cast<const float4*>(a.part_stats + ((size_t)c * 32 + t) * 4);
-      const float e = expf(ps.x - M);
-      w[c][t] = a.given ? 1.f : e;
-      zs += ps.y * e;
-      as += ps.z * e;
-      if (ps.w > mx) { mx = ps.w; mc = c; }  // clusters visited in increasing order
-    }
-    zs = warp_sum(zs);
-    as = warp_sum(as);
+  extern __shared__ __align__(16) float sm_f[];
+  float(*w)[32] = reinterpret_cast<float(*)[32]>(sm_f);                         // [clusters][32]
+  float(*red)[32][33] = reinterpret_cast<float(*)[32][33]>(sm_f + kLmMaxClusters * 32);  // [warps][32][33]
+  float* cm = sm_f + kLmMaxClusters * 32 + kLmfWarps * 32 * 33;                 // [4][warps][32]
+  __shared__ float Mt[32], iZ[32];
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  // 1. per token: thread (chunk = warp, token = lane) takes clusters chunk, chunk + 16, ...
+  {
+    const int t = lane, ch = warp;
+    float4 ps[5];
+    int nc = 0;
+    float rmax = -INFINITY;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, mx, o);
-      const int c2 = __shfl_xor_sync(0xffffffffu, mc, o);
-      if (m2 > mx || (m2 == mx && c2 < mc)) { mx = m2; mc = c2; }
+    for (int k = 0; k < 5; ++k) {
+      const int c = ch + k * kLmfWarps;
+      if (c < a.n_clu) {
+        ps[k] = *reinterpret_cast<const float4*>(a.part_stats + ((size_t)c * 32 + t) * 4);
+        rmax = fmaxf(rmax, ps[k].x);
+        nc = k + 1;
+      }
     }
-    if (lane == 0) {
-      iZ[t] = a.given ? 1.f : 1.f / zs;
-      if (blockIdx.x == 0 && t < a.T) {
-        const float lse = M + logf(zs);
-        stats.m[t] = mx;
-        stats.lse[t] = lse;
-        stats.maxprob[t] = expf(mx - lse);
-        stats.entropy[t] = lse - as / zs;
-        stats.argmax[t] = a.part_arg[(size_t)mc * 32 + t];
+    cm[(0 * kLmfWarps + ch) * 32 + t] = rmax;
+    __syncthreads();
+    if (tid < 32) {
+      float M = -INFINITY;
+      for (int q = 0; q < kLmfWarps; ++q) M = fmaxf(M, cm[q * 32 + tid]);
+      Mt[tid] = M;
+    }
+    __syncthreads();
+    const float M = Mt[t];
+    float zs = 0.f, as = 0.f, mx = -INFINITY, mc = 0.f;  // mc: cluster index of mx (as float)
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+      if (k < nc) {
+        const int c = ch + k * kLmfWarps;
+        const float e = expf(ps[k].x - M);
+        w[c][t] = a.given ? 1.f : e;
+        zs += ps[k].y * e;
+        as += ps[k].z * e;
+        if (ps[k].w > mx) { mx = ps[k].w; mc = (float)c; }
+      }
+    }
+    cm[(0 * kLmfWarps + ch) * 32 + t] = zs;
+    cm[(1 * kLmfWarps + ch) * 32 + t] = as;
+    cm[(2 * kLmfWarps + ch) * 32 + t] = mx;
+    cm[(3 * kLmfWarps + ch) * 32 + t] = mc;
+    __syncthreads();
+    if (tid < 32) {
+      float Z = 0.f, A = 0.f, bm = -INFINITY, bc = 1e30f;
+      for (int q = 0; q < kLmfWarps; ++q) {  // chunks in order; ties -> lowest cluster index
+        Z += cm[(0 * kLmfWarps + q) * 32 + tid];
+        A += cm[(1 * kLmfWarps + q) * 32 + tid];
+        const float m2 = cm[(2 * kLmfWarps + q) * 32 + tid], c2 = cm[(3 * kLmfWarps + q) * 32 + tid];
+        if (m2 > bm || (m2 == bm && c2 < bc)) { bm = m2; bc = c2; }
+      }
+      iZ[tid] = a.given ? 1.f : 1.f / Z;
+      if (blockIdx.x == 0 && tid < a.T) {
+        const float lse = Mt[tid] + logf(Z);
+        stats.m[tid] = bm;
+        stats.lse[tid] = lse;
+        stats.maxprob[tid] = expf(bm - lse);
+        stats.entropy[tid] = lse - A / Z;
+        stats.argmax[tid] = a.part_arg[(size_t)(bc < (float)a.n_clu ? (int)bc : 0) * 32 + tid];  // NaN rows: cluster 0
       }
     }
   }
   __syncthreads();
-  // 2. s: lane = feature blockIdx.x * 32 + lane, warp = clusters warp, warp + 8, ...; the next
-  //    cluster's 128 bytes are loaded while the current one is accumulated
+  // 2. s: lane = feature blockIdx.x * 32 + lane, warp = clusters warp, warp + 16, ...
   const int f = blockIdx.x * 32 + lane;
   float acc[32];
 #pragma unroll
@@ -527,8 +578,8 @@ __global__ void __launch_bounds__(256) k_lmf_combine(LmfArgs a, dlm_row_stats st
 #pragma unroll
     for (int u = 0; u < 8; ++u) cur[u] = __ldcg(src + u);
   }
-  for (; c < a.n_clu; c += 8) {
-    const int cn = c + 8;
+  for (; c < a.n_clu; c += kLmfWarps) {
+    const int cn = c + kLmfWarps;
     if (cn < a.n_clu) {
       const float4* src = reinterpret_cast<const float4*>(a.part_s + ((size_t)cn * a.d + f) * 32);
 #pragma unroll
@@ -549,11 +600,11 @@ __global__ void __launch_bounds__(256) k_lmf_combine(LmfArgs a, dlm_row_stats st
 #pragma unroll
   for (int t = 0; t < 32; ++t) red[warp][lane][t] = acc[t];
   __syncthreads();
-  for (int i = threadIdx.x; i < 32 * 32; i += blockDim.x) {
+  for (int i = tid; i < 32 * 32; i += blockDim.x) {
     const int t = i / 32, fl = i % 32;
     if (t >= a.T) continue;
     float v = 0.f;
-    for (int wv = 0; wv < 8; ++wv) v += red[wv][fl][t];  // warps in order
+    for (int wv = 0; wv < kLmfWarps; ++wv) v += red[wv][fl][t];  // warps in order
     s[(size_t)t * a.d + blockIdx.x * 32 + fl] = v * iZ[t];
   }
 }
@@ -583,6 +634,7 @@ cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_giv
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k_lmhead_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmSmem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_lmf_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmfSmem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
@@ -624,7 +676,7 @@ cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_giv
   cfg.numAttrs = g_pdl ? 2 : 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, k_lmhead_fused, tek, tem, tx, tp, a);
   if (e != cudaSuccess) return e;
-  return launch_k(k_lmf_combine, dim3(d / 32), dim3(256), 0, st, a, stats, s);
+  return launch_k(k_lmf_combine, dim3(d / 32), dim3(kLmfWarps * 32), kLmfSmem, st, a, stats, s);
 }
 
 }  // namespace dlm

@@ -238,7 +238,7 @@ dlm_status dlm_bd_attention(const void* d_q, const void* d_k_cache, const void* 
  * in a fixed 16 MiB array of static device memory per device; calls whose partials
  * (split count x T x Hq x (hd + 2) x 4 bytes, the split count as dlm_bd_attention picks it
  * from T, Hq, Hkv and max_ctx) exceed 16 MiB - 256 B are rejected with DLM_ENOMEM_WS.  The
- * 4B-class shapes (T <= 64, 32/8 heads, hd 128) need at most 10.7 MB.  The first call on a
+ * 4B-class shapes (T <= 64, 32/8 heads, hd 128) need at most 9.9 MB.  The first call on a
  * device looks the array up and sets kernel attributes: make it before starting any stream
  * capture on that device.  Every call clears the array's status word on `stream`.  The
  * array is shared: calls that may overlap in time race on it and must be serialised by the

@@ -39,8 +39,8 @@ def test_noalloc_matches_scratch_entry_twice(D, T, L, causal):
 def test_noalloc_rejects_oversized_call(D):
     import torch
     from block_diffusion_decoding_denoising_b200.dlm import DLM_ENOMEM_WS, DlmError
-    # 64 queries x 256 heads of 128: the split partials exceed the 16 MiB array
-    T, Hq, Hkv, hd, L = 64, 256, 32, 128, 8192
+    # 64 queries x 512 heads of 128 (one split): the partials exceed the 16 MiB array
+    T, Hq, Hkv, hd, L = 64, 512, 64, 128, 8192
     q = torch.zeros((T, Hq, hd), dtype=torch.bfloat16, device="cuda")
     kc = torch.zeros((Hkv, L + T, hd), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(DlmError) as ei:
