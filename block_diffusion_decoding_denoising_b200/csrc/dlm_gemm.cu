@@ -147,8 +147,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
     // never leave the CTA with copies in flight: wait (bounded) for every armed stage
     for (int i = 0; i < S; ++i)
       if (armed[i]) mbar_wait(&full[i], armed_parity[i], args.err);
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
+  } else if (warp == 1) {
+    // ---------------- MMA issuer: the whole warp runs the loop and waits (outcomes made
+    // warp-uniform); one elected lane issues the MMAs and the commits
     const uint32_t idesc = idesc_bf16(128, NT, args.a_mode == A_MNMAJOR, false);
     int stage = 0;
     uint32_t phase = 0;
@@ -159,33 +160,40 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
     while (u < u_end && ok) {
       const int tile = (int)(u / o.n_kb);
       const long seg_end = ((long)tile + 1) * o.n_kb < u_end ? ((long)tile + 1) * o.n_kb : u_end;
-      if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, args.err)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_empty[acc], acc_phase ^ 1, args.err))) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * NT;
       for (long uu = u; uu < seg_end; ++uu) {
-        if (!mbar_wait(&full[stage], phase, args.err)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, args.err))) { ok = false; break; }
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
         const uint32_t sb = sa + Cfg::kABytes;
+        // K step k: +32 B (K-major A and B) or +2048 B (MN-major A: 16 rows of 128 B)
+        const uint64_t ad = (args.a_mode == A_MNMAJOR) ? sw128_desc(sa, Cfg::kABytes / 2, 1024)
+                                                        : sw128_desc(sa, 16, 1024);
+        const uint32_t astep = (args.a_mode == A_MNMAJOR) ? 128u : 2u;
+        const uint64_t bd = sw128_desc(sb, 16, 1024);
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < kTileK / 16; ++k) {
-          uint64_t adesc = (args.a_mode == A_MNMAJOR)
-                               ? sw128_desc(sa + k * 2048, Cfg::kABytes / 2, 1024)
-                               : sw128_desc(sa + k * 32, 16, 1024);
-          uint64_t bdesc = sw128_desc(sb + k * 32, 16, 1024);
-          mma_bf16(d_tmem, adesc, bdesc, idesc, (uu > u || k > 0) ? 1u : 0u);
+          for (int k = 0; k < kTileK / 16; ++k)
+            mma_bf16(d_tmem, ad + astep * k, bd + 2 * k, idesc, (uu > u || k > 0) ? 1u : 0u);
+          mma_commit(&empty[stage]);
         }
-        mma_commit(&empty[stage]);
+        __syncwarp();
         if (++stage == S) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
-      mma_commit(&acc_full[acc]);
+      if (elect_one()) mma_commit(&acc_full[acc]);
+      __syncwarp();
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       u = seg_end;
     }
-    // all MMAs of this thread complete before TMEM is released
-    mma_commit(mma_done);
-    mbar_wait(mma_done, 0, args.err);
+    // all MMAs of the issuing lane complete before TMEM is released
+    if (elect_one()) {
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, args.err);
+    }
+    __syncwarp();
   } else if (warp >= 2) {
     // ---------------- epilogue: TMEM -> partial sums / finished tiles
     const int quarter = warp % 4;

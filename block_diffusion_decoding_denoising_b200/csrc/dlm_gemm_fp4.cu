@@ -195,8 +195,10 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tc0, const __grid_constant__ CUt
     pdl_trigger();
     for (int i = 0; i < S; ++i)
       if (armed[i]) mbar_wait(&full[i], armed_parity[i], args.err);
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer: scales to TMEM, four K = 64 block-scaled MMAs per stage
+  } else if (warp == 1) {
+    // ---------------- MMA issuer: scales to TMEM, four K = 64 block-scaled MMAs per stage.
+    // The whole warp runs the loop and waits (outcomes made warp-uniform); one elected lane
+    // issues the copies, the MMAs and the commits.
     constexpr uint32_t idesc = idesc_nvf4(128, 32);
     int stage = 0, acc = 0;
     uint32_t phase = 0, acc_phase = 0;
@@ -205,36 +207,43 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tc0, const __grid_constant__ CUt
     while (u < u_end && ok) {
       const int tile = (int)(u / o.n_kb);
       const long seg_end = ((long)tile + 1) * o.n_kb < u_end ? ((long)tile + 1) * o.n_kb : u_end;
-      if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, args.err)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_empty[acc], acc_phase ^ 1, args.err))) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * 32;
       for (long uu = u; uu < seg_end; ++uu) {
-        if (!mbar_wait(&full[stage], phase, args.err)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, args.err))) { ok = false; break; }
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + stage * kF4StageBytes);
         const uint32_t sfa_col = tmem_base + kF4SfCol + stage * kF4SfColsPerStage;
         const uint32_t sfb_col = sfa_col + 4 * kF4Mmas;
+        const uint64_t ad = sw128_desc(sa, 16, 1024), bd = sw128_desc(sa + kF4OffB, 16, 1024);
+        const uint64_t fa = sf_desc(sa + kF4OffSfA), fb = sf_desc(sa + kF4OffSfB);
+        if (elect_one()) {
 #pragma unroll
-        for (int j = 0; j < kF4Mmas; ++j) {
-          tmem_cp_32x128(sfa_col + 4 * j, sf_desc(sa + kF4OffSfA + j * 512));
-          tmem_cp_32x128(sfb_col + 4 * j, sf_desc(sa + kF4OffSfB + j * 512));
-        }
+          for (int j = 0; j < kF4Mmas; ++j) {  // +512 B per copy source
+            tmem_cp_32x128(sfa_col + 4 * j, fa + 32 * j);
+            tmem_cp_32x128(sfb_col + 4 * j, fb + 32 * j);
+          }
 #pragma unroll
-        for (int j = 0; j < kF4Mmas; ++j) {
-          const uint64_t adesc = sw128_desc(sa + j * 32, 16, 1024);
-          const uint64_t bdesc = sw128_desc(sa + kF4OffB + j * 32, 16, 1024);
-          mma_nvf4(d_tmem, adesc, bdesc, idesc, sfa_col + 4 * j, sfb_col + 4 * j, (uu > u || j > 0) ? 1u : 0u);
+          for (int j = 0; j < kF4Mmas; ++j)  // +32 B per K = 64 step
+            mma_nvf4(d_tmem, ad + 2 * j, bd + 2 * j, idesc, sfa_col + 4 * j, sfb_col + 4 * j,
+                     (uu > u || j > 0) ? 1u : 0u);
+          mma_commit(&empty[stage]);
         }
-        mma_commit(&empty[stage]);
+        __syncwarp();
         if (++stage == S) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
-      mma_commit(&acc_full[acc]);
+      if (elect_one()) mma_commit(&acc_full[acc]);
+      __syncwarp();
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       u = seg_end;
     }
-    mma_commit(mma_done);
-    mbar_wait(mma_done, 0, args.err);
+    if (elect_one()) {
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, args.err);
+    }
+    __syncwarp();
   } else if (warp >= 2) {
     // ---------------- epilogue: TMEM -> scaled partial sums
     const int quarter = warp % 4;

@@ -35,7 +35,7 @@ namespace dlm {
 namespace {
 
 constexpr int kLmT = 32;                // tokens (MMA N)
-constexpr int kLmStages = 5;
+constexpr int kLmStages = 6;
 constexpr int kLmStageBytes = 24576;    // E box 16 KB + x box 8 KB (L) / 2 E boxes + P box (PE)
 constexpr int kLmPBytes = 16384;        // P tile: 64 rows (hi, lo) x 128 vocab, 2 swizzle atoms
 constexpr int kLmXBytes = kLmT * 128 * 4;  // one partial-logit tile [32][128] fp32
@@ -43,7 +43,8 @@ constexpr int kLmMaxChunks = 12;        // d / 2 <= 1536 (TMEM: 128 + 12 x 32 co
 constexpr int kLmMaxClusters = kSMs / 2;  // clusters of two CTAs (<= 80: five per merge chunk)
 constexpr int kLmSCol = 128;            // TMEM column of the first s accumulator
 constexpr float kLmRescale = 8.0f;      // raise the reference when a max exceeds it by this
-constexpr int kLmSmem = kLmStages * kLmStageBytes + 2 * kLmPBytes + 4 * kLmXBytes + 1024 + 1024;
+constexpr int kLmSmem = kLmStages * kLmStageBytes + 2 * kLmPBytes + 3 * kLmXBytes + 1024 + 1024;
+static_assert(kLmSmem <= 232448, "fused LM head shared memory");
 
 struct LmfArgs {
   int V, d, T, mask_id;
@@ -138,8 +139,11 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = smem;
   uint8_t* pbuf = smem + kLmStages * kLmStageBytes;                     // [2][16 KB]
-  float* mine = (float*)(pbuf + 2 * kLmPBytes);                         // [2][32][128]
-  float* theirs = mine + 2 * kLmT * 128;                                // [2][32][128]
+  // mine: this CTA's own partial logits of the current tile (one buffer: every epilogue
+  // thread has finished reading tile i, a barrier later, before any writes tile i + 1);
+  // theirs: the peer's, written remotely and possibly one tile ahead (two buffers)
+  float* mine = (float*)(pbuf + 2 * kLmPBytes);                         // [32][128]
+  float* theirs = mine + kLmT * 128;                                    // [2][32][128]
   uint64_t* bars = (uint64_t*)(theirs + 2 * kLmT * 128);
   uint64_t* full = bars;                      // [S]
   uint64_t* empty = bars + kLmStages;         // [S]
@@ -348,7 +352,7 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
       tc_fence_before();
       mbar_arrive(&accl_empty[b]);
       // 2. swap with the peer: own copy locally, the peer's copy by remote stores
-      float* mb = mine + b * kLmT * 128;
+      float* mb = mine;
       const uint32_t tpeer = theirs_peer + (uint32_t)(b * kLmT * 128 * 4);
 #pragma unroll
       for (int t = 0; t < 32; ++t) {
@@ -359,10 +363,14 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
       // every thread acquires the peer's tile itself; the barrier also publishes the local
       // partial writes to the transposed reads
       if (epi_any(!mbar_wait_cluster(&xfull[b], (i >> 1) & 1, a.err))) { ok = false; break; }
-      // 3. per-token statistics over the tile: warp tw, tokens 8 tw + j, lane: vocab 4 lane .. +3
+      // 3. P(i) goes into pbuf[b], so PE(i - 2) must be done with it (it is: tcgen05 work
+      //    completes in issue order and L(i), issued after it, has completed)
+      if (epi_any(i >= 2 && !mbar_wait(&pe_done[b], ((i - 2) >> 1) & 1, a.err))) { ok = false; break; }
+      // 4. per-token statistics over the tile, P written as it is formed: warp tw, tokens
+      //    8 tw + j, lane: vocab 4 lane .. +3
       const float* tb_ = theirs + b * kLmT * 128;
+      uint8_t* pt = pbuf + b * kLmPBytes;
       int need = 0;
-      float pv[8][4];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int t = tw * 8 + j;
@@ -396,27 +404,30 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
         }
         if (lane == 0) fac[t] = f;
         float zs = 0.f, as = 0.f;
+        __align__(8) __nv_bfloat16 hi[4], lo[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const float p = (l[u] == -INFINITY) ? 0.f : expf(l[u] - ref[j]);
-          pv[j][u] = p;
           zs += p;
           as += (p > 0.f) ? p * l[u] : 0.f;
+          const float pw = (t < a.T) ? p : 0.f;
+          hi[u] = f2bf(pw);
+          lo[u] = f2bf(pw - bf2f(hi[u]));
+        }
+        if (!a.given) {
+          *reinterpret_cast<uint2*>(pt + p_offset(t, lane * 4)) = *reinterpret_cast<const uint2*>(hi);
+          *reinterpret_cast<uint2*>(pt + p_offset(32 + t, lane * 4)) = *reinterpret_cast<const uint2*>(lo);
         }
         Z[j] += warp_sum(zs);
         A[j] += warp_sum(as);
       }
-      // 4. P(i) goes into pbuf[b]: PE(i - 2) must be done with it; a rescale also needs
-      //    PE(i - 1) done (s final up to tile i - 1).  With a given P nothing is written or
-      //    rescaled, but PE(i) still waits for this point, which keeps the MMA warp at most
-      //    one PE ahead of these waits.
+      // 5. a raised reference rescales s (final up to tile i - 1: PE(i - 1) done) before
+      //    PE(i) adds to it.  With a given P nothing is written or rescaled, but PE(i) still
+      //    waits for this point, which keeps the MMA warp at most one PE ahead of these waits.
       const bool rescale = !a.given && epi_any(need != 0);  // also publishes fac[]
-      bool fail = false;
-      if (rescale && i >= 1) fail = !mbar_wait(&pe_done[(i - 1) & 1], ((i - 1) >> 1) & 1, a.err);
-      else if (i >= 2) fail = !mbar_wait(&pe_done[b], ((i - 2) >> 1) & 1, a.err);
-      if (epi_any(fail)) { ok = false; break; }
-      tc_fence_after();
       if (rescale) {
+        if (epi_any(i >= 1 && !mbar_wait(&pe_done[(i - 1) & 1], ((i - 1) >> 1) & 1, a.err))) { ok = false; break; }
+        tc_fence_after();
         float fv[32];
 #pragma unroll
         for (int t = 0; t < 32; ++t) fv[t] = fac[t];
@@ -430,26 +441,11 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
         }
         tc_fence_before();
       }
-      uint8_t* pt = pbuf + b * kLmPBytes;
-#pragma unroll
-      for (int j = 0; j < 8 && !a.given; ++j) {
-        const int t = tw * 8 + j;
-        const bool live = t < a.T;
-        __align__(8) __nv_bfloat16 hi[4], lo[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float p = live ? pv[j][u] : 0.f;
-          hi[u] = f2bf(p);
-          lo[u] = f2bf(p - bf2f(hi[u]));
-        }
-        *reinterpret_cast<uint2*>(pt + p_offset(t, lane * 4)) = *reinterpret_cast<const uint2*>(hi);
-        *reinterpret_cast<uint2*>(pt + p_offset(32 + t, lane * 4)) = *reinterpret_cast<const uint2*>(lo);
-      }
       fence_proxy_async_smem();  // generic-proxy writes of P visible to the tensor cores
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_ready[b]);
     }
-    // 5. outputs of the cluster: s half (every CTA), statistics (rank 0)
+    // 6. outputs of the cluster: s half (every CTA), statistics (rank 0)
     if (ok && nt > 0) {
       const int last = nt - 1;
       if (et == 0) *flag = mbar_wait(&pe_done[last & 1], (last >> 1) & 1, a.err) ? 1 : 0;
