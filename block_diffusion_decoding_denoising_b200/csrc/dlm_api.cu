@@ -553,7 +553,7 @@ dlm_status launch_commit(Runner& r, const dlm_block_state& st, float tau, int mo
   ca.k = k;
   ca.use_cond = use_cond ? 1 : 0;
   ca.cond = h;
-  CU_LAUNCH(launch_k(k_commit, dim3(1), dim3(64), 0, r.s, ca));
+  CU_LAUNCH(launch_k(k_commit, dim3(1), dim3(kCommitThreads), 0, r.s, ca));
   return r.check();
 }
 
@@ -735,6 +735,7 @@ dlm_status dlm_ctx_create(const dlm_config* cfg, const dlm_weights* w, void* d_w
   if (e == cudaSuccess) e = (cudaError_t)gemm_init_attributes();
   if (e == cudaSuccess && fp4) e = (cudaError_t)gemm_fp4_init_attributes();
   if (e == cudaSuccess) e = (cudaError_t)attention_init_attributes();
+  if (e == cudaSuccess) e = (cudaError_t)ops_init_attributes();
   if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->cap_stream);
   if (e != cudaSuccess) {
     if (ctx->cap_stream) cudaStreamDestroy(ctx->cap_stream);
@@ -1144,7 +1145,7 @@ dlm_status dlm_commit(const float* d_maxprob, const int32_t* d_argmax, int32_t* 
   ca.tau = tau;
   ca.mode = commit_mode;
   ca.k = tpf_k;
-  CU_LAUNCH(launch_k(k_commit, dim3(1), dim3(64), 0, (cudaStream_t)stream, ca));
+  CU_LAUNCH(launch_k(k_commit, dim3(1), dim3(kCommitThreads), 0, (cudaStream_t)stream, ca));
   return cudaGetLastError() == cudaSuccess ? DLM_OK : DLM_ECUDA;
 }
 

@@ -381,6 +381,12 @@ int attention_init_attributes() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_bd_attention<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnSmem<128>::kBytes);
+  // the largest shared-memory carve-out, as the GEMMs (see ops_init_attributes)
+  const void* ks[] = {(const void*)k_bd_attention<32>, (const void*)k_bd_attention<64>,
+                      (const void*)k_bd_attention<128>, (const void*)k_attn_combine};
+  for (const void* k : ks)
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess) done = true;
   return (int)e;
 }

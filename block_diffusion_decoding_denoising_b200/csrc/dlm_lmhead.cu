@@ -631,6 +631,9 @@ cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_giv
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k_lmhead_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmSmem);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k_lmf_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmfSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_lmf_combine, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     attr = true;
   }

@@ -382,7 +382,7 @@ __global__ void k_rowstats_final(RowStatsArgs a) {
   }
 }
 
-// Commit rule for one block (one CTA, blockDim >= B).  Threshold mode: every uncommitted
+// Commit rule for one block (one CTA of kCommitThreads >= B threads).  Threshold mode: every uncommitted
 // position with maxprob >= tau, or if none qualifies the single uncommitted position with
 // the largest maxprob (ties -> lowest position).  Top-k mode: the min(k, remaining)
 // uncommitted positions of largest maxprob (ties -> lowest position).  Newly committed
@@ -428,10 +428,20 @@ __global__ void k_commit(CommitArgs a) {
     a.committed[i] = 1;
   }
   __syncthreads();
-  // committed positions (old and new) carry no residual into the next round
-  for (int r = 0; r < B; ++r) {
-    if (unc[r] && !sel[r]) continue;
-    for (int n = threadIdx.x; n < a.d; n += blockDim.x) a.s[(size_t)r * a.d + n] = 0.f;
+  // committed positions (old and new) carry no residual into the next round: every thread
+  // zeroes a strided share of those rows (float4 stores when s is 16-byte aligned)
+  if (((uintptr_t)a.s & 15) == 0 && (a.d & 3) == 0) {
+    const int d4 = a.d / 4;
+    float4* s4 = reinterpret_cast<float4*>(a.s);
+    for (int e = threadIdx.x; e < B * d4; e += blockDim.x) {
+      const int r = e / d4;
+      if (!unc[r] || sel[r]) s4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  } else {
+    for (int e = threadIdx.x; e < B * a.d; e += blockDim.x) {
+      const int r = e / a.d;
+      if (!unc[r] || sel[r]) a.s[e] = 0.f;
+    }
   }
   int left = (i < B && unc[i] && !sel[i]) ? 1 : 0;
   int nleft = __syncthreads_count(left);
@@ -613,6 +623,26 @@ __global__ void k_nvfp4_dequant_bf16(const uint8_t* codes, const uint8_t* scales
   uint4* dst = reinterpret_cast<uint4*>(out + b * 16);
   dst[0] = reinterpret_cast<const uint4*>(o)[0];
   dst[1] = reinterpret_cast<const uint4*>(o)[1];
+}
+
+// Every kernel of a round prefers the largest shared-memory carve-out, the one the GEMMs run
+// with: an SM can then host a GEMM CTA beside the CTAs of the kernel before it without
+// reconfiguring its L1 / shared-memory split, so the GEMM's early weight loads (issued before
+// its dependency wait) overlap that kernel.
+int ops_init_attributes() {
+  static bool done = false;
+  if (done) return 0;
+  const void* ks[] = {(const void*)k_finish_qkv,  (const void*)k_finish_silu,   (const void*)k_finish_store,
+                      (const void*)k_resid_norm,  (const void*)k_act_quant,     (const void*)k_to_bf16,
+                      (const void*)k_rowstats_part, (const void*)k_rowstats_final, (const void*)k_commit,
+                      (const void*)k_block_init,  (const void*)k_block_finish};
+  for (const void* k : ks) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return (int)e;
+  }
+  done = true;
+  return 0;
 }
 
 }  // namespace dlm

@@ -59,6 +59,10 @@ struct ActQuantArgs {
   float* sx;
 };
 
+int ops_init_attributes();
+
+constexpr int kCommitThreads = 256;  // k_commit's block (B <= 64)
+
 struct CommitArgs {
   const float* maxprob;
   const int32_t* argmax;
