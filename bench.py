@@ -34,7 +34,7 @@ TPF_K = 11
 TAU = 0.9
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3)
@@ -50,7 +50,7 @@ def parse():
     # (same kernels; ncu cannot profile kernel nodes of graphs with conditional nodes)
     ap.add_argument("--eager", action="store_true")
     ap.add_argument("--pdl", type=int, default=1, help=argparse.SUPPRESS)
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def peaks():
@@ -149,6 +149,22 @@ def oracle_sample(cfg, seconds=10.0):
         if el >= seconds:
             break
     return el / reps * nl, reps, O.hw_threads()
+
+
+def max_over_ranks(x, world, dev):
+    """The largest of a float over all ranks (the slowest rank sets a multi-GPU time)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, units_per_rank, seconds):
+    """Units all ranks processed per second of the (max-over-ranks) time."""
+    return world * units_per_rank / seconds
 
 
 def reference_arm(args, cfg):
@@ -462,15 +478,12 @@ def main():
     barrier()
     ms = ev0.elapsed_time(ev1)
     ck = clocks.stop()
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     rb = rounds_out.cpu().numpy()
     assert np.all(rb[:, 1] == 0), "device status %s" % rb[:, 1]
     rounds_per_step = int(rb[:, 0].sum())
     ms_step = ms / args.steps
-    tps = world * GEN / (ms_step / 1e3)
+    tps = whole_job_rate(world, GEN, ms_step / 1e3)
     if args.case == "quick":
         if rank == 0:
             print(json.dumps({"case": "quick", "tokens_per_s": tps, "ms_per_step": ms_step,
@@ -556,11 +569,8 @@ def main():
         if i >= args.warmup:
             e2e_times.append(t1 - t0)
     e2e_s = max(e2e_times) if e2e_times else float("nan")
-    if world > 1:
-        t = torch.tensor([e2e_s], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
-    e2e_tps = world * GEN / e2e_s
+    e2e_s = max_over_ranks(e2e_s, world, dev)
+    e2e_tps = whole_job_rate(world, GEN, e2e_s)
 
     weight_bytes = sum(v.numel() * 2 for k, v in w.items() if k != "layers") + sum(
         v.numel() * 2 for l in w["layers"] for v in l.values())
