@@ -201,6 +201,52 @@ def test_linear_exact_on_integers_and_matches_matmul():
     np.testing.assert_allclose(O.linear(x2, W2), x2 @ gen.bf16_to_f64(W2).T, rtol=1e-12, atol=1e-12)
 
 
+def _on_grid_rows(rows, cols, seed):
+    """Rows whose 16-element blocks are e2m1 grid points x an e4m3 block scale x 2^-10, with a
+    block at 6 x 448 x 2^-10 in every row: the NVFP4 round trip reproduces them exactly
+    (row scale 2^-10, block scales exact)."""
+    grid = np.array([O.e2m1_value(c) for c in range(16)])
+    rng = np.random.default_rng(seed)
+    sig_choices = np.array([448.0, 1.0, 2.0, 0.5, 64.0, 2.0 ** -6, 8.0, 16.0])
+    out = np.zeros((rows, cols))
+    for r in range(rows):
+        for b in range(cols // 16):
+            blk = grid[rng.integers(0, 16, 16)]
+            blk[0] = 6.0
+            sig = 448.0 if b == 0 else sig_choices[rng.integers(0, len(sig_choices))]
+            out[r, b * 16:(b + 1) * 16] = blk * sig * 2.0 ** -10
+    return out
+
+
+def test_linear_nvfp4_exact_on_grid_operands():
+    # weights and activations both exactly representable: the NVFP4 linear is the exact
+    # fp64 product of the two (activation row scales, block scales and codes all exact)
+    K, N = 64, 24
+    w = _on_grid_rows(N, K, 7)
+    codes, scales, S = O.nvfp4_quantize(w.astype(np.float32))
+    assert S == 2.0 ** -10
+    Wq = dict(codes=codes, scales=scales, tscale=S, rows=N, cols=K)
+    x = _on_grid_rows(3, K, 8)
+    np.testing.assert_array_equal(O.linear(x, Wq, act_fp4=True), x @ w.T)
+    # weights alone: the activations stay fp64
+    xr = gen.normal_np(9, 3 * K).reshape(3, K)
+    np.testing.assert_allclose(O.linear(xr, Wq, act_fp4=False), xr @ w.T, rtol=1e-13, atol=1e-15)
+
+
+def test_linear_nvfp4_quantizes_each_activation_row_by_itself():
+    # act_fp4 = quantize every row with its own row scale, then the product with the
+    # dequantized weights (a second row scaled by 2^20 changes nothing in the first)
+    K, N = 64, 16
+    w = gen.normal_np(10, N * K, 0.02).reshape(N, K).astype(np.float32)
+    codes, scales, S = O.nvfp4_quantize(w)
+    Wq = dict(codes=codes, scales=scales, tscale=S, rows=N, cols=K)
+    wd = O.nvfp4_dequant(codes, scales, S, N, K)
+    x = gen.normal_np(11, 2 * K).reshape(2, K)
+    x[1] *= 2.0 ** 20
+    xq = np.stack([O.nvfp4_dequant(*O.nvfp4_quantize(x[t:t + 1].astype(np.float32)), 1, K)[0] for t in range(2)])
+    np.testing.assert_allclose(O.linear(x, Wq, act_fp4=True), xq @ wd.T, rtol=1e-12, atol=0)
+
+
 def test_rmsnorm_constant_vector():
     g = bits(np.linspace(0.5, 2.0, 16))
     for c in (3.0, -0.25):
