@@ -191,6 +191,26 @@ def test_lmhead_uniform_p_gives_column_mean_and_logits_match_matmul():
     np.testing.assert_allclose(out2["s"], p @ Ef, rtol=1e-10, atol=1e-14)
 
 
+def test_lmhead_nvfp4_uses_the_dequantized_embedding():
+    # NVFP4 E: a one-hot P reproduces the dequantized row (s = P E with E = q sigma S), and
+    # with grid-representable x and E the logits are their exact product
+    V, d = 96, 64
+    Eg = _on_grid_rows(V, d, 21)
+    codes, scales, S = O.nvfp4_quantize(Eg.astype(np.float32))
+    Eq = dict(codes=codes, scales=scales, tscale=S, rows=V, cols=d)
+    x = _on_grid_rows(2, d, 22)
+    P = np.zeros((2, V))
+    P[0, 5] = 1.0
+    P[1, 95] = 1.0
+    out = O.lmhead(x, Eq, p_given=P, act_fp4=True, want_logits=True)
+    np.testing.assert_array_equal(out["s"][0], Eg[5])
+    np.testing.assert_array_equal(out["s"][1], Eg[95])
+    np.testing.assert_array_equal(out["logits"], x @ Eg.T)
+    ref = O.rowstats(x @ Eg.T)
+    np.testing.assert_array_equal(out["argmax"], ref["argmax"])
+    np.testing.assert_allclose(out["lse"], ref["lse"], rtol=1e-12)
+
+
 # ------------------------------------------------------------------ layers
 def test_linear_exact_on_integers_and_matches_matmul():
     W = bits(np.arange(-6, 6, dtype=np.float64).reshape(3, 4))
