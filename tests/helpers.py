@@ -3,7 +3,7 @@ import numpy as np
 
 # Float parity bar: |gpu - ref| <= RTOL * (|ref| + rms(ref)) element by element, i.e. a
 # relative error of 2e-2 with a floor at the tensor's RMS so that entries near zero are
-# judged on the tensor's scale.  bf16 path: 2e-2; NVFP4 path: 6e-2.
+# compared on the tensor's scale.  bf16 path: 2e-2; NVFP4 path: 6e-2.
 RTOL_BF16 = 2e-2
 RTOL_NVFP4 = 6e-2
 
