@@ -52,7 +52,7 @@ typedef int dlm_status;
 #define DLM_ECUDA 4         /* a CUDA runtime/driver error; see dlm_last_error */
 #define DLM_EROUNDCAP 5     /* a block reached B rounds with positions uncommitted */
 #define DLM_ETIMEOUT 6      /* a device-side bounded wait gave up (kernel returned early) */
-#define DLM_EUNSUPPORTED 7  /* shape or format this build does not handle */
+#define DLM_EUNSUPPORTED 7  /* shape or format the library does not handle */
 
 #define DLM_COMMIT_THRESHOLD 0 /* commit max-prob >= tau, at least one per round */
 #define DLM_COMMIT_TOPK 1      /* commit the top min(k, remaining) by max-prob */
