@@ -237,14 +237,33 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
       bool finisher = true;
       if (nslots > 1 || e.op == EPI_PARTIAL) {
         float* dst = tile_part + (size_t)slot * kTileM * TP;
-#pragma unroll 1
-        for (int cb = 0; cb < ncb; ++cb) {
-          load_block(taddr, cb);
+        float* const blk = dst - row;  // the (tile, slot) block: [TP][128] fp32, contiguous
+        if (e.op == EPI_PARTIAL && ncb == 1 && ((uintptr_t)blk & 15) == 0) {
+          // 32 tokens: the 16 KB block goes out through shared memory as one bulk copy
+          load_block(taddr, 0);
+          tc_fence_before();
+          mbar_arrive(&acc_empty[acc]);  // the accumulator can take the next tile now
+          if (et == 0) bulk_wait_read_all();  // the previous segment's copy has left the buffer
+          epi_sync();
+          float* const stg = &xch[0][0];  // [32][128] fp32 inside the exchange buffer
 #pragma unroll
-          for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * kTileM] = v[j];
+          for (int j = 0; j < 32; ++j) stg[j * kTileM + row] = v[j];
+          fence_async_shared();
+          epi_sync();
+          if (et == 0) {
+            bulk_store_s2g(blk, smem_u32(stg), 32 * kTileM * 4);
+            bulk_commit();
+          }
+        } else {
+#pragma unroll 1
+          for (int cb = 0; cb < ncb; ++cb) {
+            load_block(taddr, cb);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) dst[(size_t)(cb * 32 + j) * kTileM] = v[j];
+          }
+          tc_fence_before();
+          mbar_arrive(&acc_empty[acc]);  // the accumulator can take the next tile now
         }
-        tc_fence_before();
-        mbar_arrive(&acc_empty[acc]);  // the accumulator can take the next tile now
         if (e.op == EPI_PARTIAL) {
           finisher = false;
         } else {
@@ -277,6 +296,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       u = seg_end;
     }
+    if (et == 0) bulk_wait_all();  // partial sums written before the CTA ends
   }
   tc_fence_before();
   __syncthreads();
