@@ -528,3 +528,128 @@ def test_qmargin_pins():
     assert abs(qm[0] - 16.0 / 432.0) < 1e-5, qm
     assert qm[1] < 1e-5 and qm[2] < 1e-5, qm
     assert np.all(np.isinf(qm_off))
+
+
+# ------------------------------------------------------------------ layer composition
+# Closed forms of one pre-norm layer (reading R6) with structured weights: scaled identity
+# and permutation blocks make every sub-block's output a formula in the input row, so that
+# a slip in the forward pass's composition (silu on the wrong operand, a sigmoid for the
+# SiLU, the gate and up rows exchanged, the wrong norm gain, RoPE applied to v or missing
+# on q, the q/k/v rows taken in the wrong order, W_o transposed, a dropped residual) moves
+# the result far outside the rounding error of the fp64 oracle.
+def _closed_form_layer_setup(tiny):
+    cfg, w = tiny
+    d, F, hd = cfg["d"], cfg["ffn"], cfg["head_dim"]
+    ga = 0.5 + 0.25 * (np.arange(d) % 4)           # attn_norm gains (bf16-exact)
+    gm = 2.0 - 0.25 * (np.arange(d) % 5)           # mlp_norm gains
+    gf = 1.0 + 0.125 * (np.arange(d) % 3)          # final_norm gains
+    lw = dict(w["layers"][0], attn_norm=bits(ga), mlp_norm=bits(gm))
+    w2 = dict(w, final_norm=bits(gf))
+    return cfg, w2, lw, ga, gm, gf
+
+
+def _rms(x, g, eps):
+    return x / np.sqrt(np.mean(x * x) + eps) * g
+
+
+def _silu(x):
+    return x / (1.0 + np.exp(-x))
+
+
+def test_pin_mlp_sub_block_closed_form(tiny):
+    # W_qkv = 0: q = k = v = 0, the attention output is the mean of zero values, so W_o
+    # (left random) adds nothing and the MLP sees RMSNorm(E[x]) * g_mlp.  With
+    # W_gate = a [I 0], W_up = b [P 0] (P a permutation) and W_down = c [I 0]:
+    #   h = E[x] + c * silu(a xn) * (b xn[pi]),  xf = RMSNorm(h) * g_final.
+    cfg, w2, lw, ga, gm, gf = _closed_form_layer_setup(tiny)
+    d, F = cfg["d"], cfg["ffn"]
+    a, b, c = 2.0, 1.5, 0.75
+    pi = (np.arange(d) * 7 + 3) % d                 # a permutation of 0..d-1 (7 is odd, d = 64)
+    Wg = np.zeros((F, d)); Wg[np.arange(d), np.arange(d)] = a
+    Wu = np.zeros((F, d)); Wu[np.arange(d), pi] = b
+    Wd = np.zeros((d, F)); Wd[np.arange(d), np.arange(d)] = c
+    lw.update(w_qkv=bits(np.zeros((cfg["n_q_heads"] + 2 * cfg["n_kv_heads"]) * cfg["head_dim"] * d)
+                         .reshape(-1, d)), w_gate=bits(Wg), w_up=bits(Wu), w_down=bits(Wd))
+    w2["layers"] = [lw]
+    m = O.OracleModel(cfg, w2, act_round=False)
+    E = gen.bf16_to_f64(w2["embed"])
+    toks = np.array([3, 77, 200, 5], np.int32)
+    xf = m.forward(toks, None, 7)
+    eps = cfg["rms_eps"]
+    for i, t in enumerate(toks):
+        xn = _rms(E[t], gm, eps)
+        h = E[t] + c * _silu(a * xn) * (b * xn[pi])
+        np.testing.assert_allclose(xf[i], _rms(h, gf, eps), rtol=1e-11, atol=1e-13)
+    # the gate and up roles are not interchangeable here: silu(u) * g is far away
+    xn = _rms(E[toks[0]], gm, eps)
+    swapped = _rms(E[toks[0]] + c * _silu(b * xn[pi]) * (a * xn), gf, eps)
+    assert np.abs(swapped - xf[0]).max() > 1e-3
+
+
+def _rope_np(x, pos, base):
+    """NeoX rotate-half rotation of one head vector (pairs j, j + hd/2)."""
+    half = len(x) // 2
+    th = base ** (-2.0 * np.arange(half) / len(x))
+    c, s = np.cos(pos * th), np.sin(pos * th)
+    return np.concatenate([x[:half] * c - x[half:] * s, x[:half] * s + x[half:] * c])
+
+
+def test_pin_attention_sub_block_closed_form(tiny):
+    # One block token at position p over an injected prefix of p keys (layer 0, one kv head
+    # shared by both q heads).  Structured W_qkv rows (q heads, then the k head, then the v
+    # head), each reading a different slice of xn = RMSNorm(E[x]) * g_attn:
+    #   q0 = al xn[0:32], q1 = be xn[32:64], k = xn[16:48], v = ga_ xn[perm]
+    # RoPE rotates q0, q1 and k at position p, not v.  W_o is a scaled cyclic shift
+    # ((W_o o)[n] = de o[(n+1) % 64]) and W_down = 0, so
+    #   h = E[x] + de shift(concat(o0, o1)),  o_h = softmax(rope(q_h) . K / sqrt(32)) V
+    # with K, V the injected rows followed by the block's own (rope(k), v).
+    cfg, w2, lw, ga, gm, gf = _closed_form_layer_setup(tiny)
+    d, hd, F = cfg["d"], cfg["head_dim"], cfg["ffn"]
+    Hq, Hkv = cfg["n_q_heads"], cfg["n_kv_heads"]
+    assert (Hq, Hkv, hd, d) == (2, 1, 32, 64)
+    al, be, ga_, de = 1.5, 0.75, 2.0, 0.5
+    perm = (np.arange(hd) * 5 + 11) % d
+    Wqkv = np.zeros(((Hq + 2 * Hkv) * hd, d))
+    Wqkv[np.arange(32), np.arange(32)] = al
+    Wqkv[32 + np.arange(32), 32 + np.arange(32)] = be
+    Wqkv[64 + np.arange(32), 16 + np.arange(32)] = 1.0
+    Wqkv[96 + np.arange(32), perm] = ga_
+    Wo = np.zeros((d, Hq * hd))
+    Wo[np.arange(d), (np.arange(d) + 1) % d] = de
+    lw.update(w_qkv=bits(Wqkv), w_o=bits(Wo), w_down=bits(np.zeros((d, F))))
+    w2["layers"] = [lw]
+    m = O.OracleModel(cfg, w2, act_round=False)
+    p, base, eps = 3, cfg["rope_theta"], cfg["rms_eps"]
+    Kp = gen.normal_np(61, p * hd).reshape(p, hd)
+    Vp = gen.normal_np(62, p * hd).reshape(p, hd)
+    m.kc[0, 0, :p] = Kp
+    m.vc[0, 0, :p] = Vp
+    tok = 123
+    xf = m.forward(np.array([tok], np.int32), None, p)
+    E = gen.bf16_to_f64(w2["embed"])
+    xn = _rms(E[tok], ga, eps)
+    q = [_rope_np(al * xn[0:32], p, base), _rope_np(be * xn[32:64], p, base)]
+    k = _rope_np(xn[16:48], p, base)
+    v = ga_ * xn[perm]
+    # the block's K/V rows in the cache: k rotated, v as projected
+    np.testing.assert_allclose(m.kc[0, 0, p], k, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(m.vc[0, 0, p], v, rtol=1e-12, atol=1e-14)
+    K = np.vstack([Kp, k])
+    V = np.vstack([Vp, v])
+    o = []
+    for qh in q:
+        sc = K @ qh / np.sqrt(hd)
+        e = np.exp(sc - sc.max())
+        o.append(e @ V / e.sum())
+    oc = np.concatenate(o)
+    h = E[tok] + de * oc[(np.arange(d) + 1) % d]
+    np.testing.assert_allclose(xf[0], _rms(h, gf, eps), rtol=1e-11, atol=1e-13)
+    # unrotated queries (a plausible slip) give a visibly different row
+    o_bad = []
+    for qh in (al * xn[0:32], be * xn[32:64]):
+        sc = K @ qh / np.sqrt(hd)
+        e = np.exp(sc - sc.max())
+        o_bad.append(e @ V / e.sum())
+    ob = np.concatenate(o_bad)
+    bad = _rms(E[tok] + de * ob[(np.arange(d) + 1) % d], gf, eps)
+    assert np.abs(bad - xf[0]).max() > 1e-4
