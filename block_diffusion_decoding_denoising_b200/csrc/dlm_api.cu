@@ -982,6 +982,29 @@ dlm_status dlm_gemm_bf16x2(const void* d_x2, const void* d_w, float* d_y, int T,
   return gemm_op(d_x2, d_w, d_y, T, N, K, d_scratch, scratch_bytes, stream, true);
 }
 
+size_t dlm_gemm_f32_scratch_size(int T, int N, int K) {
+  if (T < 1 || T > kMaxSplitTokens || K < 1) return 0;
+  return dlm_gemm_scratch_size(T, N, K) + align256((size_t)2 * split_pad(T) * K * 2);
+}
+
+dlm_status dlm_gemm_f32(const float* d_x, const void* d_w, float* d_y, int T, int N, int K, void* d_scratch,
+                        size_t scratch_bytes, void* stream) {
+  dlm_ctx* ctx = nullptr;
+  if (!d_x || !d_w || !d_y || !d_scratch || T < 1 || T > kMaxSplitTokens || N < 1 || K < 64 || K % 8)
+    return DLM_EINVAL;
+  if (scratch_bytes < dlm_gemm_f32_scratch_size(T, N, K)) return DLM_ENOMEM_WS;
+  cudaStream_t s = (cudaStream_t)stream;
+  // the split pair x = hi + lo goes after the GEMM's own scratch: rows [0, T) high halves,
+  // rows [pad, pad + T) low halves, the padding rows zero
+  const size_t gemm_sc = dlm_gemm_scratch_size(T, N, K);
+  const long pad = split_pad(T);
+  __nv_bfloat16* x2 = (__nv_bfloat16*)((uint8_t*)d_scratch + gemm_sc);
+  CU(cudaMemsetAsync(x2, 0, (size_t)2 * pad * K * 2, s));
+  const long n = (long)T * K;
+  CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, d_x, x2, n, pad * K));
+  return gemm_op(x2, d_w, d_y, T, N, K, d_scratch, gemm_sc, stream, true);
+}
+
 size_t dlm_lmhead_scratch_size(int B, int V, int d) {
   const int nch = (V + kRowChunk - 1) / kRowChunk;
   size_t unfused = op_header() + op_counters(V > d ? V : d) + align256(lmhead_partial(B, V, d)) +
@@ -1117,8 +1140,7 @@ dlm_status dlm_bd_attention(const void* d_q, const void* d_k_cache, const void* 
   a.max_splits = attention_max_splits(T, Hq, Hkv, max_ctx);
   a.part_o = (float*)(sc + op_header());
   a.part_ml = a.part_o + (size_t)a.max_splits * T * Hq * hd;
-  a.err = (int*)sc;
-  CU(cudaMemsetAsync(sc, 0, 4, s));
+  a.err = nullptr;  // the attention kernels have no waits and report nothing on the device
   CU(attention_launch(a, s));
   return DLM_OK;
 }

@@ -372,8 +372,8 @@ size_t attention_scratch_bytes(int T, int Hq, int hd, int max_splits) {
 }
 
 int attention_init_attributes() {
-  static bool done = false;
-  if (done) return 0;
+  static PerDeviceOnce once;
+  return once_on_current_device(once, [] {
   cudaError_t e = cudaFuncSetAttribute(k_bd_attention<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        AttnSmem<32>::kBytes);
   if (e == cudaSuccess)
@@ -387,8 +387,8 @@ int attention_init_attributes() {
   for (const void* k : ks)
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
-  if (e == cudaSuccess) done = true;
   return (int)e;
+  });
 }
 
 int attention_split_cap(int T, int max_ctx) {

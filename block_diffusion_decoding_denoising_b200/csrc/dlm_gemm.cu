@@ -436,17 +436,17 @@ static cudaError_t set_smem_attr() {
   return cudaFuncSetAttribute(k_gemm_tc<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmCfg<NT>::kSmem);
 }
 
-// Sets the dynamic shared-memory limits of every GEMM instantiation once per process
-// (must happen outside stream capture).
+// Sets the dynamic shared-memory limits of every GEMM instantiation once per device (must
+// happen outside stream capture).
 int gemm_init_attributes() {
-  static bool done = false;
-  if (done) return 0;
-  cudaError_t e = set_smem_attr<32>();
-  if (e == cudaSuccess) e = set_smem_attr<64>();
-  if (e == cudaSuccess) e = set_smem_attr<128>();
-  if (e == cudaSuccess) e = set_smem_attr<256>();
-  if (e == cudaSuccess) done = true;
-  return (int)e;
+  static PerDeviceOnce once;
+  return once_on_current_device(once, [] {
+    cudaError_t e = set_smem_attr<32>();
+    if (e == cudaSuccess) e = set_smem_attr<64>();
+    if (e == cudaSuccess) e = set_smem_attr<128>();
+    if (e == cudaSuccess) e = set_smem_attr<256>();
+    return (int)e;
+  });
 }
 
 cudaError_t gemm_launch(const GemmPlan& p, int* d_err, cudaStream_t s) {

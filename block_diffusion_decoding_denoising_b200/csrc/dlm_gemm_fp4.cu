@@ -442,11 +442,10 @@ cudaError_t gemm_fp4_launch(const GemmF4Plan& p, int* d_err, cudaStream_t s) {
 }
 
 int gemm_fp4_init_attributes() {
-  static bool done = false;
-  if (done) return 0;
-  cudaError_t e = cudaFuncSetAttribute(k_gemm_nvf4, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4Smem);
-  if (e == cudaSuccess) done = true;
-  return (int)e;
+  static PerDeviceOnce once;
+  return once_on_current_device(once, [] {
+    return (int)cudaFuncSetAttribute(k_gemm_nvf4, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4Smem);
+  });
 }
 
 }  // namespace dlm

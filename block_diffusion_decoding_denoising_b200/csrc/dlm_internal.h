@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include "../../include/dlm.h"
+#include "dlm_per_device.h"
 
 namespace dlm {
 
@@ -50,6 +51,17 @@ inline cudaError_t launch_k_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 bl
   cfg.attrs = attr;
   cfg.numAttrs = g_pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Runs init() once on the calling thread's current device (see PerDeviceOnce) and returns a
+// cudaError_t value: kernel attributes and symbol addresses are per device.
+template <class F>
+inline int once_on_current_device(PerDeviceOnce& once, F init) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return (int)e;
+  const int r = once.run(dev, init);
+  return r == PerDeviceOnce::kBadDevice ? (int)cudaErrorInvalidDevice : r;
 }
 
 constexpr int kSMs = 148;        // B200 streaming multiprocessors

@@ -627,15 +627,18 @@ bool lmhead_fused_supported(int T, int d) {
 cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_given, int T, int V, int d,
                                 int mask_id, dlm_row_stats stats, float* s, void* scratch, int* d_err,
                                 cudaStream_t st, char* err, size_t errlen) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_lmhead_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmSmem);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_lmf_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmfSmem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_lmf_combine, cudaFuncAttributePreferredSharedMemoryCarveout,
-                               (int)cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    attr = true;
+  {
+    static PerDeviceOnce once;
+    const int r = once_on_current_device(once, [] {
+      cudaError_t e = cudaFuncSetAttribute(k_lmhead_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmSmem);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_lmf_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmfSmem);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_lmf_combine, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+      return (int)e;
+    });
+    if (r != 0) return (cudaError_t)r;
   }
   LmfArgs a{};
   a.V = V;

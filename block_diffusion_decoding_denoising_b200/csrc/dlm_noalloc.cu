@@ -12,45 +12,47 @@
 //  - calls whose split-KV partials do not fit in kNoAllocScratchBytes are rejected with
 //    DLM_ENOMEM_WS before anything is launched;
 //  - the first call on a device looks up the array's device address
-//    (cudaGetSymbolAddress) and sets the kernels' shared-memory limits; make that first
-//    call before any stream capture is started on that device;
-//  - the status word at the start of the array must be zero when the kernels run: every
-//    call clears it with a cudaMemsetAsync on the caller's stream; the partial results
-//    need no initial value;
+//    (cudaGetSymbolAddress) and sets the kernels' shared-memory limits on that device;
+//    make that first call before any stream capture is started on that device;
+//  - the split partials need no initial value (every element read by the merge is written
+//    first by the same call), so a call launches the attention kernels and nothing else;
 //  - the array is shared by every call on a device: calls that may overlap in time (on
 //    different streams, or from several host threads) race on it and must be serialised
 //    by the caller.
 #include <cuda_runtime.h>
+
+#include <atomic>
 
 #include "dlm_internal.h"
 
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
-constexpr size_t kNoAllocStatusBytes = 256;                // status word, padded
-constexpr int kNoAllocMaxDevices = 64;
+constexpr size_t kNoAllocHeaderBytes = 256;                // unused head of the array (alignment)
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch per device, filled by the first call on each device
-// (two threads racing on the first call store the same value).
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+// Device address of g_noalloc_scratch per device (the name is only a host-side handle in
+// host code), looked up by the first call on each device together with the kernels'
+// attributes on that device.
+std::atomic<void*> g_noalloc_ptr[dlm::kMaxDevices];
+dlm::PerDeviceOnce g_noalloc_once;
 
 cudaError_t noalloc_scratch(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
-  if (!g_noalloc_ptr[dev]) {
+  const int r = g_noalloc_once.run(dev, [dev] {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    e = (cudaError_t)dlm::attention_init_attributes();
-    if (e != cudaSuccess) return e;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
-  return cudaSuccess;
+    cudaError_t e2 = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e2 == cudaSuccess) e2 = (cudaError_t)dlm::attention_init_attributes();
+    if (e2 == cudaSuccess) g_noalloc_ptr[dev].store(p, std::memory_order_release);
+    return (int)e2;
+  });
+  if (r == dlm::PerDeviceOnce::kBadDevice) return cudaErrorInvalidDevice;
+  if (r != 0) return (cudaError_t)r;
+  *out = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  return *out ? cudaSuccess : cudaErrorInvalidDevice;
 }
 
 }  // namespace
@@ -64,7 +66,7 @@ dlm_status dlm_bd_attention_noalloc(const void* d_q, const void* d_k_cache, cons
       !(hd == 32 || hd == 64 || hd == 128) || L + T > max_ctx)
     return DLM_EINVAL;
   const int splits = dlm::attention_max_splits(T, Hq, Hkv, max_ctx);
-  if (dlm::attention_scratch_bytes(T, Hq, hd, splits) > kNoAllocScratchBytes - kNoAllocStatusBytes)
+  if (dlm::attention_scratch_bytes(T, Hq, hd, splits) > kNoAllocScratchBytes - kNoAllocHeaderBytes)
     return DLM_ENOMEM_WS;
   void* base = nullptr;
   if (noalloc_scratch(&base) != cudaSuccess) return DLM_ECUDA;
@@ -83,10 +85,9 @@ dlm_status dlm_bd_attention_noalloc(const void* d_q, const void* d_k_cache, cons
   a.pos0 = L;
   a.causal = causal ? 1 : 0;
   a.max_splits = splits;
-  a.part_o = (float*)(sc + kNoAllocStatusBytes);
+  a.part_o = (float*)(sc + kNoAllocHeaderBytes);
   a.part_ml = a.part_o + (size_t)splits * T * Hq * hd;
-  a.err = (int*)sc;
-  if (cudaMemsetAsync(sc, 0, sizeof(int), s) != cudaSuccess) return DLM_ECUDA;
+  a.err = nullptr;
   if (dlm::attention_launch(a, s) != cudaSuccess) return DLM_ECUDA;
   return DLM_OK;
 }

@@ -630,8 +630,8 @@ __global__ void k_nvfp4_dequant_bf16(const uint8_t* codes, const uint8_t* scales
 // reconfiguring its L1 / shared-memory split, so the GEMM's early weight loads (issued before
 // its dependency wait) overlap that kernel.
 int ops_init_attributes() {
-  static bool done = false;
-  if (done) return 0;
+  static PerDeviceOnce once;
+  return once_on_current_device(once, [] {
   const void* ks[] = {(const void*)k_finish_qkv,  (const void*)k_finish_silu,   (const void*)k_finish_store,
                       (const void*)k_resid_norm,  (const void*)k_act_quant,     (const void*)k_to_bf16,
                       (const void*)k_rowstats_part, (const void*)k_rowstats_final, (const void*)k_commit,
@@ -641,8 +641,8 @@ int ops_init_attributes() {
                                          (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return (int)e;
   }
-  done = true;
   return 0;
+  });
 }
 
 }  // namespace dlm

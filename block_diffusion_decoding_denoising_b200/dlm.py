@@ -101,6 +101,9 @@ def lib():
         L.dlm_gemm_bf16.argtypes = [p, p, p, i, i, i, p, z, p]
         L.dlm_gemm_bf16x2.argtypes = [p, p, p, i, i, i, p, z, p]
         L.dlm_split_pad.argtypes = [i]
+        L.dlm_gemm_f32_scratch_size.restype = z
+        L.dlm_gemm_f32_scratch_size.argtypes = [i, i, i]
+        L.dlm_gemm_f32.argtypes = [p, p, p, i, i, i, p, z, p]
         L.dlm_lmhead_scratch_size.restype = z
         L.dlm_lmhead_scratch_size.argtypes = [i, i, i]
         L.dlm_lmhead_rowstats.argtypes = [p, p, i, i, i, i, p, RowStats, p, p, z, p]
@@ -167,19 +170,17 @@ def gemm_bf16(x, w, stream=None):
 
 
 def gemm_bf16x2(x, w, stream=None):
-    """y[T][N] fp32 = x[T][K] (fp32, carried as a bf16 hi + lo pair) @ w[N][K]^T (bf16)."""
+    """y[T][N] fp32 = x[T][K] (fp32, split by the library into a bf16 hi + lo pair) @ w[N][K]^T
+    (bf16): dlm_gemm_f32."""
     import torch
     T, K = x.shape
     N = w.shape[0]
-    pad = lib().dlm_split_pad(T)
-    x2 = torch.zeros((2 * pad, K), dtype=torch.bfloat16, device=x.device)
-    hi = x.to(torch.bfloat16)
-    x2[:T] = hi
-    x2[pad:pad + T] = (x - hi.float()).to(torch.bfloat16)
     y = torch.empty((T, N), dtype=torch.float32, device=x.device)
-    n = lib().dlm_gemm_scratch_size(T, N, K)
+    n = lib().dlm_gemm_f32_scratch_size(T, N, K)
+    if n == 0:
+        raise DlmError(DLM_EINVAL, "unsupported gemm shape")
     sc = _scratch(n, x.device)
-    _check(lib().dlm_gemm_bf16x2(_ptr(x2), _ptr(w), _ptr(y), T, N, K, _ptr(sc), n, _stream(stream)))
+    _check(lib().dlm_gemm_f32(_ptr(x.contiguous()), _ptr(w), _ptr(y), T, N, K, _ptr(sc), n, _stream(stream)))
     return y
 
 

@@ -165,6 +165,10 @@ dlm_status dlm_block_init(dlm_ctx* ctx, const dlm_block_state* st, void* stream)
  * DLM_COMMIT_THRESHOLD, tpf_k by DLM_COMMIT_TOPK. */
 dlm_status dlm_round(dlm_ctx* ctx, const dlm_block_state* st, float tau, int commit_mode,
                      int tpf_k, void* stream);
+/*   [blog "ORL: diffusion LLMs get a learnable 'tokens per forward'", "What shipped": a
+ *   round predicts the still-unresolved positions and feeds its distribution back through
+ *   the tied embedding ("On-policy residual learning"); card "QwenDLM-4B-ORL", "The paper's
+ *   evaluation pipeline": SDARPrefixKV attention, SDAR_FUSED_ROW_STATS, SDAR_COMMIT_GRAPH] */
 
 /* Clean forward of a committed block (s = 0, no LM head) writing its K/V to rows
  * [L, L+B); then L += B.  d_tokens int32 [B]. */
@@ -177,6 +181,9 @@ dlm_status dlm_kv_fill(dlm_ctx* ctx, const int32_t* d_tokens, void* stream);
  * is instantiated on first use per (commit mode, tau, k) and reused. */
 dlm_status dlm_decode_block(dlm_ctx* ctx, float tau, int commit_mode, int tpf_k,
                             int32_t* d_tokens_out, int32_t* d_rounds_out, void* stream);
+/*   [blog, "What shipped", "dlmrt, the inference engine": one CUDA graph per block with a
+ *   conditional node deciding after each round whether to go on; the host launches the
+ *   block and reads back tokens] */
 
 /* Host-level generation: copies the prompt to the device, prefills it at L = 0, decodes
  * ceil(max_new / B) blocks with dlm_decode_block, reading each block's tokens back, and
@@ -186,6 +193,8 @@ dlm_status dlm_decode_block(dlm_ctx* ctx, float tau, int commit_mode, int tpf_k,
 dlm_status dlm_generate(dlm_ctx* ctx, const int32_t* h_prompt, int prompt_len, int max_new,
                         float tau, int commit_mode, int tpf_k, int32_t* h_tokens_out,
                         int32_t* h_rounds_per_block, dlm_timing* h_timing, void* stream);
+/*   [card "QwenDLM-4B-ORL", usage section: generate(prompt, max_new_tokens) on one request;
+ *   blog, "What shipped": block-wise decoding over a prefix KV cache] */
 
 /* ---------------------------------------------------------------- single operations
  * Stand-alone entry points of the kernels one round is made of, used by the parity tests
@@ -206,6 +215,12 @@ dlm_status dlm_gemm_bf16(const void* d_x, const void* d_w, float* d_y, int T, in
 int dlm_split_pad(int T);
 dlm_status dlm_gemm_bf16x2(const void* d_x2, const void* d_w, float* d_y, int T, int N, int K,
                            void* d_scratch, size_t scratch_bytes, void* stream);
+
+/* The same GEMM taking fp32 activations x[T][K]: the library splits them into the
+ * hi + lo bf16 pair itself (in the scratch) and runs dlm_gemm_bf16x2.  T <= 128. */
+size_t dlm_gemm_f32_scratch_size(int T, int N, int K);
+dlm_status dlm_gemm_f32(const float* d_x, const void* d_w, float* d_y, int T, int N, int K,
+                        void* d_scratch, size_t scratch_bytes, void* stream);
 
 /* LM head fused with row statistics and the residual contraction:
  *   logits = x E^T (x: bf16 [B][d], already normalised), stats of every row with the
@@ -238,11 +253,11 @@ dlm_status dlm_bd_attention(const void* d_q, const void* d_k_cache, const void* 
  * in a fixed 16 MiB array of static device memory per device; calls whose partials
  * (split count x T x Hq x (hd + 2) x 4 bytes, the split count as dlm_bd_attention picks it
  * from T, Hq, Hkv and max_ctx) exceed 16 MiB - 256 B are rejected with DLM_ENOMEM_WS.  The
- * 4B-class shapes (T <= 64, 32/8 heads, hd 128) need at most 9.9 MB.  The first call on a
- * device looks the array up and sets kernel attributes: make it before starting any stream
- * capture on that device.  Every call clears the array's status word on `stream`.  The
- * array is shared: calls that may overlap in time race on it and must be serialised by the
- * caller. */
+ * 4B-class shapes (T <= 64, 32/8 heads, hd 128) need at most 9.9 MB.  The first call on
+ * each device looks the array up and sets the kernels' attributes on that device: make it
+ * before starting any stream capture on that device.  A call launches the attention kernels
+ * only (the partials need no clearing).  The array is shared: calls that may overlap in
+ * time race on it and must be serialised by the caller. */
 dlm_status dlm_bd_attention_noalloc(const void* d_q, const void* d_k_cache, const void* d_v_cache,
                                     void* d_o, int T, int L, int Hq, int Hkv, int hd, int max_ctx,
                                     int causal, void* stream);

@@ -98,6 +98,11 @@ def test_single_op_argument_checks(L):
     assert L.dlm_gemm_bf16(None, p, p, 8, 128, 128, p, 1 << 20, None) == dlm.DLM_EINVAL
     assert L.dlm_gemm_bf16(p, p, p, 8, 128, 100, p, 1 << 20, None) == dlm.DLM_EINVAL
     assert L.dlm_gemm_bf16(p, p, p, 8, 128, 128, p, 16, None) == dlm.DLM_ENOMEM_WS
+    assert L.dlm_gemm_f32(p, p, p, 129, 128, 128, p, 1 << 20, None) == dlm.DLM_EINVAL
+    assert L.dlm_gemm_f32(p, p, None, 8, 128, 128, p, 1 << 20, None) == dlm.DLM_EINVAL
+    assert L.dlm_gemm_f32(p, p, p, 8, 128, 128, p, 16, None) == dlm.DLM_ENOMEM_WS
+    assert L.dlm_gemm_f32_scratch_size(8, 128, 128) > L.dlm_gemm_scratch_size(8, 128, 128)
+    assert L.dlm_gemm_f32_scratch_size(129, 128, 128) == 0
     # attention: L + T beyond the cache, bad head dim
     assert L.dlm_bd_attention(p, p, p, p, 8, 100, 4, 2, 128, 64, 0, p, 1 << 20, None) == dlm.DLM_EINVAL
     assert L.dlm_bd_attention(p, p, p, p, 8, 0, 4, 2, 96, 64, 0, p, 1 << 20, None) == dlm.DLM_EINVAL
