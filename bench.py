@@ -53,6 +53,9 @@ def parse(argv=None):
     return ap.parse_args(argv)
 
 
+NOMINAL_HBM_GBS = 8000.0  # the ~8 TB/s HBM3e figure the fractions are also given against
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -105,12 +108,39 @@ class Clocks:
 
 
 # ------------------------------------------------------------------ launch accounting
-def launches_per_step(cfg, rounds, blocks, attn_combine_layers):
-    """Kernels of this library launched in one step (the schedule of dlm_api.cu)."""
+def step_algorithmic_bytes(cfg, w, rounds, fills):
+    """Bytes one decode step must move at least, forward by forward, at the mean prefix
+    length: a denoising round streams every layer's weights, W_a and E (LM head) and reads
+    the K/V of all layers; a KV-fill forward streams the layer weights without W_a and E, and
+    its last layer stops after the QKV projection (no attention, O or MLP there).  KV per
+    layer and position: 2 (K, V) x Hkv x hd x 2 bytes."""
     nl = cfg["n_layers"]
-    per_round = 3 + nl * 10 + attn_combine_layers + 5 + 1
-    per_fill = 1 + (nl - 1) * 10 + attn_combine_layers * (nl - 1) // max(nl, 1) + 2
-    return rounds * per_round + blocks * (per_fill + 2)
+    layer = [sum(v.numel() * 2 for v in l.values()) for l in w["layers"]]
+    last = w["layers"][-1]
+    last_qkv_only = last["attn_norm"].numel() * 2 + last["w_qkv"].numel() * 2
+    E = w["embed"].numel() * 2
+    Wa = w["w_adapter"].numel() * 2
+    fn = w["final_norm"].numel() * 2
+    kv_pos = 2 * cfg["n_kv_heads"] * cfg["head_dim"] * 2
+    mean_L = PROMPT + GEN / 2
+    round_b = sum(layer) + E + Wa + fn + kv_pos * nl * mean_L
+    fill_b = sum(layer[:-1]) + last_qkv_only + kv_pos * (nl - 1) * mean_L
+    return rounds * round_b + fills * fill_b, round_b, fill_b
+
+
+def launches_per_step(cfg, rounds, fills, blocks):
+    """Kernels of this library launched in one step, counted from the forward pass of
+    dlm_api.cu: per layer the QKV GEMM, its finisher, attention and its split merge, the O
+    GEMM, residual+RMSNorm, the gate/up GEMM, the SiLU finisher, the down GEMM and
+    residual+RMSNorm (10); a round adds the adapter (split copy, W_a GEMM, residual+RMSNorm),
+    the fused LM head and its merge, and the commit; a stand-alone KV-fill forward adds the
+    embedding + RMSNorm and stops after the last layer's QKV finisher; each block graph adds
+    its init and finish kernels, each step one prefix-length reset."""
+    nl = cfg["n_layers"]
+    per_layer = 10
+    per_round = 3 + nl * per_layer + 2 + 1
+    per_fill = 1 + (nl - 1) * per_layer + 2
+    return rounds * per_round + fills * per_fill + blocks * 2 + 1
 
 
 # ------------------------------------------------------------------ oracle baseline
@@ -216,6 +246,7 @@ def nvfp4_measure(args, cfg, w, prompt, dev, stream):
         m.set_prefix_len(PROMPT)
         for b in range(blocks):
             m.decode_block(TAU, dlm.COMMIT_TOPK, TPF_K, tok[b], rr[b])
+        m.kv_flush()
 
     for _ in range(args.warmup):
         step()
@@ -259,10 +290,104 @@ def nvfp4_measure(args, cfg, w, prompt, dev, stream):
     hbm, _, kind = peaks()
     out["gemm"] = gb
     out["gemm_frac"] = max(g["GBs"] for g in gb) / hbm
-    round_bytes = 3.632e9
-    out["round_ms"] = ms / (rounds + blocks)
-    out["round_roofline_frac"] = round_bytes / (out["round_ms"] / 1e3) / 1e9 / hbm
+    # algorithmic bytes: attention projections and W_a in bf16, MLP and E in NVFP4 (0.5625
+    # bytes per weight: e2m1 codes and an e4m3 scale per 16), KV at the mean prefix length
+    d, F, nl = cfg["d"], cfg["ffn"], cfg["n_layers"]
+    qkv = (cfg["n_q_heads"] + 2 * cfg["n_kv_heads"]) * cfg["head_dim"] * d * 2
+    wo = d * cfg["n_q_heads"] * cfg["head_dim"] * 2
+    layer = qkv + wo + 3 * F * d * 0.5625 + 2 * d * 2
+    kv_pos = 2 * cfg["n_kv_heads"] * cfg["head_dim"] * 2
+    mean_L = PROMPT + GEN / 2
+    round_b = nl * layer + cfg["vocab"] * d * 0.5625 + d * d * 2 + d * 2 + kv_pos * nl * mean_L
+    fill_b = (nl - 1) * layer + qkv + d * 2 + kv_pos * (nl - 1) * mean_L
+    fills = blocks  # NVFP4 contexts run each block's KV-fill as its own forward
+    step_b = rounds * round_b + fills * fill_b
+    out["round_bytes_mean_L"] = round_b
+    out["round_ms"] = ms / (rounds + fills)
+    out["round_roofline_frac"] = step_b / (ms / 1e3) / 1e9 / hbm
+    out["round_roofline_frac_nominal"] = step_b / (ms / 1e3) / 1e9 / NOMINAL_HBM_GBS
     return out
+
+
+def _timed_calls(fn, reps, flush=None):
+    """Mean device time (s) of fn() over `reps` calls, each bracketed by its own CUDA events on
+    the current stream; `flush` (untimed) runs between calls."""
+    import torch
+    total = 0.0
+    for _ in range(reps):
+        if flush is not None:
+            flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        total += e0.elapsed_time(e1) / 1e3
+    return total / reps
+
+
+def _l2_flusher(dev):
+    """Writes 256 MB (twice the 126 MB L2) so that the next call reads its inputs from HBM."""
+    import torch
+    buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    return lambda: buf.fill_(1)
+
+
+def config2_measure(args, dev):
+    """The single-round LM-head workload at 4B-class shapes (B 32, d 2560, V 151936): the fused
+    LM head with the given P_prev (row statistics of H E^T, s = P_prev E) plus the adapter step
+    h0 = E[x] + W_a s.  Algorithmic bytes: E once, P_prev, W_a (and the small B-row vectors)."""
+    from block_diffusion_decoding_denoising_b200 import dlm, gen
+    import torch
+    B, d, V = 32, 2560, 151936
+    H, E, Wa, P = gen.lmhead_inputs_torch(B, d, V, device=dev)
+    x = H.to(torch.bfloat16)
+    tokens = torch.full((B,), V - 1, dtype=torch.int32, device=dev)
+    st = {}
+
+    def call():
+        st["s"] = dlm.lmhead_rowstats(x, E, mask_id=V - 1, p_given=P)["s"]
+        dlm.adapter_embed(E, Wa, tokens, st["s"])
+
+    for _ in range(max(args.warmup, 3)):
+        call()
+    torch.cuda.synchronize()
+    flush = _l2_flusher(dev)
+    t = _timed_calls(call, 5, flush)
+    t_lm = _timed_calls(lambda: dlm.lmhead_rowstats(x, E, mask_id=V - 1, p_given=P), 5, flush)
+    hbm, _, kind = peaks()
+    nbytes = V * d * 2 + B * V * 2 + d * d * 2 + B * d * (2 + 4 + 4 + 4)
+    gbs = nbytes / t / 1e9
+    return {"workload": "LM head + row stats + P_prev E + adapter, B 32, d 2560, V 151936, P_prev = softmax "
+                        "of N(0,3) logits", "us_per_call": t * 1e6, "lmhead_given_p_us": t_lm * 1e6,
+            "algorithmic_bytes": nbytes, "GBs": gbs, "frac": gbs / hbm, "frac_nominal": gbs / NOMINAL_HBM_GBS,
+            "l2": "flushed (256 MB written) before every call"}
+
+
+def attention_sweep(args, dev):
+    """Block-diffusion attention of one layer (32 q / 8 kv heads, hd 128, bf16): block size
+    B in {4, 16, 32, 64} against prefix lengths L in {1K, 4K, 16K, 64K}.  Algorithmic bytes
+    per call: the K/V rows read once, 4096 (L + B), plus q read and o written, 16384 B."""
+    from block_diffusion_decoding_denoising_b200 import dlm, gen
+    import torch
+    hbm, _, kind = peaks()
+    flush = _l2_flusher(dev)
+    cells = []
+    for L in (1024, 4096, 16384, 65536):
+        for B in (4, 16, 32, 64):
+            q, kc, vc = gen.attention_inputs_torch(B, L, device=dev, seed=3)
+            fn = lambda: dlm.bd_attention(q, kc, vc, L)
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            t = _timed_calls(fn, 5, flush)
+            nbytes = 4096 * (L + B) + 16384 * B
+            gbs = nbytes / t / 1e9
+            cells.append({"B": B, "L": L, "us": round(t * 1e6, 2), "GBs": round(gbs, 1),
+                          "frac": round(gbs / hbm, 4), "frac_nominal": round(gbs / NOMINAL_HBM_GBS, 4)})
+            del q, kc, vc
+    return {"workload": "block-diffusion attention, 32/8 heads, hd 128, bf16, q/K/V N(0,1)",
+            "l2": "flushed (256 MB written) before every call", "cells": cells}
 
 
 def lmhead_measure(args, w, dev):
@@ -445,10 +570,14 @@ def main():
     rounds_out = torch.zeros((blocks, 2), dtype=torch.int32, device=dev)
     m.prefill(prompt)
     torch.cuda.synchronize()
+    m.decode_block(TAU, dlm.COMMIT_TOPK, TPF_K, tokens_out[0], rounds_out[0])
+    folded = m.fill_pending  # this context folds each block's KV-fill into the next round
 
     est = m.new_block_state()
 
     def step(mode=dlm.COMMIT_TOPK, k=TPF_K, nblk=blocks):
+        # every block's KV-fill: folded into the next block's first round, the last one
+        # flushed at the end of the step (the cache holds all blocks, as after dlm_generate)
         m.set_prefix_len(PROMPT)
         for b in range(nblk):
             if args.eager and mode == dlm.COMMIT_TOPK:
@@ -459,6 +588,7 @@ def main():
                 rounds_out[b, 0] = (B + k - 1) // k
             else:
                 m.decode_block(TAU, mode, k, tokens_out[b], rounds_out[b])
+        m.kv_flush()
 
     def barrier():
         if world > 1:
@@ -572,11 +702,11 @@ def main():
     e2e_s = max_over_ranks(e2e_s, world, dev)
     e2e_tps = whole_job_rate(world, GEN, e2e_s)
 
-    weight_bytes = sum(v.numel() * 2 for k, v in w.items() if k != "layers") + sum(
-        v.numel() * 2 for l in w["layers"] for v in l.values())
-    mean_L = PROMPT + GEN / 2
-    round_bytes = weight_bytes + 147456 * mean_L * cfg["n_layers"] / 36
-    round_ms = ms_step / (rounds_per_step + blocks)  # rounds and KV-fill forwards of the step
+    # stand-alone KV-fill forwards per step: one (the last block's flush) when the fills are
+    # folded into the next block's first round, else one per block
+    fills = 1 if folded else blocks
+    step_bytes, round_bytes, fill_bytes = step_algorithmic_bytes(cfg, w, rounds_per_step, fills)
+    round_ms = ms_step / (rounds_per_step + fills)  # rounds and stand-alone KV-fill forwards
 
     # NVFP4 weights (MLP and E; attention bf16): the same decode, and the NVFP4 GEMM alone
     # on the MLP shapes (partial sums only, inputs quantized per row)
@@ -584,6 +714,10 @@ def main():
     nv = nvfp4_measure(args, cfg, w, prompt, dev, stream)
     # the fused LM head alone (LM-head configuration shapes: B 32, d 2560, V 151936, P = softmax)
     lm = lmhead_measure(args, w, dev)
+    del w
+    torch.cuda.empty_cache()
+    c2 = config2_measure(args, dev)
+    c3 = attention_sweep(args, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -606,14 +740,18 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_tps, "unit": "tokens/s", "h2d_bytes_per_step": PROMPT * 4,
                     "d2h_bytes_per_step": GEN * 4 + blocks * 8},
-            "gpu_launches": args.steps * launches_per_step(cfg, rounds_per_step, blocks, cfg["n_layers"]),
+            "gpu_launches": args.steps * launches_per_step(cfg, rounds_per_step, fills, blocks),
             "clocks": ck,
             "extra": {"rounds_per_step": rounds_per_step, "tpf": GEN / rounds_per_step,
-                      "round_or_fill_ms": round_ms,
-                      "round_roofline_frac": (round_bytes / (round_ms / 1e3) / 1e9) / hbm,
+                      "kv_fill": "folded into the next block's first round" if folded else "one forward per block",
+                      "standalone_fills_per_step": fills, "round_or_fill_ms": round_ms,
+                      "step_algorithmic_bytes": step_bytes, "round_bytes_mean_L": round_bytes,
+                      "fill_bytes_mean_L": fill_bytes,
+                      "round_roofline_frac": step_bytes / (ms_step / 1e3) / 1e9 / hbm,
+                      "round_roofline_frac_nominal": step_bytes / (ms_step / 1e3) / 1e9 / NOMINAL_HBM_GBS,
                       "tau0.9_rounds_per_s": tau_rounds_per_s, "tau0.9_rounds_per_block": tau_rounds / 4,
                       "gemm_avg_launch_us": gemm_s * 1e6, "gemm_all_shapes_GBs": gemm_avg_gbs,
-                      "nvfp4": nv, "lmhead_fused": lm},
+                      "nvfp4": nv, "lmhead_fused": lm, "config2_lmhead_given_p": c2, "config3_attention": c3},
         }
         print(json.dumps(line), flush=True)
     if world > 1:
