@@ -372,11 +372,22 @@ def attention_sweep(args, dev):
     import torch
     hbm, _, kind = peaks()
     flush = _l2_flusher(dev)
+    import ctypes as C
+    lib = dlm.lib()
+    sp = C.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     cells = []
     for L in (1024, 4096, 16384, 65536):
         for B in (4, 16, 32, 64):
             q, kc, vc = gen.attention_inputs_torch(B, L, device=dev, seed=3)
-            fn = lambda: dlm.bd_attention(q, kc, vc, L)
+            o = torch.empty_like(q)
+            Hq, hd = q.shape[1], q.shape[2]
+            Hkv, mc = kc.shape[0], kc.shape[1]
+            n = lib.dlm_attention_scratch_size(B, Hq, hd, mc)
+            sc = torch.empty(n, dtype=torch.uint8, device=dev)
+            args_c = [C.c_void_p(t.data_ptr()) for t in (q, kc, vc, o)] + [B, L, Hq, Hkv, hd, mc, 0,
+                                                                           C.c_void_p(sc.data_ptr()), n, sp]
+            # the call alone (arguments prepared): the event pair brackets only the launch
+            fn = lambda: lib.dlm_bd_attention(*args_c)
             for _ in range(3):
                 fn()
             torch.cuda.synchronize()
@@ -385,7 +396,7 @@ def attention_sweep(args, dev):
             gbs = nbytes / t / 1e9
             cells.append({"B": B, "L": L, "us": round(t * 1e6, 2), "GBs": round(gbs, 1),
                           "frac": round(gbs / hbm, 4), "frac_nominal": round(gbs / NOMINAL_HBM_GBS, 4)})
-            del q, kc, vc
+            del q, kc, vc, o, sc
     return {"workload": "block-diffusion attention, 32/8 heads, hd 128, bf16, q/K/V N(0,1)",
             "l2": "flushed (256 MB written) before every call", "cells": cells}
 

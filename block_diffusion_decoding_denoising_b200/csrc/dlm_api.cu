@@ -32,10 +32,16 @@ namespace {
 constexpr int kPrefillChunk = kMaxSplitTokens;  // prefill tokens per forward pass (bf16 weights)
 constexpr int kRowChunk = 4096;                  // vocabulary entries per row-statistics CTA
 
+// Per-block graph variants: the KV-fill of the block runs inside its own graph (EAGER), or
+// is left pending and carried by the first round of the next block (FIRST: no block pending
+// at launch, FOLD: one pending block folded into the first round).
+enum GraphVariant : int { GV_EAGER = 0, GV_FIRST = 1, GV_FOLD = 2 };
+
 struct GraphEntry {
   int mode;
   float tau;
   int k;
+  int variant;
   cudaGraph_t graph;
   cudaGraphExec_t exec;
 };
@@ -68,7 +74,12 @@ struct dlm_ctx {
   float* rs_part = nullptr;  // row-statistics chunk partials
   float2* rope_tab = nullptr;  // [max_ctx][hd/2] (cos, sin)
   float* attn_part = nullptr;
-  int attn_splits_B = 1, attn_splits_T = 1;
+  int attn_splits_B = 1, attn_splits_T = 1, attn_splits_2B = 1;
+  // deferred KV-fill: a committed block whose clean forward has not run yet (its K/V rows
+  // [L - B, L) are not valid); the next round carries it, dlm_kv_flush runs it alone
+  int32_t* pend_tokens = nullptr;  // device [B]
+  bool pending = false;
+  bool fill_deferred = true;       // dlm_set_fill_mode
   float* logits = nullptr;
   __nv_bfloat16* P = nullptr;
   int32_t* tok_buf = nullptr;
@@ -179,7 +190,7 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   auto* q = cv.take<__nv_bfloat16>((size_t)Tmax * ho);
   auto* o = cv.take<__nv_bfloat16>(R2 * ho);
   auto* act = cv.take<__nv_bfloat16>(R2 * c.ffn);
-  auto* sbf = cv.take<__nv_bfloat16>(B2 * c.d);
+  auto* sbf = cv.take<__nv_bfloat16>(R2 * c.d);  // W_a input of a pass of up to Tmax rows
   size_t pb = max_partial_bytes(c, Tmax);
   float* partial = cv.take<float>(pb / sizeof(float));
   int* cnt = cv.take<int>((size_t)(c.vocab + 63) / 64 + (c.ffn + 63) / 64 + 64);
@@ -188,9 +199,13 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   float2* rtab = cv.take<float2>((size_t)c.max_ctx * (c.head_dim / 2));
   int sB = attention_max_splits(B, c.n_q_heads, c.n_kv_heads, c.max_ctx);
   int sT = attention_max_splits(Tmax, c.n_q_heads, c.n_kv_heads, c.max_ctx);
+  int s2 = attention_max_splits(2 * B, c.n_q_heads, c.n_kv_heads, c.max_ctx);
   size_t ab = attention_scratch_bytes(B, c.n_q_heads, c.head_dim, sB);
   size_t at = attention_scratch_bytes(Tmax, c.n_q_heads, c.head_dim, sT);
-  float* attn = cv.take<float>((ab > at ? ab : at) / sizeof(float));
+  size_t a2 = attention_scratch_bytes(2 * B, c.n_q_heads, c.head_dim, s2);
+  size_t amax = ab > at ? ab : at;
+  amax = a2 > amax ? a2 : amax;
+  float* attn = cv.take<float>(amax / sizeof(float));
   float* logits = cv.take<float>((size_t)B * c.vocab);
   auto* P = cv.take<__nv_bfloat16>(B2 * c.vocab);
   int32_t* tok = cv.take<int32_t>((size_t)c.max_ctx);
@@ -202,6 +217,7 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   int32_t* sa = cv.take<int32_t>(B);
   int32_t* ot = cv.take<int32_t>(B);
   int32_t* orr = cv.take<int32_t>(4);
+  int32_t* pend = cv.take<int32_t>(B);
   const bool fp4 = c.weight_fmt == DLM_WEIGHTS_NVFP4;
   const size_t kmax = c.d > c.ffn ? c.d : c.ffn;
   uint8_t* xcodes = fp4 ? cv.take<uint8_t>((size_t)kMaxF4Tokens * kmax / 2) : nullptr;
@@ -242,6 +258,8 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
     x->attn_part = attn;
     x->attn_splits_B = sB;
     x->attn_splits_T = sT;
+    x->attn_splits_2B = s2;
+    x->pend_tokens = pend;
     x->logits = logits;
     x->P = P;
     x->tok_buf = tok;
@@ -335,6 +353,12 @@ struct Runner {
 struct FwdSpec {
   int T;
   const int32_t* tokens;  // device [T]
+  // A pending committed block (T_pend = B rows, or 0) computed ahead of the T rows in the same
+  // pass: its clean forward (s = 0) at positions [pos - T_pend, pos), each of its rows seeing
+  // the prefix and its own block, while the T rows see everything.  Its K/V rows are what a
+  // separate KV-fill forward would write; the LM head runs on the T rows only.
+  int T_pend;
+  const int32_t* pend_tokens;  // device [T_pend]
   const float* s;         // device fp32 [T][d], or nullptr (no adapter)
   int pos0;               // used when !dev_L
   bool dev_L;             // positions from ctx->d_L (graph mode)
@@ -346,7 +370,7 @@ struct FwdSpec {
 
 // h update + RMSNorm into the split GEMM input xn, a 4-CTA cluster per token (see k_resid_norm).
 dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_tokens, const void* gain,
-                      bool quantize = false) {
+                      bool quantize = false, const int32_t* embed_tokens2 = nullptr, int tok_split = 0) {
   dlm_ctx* ctx = r.ctx;
   const dlm_config& c = ctx->cfg;
   ResNormArgs a{};
@@ -355,6 +379,8 @@ dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_t
   a.h = ctx->h;
   a.embed = embed_tokens ? (ctx->fp4 ? ctx->e_deq : (const __nv_bfloat16*)ctx->w.embed) : nullptr;
   a.tokens = embed_tokens;
+  a.tokens2 = embed_tokens2;
+  a.tok_split = tok_split;
   a.embed_scale = ctx->fp4 ? ctx->w.q_embed.tensor_scale : 1.0f;
   a.gain = (const __nv_bfloat16*)gain;
   a.xn = ctx->xn;
@@ -394,29 +420,63 @@ dlm_status finish_tiles(Runner& r, const GemmOut& y, int N, const EpiArgs& epi) 
   return DLM_OK;
 }
 
+// The MLP of layer l on the normed input in ctx->xn (and, for NVFP4 weights, its codes):
+// gate/up GEMM -> SiLU gate -> [input quantizer ->] down GEMM; the down projection's
+// partial sums are left in *y for the residual update.
+dlm_status mlp_sub_block(Runner& r, int l, int T, GemmOut* y) {
+  dlm_ctx* ctx = r.ctx;
+  const dlm_config& c = ctx->cfg;
+  const int d = c.d, F = c.ffn;
+  const long pad = split_pad(T);
+  const dlm_layer_weights& W = ctx->layers[l];
+  if (ctx->fp4) {  // input quantized by the residual+RMSNorm before
+    TRY(r.gemm_fp4(A_PAIR, W.q_gate, &W.q_up, ctx->sf + l * (ctx->sf_pair + ctx->sf_down), T, F, d, y));
+  } else {
+    TRY(r.gemm_partial(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, y));
+  }
+  EpiArgs es{};
+  es.op = EPI_SILU;
+  es.act = ctx->act;
+  es.act_lo = pad * F;
+  TRY(finish_tiles(r, *y, F, es));
+  if (ctx->fp4) {
+    TRY(act_quant(r, T, ctx->act, pad * F, F));
+    return r.gemm_fp4(A_KMAJOR, W.q_down, nullptr, ctx->sf + l * (ctx->sf_pair + ctx->sf_down) + ctx->sf_pair, T, d,
+                      F, y);
+  }
+  return r.gemm_partial(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, y);
+}
+
 // One forward pass of T tokens (round, KV-fill or prefill chunk), all on stream r.s:
 //   [s -> split bf16 -> W_a GEMM] ; h = E[x] (+ W_a s) ; RMSNorm
 //   per layer: QKV GEMM ; RoPE + K/V cache ; attention ; O GEMM ; residual + RMSNorm ;
 //              gate/up GEMM ; SiLU gate ; down GEMM ; residual + RMSNorm (next gain)
-//   round only: LM head GEMM -> logits ; row statistics + P ; P E GEMM -> s_out
+//   round only: LM head with row statistics and s = P E (fused), or logits GEMM ; row
+//   statistics + P ; P E GEMM
 // The projections leave per-slot partial sums; the kernel after each one finishes them.
+// With f.T_pend > 0 the rows of a pending committed block come first (see FwdSpec).
 dlm_status forward(Runner& r, const FwdSpec& f) {
   dlm_ctx* ctx = r.ctx;
   const dlm_config& c = ctx->cfg;
-  const int T = f.T, d = c.d, Hq = c.n_q_heads, Hkv = c.n_kv_heads, hd = c.head_dim, F = c.ffn;
+  const int Tp = f.T_pend, T = Tp + f.T;  // all rows of the pass
+  const int d = c.d, Hq = c.n_q_heads, Hkv = c.n_kv_heads, hd = c.head_dim;
   const int ho = Hq * hd, nqkv = (Hq + 2 * Hkv) * hd;
   const long pad = split_pad(T);  // low halves of split activations start `pad` rows down
   const void* first_gain = c.n_layers > 0 ? ctx->layers[0].attn_norm : ctx->w.final_norm;
+  const int32_t* tok0 = Tp ? f.pend_tokens : f.tokens;  // token rows [0, Tp) then [Tp, T)
+  const int32_t* tok1 = Tp ? f.tokens : nullptr;
+  const int pos0 = f.pos0 - Tp;  // position of row 0 (eager); graph mode: *d_L - Tp
   GemmOut y;
 
-  // embedding + residual adapter
+  // embedding + residual adapter (the pending rows carry no residual: s = 0 there)
   if (f.s) {
-    long n = (long)T * d;
-    CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, r.s, f.s, ctx->sbf, n, pad * d));
+    const long n = (long)f.T * d, zn = (long)Tp * d;
+    CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((zn + n + 255) / 256)), dim3(256), 0, r.s, f.s, ctx->sbf, n,
+                       pad * d, zn));
     TRY(r.gemm_partial(A_KMAJOR, ctx->w.w_adapter, nullptr, ctx->sbf, T, d, d, &y));
-    TRY(resid_norm(r, T, &y, f.tokens, first_gain));
+    TRY(resid_norm(r, T, &y, tok0, first_gain, false, tok1, Tp));
   } else {
-    TRY(resid_norm(r, T, nullptr, f.tokens, first_gain));
+    TRY(resid_norm(r, T, nullptr, tok0, first_gain, false, tok1, Tp));
   }
 
   const size_t layer_kv = (size_t)Hkv * c.max_ctx * hd;
@@ -434,8 +494,9 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     eq.Hkv = Hkv;
     eq.hd = hd;
     eq.max_ctx = c.max_ctx;
-    eq.pos0 = f.pos0;
+    eq.pos0 = pos0;
     eq.pos0_dev = f.dev_L ? ctx->d_L : nullptr;
+    eq.pos_off = -Tp;
     eq.rope_tab = ctx->rope_tab;
     TRY(finish_tiles(r, y, nqkv, eq));
     // the last layer's K/V do not depend on anything after its QKV projection
@@ -453,10 +514,13 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     aa.Hkv = Hkv;
     aa.hd = hd;
     aa.max_ctx = c.max_ctx;
-    aa.pos0 = f.pos0;
+    aa.pos0 = pos0;
     aa.pos0_dev = f.dev_L ? ctx->d_L : nullptr;
+    aa.pos_off = -Tp;
     aa.causal = f.causal ? 1 : 0;
-    aa.max_splits = (T <= c.block_size) ? ctx->attn_splits_B : ctx->attn_splits_T;
+    aa.blk = Tp ? Tp : 0;  // pending block, then the new block; else one block
+    aa.max_splits = (T <= c.block_size) ? ctx->attn_splits_B
+                                        : (T <= 2 * c.block_size ? ctx->attn_splits_2B : ctx->attn_splits_T);
     aa.part_ml = ctx->attn_part + (size_t)aa.max_splits * T * Hq * hd;
     aa.err = ctx->d_err;
     cudaError_t e = attention_launch(aa, r.s);
@@ -465,40 +529,26 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     TRY(r.gemm_partial(A_KMAJOR, W.w_o, nullptr, ctx->o, T, d, ho, &y));
     TRY(resid_norm(r, T, &y, nullptr, W.mlp_norm, ctx->fp4));
 
-    if (ctx->fp4) {  // input quantized by the residual+RMSNorm above
-      TRY(r.gemm_fp4(A_PAIR, W.q_gate, &W.q_up, ctx->sf + l * (ctx->sf_pair + ctx->sf_down), T, F, d, &y));
-    } else {
-      TRY(r.gemm_partial(A_PAIR, W.w_gate, W.w_up, ctx->xn, T, F, d, &y));
-    }
-    EpiArgs es{};
-    es.op = EPI_SILU;
-    es.act = ctx->act;
-    es.act_lo = pad * F;
-    TRY(finish_tiles(r, y, F, es));
-
-    if (ctx->fp4) {
-      TRY(act_quant(r, T, ctx->act, pad * F, F));
-      TRY(r.gemm_fp4(A_KMAJOR, W.q_down, nullptr, ctx->sf + l * (ctx->sf_pair + ctx->sf_down) + ctx->sf_pair, T,
-                     d, F, &y));
-    } else {
-      TRY(r.gemm_partial(A_KMAJOR, W.w_down, nullptr, ctx->act, T, d, F, &y));
-    }
+    TRY(mlp_sub_block(r, l, T, &y));
     const bool last = l + 1 == c.n_layers;
     TRY(resid_norm(r, T, &y, nullptr, last ? ctx->w.final_norm : ctx->layers[l + 1].attn_norm,
                    last && ctx->fp4 && f.lm_head));
   }
   if (!f.lm_head) return DLM_OK;
+  const int Tl = f.T;  // LM head rows: the new block's
 
   // LM head: logits (finished inside the GEMM: its tiles are mostly single-slot), row
   // statistics, P = softmax (split bf16), s = P E
-  if (ctx->lmf && T <= 32) {
-    // one pass over E: logits, row statistics and s = P E (split x: pad = 32 for T <= 32)
+  if (ctx->lmf && Tl <= 32) {
+    // one pass over E: logits, row statistics and s = P E on the rows [Tp, T) of the split x
     char msg[256];
-    cudaError_t e = lmhead_fused_launch(ctx->xn, ctx->w.embed, nullptr, T, c.vocab, d, c.mask_id, f.stats, f.s_out,
-                                        ctx->lmf, ctx->d_err, r.s, msg, sizeof(msg));
+    cudaError_t e = lmhead_fused_launch(ctx->xn, (int)(2 * pad), Tp, (int)(pad + Tp), ctx->w.embed, nullptr, Tl,
+                                        c.vocab, d, c.mask_id, f.stats, f.s_out, ctx->lmf, ctx->d_err, r.s, msg,
+                                        sizeof(msg));
     if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "fused lm head: %s %s", cudaGetErrorString(e), msg);
     return DLM_OK;
   }
+  if (Tp) return fail(ctx, DLM_EUNSUPPORTED, "a pending block needs the fused LM head");
   EpiArgs el{};
   el.op = EPI_STORE;
   el.out = ctx->logits;
@@ -532,6 +582,13 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
   ep.ld = d;
   ep.scale = ctx->fp4 ? ctx->w.q_embed.tensor_scale : 0.f;
   return finish_tiles(r, y, d, ep);
+}
+
+// Whether the context can carry a pending block in the next round: the pass then has 2B
+// rows (split GEMM inputs up to 128 rows) and must use the fused LM head.
+bool fold_supported(const dlm_ctx* ctx) {
+  const dlm_config& c = ctx->cfg;
+  return !ctx->fp4 && ctx->lmf != nullptr && 2 * c.block_size <= kMaxSplitTokens && c.block_size <= 32;
 }
 
 dlm_status launch_commit(Runner& r, const dlm_block_state& st, float tau, int mode, int k,
@@ -584,34 +641,46 @@ dlm_status launch_block_init(Runner& r, const dlm_block_state& st) {
   return r.check();
 }
 
-dlm_status build_block_graph(dlm_ctx* ctx, int mode, float tau, int k, GraphEntry* out) {
-  cudaGraph_t g = nullptr, g_init = nullptr, g_fill = nullptr;
+// One graph per (commit mode, tau / k, variant):
+//   GV_EAGER: init -> WHILE { round } -> KV-fill forward -> finish
+//   GV_FIRST: init -> WHILE { round } -> finish (the block's KV-fill is left pending)
+//   GV_FOLD:  init -> first round carrying the pending block (its commit sets the loop
+//             condition) -> WHILE { round } -> finish (this block's KV-fill left pending)
+// finish copies tokens and rounds out and advances the device prefix length by B.
+// Captures what `body` enqueues on the capture stream into graph g after the nodes `deps`
+// (cudaStreamBeginCaptureToGraph), and returns the capture's leaf nodes in *leaves.
+template <class Body>
+dlm_status capture_into(dlm_ctx* ctx, cudaGraph_t g, const std::vector<cudaGraphNode_t>& deps, Body body,
+                        std::vector<cudaGraphNode_t>* leaves) {
+  cudaStream_t cs = ctx->cap_stream;
+  CU(cudaStreamBeginCaptureToGraph(cs, g, deps.empty() ? nullptr : deps.data(), nullptr, deps.size(),
+                                   cudaStreamCaptureModeThreadLocal));
+  dlm_status st = body();
+  if (st == DLM_OK && leaves) {
+    cudaStreamCaptureStatus cst;
+    const cudaGraphNode_t* d = nullptr;
+    size_t nd = 0;
+    cudaError_t e = cudaStreamGetCaptureInfo(cs, &cst, nullptr, nullptr, &d, &nd);
+    if (e == cudaSuccess) leaves->assign(d, d + nd);
+    else st = fail(ctx, DLM_ECUDA, "capture info: %s", cudaGetErrorString(e));
+  }
+  cudaGraph_t same = nullptr;
+  cudaError_t e = cudaStreamEndCapture(cs, &same);
+  if (st != DLM_OK) return st;
+  CU(e);
+  return DLM_OK;
+}
+
+dlm_status build_block_graph(dlm_ctx* ctx, int mode, float tau, int k, int variant, GraphEntry* out) {
+  cudaGraph_t g = nullptr;
   CU(cudaGraphCreate(&g, 0));
   cudaGraphConditionalHandle h;
   CU(cudaGraphConditionalHandleCreate(&h, g, 1, cudaGraphCondAssignDefault));
-  cudaStream_t cs = ctx->cap_stream;
-  Runner r{ctx, cs, {}};
+  Runner r{ctx, ctx->cap_stream, {}};
   dlm_block_state st = internal_state(ctx);
   const dlm_config& c = ctx->cfg;
+  std::vector<cudaGraphNode_t> leaves;
 
-  // init
-  CU(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
-  dlm_status s1 = launch_block_init(r, st);
-  cudaError_t e = cudaStreamEndCapture(cs, &g_init);
-  if (s1 != DLM_OK) return s1;
-  CU(e);
-  cudaGraphNode_t n_init, n_while, n_fill;
-  CU(cudaGraphAddChildGraphNode(&n_init, g, nullptr, 0, g_init));
-
-  // while node with the round as its body
-  cudaGraphNodeParams cp = {};
-  cp.type = cudaGraphNodeTypeConditional;
-  cp.conditional.handle = h;
-  cp.conditional.type = cudaGraphCondTypeWhile;
-  cp.conditional.size = 1;
-  CU(cudaGraphAddNode(&n_while, g, &n_init, 1, &cp));
-  cudaGraph_t body = cp.conditional.phGraph_out[0];
-  CU(cudaStreamBeginCaptureToGraph(cs, body, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal));
   FwdSpec f{};
   f.T = c.block_size;
   f.tokens = st.tokens;
@@ -620,34 +689,71 @@ dlm_status build_block_graph(dlm_ctx* ctx, int mode, float tau, int k, GraphEntr
   f.lm_head = true;
   f.stats = st.stats;
   f.s_out = st.s;
-  dlm_status s2 = forward(r, f);
-  if (s2 == DLM_OK) s2 = launch_commit(r, st, tau, mode, k, true, h);
-  e = cudaStreamEndCapture(cs, nullptr);
-  if (s2 != DLM_OK) return s2;
-  CU(e);
+  // init [-> the first round carrying the pending block's rows; its commit sets the loop
+  // condition]
+  TRY(capture_into(ctx, g, {}, [&]() -> dlm_status {
+    TRY(launch_block_init(r, st));
+    if (variant != GV_FOLD) return DLM_OK;
+    FwdSpec f1 = f;
+    f1.T_pend = c.block_size;
+    f1.pend_tokens = ctx->pend_tokens;
+    TRY(forward(r, f1));
+    return launch_commit(r, st, tau, mode, k, true, h);
+  }, &leaves));
 
-  // KV-fill of the committed block, then the block outputs and L += B
-  CU(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
-  FwdSpec kf{};
-  kf.T = c.block_size;
-  kf.tokens = st.tokens;
-  kf.dev_L = true;
-  dlm_status s3 = forward(r, kf);
-  if (s3 == DLM_OK) {
+  // while node with one round as its body
+  cudaGraphNode_t n_while;
+  cudaGraphNodeParams cp = {};
+  cp.type = cudaGraphNodeTypeConditional;
+  cp.conditional.handle = h;
+  cp.conditional.type = cudaGraphCondTypeWhile;
+  cp.conditional.size = 1;
+  CU(cudaGraphAddNode(&n_while, g, leaves.data(), leaves.size(), &cp));
+  cudaGraph_t body = cp.conditional.phGraph_out[0];
+  TRY(capture_into(ctx, body, {}, [&]() -> dlm_status {
+    TRY(forward(r, f));
+    return launch_commit(r, st, tau, mode, k, true, h);
+  }, nullptr));
+
+  // [KV-fill of the committed block,] the block outputs and L += B
+  TRY(capture_into(ctx, g, {n_while}, [&]() -> dlm_status {
+    if (variant == GV_EAGER) {
+      FwdSpec kf{};
+      kf.T = c.block_size;
+      kf.tokens = st.tokens;
+      kf.dev_L = true;
+      TRY(forward(r, kf));
+    }
     BlockFinishArgs fa{st.tokens, st.round, st.status, ctx->d_err, ctx->out_tokens, ctx->out_rounds,
-                       ctx->d_L, c.block_size};
-    CU_LAUNCH(launch_k(k_block_finish, dim3(1), dim3(64), 0, cs, fa));
-    s3 = r.check();
-  }
-  e = cudaStreamEndCapture(cs, &g_fill);
-  if (s3 != DLM_OK) return s3;
-  CU(e);
-  CU(cudaGraphAddChildGraphNode(&n_fill, g, &n_while, 1, g_fill));
+                       ctx->d_L, variant == GV_EAGER ? nullptr : ctx->pend_tokens, c.block_size};
+    CU_LAUNCH(launch_k(k_block_finish, dim3(1), dim3(64), 0, ctx->cap_stream, fa));
+    return r.check();
+  }, nullptr));
   cudaGraphExec_t ex;
   CU(cudaGraphInstantiate(&ex, g, 0));
-  cudaGraphDestroy(g_init);
-  cudaGraphDestroy(g_fill);
-  *out = GraphEntry{mode, tau, k, g, ex};
+  *out = GraphEntry{mode, tau, k, variant, g, ex};
+  return DLM_OK;
+}
+
+// Sets the prefix length on the host and the device (no pending-fill handling).
+dlm_status set_L(dlm_ctx* ctx, int L, cudaStream_t s) {
+  CU_LAUNCH(launch_k(k_set_int, dim3(1), dim3(1), 0, s, ctx->d_L, L));
+  CU(cudaGetLastError());
+  ctx->L = L;
+  return DLM_OK;
+}
+
+// Runs a pending KV-fill on its own: the clean forward of the pending block at positions
+// [L - B, L) (no LM head).
+dlm_status flush_pending(dlm_ctx* ctx, cudaStream_t s) {
+  if (!ctx->pending) return DLM_OK;
+  Runner r{ctx, s, {}};
+  FwdSpec f{};
+  f.T = ctx->cfg.block_size;
+  f.tokens = ctx->pend_tokens;
+  f.pos0 = ctx->L - ctx->cfg.block_size;
+  TRY(forward(r, f));
+  ctx->pending = false;
   return DLM_OK;
 }
 
@@ -764,16 +870,35 @@ int dlm_prefix_len(const dlm_ctx* ctx) { return ctx ? ctx->L : -1; }
 dlm_status dlm_set_prefix_len(dlm_ctx* ctx, int L, void* stream) {
   if (!ctx) return DLM_EINVAL;
   if (L < 0 || L > ctx->cfg.max_ctx) return fail(ctx, DLM_EINVAL, "L=%d", L);
-  CU_LAUNCH(launch_k(k_set_int, dim3(1), dim3(1), 0, (cudaStream_t)stream, ctx->d_L, L));
-  CU(cudaGetLastError());
-  ctx->L = L;
+  if (ctx->pending) {
+    // the pending block's rows [L_old - B, L_old): free when the new prefix ends before them,
+    // else written now
+    if (L <= ctx->L - ctx->cfg.block_size) ctx->pending = false;
+    else TRY(flush_pending(ctx, (cudaStream_t)stream));
+  }
+  return set_L(ctx, L, (cudaStream_t)stream);
+}
+
+dlm_status dlm_kv_flush(dlm_ctx* ctx, void* stream) {
+  if (!ctx) return DLM_EINVAL;
+  return flush_pending(ctx, (cudaStream_t)stream);
+}
+
+dlm_status dlm_set_fill_mode(dlm_ctx* ctx, int mode, void* stream) {
+  if (!ctx) return DLM_EINVAL;
+  if (mode != DLM_FILL_EAGER && mode != DLM_FILL_DEFERRED) return fail(ctx, DLM_EINVAL, "fill mode %d", mode);
+  if (mode == DLM_FILL_EAGER) TRY(flush_pending(ctx, (cudaStream_t)stream));
+  ctx->fill_deferred = mode == DLM_FILL_DEFERRED;
   return DLM_OK;
 }
+
+int dlm_fill_pending(const dlm_ctx* ctx) { return ctx ? (ctx->pending ? 1 : 0) : -1; }
 
 dlm_status dlm_prefill(dlm_ctx* ctx, const int32_t* d_tokens, int n, void* stream) {
   if (!ctx) return DLM_EINVAL;
   if (!d_tokens || n < 0) return fail(ctx, DLM_EINVAL, "prefill args");
   if (ctx->L + n > ctx->cfg.max_ctx) return fail(ctx, DLM_EKVCAP, "prefill: %d + %d > %d", ctx->L, n, ctx->cfg.max_ctx);
+  TRY(flush_pending(ctx, (cudaStream_t)stream));
   Runner r{ctx, (cudaStream_t)stream, {}};
   const int chunk = prefill_chunk(ctx->cfg);
   for (int off = 0; off < n; off += chunk) {
@@ -785,7 +910,7 @@ dlm_status dlm_prefill(dlm_ctx* ctx, const int32_t* d_tokens, int n, void* strea
     f.causal = true;
     TRY(forward(r, f));
   }
-  return dlm_set_prefix_len(ctx, ctx->L + n, stream);
+  return set_L(ctx, ctx->L + n, (cudaStream_t)stream);
 }
 
 dlm_status dlm_block_init(dlm_ctx* ctx, const dlm_block_state* st, void* stream) {
@@ -814,7 +939,12 @@ dlm_status dlm_round(dlm_ctx* ctx, const dlm_block_state* st, float tau, int com
   f.lm_head = true;
   f.stats = st->stats;
   f.s_out = st->s;
+  if (ctx->pending) {  // the pending KV-fill rides along (see FwdSpec)
+    f.T_pend = c.block_size;
+    f.pend_tokens = ctx->pend_tokens;
+  }
   TRY(forward(r, f));
+  ctx->pending = false;
   return launch_commit(r, *st, tau, commit_mode, tpf_k, false, 0);
 }
 
@@ -823,13 +953,42 @@ dlm_status dlm_kv_fill(dlm_ctx* ctx, const int32_t* d_tokens, void* stream) {
   if (!d_tokens) return fail(ctx, DLM_EINVAL, "kv_fill tokens");
   const dlm_config& c = ctx->cfg;
   if (ctx->L + c.block_size > c.max_ctx) return fail(ctx, DLM_EKVCAP, "kv_fill: capacity");
-  Runner r{ctx, (cudaStream_t)stream, {}};
+  cudaStream_t s = (cudaStream_t)stream;
+  TRY(flush_pending(ctx, s));  // at most one block pending
+  if (ctx->fill_deferred && fold_supported(ctx)) {
+    // deferred: keep the tokens; the next round (or dlm_kv_flush) writes the rows
+    CU(cudaMemcpyAsync(ctx->pend_tokens, d_tokens, (size_t)c.block_size * 4, cudaMemcpyDeviceToDevice, s));
+    TRY(set_L(ctx, ctx->L + c.block_size, s));
+    ctx->pending = true;
+    return DLM_OK;
+  }
+  Runner r{ctx, s, {}};
   FwdSpec f{};
   f.T = c.block_size;
   f.tokens = d_tokens;
   f.pos0 = ctx->L;
   TRY(forward(r, f));
-  return dlm_set_prefix_len(ctx, ctx->L + c.block_size, stream);
+  return set_L(ctx, ctx->L + c.block_size, s);
+}
+
+dlm_status dlm_mlp_block(dlm_ctx* ctx, int layer, const float* d_h_in, float* d_h_out, int T, void* stream) {
+  if (!ctx) return DLM_EINVAL;
+  const dlm_config& c = ctx->cfg;
+  const int tmax = ctx->fp4 ? kMaxF4Tokens : ctx->Tmax;
+  if (!d_h_in || !d_h_out || layer < 0 || layer >= c.n_layers || T < 1 || T > tmax)
+    return fail(ctx, DLM_EINVAL, "mlp_block: layer %d, T %d", layer, T);
+  cudaStream_t s = (cudaStream_t)stream;
+  Runner r{ctx, s, {}};
+  const size_t bytes = (size_t)T * c.d * sizeof(float);
+  CU(cudaMemcpyAsync(ctx->h, d_h_in, bytes, cudaMemcpyDeviceToDevice, s));
+  // h unchanged (no projection to add), xn = RMSNorm(h) g_mlp (quantized for NVFP4 weights)
+  TRY(resid_norm(r, T, nullptr, nullptr, ctx->layers[layer].mlp_norm, ctx->fp4));
+  GemmOut y;
+  TRY(mlp_sub_block(r, layer, T, &y));
+  const bool last = layer + 1 == c.n_layers;
+  TRY(resid_norm(r, T, &y, nullptr, last ? ctx->w.final_norm : ctx->layers[layer + 1].attn_norm));
+  CU(cudaMemcpyAsync(d_h_out, ctx->h, bytes, cudaMemcpyDeviceToDevice, s));
+  return DLM_OK;
 }
 
 dlm_status dlm_decode_block(dlm_ctx* ctx, float tau, int commit_mode, int tpf_k, int32_t* d_tokens_out,
@@ -839,20 +998,25 @@ dlm_status dlm_decode_block(dlm_ctx* ctx, float tau, int commit_mode, int tpf_k,
   const dlm_config& c = ctx->cfg;
   if (ctx->L + c.block_size > c.max_ctx)
     return fail(ctx, DLM_EKVCAP, "decode_block: L %d + B %d > %d", ctx->L, c.block_size, c.max_ctx);
+  cudaStream_t s = (cudaStream_t)stream;
+  const bool defer = ctx->fill_deferred && fold_supported(ctx);
+  if (!defer) TRY(flush_pending(ctx, s));
+  const int variant = !defer ? GV_EAGER : (ctx->pending ? GV_FOLD : GV_FIRST);
   GraphEntry* ge = nullptr;
   for (auto& g : ctx->graphs)
-    if (g.mode == commit_mode && (commit_mode == DLM_COMMIT_TOPK ? g.k == tpf_k : g.tau == tau)) ge = &g;
+    if (g.mode == commit_mode && g.variant == variant && (commit_mode == DLM_COMMIT_TOPK ? g.k == tpf_k : g.tau == tau))
+      ge = &g;
   if (!ge) {
     GraphEntry ne{};
-    TRY(build_block_graph(ctx, commit_mode, tau, tpf_k, &ne));
+    TRY(build_block_graph(ctx, commit_mode, tau, tpf_k, variant, &ne));
     ctx->graphs.push_back(ne);
     ge = &ctx->graphs.back();
   }
-  cudaStream_t s = (cudaStream_t)stream;
   CU(cudaGraphLaunch(ge->exec, s));
   if (d_tokens_out) CU(cudaMemcpyAsync(d_tokens_out, ctx->out_tokens, c.block_size * 4, cudaMemcpyDeviceToDevice, s));
   if (d_rounds_out) CU(cudaMemcpyAsync(d_rounds_out, ctx->out_rounds, 2 * 4, cudaMemcpyDeviceToDevice, s));
   ctx->L += c.block_size;
+  ctx->pending = defer;
   return DLM_OK;
 }
 
@@ -889,6 +1053,8 @@ dlm_status dlm_generate(dlm_ctx* ctx, const int32_t* h_prompt, int prompt_len, i
     if (h_rounds_per_block) h_rounds_per_block[b] = rb[0];
     total_rounds += rb[0];
   }
+  TRY(flush_pending(ctx, s));  // the last block's KV-fill: the cache is complete on return
+  CU(cudaStreamSynchronize(s));
   auto t2 = std::chrono::steady_clock::now();
   if (h_timing) {
     h_timing->prefill_ms = std::chrono::duration<double, std::milli>(t1 - t0).count();
@@ -1001,7 +1167,7 @@ dlm_status dlm_gemm_f32(const float* d_x, const void* d_w, float* d_y, int T, in
   __nv_bfloat16* x2 = (__nv_bfloat16*)((uint8_t*)d_scratch + gemm_sc);
   CU(cudaMemsetAsync(x2, 0, (size_t)2 * pad * K * 2, s));
   const long n = (long)T * K;
-  CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, d_x, x2, n, pad * K));
+  CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, d_x, x2, n, pad * K, 0L));
   return gemm_op(x2, d_w, d_y, T, N, K, d_scratch, gemm_sc, stream, true);
 }
 
@@ -1032,8 +1198,8 @@ dlm_status dlm_lmhead_rowstats(const void* d_x, const void* d_embed, int B, int 
     CU(cudaMemsetAsync(base, 0, op_header() + (size_t)64 * d * 2, s));
     CU(cudaMemcpyAsync(x2, d_x, (size_t)B * d * 2, cudaMemcpyDeviceToDevice, s));
     char msg[256];
-    cudaError_t e = lmhead_fused_launch(x2, d_embed, d_p_given, B, V, d, mask_id, stats, d_s, lmf, (int*)base, s,
-                                        msg, sizeof(msg));
+    cudaError_t e = lmhead_fused_launch(x2, 64, 0, 32, d_embed, d_p_given, B, V, d, mask_id, stats, d_s, lmf,
+                                        (int*)base, s, msg, sizeof(msg));
     return e == cudaSuccess ? DLM_OK : DLM_ECUDA;
   }
   CU((cudaError_t)gemm_init_attributes());
@@ -1095,7 +1261,7 @@ dlm_status dlm_adapter_embed(const void* d_embed, const void* d_w_adapter, const
   CU(cudaMemsetAsync(d_scratch, 0, op_header() + op_counters(d), s));
   long n = (long)B * d;
   CU_LAUNCH(launch_k(k_to_bf16, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, d_s, sbf, n,
-                     (long)split_pad(B) * d));
+                     (long)split_pad(B) * d, 0L));
   char msg[256];
   GemmPlan p;
   if (!gemm_plan(&p, A_KMAJOR, d_w_adapter, nullptr, sbf, B, d, d, sc.partial, msg, sizeof(msg), true))

@@ -87,8 +87,12 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
   const int G = a.Hq / a.Hkv;
   const int rows_total = a.T * G;
   const int g = blockIdx.y, qt = blockIdx.x, split = blockIdx.z;
-  const int L = a.pos0_dev ? *a.pos0_dev : a.pos0;
+  const int L = a.pos0_dev ? *a.pos0_dev + a.pos_off : a.pos0;
   const int nkeys = L + a.T;
+  // query token t sees keys [0, L + min(T, (t / blk + 1) blk)): causal is blk = 1, one
+  // bidirectional block blk = T, a pending block followed by a new one blk = B
+  const int blk = a.causal ? 1 : ((a.blk > 0 && a.blk < a.T) ? a.blk : a.T);
+  auto key_end = [&](int t) { const int e = (t / blk + 1) * blk; return L + (e < a.T ? e : a.T); };
   const int nsplit = attn_splits(nkeys, a.max_splits);
   if (split >= nsplit) return;
   int chunk = (nkeys + nsplit - 1) / nsplit;
@@ -96,10 +100,10 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
   const int k0 = split * chunk;
   int k1 = min(nkeys, k0 + chunk);
   const int row0 = qt * kAttnRows;
-  if (a.causal) {
-    // the last valid row of this CTA sees keys up to L + t_max
-    int rlast = min(rows_total, row0 + kAttnRows) - 1;
-    k1 = min(k1, L + rlast / G + 1);
+  {
+    // the last valid row of this CTA sees the most keys
+    const int rlast = min(rows_total, row0 + kAttnRows) - 1;
+    k1 = min(k1, key_end(rlast / G));
   }
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -151,8 +155,8 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
 
   // per-thread rows: gid and gid + 8 of the warp's 16
   const int rA = row0 + warp * 16 + gid, rB = rA + 8;
-  const int lim_A = a.causal ? (L + min(rA, rows_total - 1) / G) : (nkeys - 1);
-  const int lim_B = a.causal ? (L + min(rB, rows_total - 1) / G) : (nkeys - 1);
+  const int lim_A = key_end(min(rA, rows_total - 1) / G) - 1;
+  const int lim_B = key_end(min(rB, rows_total - 1) / G) - 1;
   const float sl2 = 1.4426950408889634f / sqrtf((float)HD);  // log2(e) / sqrt(hd)
   float m_A = -INFINITY, m_B = -INFINITY, l_A = 0.f, l_B = 0.f;
   float acc[HD / 8][4];
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(128) k_attn_combine(AttnArgs a) {
   const int G = a.Hq / a.Hkv;
   const int rows_total = a.T * G;
   const int Rows = a.Hkv * rows_total;
-  const int L = a.pos0_dev ? *a.pos0_dev : a.pos0;
+  const int L = a.pos0_dev ? *a.pos0_dev + a.pos_off : a.pos0;
   const int nsplit = attn_splits(L + a.T, a.max_splits);
   if (nsplit == 1) return;
   const int row = blockIdx.x;  // over Rows

@@ -200,7 +200,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUten
     const int row = quarter * 32 + lane;  // tile row = TMEM lane
     const int et = threadIdx.x - 64;      // 0 .. 127
     const EpiArgs& e = args.epi;
-    const int L = (e.op == EPI_QKV) ? (e.pos0_dev ? *e.pos0_dev : e.pos0) : 0;
+    const int L = (e.op == EPI_QKV) ? (e.pos0_dev ? *e.pos0_dev + e.pos_off : e.pos0) : 0;
     const int ncb = (args.T + 31) / 32;
     int acc = 0;
     uint32_t acc_phase = 0;

@@ -114,6 +114,7 @@ struct EpiArgs {
   int Hq, Hkv, hd, max_ctx;
   int pos0;
   const int* pos0_dev;
+  int pos_off;                  // added to *pos0_dev (graph mode): position of token 0
   const float2* rope_tab;       // (cos, sin) of position p, pair j at [p][j], j < hd/2
   float scale;                  // EPI_STORE: out = scale * y (0 means 1)
   float* h;                     // EPI_RESID / EPI_EMBED: [T][d]
@@ -174,13 +175,16 @@ cudaError_t gemm_fp4_launch(const GemmF4Plan& p, int* d_err, cudaStream_t s);
 int gemm_fp4_init_attributes();
 
 // LM head fused with the row statistics and s = P E (dlm_lmhead.cu), one pass over E.
-// x2: split bf16 pair, rows [0, T) high halves, rows [32, 32 + T) low halves; p_given:
-// bf16 [T][V] or nullptr (P = softmax of the logits).  T <= 32, d % 256 == 0, d <= 3072.
+// x2: split bf16 pair of x2_rows rows of d: the T high halves start at row hi_row, the T low
+// halves at row lo_row (both multiples of 8; rows past T up to 32 are read and dropped);
+// p_given: bf16 [T][V] or nullptr (P = softmax of the logits).  T <= 32, d % 256 == 0,
+// d <= 3072.
 bool lmhead_fused_supported(int T, int d);
 size_t lmhead_fused_scratch_bytes(int V, int d);
-cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_given, int T, int V, int d,
-                                int mask_id, dlm_row_stats stats, float* s, void* scratch, int* d_err,
-                                cudaStream_t st, char* err, size_t errlen);
+cudaError_t lmhead_fused_launch(const void* x2, int x2_rows, int hi_row, int lo_row, const void* E,
+                                const void* p_given, int T, int V, int d, int mask_id, dlm_row_stats stats,
+                                float* s, void* scratch, int* d_err, cudaStream_t st, char* err,
+                                size_t errlen);
 
 // attention (dlm_attention.cu)
 struct AttnArgs {
@@ -192,9 +196,12 @@ struct AttnArgs {
   float* part_o;             // [max_splits][Hkv * T * G][hd]
   float* part_ml;            // [max_splits][Hkv * T * G][2]
   int T, Hq, Hkv, hd, max_ctx;
-  int pos0;                  // prefix length L when pos0_dev == nullptr
-  const int* pos0_dev;       // device L (graph mode)
-  int causal;
+  int pos0;                  // position of query 0 when pos0_dev == nullptr
+  const int* pos0_dev;       // device prefix length (graph mode); query 0 at *pos0_dev + pos_off
+  int pos_off;
+  int causal;                // query t sees keys [0, pos0 + t]
+  int blk;                   // causal == 0: query t sees keys [0, pos0 + min(T, (t / blk + 1) blk));
+                             // blk == 0 or T: every query sees [0, pos0 + T) (one block)
   int max_splits;
   int* err;
 };

@@ -48,6 +48,7 @@ static_assert(kLmSmem <= 232448, "fused LM head shared memory");
 
 struct LmfArgs {
   int V, d, T, mask_id;
+  int x_hi_row, x_lo_row;  // rows of the split x where the high / low halves start
   int n_tiles, n_clu;
   int given;            // 1: P comes from memory (tp), s = P E without normalisation
   float* part_stats;    // [n_clu][32][4]: reference, Z, A, max
@@ -214,7 +215,9 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
         if (!ok) break;
         mbar_arrive_expect_tx(&full[stage], 16384 + 8192);
         tma_load_2d_hint(st, &tek, &full[stage], d0 + kb * 64, tile * 128, keep);
-        tma_load_2d_hint(st + 16384, &tx, &full[stage], d0 + kb * 64, 0, keep);
+        // x: 32 rows of high halves, then 32 rows of low halves (a 64-row K-major B operand)
+        tma_load_2d_hint(st + 16384, &tx, &full[stage], d0 + kb * 64, a.x_hi_row, keep);
+        tma_load_2d_hint(st + 16384 + 4096, &tx, &full[stage], d0 + kb * 64, a.x_lo_row, keep);
         advance();
       }
     };
@@ -623,10 +626,16 @@ bool lmhead_fused_supported(int T, int d) {
   return T >= 1 && T <= kLmT && d % 256 == 0 && d / 256 <= kLmMaxChunks;
 }
 
-// x2: split bf16 pair, rows [0, T) high halves and [32, 32 + T) low halves (pad = 32).
-cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_given, int T, int V, int d,
-                                int mask_id, dlm_row_stats stats, float* s, void* scratch, int* d_err,
-                                cudaStream_t st, char* err, size_t errlen) {
+// x2: split bf16 pair of x2_rows rows: the T high halves from row hi_row, the T low halves
+// from row lo_row.
+cudaError_t lmhead_fused_launch(const void* x2, int x2_rows, int hi_row, int lo_row, const void* E,
+                                const void* p_given, int T, int V, int d, int mask_id, dlm_row_stats stats,
+                                float* s, void* scratch, int* d_err, cudaStream_t st, char* err,
+                                size_t errlen) {
+  if (hi_row % 8 || lo_row % 8 || hi_row + 32 > x2_rows || lo_row + 32 > x2_rows) {
+    snprintf(err, errlen, "lm head: x rows %d / %d of %d", hi_row, lo_row, x2_rows);
+    return cudaErrorInvalidValue;
+  }
   {
     static PerDeviceOnce once;
     const int r = once_on_current_device(once, [] {
@@ -645,6 +654,8 @@ cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_giv
   a.d = d;
   a.T = T;
   a.mask_id = mask_id;
+  a.x_hi_row = hi_row;
+  a.x_lo_row = lo_row;
   a.n_tiles = (V + 127) / 128;
   a.n_clu = a.n_tiles < kLmMaxClusters ? a.n_tiles : kLmMaxClusters;
   a.given = p_given != nullptr;
@@ -655,7 +666,7 @@ cudaError_t lmhead_fused_launch(const void* x2, const void* E, const void* p_giv
   a.err = d_err;
   CUtensorMap tek, tem, tx, tp;
   if (!encode_bf16_2d(&tek, E, d, V, 64, 128, err, errlen) || !encode_bf16_2d(&tem, E, d, V, 64, 64, err, errlen) ||
-      !encode_bf16_2d(&tx, x2, d, 64, 64, 64, err, errlen))
+      !encode_bf16_2d(&tx, x2, d, x2_rows, 64, 32, err, errlen))
     return cudaErrorInvalidValue;
   if (p_given) {
     if (!encode_bf16_2d(&tp, p_given, V, T, 64, 32, err, errlen)) return cudaErrorInvalidValue;

@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(256) k_finish_qkv(FinishArgs a) {
   const int ra = (p / half) * e.hd + p % half, rb = ra + half;  // rows of the pair in the tile
   const int n = tile * kTileM + ra;                              // feature of row ra
   if (n >= a.N || t0 >= a.out.T) return;
-  const int L = e.pos0_dev ? *e.pos0_dev : e.pos0;
+  const int L = e.pos0_dev ? *e.pos0_dev + e.pos_off : e.pos0;
   float va[kFinTok], vb[kFinTok];
   finish_load_pair(a.out, tile, ra, rb, t0, va, vb);
   const int hh = n / e.hd, jj = n % e.hd;  // jj < half
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kRnThreads) k_resid_norm(ResNormArgs a) {
   const int tile0 = f0 >> 7, ntl = ((f0 + dq - 1) >> 7) - tile0 + 1;  // tiles of this CTA's features
   if (has_y && (int)threadIdx.x < ntl) nsl[threadIdx.x] = tile_slots(o, tile0 + threadIdx.x);
   __syncthreads();
-  const int tok = a.embed ? a.tokens[t] : 0;
+  const int tok = !a.embed ? 0 : ((a.tokens2 && t >= a.tok_split) ? a.tokens2[t - a.tok_split] : a.tokens[t]);
   float base[kFeat], x[kFeat][kSlotsReg];
   int ns[kFeat];
   const float* pp[kFeat];
@@ -274,12 +274,15 @@ __global__ void __launch_bounds__(kRnThreads) k_resid_norm(ResNormArgs a) {
   }
 }
 
-// Split bf16 copy of s (the W_a GEMM input): high halves at y[i], low halves at y[i + lo].
-__global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo) {
+// Split bf16 copy of s (the W_a GEMM input): high halves at y[i], low halves at y[i + lo];
+// the first zero_n elements of y are zero (rows without a residual input), x fills the n
+// after them.
+__global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo, long zero_n) {
   pdl_trigger();
   pdl_wait();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) store_split(y + i, lo, x[i]);
+  if (i < zero_n) store_split(y + i, lo, 0.f);
+  else if (i < zero_n + n) store_split(y + i, lo, x[i - zero_n]);
 }
 
 // Row statistics, phase 1: for logits[b][chunk] (mask id excluded) the chunk's max m_c,
@@ -470,13 +473,15 @@ __global__ void k_block_init(BlockInitArgs a) {
   for (long n = i; n < (long)a.B * a.d; n += (long)gridDim.x * blockDim.x) a.s[n] = 0.f;
 }
 
-// End of a block: copy tokens and {round, status} out, merge the kernel error flag into
-// the status, and advance the device prefix length by B.
+// End of a block: copy tokens and {round, status} out (and keep the tokens for the block's
+// deferred KV-fill), merge the kernel error flag into the status, and advance the device
+// prefix length by B.
 __global__ void k_block_finish(BlockFinishArgs a) {
   pdl_trigger();
   pdl_wait();
   const int i = threadIdx.x;
   if (i < a.B) a.tokens_out[i] = a.tokens[i];
+  if (i < a.B && a.pend_tokens) a.pend_tokens[i] = a.tokens[i];
   if (i == 0) {
     a.rounds_out[0] = *a.round;
     int st = *a.status;

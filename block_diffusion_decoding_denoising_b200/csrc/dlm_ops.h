@@ -20,7 +20,9 @@ struct ResNormArgs {
   GemmOut out;                 // partial sums of a GEMM with N = d (partial == nullptr: y = 0)
   float* h;                    // [T][d] residual stream
   const __nv_bfloat16* embed;  // non-null: h = E[tokens] + y instead of h += y
-  const int32_t* tokens;
+  const int32_t* tokens;       // token of row t < tok_split (all rows when tokens2 is null)
+  const int32_t* tokens2;      // token of row t >= tok_split: tokens2[t - tok_split]
+  int tok_split;
   float embed_scale;           // E rows are multiplied by it (1 for bf16 weights)
   const __nv_bfloat16* gain;   // [d]
   __nv_bfloat16* xn;           // [T][d] high halves
@@ -95,6 +97,7 @@ struct BlockFinishArgs {
   int32_t* tokens_out;
   int32_t* rounds_out;
   int* L_dev;
+  int32_t* pend_tokens;  // non-null: the block's tokens are kept for its deferred KV-fill
   int B;
 };
 
@@ -102,7 +105,7 @@ __global__ void k_finish_qkv(FinishArgs a);
 __global__ void k_finish_silu(FinishArgs a);
 __global__ void k_finish_store(FinishArgs a);
 __global__ void k_resid_norm(ResNormArgs a);
-__global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo);
+__global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo, long zero_n);
 __global__ void k_rowstats_part(RowStatsArgs a);
 __global__ void k_rowstats_final(RowStatsArgs a);
 __global__ void k_commit(CommitArgs a);

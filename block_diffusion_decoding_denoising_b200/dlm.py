@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(HERE, "libdlm.so")
 
 DLM_OK, DLM_EINVAL, DLM_ENOMEM_WS, DLM_EKVCAP, DLM_ECUDA, DLM_EROUNDCAP, DLM_ETIMEOUT, DLM_EUNSUPPORTED = range(8)
 COMMIT_THRESHOLD, COMMIT_TOPK = 0, 1
+FILL_EAGER, FILL_DEFERRED = 0, 1
 WEIGHTS_BF16, WEIGHTS_NVFP4 = 0, 1
 STATUS_NAMES = {0: "DLM_OK", 1: "DLM_EINVAL", 2: "DLM_ENOMEM_WS", 3: "DLM_EKVCAP", 4: "DLM_ECUDA",
                 5: "DLM_EROUNDCAP", 6: "DLM_ETIMEOUT", 7: "DLM_EUNSUPPORTED"}
@@ -94,6 +95,10 @@ def lib():
         L.dlm_block_init.argtypes = [p, C.POINTER(BlockState), p]
         L.dlm_round.argtypes = [p, C.POINTER(BlockState), f, i, i, p]
         L.dlm_kv_fill.argtypes = [p, p, p]
+        L.dlm_kv_flush.argtypes = [p, p]
+        L.dlm_fill_pending.argtypes = [p]
+        L.dlm_set_fill_mode.argtypes = [p, i, p]
+        L.dlm_mlp_block.argtypes = [p, i, p, p, i, p]
         L.dlm_decode_block.argtypes = [p, f, i, i, p, p, p]
         L.dlm_generate.argtypes = [p, p, i, i, f, i, i, p, p, C.POINTER(Timing), p]
         L.dlm_gemm_scratch_size.restype = z
@@ -391,6 +396,25 @@ class Model:
 
     def kv_fill(self, tokens, stream=None):
         _check(lib().dlm_kv_fill(self.ctx, _ptr(tokens), _stream(stream)), self.ctx)
+
+    def kv_flush(self, stream=None):
+        _check(lib().dlm_kv_flush(self.ctx, _stream(stream)), self.ctx)
+
+    @property
+    def fill_pending(self):
+        return bool(lib().dlm_fill_pending(self.ctx))
+
+    def set_fill_mode(self, mode, stream=None):
+        _check(lib().dlm_set_fill_mode(self.ctx, int(mode), _stream(stream)), self.ctx)
+
+    def mlp_block(self, layer, h, stream=None):
+        """One layer's MLP sub-block on fp32 residual rows h [T][d] (dlm_mlp_block)."""
+        import torch
+        h = h.contiguous()
+        out = torch.empty_like(h)
+        _check(lib().dlm_mlp_block(self.ctx, int(layer), _ptr(h), _ptr(out), int(h.shape[0]), _stream(stream)),
+               self.ctx)
+        return out
 
     def decode_block(self, tau, mode=COMMIT_THRESHOLD, k=1, tokens_out=None, rounds_out=None, stream=None):
         _check(lib().dlm_decode_block(self.ctx, float(tau), int(mode), int(k), _ptr(tokens_out), _ptr(rounds_out),

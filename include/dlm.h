@@ -57,6 +57,9 @@ typedef int dlm_status;
 #define DLM_COMMIT_THRESHOLD 0 /* commit max-prob >= tau, at least one per round */
 #define DLM_COMMIT_TOPK 1      /* commit the top min(k, remaining) by max-prob */
 
+#define DLM_FILL_EAGER 0    /* a block's KV-fill forward runs as soon as the block commits */
+#define DLM_FILL_DEFERRED 1 /* it is carried by the next round (default; see dlm_kv_fill) */
+
 #define DLM_WEIGHTS_BF16 0
 #define DLM_WEIGHTS_NVFP4 1 /* MLP and LM head in NVFP4, attention projections bf16 */
 
@@ -148,7 +151,9 @@ dlm_status dlm_ctx_destroy(dlm_ctx* ctx);
 const char* dlm_last_error(const dlm_ctx* ctx);
 /* Current prefix length L (positions of the KV cache holding committed context). */
 int dlm_prefix_len(const dlm_ctx* ctx);
-/* Sets L (0 <= L <= max_ctx - B).  Rows >= L of the KV cache are treated as free. */
+/* Sets L (0 <= L <= max_ctx - B).  Rows >= L of the KV cache are treated as free.  A pending
+ * KV-fill (see dlm_kv_fill) whose rows lie at or above the new L is dropped; otherwise it is
+ * run first. */
 dlm_status dlm_set_prefix_len(dlm_ctx* ctx, int L, void* stream);
 
 /* ---------------------------------------------------------------- decoding */
@@ -162,7 +167,8 @@ dlm_status dlm_block_init(dlm_ctx* ctx, const dlm_block_state* st, void* stream)
  * caller's state in place: embedding + residual adapter, the transformer layers with
  * block-diffusion attention (block K/V written to cache rows [L, L+B)), fused LM head
  * with row statistics and s = softmax(logits) E, then the commit rule.  tau is used by
- * DLM_COMMIT_THRESHOLD, tpf_k by DLM_COMMIT_TOPK. */
+ * DLM_COMMIT_THRESHOLD, tpf_k by DLM_COMMIT_TOPK.  If a KV-fill is pending, this round
+ * computes it in the same pass (see dlm_kv_fill). */
 dlm_status dlm_round(dlm_ctx* ctx, const dlm_block_state* st, float tau, int commit_mode,
                      int tpf_k, void* stream);
 /*   [blog "ORL: diffusion LLMs get a learnable 'tokens per forward'", "What shipped": a
@@ -171,14 +177,30 @@ dlm_status dlm_round(dlm_ctx* ctx, const dlm_block_state* st, float tau, int com
  *   evaluation pipeline": SDARPrefixKV attention, SDAR_FUSED_ROW_STATS, SDAR_COMMIT_GRAPH] */
 
 /* Clean forward of a committed block (s = 0, no LM head) writing its K/V to rows
- * [L, L+B); then L += B.  d_tokens int32 [B]. */
+ * [L, L+B); then L += B.  d_tokens int32 [B].
+ * In DLM_FILL_DEFERRED mode (the default, on contexts with bf16 weights, B <= 32 and the
+ * fused LM head) the call only records the block as pending: the next dlm_round (or the
+ * next block's graph) prepends the pending block's B rows to its own B rows and computes
+ * both in one pass over the weights; the pending rows see the prefix and their own block,
+ * the new rows see everything, so the K/V rows written are those of the separate forward
+ * (up to fp32 summation order).  Until then rows [L - B, L) of the cache are not valid:
+ * dlm_kv_flush writes them.  Other contexts run the forward at once. */
 dlm_status dlm_kv_fill(dlm_ctx* ctx, const int32_t* d_tokens, void* stream);
+
+/* Runs a pending KV-fill on its own (no-op if none is pending). */
+dlm_status dlm_kv_flush(dlm_ctx* ctx, void* stream);
+/* 1 if a KV-fill is pending, 0 if not, -1 for a null context. */
+int dlm_fill_pending(const dlm_ctx* ctx);
+/* DLM_FILL_EAGER or DLM_FILL_DEFERRED (switching to eager runs a pending fill first). */
+dlm_status dlm_set_fill_mode(dlm_ctx* ctx, int mode, void* stream);
 
 /* Decodes one whole block on the device: one launch of a CUDA graph that initialises
  * the block, loops rounds in a while-conditional node until every position is committed
- * (or B rounds), then runs the KV-fill forward.  Writes d_tokens_out int32 [B] and
- * d_rounds_out int32 [2] = {rounds, device status}.  L += B (host and device).  The graph
- * is instantiated on first use per (commit mode, tau, k) and reused. */
+ * (or B rounds), then runs the block's KV-fill.  Writes d_tokens_out int32 [B] and
+ * d_rounds_out int32 [2] = {rounds, device status}.  L += B (host and device).  In
+ * DLM_FILL_DEFERRED mode the KV-fill is left pending (see dlm_kv_fill) and the next block's
+ * graph carries it in its first round: one weight stream per block less.  The graph is
+ * instantiated on first use per (commit mode, tau, k, fill variant) and reused. */
 dlm_status dlm_decode_block(dlm_ctx* ctx, float tau, int commit_mode, int tpf_k,
                             int32_t* d_tokens_out, int32_t* d_rounds_out, void* stream);
 /*   [blog, "What shipped", "dlmrt, the inference engine": one CUDA graph per block with a
@@ -186,8 +208,9 @@ dlm_status dlm_decode_block(dlm_ctx* ctx, float tau, int commit_mode, int tpf_k,
  *   block and reads back tokens] */
 
 /* Host-level generation: copies the prompt to the device, prefills it at L = 0, decodes
- * ceil(max_new / B) blocks with dlm_decode_block, reading each block's tokens back, and
- * returns max_new tokens (the last block truncated) and the rounds of every block.
+ * ceil(max_new / B) blocks with dlm_decode_block, reading each block's tokens back, runs the
+ * last block's pending KV-fill (the cache holds every block on return), and returns max_new
+ * tokens (the last block truncated) and the rounds of every block.
  * Synchronizes.  h_prompt int32 [prompt_len]; h_tokens_out int32 [max_new];
  * h_rounds_per_block int32 [ceil(max_new/B)] (may be NULL); h_timing may be NULL. */
 dlm_status dlm_generate(dlm_ctx* ctx, const int32_t* h_prompt, int prompt_len, int max_new,
@@ -261,6 +284,13 @@ dlm_status dlm_bd_attention(const void* d_q, const void* d_k_cache, const void* 
 dlm_status dlm_bd_attention_noalloc(const void* d_q, const void* d_k_cache, const void* d_v_cache,
                                     void* d_o, int T, int L, int Hq, int Hkv, int hd, int max_ctx,
                                     int causal, void* stream);
+
+/* One layer's MLP sub-block on given residual rows (single operation for parity tests):
+ * h_out = h_in + W_down (silu(W_gate x) * (W_up x)), x = RMSNorm(h_in) g_mlp, with the
+ * context's weights of that layer (for NVFP4 weights x and the SiLU output are quantized per
+ * row, as in a round).  d_h_in, d_h_out fp32 [T][d]; T <= 32 (NVFP4) or <= 128.  Uses the
+ * context's workspace: not concurrent with other calls on the context. */
+dlm_status dlm_mlp_block(dlm_ctx* ctx, int layer, const float* d_h_in, float* d_h_out, int T, void* stream);
 
 /* Commit rule on device arrays (one block of B positions).  Updates tokens, committed,
  * zeroes the s rows of newly committed positions, increments *d_round. */

@@ -82,6 +82,10 @@ def test_null_context_calls(L):
     assert L.dlm_generate(None, None, 0, 0, 0.9, 0, 1, None, None, None, None) == dlm.DLM_EINVAL
     assert L.dlm_prefill(None, None, 0, None) == dlm.DLM_EINVAL
     assert L.dlm_kv_fill(None, None, None) == dlm.DLM_EINVAL
+    assert L.dlm_kv_flush(None, None) == dlm.DLM_EINVAL
+    assert L.dlm_fill_pending(None) == -1
+    assert L.dlm_set_fill_mode(None, dlm.FILL_DEFERRED, None) == dlm.DLM_EINVAL
+    assert L.dlm_mlp_block(None, 0, None, None, 1, None) == dlm.DLM_EINVAL
     assert L.dlm_set_prefix_len(None, 0, None) == dlm.DLM_EINVAL
 
 
