@@ -176,7 +176,8 @@ int gemm_fp4_init_attributes();
 
 // LM head fused with the row statistics and s = P E (dlm_lmhead.cu), one pass over E.
 // x2: split bf16 pair of x2_rows rows of d: the T high halves start at row hi_row, the T low
-// halves at row lo_row (both multiples of 8; rows past T up to 32 are read and dropped);
+// halves at row lo_row (both multiples of 8; the 32 rows from each are read, those past T
+// dropped, those past x2_rows read as zeros);
 // p_given: bf16 [T][V] or nullptr (P = softmax of the logits).  T <= 32, d % 256 == 0,
 // d <= 3072.
 bool lmhead_fused_supported(int T, int d);

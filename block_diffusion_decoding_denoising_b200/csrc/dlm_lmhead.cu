@@ -632,8 +632,10 @@ cudaError_t lmhead_fused_launch(const void* x2, int x2_rows, int hi_row, int lo_
                                 const void* p_given, int T, int V, int d, int mask_id, dlm_row_stats stats,
                                 float* s, void* scratch, int* d_err, cudaStream_t st, char* err,
                                 size_t errlen) {
-  if (hi_row % 8 || lo_row % 8 || hi_row + 32 > x2_rows || lo_row + 32 > x2_rows) {
-    snprintf(err, errlen, "lm head: x rows %d / %d of %d", hi_row, lo_row, x2_rows);
+  // the 32-row boxes may reach past the buffer (TMA fills those rows with zeros, and columns
+  // past T are dropped); the T live rows of each half must lie inside it
+  if (hi_row % 8 || lo_row % 8 || hi_row < 0 || lo_row < 0 || hi_row + T > x2_rows || lo_row + T > x2_rows) {
+    snprintf(err, errlen, "lm head: x rows %d / %d (+%d) of %d", hi_row, lo_row, T, x2_rows);
     return cudaErrorInvalidValue;
   }
   {
