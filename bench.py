@@ -45,7 +45,7 @@ def parse(argv=None):
     # profiling cases (small, for ncu): "quick" = the decode loop on 256 generated tokens
     # without the extra measurements; "gemm" = every projection GEMM of two layers plus
     # the LM-head GEMM, `--steps` launches each
-    ap.add_argument("--case", default="full", choices=["full", "quick", "gemm", "lmhead"])
+    ap.add_argument("--case", default="full", choices=["full", "quick", "gemm", "lmhead", "attention"])
     # the quick case with eager dlm_round / dlm_kv_fill calls instead of the block graph
     # (same kernels; ncu cannot profile kernel nodes of graphs with conditional nodes)
     ap.add_argument("--eager", action="store_true")
@@ -397,8 +397,52 @@ def attention_sweep(args, dev):
             cells.append({"B": B, "L": L, "us": round(t * 1e6, 2), "GBs": round(gbs, 1),
                           "frac": round(gbs / hbm, 4), "frac_nominal": round(gbs / NOMINAL_HBM_GBS, 4)})
             del q, kc, vc, o, sc
-    return {"workload": "block-diffusion attention, 32/8 heads, hd 128, bf16, q/K/V N(0,1)",
+    return {"workload": "block-diffusion attention (dlm_bd_attention: split key range + merge), 32/8 heads, hd 128, "
+                        "bf16, q/K/V N(0,1)",
             "l2": "flushed (256 MB written) before every call", "cells": cells}
+
+
+def attention_case(args):
+    """The attention of the rounds (split key range + merge, dlm_bd_attention) on 32/8 heads,
+    hd 128: T in {32, 64} against L in {512, 2560, 4096, 16384, 65536}, `--steps` calls each,
+    warm (back to back) and cold (L2 flushed before each call)."""
+    import ctypes as C
+
+    import torch
+
+    from block_diffusion_decoding_denoising_b200 import build, dlm, gen
+    build.build()
+    dev = torch.device("cuda", 0)
+    lib = dlm.lib()
+    sp = C.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    flush = _l2_flusher(dev)
+    out = []
+    for T in (32, 64):
+        for L in (512, 2560, 4096, 16384, 65536):
+            q, kc, vc = gen.attention_inputs_torch(T, L, device=dev, seed=3)
+            o = torch.empty_like(q)
+            Hq, hd, Hkv, mc = q.shape[1], q.shape[2], kc.shape[0], kc.shape[1]
+            n = lib.dlm_attention_scratch_size(T, Hq, hd, mc)
+            sc = torch.empty(n, dtype=torch.uint8, device=dev)
+            p = [C.c_void_p(t.data_ptr()) for t in (q, kc, vc, o)]
+            calls = {"split": lambda: lib.dlm_bd_attention(*p, T, L, Hq, Hkv, hd, mc, 0, C.c_void_p(sc.data_ptr()),
+                                                           n, sp)}
+            row = {"T": T, "L": L}
+            for name, fn in calls.items():
+                for _ in range(3):
+                    fn()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(args.steps):
+                    fn()
+                e1.record()
+                torch.cuda.synchronize()
+                row[name + "_warm_us"] = round(e0.elapsed_time(e1) * 1e3 / args.steps, 2)
+                row[name + "_cold_us"] = round(_timed_calls(fn, args.steps, flush) * 1e6, 2)
+            out.append(row)
+            del q, kc, vc, o, sc
+    print(json.dumps({"case": "attention", "rows": out}), flush=True)
 
 
 def lmhead_measure(args, w, dev):
@@ -547,6 +591,9 @@ def main():
         return
     if args.case == "lmhead":
         lmhead_case(args)
+        return
+    if args.case == "attention":
+        attention_case(args)
         return
     if args.case == "quick":
         GEN = 256
