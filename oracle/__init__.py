@@ -41,7 +41,7 @@ class Cfg(C.Structure):
                 ("n_kv_heads", C.c_int), ("head_dim", C.c_int), ("ffn", C.c_int),
                 ("vocab", C.c_int), ("mask_id", C.c_int), ("block_size", C.c_int),
                 ("rope_theta", C.c_double), ("rms_eps", C.c_double),
-                ("act_round", C.c_int), ("act_fp4", C.c_int)]
+                ("act_round", C.c_int), ("act_fp4", C.c_int), ("kv_fp8", C.c_int)]
 
 
 class Layer(C.Structure):
@@ -101,6 +101,8 @@ def lib():
         L.orc_rope.argtypes = [p, i, C.c_long, d]
         L.orc_attention.argtypes = [p, i, i, i, i, p, p, i, i, i, p]
         L.orc_rowstats.argtypes = [p, i, i, i, C.POINTER(Stats)]
+        L.orc_kv_quantize_row.restype = C.c_float
+        L.orc_kv_quantize_row.argtypes = [p, i, p, p]
         L.orc_lmhead.argtypes = [p, i, C.POINTER(Mat), i, i, p, C.POINTER(Stats), p, p]
         L.orc_commit.restype = i
         L.orc_commit.argtypes = [i, p, p, d, i, i, p, p]
@@ -155,6 +157,22 @@ def e4m3_round(x: float) -> float:
 
 def e4m3_bits(v: float) -> int:
     return int(lib().orc_e4m3_bits(float(v)))
+
+
+def kv_quantize(rows):
+    """FP8 KV rows (R13): float [n][hd] -> (codes uint8 [n][hd], scales fp32 [n], values [n][hd])."""
+    x = _c(np.atleast_2d(rows), np.float64)
+    n, hd = x.shape
+    codes = np.zeros((n, hd), np.uint8)
+    vals = np.zeros((n, hd), np.float64)
+    scales = np.zeros(n, np.float32)
+    for r in range(n):
+        xr = np.ascontiguousarray(x[r])
+        cr = np.zeros(hd, np.uint8)
+        vr = np.zeros(hd, np.float64)
+        scales[r] = lib().orc_kv_quantize_row(_ptr(xr), hd, _ptr(cr), _ptr(vr))
+        codes[r], vals[r] = cr, vr
+    return codes, scales, vals
 
 
 def e4m3_value(b: int) -> float:
@@ -297,7 +315,7 @@ class OracleModel:
         nvfp4 = bool(c.get("weight_fmt", 0))
         self.cfg = Cfg(c["n_layers"], c["d"], c["n_q_heads"], c["n_kv_heads"], c["head_dim"],
                        c["ffn"], c["vocab"], c["mask_id"], c["block_size"], float(c["rope_theta"]),
-                       float(c["rms_eps"]), int(act_round), int(nvfp4))
+                       float(c["rms_eps"]), int(act_round), int(nvfp4), int(c.get("kv_fmt", 0)))
         layers = (Layer * c["n_layers"])()
         for i, lw in enumerate(weights["layers"]):
             layers[i] = Layer(self.wk.vec(lw["attn_norm"]), self.wk.mat(lw["w_qkv"]),

@@ -51,6 +51,11 @@
 //      the attention takes bf16 queries, so with act_round set the oracle rounds q, k and v
 //      to bf16 (round-to-nearest-even) after RoPE, as they are stored; integer decisions
 //      are then taken on the same attention operands.  Every other value stays fp64.
+//   R13 FP8 KV cache (option kv_fp8; [blog] "What shipped", "dlmrt, the inference engine":
+//      the KV cache is FP8): every K and V row of hd values (one layer, one KV head, one
+//      position) is stored as OCP e4m3 codes with one fp32 scale s = amax(|row|) / 448, code =
+//      RNE_e4m3(x / s) saturating at 448, value = e4m3(code) * s.  q stays bf16 (R9); the K
+//      and V rows are quantized from their unrounded values.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -246,6 +251,7 @@ typedef struct orc_cfg {
   double rope_theta, rms_eps;
   int act_round;      // R9
   int act_fp4;        // NVFP4 GEMMs quantize their input rows (R8); 0 for bf16 models
+  int kv_fp8;         // R13
 } orc_cfg;
 
 typedef struct orc_layer {
@@ -279,6 +285,27 @@ typedef struct orc_stats {
   double qmargin;  // smallest margin of the row's NVFP4 activation rounding decisions
                    // (e2m1_margin / e4m3_margin) in the forward pass; +inf without any
 } orc_stats;
+
+// FP8 KV row (R13): n values -> e4m3 codes and one fp32 scale amax / 448; `out` (optional)
+// receives the stored values e4m3(code) * scale.  Returns the scale.
+float orc_kv_quantize_row(const double* x, int n, uint8_t* codes, double* out) {
+  float amax = 0.0f;
+  for (int i = 0; i < n; ++i) amax = std::max(amax, std::fabs(float(x[i])));
+  const float s = amax / 448.0f;
+  for (int i = 0; i < n; ++i) {
+    double v = 0.0;
+    uint8_t c = 0;
+    if (s > 0.0f) {
+      const float r = float(x[i]) / s;
+      const double q = round_e4m3_nonneg(std::fabs(r));  // magnitude, RNE, saturating
+      c = uint8_t(e4m3_bits(q) | (r < 0.0f ? 0x80 : 0));
+      v = (r < 0.0f ? -q : q) * double(s);
+    }
+    if (codes) codes[i] = c;
+    if (out) out[i] = v;
+  }
+  return s;
+}
 
 void orc_set_threads(int n) { g_threads = n; }
 int orc_hw_threads(void) { return int(std::thread::hardware_concurrency()); }
@@ -592,7 +619,11 @@ void forward(const orc_model& M, const orc_cfg& C, const int* tokens, const doub
       double* row = qkv.data() + size_t(i) * nqkv;
       long pos = pos0 + i;
       for (int hh = 0; hh < Hq + Hkv; ++hh) rope(row + hh * hd, hd, pos, C.rope_theta);
-      for (int e = 0; e < nqkv; ++e) row[e] = maybe_round(row[e], rnd);
+      const bool fp8 = C.kv_fp8 != 0;
+      for (int e = 0; e < nqkv; ++e)
+        if (!(fp8 && e >= Hq * hd)) row[e] = maybe_round(row[e], rnd);  // K/V rows: see R13 below
+      if (fp8)
+        for (int hh = Hq; hh < Hq + 2 * Hkv; ++hh) orc_kv_quantize_row(row + hh * hd, hd, nullptr, row + hh * hd);
       for (int hh = 0; hh < Hq; ++hh)
         std::memcpy(q.data() + (size_t(i) * Hq + hh) * hd, row + hh * hd, hd * sizeof(double));
       for (int gg = 0; gg < Hkv; ++gg) {

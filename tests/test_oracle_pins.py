@@ -653,3 +653,81 @@ def test_pin_attention_sub_block_closed_form(tiny):
     ob = np.concatenate(o_bad)
     bad = _rms(E[tok] + de * ob[(np.arange(d) + 1) % d], gf, eps)
     assert np.abs(bad - xf[0]).max() > 1e-4
+
+
+# ------------------------------------------------------------------ FP8 KV cache (reading R13)
+def test_kv_fp8_rows_on_the_e4m3_grid_round_trip():
+    # rows made of golden e4m3 values (OCP OFP8 E4M3, tests/golden/e4m3_values.txt) times a
+    # power of two, with 448 present: the scale is exactly that power of two and every value
+    # and code comes back unchanged
+    table = [(int(b, 0), float(v)) for b, v in _golden_table("e4m3_values.txt")]
+    vals = np.array([v for _, v in table] + [448.0])
+    signs = np.where(np.arange(len(vals)) % 3 == 1, -1.0, 1.0)
+    for p2 in (2.0 ** -7, 1.0, 2.0 ** 5):
+        row = np.resize(vals * signs, 32) * p2
+        row[5] = 448.0 * p2
+        codes, scales, out = O.kv_quantize(row)
+        assert scales[0] == np.float32(p2)
+        np.testing.assert_array_equal(out[0], row)
+        for c, x in zip(codes[0], row / p2):
+            assert O.e4m3_value(int(c) & 0x7F) == abs(x) and (int(c) >> 7) == (1 if x < 0 else 0)
+
+
+def test_kv_fp8_idempotent_error_bound_saturation_and_zero_rows():
+    x = gen.normal_np(91, 8 * 128, 1.7).reshape(8, 128)
+    x[3] *= 1e-3
+    x[5] = 0.0
+    codes, scales, out = O.kv_quantize(x)
+    for r in range(8):
+        if r == 5:
+            assert scales[r] == 0.0 and np.all(codes[r] == 0) and np.all(out[r] == 0.0)
+            continue
+        s = float(scales[r])
+        assert s == np.float32(np.float32(np.abs(x[r]).max()) / np.float32(448.0))
+        j = int(np.argmax(np.abs(x[r])))
+        assert int(codes[r][j]) & 0x7F == 0x7E  # the amax element is +-448 * s
+        # e4m3 keeps 4 significant bits: relative error at most 2^-4 in the normal range, and at
+        # most half the subnormal quantum (2^-10 * s) below it
+        err = np.abs(out[r] - x[r])
+        assert np.all(err <= np.maximum(np.abs(x[r]) * 2.0 ** -4, 2.0 ** -10 * s) * (1 + 1e-6))
+        c2, s2, out2 = O.kv_quantize(out[r])
+        np.testing.assert_array_equal(out2[0], out[r])
+
+
+def test_pin_kv_fp8_applies_to_k_and_v_rows_only(tiny):
+    # the structured attention sub-block above with an FP8 KV cache: the cached K and V rows are
+    # the quantized closed forms, and the attention reads those stored values
+    cfg, w2, lw, ga, gm, gf = _closed_form_layer_setup(tiny)
+    cfg = dict(cfg, kv_fmt=1)
+    d, hd, F = cfg["d"], cfg["head_dim"], cfg["ffn"]
+    perm = (np.arange(hd) * 5 + 11) % d
+    Wqkv = np.zeros((4 * hd, d))
+    Wqkv[np.arange(32), np.arange(32)] = 1.5
+    Wqkv[32 + np.arange(32), 32 + np.arange(32)] = 0.75
+    Wqkv[64 + np.arange(32), 16 + np.arange(32)] = 1.0
+    Wqkv[96 + np.arange(32), perm] = 2.0
+    Wo = np.zeros((d, 2 * hd))
+    Wo[np.arange(d), np.arange(d)] = 1.0
+    lw.update(w_qkv=bits(Wqkv), w_o=bits(Wo), w_down=bits(np.zeros((d, F))))
+    w2["layers"] = [lw]
+    m = O.OracleModel(cfg, w2, act_round=False)
+    p, base, eps, tok = 3, cfg["rope_theta"], cfg["rms_eps"], 123
+    Kp = O.kv_quantize(gen.normal_np(63, p * hd).reshape(p, hd))[2]
+    Vp = O.kv_quantize(gen.normal_np(64, p * hd).reshape(p, hd))[2]
+    m.kc[0, 0, :p] = Kp
+    m.vc[0, 0, :p] = Vp
+    xf = m.forward(np.array([tok], np.int32), None, p)
+    E = gen.bf16_to_f64(w2["embed"])
+    xn = _rms(E[tok], ga, eps)
+    k = O.kv_quantize(_rope_np(xn[16:48], p, base))[2][0]
+    v = O.kv_quantize(2.0 * xn[perm])[2][0]
+    np.testing.assert_array_equal(m.kc[0, 0, p], k)
+    np.testing.assert_array_equal(m.vc[0, 0, p], v)
+    q = [_rope_np(1.5 * xn[0:32], p, base), _rope_np(0.75 * xn[32:64], p, base)]  # q not quantized
+    K, V = np.vstack([Kp, k]), np.vstack([Vp, v])
+    o = []
+    for qh in q:
+        sc = K @ qh / np.sqrt(hd)
+        e = np.exp(sc - sc.max())
+        o.append(e @ V / e.sum())
+    np.testing.assert_allclose(xf[0], _rms(E[tok] + np.concatenate(o), gf, eps), rtol=1e-11, atol=1e-13)
