@@ -445,6 +445,84 @@ def attention_case(args):
     print(json.dumps({"case": "attention", "rows": out}), flush=True)
 
 
+def fp8_kv_measure(args, cfg, w, prompt, dev, stream):
+    """Decode tokens/s with the FP8 KV cache (bf16 weights; same schedule as the main line)."""
+    import torch
+
+    from block_diffusion_decoding_denoising_b200 import dlm
+    c8 = dict(cfg)
+    c8["kv_fmt"] = dlm.KV_FP8
+    m = dlm.Model(c8, w, device=dev)
+    B = c8["block_size"]
+    blocks = GEN // B
+    tok = torch.zeros((blocks, B), dtype=torch.int32, device=dev)
+    rr = torch.zeros((blocks, 2), dtype=torch.int32, device=dev)
+    m.prefill(prompt)
+
+    def step():
+        m.set_prefix_len(PROMPT)
+        for b in range(blocks):
+            m.decode_block(TAU, dlm.COMMIT_TOPK, TPF_K, tok[b], rr[b])
+        m.kv_flush()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert int(rr[:, 1].abs().sum().item()) == 0, "device status"
+    ms = e0.elapsed_time(e1) / args.steps
+    m.close()
+    return {"tokens_per_s": GEN / (ms / 1e3), "ms_per_step": ms,
+            "kv_cache_bytes_per_position": 2 * cfg["n_layers"] * cfg["n_kv_heads"] * (cfg["head_dim"] + 4)}
+
+
+def attention_fp8_cells(args, dev):
+    """Config-3 cells on an FP8 KV cache (e4m3 rows + fp32 row scales): algorithmic bytes
+    8 (L + B) (hd + 4) for K/V and their scales + 16384 B for q and o."""
+    import ctypes as C
+
+    import torch
+
+    from block_diffusion_decoding_denoising_b200 import dlm, gen
+    lib = dlm.lib()
+    sp = C.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    hbm, _, kind = peaks()
+    flush = _l2_flusher(dev)
+    cells = []
+    for L in (16384, 65536):
+        for B in (4, 32):
+            q, kc, vc = gen.attention_inputs_torch(B, L, device=dev, seed=3)
+            Hq, hd, Hkv, mc = q.shape[1], q.shape[2], kc.shape[0], kc.shape[1]
+            mc4 = (mc + 3) // 4 * 4
+            # synthetic e4m3 rows (NaN codes excluded) with one scale per row
+            g = torch.Generator(device=dev)
+            g.manual_seed(5)
+            codes = [torch.randint(0, 126, (Hkv, mc4, hd), generator=g, device=dev, dtype=torch.int32).to(torch.uint8)
+                     for _ in range(2)]
+            scales = [torch.full((Hkv, mc4), 3.0 / 448.0, device=dev) for _ in range(2)]
+            o = torch.empty_like(q)
+            n = lib.dlm_attention_scratch_size(B, Hq, hd, mc4)
+            sc = torch.empty(n, dtype=torch.uint8, device=dev)
+            p = [C.c_void_p(t.data_ptr()) for t in (q, codes[0], scales[0], codes[1], scales[1], o)]
+            fn = lambda: lib.dlm_bd_attention_fp8(*p, B, L, Hq, Hkv, hd, mc4, 0, C.c_void_p(sc.data_ptr()), n, sp)
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            t = _timed_calls(fn, 5, flush)
+            nbytes = 2 * Hkv * (L + B) * (hd + 4) + 16384 * B
+            gbs = nbytes / t / 1e9
+            cells.append({"B": B, "L": L, "us": round(t * 1e6, 2), "GBs": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                          "frac_nominal": round(gbs / NOMINAL_HBM_GBS, 4)})
+            del q, kc, vc, codes, scales, o, sc
+    return {"workload": "block-diffusion attention on an FP8 KV cache (dlm_bd_attention_fp8), 32/8 heads, hd 128",
+            "l2": "flushed (256 MB written) before every call", "cells": cells}
+
+
 def lmhead_measure(args, w, dev):
     """The fused LM head (row statistics and s = P E in one pass over E) on the model's E."""
     import torch
@@ -770,12 +848,15 @@ def main():
     # on the MLP shapes (partial sums only, inputs quantized per row)
     m.close()
     nv = nvfp4_measure(args, cfg, w, prompt, dev, stream)
+    # the same decode on an FP8 KV cache
+    kv8 = fp8_kv_measure(args, cfg, w, prompt, dev, stream)
     # the fused LM head alone (LM-head configuration shapes: B 32, d 2560, V 151936, P = softmax)
     lm = lmhead_measure(args, w, dev)
     del w
     torch.cuda.empty_cache()
     c2 = config2_measure(args, dev)
     c3 = attention_sweep(args, dev)
+    c3["fp8_kv"] = attention_fp8_cells(args, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -809,7 +890,7 @@ def main():
                       "round_roofline_frac_nominal": step_bytes / (ms_step / 1e3) / 1e9 / NOMINAL_HBM_GBS,
                       "tau0.9_rounds_per_s": tau_rounds_per_s, "tau0.9_rounds_per_block": tau_rounds / 4,
                       "gemm_avg_launch_us": gemm_s * 1e6, "gemm_all_shapes_GBs": gemm_avg_gbs,
-                      "nvfp4": nv, "lmhead_fused": lm, "config2_lmhead_given_p": c2, "config3_attention": c3},
+                      "nvfp4": nv, "fp8_kv": kv8, "lmhead_fused": lm, "config2_lmhead_given_p": c2, "config3_attention": c3},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -54,7 +54,7 @@ struct dlm_ctx {
   std::vector<dlm_layer_weights> layers;
   uint8_t* ws = nullptr;
   size_t ws_bytes = 0;
-  __nv_bfloat16* kv = nullptr;
+  uint8_t* kv = nullptr;   // KV cache values (bf16 or e4m3), then for FP8 the row scales
   size_t kv_bytes = 0;
   int L = 0;
   int Tmax = 0;
@@ -291,6 +291,11 @@ bool valid_cfg(const dlm_config* c, char* msg, size_t n) {
     snprintf(msg, n, "invalid weight_fmt %d", c->weight_fmt);
     return false;
   }
+  // FP8 cache: the row scales are read in 16-byte groups of 4 (max_ctx a multiple of 4)
+  if ((c->kv_fmt != DLM_KV_BF16 && c->kv_fmt != DLM_KV_FP8) || (c->kv_fmt == DLM_KV_FP8 && c->max_ctx % 4)) {
+    snprintf(msg, n, "invalid kv_fmt %d (FP8 needs max_ctx %% 4 == 0)", c->kv_fmt);
+    return false;
+  }
   return true;
 }
 
@@ -479,17 +484,30 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     TRY(resid_norm(r, T, nullptr, tok0, first_gain, false, tok1, Tp));
   }
 
-  const size_t layer_kv = (size_t)Hkv * c.max_ctx * hd;
+  // KV cache planes of layer l: [K|V][Hkv][max_ctx][hd] values (bf16, or e4m3 bytes followed,
+  // after all layers' values, by the fp32 row scales [layer][K|V][Hkv][max_ctx])
+  const bool kv8 = c.kv_fmt == DLM_KV_FP8;
+  const size_t plane_rows = (size_t)Hkv * c.max_ctx;
+  const size_t plane_bytes = plane_rows * hd * (kv8 ? 1 : 2);
+  float* const kv_scales = kv8 ? reinterpret_cast<float*>(ctx->kv + (size_t)2 * c.n_layers * plane_bytes) : nullptr;
   for (int l = 0; l < c.n_layers; ++l) {
     const dlm_layer_weights& W = ctx->layers[l];
-    __nv_bfloat16* kc = ctx->kv + (size_t)(2 * l) * layer_kv;
-    __nv_bfloat16* vc = ctx->kv + (size_t)(2 * l + 1) * layer_kv;
+    uint8_t* kp = ctx->kv + (size_t)(2 * l) * plane_bytes;
+    uint8_t* vp = ctx->kv + (size_t)(2 * l + 1) * plane_bytes;
+    __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(kp);
+    __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(vp);
+    float* ks = kv8 ? kv_scales + (size_t)(2 * l) * plane_rows : nullptr;
+    float* vs = kv8 ? kv_scales + (size_t)(2 * l + 1) * plane_rows : nullptr;
     TRY(r.gemm_partial(A_KMAJOR, W.w_qkv, nullptr, ctx->xn, T, nqkv, d, &y));
     EpiArgs eq{};
     eq.op = EPI_QKV;
     eq.q = ctx->q;
-    eq.kc = kc;
-    eq.vc = vc;
+    eq.kc = kv8 ? nullptr : kc;
+    eq.vc = kv8 ? nullptr : vc;
+    eq.kc8 = kv8 ? kp : nullptr;
+    eq.vc8 = kv8 ? vp : nullptr;
+    eq.ks = ks;
+    eq.vs = vs;
     eq.Hq = Hq;
     eq.Hkv = Hkv;
     eq.hd = hd;
@@ -506,6 +524,8 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
     aa.q = ctx->q;
     aa.kc = kc;
     aa.vc = vc;
+    aa.ks = ks;
+    aa.vs = vs;
     aa.o = ctx->o;
     aa.o_lo = pad * ho;
     aa.part_o = ctx->attn_part;
@@ -775,7 +795,8 @@ size_t dlm_workspace_size(const dlm_config* cfg) {
 size_t dlm_kv_cache_size(const dlm_config* c) {
   char msg[128];
   if (!valid_cfg(c, msg, sizeof(msg))) return 0;
-  return (size_t)2 * c->n_layers * c->n_kv_heads * c->max_ctx * c->head_dim * 2;
+  const size_t rows = (size_t)2 * c->n_layers * c->n_kv_heads * c->max_ctx;
+  return c->kv_fmt == DLM_KV_FP8 ? rows * c->head_dim + rows * 4 : rows * c->head_dim * 2;
 }
 
 dlm_status dlm_ctx_create(const dlm_config* cfg, const dlm_weights* w, void* d_workspace,
@@ -809,7 +830,7 @@ dlm_status dlm_ctx_create(const dlm_config* cfg, const dlm_weights* w, void* d_w
   ctx->w.layers = ctx->layers.data();
   ctx->ws = (uint8_t*)d_workspace;
   ctx->ws_bytes = ws_bytes;
-  ctx->kv = (__nv_bfloat16*)d_kv_cache;
+  ctx->kv = (uint8_t*)d_kv_cache;
   ctx->kv_bytes = kv_bytes;
   carve(ctx, *cfg, ctx->ws);
   cudaError_t e = cudaStreamCreateWithFlags(&ctx->cap_stream, cudaStreamNonBlocking);
@@ -1308,6 +1329,37 @@ dlm_status dlm_bd_attention(const void* d_q, const void* d_k_cache, const void* 
   a.part_ml = a.part_o + (size_t)a.max_splits * T * Hq * hd;
   a.err = nullptr;  // the attention kernels have no waits and report nothing on the device
   CU(attention_launch(a, s));
+  return DLM_OK;
+}
+
+dlm_status dlm_bd_attention_fp8(const void* d_q, const void* d_k_codes, const float* d_k_scales, const void* d_v_codes,
+                                const float* d_v_scales, void* d_o, int T, int L, int Hq, int Hkv, int hd, int max_ctx,
+                                int causal, void* d_scratch, size_t scratch_bytes, void* stream) {
+  dlm_ctx* ctx = nullptr;
+  if (!d_q || !d_k_codes || !d_v_codes || !d_k_scales || !d_v_scales || !d_o || !d_scratch || T < 1 || L < 0 ||
+      Hq < 1 || Hkv < 1 || Hq % Hkv || !(hd == 32 || hd == 64 || hd == 128) || L + T > max_ctx || max_ctx % 4)
+    return DLM_EINVAL;
+  if (scratch_bytes < dlm_attention_scratch_size(T, Hq, hd, max_ctx)) return DLM_ENOMEM_WS;
+  CU((cudaError_t)attention_init_attributes());
+  uint8_t* sc = (uint8_t*)d_scratch;
+  AttnArgs a{};
+  a.q = (const __nv_bfloat16*)d_q;
+  a.kc = (const __nv_bfloat16*)d_k_codes;
+  a.vc = (const __nv_bfloat16*)d_v_codes;
+  a.ks = d_k_scales;
+  a.vs = d_v_scales;
+  a.o = (__nv_bfloat16*)d_o;
+  a.T = T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.hd = hd;
+  a.max_ctx = max_ctx;
+  a.pos0 = L;
+  a.causal = causal ? 1 : 0;
+  a.max_splits = attention_max_splits(T, Hq, Hkv, max_ctx);
+  a.part_o = (float*)(sc + op_header());
+  a.part_ml = a.part_o + (size_t)a.max_splits * T * Hq * hd;
+  CU(attention_launch(a, (cudaStream_t)stream));
   return DLM_OK;
 }
 

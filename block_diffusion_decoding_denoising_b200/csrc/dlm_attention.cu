@@ -24,11 +24,24 @@ constexpr int kAttnRows = 64;   // query rows per CTA
 constexpr int kAttnKeys = 64;   // keys per tile
 constexpr int kMinKeysPerSplit = 128;
 
-template <int HD>
+template <int HD, bool FP8 = false>
 struct AttnSmem {
   static constexpr int kTileBytes = 64 * HD * 2;
-  static constexpr int kBytes = kTileBytes /*Q*/ + 4 * kTileBytes /*K,V double-buffered*/;
+  // bf16 cache: Q + K, V double-buffered.  FP8 cache: Q + one bf16 K, V tile + the raw e4m3
+  // K, V tiles and their 64 + 64 row scales double-buffered
+  static constexpr int kRawBytes = 2 * 64 * HD + 2 * 64 * 4;
+  static constexpr int kBytes = FP8 ? kTileBytes + 2 * kTileBytes + 2 * kRawBytes : kTileBytes + 4 * kTileBytes;
 };
+
+// Two e4m3 codes (low byte first) -> their values as a bf16 pair, exactly (e4m3 values are
+// f16 values, and at most 4 significant bits fit bf16).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(two));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
 
 // 16-byte chunk swizzle inside a [64][HD] bf16 tile (row stride HD*2 bytes) that keeps
 // ldmatrix reads of 8 consecutive rows free of bank conflicts.
@@ -79,7 +92,7 @@ __host__ __device__ __forceinline__ int attn_splits(int nkeys, int max_splits) {
   return s;
 }
 
-template <int HD>
+template <int HD, bool FP8>
 __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
   pdl_trigger();
   pdl_wait();
@@ -109,8 +122,12 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int gid = lane / 4, tig = lane % 4;
   const uint32_t sQ = smem_u32(sm);
-  const uint32_t sK[2] = {sQ + AttnSmem<HD>::kTileBytes, sQ + 3 * AttnSmem<HD>::kTileBytes};
-  const uint32_t sV[2] = {sQ + 2 * AttnSmem<HD>::kTileBytes, sQ + 4 * AttnSmem<HD>::kTileBytes};
+  constexpr int TB = AttnSmem<HD>::kTileBytes;
+  // FP8: one bf16 K and V tile (index 0) converted from raw[buf] each step
+  const uint32_t sK[2] = {sQ + TB, sQ + (FP8 ? TB : 3 * TB)};
+  const uint32_t sV[2] = {sQ + 2 * TB, sQ + (FP8 ? 2 * TB : 4 * TB)};
+  uint8_t* const raw0 = sm + 3 * TB;  // FP8: [buf][K codes 64 x HD | V codes | K scales 64 | V scales 64]
+  constexpr int RB = AttnSmem<HD, true>::kRawBytes;
   constexpr int CH = HD / 8;  // 16-byte chunks per row
 
   // ---- Q tile: row r <-> (token t = r / G, head g*G + r % G)
@@ -127,15 +144,66 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
   const __nv_bfloat16* kbase = a.kc + (size_t)g * a.max_ctx * HD;
   const __nv_bfloat16* vbase = a.vc + (size_t)g * a.max_ctx * HD;
   auto load_kv = [&](int buf, int kt0) {
-    for (int i = threadIdx.x; i < kAttnKeys * CH; i += 128) {
-      int r = i / CH, ch = i % CH;
-      int key = kt0 + r;
-      bool v = key < k1;
-      size_t off = (size_t)(v ? key : 0) * HD + ch * 8;
-      cp_async16(sK[buf] + r * (HD * 2) + swz<HD>(r, ch) * 16, kbase + off, v);
-      cp_async16(sV[buf] + r * (HD * 2) + swz<HD>(r, ch) * 16, vbase + off, v);
+    if constexpr (FP8) {
+      // raw e4m3 rows (HD bytes per key) and the 64 K / V row scales of the tile
+      const uint8_t* kb8 = reinterpret_cast<const uint8_t*>(a.kc) + (size_t)g * a.max_ctx * HD;
+      const uint8_t* vb8 = reinterpret_cast<const uint8_t*>(a.vc) + (size_t)g * a.max_ctx * HD;
+      const uint32_t rb = smem_u32(raw0 + buf * RB);
+      constexpr int C8 = HD / 16;  // 16-byte chunks per key
+      for (int i = threadIdx.x; i < kAttnKeys * C8; i += 128) {
+        const int r = i / C8, ch = i % C8;
+        const int key = kt0 + r;
+        const bool v = key < k1;
+        const size_t off = (size_t)(v ? key : 0) * HD + ch * 16;
+        cp_async16(rb + r * HD + ch * 16, kb8 + off, v);
+        cp_async16(rb + kAttnKeys * HD + r * HD + ch * 16, vb8 + off, v);
+      }
+      if (threadIdx.x < 32) {  // 16 chunks of 4 scales each for K, then for V
+        const int which = threadIdx.x / 16, ch = threadIdx.x % 16;
+        const float* sc = (which ? a.vs : a.ks) + (size_t)g * a.max_ctx + kt0 + ch * 4;
+        const bool v = kt0 + ch * 4 + 3 < k1;
+        if (v) {
+          cp_async16(rb + 2 * kAttnKeys * HD + which * 256 + ch * 16, sc, true);
+        } else {
+          // the tile's last keys: element-wise (zero past k1), no 16-byte read past the row
+          float* d = reinterpret_cast<float*>(raw0 + buf * RB + 2 * kAttnKeys * HD + which * 256) + ch * 4;
+          for (int u = 0; u < 4; ++u) d[u] = (kt0 + ch * 4 + u < k1) ? sc[u] : 0.f;
+        }
+      }
+    } else {
+      for (int i = threadIdx.x; i < kAttnKeys * CH; i += 128) {
+        int r = i / CH, ch = i % CH;
+        int key = kt0 + r;
+        bool v = key < k1;
+        size_t off = (size_t)(v ? key : 0) * HD + ch * 8;
+        cp_async16(sK[buf] + r * (HD * 2) + swz<HD>(r, ch) * 16, kbase + off, v);
+        cp_async16(sV[buf] + r * (HD * 2) + swz<HD>(r, ch) * 16, vbase + off, v);
+      }
     }
     cp_commit();
+  };
+  // FP8: raw[buf] -> the bf16 K and V tiles, exactly (16 codes -> two 16-byte chunks)
+  auto convert = [&](int buf) {
+    const uint8_t* rk = raw0 + buf * RB;
+    constexpr int C8 = HD / 16;
+    for (int i = threadIdx.x; i < 2 * kAttnKeys * C8; i += 128) {
+      const int which = i / (kAttnKeys * C8), j = i % (kAttnKeys * C8);
+      const int r = j / C8, ch = j % C8;
+      const uint4 src = *reinterpret_cast<const uint4*>(rk + which * kAttnKeys * HD + r * HD + ch * 16);
+      const uint32_t w[4] = {src.x, src.y, src.z, src.w};
+      uint32_t o[8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        o[2 * u] = e4m3x2_to_bf16x2((uint16_t)(w[u] & 0xFFFFu));
+        o[2 * u + 1] = e4m3x2_to_bf16x2((uint16_t)(w[u] >> 16));
+      }
+      const uint32_t base = which ? sV[0] : sK[0];
+      const int c0 = ch * 2;  // 8-element (16-byte) chunk index of the first 8 values
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + r * (HD * 2) + swz<HD>(r, c0) * 16),
+                   "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]) : "memory");
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + r * (HD * 2) + swz<HD>(r, c0 + 1) * 16),
+                   "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7]) : "memory");
+    }
   };
 
   const int ntiles = (k1 > k0) ? (k1 - k0 + kAttnKeys - 1) / kAttnKeys : 0;
@@ -166,13 +234,26 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
   for (int it = 0; it < ntiles; ++it) {
     const int buf = it & 1;
     const int kt0 = k0 + it * kAttnKeys;
-    if (it + 1 < ntiles) {
-      load_kv(buf ^ 1, kt0 + kAttnKeys);
-      cp_wait<1>();
+    const float* ksc = nullptr;
+    const float* vsc = nullptr;
+    if constexpr (FP8) {
+      cp_wait<0>();     // raw[buf] (the one group in flight) has landed for this thread
+      __syncthreads();  // ... for every thread; and tile it - 1 is done with the bf16 tiles
+      if (it + 1 < ntiles) load_kv(buf ^ 1, kt0 + kAttnKeys);  // overlaps this tile's work
+      convert(buf);
+      __syncthreads();
+      ksc = reinterpret_cast<const float*>(raw0 + buf * RB + 2 * kAttnKeys * HD);
+      vsc = ksc + kAttnKeys;
     } else {
-      cp_wait<0>();
+      if (it + 1 < ntiles) {
+        load_kv(buf ^ 1, kt0 + kAttnKeys);
+        cp_wait<1>();
+      } else {
+        cp_wait<0>();
+      }
+      __syncthreads();
     }
-    __syncthreads();
+    const int kb = FP8 ? 0 : buf;  // bf16 tile of this step
 
     // S = Q K^T for 16 rows x 64 keys
     float s[8][4];
@@ -187,10 +268,21 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
         int key = nb2 * 16 + (m / 2) * 8 + (lane % 8);
         int col = ks * 16 + (m % 2) * 8;
         uint32_t b0, b1, b2, b3;
-        ldsm_x4(tile_addr<HD>(sK[buf], key, col), b0, b1, b2, b3);
+        ldsm_x4(tile_addr<HD>(sK[kb], key, col), b0, b1, b2, b3);
         mma16816(s[nb2 * 2], qf[ks], b0, b1);
         mma16816(s[nb2 * 2 + 1], qf[ks], b2, b3);
       }
+    }
+    // FP8: the K row scale of each key multiplies its scores
+    if constexpr (FP8) {
+#pragma unroll
+      for (int nb = 0; nb < 8; ++nb)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float sk = ksc[nb * 8 + tig * 2 + j];
+          s[nb][j] *= sk;
+          s[nb][2 + j] *= sk;
+        }
     }
     // mask, running max
     float mx_A = -INFINITY, mx_B = -INFINITY;
@@ -229,6 +321,18 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
     }
     l_A = l_A * al_A + rs_A;
     l_B = l_B * al_B + rs_B;
+    // FP8: the V row scale of each key multiplies its weight in O = P V (the sums above stay
+    // the softmax normaliser)
+    if constexpr (FP8) {
+#pragma unroll
+      for (int nb = 0; nb < 8; ++nb)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float sv = vsc[nb * 8 + tig * 2 + j];
+          s[nb][j] *= sv;
+          s[nb][2 + j] *= sv;
+        }
+    }
 #pragma unroll
     for (int i = 0; i < HD / 8; ++i) {
       acc[i][0] *= al_A;
@@ -255,7 +359,7 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
         int key = ks * 16 + (m % 2) * 8 + (lane % 8);
         int col = nb2 * 16 + (m / 2) * 8;
         uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(tile_addr<HD>(sV[buf], key, col), b0, b1, b2, b3);
+        ldsm_x4_t(tile_addr<HD>(sV[kb], key, col), b0, b1, b2, b3);
         mma16816(acc[nb2 * 2], pa, b0, b1);
         mma16816(acc[nb2 * 2 + 1], pa, b2, b3);
         mma16816(acc[nb2 * 2], pl, b0, b1);
@@ -375,23 +479,30 @@ size_t attention_scratch_bytes(int T, int Hq, int hd, int max_splits) {
   return (size_t)max_splits * rows * (hd + 2) * sizeof(float);
 }
 
+template <int HD, bool FP8>
+static cudaError_t attn_attr() {
+  cudaError_t e = cudaFuncSetAttribute(k_bd_attention<HD, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       AttnSmem<HD, FP8>::kBytes);
+  // the largest shared-memory carve-out, as the GEMMs (see ops_init_attributes)
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_bd_attention<HD, FP8>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+  return e;
+}
+
 int attention_init_attributes() {
   static PerDeviceOnce once;
   return once_on_current_device(once, [] {
-  cudaError_t e = cudaFuncSetAttribute(k_bd_attention<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       AttnSmem<32>::kBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_bd_attention<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem<64>::kBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_bd_attention<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             AttnSmem<128>::kBytes);
-  // the largest shared-memory carve-out, as the GEMMs (see ops_init_attributes)
-  const void* ks[] = {(const void*)k_bd_attention<32>, (const void*)k_bd_attention<64>,
-                      (const void*)k_bd_attention<128>, (const void*)k_attn_combine};
-  for (const void* k : ks)
+    cudaError_t e = attn_attr<32, false>();
+    if (e == cudaSuccess) e = attn_attr<64, false>();
+    if (e == cudaSuccess) e = attn_attr<128, false>();
+    if (e == cudaSuccess) e = attn_attr<32, true>();
+    if (e == cudaSuccess) e = attn_attr<64, true>();
+    if (e == cudaSuccess) e = attn_attr<128, true>();
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
-  return (int)e;
+      e = cudaFuncSetAttribute(k_attn_combine, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    return (int)e;
   });
 }
 
@@ -404,7 +515,8 @@ template <int HD>
 static cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   const int G = a.Hq / a.Hkv;
   dim3 grid((a.T * G + kAttnRows - 1) / kAttnRows, a.Hkv, a.max_splits);
-  cudaError_t e = launch_k(k_bd_attention<HD>, grid, dim3(128), AttnSmem<HD>::kBytes, s, a);
+  cudaError_t e = a.ks ? launch_k(k_bd_attention<HD, true>, grid, dim3(128), AttnSmem<HD, true>::kBytes, s, a)
+                       : launch_k(k_bd_attention<HD, false>, grid, dim3(128), AttnSmem<HD, false>::kBytes, s, a);
   if (e != cudaSuccess) return e;
   if (a.max_splits > 1) e = launch_k(k_attn_combine, dim3(a.Hkv * a.T * G), dim3(128), 0, s, a);
   return e;

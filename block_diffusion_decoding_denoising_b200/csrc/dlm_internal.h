@@ -110,7 +110,9 @@ struct EpiArgs {
   int* tile_cnt;                // [n_tiles] arrival counters, zero between GEMMs
   float* out;                   // EPI_STORE
   int ld;
-  __nv_bfloat16 *q, *kc, *vc;   // EPI_QKV
+  __nv_bfloat16 *q, *kc, *vc;   // EPI_QKV (bf16 K/V cache)
+  uint8_t *kc8, *vc8;           // EPI_QKV with an FP8 KV cache: e4m3 rows ...
+  float *ks, *vs;               // ... and their scales [Hkv][max_ctx]
   int Hq, Hkv, hd, max_ctx;
   int pos0;
   const int* pos0_dev;
@@ -190,8 +192,10 @@ cudaError_t lmhead_fused_launch(const void* x2, int x2_rows, int hi_row, int lo_
 // attention (dlm_attention.cu)
 struct AttnArgs {
   const __nv_bfloat16* q;    // [T][Hq][hd]
-  const __nv_bfloat16* kc;   // [Hkv][max_ctx][hd] (one layer)
+  const __nv_bfloat16* kc;   // [Hkv][max_ctx][hd] (one layer; e4m3 bytes when ks != nullptr)
   const __nv_bfloat16* vc;
+  const float* ks;           // FP8 KV cache: K / V row scales [Hkv][max_ctx], else nullptr
+  const float* vs;
   __nv_bfloat16* o;          // [T][Hq][hd] (high halves when o_lo != 0)
   long o_lo;                 // elements to the low halves of a split output, 0 = plain bf16
   float* part_o;             // [max_splits][Hkv * T * G][hd]

@@ -71,45 +71,102 @@ __device__ __forceinline__ void finish_load_pair(const GemmOut& o, int tile, int
 }
 
 // QKV: RoPE (NeoX pairs j, j + hd/2, angles from the fp64-built table) on q and k heads;
-// q as bf16 [T][Hq][hd], K and V rows into the cache at positions L + t.
+// q as bf16 [T][Hq][hd], K and V rows into the cache at positions L + t: bf16, or for an FP8
+// cache e4m3 codes with one fp32 scale amax / 448 per (KV head, position) row.  A thread owns
+// the pair (jj, jj + hd/2) of one head for 8 tokens; the pairs of one head row are held by
+// min(32, hd/2) consecutive lanes, and by two warps for hd = 128 (their maxima meet in shared
+// memory).
 __global__ void __launch_bounds__(256) k_finish_qkv(FinishArgs a) {
   pdl_trigger();
   pdl_wait();
+  __shared__ float amax2[4][kFinTok][2];  // [token group][token][warp of the pair] (hd = 128)
   const EpiArgs& e = a.epi;
+  const bool fp8 = e.kc8 != nullptr;
   const int tile = blockIdx.x, p = threadIdx.x % 64, tg = threadIdx.x / 64;
   const int t0 = blockIdx.y * 32 + tg * kFinTok;
   const int half = e.hd / 2;
   const int ra = (p / half) * e.hd + p % half, rb = ra + half;  // rows of the pair in the tile
   const int n = tile * kTileM + ra;                              // feature of row ra
-  if (n >= a.N || t0 >= a.out.T) return;
+  const bool active = n < a.N && t0 < a.out.T;
+  if (!active && !fp8) return;  // (the FP8 path reduces across threads: no early exit)
   const int L = e.pos0_dev ? *e.pos0_dev + e.pos_off : e.pos0;
   float va[kFinTok], vb[kFinTok];
-  finish_load_pair(a.out, tile, ra, rb, t0, va, vb);
+  if (active) {
+    finish_load_pair(a.out, tile, ra, rb, t0, va, vb);
+  } else {
+#pragma unroll
+    for (int j = 0; j < kFinTok; ++j) va[j] = vb[j] = 0.f;
+  }
   const int hh = n / e.hd, jj = n % e.hd;  // jj < half
   const bool rope = hh < e.Hq + e.Hkv;
-  float2 cs[kFinTok];
-#pragma unroll
-  for (int j = 0; j < kFinTok; ++j)
-    cs[j] = (rope && t0 + j < a.out.T) ? e.rope_tab[(size_t)(L + t0 + j) * half + jj] : make_float2(1.f, 0.f);
-  __nv_bfloat16* dst;
-  size_t stride_t;
-  if (hh < e.Hq) {
-    dst = e.q + (size_t)t0 * e.Hq * e.hd + (size_t)hh * e.hd + jj;
-    stride_t = (size_t)e.Hq * e.hd;
-  } else if (hh < e.Hq + e.Hkv) {
-    dst = e.kc + ((size_t)(hh - e.Hq) * e.max_ctx + L + t0) * e.hd + jj;
-    stride_t = e.hd;
-  } else {
-    dst = e.vc + ((size_t)(hh - e.Hq - e.Hkv) * e.max_ctx + L + t0) * e.hd + jj;
-    stride_t = e.hd;
-  }
+  float x0[kFinTok], x1[kFinTok];
 #pragma unroll
   for (int j = 0; j < kFinTok; ++j) {
-    if (t0 + j < a.out.T) {
-      const float x0 = va[j], x1 = vb[j];
-      dst[(size_t)j * stride_t] = f2bf(x0 * cs[j].x - x1 * cs[j].y);
-      dst[(size_t)j * stride_t + half] = f2bf(x0 * cs[j].y + x1 * cs[j].x);
+    const bool in = active && t0 + j < a.out.T;
+    const float2 cs = (rope && in) ? e.rope_tab[(size_t)(L + t0 + j) * half + jj] : make_float2(1.f, 0.f);
+    x0[j] = va[j] * cs.x - vb[j] * cs.y;
+    x1[j] = va[j] * cs.y + vb[j] * cs.x;
+  }
+  if (active && hh < e.Hq) {
+    __nv_bfloat16* dst = e.q + (size_t)t0 * e.Hq * e.hd + (size_t)hh * e.hd + jj;
+    const size_t stride_t = (size_t)e.Hq * e.hd;
+#pragma unroll
+    for (int j = 0; j < kFinTok; ++j) {
+      if (t0 + j < a.out.T) {
+        dst[(size_t)j * stride_t] = f2bf(x0[j]);
+        dst[(size_t)j * stride_t + half] = f2bf(x1[j]);
+      }
     }
+  }
+  const bool is_k = hh >= e.Hq && hh < e.Hq + e.Hkv;
+  const int kvh = is_k ? hh - e.Hq : hh - e.Hq - e.Hkv;  // KV head of a K or V row
+  if (!fp8) {
+    if (!active || hh < e.Hq) return;
+    __nv_bfloat16* dst = (is_k ? e.kc : e.vc) + ((size_t)kvh * e.max_ctx + L + t0) * e.hd + jj;
+#pragma unroll
+    for (int j = 0; j < kFinTok; ++j) {
+      if (t0 + j < a.out.T) {
+        dst[(size_t)j * e.hd] = f2bf(x0[j]);
+        dst[(size_t)j * e.hd + half] = f2bf(x1[j]);
+      }
+    }
+    return;
+  }
+  // FP8: row amax over the head's pairs (every thread takes part; inactive ones carry 0)
+  const int lane = threadIdx.x % 32;
+  const int group = half < 32 ? half : 32;  // lanes of one head row within a warp
+  float am[kFinTok];
+#pragma unroll
+  for (int j = 0; j < kFinTok; ++j) {
+    float v = fmaxf(fabsf(x0[j]), fabsf(x1[j]));
+    for (int o = group / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    am[j] = v;
+  }
+  if (half == 64) {  // the row spans the two warps of this token group
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < kFinTok; ++j) amax2[tg][j][(threadIdx.x / 32) % 2] = am[j];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kFinTok; ++j) am[j] = fmaxf(amax2[tg][j][0], amax2[tg][j][1]);
+  }
+  if (!active || hh < e.Hq) return;
+  uint8_t* dst = (is_k ? e.kc8 : e.vc8) + ((size_t)kvh * e.max_ctx + L + t0) * e.hd + jj;
+  float* sdst = (is_k ? e.ks : e.vs) + (size_t)kvh * e.max_ctx + L + t0;
+#pragma unroll
+  for (int j = 0; j < kFinTok; ++j) {
+    if (t0 + j >= a.out.T) continue;
+    const float sc = am[j] / 448.0f;
+    uint8_t c0 = 0, c1 = 0;
+    if (sc > 0.f) {
+      const float r0 = x0[j] / sc, r1 = x1[j] / sc;
+      c0 = (uint8_t)(e4m3_rne_bits(fabsf(r0)) | (r0 < 0.f ? 0x80 : 0));
+      c1 = (uint8_t)(e4m3_rne_bits(fabsf(r1)) | (r1 < 0.f ? 0x80 : 0));
+    }
+    dst[(size_t)j * e.hd] = c0;
+    dst[(size_t)j * e.hd + half] = c1;
+    if (jj == 0) sdst[j] = sc;
   }
 }
 

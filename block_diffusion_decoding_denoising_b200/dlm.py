@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(HERE, "libdlm.so")
 DLM_OK, DLM_EINVAL, DLM_ENOMEM_WS, DLM_EKVCAP, DLM_ECUDA, DLM_EROUNDCAP, DLM_ETIMEOUT, DLM_EUNSUPPORTED = range(8)
 COMMIT_THRESHOLD, COMMIT_TOPK = 0, 1
 FILL_EAGER, FILL_DEFERRED = 0, 1
+KV_BF16, KV_FP8 = 0, 1
 WEIGHTS_BF16, WEIGHTS_NVFP4 = 0, 1
 STATUS_NAMES = {0: "DLM_OK", 1: "DLM_EINVAL", 2: "DLM_ENOMEM_WS", 3: "DLM_EKVCAP", 4: "DLM_ECUDA",
                 5: "DLM_EROUNDCAP", 6: "DLM_ETIMEOUT", 7: "DLM_EUNSUPPORTED"}
@@ -30,13 +31,13 @@ class Config(C.Structure):
     _fields_ = [("n_layers", C.c_int), ("d", C.c_int), ("n_q_heads", C.c_int), ("n_kv_heads", C.c_int),
                 ("head_dim", C.c_int), ("ffn", C.c_int), ("vocab", C.c_int), ("mask_id", C.c_int),
                 ("max_ctx", C.c_int), ("block_size", C.c_int), ("rope_theta", C.c_float),
-                ("rms_eps", C.c_float), ("weight_fmt", C.c_int)]
+                ("rms_eps", C.c_float), ("weight_fmt", C.c_int), ("kv_fmt", C.c_int)]
 
     @classmethod
     def from_dict(cls, c):
         return cls(c["n_layers"], c["d"], c["n_q_heads"], c["n_kv_heads"], c["head_dim"], c["ffn"],
                    c["vocab"], c["mask_id"], c["max_ctx"], c["block_size"], float(c["rope_theta"]),
-                   float(c["rms_eps"]), int(c.get("weight_fmt", 0)))
+                   float(c["rms_eps"]), int(c.get("weight_fmt", 0)), int(c.get("kv_fmt", 0)))
 
 
 class Nvfp4Matrix(C.Structure):
@@ -119,6 +120,7 @@ def lib():
         L.dlm_attention_scratch_size.argtypes = [i, i, i, i]
         L.dlm_bd_attention.argtypes = [p, p, p, p, i, i, i, i, i, i, i, p, z, p]
         L.dlm_bd_attention_noalloc.argtypes = [p, p, p, p, i, i, i, i, i, i, i, p]
+        L.dlm_bd_attention_fp8.argtypes = [p, p, p, p, p, p, i, i, i, i, i, i, i, p, z, p]
         L.dlm_commit.argtypes = [p, p, p, p, p, p, p, i, i, f, i, i, p]
         L.dlm_nvfp4_quantize.argtypes = [p, i, i, p, p, p, p]
         L.dlm_gemm_nvfp4_scratch_size.restype = z
@@ -239,6 +241,20 @@ def bd_attention(q, k_cache, v_cache, L, causal=False, stream=None):
     return o
 
 
+def bd_attention_fp8(q, k_codes, k_scales, v_codes, v_scales, L, causal=False, stream=None):
+    """Attention on an FP8 KV cache: codes uint8 [Hkv][max_ctx][hd] (e4m3), scales fp32
+    [Hkv][max_ctx] -> o bf16 [T][Hq][hd]."""
+    import torch
+    T, Hq, hd = q.shape
+    Hkv, max_ctx, _ = k_codes.shape
+    o = torch.empty_like(q)
+    n = lib().dlm_attention_scratch_size(T, Hq, hd, max_ctx)
+    sc = _scratch(n, q.device)
+    _check(lib().dlm_bd_attention_fp8(_ptr(q), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales), _ptr(o),
+                                      T, int(L), Hq, Hkv, hd, max_ctx, int(causal), _ptr(sc), n, _stream(stream)))
+    return o
+
+
 def bd_attention_noalloc(q, k_cache, v_cache, L, causal=False, o=None, stream=None):
     """bd_attention through the entry point that takes no scratch (library-owned static
     device memory; see dlm_bd_attention_noalloc).  `o` may be given to reuse an output."""
@@ -338,7 +354,7 @@ class Model:
         if ws == 0:
             raise DlmError(DLM_EINVAL, "invalid config")
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=self.device)
-        self.kv = torch.zeros(max(kv, 256) // 2, dtype=torch.bfloat16, device=self.device)
+        self.kv = torch.zeros(max(kv, 256), dtype=torch.uint8, device=self.device)
         ctx = C.c_void_p()
         _check(L.dlm_ctx_create(C.byref(self.cfg), C.byref(self._w), _ptr(self.workspace), ws, _ptr(self.kv),
                                 kv, C.byref(ctx)))
@@ -357,9 +373,25 @@ class Model:
 
     # KV cache views: [layer][K|V][kv_head][max_ctx][head_dim]
     def kv_view(self):
+        """bf16 cache values (DLM_KV_BF16 contexts)."""
         c = self.cfg_d
-        return self.kv[: 2 * c["n_layers"] * c["n_kv_heads"] * c["max_ctx"] * c["head_dim"]].view(
-            c["n_layers"], 2, c["n_kv_heads"], c["max_ctx"], c["head_dim"])
+        assert int(c.get("kv_fmt", 0)) == KV_BF16
+        import torch
+        n = 2 * c["n_layers"] * c["n_kv_heads"] * c["max_ctx"] * c["head_dim"]
+        return self.kv[: 2 * n].view(torch.bfloat16).view(c["n_layers"], 2, c["n_kv_heads"], c["max_ctx"],
+                                                          c["head_dim"])
+
+    def kv_view_fp8(self):
+        """(codes uint8 [layer][K|V][kv_head][max_ctx][head_dim], scales fp32
+        [layer][K|V][kv_head][max_ctx]) of a DLM_KV_FP8 context."""
+        import torch
+        c = self.cfg_d
+        assert int(c.get("kv_fmt", 0)) == KV_FP8
+        rows = 2 * c["n_layers"] * c["n_kv_heads"] * c["max_ctx"]
+        codes = self.kv[: rows * c["head_dim"]].view(c["n_layers"], 2, c["n_kv_heads"], c["max_ctx"], c["head_dim"])
+        scales = self.kv[rows * c["head_dim"]: rows * c["head_dim"] + 4 * rows].view(torch.float32).view(
+            c["n_layers"], 2, c["n_kv_heads"], c["max_ctx"])
+        return codes, scales
 
     @property
     def prefix_len(self):

@@ -60,6 +60,9 @@ typedef int dlm_status;
 #define DLM_FILL_EAGER 0    /* a block's KV-fill forward runs as soon as the block commits */
 #define DLM_FILL_DEFERRED 1 /* it is carried by the next round (default; see dlm_kv_fill) */
 
+#define DLM_KV_BF16 0 /* K/V cache rows in bf16 */
+#define DLM_KV_FP8 1  /* e4m3 K/V rows, one fp32 scale amax / 448 per row (see dlm_kv_cache_size) */
+
 #define DLM_WEIGHTS_BF16 0
 #define DLM_WEIGHTS_NVFP4 1 /* MLP and LM head in NVFP4, attention projections bf16 */
 
@@ -77,6 +80,7 @@ typedef struct dlm_config {
   float rope_theta;/* RoPE base (NeoX rotate-half pairing (j, j + hd/2)) */
   float rms_eps;   /* RMSNorm epsilon */
   int weight_fmt;  /* DLM_WEIGHTS_BF16 or DLM_WEIGHTS_NVFP4 */
+  int kv_fmt;      /* DLM_KV_BF16 or DLM_KV_FP8 */
 } dlm_config;
 
 /* One NVFP4 matrix [rows][cols]: e2m1 codes (2 per byte, element 2j in the low nibble),
@@ -140,7 +144,11 @@ typedef struct dlm_ctx dlm_ctx;
 /* ---------------------------------------------------------------- context */
 /* Bytes of device workspace a context needs (256-byte aligned base). */
 size_t dlm_workspace_size(const dlm_config* cfg);
-/* Bytes of the bf16 KV cache: 2 * n_layers * n_kv_heads * max_ctx * head_dim * 2. */
+/* Bytes of the KV cache.  DLM_KV_BF16: values bf16 [layer][K|V][kv_head][max_ctx][head_dim].
+ * DLM_KV_FP8 ("ORL: diffusion LLMs get a learnable 'tokens per forward'", "What shipped",
+ * "dlmrt, the inference engine": the KV cache is FP8): values e4m3 bytes in the same layout,
+ * followed by fp32 scales [layer][K|V][kv_head][max_ctx], one per row of head_dim values:
+ * scale = amax(|row|) / 448, value = e4m3(code) * scale (K after RoPE). */
 size_t dlm_kv_cache_size(const dlm_config* cfg);
 /* Validates cfg, copies the weight pointer table, carves the workspace.  The KV cache
  * layout is [layer][K|V][kv_head][max_ctx][head_dim] bf16.  Sets the prefix length L = 0. */
@@ -291,6 +299,15 @@ dlm_status dlm_bd_attention_noalloc(const void* d_q, const void* d_k_cache, cons
  * row, as in a round).  d_h_in, d_h_out fp32 [T][d]; T <= 32 (NVFP4) or <= 128.  Uses the
  * context's workspace: not concurrent with other calls on the context. */
 dlm_status dlm_mlp_block(dlm_ctx* ctx, int layer, const float* d_h_in, float* d_h_out, int T, void* stream);
+
+/* The same attention on an FP8 KV cache (see dlm_kv_cache_size): k_codes, v_codes uint8
+ * [Hkv][max_ctx][hd] e4m3; k_scales, v_scales fp32 [Hkv][max_ctx].  The e4m3 values enter
+ * the tensor cores exactly (as bf16); the K row scales multiply the scores and the V row
+ * scales the softmax weights.  Scratch as dlm_bd_attention. */
+dlm_status dlm_bd_attention_fp8(const void* d_q, const void* d_k_codes, const float* d_k_scales,
+                                const void* d_v_codes, const float* d_v_scales, void* d_o, int T, int L,
+                                int Hq, int Hkv, int hd, int max_ctx, int causal, void* d_scratch,
+                                size_t scratch_bytes, void* stream);
 
 /* Commit rule on device arrays (one block of B positions).  Updates tokens, committed,
  * zeroes the s rows of newly committed positions, increments *d_round. */

@@ -105,6 +105,58 @@ def test_attention_causal_prefill(lib, T, L):
     assert_close(got, ref, RTOL_BF16, "causal T=%d L=%d" % (T, L))
 
 
+# ------------------------------------------------------------------ attention on an FP8 KV cache
+def _fp8_attn_case(lib, B, L, Hq=32, Hkv=8, hd=128, causal=False, rows=None, seed=0):
+    """K and V quantized per row by the oracle's FP8 KV quantizer (reading R13); the GPU reads
+    the codes and scales, the oracle attends over the stored values."""
+    import torch
+    q, k, v = gen.attention_inputs_torch(B, L, Hq, Hkv, hd, seed=seed)
+    mc = k.shape[1]
+    mc4 = (mc + 3) // 4 * 4
+    kf = bf16_f64(from_torch_bf16(k))
+    vf = bf16_f64(from_torch_bf16(v))
+    kc, ks, kq = O.kv_quantize(kf.reshape(-1, hd))
+    vc, vs, vq = O.kv_quantize(vf.reshape(-1, hd))
+
+    def dev(codes, scales):
+        c = np.zeros((Hkv, mc4, hd), np.uint8)
+        sc = np.zeros((Hkv, mc4), np.float32)
+        c[:, :mc] = codes.reshape(Hkv, mc, hd)
+        sc[:, :mc] = scales.reshape(Hkv, mc)
+        return torch.from_numpy(c).cuda(), torch.from_numpy(sc).cuda()
+
+    kcd, ksd = dev(kc, ks)
+    vcd, vsd = dev(vc, vs)
+    o = lib.bd_attention_fp8(q, kcd, ksd, vcd, vsd, L, causal=causal)
+    torch.cuda.synchronize()
+    qf = bf16_f64(from_torch_bf16(q))
+    of = bf16_f64(from_torch_bf16(o))
+    kq, vq = kq.reshape(Hkv, mc, hd), vq.reshape(Hkv, mc, hd)
+    if rows is None:
+        return of, O.attention(qf, kq, vq, L, causal)
+    sel = np.array(rows)
+    return of[sel], O.attention(qf[sel], kq, vq, L + B - len(sel), False)
+
+
+@pytest.mark.parametrize("B,L", [(32, 1024), (64, 4096), (4, 2048), (1, 0), (16, 300)])
+def test_attention_fp8_kv(lib, B, L):
+    got, ref = _fp8_attn_case(lib, B, L)
+    assert_close(got, ref, RTOL_BF16, "fp8 attention B=%d L=%d" % (B, L))
+
+
+@pytest.mark.parametrize("B,L", [(32, 16384), (4, 65536)])
+def test_attention_fp8_kv_sampled_rows(lib, B, L):
+    rows = sorted({0, B // 2, B - 1})
+    got, ref = _fp8_attn_case(lib, B, L, rows=rows)
+    assert_close(got, ref, RTOL_BF16, "fp8 attention B=%d L=%d rows" % (B, L))
+
+
+@pytest.mark.parametrize("T,L,Hq,Hkv,hd", [(100, 37, 8, 2, 128), (24, 0, 4, 4, 64), (16, 20, 2, 1, 32)])
+def test_attention_fp8_kv_causal_and_head_dims(lib, T, L, Hq, Hkv, hd):
+    got, ref = _fp8_attn_case(lib, T, L, Hq=Hq, Hkv=Hkv, hd=hd, causal=True)
+    assert_close(got, ref, RTOL_BF16, "fp8 causal T=%d L=%d hd=%d" % (T, L, hd))
+
+
 # ------------------------------------------------------------------ LM head + row stats + P E
 def _check_stats(st, ref, what, logits=None):
     for k in ("m", "lse", "maxprob", "entropy"):

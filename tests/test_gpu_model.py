@@ -61,9 +61,11 @@ def torch_weights(w_np):
     return out
 
 
-def small_model(std=0.02, n_layers=1, d=64, Hq=2, Hkv=1, hd=32, F=256, V=512, B=8, seed=0, max_ctx=256, fmt=0):
+def small_model(std=0.02, n_layers=1, d=64, Hq=2, Hkv=1, hd=32, F=256, V=512, B=8, seed=0, max_ctx=256, fmt=0,
+                kv=0):
     cfg = dict(n_layers=n_layers, d=d, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=hd, ffn=F, vocab=V,
-               mask_id=V - 1, max_ctx=max_ctx, block_size=B, rope_theta=10000.0, rms_eps=1e-6, weight_fmt=fmt)
+               mask_id=V - 1, max_ctx=max_ctx, block_size=B, rope_theta=10000.0, rms_eps=1e-6, weight_fmt=fmt,
+               kv_fmt=kv)
     w = gen.model_weights_np(cfg, seed, std=std, embed_std=8.0 / np.sqrt(d))
     return cfg, w
 
@@ -77,6 +79,9 @@ MODELS = {
                                                fmt=1),
     # block of 32 as in the 4B-class configuration: a folded round carries 64 rows
     "gqa_b32": lambda: small_model(0.06, n_layers=2, d=256, Hq=4, Hkv=2, hd=64, F=512, V=1024, B=32, max_ctx=320),
+    # FP8 KV cache (reading R13)
+    "two_layer_gqa_fp8kv": lambda: small_model(0.06, n_layers=2, d=256, Hq=4, Hkv=2, hd=64, F=512, V=1024, B=16,
+                                               kv=1),
 }
 
 
@@ -116,11 +121,52 @@ def gpu_weights(D, cfg, w):
     return D.quantize_model(tw) if is_fp4(cfg) else tw
 
 
+def is_kv8(cfg):
+    return int(cfg.get("kv_fmt", 0)) == 1
+
+
 def inject_kv(m, orc, upto):
+    """The oracle's K/V rows [0, upto) into the GPU cache (FP8: its stored values re-quantized,
+    which gives back the same codes and scales: each row is a fixed point of the quantizer)."""
     import torch
-    kv = m.kv_view()
-    kv[:, 0, :, :upto] = torch.from_numpy(orc.kc[:, :, :upto]).to(torch.bfloat16).cuda()
-    kv[:, 1, :, :upto] = torch.from_numpy(orc.vc[:, :, :upto]).to(torch.bfloat16).cuda()
+    if not is_kv8(m.cfg_d):
+        kv = m.kv_view()
+        kv[:, 0, :, :upto] = torch.from_numpy(orc.kc[:, :, :upto]).to(torch.bfloat16).cuda()
+        kv[:, 1, :, :upto] = torch.from_numpy(orc.vc[:, :, :upto]).to(torch.bfloat16).cuda()
+        return
+    codes, scales = m.kv_view_fp8()
+    for j, src in enumerate((orc.kc, orc.vc)):
+        nl, hk, _, hd = src.shape
+        c, sc, _ = O.kv_quantize(src[:, :, :upto].reshape(-1, hd))
+        codes[:, j, :, :upto] = torch.from_numpy(c.reshape(nl, hk, upto, hd)).cuda()
+        scales[:, j, :, :upto] = torch.from_numpy(sc.reshape(nl, hk, upto)).cuda()
+
+
+def gpu_kv(m, rows):
+    """The GPU cache's K and V values of positions `rows` as float arrays [layer][head][row][hd]."""
+    if not is_kv8(m.cfg_d):
+        kv = m.kv_view()
+        return kv[:, 0, :, rows].float().cpu().numpy(), kv[:, 1, :, rows].float().cpu().numpy()
+    codes, scales = m.kv_view_fp8()
+    out = []
+    for j in (0, 1):
+        c = codes[:, j, :, rows].cpu().numpy()
+        sc = scales[:, j, :, rows].cpu().numpy().astype(np.float64)
+        mag = np.array([O.e4m3_value(b) for b in range(128)])[c & 0x7F]
+        out.append(np.where(c >= 128, -mag, mag) * sc[..., None])
+    return out[0], out[1]
+
+
+def assert_kv_close(got, ref, cfg, what):
+    """bf16 cache: the tolerance.  FP8 cache: each value within one e4m3 step of the oracle's
+    (a value near a rounding tie may take the neighbouring code) and at most 1 % of them off."""
+    if not is_kv8(cfg):
+        assert_close(got, ref, rtol(cfg), what)
+        return
+    step = np.abs(ref) * 2.0 ** -3 + np.abs(ref).max(axis=-1, keepdims=True) / 448.0 * 2.0 ** -9 + 1e-30
+    off = np.abs(got - ref) > 1e-6 * np.abs(ref) + 1e-30
+    assert np.all(np.abs(got - ref) <= step * 1.001), what + ": beyond one e4m3 step"
+    assert off.mean() <= 0.01, "%s: %.3f of the values off" % (what, off.mean())
 
 
 def set_state(st, tokens, committed, s, rnd):
@@ -256,7 +302,8 @@ def compare_round(st, ost, com, new, tau, mode, k, cfg, what):
 # so most of its min-1 / top-k rankings are inside the uncertainty.
 MIN_DECIDED = {("tiny", 0): 4, ("tiny", 1): 4, ("tiny_distinct", 0): 20, ("tiny_distinct", 1): 10,
                ("two_layer_gqa", 0): 26, ("two_layer_gqa", 1): 21, ("two_layer_gqa_nvfp4", 0): 0,
-               ("two_layer_gqa_nvfp4", 1): 0, ("gqa_b32", 0): 32, ("gqa_b32", 1): 36}
+               ("two_layer_gqa_nvfp4", 1): 0, ("gqa_b32", 0): 32, ("gqa_b32", 1): 36,
+               ("two_layer_gqa_fp8kv", 0): 32, ("two_layer_gqa_fp8kv", 1): 20}
 
 
 def lockstep(D, name, mode, tau, k, prompt_len=32, n_blocks=4):
@@ -279,15 +326,13 @@ def lockstep(D, name, mode, tau, k, prompt_len=32, n_blocks=4):
 
     def check_kv(rows, what):
         torch.cuda.synchronize()
-        kv = m.kv_view()
-        gk = kv[:, 0, :, rows].float().cpu().numpy()
-        gv = kv[:, 1, :, rows].float().cpu().numpy()
+        gk, gv = gpu_kv(m, rows)
         if is_fp4(cfg):  # layer 0 is upstream of every quantized GEMM input
             assert_close(gk[0], orc.kc[0, :, rows], rtol(cfg), what + " K layer 0")
             assert median_pos_err(gk[1:], orc.kc[1:, :, rows]) <= rtol(cfg), what + " K"
         else:
-            assert_close(gk, orc.kc[:, :, rows], rtol(cfg), what + " K")
-            assert_close(gv, orc.vc[:, :, rows], rtol(cfg), what + " V")
+            assert_kv_close(gk, orc.kc[:, :, rows], cfg, what + " K")
+            assert_kv_close(gv, orc.vc[:, :, rows], cfg, what + " V")
 
     for blk in range(n_blocks):
         pending = m.fill_pending
@@ -346,8 +391,7 @@ def test_prefill_kv_parity(dlm, name):
     m.prefill(torch.from_numpy(prompt).cuda())
     torch.cuda.synchronize()
     assert m.prefix_len == P
-    kv = m.kv_view()
-    gk, gv = kv[:, 0, :, :P].float().cpu().numpy(), kv[:, 1, :, :P].float().cpu().numpy()
+    gk, gv = gpu_kv(m, slice(0, P))
     if is_fp4(cfg):
         # layer 0 is upstream of every quantized GEMM input; later layers on the median
         # position (a position whose quantization decision flipped moves as a whole)
@@ -356,8 +400,8 @@ def test_prefill_kv_parity(dlm, name):
         assert median_pos_err(gk[1:], orc.kc[1:, :, :P]) <= rtol(cfg)
         assert median_pos_err(gv[1:], orc.vc[1:, :, :P]) <= rtol(cfg)
     else:
-        assert_close(gk, orc.kc[:, :, :P], rtol(cfg), "prefill K")
-        assert_close(gv, orc.vc[:, :, :P], rtol(cfg), "prefill V")
+        assert_kv_close(gk, orc.kc[:, :, :P], cfg, "prefill K")
+        assert_kv_close(gv, orc.vc[:, :, :P], cfg, "prefill V")
 
 
 @pytest.mark.parametrize("name", list(MODELS))
@@ -366,7 +410,7 @@ def test_round_lockstep(dlm, name, mode, tau, k):
     lockstep(dlm, name, mode, tau, k)
 
 
-@pytest.mark.parametrize("name", ["tiny_distinct", "two_layer_gqa", "two_layer_gqa_nvfp4"])
+@pytest.mark.parametrize("name", ["tiny_distinct", "two_layer_gqa", "two_layer_gqa_nvfp4", "two_layer_gqa_fp8kv"])
 def test_graph_decode_matches_eager_rounds(dlm, name):
     """The per-block CUDA graph (while node) and eager dlm_round calls run the same
     kernels on the same inputs: tokens, round counts and the KV cache must be identical,
@@ -403,7 +447,7 @@ def test_graph_decode_matches_eager_rounds(dlm, name):
     b.kv_flush()
     torch.cuda.synchronize()
     assert not a.fill_pending and not b.fill_pending
-    assert torch.equal(a.kv_view(), b.kv_view())
+    assert torch.equal(a.kv, b.kv)  # the cache bytes (values, and scales for FP8)
 
 
 @pytest.mark.parametrize("name", [n for n in MODELS if folds(MODELS[n]()[0])])
@@ -595,26 +639,62 @@ def test_round_4b_lockstep_sampled(dlm, fmt):
     assert_close(st["s"].cpu().numpy()[unc], new["s"][unc], rtol(cfg), "4b s")
 
 
-def _model_4b_with_prefix(dlm, L, n_layers=36, fmt=0, extra_ctx=64):
+def _model_4b_with_prefix(dlm, L, n_layers=36, fmt=0, extra_ctx=64, kv_fmt=0):
     """The 4B-class model (random weights on the device) with a seeded synthetic prefix K/V of
-    L rows, and the oracle bound to the same weights and prefix."""
+    L rows, and the oracle bound to the same weights and prefix.  FP8 cache: random e4m3 codes
+    (the two NaN codes excluded) with one scale per row."""
     import torch
     cfg = gen.config_4b(max_ctx=L + extra_ctx, n_layers=n_layers)
     cfg["weight_fmt"] = fmt
+    cfg["kv_fmt"] = kv_fmt
     tw = gen.model_weights_torch(cfg, seed=0, device="cuda")
     m = dlm.Model(cfg, dlm.quantize_model(tw) if fmt else tw)
-    kv = m.kv_view()
     g = torch.Generator(device="cuda")
     g.manual_seed(1234)
-    kv[:, :, :, :L] = torch.randn(kv[:, :, :, :L].shape, generator=g, device="cuda").to(torch.bfloat16)
-    m.set_prefix_len(L)
+    if kv_fmt:
+        codes, scales = m.kv_view_fp8()
+        c = torch.randint(0, 254, codes[:, :, :, :L].shape, generator=g, device="cuda", dtype=torch.int32)
+        c = torch.where(c >= 127, c + 1, c)  # skip 0x7F (and 0xFF: 254 + 1 = 255 never drawn)
+        codes[:, :, :, :L] = c.to(torch.uint8)
+        scales[:, :, :, :L] = 2.5 / 448.0 + 0.5 / 448.0 * torch.rand(scales[:, :, :, :L].shape, generator=g,
+                                                                     device="cuda")
+        m.set_prefix_len(L)
+        kh, vh = gpu_kv(m, slice(0, L))
+    else:
+        kv = m.kv_view()
+        kv[:, :, :, :L] = torch.randn(kv[:, :, :, :L].shape, generator=g, device="cuda").to(torch.bfloat16)
+        m.set_prefix_len(L)
+        kvh = kv[:, :, :, :L].float().cpu().numpy()
+        kh, vh = kvh[:, 0], kvh[:, 1]
     w_np = {k: from_torch_bf16(tw[k]) for k in ("embed", "w_adapter", "final_norm")}
     w_np["layers"] = [{k: from_torch_bf16(v) for k, v in l.items()} for l in tw["layers"]]
     orc = O.OracleModel(cfg, oracle_weights(cfg, w_np), act_round=True, max_ctx=L + extra_ctx)
-    kvh = kv[:, :, :, :L].float().cpu().numpy()
-    orc.kc[:, :, :L] = kvh[:, 0]
-    orc.vc[:, :, :L] = kvh[:, 1]
+    orc.kc[:, :, :L] = kh
+    orc.vc[:, :, :L] = vh
     return cfg, tw, w_np, m, orc
+
+
+def test_round_4b_fp8_kv_lockstep(dlm):
+    """One lock-step round of the 4B-class bf16 model on an FP8 KV cache at prefix length 512
+    (synthetic e4m3 prefix), then the K/V rows that round wrote for the block."""
+    import torch
+    L = 512
+    cfg, tw, w_np, m, orc = _model_4b_with_prefix(dlm, L, kv_fmt=1)
+    B, d = cfg["block_size"], cfg["d"]
+    st = m.new_block_state()
+    rng = np.random.default_rng(0)
+    com = (rng.random(B) < 0.25).astype(np.uint8)
+    tok = np.where(com == 1, rng.integers(0, cfg["vocab"] - 1, B), cfg["mask_id"]).astype(np.int32)
+    s = np.where(com[:, None] == 1, 0.0, rng.normal(0, 0.02, (B, d)))
+    set_state(st, tok, com, s.astype(np.float32), 1)
+    m.round(st, 0.9, 0, 1)
+    n, new, ost = orc.round(tok, com, s, 1, L, 0.9, 0, 1)
+    torch.cuda.synchronize()
+    compare_round(st, ost, com, new, 0.9, 0, 1, cfg, "4b fp8 kv")
+    gk, gv = gpu_kv(m, slice(L, L + B))
+    for layer in (0, cfg["n_layers"] - 1):
+        assert_kv_close(gk[layer], orc.kc[layer, :, L:L + B], cfg, "4b fp8 K layer %d" % layer)
+        assert_kv_close(gv[layer], orc.vc[layer, :, L:L + B], cfg, "4b fp8 V layer %d" % layer)
 
 
 def test_block_4b_fixed_tpf_lockstep_with_folded_fill(dlm):
