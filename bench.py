@@ -50,6 +50,9 @@ def parse(argv=None):
     # (same kernels; ncu cannot profile kernel nodes of graphs with conditional nodes)
     ap.add_argument("--eager", action="store_true")
     ap.add_argument("--pdl", type=int, default=1, help=argparse.SUPPRESS)
+    # the quick case on the NVFP4 model (MLP and E in NVFP4) or on an FP8 KV cache
+    ap.add_argument("--fmt", default="bf16", choices=["bf16", "nvfp4"])
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"])
     return ap.parse_args(argv)
 
 
@@ -698,7 +701,12 @@ def main():
     B = cfg["block_size"]
     blocks = GEN // B
     w = gen.model_weights_torch(cfg, seed=0, device=dev)
-    m = dlm.Model(cfg, w, device=dev)
+    if args.case == "quick" and (args.fmt != "bf16" or args.kv != "bf16"):
+        cq = dict(cfg, weight_fmt=dlm.WEIGHTS_NVFP4 if args.fmt == "nvfp4" else 0,
+                  kv_fmt=dlm.KV_FP8 if args.kv == "fp8" else 0)
+        m = dlm.Model(cq, dlm.quantize_model(w) if args.fmt == "nvfp4" else w, device=dev)
+    else:
+        m = dlm.Model(cfg, w, device=dev)
     prompt_np = gen.prompt_np(cfg, PROMPT, seed=rank)
     prompt = torch.from_numpy(prompt_np).to(dev)
     stream = torch.cuda.current_stream(dev)

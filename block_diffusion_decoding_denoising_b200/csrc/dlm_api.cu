@@ -90,6 +90,7 @@ struct dlm_ctx {
   uint8_t* xcodes = nullptr;   // [32][max(d, F) / 2] e2m1 codes of the GEMM input
   uint8_t* xscales = nullptr;  // e4m3 scales, tiled [max(d, F) / 64][32][16 B]
   float* sx = nullptr;
+  float* act_amax = nullptr;   // [F / 64][Tmax] partial maxima of the SiLU output (NVFP4)
   __nv_bfloat16* e_deq = nullptr;
   uint8_t* sf = nullptr;       // weight scales re-tiled for the FP4 MMA: per layer (gate/up, down), then E
   size_t sf_pair = 0, sf_down = 0;
@@ -223,6 +224,7 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   uint8_t* xcodes = fp4 ? cv.take<uint8_t>((size_t)kMaxF4Tokens * kmax / 2) : nullptr;
   uint8_t* xscales = fp4 ? cv.take<uint8_t>(kmax / 64 * 512) : nullptr;
   float* sx = fp4 ? cv.take<float>(kMaxF4Tokens) : nullptr;
+  float* aam = fp4 ? cv.take<float>((size_t)((c.ffn + 63) / 64) * Tmax) : nullptr;
   __nv_bfloat16* edq = fp4 ? cv.take<__nv_bfloat16>((size_t)c.vocab * c.d) : nullptr;
   const bool fp4_shapes = fp4 && c.d % 256 == 0 && c.ffn % 256 == 0;
   const size_t sfp = fp4_shapes ? align256(nvf4_sf_tile_bytes(c.ffn, c.d, A_PAIR)) : 0;
@@ -237,6 +239,7 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
     x->xcodes = xcodes;
     x->xscales = xscales;
     x->sx = sx;
+    x->act_amax = aam;
     x->sf = sf;
     x->sf_pair = sfp;
     x->sf_down = sfd;
@@ -443,9 +446,20 @@ dlm_status mlp_sub_block(Runner& r, int l, int T, GemmOut* y) {
   es.op = EPI_SILU;
   es.act = ctx->act;
   es.act_lo = pad * F;
+  es.act_amax = ctx->fp4 ? ctx->act_amax : nullptr;
   TRY(finish_tiles(r, *y, F, es));
   if (ctx->fp4) {
-    TRY(act_quant(r, T, ctx->act, pad * F, F));
+    ActQuantArgs q{};
+    q.xb = ctx->act;
+    q.xb_lo = pad * F;
+    q.K = F;
+    q.codes = ctx->xcodes;
+    q.scales = ctx->xscales;
+    q.sx = ctx->sx;
+    q.amax = ctx->act_amax;
+    q.n_amax = (F + 63) / 64;
+    q.T = T;
+    CU_LAUNCH(launch_k(k_act_quant_wide, dim3((unsigned)((F / 16 + 255) / 256), T), dim3(256), 0, r.s, q));
     return r.gemm_fp4(A_KMAJOR, W.q_down, nullptr, ctx->sf + l * (ctx->sf_pair + ctx->sf_down) + ctx->sf_pair, T, d,
                       F, y);
   }

@@ -125,6 +125,7 @@ struct EpiArgs {
   const int32_t* tokens;
   __nv_bfloat16* act;           // EPI_SILU: [T][F] high halves
   long act_lo;
+  float* act_amax;              // EPI_SILU (optional): [F / 64][T] amax of each tile's stored values
 };
 
 struct GemmPlan {

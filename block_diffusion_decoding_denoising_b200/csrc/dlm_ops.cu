@@ -171,20 +171,46 @@ __global__ void __launch_bounds__(256) k_finish_qkv(FinishArgs a) {
 }
 
 // gate/up pair tile (gate features in rows 0..63, up in 64..127): act = silu(g) u as a split
-// bf16 pair.
+// bf16 pair.  With act_amax set (the down projection is NVFP4) the tile also leaves, per
+// token, the largest magnitude of the values it stored (hi + lo), the partial maxima the
+// wide quantizer takes the row scale from.
 __global__ void __launch_bounds__(256) k_finish_silu(FinishArgs a) {
   pdl_trigger();
   pdl_wait();
+  __shared__ float am2[4][kFinTok][2];
   const EpiArgs& e = a.epi;
   const int tile = blockIdx.x, r = threadIdx.x % 64, tg = threadIdx.x / 64;
   const int t0 = blockIdx.y * 32 + tg * kFinTok;
   const int f = tile * 64 + r;
-  if (f >= a.N || t0 >= a.out.T) return;
-  float g[kFinTok], u[kFinTok];
-  finish_load_pair(a.out, tile, r, r + 64, t0, g, u);
+  const bool active = f < a.N && t0 < a.out.T;
+  if (!active && !e.act_amax) return;
+  float g[kFinTok], u[kFinTok], am[kFinTok];
+  if (active) finish_load_pair(a.out, tile, r, r + 64, t0, g, u);
 #pragma unroll
-  for (int j = 0; j < kFinTok; ++j)
-    if (t0 + j < a.out.T) store_split(e.act + (size_t)(t0 + j) * a.N + f, e.act_lo, g[j] / (1.0f + expf(-g[j])) * u[j]);
+  for (int j = 0; j < kFinTok; ++j) {
+    am[j] = 0.f;
+    if (active && t0 + j < a.out.T) {
+      const float v = g[j] / (1.0f + expf(-g[j])) * u[j];
+      __nv_bfloat16* p = e.act + (size_t)(t0 + j) * a.N + f;
+      store_split(p, e.act_lo, v);
+      if (e.act_amax) {
+        const __nv_bfloat16 h = f2bf(v);
+        am[j] = fabsf(bf2f(h) + bf2f(f2bf(v - bf2f(h))));  // the value the quantizer reads
+      }
+    }
+  }
+  if (!e.act_amax) return;
+  // tile maximum per token: 64 features = the two warps of this token group
+#pragma unroll
+  for (int j = 0; j < kFinTok; ++j) am[j] = warp_max(am[j]);
+  if (threadIdx.x % 32 == 0)
+#pragma unroll
+    for (int j = 0; j < kFinTok; ++j) am2[tg][j][(threadIdx.x / 32) % 2] = am[j];
+  __syncthreads();
+  if (threadIdx.x % 64 == 0)
+#pragma unroll
+    for (int j = 0; j < kFinTok; ++j)
+      if (t0 + j < a.out.T) e.act_amax[(size_t)tile * a.out.T + t0 + j] = fmaxf(am2[tg][j][0], am2[tg][j][1]);
 }
 
 // out[t][n] = scale * y (scale 0 means 1), rows r and r + 64 of the tile per thread.
@@ -668,6 +694,46 @@ __global__ void __launch_bounds__(256) k_act_quant(ActQuantArgs a) {
   }
 }
 
+// Wide NVFP4 quantizer of a split bf16 GEMM input: one thread per 16-element block, grid
+// (ceil(K / 16 / 256), T).  The row scale S = amax / (6 * 448) comes from the row's partial
+// maxima (a.amax[i][t], i < n_amax), reduced by every CTA in the same order.
+__global__ void __launch_bounds__(256) k_act_quant_wide(ActQuantArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float red[8];
+  const int t = blockIdx.y, nb = a.K / 16;
+  float m = 0.f;
+  for (int i = threadIdx.x; i < a.n_amax; i += 256) m = fmaxf(m, a.amax[(size_t)i * a.T + t]);
+  m = warp_max(m);
+  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = m;
+  __syncthreads();
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  const float S = amax / (6.0f * 448.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.sx[t] = S;
+  const int b = blockIdx.x * 256 + threadIdx.x;
+  if (b >= nb) return;
+  const size_t off = (size_t)t * a.K + (size_t)b * 16;
+  float v[16];
+  float bm = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    v[j] = bf2f(a.xb[off + j]) + bf2f(a.xb[off + j + a.xb_lo]);
+    bm = fmaxf(bm, fabsf(v[j]));
+  }
+  const uint8_t sb = (S > 0.f) ? e4m3_rne_bits(bm / (6.0f * S)) : 0;
+  const float denom = e4m3_value_dev(sb) * S;
+  uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t c = denom > 0.f ? e2m1_rne(v[j] / denom) : 0u;
+    packed[j / 8] |= c << (4 * (j % 8));
+  }
+  a.scales[((size_t)(b / 4) * 32 + t) * 16 + (b % 4)] = sb;
+  *reinterpret_cast<uint2*>(a.codes + (size_t)t * (a.K / 2) + (size_t)b * 8) = make_uint2(packed[0], packed[1]);
+}
+
 // NVFP4 matrix -> bf16 values q sigma (without the tensor scale; exact in bf16), one thread
 // per 16-element block.
 __global__ void k_nvfp4_dequant_bf16(const uint8_t* codes, const uint8_t* scales, long n_blocks,
@@ -696,6 +762,7 @@ int ops_init_attributes() {
   return once_on_current_device(once, [] {
   const void* ks[] = {(const void*)k_finish_qkv,  (const void*)k_finish_silu,   (const void*)k_finish_store,
                       (const void*)k_resid_norm,  (const void*)k_act_quant,     (const void*)k_to_bf16,
+                      (const void*)k_act_quant_wide,
                       (const void*)k_rowstats_part, (const void*)k_rowstats_final, (const void*)k_commit,
                       (const void*)k_block_init,  (const void*)k_block_finish};
   for (const void* k : ks) {

@@ -59,6 +59,11 @@ struct ActQuantArgs {
   uint8_t* codes;
   uint8_t* scales;
   float* sx;
+  // Wide form (k_act_quant_wide, split bf16 input): the row amax is the max of n_amax partial
+  // maxima amax[i][t] (one per 64-feature tile, written by the SiLU finisher); T rows.
+  const float* amax;
+  int n_amax;
+  int T;
 };
 
 int ops_init_attributes();
@@ -113,6 +118,7 @@ __global__ void k_block_init(BlockInitArgs a);
 __global__ void k_block_finish(BlockFinishArgs a);
 __global__ void k_set_int(int* p, int v);
 __global__ void k_act_quant(ActQuantArgs a);
+__global__ void k_act_quant_wide(ActQuantArgs a);
 __global__ void k_nvfp4_dequant_bf16(const uint8_t* codes, const uint8_t* scales, long n_blocks,
                                      __nv_bfloat16* out);
 __global__ void k_rope_table(float2* tab, int max_ctx, int hd, double base);
