@@ -1419,6 +1419,53 @@ dlm_status dlm_nvfp4_quantize(const void* d_w, int rows, int cols, void* d_codes
   return cudaGetLastError() == cudaSuccess ? DLM_OK : DLM_ECUDA;
 }
 
+size_t dlm_lmhead_nvfp4_scratch_size(int B, int V, int d) {
+  if (!lmhead_fused_f4_supported(B, d) || V < 2) return 0;
+  return op_header() + align256((size_t)kMaxF4Tokens * d / 2) + align256((size_t)d / 64 * 512) +
+         align256(kMaxF4Tokens * 4) + align256(nvf4_sf_tile_bytes(V, d, A_KMAJOR)) +
+         align256(lmhead_fused_scratch_bytes(V, d));
+}
+
+dlm_status dlm_lmhead_rowstats_nvfp4(const float* d_x, const dlm_nvfp4_matrix* E, int B, int V, int d, int mask_id,
+                                     dlm_row_stats stats, float* d_s, void* d_scratch, size_t scratch_bytes,
+                                     void* stream) {
+  dlm_ctx* ctx = nullptr;
+  if (!d_x || !E || !E->codes || !E->scales || !std::isfinite(E->tensor_scale) || !d_s || !d_scratch || B < 1 ||
+      V < 2 || d < 64 || !stats.m || !stats.lse || !stats.maxprob || !stats.entropy || !stats.argmax)
+    return DLM_EINVAL;
+  if (!lmhead_fused_f4_supported(B, d)) return DLM_EUNSUPPORTED;
+  if (scratch_bytes < dlm_lmhead_nvfp4_scratch_size(B, V, d)) return DLM_ENOMEM_WS;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* base = (uint8_t*)d_scratch;
+  size_t off = op_header();
+  auto take = [&](size_t bytes) {
+    uint8_t* q = base + off;
+    off += align256(bytes);
+    return q;
+  };
+  uint8_t* xcodes = take((size_t)kMaxF4Tokens * d / 2);
+  uint8_t* xscales = take((size_t)d / 64 * 512);
+  float* sx = (float*)take(kMaxF4Tokens * 4);
+  uint8_t* sfe = take(nvf4_sf_tile_bytes(V, d, A_KMAJOR));
+  void* lmf = take(lmhead_fused_scratch_bytes(V, d));
+  // the status word, and the token codes and scales of the rows past B (read by the MMA, their
+  // columns dropped), start at zero
+  CU(cudaMemsetAsync(base, 0, op_header() + align256((size_t)kMaxF4Tokens * d / 2) + align256((size_t)d / 64 * 512),
+                     s));
+  CU(nvf4_sf_tile(*E, nullptr, V, d, A_KMAJOR, sfe, s));
+  ActQuantArgs q{};
+  q.xf = d_x;
+  q.K = d;
+  q.codes = xcodes;
+  q.scales = xscales;
+  q.sx = sx;
+  CU_LAUNCH(launch_k(k_act_quant, dim3(B), dim3(256), 0, s, q));
+  char msg[256];
+  CU(lmhead_fused_f4_launch(*E, sfe, xcodes, kMaxF4Tokens, xscales, sx, B, V, d, mask_id, stats, d_s, lmf,
+                            (int*)base, s, msg, sizeof(msg)));
+  return DLM_OK;
+}
+
 size_t dlm_gemm_nvfp4_scratch_size(int T, int N, int K) {
   if (T < 1 || T > kMaxF4Tokens || N < 1 || K < 256 || K % 256 || K > 16384) return 0;
   return op_header() + op_counters(N) + align256(gemm_fp4_partial_bytes(T, N, K, A_KMAJOR)) +

@@ -239,6 +239,60 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool a_mn_major,
          | (uint32_t(m >> 4) << 24);     // M / 16
 }
 
+// ---------------------------------------------------------------- block-scaled FP4 MMA
+// Shared-memory descriptor of a 32-row x 16-byte block without swizzle (the tcgen05.cp
+// source): core matrices of 8 rows x 16 bytes, 128 bytes apart.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= uint64_t((smem_addr >> 4) & 0x3FFF);
+  d |= uint64_t(128 >> 4) << 16;  // leading byte offset (one core matrix along K: unused)
+  d |= uint64_t(128 >> 4) << 32;  // stride byte offset: next 8 rows
+  d |= uint64_t(1) << 46;         // descriptor version for sm_100
+  return d;                       // layout type 0: no swizzle
+}
+
+__device__ __forceinline__ void tmem_cp_32x128(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T with e2m1 operands and e4m3 scales per 16 elements.
+__device__ __forceinline__ void mma_nvf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Instruction descriptor of kind::mxf4nvf4: A and B e2m1 (format 1), K-major, e4m3 scales,
+// M = m, N = n, K = 64.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
+  return (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+
+// Instruction descriptor of kind::f16 with f16 A/B, fp32 D, M = m, N = n.
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                       // D format fp32
+         | (0u << 7)                     // A f16
+         | (0u << 10)                    // B f16
+         | (uint32_t(a_mn_major) << 15)
+         | (uint32_t(b_mn_major) << 16)
+         | (uint32_t(n >> 3) << 17)
+         | (uint32_t(m >> 4) << 24);
+}
+
 // ---------------------------------------------------------------- stream-K partition
 // The (tile, k-block) units of a GEMM are cut into `grid` contiguous ranges; CTA c owns
 // units [unit_begin(c), unit_begin(c + 1)).

@@ -66,47 +66,6 @@ struct F4KArgs {
   int* err;
 };
 
-// Shared-memory descriptor of a 32-row x 16-byte block without swizzle (the tcgen05.cp
-// source): core matrices of 8 rows x 16 bytes, 128 bytes apart.
-__device__ __forceinline__ uint64_t sf_desc(uint32_t smem_addr) {
-  uint64_t d = 0;
-  d |= uint64_t((smem_addr >> 4) & 0x3FFF);
-  d |= uint64_t(128 >> 4) << 16;  // leading byte offset (one core matrix along K: unused)
-  d |= uint64_t(128 >> 4) << 32;  // stride byte offset: next 8 rows
-  d |= uint64_t(1) << 46;         // descriptor version for sm_100
-  return d;                       // layout type 0: no swizzle
-}
-
-__device__ __forceinline__ void tmem_cp_32x128(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
-// D[tmem] (+)= A[smem] * B[smem]^T with e2m1 operands and e4m3 scales per 16 elements.
-__device__ __forceinline__ void mma_nvf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
-          tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
-      : "memory");
-}
-
-// Instruction descriptor of kind::mxf4nvf4: A and B e2m1 (format 1), K-major, e4m3 scales,
-// M = m, N = n, K = 64.
-__host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
-  return (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
-}
-
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 __device__ __forceinline__ void epi_sync_f4() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __global__ void __launch_bounds__(192, 1)
@@ -363,6 +322,12 @@ void partition_f4(int T, int N, int K, int a_mode, GemmOut* o) {
 }
 
 }  // namespace
+
+bool encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                  uint32_t box_outer, bool swizzle128, char* err, size_t errlen) {
+  return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner, outer, inner, box_inner, box_outer,
+                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, err, errlen);
+}
 
 size_t gemm_fp4_partial_bytes(int T, int N, int K, int a_mode) {
   GemmOut o;

@@ -190,6 +190,18 @@ cudaError_t lmhead_fused_launch(const void* x2, int x2_rows, int hi_row, int lo_
                                 float* s, void* scratch, int* d_err, cudaStream_t st, char* err,
                                 size_t errlen);
 
+// The same pass with NVFP4 E (codes [V][d/2], e4m3 scales [V][d/16], tensor scale; sfe_tiled
+// its scales re-tiled by nvf4_sf_tile) and x quantized by the last RMSNorm (codes [x_rows][d/2],
+// token t in row t; tiled scales; row scales sx[T]).  T <= 32, d % 512 == 0, d <= 2560.
+bool lmhead_fused_f4_supported(int T, int d);
+cudaError_t lmhead_fused_f4_launch(const dlm_nvfp4_matrix& E, const uint8_t* sfe_tiled, const uint8_t* xcodes,
+                                   int x_rows, const uint8_t* xscales, const float* sx, int T, int V, int d,
+                                   int mask_id, dlm_row_stats stats, float* s, void* scratch, int* d_err,
+                                   cudaStream_t st, char* err, size_t errlen);
+// 2-D tensor map of a byte matrix [outer][inner] (rows of `inner` bytes).
+bool encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                  uint32_t box_outer, bool swizzle128, char* err, size_t errlen);
+
 // attention (dlm_attention.cu)
 struct AttnArgs {
   const __nv_bfloat16* q;    // [T][Hq][hd]

@@ -55,6 +55,9 @@ struct LmfArgs {
   int* part_arg;        // [n_clu][32]
   float* part_s;        // [n_clu][d][32]
   int* err;
+  float s_scale;        // multiplies s (the NVFP4 E tensor scale; 1 for bf16 E)
+  const float* sx;      // NVFP4: per-token scales of the quantized x
+  float se;             // NVFP4: tensor scale of E
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -553,7 +556,7 @@ __global__ void __launch_bounds__(kLmfWarps * 32) k_lmf_combine(LmfArgs a, dlm_r
         const float m2 = cm[(2 * kLmfWarps + q) * 32 + tid], c2 = cm[(3 * kLmfWarps + q) * 32 + tid];
         if (m2 > bm || (m2 == bm && c2 < bc)) { bm = m2; bc = c2; }
       }
-      iZ[tid] = a.given ? 1.f : 1.f / Z;
+      iZ[tid] = (a.given ? 1.f : 1.f / Z) * a.s_scale;
       if (blockIdx.x == 0 && tid < a.T) {
         const float lse = Mt[tid] + logf(Z);
         stats.m[tid] = bm;
@@ -606,6 +609,432 @@ __global__ void __launch_bounds__(kLmfWarps * 32) k_lmf_combine(LmfArgs a, dlm_r
     for (int wv = 0; wv < kLmfWarps; ++wv) v += red[wv][fl][t];  // warps in order
     s[(size_t)t * a.d + blockIdx.x * 32 + fl] = v * iZ[t];
   }
+}
+
+// ------------------------------------------------------------------------------------------
+// NVFP4 E: the same pass with E stored as e2m1 codes, e4m3 scales per 16 and an fp32 tensor
+// scale S_E, and x quantized the same way per row (scale S_x[t]) by the last RMSNorm:
+//   L  partial logits on the block-scaled FP4 tensor cores (kind::mxf4nvf4, 256 reduction
+//      elements per stage: E codes 16 KB, x codes 4 KB, both operands' scales re-tiled for
+//      tcgen05.cp), times S_E S_x[t] in the epilogue;
+//   X  exchange and row statistics as above; P is written as f16 (one operand, N = 32);
+//   PE s^T += E^T P with kind::f16 MMAs: four dequantisation warps re-read the E tile's codes
+//      and scales (64 vocabulary rows x 128 features per step, from L2), turn them into f16
+//      (e2m1 x e4m3 values are exact in f16) in the MN-major layout the MMA reads, and hand
+//      them over through a two-slot ring.  The combine multiplies s by S_E.
+// Warps: 0 lane 0 = producer of the L ring, lane 1 = producer of the PE code ring; 1 = MMA;
+// 2..5 = statistics; 6..9 = dequantisation.
+constexpr int kF4LmStages = 4;
+constexpr int kF4LmStageBytes = 24576;  // E codes 16 KB | x codes 4 KB | E scales 2 KB | x scales 2 KB
+constexpr int kF4LmPcStages = 4;
+constexpr int kF4LmPcBytes = 5120;      // E codes [64 vocab][64 B] | E scales [64 vocab][16 B]
+constexpr int kF4LmPhBytes = 16384;     // f16 E^T tile: 2 boxes [64 vocab][64 features]
+constexpr int kF4LmPBytes = 8192;       // P f16 [32 tokens][128 vocab]: 2 atoms of 64
+constexpr int kF4LmMaxChunks = 10;      // d / 2 <= 1280 (TMEM: 64 + 10 x 32 + 128 columns)
+constexpr int kF4LmSCol = 64;           // TMEM column of the first s accumulator
+constexpr int kF4LmSfCol = 384;         // TMEM columns of the scale-factor slots
+constexpr int kF4LmThreads = 320;
+constexpr float kF4PScale = 16.f;       // P is stored as f16 times this (p <= e^8 stays finite)
+constexpr int kF4LmSmem = kF4LmStages * kF4LmStageBytes + kF4LmPcStages * kF4LmPcBytes + 2 * kF4LmPhBytes +
+                          2 * kF4LmPBytes + 3 * kLmXBytes + 1024 + 1024;
+static_assert(kF4LmSmem <= 232448, "fused NVFP4 LM head shared memory");
+
+__device__ __forceinline__ uint32_t f16x2_from_e2m1x2(uint32_t two) {
+  uint32_t h;
+  asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(h) : "r"(two));
+  return h;
+}
+__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint32_t two) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 b;\n\tcvt.u16.u32 b, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, b;\n\t}" : "=r"(h) : "r"(two));
+  return h;
+}
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// Offset of element (row, v) of the f16 P tile (K-major B operand, 128-byte swizzle, two
+// 64-wide atoms of 32 rows each).
+__device__ __forceinline__ uint32_t p16_offset(int row, int v) {
+  const int atom = v >> 6, c = v & 63;
+  return (uint32_t)(atom * 4096 + row * 128 + ((((c >> 3) ^ (row & 7)) << 4) | ((c & 7) << 1)));
+}
+
+__global__ void __launch_bounds__(kF4LmThreads, 1)
+k_lmhead_fused_f4(const __grid_constant__ CUtensorMap tec, const __grid_constant__ CUtensorMap tep,
+                  const __grid_constant__ CUtensorMap tes, const __grid_constant__ CUtensorMap txc,
+                  const uint8_t* __restrict__ sfe, const uint8_t* __restrict__ sfx, LmfArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* ring = smem;                                                  // L ring
+  uint8_t* pcr = ring + kF4LmStages * kF4LmStageBytes;                   // PE code ring
+  uint8_t* phr = pcr + kF4LmPcStages * kF4LmPcBytes;                     // f16 E^T ring [2]
+  uint8_t* pbuf = phr + 2 * kF4LmPhBytes;                                // P [2]
+  float* mine = (float*)(pbuf + 2 * kF4LmPBytes);                        // [32][128]
+  float* theirs = mine + kLmT * 128;                                     // [2][32][128]
+  uint64_t* bars = (uint64_t*)(theirs + 2 * kLmT * 128);
+  uint64_t* full = bars;                          // [S]
+  uint64_t* empty = full + kF4LmStages;           // [S]
+  uint64_t* pc_full = empty + kF4LmStages;        // [PS]
+  uint64_t* pc_empty = pc_full + kF4LmPcStages;   // [PS] (128 arrivals)
+  uint64_t* ph_full = pc_empty + kF4LmPcStages;   // [2] (128 arrivals)
+  uint64_t* ph_empty = ph_full + 2;               // [2] (MMA commit)
+  uint64_t* accl_full = ph_empty + 2;             // [2]
+  uint64_t* accl_empty = accl_full + 2;           // [2] (128 arrivals)
+  uint64_t* p_ready = accl_empty + 2;             // [2] (4 arrivals)
+  uint64_t* pe_done = p_ready + 2;                // [2]
+  uint64_t* xfull = pe_done + 2;                  // [2] (128 remote arrivals)
+  uint64_t* mma_done = xfull + 2;
+  uint32_t* tmem_holder = (uint32_t*)(mma_done + 1);
+  int* flag = (int*)(mma_done + 2);
+  float* fac = (float*)(mma_done + 3);            // [32]
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
+  const int clu = blockIdx.x / 2;
+  const int dh = a.d / 2, d0 = (int)rank * dh;
+  const int KB = dh / 256, CH = dh / 128, NB64 = a.d / 64;
+  const int tb = lm_tile_begin(clu, a.n_tiles, a.n_clu), te = lm_tile_begin(clu + 1, a.n_tiles, a.n_clu);
+  const int nt = te - tb;
+
+  if (warp == 1 && lane == 0) {
+    for (int i = 0; i < kF4LmStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < kF4LmPcStages; ++i) { mbar_init(&pc_full[i], 1); mbar_init(&pc_empty[i], 128); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ph_full[i], 128);
+      mbar_init(&ph_empty[i], 1);
+      mbar_init(&accl_full[i], 1);
+      mbar_init(&accl_empty[i], 128);
+      mbar_init(&p_ready[i], 4);
+      mbar_init(&pe_done[i], 1);
+      mbar_init(&xfull[i], 128);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tec);
+    prefetch_tmap(&tep);
+    prefetch_tmap(&tes);
+    prefetch_tmap(&txc);
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  pdl_trigger();
+  pdl_wait();
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- L producer: per tile, KB stages of 256 reduction elements
+    const uint64_t keep = l2_policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int i = 0; i < nt && ok; ++i) {
+      const int tile = tb + i;
+      for (int kb = 0; kb < KB && ok; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, a.err)) { ok = false; break; }
+        uint8_t* st = ring + stage * kF4LmStageBytes;
+        const int kc = (d0 + kb * 256) / 2;         // code byte of the stage's first element
+        const int b64 = (d0 + kb * 256) / 64;       // its 64-element block
+        mbar_arrive_expect_tx(&full[stage], kF4LmStageBytes);
+        tma_load_2d_hint(st, &tec, &full[stage], kc, tile * 128, keep);
+        tma_load_2d(st + 16384, &txc, &full[stage], kc, 0);
+        bulk_load(st + 20480, sfe + ((size_t)tile * NB64 + b64) * 512, 2048, &full[stage]);
+        bulk_load(st + 22528, sfx + (size_t)b64 * 512, 2048, &full[stage]);
+        if (++stage == kF4LmStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    for (int i = 0; i < kF4LmStages && ok; ++i) {  // no copy left in flight
+      if (!mbar_wait(&empty[stage], phase ^ 1, a.err)) break;
+      if (++stage == kF4LmStages) { stage = 0; phase ^= 1; }
+    }
+  } else if (warp == 0 && lane == 1) {
+    // ---------------- PE producer: per tile, CH x 2 steps of E codes [64 vocab][128 features]
+    // and their scales (a 16-byte box holding this step's 8 scale bytes)
+    const uint64_t drop = l2_policy_evict_first();
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int i = 0; i < nt && ok; ++i) {
+      const int tile = tb + i;
+      for (int ch = 0; ch < CH && ok; ++ch)
+        for (int vh = 0; vh < 2 && ok; ++vh) {
+          if (!mbar_wait(&pc_empty[stage], phase ^ 1, a.err)) { ok = false; break; }
+          uint8_t* st = pcr + stage * kF4LmPcBytes;
+          const int f0 = d0 + ch * 128;
+          mbar_arrive_expect_tx(&pc_full[stage], kF4LmPcBytes);
+          tma_load_2d_hint(st, &tep, &pc_full[stage], f0 / 2, tile * 128 + vh * 64, drop);
+          tma_load_2d_hint(st + 4096, &tes, &pc_full[stage], (f0 / 16) & ~15, tile * 128 + vh * 64, drop);
+          if (++stage == kF4LmPcStages) { stage = 0; phase ^= 1; }
+        }
+    }
+    for (int i = 0; i < kF4LmPcStages && ok; ++i) {
+      if (!mbar_wait(&pc_empty[stage], phase ^ 1, a.err)) break;
+      if (++stage == kF4LmPcStages) { stage = 0; phase ^= 1; }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc_l = idesc_nvf4(128, kLmT);
+    const uint32_t idesc_pe = idesc_f16(128, kLmT, true, false);
+    int stage = 0, fs = 0;
+    uint32_t phase = 0, fphase = 0;
+    bool ok = true;
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, a.err)) != 0;
+    };
+    auto mma_l = [&](int i) {
+      const int b = i & 1;
+      if (!wait_all(&accl_empty[b], ((i >> 1) & 1) ^ 1)) { ok = false; return; }
+      tc_fence_after();
+      const uint32_t dl = tmem + b * kLmT;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!wait_all(&full[stage], phase)) { ok = false; return; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(ring + stage * kF4LmStageBytes);
+        const uint32_t sfa_col = tmem + kF4LmSfCol + stage * 32, sfb_col = sfa_col + 16;
+        const uint64_t ad = sw128_desc(sa, 16, 1024), bd = sw128_desc(sa + 16384, 16, 1024);
+        const uint64_t fa = sf_desc(sa + 20480), fb = sf_desc(sa + 22528);
+        if (elect_one()) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tmem_cp_32x128(sfa_col + 4 * j, fa + 32 * j);
+            tmem_cp_32x128(sfb_col + 4 * j, fb + 32 * j);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            mma_nvf4(dl, ad + 2 * j, bd + 2 * j, idesc_l, sfa_col + 4 * j, sfb_col + 4 * j, (kb | j) ? 1u : 0u);
+          mma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == kF4LmStages) { stage = 0; phase ^= 1; }
+      }
+      if (elect_one()) mma_commit(&accl_full[b]);
+      __syncwarp();
+    };
+    auto mma_pe = [&](int i) {
+      const int b = i & 1;
+      if (!wait_all(&p_ready[b], (i >> 1) & 1)) { ok = false; return; }
+      tc_fence_after();
+      const uint64_t pd = sw128_desc(smem_u32(pbuf + b * kF4LmPBytes), 16, 1024);
+      for (int ch = 0; ch < CH; ++ch) {
+        const uint32_t ds = tmem + kF4LmSCol + ch * kLmT;
+        for (int vh = 0; vh < 2; ++vh) {
+          if (!wait_all(&ph_full[fs], fphase)) { ok = false; return; }
+          tc_fence_after();
+          const uint64_t ad0 = sw128_desc(smem_u32(phr + fs * kF4LmPhBytes), 8192, 1024);
+          if (elect_one()) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)  // 16 vocabulary rows (2048 B of E^T, 32 B of P) per step
+              mma_bf16(ds, ad0 + 128 * k, pd + (vh * 4096 + k * 32) / 16, idesc_pe,
+                       (i == 0 && vh == 0 && k == 0) ? 0u : 1u);
+            mma_commit(&ph_empty[fs]);
+          }
+          __syncwarp();
+          if (++fs == 2) { fs = 0; fphase ^= 1; }
+        }
+      }
+      if (elect_one()) mma_commit(&pe_done[b]);
+      __syncwarp();
+    };
+    for (int i = 0; i < nt && ok; ++i) {
+      mma_l(i);
+      if (ok && i >= 1) mma_pe(i - 1);
+    }
+    if (ok && nt > 0) mma_pe(nt - 1);
+    if (elect_one()) {
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, a.err);
+    }
+    __syncwarp();
+  } else if (warp >= 6) {
+    // ---------------- dequantisation: thread dt owns vocabulary row dt / 2 and features
+    // [64 (dt % 2), + 64) of each step's 128
+    const int dt = threadIdx.x - 192, v = dt / 2, hf = dt % 2;
+    int stage = 0, fs = 0;
+    uint32_t phase = 0, fphase = 0;
+    bool ok = true;
+    for (int i = 0; i < nt && ok; ++i)
+      for (int ch = 0; ch < CH && ok; ++ch)
+        for (int vh = 0; vh < 2 && ok; ++vh) {
+          const int sofs = ((d0 + ch * 128) / 16) & 15;  // this step's first scale in the 16-byte box
+          if (!mbar_wait(&ph_empty[fs], fphase ^ 1, a.err)) { ok = false; break; }
+          if (!mbar_wait(&pc_full[stage], phase, a.err)) { ok = false; break; }
+          const uint8_t* st = pcr + stage * kF4LmPcBytes;
+          const uint4 c0 = *reinterpret_cast<const uint4*>(st + v * 64 + hf * 32);
+          const uint4 c1 = *reinterpret_cast<const uint4*>(st + v * 64 + hf * 32 + 16);
+          const uint32_t sc4 = *reinterpret_cast<const uint32_t*>(st + 4096 + v * 16 + sofs + hf * 4);
+          mbar_arrive(&pc_empty[stage]);  // the codes and scales are in registers now
+          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          const uint32_t tile_b = smem_u32(phr + fs * kF4LmPhBytes) + hf * 8192 + v * 128;
+#pragma unroll
+          for (int blk = 0; blk < 4; ++blk) {  // 16 features: two code words, one scale
+            const uint32_t sb = (sc4 >> (8 * blk)) & 0xFFu;
+            const uint32_t sig = f16x2_from_e4m3x2(sb | (sb << 8));
+            uint32_t o[8];
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+              const uint32_t word = cw[2 * blk + w];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) o[4 * w + q] = hmul2(f16x2_from_e2m1x2((word >> (8 * q)) & 0xFFu), sig);
+            }
+            const int c = 2 * blk;  // 16-byte chunk of the 128-byte row (8 features each)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(tile_b + (((c) ^ (v & 7)) << 4)),
+                         "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]) : "memory");
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(tile_b + (((c + 1) ^ (v & 7)) << 4)),
+                         "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7]) : "memory");
+          }
+          fence_proxy_async_smem();  // generic-proxy writes visible to the tensor cores
+          mbar_arrive(&ph_full[fs]);
+          if (++stage == kF4LmPcStages) { stage = 0; phase ^= 1; }
+          if (++fs == 2) { fs = 0; fphase ^= 1; }
+        }
+  } else if (warp >= 2) {
+    // ---------------- statistics: exchange, running reference, P (f16), rescale, outputs
+    const int et = threadIdx.x - 64;
+    const int q = warp % 4, row = q * 32 + lane;
+    const int tw = et / 32;
+    float ref[8], Z[8], A[8], mbest[8];
+    int arg[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { ref[j] = -INFINITY; Z[j] = 0.f; A[j] = 0.f; mbest[j] = -INFINITY; arg[j] = 0x7fffffff; }
+    float sct[8];  // S_E S_x[t] of this warp's tokens (0 past T)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sct[j] = tw * 8 + j < a.T ? a.se * a.sx[tw * 8 + j] : 0.f;
+    const uint32_t theirs_peer = map_peer(smem_u32(theirs), peer);
+    const uint32_t xfull_peer = map_peer(smem_u32(xfull), peer);
+    bool ok = true;
+    for (int i = 0; i < nt && ok; ++i) {
+      const int b = i & 1, tile = tb + i;
+      if (et == 0) *flag = mbar_wait(&accl_full[b], (i >> 1) & 1, a.err) ? 1 : 0;
+      epi_bar();
+      ok = *flag != 0;
+      epi_bar();
+      if (!ok) break;
+      tc_fence_after();
+      float lp[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * kLmT, lp);
+      tc_fence_before();
+      mbar_arrive(&accl_empty[b]);
+      const uint32_t tpeer = theirs_peer + (uint32_t)(b * kLmT * 128 * 4);
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        mine[t * 128 + row] = lp[t];
+        st_cluster_f32(tpeer + (uint32_t)((t * 128 + row) * 4), lp[t]);
+      }
+      mbar_arrive_remote(xfull_peer + b * 8);
+      if (epi_any(!mbar_wait_cluster(&xfull[b], (i >> 1) & 1, a.err))) { ok = false; break; }
+      if (epi_any(i >= 2 && !mbar_wait(&pe_done[b], ((i - 2) >> 1) & 1, a.err))) { ok = false; break; }
+      const float* tb_ = theirs + b * kLmT * 128;
+      uint8_t* pt = pbuf + b * kF4LmPBytes;
+      int need = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int t = tw * 8 + j;
+        const float4 x0 = *reinterpret_cast<const float4*>(mine + t * 128 + lane * 4);
+        const float4 x1 = *reinterpret_cast<const float4*>(tb_ + t * 128 + lane * 4);
+        float l[4] = {(x0.x + x1.x) * sct[j], (x0.y + x1.y) * sct[j], (x0.z + x1.z) * sct[j], (x0.w + x1.w) * sct[j]};
+        float mx = -INFINITY;
+        int ax = 0x7fffffff;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int vv = tile * 128 + lane * 4 + u;
+          if (vv >= a.V || vv == a.mask_id || t >= a.T) l[u] = -INFINITY;
+          if (l[u] > mx) { mx = l[u]; ax = vv; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const float m2 = __shfl_xor_sync(0xffffffffu, mx, o);
+          const int a2 = __shfl_xor_sync(0xffffffffu, ax, o);
+          if (m2 > mx || (m2 == mx && a2 < ax)) { mx = m2; ax = a2; }
+        }
+        if (mx > mbest[j]) { mbest[j] = mx; arg[j] = ax; }
+        float f = 1.f;
+        if (i == 0) {
+          ref[j] = mx;
+        } else if (mx > ref[j] + kLmRescale) {
+          f = expf(ref[j] - mx);
+          ref[j] = mx;
+          Z[j] *= f;
+          A[j] *= f;
+          need = 1;
+        }
+        if (lane == 0) fac[t] = f;
+        float zs = 0.f, as = 0.f;
+        __align__(8) __half hv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float p = (l[u] == -INFINITY) ? 0.f : expf(l[u] - ref[j]);
+          zs += p;
+          as += (p > 0.f) ? p * l[u] : 0.f;
+          hv[u] = __float2half_rn(t < a.T ? p * kF4PScale : 0.f);
+        }
+        *reinterpret_cast<uint2*>(pt + p16_offset(t, lane * 4)) = *reinterpret_cast<const uint2*>(hv);
+        Z[j] += warp_sum(zs);
+        A[j] += warp_sum(as);
+      }
+      const bool rescale = epi_any(need != 0);
+      if (rescale) {
+        if (epi_any(i >= 1 && !mbar_wait(&pe_done[(i - 1) & 1], ((i - 1) >> 1) & 1, a.err))) { ok = false; break; }
+        tc_fence_after();
+        float fv[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) fv[t] = fac[t];
+        for (int ch = 0; ch < CH; ++ch) {
+          float sv[32];
+          const uint32_t sa = tmem + ((uint32_t)(q * 32) << 16) + kF4LmSCol + ch * kLmT;
+          tmem_ld32(sa, sv);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) sv[t] *= fv[t];
+          tmem_st32_f(sa, sv);
+        }
+        tc_fence_before();
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready[b]);
+    }
+    if (ok && nt > 0) {
+      const int last = nt - 1;
+      if (et == 0) *flag = mbar_wait(&pe_done[last & 1], (last >> 1) & 1, a.err) ? 1 : 0;
+      epi_bar();
+      ok = *flag != 0;
+      epi_bar();
+      if (ok) {
+        tc_fence_after();
+        for (int ch = 0; ch < CH; ++ch) {
+          float sv[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + kF4LmSCol + ch * kLmT, sv);
+          float4* dst = reinterpret_cast<float4*>(a.part_s + ((size_t)clu * a.d + d0 + ch * 128 + row) * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) dst[u] = make_float4(sv[4 * u], sv[4 * u + 1], sv[4 * u + 2], sv[4 * u + 3]);
+        }
+        if (rank == 0 && lane == 0) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int t = tw * 8 + j;
+            float* ps = a.part_stats + ((size_t)clu * 32 + t) * 4;
+            ps[0] = ref[j];
+            ps[1] = Z[j];
+            ps[2] = A[j];
+            ps[3] = mbest[j];
+            a.part_arg[(size_t)clu * 32 + t] = arg[j];
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
@@ -661,6 +1090,7 @@ cudaError_t lmhead_fused_launch(const void* x2, int x2_rows, int hi_row, int lo_
   a.n_tiles = (V + 127) / 128;
   a.n_clu = a.n_tiles < kLmMaxClusters ? a.n_tiles : kLmMaxClusters;
   a.given = p_given != nullptr;
+  a.s_scale = 1.f;
   uint8_t* sc = (uint8_t*)scratch;
   a.part_stats = (float*)sc;
   a.part_arg = (int*)(sc + (size_t)a.n_clu * 32 * 4 * sizeof(float));
@@ -690,6 +1120,76 @@ cudaError_t lmhead_fused_launch(const void* x2, int x2_rows, int hi_row, int lo_
   cfg.attrs = at;
   cfg.numAttrs = g_pdl ? 2 : 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, k_lmhead_fused, tek, tem, tx, tp, a);
+  if (e != cudaSuccess) return e;
+  return launch_k(k_lmf_combine, dim3(d / 32), dim3(kLmfWarps * 32), kLmfSmem, st, a, stats, s);
+}
+
+bool lmhead_fused_f4_supported(int T, int d) {
+  return T >= 1 && T <= kLmT && d % 512 == 0 && d / 256 <= kF4LmMaxChunks;
+}
+
+// E: NVFP4 codes [V][d/2], scales [V][d/16], tensor scale; sfe_tiled: its scales re-tiled for
+// the block-scaled MMA; x: codes [x_rows][d/2] (token t in row t), tiled scales and row scales
+// sx[T] as the quantizer of the last RMSNorm leaves them.
+cudaError_t lmhead_fused_f4_launch(const dlm_nvfp4_matrix& E, const uint8_t* sfe_tiled, const uint8_t* xcodes,
+                                   int x_rows, const uint8_t* xscales, const float* sx, int T, int V, int d,
+                                   int mask_id, dlm_row_stats stats, float* s, void* scratch, int* d_err,
+                                   cudaStream_t st, char* err, size_t errlen) {
+  if (!lmhead_fused_f4_supported(T, d) || !E.codes || !E.scales || !sfe_tiled || !xcodes || !xscales || !sx ||
+      x_rows < T) {
+    snprintf(err, errlen, "nvfp4 lm head: unsupported arguments T=%d d=%d x_rows=%d", T, d, x_rows);
+    return cudaErrorInvalidValue;
+  }
+  {
+    static PerDeviceOnce once;
+    const int r = once_on_current_device(once, [] {
+      cudaError_t e = cudaFuncSetAttribute(k_lmhead_fused_f4, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4LmSmem);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_lmf_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, kLmfSmem);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_lmf_combine, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+      return (int)e;
+    });
+    if (r != 0) return (cudaError_t)r;
+  }
+  LmfArgs a{};
+  a.V = V;
+  a.d = d;
+  a.T = T;
+  a.mask_id = mask_id;
+  a.n_tiles = (V + 127) / 128;
+  a.n_clu = a.n_tiles < kLmMaxClusters ? a.n_tiles : kLmMaxClusters;
+  a.given = 0;
+  a.se = E.tensor_scale;
+  a.sx = sx;
+  a.s_scale = E.tensor_scale / kF4PScale;
+  uint8_t* sc = (uint8_t*)scratch;
+  a.part_stats = (float*)sc;
+  a.part_arg = (int*)(sc + (size_t)a.n_clu * 32 * 4 * sizeof(float));
+  a.part_s = (float*)(sc + (((size_t)a.n_clu * 32 * 5 * 4 + 255) & ~(size_t)255));
+  a.err = d_err;
+  CUtensorMap tec, tep, tes, txc;
+  bool ok = encode_u8_2d(&tec, E.codes, (uint64_t)d / 2, V, 128, 128, true, err, errlen);
+  ok = ok && encode_u8_2d(&tep, E.codes, (uint64_t)d / 2, V, 64, 64, false, err, errlen);
+  ok = ok && encode_u8_2d(&tes, E.scales, (uint64_t)d / 16, V, 16, 64, false, err, errlen);
+  ok = ok && encode_u8_2d(&txc, xcodes, (uint64_t)d / 2, x_rows, 128, 32, true, err, errlen);
+  if (!ok) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * a.n_clu);
+  cfg.blockDim = dim3(kF4LmThreads);
+  cfg.dynamicSmemBytes = kF4LmSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = g_pdl ? 2 : 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_lmhead_fused_f4, tec, tep, tes, txc, sfe_tiled, xscales, a);
   if (e != cudaSuccess) return e;
   return launch_k(k_lmf_combine, dim3(d / 32), dim3(kLmfWarps * 32), kLmfSmem, st, a, stats, s);
 }

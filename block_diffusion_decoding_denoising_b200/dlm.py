@@ -123,6 +123,9 @@ def lib():
         L.dlm_bd_attention_fp8.argtypes = [p, p, p, p, p, p, i, i, i, i, i, i, i, p, z, p]
         L.dlm_commit.argtypes = [p, p, p, p, p, p, p, i, i, f, i, i, p]
         L.dlm_nvfp4_quantize.argtypes = [p, i, i, p, p, p, p]
+        L.dlm_lmhead_nvfp4_scratch_size.restype = z
+        L.dlm_lmhead_nvfp4_scratch_size.argtypes = [i, i, i]
+        L.dlm_lmhead_rowstats_nvfp4.argtypes = [p, C.POINTER(Nvfp4Matrix), i, i, i, i, RowStats, p, p, z, p]
         L.dlm_gemm_nvfp4_scratch_size.restype = z
         L.dlm_gemm_nvfp4_scratch_size.argtypes = [i, i, i]
         L.dlm_gemm_nvfp4.argtypes = [p, C.POINTER(Nvfp4Matrix), p, i, i, i, p, z, p]
@@ -213,6 +216,26 @@ def lmhead_rowstats(x, E, mask_id=-1, p_given=None, stream=None):
     sc = _scratch(n, x.device)
     _check(lib().dlm_lmhead_rowstats(_ptr(x), _ptr(E), B, V, d, int(mask_id), _ptr(p_given), _rowstats(st),
                                      _ptr(s), _ptr(sc), n, _stream(stream)))
+    st["s"] = s
+    return st
+
+
+def lmhead_rowstats_nvfp4(x, Eq, mask_id=-1, stream=None):
+    """Fused LM head on an NVFP4 embedding: stats of Q(x) E^T and s = P E.  x fp32 [B][d]
+    (normalised, quantized per row by the library); Eq a dict with device codes, scales,
+    tscale, rows (V) and cols (d)."""
+    import torch
+    B, d = x.shape
+    V = Eq["rows"]
+    st = new_stats(B, x.device)
+    s = torch.empty((B, d), dtype=torch.float32, device=x.device)
+    n = lib().dlm_lmhead_nvfp4_scratch_size(B, V, d)
+    if n == 0:
+        raise DlmError(DLM_EUNSUPPORTED, "nvfp4 lm head: unsupported shape B=%d V=%d d=%d" % (B, V, d))
+    sc = _scratch(n, x.device)
+    m = _q_matrix(Eq)
+    _check(lib().dlm_lmhead_rowstats_nvfp4(_ptr(x), C.byref(m), B, V, d, int(mask_id), _rowstats(st), _ptr(s),
+                                           _ptr(sc), n, _stream(stream)))
     st["s"] = s
     return st
 

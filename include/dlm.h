@@ -332,6 +332,20 @@ size_t dlm_gemm_nvfp4_scratch_size(int T, int N, int K);
 dlm_status dlm_gemm_nvfp4(const float* d_x, const dlm_nvfp4_matrix* w, float* d_y, int T, int N, int K,
                           void* d_scratch, size_t scratch_bytes, void* stream);
 
+/* The fused LM head of dlm_lmhead_rowstats with an NVFP4 embedding E [V][d] (see
+ * dlm_nvfp4_matrix; host struct, device arrays): x (fp32 [B][d], already normalised) is
+ * quantized per row as for dlm_gemm_nvfp4, the logits S_E S_x[t] (q_x sigma_x)(q_E sigma_E)^T
+ * run on the block-scaled FP4 tensor cores and are never stored, and s = P E uses the
+ * dequantized E (e2m1 x e4m3 values, exact in f16) with P = softmax(logits) carried as f16,
+ * in the same pass over E ("QwenDLM-4B-ORL" model card, "The paper's evaluation pipeline": the
+ * LM head with fused row statistics; "ORL: diffusion LLMs get a learnable 'tokens per
+ * forward'", "What shipped": NVFP4 weights).  Mask id as dlm_lmhead_rowstats.  B <= 32,
+ * d % 512 == 0, d <= 2560; other shapes return DLM_EUNSUPPORTED (scratch size 0). */
+size_t dlm_lmhead_nvfp4_scratch_size(int B, int V, int d);
+dlm_status dlm_lmhead_rowstats_nvfp4(const float* d_x, const dlm_nvfp4_matrix* E, int B, int V, int d, int mask_id,
+                                     dlm_row_stats stats, float* d_s, void* d_scratch, size_t scratch_bytes,
+                                     void* stream);
+
 /* Version string of the build. */
 const char* dlm_version(void);
 
