@@ -643,9 +643,17 @@ def lmhead_case(args):
     tokens = torch.full((B,), V - 1, dtype=torch.int32, device="cuda")
     s = torch.zeros((B, d), dtype=torch.float32, device="cuda")
     out = {}
-    for name, fn in (("lmhead_given_p", lambda: dlm.lmhead_rowstats(x, E, mask_id=V - 1, p_given=P)),
-                     ("lmhead_softmax", lambda: dlm.lmhead_rowstats(x, E, mask_id=V - 1)),
-                     ("adapter", lambda: dlm.adapter_embed(E, Wa, tokens, s))):
+    if args.fmt == "nvfp4":
+        # E in NVFP4 (quantized on the device), x fp32 quantized per row by the call
+        Eq = dlm.nvfp4_matrix(E)
+        xf = H.float().contiguous()
+        del E
+        calls = (("lmhead_nvfp4_softmax", lambda: dlm.lmhead_rowstats_nvfp4(xf, Eq, mask_id=V - 1)),)
+    else:
+        calls = (("lmhead_given_p", lambda: dlm.lmhead_rowstats(x, E, mask_id=V - 1, p_given=P)),
+                 ("lmhead_softmax", lambda: dlm.lmhead_rowstats(x, E, mask_id=V - 1)),
+                 ("adapter", lambda: dlm.adapter_embed(E, Wa, tokens, s)))
+    for name, fn in calls:
         for _ in range(max(args.warmup, 1)):
             fn()
         torch.cuda.synchronize()
@@ -656,8 +664,15 @@ def lmhead_case(args):
         ev[1].record()
         torch.cuda.synchronize()
         out[name] = ev[0].elapsed_time(ev[1]) * 1e3 / args.steps
-    e_bytes = V * d * 2
     hbm, _, kind = peaks()
+    if args.fmt == "nvfp4":
+        e_bytes = V * d // 2 + V * d // 16  # codes and e4m3 scales, read once
+        gbs = e_bytes / (out["lmhead_nvfp4_softmax"] * 1e-6) / 1e9
+        print(json.dumps({"case": "lmhead", "fmt": "nvfp4", "us_per_call": out, "GBs": gbs, "frac": gbs / hbm,
+                          "peak": hbm, "peak_kind": kind,
+                          "note": "per call: scale re-tiling and x quantization besides the fused kernel"}), flush=True)
+        return
+    e_bytes = V * d * 2
     gbs = (e_bytes + B * V * 2) / (out["lmhead_given_p"] * 1e-6) / 1e9
     print(json.dumps({"case": "lmhead", "us_per_call": out, "given_p_GBs": gbs, "frac": gbs / hbm,
                       "peak": hbm, "peak_kind": kind}), flush=True)

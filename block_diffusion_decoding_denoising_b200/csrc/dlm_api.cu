@@ -231,7 +231,7 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   const size_t sfd = fp4_shapes ? align256(nvf4_sf_tile_bytes(c.d, c.ffn, A_KMAJOR)) : 0;
   const size_t sfe = fp4_shapes ? align256(nvf4_sf_tile_bytes(c.vocab, c.d, A_KMAJOR)) : 0;
   uint8_t* sf = fp4_shapes ? cv.take<uint8_t>((size_t)c.n_layers * (sfp + sfd) + sfe) : nullptr;
-  const bool fused = !fp4 && lmhead_fused_supported(B, c.d);
+  const bool fused = fp4 ? fp4_shapes && lmhead_fused_f4_supported(B, c.d) : lmhead_fused_supported(B, c.d);
   uint8_t* lmf = fused ? cv.take<uint8_t>(lmhead_fused_scratch_bytes(c.vocab, c.d)) : nullptr;
   if (x && base) {
     x->lmf = lmf;
@@ -573,7 +573,17 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
 
   // LM head: logits (finished inside the GEMM: its tiles are mostly single-slot), row
   // statistics, P = softmax (split bf16), s = P E
-  if (ctx->lmf && Tl <= 32) {
+  if (ctx->lmf && ctx->fp4 && Tp == 0) {
+    // one pass over the NVFP4 E: the rows of x were quantized by the last residual+RMSNorm
+    if (c.n_layers == 0) TRY(act_quant(r, T, ctx->xn, pad * d, d));
+    char msg[256];
+    cudaError_t e = lmhead_fused_f4_launch(ctx->w.q_embed, ctx->sf + c.n_layers * (ctx->sf_pair + ctx->sf_down),
+                                           ctx->xcodes, kMaxF4Tokens, ctx->xscales, ctx->sx, Tl, c.vocab, d,
+                                           c.mask_id, f.stats, f.s_out, ctx->lmf, ctx->d_err, r.s, msg, sizeof(msg));
+    if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "fused nvfp4 lm head: %s %s", cudaGetErrorString(e), msg);
+    return DLM_OK;
+  }
+  if (ctx->lmf && !ctx->fp4 && Tl <= 32) {
     // one pass over E: logits, row statistics and s = P E on the rows [Tp, T) of the split x
     char msg[256];
     cudaError_t e = lmhead_fused_launch(ctx->xn, (int)(2 * pad), Tp, (int)(pad + Tp), ctx->w.embed, nullptr, Tl,

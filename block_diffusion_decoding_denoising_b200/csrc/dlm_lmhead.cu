@@ -76,6 +76,10 @@ __device__ __forceinline__ uint32_t map_peer(uint32_t local_addr, uint32_t peer)
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
@@ -671,8 +675,8 @@ k_lmhead_fused_f4(const __grid_constant__ CUtensorMap tec, const __grid_constant
   uint8_t* pcr = ring + kF4LmStages * kF4LmStageBytes;                   // PE code ring
   uint8_t* phr = pcr + kF4LmPcStages * kF4LmPcBytes;                     // f16 E^T ring [2]
   uint8_t* pbuf = phr + 2 * kF4LmPhBytes;                                // P [2]
-  float* mine = (float*)(pbuf + 2 * kF4LmPBytes);                        // [32][128]
-  float* theirs = mine + kLmT * 128;                                     // [2][32][128]
+  float* mine = (float*)(pbuf + 2 * kF4LmPBytes);                        // [128][32]
+  float* theirs = mine + kLmT * 128;                                     // [2][128][32]
   uint64_t* bars = (uint64_t*)(theirs + 2 * kLmT * 128);
   uint64_t* full = bars;                          // [S]
   uint64_t* empty = full + kF4LmStages;           // [S]
@@ -688,7 +692,7 @@ k_lmhead_fused_f4(const __grid_constant__ CUtensorMap tec, const __grid_constant
   uint64_t* mma_done = xfull + 2;
   uint32_t* tmem_holder = (uint32_t*)(mma_done + 1);
   int* flag = (int*)(mma_done + 2);
-  float* fac = (float*)(mma_done + 3);            // [32]
+  float* fac = (float*)(mma_done + 3);            // [32] rescale factors, then [4][32] quarter maxima
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
@@ -870,7 +874,6 @@ k_lmhead_fused_f4(const __grid_constant__ CUtensorMap tec, const __grid_constant
           const uint4 c0 = *reinterpret_cast<const uint4*>(st + v * 64 + hf * 32);
           const uint4 c1 = *reinterpret_cast<const uint4*>(st + v * 64 + hf * 32 + 16);
           const uint32_t sc4 = *reinterpret_cast<const uint32_t*>(st + 4096 + v * 16 + sofs + hf * 4);
-          mbar_arrive(&pc_empty[stage]);  // the codes and scales are in registers now
           const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
           const uint32_t tile_b = smem_u32(phr + fs * kF4LmPhBytes) + hf * 8192 + v * 128;
 #pragma unroll
@@ -891,118 +894,129 @@ k_lmhead_fused_f4(const __grid_constant__ CUtensorMap tec, const __grid_constant
                          "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7]) : "memory");
           }
           fence_proxy_async_smem();  // generic-proxy writes visible to the tensor cores
+          // the code slot goes back only now that its values have been used: released right
+          // after the loads were issued, the next TMA into the slot sometimes landed first
+          mbar_arrive(&pc_empty[stage]);
           mbar_arrive(&ph_full[fs]);
           if (++stage == kF4LmPcStages) { stage = 0; phase ^= 1; }
           if (++fs == 2) { fs = 0; fphase ^= 1; }
         }
   } else if (warp >= 2) {
-    // ---------------- statistics: exchange, running reference, P (f16), rescale, outputs
-    const int et = threadIdx.x - 64;
-    const int q = warp % 4, row = q * 32 + lane;
-    const int tw = et / 32;
-    float ref[8], Z[8], A[8], mbest[8];
-    int arg[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) { ref[j] = -INFINITY; Z[j] = 0.f; A[j] = 0.f; mbest[j] = -INFINITY; arg[j] = 0x7fffffff; }
-    float sct[8];  // S_E S_x[t] of this warp's tokens (0 past T)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) sct[j] = tw * 8 + j < a.T ? a.se * a.sx[tw * 8 + j] : 0.f;
+    // ---------------- statistics.  Phase 1 (thread = vocabulary row q*32 + lane of the tile): the
+    // CTA's partial logits of the 32 tokens go to `mine` and to the peer's `theirs`, both laid
+    // out [vocab 128][token 32] with the 16-byte chunks of a row rotated by (row & 7) (no bank
+    // conflicts either way).  Phase 2 (thread = token t = lane, warp = vocabulary quarter q):
+    // the full logits of its 32 rows, their max and lowest argmax, all in registers; the four
+    // quarters agree on the tile max through shared memory, so every warp applies the same
+    // running reference r_t; per-quarter sums Z_q, A_q and (max, argmax) are merged once,
+    // after the last tile.
+    const int q = warp % 4, row = q * 32 + lane, t = lane;
+    const bool live = t < a.T;
+    const float sct = live ? a.se * a.sx[t] : 0.f;  // S_E S_x[t]
+    float ref = -INFINITY, Z = 0.f, A = 0.f, mbest = -INFINITY;
+    int arg = 0x7fffffff;
+    float* qmax = fac + 32;  // [4][32] quarter maxima of the current tile
     const uint32_t theirs_peer = map_peer(smem_u32(theirs), peer);
     const uint32_t xfull_peer = map_peer(smem_u32(xfull), peer);
     bool ok = true;
     for (int i = 0; i < nt && ok; ++i) {
       const int b = i & 1, tile = tb + i;
-      if (et == 0) *flag = mbar_wait(&accl_full[b], (i >> 1) & 1, a.err) ? 1 : 0;
+      if (threadIdx.x == 64) *flag = mbar_wait(&accl_full[b], (i >> 1) & 1, a.err) ? 1 : 0;
       epi_bar();
       ok = *flag != 0;
       epi_bar();
       if (!ok) break;
       tc_fence_after();
-      float lp[32];
-      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * kLmT, lp);
-      tc_fence_before();
-      mbar_arrive(&accl_empty[b]);
-      const uint32_t tpeer = theirs_peer + (uint32_t)(b * kLmT * 128 * 4);
+      {
+        float lp[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * kLmT, lp);
+        tc_fence_before();
+        mbar_arrive(&accl_empty[b]);
+        float4* mrow = reinterpret_cast<float4*>(mine + row * 32);
+        const uint32_t tpeer = theirs_peer + (uint32_t)((b * kLmT * 128 + row * 32) * 4);
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        mine[t * 128 + row] = lp[t];
-        st_cluster_f32(tpeer + (uint32_t)((t * 128 + row) * 4), lp[t]);
+        for (int u = 0; u < 8; ++u) {
+          const float4 v4 = make_float4(lp[4 * u], lp[4 * u + 1], lp[4 * u + 2], lp[4 * u + 3]);
+          const int cu = u ^ (row & 7);
+          mrow[cu] = v4;
+          st_cluster_v4(tpeer + (uint32_t)(cu * 16), v4);
+        }
       }
       mbar_arrive_remote(xfull_peer + b * 8);
       if (epi_any(!mbar_wait_cluster(&xfull[b], (i >> 1) & 1, a.err))) { ok = false; break; }
+      // P(i) goes into pbuf[b]: PE(i - 2) must be done with it
       if (epi_any(i >= 2 && !mbar_wait(&pe_done[b], ((i - 2) >> 1) & 1, a.err))) { ok = false; break; }
       const float* tb_ = theirs + b * kLmT * 128;
-      uint8_t* pt = pbuf + b * kF4LmPBytes;
-      int need = 0;
+      float l[32];
+      float mx = -INFINITY;
+      int ax = 0x7fffffff;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int t = tw * 8 + j;
-        const float4 x0 = *reinterpret_cast<const float4*>(mine + t * 128 + lane * 4);
-        const float4 x1 = *reinterpret_cast<const float4*>(tb_ + t * 128 + lane * 4);
-        float l[4] = {(x0.x + x1.x) * sct[j], (x0.y + x1.y) * sct[j], (x0.z + x1.z) * sct[j], (x0.w + x1.w) * sct[j]};
-        float mx = -INFINITY;
-        int ax = 0x7fffffff;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int vv = tile * 128 + lane * 4 + u;
-          if (vv >= a.V || vv == a.mask_id || t >= a.T) l[u] = -INFINITY;
-          if (l[u] > mx) { mx = l[u]; ax = vv; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const float m2 = __shfl_xor_sync(0xffffffffu, mx, o);
-          const int a2 = __shfl_xor_sync(0xffffffffu, ax, o);
-          if (m2 > mx || (m2 == mx && a2 < ax)) { mx = m2; ax = a2; }
-        }
-        if (mx > mbest[j]) { mbest[j] = mx; arg[j] = ax; }
-        float f = 1.f;
-        if (i == 0) {
-          ref[j] = mx;
-        } else if (mx > ref[j] + kLmRescale) {
-          f = expf(ref[j] - mx);
-          ref[j] = mx;
-          Z[j] *= f;
-          A[j] *= f;
-          need = 1;
-        }
-        if (lane == 0) fac[t] = f;
-        float zs = 0.f, as = 0.f;
-        __align__(8) __half hv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float p = (l[u] == -INFINITY) ? 0.f : expf(l[u] - ref[j]);
-          zs += p;
-          as += (p > 0.f) ? p * l[u] : 0.f;
-          hv[u] = __float2half_rn(t < a.T ? p * kF4PScale : 0.f);
-        }
-        *reinterpret_cast<uint2*>(pt + p16_offset(t, lane * 4)) = *reinterpret_cast<const uint2*>(hv);
-        Z[j] += warp_sum(zs);
-        A[j] += warp_sum(as);
+      for (int k = 0; k < 32; ++k) {
+        const int v = q * 32 + k, vv = tile * 128 + v;
+        const int o = v * 32 + ((((t >> 2) ^ (v & 7))) << 2) + (t & 3);
+        float x = (mine[o] + tb_[o]) * sct;
+        if (vv >= a.V || vv == a.mask_id || !live) x = -INFINITY;
+        l[k] = x;
+        if (x > mx) { mx = x; ax = vv; }
       }
+      if (mx > mbest) { mbest = mx; arg = ax; }
+      qmax[q * 32 + t] = mx;
+      epi_bar();
+      const float tmx = fmaxf(fmaxf(qmax[t], qmax[32 + t]), fmaxf(qmax[64 + t], qmax[96 + t]));
+      float f = 1.f;
+      int need = 0;
+      if (i == 0) {
+        ref = tmx;
+      } else if (tmx > ref + kLmRescale) {
+        f = expf(ref - tmx);
+        ref = tmx;
+        Z *= f;
+        A *= f;
+        need = 1;
+      }
+      if (q == 0) fac[t] = f;
+      uint32_t hw[16];
+#pragma unroll
+      for (int k = 0; k < 32; k += 2) {
+        const float p0 = (l[k] == -INFINITY) ? 0.f : expf(l[k] - ref);
+        const float p1 = (l[k + 1] == -INFINITY) ? 0.f : expf(l[k + 1] - ref);
+        Z += p0;
+        Z += p1;
+        A += (p0 > 0.f) ? p0 * l[k] : 0.f;
+        A += (p1 > 0.f) ? p1 * l[k + 1] : 0.f;
+        const __half2 h = __floats2half2_rn(p0 * kF4PScale, p1 * kF4PScale);
+        hw[k / 2] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      {  // row t of P, vocabulary 32 q .. 32 q + 31: four 16-byte chunks of atom q / 2
+        uint8_t* prow = pbuf + b * kF4LmPBytes + (q >> 1) * 4096 + t * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(prow + ((((q & 1) * 4 + j) ^ (t & 7)) << 4)) =
+              make_uint4(hw[4 * j], hw[4 * j + 1], hw[4 * j + 2], hw[4 * j + 3]);
+      }
+      // a raised reference rescales s (final up to tile i - 1: PE(i - 1) done) before PE(i)
+      // adds to it; the barrier also ends this tile's reads of mine, theirs[b] and qmax
       const bool rescale = epi_any(need != 0);
       if (rescale) {
         if (epi_any(i >= 1 && !mbar_wait(&pe_done[(i - 1) & 1], ((i - 1) >> 1) & 1, a.err))) { ok = false; break; }
         tc_fence_after();
-        float fv[32];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) fv[t] = fac[t];
         for (int ch = 0; ch < CH; ++ch) {
           float sv[32];
           const uint32_t sa = tmem + ((uint32_t)(q * 32) << 16) + kF4LmSCol + ch * kLmT;
           tmem_ld32(sa, sv);
 #pragma unroll
-          for (int t = 0; t < 32; ++t) sv[t] *= fv[t];
+          for (int u = 0; u < 32; ++u) sv[u] *= fac[u];
           tmem_st32_f(sa, sv);
         }
         tc_fence_before();
       }
-      fence_proxy_async_smem();
+      fence_proxy_async_smem();  // generic-proxy writes of P visible to the tensor cores
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_ready[b]);
     }
     if (ok && nt > 0) {
       const int last = nt - 1;
-      if (et == 0) *flag = mbar_wait(&pe_done[last & 1], (last >> 1) & 1, a.err) ? 1 : 0;
+      if (threadIdx.x == 64) *flag = mbar_wait(&pe_done[last & 1], (last >> 1) & 1, a.err) ? 1 : 0;
       epi_bar();
       ok = *flag != 0;
       epi_bar();
@@ -1015,17 +1029,29 @@ k_lmhead_fused_f4(const __grid_constant__ CUtensorMap tec, const __grid_constant
 #pragma unroll
           for (int u = 0; u < 8; ++u) dst[u] = make_float4(sv[4 * u], sv[4 * u + 1], sv[4 * u + 2], sv[4 * u + 3]);
         }
-        if (rank == 0 && lane == 0) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int t = tw * 8 + j;
-            float* ps = a.part_stats + ((size_t)clu * 32 + t) * 4;
-            ps[0] = ref[j];
-            ps[1] = Z[j];
-            ps[2] = A[j];
-            ps[3] = mbest[j];
-            a.part_arg[(size_t)clu * 32 + t] = arg[j];
+        // the quarters' statistics of token t, merged in quarter order (`mine` is free now)
+        float* ms = mine;  // [Z, A, max, argmax][quarter 4][token 32]
+        ms[(0 * 4 + q) * 32 + t] = Z;
+        ms[(1 * 4 + q) * 32 + t] = A;
+        ms[(2 * 4 + q) * 32 + t] = mbest;
+        reinterpret_cast<int*>(ms)[(3 * 4 + q) * 32 + t] = arg;
+        epi_bar();
+        if (rank == 0 && q == 0) {
+          float zs = 0.f, as = 0.f, mb = -INFINITY;
+          int ab = 0x7fffffff;
+          for (int w = 0; w < 4; ++w) {
+            zs += ms[(0 * 4 + w) * 32 + t];
+            as += ms[(1 * 4 + w) * 32 + t];
+            const float m = ms[(2 * 4 + w) * 32 + t];
+            const int am = reinterpret_cast<const int*>(ms)[(3 * 4 + w) * 32 + t];
+            if (m > mb || (m == mb && am < ab)) { mb = m; ab = am; }
           }
+          float* ps = a.part_stats + ((size_t)clu * 32 + t) * 4;
+          ps[0] = ref;
+          ps[1] = zs;
+          ps[2] = as;
+          ps[3] = mb;
+          a.part_arg[(size_t)clu * 32 + t] = ab;
         }
       }
     }

@@ -77,6 +77,9 @@ MODELS = {
     # MLP and E in NVFP4 (the format of the 4B-class NVFP4 configuration), attention in bf16
     "two_layer_gqa_nvfp4": lambda: small_model(0.06, n_layers=2, d=256, Hq=4, Hkv=2, hd=64, F=512, V=1024, B=16,
                                                fmt=1),
+    # d a multiple of 512: the LM head runs as the fused NVFP4 kernel
+    "two_layer_nvfp4_d512": lambda: small_model(0.06, n_layers=2, d=512, Hq=4, Hkv=2, hd=64, F=1024, V=1024, B=16,
+                                                fmt=1),
     # block of 32 as in the 4B-class configuration: a folded round carries 64 rows
     "gqa_b32": lambda: small_model(0.06, n_layers=2, d=256, Hq=4, Hkv=2, hd=64, F=512, V=1024, B=32, max_ctx=320),
     # FP8 KV cache (reading R13)
@@ -315,7 +318,8 @@ def compare_round(st, ost, com, new, tau, mode, k, cfg, what):
 # so most of its min-1 / top-k rankings are inside the uncertainty.
 MIN_DECIDED = {("tiny", 0): 4, ("tiny", 1): 4, ("tiny_distinct", 0): 20, ("tiny_distinct", 1): 10,
                ("two_layer_gqa", 0): 26, ("two_layer_gqa", 1): 21, ("two_layer_gqa_nvfp4", 0): 0,
-               ("two_layer_gqa_nvfp4", 1): 0, ("gqa_b32", 0): 32, ("gqa_b32", 1): 36,
+               ("two_layer_gqa_nvfp4", 1): 0, ("two_layer_nvfp4_d512", 0): 0, ("two_layer_nvfp4_d512", 1): 0,
+               ("gqa_b32", 0): 32, ("gqa_b32", 1): 36,
                ("two_layer_gqa_fp8kv", 0): 32, ("two_layer_gqa_fp8kv", 1): 20}
 
 
@@ -423,7 +427,8 @@ def test_round_lockstep(dlm, name, mode, tau, k):
     lockstep(dlm, name, mode, tau, k)
 
 
-@pytest.mark.parametrize("name", ["tiny_distinct", "two_layer_gqa", "two_layer_gqa_nvfp4", "two_layer_gqa_fp8kv"])
+@pytest.mark.parametrize("name", ["tiny_distinct", "two_layer_gqa", "two_layer_gqa_nvfp4", "two_layer_nvfp4_d512",
+                                  "two_layer_gqa_fp8kv"])
 def test_graph_decode_matches_eager_rounds(dlm, name):
     """The per-block CUDA graph (while node) and eager dlm_round calls run the same
     kernels on the same inputs: tokens, round counts and the KV cache must be identical,
