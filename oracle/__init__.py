@@ -54,6 +54,12 @@ class Model(C.Structure):
                 ("layers", C.POINTER(Layer))]
 
 
+class Moe(C.Structure):
+    _fields_ = [("n_experts", C.c_int), ("top_k", C.c_int), ("ffn_expert", C.c_int),
+                ("w_router", C.c_void_p), ("norm", C.c_void_p), ("gate", Mat), ("up", Mat),
+                ("down", Mat)]
+
+
 class KV(C.Structure):
     _fields_ = [("max_ctx", C.c_int), ("k", C.c_void_p), ("v", C.c_void_p)]
 
@@ -104,6 +110,7 @@ def lib():
         L.orc_kv_quantize_row.restype = C.c_float
         L.orc_kv_quantize_row.argtypes = [p, i, p, p]
         L.orc_lmhead.argtypes = [p, i, C.POINTER(Mat), i, i, p, C.POINTER(Stats), p, p]
+        L.orc_moe_mlp.argtypes = [p, i, i, d, C.POINTER(Moe), i, p, p, p, p, p]
         L.orc_commit.restype = i
         L.orc_commit.argtypes = [i, p, p, d, i, i, p, p]
         L.orc_forward.argtypes = [C.POINTER(Model), C.POINTER(Cfg), p, p, i, i, i,
@@ -291,6 +298,27 @@ def lmhead(x, E, mask_id=-1, p_given=None, act_fp4=False, want_logits=False):
     if want_logits:
         out["logits"] = logits
     return out
+
+
+def moe_mlp(h_in, moe, eps=1e-6, act_fp4=True):
+    """Routed-expert MLP sub-block (R14).  h_in [T][d]; moe: dict(n_experts, top_k,
+    ffn_expert, w_router (bf16 bits [E][d]), norm (bf16 bits [d]), gate, up ([E F][d]) and
+    down ([d][E F]) as bf16 bits or NVFP4 dicts).  Returns dict(h_out, logits [T][E],
+    idx [T][k], w [T][k], qmargin [T])."""
+    h = _c(h_in, np.float64)
+    T, d = h.shape
+    E, k, F = int(moe["n_experts"]), int(moe["top_k"]), int(moe["ffn_expert"])
+    wk = Weights()
+    m = Moe(E, k, F, wk.vec(moe["w_router"]), wk.vec(moe["norm"]), wk.mat(moe["gate"]),
+            wk.mat(moe["up"]), wk.mat(moe["down"]))
+    out = np.zeros_like(h)
+    logits = np.zeros((T, E), np.float64)
+    idx = np.zeros((T, k), np.int32)
+    w = np.zeros((T, k), np.float64)
+    qm = np.zeros(T, np.float64)
+    lib().orc_moe_mlp(_ptr(h), T, d, float(eps), C.byref(m), int(act_fp4), _ptr(out), _ptr(logits),
+                      _ptr(idx), _ptr(w), _ptr(qm))
+    return {"h_out": out, "logits": logits, "idx": idx, "w": w, "qmargin": qm}
 
 
 def commit(maxprob, argmax, tau, mode, k, tokens, committed):

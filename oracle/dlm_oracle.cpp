@@ -56,6 +56,19 @@
 //      position) is stored as OCP e4m3 codes with one fp32 scale s = amax(|row|) / 448, code =
 //      RNE_e4m3(x / s) saturating at 448, value = e4m3(code) * s.  q stays bf16 (R9); the K
 //      and V rows are quantized from their unrounded values.
+//   R14 routed-expert MLP ([blog] "What shipped", "dlmrt, the inference engine": routed
+//      experts run NVFP4 on FP4 tensor cores; the pages give neither the routing rule nor
+//      the expert shapes, so this is the plainest reading): x = RMSNorm(h) g; router logits
+//      l = x W_r^T (W_r bf16 [E][d]); p = softmax(l) over the E experts; the k experts of
+//      largest p are selected (ties to the lower index) with weights w_e = p_e / sum of the
+//      selected p; every expert is a SiLU-gated MLP (gate, up [F][d], down [d][F]) and the
+//      sub-block adds h += sum_e w_e down_e(silu(gate_e x) * up_e x).  The experts' gate and
+//      up matrices are stacked along rows ([E F][d], expert e in rows [e F, (e + 1) F)) and
+//      their down matrices side by side along columns ([d][E F]), one NVFP4 tensor scale
+//      each; the activation row entering the down projection is the concatenation over the
+//      experts of w_e silu(.) * up(.) (zeros for the experts not selected), quantized per
+//      row like every NVFP4 GEMM input (R8), so the weighted sum over the experts is one
+//      contraction over E F.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -511,6 +524,71 @@ void orc_rowstats(const double* logits, int B, int V, int mask_id, orc_stats* st
     st[b].entropy = H;
     st[b].argmax = am;
   }
+}
+
+// Routed-expert MLP sub-block (R14).  h_in, h_out [T][d]; logits [T][E] (optional);
+// topk_idx, topk_w [T][k]; qmargin [T] (optional, act_fp4 only: the smallest distance of an
+// activation to a quantization decision boundary, as orc_lmhead reports it).
+typedef struct orc_moe {
+  int n_experts, top_k, ffn_expert;
+  const uint16_t* w_router;  // bf16 [E][d]
+  const uint16_t* norm;      // bf16 [d]
+  orc_mat gate, up;          // [E F][d]
+  orc_mat down;              // [d][E F]
+} orc_moe;
+
+void orc_moe_mlp(const double* h_in, int T, int d, double eps, const orc_moe* M, int act_fp4, double* h_out,
+                 double* logits_out, int* topk_idx, double* topk_w, double* qmargin) {
+  const int E = M->n_experts, k = M->top_k, F = M->ffn_expert, EF = E * F;
+  const bool fp4 = act_fp4 != 0;
+  std::vector<double> x(size_t(T) * d), l(size_t(T) * E), sel_w(size_t(T) * E, 0.0);
+  std::vector<double> qm(T, std::numeric_limits<double>::infinity());
+  for (int t = 0; t < T; ++t) rmsnorm(h_in + size_t(t) * d, d, M->norm, eps, x.data() + size_t(t) * d);
+  for (int t = 0; t < T; ++t) {
+    // router logits and softmax over all experts
+    double mx = -std::numeric_limits<double>::infinity();
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int c = 0; c < d; ++c) acc += x[size_t(t) * d + c] * bf16_to_double(M->w_router[size_t(e) * d + c]);
+      l[size_t(t) * E + e] = acc;
+      mx = std::max(mx, acc);
+    }
+    std::vector<double> p(E);
+    double z = 0.0;
+    for (int e = 0; e < E; ++e) z += (p[e] = std::exp(l[size_t(t) * E + e] - mx));
+    for (int e = 0; e < E; ++e) p[e] /= z;
+    // top-k by probability, ties to the lower index; weights renormalised over the chosen
+    std::vector<uint8_t> taken(E, 0);
+    double zs = 0.0;
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      for (int e = 0; e < E; ++e)
+        if (!taken[e] && (best < 0 || p[e] > p[best])) best = e;
+      taken[best] = 1;
+      topk_idx[size_t(t) * k + j] = best;
+      zs += p[best];
+    }
+    for (int j = 0; j < k; ++j) {
+      const int e = topk_idx[size_t(t) * k + j];
+      topk_w[size_t(t) * k + j] = p[e] / zs;
+      sel_w[size_t(t) * E + e] = p[e] / zs;
+    }
+  }
+  if (logits_out) std::memcpy(logits_out, l.data(), l.size() * sizeof(double));
+  // every expert on every row (the ones not selected get weight 0 below)
+  std::vector<double> g(size_t(T) * EF), u(size_t(T) * EF), a(size_t(T) * EF), y(size_t(T) * d);
+  linear(x.data(), T, M->gate, g.data(), fp4, qm.data());
+  linear(x.data(), T, M->up, u.data(), fp4, qm.data());
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < EF; ++j) {
+      const size_t i = size_t(t) * EF + j;
+      const double w = sel_w[size_t(t) * E + j / F];
+      a[i] = (w == 0.0) ? 0.0 : w * (g[i] / (1.0 + std::exp(-g[i]))) * u[i];
+    }
+  linear(a.data(), T, M->down, y.data(), fp4, qm.data());
+  for (size_t i = 0; i < y.size(); ++i) h_out[i] = h_in[i] + y[i];
+  if (qmargin)
+    for (int t = 0; t < T; ++t) qmargin[t] = qm[t];
 }
 
 // Fused-LM-head semantics, computed plainly: logits = x E^T (x already normalised),

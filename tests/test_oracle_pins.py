@@ -731,3 +731,108 @@ def test_pin_kv_fp8_applies_to_k_and_v_rows_only(tiny):
         e = np.exp(sc - sc.max())
         o.append(e @ V / e.sum())
     np.testing.assert_allclose(xf[0], _rms(E[tok] + np.concatenate(o), gf, eps), rtol=1e-11, atol=1e-13)
+
+
+# ------------------------------------------------------------------ routed-expert MLP (R14)
+def _bits_f32(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _moe(E, k, F, d, seed, router_std=0.3, w_std=0.2, fp4=False):
+    rng = np.random.default_rng(seed)
+    gate = gen.bf16_bits(rng.normal(0, w_std, (E * F, d)))
+    up = gen.bf16_bits(rng.normal(0, w_std, (E * F, d)))
+    down = gen.bf16_bits(rng.normal(0, w_std, (d, E * F)))
+    if fp4:
+        def q(w):
+            c, s, S = O.nvfp4_quantize(_bits_f32(w))
+            return {"codes": c, "scales": s, "tscale": S, "rows": w.shape[0], "cols": w.shape[1]}
+        gate, up, down = q(gate), q(up), q(down)
+    return dict(n_experts=E, top_k=k, ffn_expert=F, w_router=gen.bf16_bits(rng.normal(0, router_std, (E, d))),
+                norm=gen.bf16_bits(np.ones(d)), gate=gate, up=up, down=down)
+
+
+def test_pin_moe_uniform_router_takes_the_lowest_indices_with_equal_weights():
+    """All router logits equal (W_r = 0): every expert has probability 1/E, so the top-k rule
+    with ties to the lower index selects experts 0..k-1, each with weight 1/k."""
+    moe = _moe(6, 3, 16, 32, seed=1)
+    moe["w_router"] = np.zeros_like(moe["w_router"])
+    r = O.moe_mlp(np.random.default_rng(2).normal(0, 1, (4, 32)), moe, act_fp4=False)
+    assert np.array_equal(r["idx"], np.tile(np.arange(3, dtype=np.int32), (4, 1)))
+    np.testing.assert_array_equal(r["w"], np.full((4, 3), 1.0 / 3.0))
+    np.testing.assert_array_equal(r["logits"], 0.0)
+
+
+def test_pin_moe_expert_permutation_invariance():
+    """Relabelling the experts (router rows, gate/up row blocks and down column blocks
+    permuted together) leaves the output unchanged and maps the selections through the
+    permutation: catches an expert slice or a router row read at the wrong index."""
+    E, k, F, d, T = 5, 2, 16, 32, 6
+    moe = _moe(E, k, F, d, seed=3)
+    h = np.random.default_rng(4).normal(0, 1, (T, d))
+    perm = np.array([3, 0, 4, 1, 2])
+    pm = dict(moe)
+    pm["w_router"] = moe["w_router"][perm]
+    rows = np.concatenate([np.arange(e * F, (e + 1) * F) for e in perm])
+    pm["gate"] = moe["gate"][rows]
+    pm["up"] = moe["up"][rows]
+    pm["down"] = moe["down"][:, rows]
+    a = O.moe_mlp(h, moe, act_fp4=False)
+    b = O.moe_mlp(h, pm, act_fp4=False)
+    np.testing.assert_allclose(b["h_out"], a["h_out"], rtol=1e-12, atol=1e-12)
+    # new expert j is old expert perm[j]
+    assert np.array_equal(perm[b["idx"]], a["idx"])
+    np.testing.assert_allclose(b["w"], a["w"], rtol=1e-12)
+
+
+def test_pin_moe_scaled_identity_experts_closed_form():
+    """Experts G_e = a_e I, U_e = b_e I, D_e = c_e I (d = F, bf16-exact scalars) make every
+    expert elementwise: out = h + sum_e w_e c_e silu(a_e x) b_e x with x = RMSNorm(h).  With a
+    router that puts one expert far ahead (k = 1) the weight is exactly 1; with W_r = 0 and
+    k = 2 the weights are 1/2 on experts 0 and 1."""
+    E, d = 3, 16
+    a = np.array([0.5, 1.0, 2.0])
+    b = np.array([1.0, -0.5, 0.25])
+    c = np.array([2.0, 1.0, -1.0])
+    I = np.eye(d)
+    gate = gen.bf16_bits(np.concatenate([a[e] * I for e in range(E)]))
+    up = gen.bf16_bits(np.concatenate([b[e] * I for e in range(E)]))
+    down = gen.bf16_bits(np.concatenate([c[e] * I for e in range(E)], axis=1))
+    h = np.random.default_rng(5).normal(0, 1, (2, d))
+    x = h / np.sqrt(np.mean(h ** 2, axis=1, keepdims=True) + 1e-6)
+    silu = lambda v: v / (1.0 + np.exp(-v))
+    # router: expert 2 far ahead for every row (logit 8 * sum(x) with x summed ... use a
+    # router row of +1 on coordinate 0 scaled by the sign of x_0 so its logit is large)
+    wr = np.zeros((E, d))
+    for_row = np.sign(x[:, 0])
+    assert np.all(for_row == for_row[0])
+    wr[2, 0] = 64.0 * for_row[0]
+    moe = dict(n_experts=E, top_k=1, ffn_expert=d, w_router=gen.bf16_bits(wr), norm=gen.bf16_bits(np.ones(d)),
+               gate=gate, up=up, down=down)
+    r = O.moe_mlp(h, moe, act_fp4=False)
+    assert np.array_equal(r["idx"][:, 0], [2, 2])
+    np.testing.assert_array_equal(r["w"], 1.0)
+    want = h + c[2] * silu(a[2] * x) * b[2] * x
+    np.testing.assert_allclose(r["h_out"], want, rtol=1e-12, atol=1e-12)
+    moe["w_router"] = gen.bf16_bits(np.zeros((E, d)))
+    moe["top_k"] = 2
+    r = O.moe_mlp(h, moe, act_fp4=False)
+    want = h + 0.5 * sum(c[e] * silu(a[e] * x) * b[e] * x for e in (0, 1))
+    np.testing.assert_allclose(r["h_out"], want, rtol=1e-12, atol=1e-12)
+
+
+def test_pin_moe_single_expert_nvfp4_is_the_dense_mlp():
+    """E = k = 1 with NVFP4 weights: the weight is exactly 1, so the sub-block is the dense
+    NVFP4 MLP built from the pinned linear (each input row quantized, R8):
+    h + Q(silu(Q(x) G^T) * Q(x) U^T) D^T."""
+    F, d = 64, 64
+    moe = _moe(1, 1, F, d, seed=6, fp4=True)
+    h = np.random.default_rng(7).normal(0, 1, (5, d))
+    r = O.moe_mlp(h, moe, act_fp4=True)
+    x = O.rmsnorm(h, moe["norm"], 1e-6)
+    g = O.linear(x, moe["gate"], act_fp4=True)
+    u = O.linear(x, moe["up"], act_fp4=True)
+    act = g / (1.0 + np.exp(-g)) * u
+    want = h + O.linear(act, moe["down"], act_fp4=True)
+    np.testing.assert_allclose(r["h_out"], want, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(r["w"], 1.0)
