@@ -45,7 +45,7 @@ def parse(argv=None):
     # profiling cases (small, for ncu): "quick" = the decode loop on 256 generated tokens
     # without the extra measurements; "gemm" = every projection GEMM of two layers plus
     # the LM-head GEMM, `--steps` launches each
-    ap.add_argument("--case", default="full", choices=["full", "quick", "gemm", "lmhead", "attention"])
+    ap.add_argument("--case", default="full", choices=["full", "quick", "gemm", "lmhead", "attention", "moe"])
     # the quick case with eager dlm_round / dlm_kv_fill calls instead of the block graph
     # (same kernels; ncu cannot profile kernel nodes of graphs with conditional nodes)
     ap.add_argument("--eager", action="store_true")
@@ -678,6 +678,46 @@ def lmhead_case(args):
                       "peak": hbm, "peak_kind": kind}), flush=True)
 
 
+def moe_case(args):
+    """Routed-expert MLP sub-block with NVFP4 experts (dlm_moe_mlp_nvfp4) on a synthetic layer
+    at the 4B-class width: d 2560, 64 experts of F 512, top-4, 32 rows, random router and
+    expert weights (quantized on the device), L2 flushed before every call.  Algorithmic
+    bytes: every expert's gate, up and down codes and scales (all are streamed) plus the
+    router (bf16)."""
+    import ctypes as C
+
+    import torch
+
+    from block_diffusion_decoding_denoising_b200 import build, dlm, gen
+    build.build()
+    dev = torch.device("cuda", 0)
+    E, k, F, d, T = 64, 4, 512, 2560, 32
+    g = torch.Generator(device=dev).manual_seed(5)
+    wr = (torch.randn((E, d), device=dev, generator=g) * 0.02).to(torch.bfloat16)
+    norm = torch.ones(d, device=dev, dtype=torch.bfloat16)
+    mk = lambda r, c: dlm.nvfp4_matrix((torch.randn((r, c), device=dev, generator=g) * 0.02).to(torch.bfloat16))
+    qg, qu, qd = mk(E * F, d), mk(E * F, d), mk(d, E * F)
+    m = dlm.Moe(E, k, F, d, wr, norm, qg, qu, qd)
+    h = torch.randn((T, d), device=dev, generator=g)
+    fn = lambda: m(h)
+    for _ in range(max(args.warmup, 3)):
+        fn()
+    torch.cuda.synchronize()
+    flush = _l2_flusher(dev)
+    t = _timed_calls(fn, max(args.steps, 5), flush)
+    _, idx, _ = m(h)
+    active = int(torch.unique(idx).numel())
+    hbm, _, kind = peaks()
+    nbytes = 3 * E * F * d // 2 + 3 * E * F * d // 16 + E * d * 2 + 2 * T * d * 4
+    gbs = nbytes / t / 1e9
+    print(json.dumps({"case": "moe", "workload": "routed-expert MLP, NVFP4 experts: d %d, %d experts of F %d, top-%d, "
+                      "%d rows" % (d, E, F, k, T), "us_per_call": t * 1e6, "algorithmic_bytes": nbytes,
+                      "GBs": gbs, "frac": gbs / hbm, "peak": hbm, "peak_kind": kind, "experts_chosen": active,
+                      "l2": "flushed (256 MB written) before every call",
+                      "note": "per call: routing, activation quantizers, two FP4 GEMMs and their finishers"}),
+          flush=True)
+
+
 def main():
     global GEN
     args = parse()
@@ -690,6 +730,9 @@ def main():
         return
     if args.case == "attention":
         attention_case(args)
+        return
+    if args.case == "moe":
+        moe_case(args)
         return
     if args.case == "quick":
         GEN = 256

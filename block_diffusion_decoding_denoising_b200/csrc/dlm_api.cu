@@ -1476,6 +1476,146 @@ dlm_status dlm_lmhead_rowstats_nvfp4(const float* d_x, const dlm_nvfp4_matrix* E
   return DLM_OK;
 }
 
+static bool moe_shape_ok(int d, const dlm_moe_weights* w) {
+  if (!w) return false;
+  const long EF = (long)w->n_experts * w->ffn_expert;
+  return w->n_experts >= 1 && w->n_experts <= 256 && w->top_k >= 1 && w->top_k <= 8 &&
+         w->top_k <= w->n_experts && w->ffn_expert >= 64 && w->ffn_expert % 64 == 0 && EF % 256 == 0 &&
+         EF <= 65536 && d >= 256 && d % 256 == 0 && d <= 8192;
+}
+static size_t moe_tile_bytes_pair(int d, const dlm_moe_weights* w) {
+  return align256(nvf4_sf_tile_bytes(w->n_experts * w->ffn_expert, d, A_PAIR));
+}
+
+size_t dlm_moe_prepare_size(int d, const dlm_moe_weights* w) {
+  if (!moe_shape_ok(d, w)) return 0;
+  const int EF = w->n_experts * w->ffn_expert;
+  return moe_tile_bytes_pair(d, w) + align256(nvf4_sf_tile_bytes(d, EF, A_KMAJOR));
+}
+
+dlm_status dlm_moe_prepare(int d, const dlm_moe_weights* w, void* d_tiles, size_t bytes, void* stream) {
+  dlm_ctx* ctx = nullptr;
+  if (!w || !d_tiles || !w->q_gate.scales || !w->q_up.scales || !w->q_down.scales) return DLM_EINVAL;
+  if (!moe_shape_ok(d, w)) return DLM_EUNSUPPORTED;
+  if (bytes < dlm_moe_prepare_size(d, w)) return DLM_ENOMEM_WS;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int EF = w->n_experts * w->ffn_expert;
+  uint8_t* base = (uint8_t*)d_tiles;
+  CU(nvf4_sf_tile(w->q_gate, &w->q_up, EF, d, A_PAIR, base, s));
+  CU(nvf4_sf_tile(w->q_down, nullptr, d, EF, A_KMAJOR, base + moe_tile_bytes_pair(d, w), s));
+  return DLM_OK;
+}
+
+static size_t moe_partial_bytes(int T, int d, int EF) {
+  const size_t a = gemm_fp4_partial_bytes(T, EF, d, A_PAIR), b = gemm_fp4_partial_bytes(T, d, EF, A_KMAJOR);
+  return a > b ? a : b;
+}
+
+size_t dlm_moe_scratch_size(int T, int d, const dlm_moe_weights* w) {
+  if (T < 1 || T > kMaxF4Tokens || !moe_shape_ok(d, w)) return 0;
+  const int E = w->n_experts, EF = E * w->ffn_expert, K = EF > d ? EF : d;
+  return op_header() + op_counters(K) + align256(moe_partial_bytes(T, d, EF)) +
+         align256((size_t)kMaxF4Tokens * K / 2) + align256((size_t)K / 64 * 512) + align256(kMaxF4Tokens * 4) +
+         align256((size_t)T * d * 4) + 2 * align256((size_t)T * E * 4) + 2 * align256((size_t)T * EF * 2) +
+         align256((size_t)(EF / 64) * T * 4);
+}
+
+dlm_status dlm_moe_mlp_nvfp4(const float* d_h_in, float* d_h_out, int T, int d, float rms_eps,
+                             const dlm_moe_weights* w, const void* d_tiles, int32_t* d_topk_idx, float* d_topk_w,
+                             void* d_scratch, size_t scratch_bytes, void* stream) {
+  dlm_ctx* ctx = nullptr;
+  if (!d_h_in || !d_h_out || d_h_in == d_h_out || !w || !d_tiles || !d_scratch || !w->w_router ||
+      !w->mlp_norm || !w->q_gate.codes || !w->q_up.codes || !w->q_down.codes || !std::isfinite(rms_eps) ||
+      T < 1 || !std::isfinite(w->q_gate.tensor_scale) || !std::isfinite(w->q_up.tensor_scale) ||
+      !std::isfinite(w->q_down.tensor_scale))
+    return DLM_EINVAL;
+  if (T > kMaxF4Tokens || !moe_shape_ok(d, w)) return DLM_EUNSUPPORTED;
+  if (scratch_bytes < dlm_moe_scratch_size(T, d, w)) return DLM_ENOMEM_WS;
+  CU((cudaError_t)gemm_fp4_init_attributes());
+  cudaStream_t s = (cudaStream_t)stream;
+  const int E = w->n_experts, F = w->ffn_expert, EF = E * F, K = EF > d ? EF : d;
+  OpScratch sc(d_scratch, K, moe_partial_bytes(T, d, EF));
+  uint8_t* xcodes = sc.take<uint8_t>((size_t)kMaxF4Tokens * K / 2);
+  uint8_t* xscales = sc.take<uint8_t>((size_t)K / 64 * 512);
+  float* sx = sc.take<float>(kMaxF4Tokens);
+  float* x = sc.take<float>((size_t)T * d);
+  float* logits = sc.take<float>((size_t)T * E);
+  float* route_w = sc.take<float>((size_t)T * E);
+  __nv_bfloat16* act = sc.take<__nv_bfloat16>((size_t)2 * T * EF);  // high halves, then low halves
+  float* act_amax = sc.take<float>((size_t)(EF / 64) * T);
+  // the status word, and the token codes and scales of the rows past T (read by the MMA,
+  // their columns dropped), start at zero
+  CU(cudaMemsetAsync(d_scratch, 0, op_header(), s));
+  CU(cudaMemsetAsync(xcodes, 0, (size_t)kMaxF4Tokens * K / 2, s));
+  CU(cudaMemsetAsync(xscales, 0, (size_t)K / 64 * 512, s));
+  MoeRouteArgs ra{};
+  ra.h = d_h_in;
+  ra.g = (const __nv_bfloat16*)w->mlp_norm;
+  ra.wr = (const __nv_bfloat16*)w->w_router;
+  ra.eps = rms_eps;
+  ra.T = T;
+  ra.d = d;
+  ra.E = E;
+  ra.k = w->top_k;
+  ra.x = x;
+  ra.logits = logits;
+  ra.route_w = route_w;
+  ra.topk_idx = d_topk_idx;
+  ra.topk_w = d_topk_w;
+  CU_LAUNCH(launch_k(k_moe_route, dim3(T), dim3(256), (d + E) * 4, s, ra));
+  ActQuantArgs q{};
+  q.xf = x;
+  q.K = d;
+  q.codes = xcodes;
+  q.scales = xscales;
+  q.sx = sx;
+  CU_LAUNCH(launch_k(k_act_quant, dim3(T), dim3(256), 0, s, q));
+  const uint8_t* tiles = (const uint8_t*)d_tiles;
+  char msg[256];
+  GemmF4Plan p;
+  // every expert's gate/up rows on every row of x
+  if (!gemm_fp4_plan(&p, A_PAIR, w->q_gate, &w->q_up, tiles, xcodes, xscales, kMaxF4Tokens, sx, T, EF, d, sc.partial,
+                     msg, sizeof(msg)))
+    return DLM_EUNSUPPORTED;
+  CU(gemm_fp4_launch(p, sc.err, s));
+  EpiArgs es{};
+  es.op = EPI_SILU;
+  es.act = act;
+  es.act_lo = (long)T * EF;
+  es.act_amax = act_amax;
+  es.route_w = route_w;
+  es.route_e = E;
+  es.route_f = F;
+  {
+    FinishArgs fa{p.out, es, EF};
+    CU_LAUNCH(launch_k(k_finish_silu, dim3(p.out.n_tiles, (T + 31) / 32), dim3(256), 0, s, fa));
+  }
+  // the weighted expert activations, one row of E F per token, quantized per row
+  ActQuantArgs qa{};
+  qa.xb = act;
+  qa.xb_lo = (long)T * EF;
+  qa.K = EF;
+  qa.codes = xcodes;
+  qa.scales = xscales;
+  qa.sx = sx;
+  qa.amax = act_amax;
+  qa.n_amax = EF / 64;
+  qa.T = T;
+  CU_LAUNCH(launch_k(k_act_quant_wide, dim3((unsigned)((EF / 16 + 255) / 256), T), dim3(256), 0, s, qa));
+  if (!gemm_fp4_plan(&p, A_KMAJOR, w->q_down, nullptr, tiles + moe_tile_bytes_pair(d, w), xcodes, xscales,
+                     kMaxF4Tokens, sx, T, d, EF, sc.partial, msg, sizeof(msg)))
+    return DLM_EUNSUPPORTED;
+  CU(gemm_fp4_launch(p, sc.err, s));
+  EpiArgs eo{};
+  eo.op = EPI_STORE;
+  eo.out = d_h_out;
+  eo.ld = d;
+  eo.add = d_h_in;
+  FinishArgs fo{p.out, eo, d};
+  CU_LAUNCH(launch_k(k_finish_store, dim3(p.out.n_tiles, (T + 31) / 32), dim3(256), 0, s, fo));
+  return DLM_OK;
+}
+
 size_t dlm_gemm_nvfp4_scratch_size(int T, int N, int K) {
   if (T < 1 || T > kMaxF4Tokens || N < 1 || K < 256 || K % 256 || K > 16384) return 0;
   return op_header() + op_counters(N) + align256(gemm_fp4_partial_bytes(T, N, K, A_KMAJOR)) +

@@ -126,6 +126,9 @@ struct EpiArgs {
   __nv_bfloat16* act;           // EPI_SILU: [T][F] high halves
   long act_lo;
   float* act_amax;              // EPI_SILU (optional): [F / 64][T] amax of each tile's stored values
+  const float* route_w;         // EPI_SILU (optional): act[t][f] *= route_w[t][f / route_f] (routed experts)
+  int route_e, route_f;         //   experts per row of route_w, features per expert
+  const float* add;             // EPI_STORE (optional): out = add + y (same layout as out)
 };
 
 struct GemmPlan {

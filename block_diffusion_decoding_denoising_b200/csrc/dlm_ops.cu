@@ -190,7 +190,8 @@ __global__ void __launch_bounds__(256) k_finish_silu(FinishArgs a) {
   for (int j = 0; j < kFinTok; ++j) {
     am[j] = 0.f;
     if (active && t0 + j < a.out.T) {
-      const float v = g[j] / (1.0f + expf(-g[j])) * u[j];
+      float v = g[j] / (1.0f + expf(-g[j])) * u[j];
+      if (e.route_w) v *= e.route_w[(size_t)(t0 + j) * e.route_e + f / e.route_f];
       __nv_bfloat16* p = e.act + (size_t)(t0 + j) * a.N + f;
       store_split(p, e.act_lo, v);
       if (e.act_amax) {
@@ -214,6 +215,88 @@ __global__ void __launch_bounds__(256) k_finish_silu(FinishArgs a) {
 }
 
 // out[t][n] = scale * y (scale 0 means 1), rows r and r + 64 of the tile per thread.
+// Routed-expert MLP front (one CTA per token row): x = h / sqrt(mean(h^2) + eps) g, router
+// logits l_e = x . W_r[e] (fp32, W_r bf16), then warp 0 picks the k largest logits (ties to
+// the lower index) and weights them by softmax renormalised over the chosen:
+// w_e = exp(l_e - m) / sum_chosen exp(l_j - m).  route_w gets the weights densely (zero for
+// the experts not chosen).
+__global__ void __launch_bounds__(256) k_moe_route(MoeRouteArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ float msm[];  // x [d] | logits [E]
+  __shared__ float red[8];
+  const int t = blockIdx.x, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const float* h = a.h + (size_t)t * a.d;
+  float ss = 0.f;
+  for (int c = tid; c < a.d; c += 256) ss += h[c] * h[c];
+  ss = warp_sum(ss);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += red[w];
+  const float r = 1.0f / sqrtf(tot / (float)a.d + a.eps);
+  float* sx = msm;
+  float* sl = msm + a.d;
+  for (int c = tid; c < a.d; c += 256) {
+    const float xv = h[c] * r * bf2f(a.g[c]);
+    sx[c] = xv;
+    a.x[(size_t)t * a.d + c] = xv;
+  }
+  __syncthreads();
+  for (int e = warp; e < a.E; e += 8) {
+    const __nv_bfloat16* wr = a.wr + (size_t)e * a.d;
+    float acc = 0.f;
+    for (int c0 = lane * 8; c0 < a.d; c0 += 256) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(wr + c0);
+      const __nv_bfloat16* wv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc += sx[c0 + u] * bf2f(wv[u]);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) {
+      sl[e] = acc;
+      if (a.logits) a.logits[(size_t)t * a.E + e] = acc;
+    }
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  // lane owns experts lane + 32 j (j < 8, E <= 256)
+  float mx = -INFINITY;
+  for (int e = lane; e < a.E; e += 32) mx = fmaxf(mx, sl[e]);
+  mx = warp_max(mx);
+  uint32_t taken = 0;
+  float zs = 0.f, pw[8];
+  int pi[8];
+  for (int s = 0; s < a.k; ++s) {
+    float best = -INFINITY;
+    int be = 0x7fffffff;
+    for (int j = 0; lane + 32 * j < a.E; ++j) {
+      const int e = lane + 32 * j;
+      if (!((taken >> j) & 1u) && (sl[e] > best || (sl[e] == best && e < be))) { best = sl[e]; be = e; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float b2 = __shfl_xor_sync(0xffffffffu, best, o);
+      const int e2 = __shfl_xor_sync(0xffffffffu, be, o);
+      if (b2 > best || (b2 == best && e2 < be)) { best = b2; be = e2; }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    pi[s] = be;
+    pw[s] = expf(best - mx);
+    zs += pw[s];
+  }
+  for (int e = lane; e < a.E; e += 32) a.route_w[(size_t)t * a.E + e] = 0.f;
+  __syncwarp();
+  if (lane == 0)
+    for (int s = 0; s < a.k; ++s) {
+      const float w = pw[s] / zs;
+      a.route_w[(size_t)t * a.E + pi[s]] = w;
+      if (a.topk_idx) a.topk_idx[(size_t)t * a.k + s] = pi[s];
+      if (a.topk_w) a.topk_w[(size_t)t * a.k + s] = w;
+    }
+}
+
 __global__ void __launch_bounds__(256) k_finish_store(FinishArgs a) {
   pdl_trigger();
   pdl_wait();
@@ -228,8 +311,9 @@ __global__ void __launch_bounds__(256) k_finish_store(FinishArgs a) {
 #pragma unroll
   for (int j = 0; j < kFinTok; ++j) {
     if (t0 + j < a.out.T) {
-      if (na < a.N) e.out[(size_t)(t0 + j) * e.ld + na] = (e.scale != 0.f) ? va[j] * sc : va[j];
-      if (nb < a.N) e.out[(size_t)(t0 + j) * e.ld + nb] = (e.scale != 0.f) ? vb[j] * sc : vb[j];
+      const size_t ia = (size_t)(t0 + j) * e.ld + na, ib = (size_t)(t0 + j) * e.ld + nb;
+      if (na < a.N) e.out[ia] = ((e.scale != 0.f) ? va[j] * sc : va[j]) + (e.add ? e.add[ia] : 0.f);
+      if (nb < a.N) e.out[ib] = ((e.scale != 0.f) ? vb[j] * sc : vb[j]) + (e.add ? e.add[ib] : 0.f);
     }
   }
 }

@@ -51,6 +51,19 @@ struct RowStatsArgs {
 // per 16 elements and e2m1 codes (codes[t][K/2], element 2j in the low nibble).  The
 // scales are written in the FP4 MMA's copy layout: byte (b / 4) * 512 + t * 16 + b % 4 holds
 // the scale of group b (tokens t < 32; the other 12 bytes of each 16 are not used).
+struct MoeRouteArgs {
+  const float* h;            // [T][d] residual rows
+  const __nv_bfloat16* g;    // [d] RMSNorm gain
+  const __nv_bfloat16* wr;   // [E][d] router
+  float eps;
+  int T, d, E, k;            // E <= 256, k <= 8, d % 8 == 0
+  float* x;                  // [T][d] normalised rows
+  float* logits;             // [T][E] (optional)
+  float* route_w;            // [T][E] weights, zero for the experts not chosen
+  int* topk_idx;             // [T][k] (optional)
+  float* topk_w;             // [T][k] (optional)
+};
+
 struct ActQuantArgs {
   const float* xf;
   const __nv_bfloat16* xb;
@@ -109,6 +122,7 @@ struct BlockFinishArgs {
 __global__ void k_finish_qkv(FinishArgs a);
 __global__ void k_finish_silu(FinishArgs a);
 __global__ void k_finish_store(FinishArgs a);
+__global__ void k_moe_route(MoeRouteArgs a);
 __global__ void k_resid_norm(ResNormArgs a);
 __global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo, long zero_n);
 __global__ void k_rowstats_part(RowStatsArgs a);

@@ -44,6 +44,12 @@ class Nvfp4Matrix(C.Structure):
     _fields_ = [("codes", C.c_void_p), ("scales", C.c_void_p), ("tensor_scale", C.c_float)]
 
 
+class MoeWeights(C.Structure):
+    _fields_ = [("n_experts", C.c_int), ("top_k", C.c_int), ("ffn_expert", C.c_int),
+                ("w_router", C.c_void_p), ("mlp_norm", C.c_void_p), ("q_gate", Nvfp4Matrix),
+                ("q_up", Nvfp4Matrix), ("q_down", Nvfp4Matrix)]
+
+
 class LayerWeights(C.Structure):
     _fields_ = [("attn_norm", C.c_void_p), ("w_qkv", C.c_void_p), ("w_o", C.c_void_p),
                 ("mlp_norm", C.c_void_p), ("w_gate", C.c_void_p), ("w_up", C.c_void_p),
@@ -123,6 +129,12 @@ def lib():
         L.dlm_bd_attention_fp8.argtypes = [p, p, p, p, p, p, i, i, i, i, i, i, i, p, z, p]
         L.dlm_commit.argtypes = [p, p, p, p, p, p, p, i, i, f, i, i, p]
         L.dlm_nvfp4_quantize.argtypes = [p, i, i, p, p, p, p]
+        L.dlm_moe_prepare_size.restype = z
+        L.dlm_moe_prepare_size.argtypes = [i, C.POINTER(MoeWeights)]
+        L.dlm_moe_prepare.argtypes = [i, C.POINTER(MoeWeights), p, z, p]
+        L.dlm_moe_scratch_size.restype = z
+        L.dlm_moe_scratch_size.argtypes = [i, i, C.POINTER(MoeWeights)]
+        L.dlm_moe_mlp_nvfp4.argtypes = [p, p, i, i, f, C.POINTER(MoeWeights), p, p, p, p, z, p]
         L.dlm_lmhead_nvfp4_scratch_size.restype = z
         L.dlm_lmhead_nvfp4_scratch_size.argtypes = [i, i, i]
         L.dlm_lmhead_rowstats_nvfp4.argtypes = [p, C.POINTER(Nvfp4Matrix), i, i, i, i, RowStats, p, p, z, p]
@@ -238,6 +250,41 @@ def lmhead_rowstats_nvfp4(x, Eq, mask_id=-1, stream=None):
                                            _ptr(sc), n, _stream(stream)))
     st["s"] = s
     return st
+
+
+class Moe:
+    """A routed-expert MLP sub-block on the device: router bf16 [E][d], norm gain bf16 [d],
+    and the experts' NVFP4 stacks gate, up [E F][d] and down [d][E F] (dicts as
+    nvfp4_matrix returns), with their scales re-tiled once (dlm_moe_prepare)."""
+
+    def __init__(self, n_experts, top_k, ffn_expert, d, w_router, mlp_norm, q_gate, q_up, q_down, stream=None):
+        import torch
+        self.d = d
+        self._keep = [w_router, mlp_norm, q_gate, q_up, q_down]
+        self.w = MoeWeights(n_experts, top_k, ffn_expert, _ptr(w_router).value, _ptr(mlp_norm).value,
+                            _q_matrix(q_gate), _q_matrix(q_up), _q_matrix(q_down))
+        n = lib().dlm_moe_prepare_size(d, C.byref(self.w))
+        if n == 0:
+            raise DlmError(DLM_EUNSUPPORTED, "moe: unsupported shape E=%d k=%d F=%d d=%d" %
+                           (n_experts, top_k, ffn_expert, d))
+        self.tiles = torch.empty(n, dtype=torch.uint8, device=w_router.device)
+        _check(lib().dlm_moe_prepare(d, C.byref(self.w), _ptr(self.tiles), n, _stream(stream)))
+        self.k = top_k
+
+    def __call__(self, h, eps=1e-6, stream=None):
+        """h fp32 [T][d] -> (h_out fp32 [T][d], chosen experts int32 [T][k], weights fp32 [T][k])."""
+        import torch
+        T, d = h.shape
+        out = torch.empty_like(h)
+        idx = torch.empty((T, self.k), dtype=torch.int32, device=h.device)
+        w = torch.empty((T, self.k), dtype=torch.float32, device=h.device)
+        n = lib().dlm_moe_scratch_size(T, d, C.byref(self.w))
+        if n == 0:
+            raise DlmError(DLM_EUNSUPPORTED, "moe: unsupported rows T=%d d=%d" % (T, d))
+        sc = _scratch(n, h.device)
+        _check(lib().dlm_moe_mlp_nvfp4(_ptr(h), _ptr(out), T, d, float(eps), C.byref(self.w), _ptr(self.tiles),
+                                       _ptr(idx), _ptr(w), _ptr(sc), n, _stream(stream)))
+        return out, idx, w
 
 
 def adapter_embed(E, Wa, tokens, s, stream=None):

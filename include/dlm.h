@@ -346,6 +346,44 @@ dlm_status dlm_lmhead_rowstats_nvfp4(const float* d_x, const dlm_nvfp4_matrix* E
                                      dlm_row_stats stats, float* d_s, void* d_scratch, size_t scratch_bytes,
                                      void* stream);
 
+/* Routed-expert MLP sub-block with NVFP4 experts ([blog] "ORL: diffusion LLMs get a learnable
+ * 'tokens per forward'", "What shipped", "dlmrt, the inference engine": routed experts run
+ * NVFP4 on FP4 tensor cores).  The pages give neither the routing rule nor the expert shapes;
+ * the library's reading:
+ *   x = RMSNorm(h) g;  l = x W_r^T;  the k experts of largest l (ties to the lower index),
+ *   weighted by softmax renormalised over the chosen: w_e = exp(l_e) / sum_chosen exp(l_j);
+ *   h_out = h + sum_e w_e down_e(silu(gate_e x) * (up_e x)).
+ * The E experts' gate and up matrices are stacked along rows ([E F][d], expert e in rows
+ * [e F, (e + 1) F)) and their down matrices side by side along columns ([d][E F]), each stack
+ * one NVFP4 matrix (see dlm_nvfp4_matrix).  x is quantized per row for the gate/up GEMM; the
+ * activation row entering the down projection is the concatenation over the experts of
+ * w_e silu(.) * up(.) (zeros for the experts not chosen), quantized per row, so the weighted
+ * sum over the experts is one FP4 contraction over E F.  Every expert's weights are streamed
+ * (at 32 rows and k of E experts most experts are chosen by some row). */
+typedef struct dlm_moe_weights {
+  int n_experts;      /* E, 1..256 */
+  int top_k;          /* k, 1..min(E, 8) */
+  int ffn_expert;     /* F, a multiple of 64; E F a multiple of 256 */
+  const void* w_router;   /* device, bf16 [E][d] */
+  const void* mlp_norm;   /* device, bf16 [d] */
+  dlm_nvfp4_matrix q_gate, q_up;  /* [E F][d] */
+  dlm_nvfp4_matrix q_down;        /* [d][E F] */
+} dlm_moe_weights;
+
+/* The experts' e4m3 scales re-tiled for the block-scaled MMA (done once per weight set):
+ * d_tiles receives dlm_moe_prepare_size(d, w) bytes. */
+size_t dlm_moe_prepare_size(int d, const dlm_moe_weights* w);
+dlm_status dlm_moe_prepare(int d, const dlm_moe_weights* w, void* d_tiles, size_t bytes, void* stream);
+
+/* One sub-block on T <= 32 rows: h_in, h_out fp32 [T][d] (distinct buffers), d % 256 == 0,
+ * d <= 8192; d_tiles from dlm_moe_prepare.  Outputs the chosen experts (int32 [T][k]) and their
+ * weights (fp32 [T][k]) when the pointers are non-null.  Scratch: dlm_moe_scratch_size bytes,
+ * DLM_ENOMEM_WS if smaller; DLM_EUNSUPPORTED for shapes outside the limits. */
+size_t dlm_moe_scratch_size(int T, int d, const dlm_moe_weights* w);
+dlm_status dlm_moe_mlp_nvfp4(const float* d_h_in, float* d_h_out, int T, int d, float rms_eps,
+                             const dlm_moe_weights* w, const void* d_tiles, int32_t* d_topk_idx,
+                             float* d_topk_w, void* d_scratch, size_t scratch_bytes, void* stream);
+
 /* Version string of the build. */
 const char* dlm_version(void);
 
