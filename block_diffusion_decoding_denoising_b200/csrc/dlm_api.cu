@@ -1562,7 +1562,8 @@ dlm_status dlm_moe_mlp_nvfp4(const float* d_h_in, float* d_h_out, int T, int d, 
   ra.route_w = route_w;
   ra.topk_idx = d_topk_idx;
   ra.topk_w = d_topk_w;
-  CU_LAUNCH(launch_k(k_moe_route, dim3(T), dim3(256), (d + E) * 4, s, ra));
+  CU_LAUNCH(launch_k(k_moe_logits, dim3(T, (E + 7) / 8), dim3(256), d * 4, s, ra));
+  CU_LAUNCH(launch_k(k_moe_topk, dim3((T + 7) / 8), dim3(256), 0, s, ra));
   ActQuantArgs q{};
   q.xf = x;
   q.K = d;

@@ -215,15 +215,14 @@ __global__ void __launch_bounds__(256) k_finish_silu(FinishArgs a) {
 }
 
 // out[t][n] = scale * y (scale 0 means 1), rows r and r + 64 of the tile per thread.
-// Routed-expert MLP front (one CTA per token row): x = h / sqrt(mean(h^2) + eps) g, router
-// logits l_e = x . W_r[e] (fp32, W_r bf16), then warp 0 picks the k largest logits (ties to
-// the lower index) and weights them by softmax renormalised over the chosen:
-// w_e = exp(l_e - m) / sum_chosen exp(l_j - m).  route_w gets the weights densely (zero for
-// the experts not chosen).
-__global__ void __launch_bounds__(256) k_moe_route(MoeRouteArgs a) {
+// Routed-expert MLP front, in two kernels.
+// k_moe_logits, grid (T, ceil(E / 8)): CTA (t, c) normalises row t, x = h / sqrt(mean(h^2) + eps)
+// g (fp32; CTA (t, 0) also stores it), and its 8 warps take the router logits of experts
+// 8 c .. 8 c + 7, l_e = x . W_r[e] (W_r bf16, fp32 sums).
+__global__ void __launch_bounds__(256) k_moe_logits(MoeRouteArgs a) {
   pdl_trigger();
   pdl_wait();
-  extern __shared__ float msm[];  // x [d] | logits [E]
+  extern __shared__ float sx[];  // x [d]
   __shared__ float red[8];
   const int t = blockIdx.x, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const float* h = a.h + (size_t)t * a.d;
@@ -236,34 +235,43 @@ __global__ void __launch_bounds__(256) k_moe_route(MoeRouteArgs a) {
 #pragma unroll
   for (int w = 0; w < 8; ++w) tot += red[w];
   const float r = 1.0f / sqrtf(tot / (float)a.d + a.eps);
-  float* sx = msm;
-  float* sl = msm + a.d;
   for (int c = tid; c < a.d; c += 256) {
     const float xv = h[c] * r * bf2f(a.g[c]);
     sx[c] = xv;
-    a.x[(size_t)t * a.d + c] = xv;
+    if (blockIdx.y == 0) a.x[(size_t)t * a.d + c] = xv;
   }
   __syncthreads();
-  for (int e = warp; e < a.E; e += 8) {
-    const __nv_bfloat16* wr = a.wr + (size_t)e * a.d;
-    float acc = 0.f;
-    for (int c0 = lane * 8; c0 < a.d; c0 += 256) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(wr + c0);
-      const __nv_bfloat16* wv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+  const int e = blockIdx.y * 8 + warp;
+  if (e >= a.E) return;
+  const __nv_bfloat16* wr = a.wr + (size_t)e * a.d;
+  float acc = 0.f;
+  for (int c0 = lane * 8; c0 < a.d; c0 += 256) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(wr + c0);
+    const __nv_bfloat16* wv = reinterpret_cast<const __nv_bfloat16*>(&raw);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) acc += sx[c0 + u] * bf2f(wv[u]);
-    }
-    acc = warp_sum(acc);
-    if (lane == 0) {
-      sl[e] = acc;
-      if (a.logits) a.logits[(size_t)t * a.E + e] = acc;
-    }
+    for (int u = 0; u < 8; ++u) acc += sx[c0 + u] * bf2f(wv[u]);
   }
-  __syncthreads();
-  if (warp != 0) return;
-  // lane owns experts lane + 32 j (j < 8, E <= 256)
+  acc = warp_sum(acc);
+  if (lane == 0) a.logits[(size_t)t * a.E + e] = acc;
+}
+
+// k_moe_topk, one warp per row: the k largest logits (ties to the lower index), weighted by
+// softmax renormalised over the chosen, w_e = exp(l_e - m) / sum_chosen exp(l_j - m); route_w
+// gets the weights densely (zero for the experts not chosen).
+__global__ void __launch_bounds__(256) k_moe_topk(MoeRouteArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const int t = blockIdx.x * 8 + threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (t >= a.T) return;
+  const float* l = a.logits + (size_t)t * a.E;
+  float lv[8];  // lane owns experts lane + 32 j (E <= 256)
   float mx = -INFINITY;
-  for (int e = lane; e < a.E; e += 32) mx = fmaxf(mx, sl[e]);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane + 32 * j;
+    lv[j] = e < a.E ? l[e] : -INFINITY;
+    mx = fmaxf(mx, lv[j]);
+  }
   mx = warp_max(mx);
   uint32_t taken = 0;
   float zs = 0.f, pw[8];
@@ -271,9 +279,10 @@ __global__ void __launch_bounds__(256) k_moe_route(MoeRouteArgs a) {
   for (int s = 0; s < a.k; ++s) {
     float best = -INFINITY;
     int be = 0x7fffffff;
-    for (int j = 0; lane + 32 * j < a.E; ++j) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
       const int e = lane + 32 * j;
-      if (!((taken >> j) & 1u) && (sl[e] > best || (sl[e] == best && e < be))) { best = sl[e]; be = e; }
+      if (e < a.E && !((taken >> j) & 1u) && (lv[j] > best || (lv[j] == best && e < be))) { best = lv[j]; be = e; }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {

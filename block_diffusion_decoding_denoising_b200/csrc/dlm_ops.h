@@ -58,7 +58,7 @@ struct MoeRouteArgs {
   float eps;
   int T, d, E, k;            // E <= 256, k <= 8, d % 8 == 0
   float* x;                  // [T][d] normalised rows
-  float* logits;             // [T][E] (optional)
+  float* logits;             // [T][E]
   float* route_w;            // [T][E] weights, zero for the experts not chosen
   int* topk_idx;             // [T][k] (optional)
   float* topk_w;             // [T][k] (optional)
@@ -122,7 +122,8 @@ struct BlockFinishArgs {
 __global__ void k_finish_qkv(FinishArgs a);
 __global__ void k_finish_silu(FinishArgs a);
 __global__ void k_finish_store(FinishArgs a);
-__global__ void k_moe_route(MoeRouteArgs a);
+__global__ void k_moe_logits(MoeRouteArgs a);
+__global__ void k_moe_topk(MoeRouteArgs a);
 __global__ void k_resid_norm(ResNormArgs a);
 __global__ void k_to_bf16(const float* x, __nv_bfloat16* y, long n, long lo, long zero_n);
 __global__ void k_rowstats_part(RowStatsArgs a);
