@@ -263,6 +263,9 @@ def nvfp4_measure(args, cfg, w, prompt, dev, stream):
     assert int(rr[:, 1].abs().sum().item()) == 0, "device status"
     ms = e0.elapsed_time(e1) / args.steps
     rounds = int(rr[:, 0].sum().item())
+    m.set_prefix_len(PROMPT)
+    m.decode_block(TAU, dlm.COMMIT_TOPK, TPF_K, tok[0], rr[0])
+    folded = m.fill_pending  # B = 32 NVFP4 contexts fold each block's KV-fill into the next round
     m.close()
     # the GEMM alone
     out = {"tokens_per_s": GEN / (ms / 1e3), "ms_per_step": ms, "rounds_per_step": rounds}
@@ -303,7 +306,10 @@ def nvfp4_measure(args, cfg, w, prompt, dev, stream):
     mean_L = PROMPT + GEN / 2
     round_b = nl * layer + cfg["vocab"] * d * 0.5625 + d * d * 2 + d * 2 + kv_pos * nl * mean_L
     fill_b = (nl - 1) * layer + qkv + d * 2 + kv_pos * (nl - 1) * mean_L
-    fills = blocks  # NVFP4 contexts run each block's KV-fill as its own forward
+    # the KV-fills: folded into the next block's first round (one flushed per step), else one
+    # forward per block
+    fills = 1 if folded else blocks
+    out["kv_fill"] = "folded into the next block's first round" if folded else "one forward per block"
     step_b = rounds * round_b + fills * fill_b
     out["round_bytes_mean_L"] = round_b
     out["round_ms"] = ms / (rounds + fills)

@@ -222,7 +222,7 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   const bool fp4 = c.weight_fmt == DLM_WEIGHTS_NVFP4;
   const size_t kmax = c.d > c.ffn ? c.d : c.ffn;
   uint8_t* xcodes = fp4 ? cv.take<uint8_t>((size_t)kMaxF4Tokens * kmax / 2) : nullptr;
-  uint8_t* xscales = fp4 ? cv.take<uint8_t>(kmax / 64 * 512) : nullptr;
+  uint8_t* xscales = fp4 ? cv.take<uint8_t>(f4_scale_bytes(kmax)) : nullptr;
   float* sx = fp4 ? cv.take<float>(kMaxF4Tokens) : nullptr;
   float* aam = fp4 ? cv.take<float>((size_t)((c.ffn + 63) / 64) * Tmax) : nullptr;
   __nv_bfloat16* edq = fp4 ? cv.take<__nv_bfloat16>((size_t)c.vocab * c.d) : nullptr;
@@ -573,12 +573,13 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
 
   // LM head: logits (finished inside the GEMM: its tiles are mostly single-slot), row
   // statistics, P = softmax (split bf16), s = P E
-  if (ctx->lmf && ctx->fp4 && Tp == 0) {
-    // one pass over the NVFP4 E: the rows of x were quantized by the last residual+RMSNorm
+  if (ctx->lmf && ctx->fp4) {
+    // one pass over the NVFP4 E: the rows of x were quantized by the last residual+RMSNorm;
+    // the round's own rows start at Tp (a pending block's rows come first)
     if (c.n_layers == 0) TRY(act_quant(r, T, ctx->xn, pad * d, d));
     char msg[256];
     cudaError_t e = lmhead_fused_f4_launch(ctx->w.q_embed, ctx->sf + c.n_layers * (ctx->sf_pair + ctx->sf_down),
-                                           ctx->xcodes, kMaxF4Tokens, ctx->xscales, ctx->sx, Tl, c.vocab, d,
+                                           ctx->xcodes, kMaxF4Tokens, Tp, ctx->xscales, ctx->sx, Tl, c.vocab, d,
                                            c.mask_id, f.stats, f.s_out, ctx->lmf, ctx->d_err, r.s, msg, sizeof(msg));
     if (e != cudaSuccess) return fail(ctx, DLM_ECUDA, "fused nvfp4 lm head: %s %s", cudaGetErrorString(e), msg);
     return DLM_OK;
@@ -629,10 +630,12 @@ dlm_status forward(Runner& r, const FwdSpec& f) {
 }
 
 // Whether the context can carry a pending block in the next round: the pass then has 2B
-// rows (split GEMM inputs up to 128 rows) and must use the fused LM head.
+// rows (split GEMM inputs up to 128 rows; NVFP4 GEMM inputs up to 64, so B = 32 and the
+// round's own rows are the second group of 32) and must use the fused LM head.
 bool fold_supported(const dlm_ctx* ctx) {
   const dlm_config& c = ctx->cfg;
-  return !ctx->fp4 && ctx->lmf != nullptr && 2 * c.block_size <= kMaxSplitTokens && c.block_size <= 32;
+  return ctx->lmf != nullptr && 2 * c.block_size <= (ctx->fp4 ? kMaxF4Tokens : kMaxSplitTokens) &&
+         c.block_size <= 32 && (!ctx->fp4 || c.block_size == 32);
 }
 
 dlm_status launch_commit(Runner& r, const dlm_block_state& st, float tau, int mode, int k,
@@ -1431,7 +1434,7 @@ dlm_status dlm_nvfp4_quantize(const void* d_w, int rows, int cols, void* d_codes
 
 size_t dlm_lmhead_nvfp4_scratch_size(int B, int V, int d) {
   if (!lmhead_fused_f4_supported(B, d) || V < 2) return 0;
-  return op_header() + align256((size_t)kMaxF4Tokens * d / 2) + align256((size_t)d / 64 * 512) +
+  return op_header() + align256((size_t)kMaxF4Tokens * d / 2) + align256(f4_scale_bytes(d)) +
          align256(kMaxF4Tokens * 4) + align256(nvf4_sf_tile_bytes(V, d, A_KMAJOR)) +
          align256(lmhead_fused_scratch_bytes(V, d));
 }
@@ -1454,13 +1457,13 @@ dlm_status dlm_lmhead_rowstats_nvfp4(const float* d_x, const dlm_nvfp4_matrix* E
     return q;
   };
   uint8_t* xcodes = take((size_t)kMaxF4Tokens * d / 2);
-  uint8_t* xscales = take((size_t)d / 64 * 512);
+  uint8_t* xscales = take(f4_scale_bytes(d));
   float* sx = (float*)take(kMaxF4Tokens * 4);
   uint8_t* sfe = take(nvf4_sf_tile_bytes(V, d, A_KMAJOR));
   void* lmf = take(lmhead_fused_scratch_bytes(V, d));
   // the status word, and the token codes and scales of the rows past B (read by the MMA, their
   // columns dropped), start at zero
-  CU(cudaMemsetAsync(base, 0, op_header() + align256((size_t)kMaxF4Tokens * d / 2) + align256((size_t)d / 64 * 512),
+  CU(cudaMemsetAsync(base, 0, op_header() + align256((size_t)kMaxF4Tokens * d / 2) + align256(f4_scale_bytes(d)),
                      s));
   CU(nvf4_sf_tile(*E, nullptr, V, d, A_KMAJOR, sfe, s));
   ActQuantArgs q{};
@@ -1471,7 +1474,7 @@ dlm_status dlm_lmhead_rowstats_nvfp4(const float* d_x, const dlm_nvfp4_matrix* E
   q.sx = sx;
   CU_LAUNCH(launch_k(k_act_quant, dim3(B), dim3(256), 0, s, q));
   char msg[256];
-  CU(lmhead_fused_f4_launch(*E, sfe, xcodes, kMaxF4Tokens, xscales, sx, B, V, d, mask_id, stats, d_s, lmf,
+  CU(lmhead_fused_f4_launch(*E, sfe, xcodes, kMaxF4Tokens, 0, xscales, sx, B, V, d, mask_id, stats, d_s, lmf,
                             (int*)base, s, msg, sizeof(msg)));
   return DLM_OK;
 }
@@ -1515,7 +1518,7 @@ size_t dlm_moe_scratch_size(int T, int d, const dlm_moe_weights* w) {
   if (T < 1 || T > kMaxF4Tokens || !moe_shape_ok(d, w)) return 0;
   const int E = w->n_experts, EF = E * w->ffn_expert, K = EF > d ? EF : d;
   return op_header() + op_counters(K) + align256(moe_partial_bytes(T, d, EF)) +
-         align256((size_t)kMaxF4Tokens * K / 2) + align256((size_t)K / 64 * 512) + align256(kMaxF4Tokens * 4) +
+         align256((size_t)kMaxF4Tokens * K / 2) + align256(f4_scale_bytes(K)) + align256(kMaxF4Tokens * 4) +
          align256((size_t)T * d * 4) + 2 * align256((size_t)T * E * 4) + 2 * align256((size_t)T * EF * 2) +
          align256((size_t)(EF / 64) * T * 4);
 }
@@ -1536,7 +1539,7 @@ dlm_status dlm_moe_mlp_nvfp4(const float* d_h_in, float* d_h_out, int T, int d, 
   const int E = w->n_experts, F = w->ffn_expert, EF = E * F, K = EF > d ? EF : d;
   OpScratch sc(d_scratch, K, moe_partial_bytes(T, d, EF));
   uint8_t* xcodes = sc.take<uint8_t>((size_t)kMaxF4Tokens * K / 2);
-  uint8_t* xscales = sc.take<uint8_t>((size_t)K / 64 * 512);
+  uint8_t* xscales = sc.take<uint8_t>(f4_scale_bytes(K));
   float* sx = sc.take<float>(kMaxF4Tokens);
   float* x = sc.take<float>((size_t)T * d);
   float* logits = sc.take<float>((size_t)T * E);
@@ -1547,7 +1550,7 @@ dlm_status dlm_moe_mlp_nvfp4(const float* d_h_in, float* d_h_out, int T, int d, 
   // their columns dropped), start at zero
   CU(cudaMemsetAsync(d_scratch, 0, op_header(), s));
   CU(cudaMemsetAsync(xcodes, 0, (size_t)kMaxF4Tokens * K / 2, s));
-  CU(cudaMemsetAsync(xscales, 0, (size_t)K / 64 * 512, s));
+  CU(cudaMemsetAsync(xscales, 0, f4_scale_bytes(K), s));
   MoeRouteArgs ra{};
   ra.h = d_h_in;
   ra.g = (const __nv_bfloat16*)w->mlp_norm;
@@ -1620,7 +1623,7 @@ dlm_status dlm_moe_mlp_nvfp4(const float* d_h_in, float* d_h_out, int T, int d, 
 size_t dlm_gemm_nvfp4_scratch_size(int T, int N, int K) {
   if (T < 1 || T > kMaxF4Tokens || N < 1 || K < 256 || K % 256 || K > 16384) return 0;
   return op_header() + op_counters(N) + align256(gemm_fp4_partial_bytes(T, N, K, A_KMAJOR)) +
-         align256((size_t)kMaxF4Tokens * K / 2) + align256((size_t)K / 64 * 512) + align256(kMaxF4Tokens * 4) +
+         align256((size_t)kMaxF4Tokens * K / 2) + align256(f4_scale_bytes(K)) + align256(kMaxF4Tokens * 4) +
          align256(nvf4_sf_tile_bytes(N, K, A_KMAJOR));
 }
 
@@ -1635,13 +1638,13 @@ dlm_status dlm_gemm_nvfp4(const float* d_x, const dlm_nvfp4_matrix* w, float* d_
   cudaStream_t s = (cudaStream_t)stream;
   OpScratch sc(d_scratch, N, gemm_fp4_partial_bytes(T, N, K, A_KMAJOR));
   uint8_t* xcodes = sc.take<uint8_t>((size_t)kMaxF4Tokens * K / 2);
-  uint8_t* xscales = sc.take<uint8_t>((size_t)K / 64 * 512);
+  uint8_t* xscales = sc.take<uint8_t>(f4_scale_bytes(K));
   float* sx = sc.take<float>(kMaxF4Tokens);
   uint8_t* sfa = sc.take<uint8_t>(nvf4_sf_tile_bytes(N, K, A_KMAJOR));
   CU(cudaMemsetAsync(d_scratch, 0, op_header(), s));
   // rows T.. of the token codes and scales are read by the MMA (their columns are dropped)
   CU(cudaMemsetAsync(xcodes, 0, (size_t)kMaxF4Tokens * K / 2, s));
-  CU(cudaMemsetAsync(xscales, 0, (size_t)K / 64 * 512, s));
+  CU(cudaMemsetAsync(xscales, 0, f4_scale_bytes(K), s));
   CU(nvf4_sf_tile(*w, nullptr, N, K, A_KMAJOR, sfa, s));
   ActQuantArgs q{};
   q.xf = d_x;

@@ -239,6 +239,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool a_mn_major,
          | (uint32_t(m >> 4) << 24);     // M / 16
 }
 
+// Token scales of an NVFP4 GEMM input (K elements per row): one plane per group of 32 tokens,
+// [group][64-element block][token % 32][16 B], byte k of a row's 16 the scale of its
+// 16-element group 4 b + k (4 of the 16 bytes used), so that a stage's four blocks of one
+// group are 2 KB of contiguous tcgen05.cp sources.  b16 = index of the 16-element block.
+__host__ __device__ __forceinline__ size_t tok_scale_index(int t, int b16, int K) {
+  return ((size_t)(t >> 5) * (size_t)(K / 64) + (size_t)(b16 >> 2)) * 512 + (size_t)(t & 31) * 16 + (size_t)(b16 & 3);
+}
+
 // ---------------------------------------------------------------- block-scaled FP4 MMA
 // Shared-memory descriptor of a 32-row x 16-byte block without swizzle (the tcgen05.cp
 // source): core matrices of 8 rows x 16 bytes, 128 bytes apart.

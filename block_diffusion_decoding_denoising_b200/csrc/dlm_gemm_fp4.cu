@@ -16,7 +16,10 @@
 // swizzle), the codes of 32 tokens (4 KB), the weight tile's scales (2 KB, pre-tiled, see
 // below) and the tokens' scales (2 KB, pre-tiled).  The MMA thread copies the scales into tensor
 // memory (tcgen05.cp, 32 lanes x 128 bits, replicated to the four lane quarters) and issues
-// four K = 64 MMAs per stage.  Work is cut stream-K over (tile, 256-element k-block) units
+// four K = 64 MMAs per stage.  Inputs of 33..64 rows (a round carrying a pending block) run as
+// two groups of 32 tokens: a stage then holds both groups' codes and scales (30 KB, 7 stages)
+// and each group issues its own four N = 32 MMAs on the shared weight tile, into its own half
+// of the accumulator.  Work is cut stream-K over (tile, 256-element k-block) units
 // exactly like the bf16 GEMM, and the epilogue writes scaled partial sums in the same
 // [tile][slot][TP][128] layout, so the same finish kernels complete it.
 //
@@ -24,9 +27,9 @@
 // group k (of 4) sits in lane m % 32 of every lane quarter, 32-bit column m / 32, byte k; the
 // 32 tokens' scales in lane t, one column.  Each MMA's scales get their own 4-column slot.
 // The weight scales are therefore re-tiled once (k_sf_tile) into [tile][64-element block]
-// [lane 32][column 4][byte 4], and the quantizer writes the token scales as [64-element
-// block][token 32][16 B] (4 bytes used), so that a stage's four blocks are 2 KB of
-// contiguous 512-byte copy sources for either operand.
+// [lane 32][column 4][byte 4], and the quantizer writes the token scales as [group of 32
+// tokens][64-element block][token % 32][16 B] (4 bytes used; tok_scale_index), so that a
+// stage's four blocks of one group are 2 KB of contiguous 512-byte copy sources.
 #include <cuda_fp16.h>
 #include <stdio.h>
 #include <string.h>
@@ -40,20 +43,31 @@ namespace {
 
 constexpr int kF4K = 256;          // reduction elements per stage (128 code bytes per row)
 constexpr int kF4Mmas = kF4K / 64; // K = 64 MMAs per stage
-constexpr int kF4Stages = 8;
 constexpr int kF4ACodes = kTileM * 128;   // 16 KB
-constexpr int kF4BCodes = 32 * 128;       // 4 KB
+constexpr int kF4BCodes = 32 * 128;       // 4 KB per group of 32 tokens
 constexpr int kF4SfA = kTileM * kF4K / 16;  // 2 KB
-constexpr int kF4SfB = kF4Mmas * 32 * 16;  // 2 KB: per MMA 32 tokens x 16 B (4 scale bytes used)
-constexpr int kF4OffB = kF4ACodes, kF4OffSfA = kF4OffB + kF4BCodes, kF4OffSfB = kF4OffSfA + kF4SfA;
-constexpr int kF4StageBytes = 24576;      // 24 KB
-static_assert(kF4OffSfB + kF4SfB <= kF4StageBytes, "stage layout");
-constexpr int kF4Smem = kF4Stages * kF4StageBytes + 1024 + 512;
+constexpr int kF4SfB = kF4Mmas * 32 * 16;  // 2 KB per group: per MMA 32 tokens x 16 B (4 scale bytes used)
 constexpr int kF4TmemCols = 512;
-constexpr int kF4SfCol = 64;              // TMEM: accumulators in [0, 64), scales from here
-// per stage and MMA, a 4-column slot for the weight scales and one for the token scales
-constexpr int kF4SfColsPerStage = 4 * kF4Mmas + 4 * kF4Mmas;
-static_assert(kF4SfCol + kF4Stages * kF4SfColsPerStage <= kF4TmemCols, "tmem budget");
+// Stage layout for G groups of 32 tokens (G = 1: up to 32 rows; G = 2: up to 64, the rows of
+// a round that carries a pending block): weight codes | G token-code boxes | weight scales |
+// G token-scale blocks.  Each group runs its own four N = 32 MMAs on the shared weight tile.
+template <int G>
+struct F4Cfg {
+  static constexpr int kOffB = kF4ACodes;
+  static constexpr int kOffSfA = kOffB + G * kF4BCodes;
+  static constexpr int kOffSfB = kOffSfA + kF4SfA;
+  static constexpr int kStageBytes = kOffSfB + G * kF4SfB;  // 24 KB / 30 KB
+  static constexpr int kStages = G == 1 ? 8 : 7;
+  static constexpr int kSmem = kStages * kStageBytes + 1024 + 512;
+  static constexpr int kAccCols = G * 32;                  // one accumulator (all groups)
+  static constexpr int kSfCol = 2 * kAccCols;              // two accumulators, then the scales
+  // per stage and MMA, a 4-column slot for the weight scales and one per group for the tokens'
+  static constexpr int kSfColsPerStage = 4 * kF4Mmas * (1 + G);
+};
+static_assert(F4Cfg<1>::kStageBytes == 24576 && F4Cfg<2>::kStageBytes == 30720, "stage layout");
+static_assert(F4Cfg<2>::kSmem <= 232448, "nvfp4 gemm shared memory");
+static_assert(F4Cfg<1>::kSfCol + F4Cfg<1>::kStages * F4Cfg<1>::kSfColsPerStage <= kF4TmemCols, "tmem budget");
+static_assert(F4Cfg<2>::kSfCol + F4Cfg<2>::kStages * F4Cfg<2>::kSfColsPerStage <= kF4TmemCols, "tmem budget");
 
 struct F4KArgs {
   int a_mode;        // A_KMAJOR or A_PAIR
@@ -62,16 +76,21 @@ struct F4KArgs {
   float sw0, sw1;    // tensor scales (rows 0..63 / 64..127 of a pair tile use sw0 / sw1)
   const float* sx;   // [T] row scales of the quantized activations
   const uint8_t* sfa;  // tiled weight scales (k_sf_tile)
-  const uint8_t* sfb;  // tiled token scales (k_act_quant)
+  const uint8_t* sfb;  // tiled token scales (k_act_quant): group g's plane at sfb + g * K / 64 * 512
+  int nb64;            // K / 64
   int* err;
 };
 
 __device__ __forceinline__ void epi_sync_f4() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+template <int G>
 __global__ void __launch_bounds__(192, 1)
 k_gemm_nvf4(const __grid_constant__ CUtensorMap tc0, const __grid_constant__ CUtensorMap tc1,
             const __grid_constant__ CUtensorMap tbc, F4KArgs args) {
-  constexpr int S = kF4Stages;
+  using Cf = F4Cfg<G>;
+  constexpr int S = Cf::kStages;
+  constexpr int kF4StageBytes = Cf::kStageBytes;
+  constexpr int kF4OffB = Cf::kOffB, kF4OffSfA = Cf::kOffSfA, kF4OffSfB = Cf::kOffSfB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(smem + S * kF4StageBytes);
@@ -125,15 +144,19 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tc0, const __grid_constant__ CUt
       }
       bulk_load(base + kF4OffSfA, args.sfa + ((size_t)tile * o.n_kb + kb) * kF4SfA, kF4SfA, &full[st]);
     };
-    auto load_x = [&](long u, int st) {  // token codes and tiled token scales
+    auto load_x = [&](long u, int st) {  // token codes and tiled token scales, per group
       const int kb = (int)(u % o.n_kb);
       uint8_t* base = smem + st * kF4StageBytes;
-      tma_load_2d(base + kF4OffB, &tbc, &full[st], kb * 128, 0);
-      bulk_load(base + kF4OffSfB, args.sfb + (size_t)kb * kF4SfB, kF4SfB, &full[st]);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        tma_load_2d(base + kF4OffB + g * kF4BCodes, &tbc, &full[st], kb * 128, g * 32);
+        bulk_load(base + kF4OffSfB + g * kF4SfB, args.sfb + ((size_t)g * args.nb64 + (size_t)kb * kF4Mmas) * 512,
+                  kF4SfB, &full[st]);
+      }
     };
     const long n_pre = (u_end - u_begin) < S ? (u_end - u_begin) : S;
     for (long i = 0; i < n_pre; ++i) {
-      mbar_arrive_expect_tx(&full[i], kF4ACodes + kF4BCodes + kF4SfA + kF4SfB);
+      mbar_arrive_expect_tx(&full[i], kF4StageBytes);
       armed[i] = true;
       armed_parity[i] = 0;
       load_w(u_begin + i, (int)i);
@@ -144,7 +167,7 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tc0, const __grid_constant__ CUt
     uint32_t phase = (n_pre == S) ? 1u : 0u;
     for (long u = u_begin + n_pre; u < u_end; ++u) {
       if (!mbar_wait(&empty[stage], phase ^ 1, args.err)) break;
-      mbar_arrive_expect_tx(&full[stage], kF4ACodes + kF4BCodes + kF4SfA + kF4SfB);
+      mbar_arrive_expect_tx(&full[stage], kF4StageBytes);
       armed[stage] = true;
       armed_parity[stage] = phase;
       load_w(u, stage);
@@ -168,25 +191,31 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tc0, const __grid_constant__ CUt
       const long seg_end = ((long)tile + 1) * o.n_kb < u_end ? ((long)tile + 1) * o.n_kb : u_end;
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_empty[acc], acc_phase ^ 1, args.err))) { ok = false; break; }
       tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * 32;
+      const uint32_t d_tmem = tmem_base + acc * Cf::kAccCols;
       for (long uu = u; uu < seg_end; ++uu) {
         if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, args.err))) { ok = false; break; }
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + stage * kF4StageBytes);
-        const uint32_t sfa_col = tmem_base + kF4SfCol + stage * kF4SfColsPerStage;
-        const uint32_t sfb_col = sfa_col + 4 * kF4Mmas;
-        const uint64_t ad = sw128_desc(sa, 16, 1024), bd = sw128_desc(sa + kF4OffB, 16, 1024);
-        const uint64_t fa = sf_desc(sa + kF4OffSfA), fb = sf_desc(sa + kF4OffSfB);
+        const uint32_t sfa_col = tmem_base + Cf::kSfCol + stage * Cf::kSfColsPerStage;
+        const uint32_t sfb_col = sfa_col + 4 * kF4Mmas;  // + 16 columns per group
+        const uint64_t ad = sw128_desc(sa, 16, 1024);
+        const uint64_t fa = sf_desc(sa + kF4OffSfA);
         if (elect_one()) {
 #pragma unroll
           for (int j = 0; j < kF4Mmas; ++j) {  // +512 B per copy source
             tmem_cp_32x128(sfa_col + 4 * j, fa + 32 * j);
-            tmem_cp_32x128(sfb_col + 4 * j, fb + 32 * j);
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+              tmem_cp_32x128(sfb_col + 16 * g + 4 * j, sf_desc(sa + kF4OffSfB + g * kF4SfB) + 32 * j);
           }
 #pragma unroll
-          for (int j = 0; j < kF4Mmas; ++j)  // +32 B per K = 64 step
-            mma_nvf4(d_tmem, ad + 2 * j, bd + 2 * j, idesc, sfa_col + 4 * j, sfb_col + 4 * j,
-                     (uu > u || j > 0) ? 1u : 0u);
+          for (int g = 0; g < G; ++g) {
+            const uint64_t bd = sw128_desc(sa + kF4OffB + g * kF4BCodes, 16, 1024);
+#pragma unroll
+            for (int j = 0; j < kF4Mmas; ++j)  // +32 B per K = 64 step
+              mma_nvf4(d_tmem + 32 * g, ad + 2 * j, bd + 2 * j, idesc, sfa_col + 4 * j, sfb_col + 16 * g + 4 * j,
+                       (uu > u || j > 0) ? 1u : 0u);
+          }
           mma_commit(&empty[stage]);
         }
         __syncwarp();
@@ -209,7 +238,7 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tc0, const __grid_constant__ CUt
     const int row = quarter * 32 + lane;
     const int et = threadIdx.x - 64;
     const float sw = (args.a_mode == A_PAIR && row >= 64) ? args.sw1 : args.sw0;
-    const int TP = 32;
+    const int TP = G * 32;
     int acc = 0;
     uint32_t acc_phase = 0;
     long u = u_begin;
@@ -226,9 +255,15 @@ k_gemm_nvf4(const __grid_constant__ CUtensorMap tc0, const __grid_constant__ CUt
       const int lo_c = cta_of_unit((long)tile * o.n_kb, o.units, o.grid);
       const int slot = c - lo_c;
       float* dst = o.partial + ((size_t)tile * o.max_slots + slot) * kTileM * TP + row;
-      tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * 32, v);
+#pragma unroll 1
+      for (int g = 0; g < G; ++g) {
+        tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * Cf::kAccCols + 32 * g, v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) dst[(size_t)j * kTileM] = (j < args.T) ? v[j] * (sw * args.sx[j]) : 0.f;
+        for (int j = 0; j < 32; ++j) {
+          const int t = 32 * g + j;
+          dst[(size_t)t * kTileM] = (t < args.T) ? v[j] * (sw * args.sx[t]) : 0.f;
+        }
+      }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
@@ -332,7 +367,7 @@ bool encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t o
 size_t gemm_fp4_partial_bytes(int T, int N, int K, int a_mode) {
   GemmOut o;
   partition_f4(T, N, K, a_mode, &o);
-  return (size_t)o.n_tiles * o.max_slots * 32 * kTileM * sizeof(float);
+  return (size_t)o.n_tiles * o.max_slots * ((T + 31) / 32 * 32) * kTileM * sizeof(float);
 }
 
 size_t nvf4_sf_tile_bytes(int N, int K, int a_mode) {
@@ -387,8 +422,9 @@ bool gemm_fp4_plan(GemmF4Plan* p, int a_mode, const dlm_nvfp4_matrix& w0, const 
     p->tc1 = p->tc0;
   // token codes [x_rows][K/2] (128-byte swizzle); token scales tiled (k_act_quant)
   p->sfb = xscales;
-  ok = ok && encode_2d(&p->tbc, CU_TENSOR_MAP_DATA_TYPE_UINT8, xcodes, (uint64_t)K / 2, 32, (uint64_t)K / 2, 128,
-                       32, CU_TENSOR_MAP_SWIZZLE_128B, err, errlen);
+  // (all x_rows rows: a 64-row input is loaded as two 32-row boxes)
+  ok = ok && encode_2d(&p->tbc, CU_TENSOR_MAP_DATA_TYPE_UINT8, xcodes, (uint64_t)K / 2, (uint64_t)x_rows,
+                       (uint64_t)K / 2, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B, err, errlen);
   return ok;
 }
 
@@ -402,14 +438,20 @@ cudaError_t gemm_fp4_launch(const GemmF4Plan& p, int* d_err, cudaStream_t s) {
   a.sx = p.sx;
   a.sfa = p.sfa;
   a.sfb = p.sfb;
+  a.nb64 = p.K / 64;
   a.err = d_err;
-  return launch_k(k_gemm_nvf4, dim3(p.out.grid), dim3(192), kF4Smem, s, p.tc0, p.tc1, p.tbc, a);
+  if (p.T > 32)
+    return launch_k(k_gemm_nvf4<2>, dim3(p.out.grid), dim3(192), F4Cfg<2>::kSmem, s, p.tc0, p.tc1, p.tbc, a);
+  return launch_k(k_gemm_nvf4<1>, dim3(p.out.grid), dim3(192), F4Cfg<1>::kSmem, s, p.tc0, p.tc1, p.tbc, a);
 }
 
 int gemm_fp4_init_attributes() {
   static PerDeviceOnce once;
   return once_on_current_device(once, [] {
-    return (int)cudaFuncSetAttribute(k_gemm_nvf4, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4Smem);
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_nvf4<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, F4Cfg<1>::kSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_gemm_nvf4<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, F4Cfg<2>::kSmem);
+    return (int)e;
   });
 }
 

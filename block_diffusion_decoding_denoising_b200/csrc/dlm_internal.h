@@ -69,7 +69,10 @@ constexpr int kTileM = 128;      // output features per GEMM tile (tcgen05 M)
 constexpr int kTileK = 64;       // reduction elements per k-block (one 128-byte swizzle atom)
 constexpr int kMaxTokens = 256;  // tokens per GEMM with plain bf16 activations (tcgen05 N <= 256)
 constexpr int kMaxSplitTokens = 128;  // tokens per GEMM with split (hi + lo) activations
-constexpr int kMaxF4Tokens = 32;      // tokens per NVFP4 GEMM (MMA N)
+constexpr int kMaxF4Tokens = 64;      // rows per NVFP4 GEMM: two groups of 32 (MMA N = 32 each)
+// Bytes of the tiled token scales of an NVFP4 GEMM input with K elements per row, kMaxF4Tokens
+// rows (one plane per group of 32; see tok_scale_index).
+inline size_t f4_scale_bytes(long K) { return (size_t)(kMaxF4Tokens / 32) * (size_t)(K / 64) * 512; }
 
 // Partial-sum layout written by the GEMM: [tile][slot][TP][128] fp32, TP = T rounded up to
 // 32 (token-major: the 128 rows of one token are contiguous).  Tile tau covers
@@ -195,11 +198,12 @@ cudaError_t lmhead_fused_launch(const void* x2, int x2_rows, int hi_row, int lo_
 
 // The same pass with NVFP4 E (codes [V][d/2], e4m3 scales [V][d/16], tensor scale; sfe_tiled
 // its scales re-tiled by nvf4_sf_tile) and x quantized by the last RMSNorm (codes [x_rows][d/2],
-// token t in row t; tiled scales; row scales sx[T]).  T <= 32, d % 512 == 0, d <= 2560.
+// tiled scales, row scales sx): the T rows from row x_row0 (a multiple of 32: the rows of a
+// round that carries a pending block start at 32).  T <= 32, d % 512 == 0, d <= 2560.
 bool lmhead_fused_f4_supported(int T, int d);
 cudaError_t lmhead_fused_f4_launch(const dlm_nvfp4_matrix& E, const uint8_t* sfe_tiled, const uint8_t* xcodes,
-                                   int x_rows, const uint8_t* xscales, const float* sx, int T, int V, int d,
-                                   int mask_id, dlm_row_stats stats, float* s, void* scratch, int* d_err,
+                                   int x_rows, int x_row0, const uint8_t* xscales, const float* sx, int T, int V,
+                                   int d, int mask_id, dlm_row_stats stats, float* s, void* scratch, int* d_err,
                                    cudaStream_t st, char* err, size_t errlen);
 // 2-D tensor map of a byte matrix [outer][inner] (rows of `inner` bytes).
 bool encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,

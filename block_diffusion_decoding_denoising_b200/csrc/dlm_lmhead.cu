@@ -749,7 +749,7 @@ k_lmhead_fused_f4(const __grid_constant__ CUtensorMap tec, const __grid_constant
         const int b64 = (d0 + kb * 256) / 64;       // its 64-element block
         mbar_arrive_expect_tx(&full[stage], kF4LmStageBytes);
         tma_load_2d_hint(st, &tec, &full[stage], kc, tile * 128, keep);
-        tma_load_2d(st + 16384, &txc, &full[stage], kc, 0);
+        tma_load_2d(st + 16384, &txc, &full[stage], kc, a.x_hi_row);
         bulk_load(st + 20480, sfe + ((size_t)tile * NB64 + b64) * 512, 2048, &full[stage]);
         bulk_load(st + 22528, sfx + (size_t)b64 * 512, 2048, &full[stage]);
         if (++stage == kF4LmStages) { stage = 0; phase ^= 1; }
@@ -1158,12 +1158,13 @@ bool lmhead_fused_f4_supported(int T, int d) {
 // the block-scaled MMA; x: codes [x_rows][d/2] (token t in row t), tiled scales and row scales
 // sx[T] as the quantizer of the last RMSNorm leaves them.
 cudaError_t lmhead_fused_f4_launch(const dlm_nvfp4_matrix& E, const uint8_t* sfe_tiled, const uint8_t* xcodes,
-                                   int x_rows, const uint8_t* xscales, const float* sx, int T, int V, int d,
-                                   int mask_id, dlm_row_stats stats, float* s, void* scratch, int* d_err,
+                                   int x_rows, int x_row0, const uint8_t* xscales, const float* sx, int T, int V,
+                                   int d, int mask_id, dlm_row_stats stats, float* s, void* scratch, int* d_err,
                                    cudaStream_t st, char* err, size_t errlen) {
   if (!lmhead_fused_f4_supported(T, d) || !E.codes || !E.scales || !sfe_tiled || !xcodes || !xscales || !sx ||
-      x_rows < T) {
-    snprintf(err, errlen, "nvfp4 lm head: unsupported arguments T=%d d=%d x_rows=%d", T, d, x_rows);
+      x_row0 < 0 || x_row0 % 32 || x_row0 + T > x_rows) {
+    snprintf(err, errlen, "nvfp4 lm head: unsupported arguments T=%d d=%d x rows %d + %d of %d", T, d, x_row0, T,
+             x_rows);
     return cudaErrorInvalidValue;
   }
   {
@@ -1188,7 +1189,9 @@ cudaError_t lmhead_fused_f4_launch(const dlm_nvfp4_matrix& E, const uint8_t* sfe
   a.n_clu = a.n_tiles < kLmMaxClusters ? a.n_tiles : kLmMaxClusters;
   a.given = 0;
   a.se = E.tensor_scale;
-  a.sx = sx;
+  a.sx = sx + x_row0;      // the T rows' scales
+  a.x_hi_row = x_row0;     // first row of their codes
+  xscales += tok_scale_index(x_row0, 0, d);  // their group's plane of token scales
   a.s_scale = E.tensor_scale / kF4PScale;
   uint8_t* sc = (uint8_t*)scratch;
   a.part_stats = (float*)sc;

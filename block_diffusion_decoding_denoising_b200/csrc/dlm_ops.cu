@@ -445,7 +445,7 @@ __global__ void __launch_bounds__(kRnThreads) k_resid_norm(ResNormArgs a) {
     if ((lane & 1) == 0) a.qcodes[(size_t)t * (a.d / 2) + n / 2] = (uint8_t)(code | (hi << 4));
     if ((lane & 15) == 0) {
       const int gi = n / 16;
-      a.qscales[((size_t)(gi / 4) * 32 + t) * 16 + (gi % 4)] = sb;
+      a.qscales[tok_scale_index(t, gi, a.d)] = sb;
     }
   }
 }
@@ -782,7 +782,7 @@ __global__ void __launch_bounds__(256) k_act_quant(ActQuantArgs a) {
       const uint32_t c = denom > 0.f ? e2m1_rne(v[i][j] / denom) : 0u;
       packed[j / 8] |= c << (4 * (j % 8));  // element 2m in the low nibble of byte m
     }
-    a.scales[((size_t)(b / 4) * 32 + t) * 16 + (b % 4)] = sb;  // [64-element block][token][16 B]
+    a.scales[tok_scale_index(t, b, a.K)] = sb;
     *reinterpret_cast<uint2*>(a.codes + (size_t)t * (a.K / 2) + (size_t)b * 8) = make_uint2(packed[0], packed[1]);
   }
 }
@@ -823,7 +823,7 @@ __global__ void __launch_bounds__(256) k_act_quant_wide(ActQuantArgs a) {
     const uint32_t c = denom > 0.f ? e2m1_rne(v[j] / denom) : 0u;
     packed[j / 8] |= c << (4 * (j % 8));
   }
-  a.scales[((size_t)(b / 4) * 32 + t) * 16 + (b % 4)] = sb;
+  a.scales[tok_scale_index(t, b, a.K)] = sb;
   *reinterpret_cast<uint2*>(a.codes + (size_t)t * (a.K / 2) + (size_t)b * 8) = make_uint2(packed[0], packed[1]);
 }
 

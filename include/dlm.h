@@ -296,7 +296,7 @@ dlm_status dlm_bd_attention_noalloc(const void* d_q, const void* d_k_cache, cons
 /* One layer's MLP sub-block on given residual rows (single operation for parity tests):
  * h_out = h_in + W_down (silu(W_gate x) * (W_up x)), x = RMSNorm(h_in) g_mlp, with the
  * context's weights of that layer (for NVFP4 weights x and the SiLU output are quantized per
- * row, as in a round).  d_h_in, d_h_out fp32 [T][d]; T <= 32 (NVFP4) or <= 128.  Uses the
+ * row, as in a round).  d_h_in, d_h_out fp32 [T][d]; T <= 64 (NVFP4) or <= 128.  Uses the
  * context's workspace: not concurrent with other calls on the context. */
 dlm_status dlm_mlp_block(dlm_ctx* ctx, int layer, const float* d_h_in, float* d_h_out, int T, void* stream);
 
@@ -326,7 +326,7 @@ dlm_status dlm_nvfp4_quantize(const void* d_w, int rows, int cols, void* d_codes
  * [T][K]) to NVFP4 with its own fp32 scale amax_row / (6 * 448), e4m3 scales per 16 elements
  * and round-to-nearest-even e2m1 codes, the format the pages' B200 numbers use ("ORL:
  * diffusion LLMs get a learnable 'tokens per forward'", "What shipped"), on the
- * block-scaled FP4 tensor cores.  T <= 32, K % 256 == 0, K <= 16384.  d_y may be NULL:
+ * block-scaled FP4 tensor cores.  T <= 64, K % 256 == 0, K <= 16384.  d_y may be NULL:
  * partial sums only (kernel timing). */
 size_t dlm_gemm_nvfp4_scratch_size(int T, int N, int K);
 dlm_status dlm_gemm_nvfp4(const float* d_x, const dlm_nvfp4_matrix* w, float* d_y, int T, int N, int K,
@@ -375,7 +375,7 @@ typedef struct dlm_moe_weights {
 size_t dlm_moe_prepare_size(int d, const dlm_moe_weights* w);
 dlm_status dlm_moe_prepare(int d, const dlm_moe_weights* w, void* d_tiles, size_t bytes, void* stream);
 
-/* One sub-block on T <= 32 rows: h_in, h_out fp32 [T][d] (distinct buffers), d % 256 == 0,
+/* One sub-block on T <= 64 rows: h_in, h_out fp32 [T][d] (distinct buffers), d % 256 == 0,
  * d <= 8192; d_tiles from dlm_moe_prepare.  Outputs the chosen experts (int32 [T][k]) and their
  * weights (fp32 [T][k]) when the pointers are non-null.  Scratch: dlm_moe_scratch_size bytes,
  * DLM_ENOMEM_WS if smaller; DLM_EUNSUPPORTED for shapes outside the limits. */

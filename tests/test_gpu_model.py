@@ -80,6 +80,9 @@ MODELS = {
     # d a multiple of 512: the LM head runs as the fused NVFP4 kernel
     "two_layer_nvfp4_d512": lambda: small_model(0.06, n_layers=2, d=512, Hq=4, Hkv=2, hd=64, F=1024, V=1024, B=16,
                                                 fmt=1),
+    # ... and with blocks of 32 the NVFP4 context folds its KV-fills (64-row rounds)
+    "nvfp4_b32_d512": lambda: small_model(0.06, n_layers=2, d=512, Hq=4, Hkv=2, hd=64, F=1024, V=1024, B=32,
+                                          fmt=1, max_ctx=320),
     # block of 32 as in the 4B-class configuration: a folded round carries 64 rows
     "gqa_b32": lambda: small_model(0.06, n_layers=2, d=256, Hq=4, Hkv=2, hd=64, F=512, V=1024, B=32, max_ctx=320),
     # FP8 KV cache (reading R13)
@@ -93,9 +96,12 @@ def is_fp4(cfg):
 
 
 def folds(cfg):
-    """Whether the library defers this model's KV-fills into the next round: bf16 weights,
-    B <= 32 and the fused LM head (d a multiple of 256, at most 3072)."""
-    return not is_fp4(cfg) and cfg["d"] % 256 == 0 and cfg["d"] <= 3072 and cfg["block_size"] <= 32
+    """Whether the library defers this model's KV-fills into the next round: the fused LM head
+    (bf16: d a multiple of 256, at most 3072, B <= 32; NVFP4: d a multiple of 512, at most 2560,
+    and B = 32, the second group of 32 rows of the NVFP4 GEMMs)."""
+    if is_fp4(cfg):
+        return cfg["d"] % 512 == 0 and cfg["d"] <= 2560 and cfg["block_size"] == 32
+    return cfg["d"] % 256 == 0 and cfg["d"] <= 3072 and cfg["block_size"] <= 32
 
 
 def rtol(cfg):
@@ -319,6 +325,7 @@ def compare_round(st, ost, com, new, tau, mode, k, cfg, what):
 MIN_DECIDED = {("tiny", 0): 4, ("tiny", 1): 4, ("tiny_distinct", 0): 20, ("tiny_distinct", 1): 10,
                ("two_layer_gqa", 0): 26, ("two_layer_gqa", 1): 21, ("two_layer_gqa_nvfp4", 0): 0,
                ("two_layer_gqa_nvfp4", 1): 0, ("two_layer_nvfp4_d512", 0): 0, ("two_layer_nvfp4_d512", 1): 0,
+               ("nvfp4_b32_d512", 0): 0, ("nvfp4_b32_d512", 1): 0,
                ("gqa_b32", 0): 32, ("gqa_b32", 1): 36,
                ("two_layer_gqa_fp8kv", 0): 32, ("two_layer_gqa_fp8kv", 1): 20}
 
@@ -428,7 +435,7 @@ def test_round_lockstep(dlm, name, mode, tau, k):
 
 
 @pytest.mark.parametrize("name", ["tiny_distinct", "two_layer_gqa", "two_layer_gqa_nvfp4", "two_layer_nvfp4_d512",
-                                  "two_layer_gqa_fp8kv"])
+                                  "nvfp4_b32_d512", "two_layer_gqa_fp8kv"])
 def test_graph_decode_matches_eager_rounds(dlm, name):
     """The per-block CUDA graph (while node) and eager dlm_round calls run the same
     kernels on the same inputs: tokens, round counts and the KV cache must be identical,
@@ -468,7 +475,10 @@ def test_graph_decode_matches_eager_rounds(dlm, name):
     assert torch.equal(a.kv, b.kv)  # the cache bytes (values, and scales for FP8)
 
 
-@pytest.mark.parametrize("name", [n for n in MODELS if folds(MODELS[n]()[0])])
+# bf16 contexts: the folded pass splits the attention key range differently, and at 4-bit
+# activations (NVFP4) such float differences flip quantization decisions (reading R12), so
+# NVFP4 folds are checked against the oracle in lock-step and graph against eager instead
+@pytest.mark.parametrize("name", [n for n in MODELS if folds(MODELS[n]()[0]) and not is_fp4(MODELS[n]()[0])])
 def test_deferred_fill_matches_eager_fill(dlm, name):
     """Blocks decoded with the KV-fill folded into the next block's first round and with a
     separate KV-fill forward per block: the same tokens and round counts, and K/V caches

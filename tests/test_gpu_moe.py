@@ -72,7 +72,7 @@ def check(D, moe, h, what, tol=2e-2):
 
 
 @pytest.mark.parametrize("E,k,F,d,T", [(4, 2, 64, 256, 5), (16, 4, 128, 512, 32), (64, 8, 64, 1024, 17),
-                                       (8, 1, 256, 768, 3)])
+                                       (8, 1, 256, 768, 3), (16, 2, 128, 512, 64)])
 def test_moe_matches_oracle(D, E, k, F, d, T):
     moe, h = make_case(E, k, F, d, T, seed=E * 100 + k * 10 + T)
     check(D, moe, h, "moe E=%d k=%d F=%d d=%d T=%d" % (E, k, F, d, T))
@@ -101,4 +101,4 @@ def test_moe_rejects_unsupported_shapes(D):
     with pytest.raises(DlmError):
         run(D, dict(moe, ffn_expert=48), h)  # F % 64 != 0
     with pytest.raises(DlmError):
-        run(D, moe, np.zeros((33, 256), np.float32))  # T > 32
+        run(D, moe, np.zeros((65, 256), np.float32))  # T > 64

@@ -47,15 +47,16 @@ def run_case(D, T, N, K, seed, std=0.02, x_std=1.0):
     return err
 
 
-@pytest.mark.parametrize("T", [1, 5, 17, 32])
+@pytest.mark.parametrize("T", [1, 5, 17, 32, 33, 48, 64])
 @pytest.mark.parametrize("N,K", [(128, 256), (384, 512), (200, 768), (640, 2560)])
 def test_gemm_nvfp4_small(lib, T, N, K):
     run_case(lib, T, N, K, seed=T * 1000 + N + K)
 
 
 @pytest.mark.parametrize("N,K", [(9728, 2560), (2560, 9728)])
-def test_gemm_nvfp4_4b_mlp_shapes(lib, N, K):
-    err = run_case(lib, 32, N, K, seed=7)
+@pytest.mark.parametrize("T", [32, 64])
+def test_gemm_nvfp4_4b_mlp_shapes(lib, N, K, T):
+    err = run_case(lib, T, N, K, seed=7 + T)
     print("nvfp4 %dx%d rel err %.2e" % (N, K, err))
 
 
@@ -83,7 +84,7 @@ def test_gemm_nvfp4_rejects_bad_shapes(lib):
         lib.gemm_nvfp4(torch.zeros((4, 320), device="cuda"), q)  # K % 256 != 0
     q2 = to_device_q(oracle_q(gen.bf16_bits(gen.normal_np(6, 128 * 256, 0.02).reshape(128, 256))))
     with pytest.raises(DlmError):
-        lib.gemm_nvfp4(torch.zeros((33, 256), device="cuda"), q2)  # T > 32
+        lib.gemm_nvfp4(torch.zeros((65, 256), device="cuda"), q2)  # T > 64
 
 
 # ------------------------------------------------------------------ fused NVFP4 LM head
