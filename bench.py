@@ -946,6 +946,7 @@ def main():
             "roofline": {"bound": "hbm", "kernel": "k_gemm_tc: 9728x2560 bf16 weight GEMM, 32 tokens as a split "
                                                      "bf16 pair (the gate projection), partial sums",
                          "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "frac_nominal": achieved / NOMINAL_HBM_GBS,
                          "peak_kind": peak_kind, "traffic": profile_traffic("k_gemm_tc_9728x2560_t32.md"),
                          "algorithmic_bytes": gate_bytes, "launch_us": gate_s * 1e6},
             "cpu_baseline": cpu,
