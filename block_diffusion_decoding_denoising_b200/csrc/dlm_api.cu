@@ -225,13 +225,15 @@ size_t carve(dlm_ctx* x, const dlm_config& c, uint8_t* base) {
   uint8_t* xscales = fp4 ? cv.take<uint8_t>(f4_scale_bytes(kmax)) : nullptr;
   float* sx = fp4 ? cv.take<float>(kMaxF4Tokens) : nullptr;
   float* aam = fp4 ? cv.take<float>((size_t)((c.ffn + 63) / 64) * Tmax) : nullptr;
-  __nv_bfloat16* edq = fp4 ? cv.take<__nv_bfloat16>((size_t)c.vocab * c.d) : nullptr;
   const bool fp4_shapes = fp4 && c.d % 256 == 0 && c.ffn % 256 == 0;
+  const bool fused = fp4 ? fp4_shapes && lmhead_fused_f4_supported(B, c.d) : lmhead_fused_supported(B, c.d);
+  // a bf16 copy of the NVFP4 E (q sigma) only for the unfused LM head's P E; the fused one and
+  // the embedding rows read the codes
+  __nv_bfloat16* edq = (fp4 && !fused) ? cv.take<__nv_bfloat16>((size_t)c.vocab * c.d) : nullptr;
   const size_t sfp = fp4_shapes ? align256(nvf4_sf_tile_bytes(c.ffn, c.d, A_PAIR)) : 0;
   const size_t sfd = fp4_shapes ? align256(nvf4_sf_tile_bytes(c.d, c.ffn, A_KMAJOR)) : 0;
   const size_t sfe = fp4_shapes ? align256(nvf4_sf_tile_bytes(c.vocab, c.d, A_KMAJOR)) : 0;
   uint8_t* sf = fp4_shapes ? cv.take<uint8_t>((size_t)c.n_layers * (sfp + sfd) + sfe) : nullptr;
-  const bool fused = fp4 ? fp4_shapes && lmhead_fused_f4_supported(B, c.d) : lmhead_fused_supported(B, c.d);
   uint8_t* lmf = fused ? cv.take<uint8_t>(lmhead_fused_scratch_bytes(c.vocab, c.d)) : nullptr;
   if (x && base) {
     x->lmf = lmf;
@@ -385,7 +387,12 @@ dlm_status resid_norm(Runner& r, int T, const GemmOut* y, const int32_t* embed_t
   if (y) a.out = *y;
   a.out.T = T;
   a.h = ctx->h;
-  a.embed = embed_tokens ? (ctx->fp4 ? ctx->e_deq : (const __nv_bfloat16*)ctx->w.embed) : nullptr;
+  if (embed_tokens && ctx->fp4 && !ctx->e_deq) {  // NVFP4 E read as codes (no bf16 copy kept)
+    a.embed_codes = (const uint8_t*)ctx->w.q_embed.codes;
+    a.embed_sc = (const uint8_t*)ctx->w.q_embed.scales;
+  } else {
+    a.embed = embed_tokens ? (ctx->fp4 ? ctx->e_deq : (const __nv_bfloat16*)ctx->w.embed) : nullptr;
+  }
   a.tokens = embed_tokens;
   a.tokens2 = embed_tokens2;
   a.tok_split = tok_split;
@@ -868,9 +875,9 @@ dlm_status dlm_ctx_create(const dlm_config* cfg, const dlm_weights* w, void* d_w
                                                                           cfg->head_dim, (double)cfg->rope_theta);
     e = cudaGetLastError();
   }
-  if (e == cudaSuccess && fp4) {
-    // E for the embedding rows and P E: q sigma in bf16 (exact); the tensor scale is applied
-    // where they are used
+  if (e == cudaSuccess && fp4 && ctx->e_deq) {
+    // E for the embedding rows and P E of the unfused LM head: q sigma in bf16 (exact); the
+    // tensor scale is applied where they are used
     const long nb = (long)cfg->vocab * (cfg->d / 16);
     k_nvfp4_dequant_bf16<<<(unsigned)((nb + 255) / 256), 256, 0, ctx->cap_stream>>>(
         (const uint8_t*)w->q_embed.codes, (const uint8_t*)w->q_embed.scales, nb, ctx->e_deq);

@@ -355,7 +355,8 @@ __global__ void __launch_bounds__(kRnThreads) k_resid_norm(ResNormArgs a) {
   const int tile0 = f0 >> 7, ntl = ((f0 + dq - 1) >> 7) - tile0 + 1;  // tiles of this CTA's features
   if (has_y && (int)threadIdx.x < ntl) nsl[threadIdx.x] = tile_slots(o, tile0 + threadIdx.x);
   __syncthreads();
-  const int tok = !a.embed ? 0 : ((a.tokens2 && t >= a.tok_split) ? a.tokens2[t - a.tok_split] : a.tokens[t]);
+  const bool emb = a.embed || a.embed_codes;
+  const int tok = !emb ? 0 : ((a.tokens2 && t >= a.tok_split) ? a.tokens2[t - a.tok_split] : a.tokens[t]);
   float base[kFeat], x[kFeat][kSlotsReg];
   int ns[kFeat];
   const float* pp[kFeat];
@@ -365,7 +366,15 @@ __global__ void __launch_bounds__(kRnThreads) k_resid_norm(ResNormArgs a) {
     const bool ok = (int)threadIdx.x + k * kRnThreads < dq;
     ns[k] = (ok && has_y) ? nsl[(n >> 7) - tile0] : 0;
     pp[k] = has_y ? o.partial + ((size_t)(n >> 7) * o.max_slots * TP + t) * kTileM + (n & 127) : nullptr;
-    base[k] = !ok ? 0.f : (a.embed ? bf2f(a.embed[(size_t)tok * a.d + n]) * a.embed_scale : a.h[(size_t)t * a.d + n]);
+    if (!ok) {
+      base[k] = 0.f;
+    } else if (a.embed_codes) {  // NVFP4 E: code x e4m3 scale (exact in fp32), times the tensor scale
+      const uint8_t cb = a.embed_codes[(size_t)tok * (a.d / 2) + n / 2];
+      base[k] = e2m1_value_dev((n & 1) ? (uint8_t)(cb >> 4) : (uint8_t)(cb & 15)) *
+                e4m3_value_dev(a.embed_sc[(size_t)tok * (a.d / 16) + n / 16]) * a.embed_scale;
+    } else {
+      base[k] = a.embed ? bf2f(a.embed[(size_t)tok * a.d + n]) * a.embed_scale : a.h[(size_t)t * a.d + n];
+    }
 #pragma unroll
     for (int sl = 0; sl < kSlotsReg; ++sl) x[k][sl] = sl < ns[k] ? __ldcg(pp[k] + sl * st) : 0.f;
   }

@@ -20,6 +20,8 @@ struct ResNormArgs {
   GemmOut out;                 // partial sums of a GEMM with N = d (partial == nullptr: y = 0)
   float* h;                    // [T][d] residual stream
   const __nv_bfloat16* embed;  // non-null: h = E[tokens] + y instead of h += y
+  const uint8_t* embed_codes;  // or, for an NVFP4 E: its codes [V][d/2] and scales [V][d/16]
+  const uint8_t* embed_sc;     //   (the rows dequantized here, q sigma, times embed_scale)
   const int32_t* tokens;       // token of row t < tok_split (all rows when tokens2 is null)
   const int32_t* tokens2;      // token of row t >= tok_split: tokens2[t - tok_split]
   int tok_split;

@@ -47,6 +47,19 @@ def test_workspace_and_kv_sizes(L):
     assert 0 < L.dlm_workspace_size(C.byref(tiny)) < ws
 
 
+def test_nvfp4_workspace_keeps_no_bf16_copy_of_e(L):
+    # With the fused NVFP4 LM head (B <= 32) the embedding rows and P E read E's codes, so the
+    # workspace holds no bf16 copy of E; the unfused head (B = 33) needs one (V x d x 2 bytes).
+    def ws(B):
+        c = gen.config_4b()
+        c["weight_fmt"], c["block_size"] = dlm.WEIGHTS_NVFP4, B
+        return L.dlm_workspace_size(C.byref(dlm.Config.from_dict(c)))
+    c = gen.config_4b()
+    e_bf16 = c["vocab"] * c["d"] * 2
+    assert ws(32) < e_bf16 // 2
+    assert ws(33) - ws(32) > 0.9 * e_bf16
+
+
 @pytest.mark.parametrize("field,value", [("d", 65), ("n_kv_heads", 3), ("head_dim", 48), ("block_size", 0),
                                          ("block_size", 65), ("mask_id", 512), ("vocab", 510), ("weight_fmt", 2),
                                          ("rms_eps", 0.0)])
