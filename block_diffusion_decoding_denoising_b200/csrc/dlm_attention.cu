@@ -13,7 +13,10 @@
 // blocks still spread the KV stream over the SMs, and a combine kernel merges the splits
 // with their (max, sum) statistics.  S = Q K^T and O = P V run on the tensor cores
 // (mma.sync m16n8k16 bf16, fp32 accumulate); softmax is online in fp32 (base-2 exponent).
+// The bf16 K/V tiles are staged by TMA (cp.async.bulk.tensor, 64 keys x 64 features per box,
+// 128-byte swizzle; 64-byte for head_dim 32) into a double buffer completed on mbarriers.
 #include <cstdio>
+#include <cstring>
 
 #include "dlm_device.cuh"
 #include "dlm_internal.h"
@@ -24,13 +27,17 @@ constexpr int kAttnRows = 64;   // query rows per CTA
 constexpr int kAttnKeys = 64;   // keys per tile
 constexpr int kMinKeysPerSplit = 128;
 
+constexpr int kKvStages = 3;  // bf16 cache: K/V ring depth (TMA)
+
 template <int HD, bool FP8 = false>
 struct AttnSmem {
   static constexpr int kTileBytes = 64 * HD * 2;
-  // bf16 cache: Q + K, V double-buffered.  FP8 cache: Q + one bf16 K, V tile + the raw e4m3
-  // K, V tiles and their 64 + 64 row scales double-buffered
+  // bf16 cache: a ring of kKvStages (K, V) tile pairs (Q goes to registers from global memory).
+  // FP8 cache: Q + one bf16 K, V tile + the raw e4m3 K, V tiles and their 64 + 64 row scales
+  // double-buffered
   static constexpr int kRawBytes = 2 * 64 * HD + 2 * 64 * 4;
-  static constexpr int kBytes = FP8 ? kTileBytes + 2 * kTileBytes + 2 * kRawBytes : kTileBytes + 4 * kTileBytes;
+  // + 1024: the tiles start on a 1024-byte boundary (the TMA swizzle atom)
+  static constexpr int kBytes = (FP8 ? kTileBytes + 2 * kTileBytes + 2 * kRawBytes : 2 * kKvStages * kTileBytes) + 1024;
 };
 
 // Two e4m3 codes (low byte first) -> their values as a bf16 pair, exactly (e4m3 values are
@@ -43,17 +50,19 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// 16-byte chunk swizzle inside a [64][HD] bf16 tile (row stride HD*2 bytes) that keeps
-// ldmatrix reads of 8 consecutive rows free of bank conflicts.
+// Byte offset of 16-byte chunk `ch` (8 features) of row `row` in a [64][HD] bf16 tile, laid out
+// as the TMA writes a box with the 128-byte swizzle (HD >= 64: rows of 128 B, HD = 128 as two
+// [64][64] halves one after the other) or the 64-byte swizzle (HD = 32: rows of 64 B).  The
+// swizzle spreads the 8 rows of an ldmatrix read over all banks.
 template <int HD>
-__device__ __forceinline__ int swz(int row, int chunk) {
-  if constexpr (HD >= 64) return chunk ^ (row & 7);
-  else return chunk ^ ((row >> 1) & 3);
+__device__ __forceinline__ uint32_t chunk_off(int row, int ch) {
+  if constexpr (HD >= 64) return (uint32_t)((ch >> 3) * 8192 + row * 128 + (((ch & 7) ^ (row & 7)) << 4));
+  else return (uint32_t)(row * 64 + (((ch & 3) ^ ((row >> 1) & 3)) << 4));
 }
 template <int HD>
 __device__ __forceinline__ uint32_t tile_addr(uint32_t base, int row, int col) {
   // col in elements, multiple of 8 for chunk-aligned accesses
-  return base + row * (HD * 2) + swz<HD>(row, col >> 3) * 16 + (col & 7) * 2;
+  return base + chunk_off<HD>(row, col >> 3) + (col & 7) * 2;
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -93,10 +102,16 @@ __host__ __device__ __forceinline__ int attn_splits(int nkeys, int max_splits) {
 }
 
 template <int HD, bool FP8>
-__global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
+__global__ void __launch_bounds__(128)
+k_bd_attention(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, AttnArgs a) {
   pdl_trigger();
-  pdl_wait();
-  extern __shared__ __align__(128) uint8_t sm[];
+  // bf16 cache: the prefix length (set between passes, never by a kernel of the pass) and the
+  // K/V rows of the prefix [0, L) (written by earlier passes) do not depend on the previous
+  // kernel, so the first prefix tiles are requested before waiting for it (below)
+  if constexpr (FP8) pdl_wait();
+  extern __shared__ uint8_t sm_raw[];
+  uint8_t* const sm = (uint8_t*)(((uintptr_t)sm_raw + 1023) & ~(uintptr_t)1023);  // swizzle atoms
+  __shared__ uint64_t kv_full[kKvStages];  // bf16 cache: the TMA K + V tiles of stage s have landed
   const int G = a.Hq / a.Hkv;
   const int rows_total = a.T * G;
   const int g = blockIdx.y, qt = blockIdx.x, split = blockIdx.z;
@@ -121,28 +136,30 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int gid = lane / 4, tig = lane % 4;
-  const uint32_t sQ = smem_u32(sm);
+  const uint32_t sQ = smem_u32(sm);  // FP8: the Q tile
   constexpr int TB = AttnSmem<HD>::kTileBytes;
-  // FP8: one bf16 K and V tile (index 0) converted from raw[buf] each step
-  const uint32_t sK[2] = {sQ + TB, sQ + (FP8 ? TB : 3 * TB)};
-  const uint32_t sV[2] = {sQ + 2 * TB, sQ + (FP8 ? 2 * TB : 4 * TB)};
+  // bf16: stage s holds K at 2 s TB and V at (2 s + 1) TB; FP8: one bf16 K and V tile (after
+  // the Q tile) converted from raw[buf] each step
+  uint32_t sK[kKvStages], sV[kKvStages];
+#pragma unroll
+  for (int st = 0; st < kKvStages; ++st) {
+    sK[st] = FP8 ? sQ + TB : sQ + 2 * st * TB;
+    sV[st] = FP8 ? sQ + 2 * TB : sQ + (2 * st + 1) * TB;
+  }
   uint8_t* const raw0 = sm + 3 * TB;  // FP8: [buf][K codes 64 x HD | V codes | K scales 64 | V scales 64]
   constexpr int RB = AttnSmem<HD, true>::kRawBytes;
   constexpr int CH = HD / 8;  // 16-byte chunks per row
 
-  // ---- Q tile: row r <-> (token t = r / G, head g*G + r % G)
-  for (int i = threadIdx.x; i < kAttnRows * CH; i += 128) {
-    int r = i / CH, ch = i % CH;
-    int R = row0 + r;
-    bool v = R < rows_total;
-    int t = v ? R / G : 0, h = g * G + (v ? R % G : 0);
-    const __nv_bfloat16* src = a.q + ((size_t)t * a.Hq + h) * HD + ch * 8;
-    cp_async16(sQ + r * (HD * 2) + swz<HD>(r, ch) * 16, src, v);
+  const int ntiles = (k1 > k0) ? (k1 - k0 + kAttnKeys - 1) / kAttnKeys : 0;
+  if constexpr (!FP8) {
+    if (threadIdx.x == 0) {
+      for (int st = 0; st < kKvStages; ++st) mbar_init(&kv_full[st], 1);
+      fence_mbar_init();
+      prefetch_tmap(&tk);
+      prefetch_tmap(&tv);
+    }
   }
-  cp_commit();
 
-  const __nv_bfloat16* kbase = a.kc + (size_t)g * a.max_ctx * HD;
-  const __nv_bfloat16* vbase = a.vc + (size_t)g * a.max_ctx * HD;
   auto load_kv = [&](int buf, int kt0) {
     if constexpr (FP8) {
       // raw e4m3 rows (HD bytes per key) and the 64 K / V row scales of the tile
@@ -170,17 +187,20 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
           for (int u = 0; u < 4; ++u) d[u] = (kt0 + ch * 4 + u < k1) ? sc[u] : 0.f;
         }
       }
+      cp_commit();
     } else {
-      for (int i = threadIdx.x; i < kAttnKeys * CH; i += 128) {
-        int r = i / CH, ch = i % CH;
-        int key = kt0 + r;
-        bool v = key < k1;
-        size_t off = (size_t)(v ? key : 0) * HD + ch * 8;
-        cp_async16(sK[buf] + r * (HD * 2) + swz<HD>(r, ch) * 16, kbase + off, v);
-        cp_async16(sV[buf] + r * (HD * 2) + swz<HD>(r, ch) * 16, vbase + off, v);
+      // one thread: the 64-key K and V boxes (rows g max_ctx + kt0 ..; rows past the cache's
+      // end read as zeros, rows past k1 are masked, and V's are zeroed before use)
+      if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(&kv_full[buf], 2 * TB);
+        const int y = g * a.max_ctx + kt0;
+#pragma unroll
+        for (int hh = 0; hh < (HD > 64 ? 2 : 1); ++hh) {
+          tma_load_2d(sm + (sK[buf] - sQ) + hh * 8192, &tk, &kv_full[buf], hh * 64, y);
+          tma_load_2d(sm + (sV[buf] - sQ) + hh * 8192, &tv, &kv_full[buf], hh * 64, y);
+        }
       }
     }
-    cp_commit();
   };
   // FP8: raw[buf] -> the bf16 K and V tiles, exactly (16 codes -> two 16-byte chunks)
   auto convert = [&](int buf) {
@@ -199,26 +219,68 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
       }
       const uint32_t base = which ? sV[0] : sK[0];
       const int c0 = ch * 2;  // 8-element (16-byte) chunk index of the first 8 values
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + r * (HD * 2) + swz<HD>(r, c0) * 16),
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + chunk_off<HD>(r, c0)),
                    "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]) : "memory");
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + r * (HD * 2) + swz<HD>(r, c0 + 1) * 16),
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + chunk_off<HD>(r, c0 + 1)),
                    "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7]) : "memory");
     }
   };
 
-  const int ntiles = (k1 > k0) ? (k1 - k0 + kAttnKeys - 1) / kAttnKeys : 0;
-  if (ntiles > 0) load_kv(0, k0);
+  // bf16: thread 0 requests the first kKvStages tiles; those that lie wholly in the prefix go
+  // out before waiting for the previous kernel (its mbarrier init precedes them in the thread)
+  int issued = 0;
+  if constexpr (!FP8) {
+    if (threadIdx.x == 0)
+      while (issued < kKvStages && issued < ntiles && k0 + (issued + 1) * kAttnKeys <= L) {
+        load_kv(issued, k0 + issued * kAttnKeys);
+        ++issued;
+      }
+    pdl_wait();
+    if (threadIdx.x == 0)
+      for (; issued < kKvStages && issued < ntiles; ++issued) load_kv(issued, k0 + issued * kAttnKeys);
+  }
 
-  // Q fragments for this warp's 16 rows
-  cp_wait<1>();
-  if (ntiles == 0) cp_wait<0>();
-  __syncthreads();
+  // ---- Q: row r <-> (token t = r / G, head g*G + r % G); the A fragments of this warp's 16 rows
   uint32_t qf[HD / 16][4];
+  if constexpr (FP8) {
+    for (int i = threadIdx.x; i < kAttnRows * CH; i += 128) {
+      int r = i / CH, ch = i % CH;
+      int R = row0 + r;
+      bool v = R < rows_total;
+      int t = v ? R / G : 0, h = g * G + (v ? R % G : 0);
+      const __nv_bfloat16* src = a.q + ((size_t)t * a.Hq + h) * HD + ch * 8;
+      cp_async16(sQ + chunk_off<HD>(r, ch), src, v);
+    }
+    cp_commit();
+    if (ntiles > 0) load_kv(0, k0);
+    cp_wait<1>();
+    if (ntiles == 0) cp_wait<0>();
+    __syncthreads();
 #pragma unroll
-  for (int ks = 0; ks < HD / 16; ++ks) {
-    int r = warp * 16 + (lane % 16);
-    int col = ks * 16 + (lane / 16) * 8;
-    ldsm_x4(tile_addr<HD>(sQ, r, col), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+    for (int ks = 0; ks < HD / 16; ++ks) {
+      int r = warp * 16 + (lane % 16);
+      int col = ks * 16 + (lane / 16) * 8;
+      ldsm_x4(tile_addr<HD>(sQ, r, col), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+    }
+  } else {
+    // straight from global memory (L2): register j of k-step ks holds row gid (+ 8 for odd j),
+    // features ks 16 + 8 (j / 2) + 2 tig and the next one
+    const uint32_t* qrow[2];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int R = row0 + warp * 16 + gid + 8 * hf;
+      qrow[hf] = R < rows_total
+                     ? reinterpret_cast<const uint32_t*>(a.q + ((size_t)(R / G) * a.Hq + g * G + R % G) * HD)
+                     : nullptr;
+    }
+#pragma unroll
+    for (int ks = 0; ks < HD / 16; ++ks)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t* qr = qrow[j & 1];
+        qf[ks][j] = qr ? __ldcg(qr + (ks * 16 + (j >> 1) * 8 + 2 * tig) / 2) : 0u;
+      }
+    __syncthreads();  // the ring's mbarriers are initialised for every thread
   }
 
   // per-thread rows: gid and gid + 8 of the warp's 16
@@ -231,8 +293,12 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
 #pragma unroll
   for (int i = 0; i < HD / 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 
+  // a thread that gave up waiting for a tile waits no more (every thread still takes every
+  // barrier); thread 0, which issues the loads, then issues no more of them
+  bool timed_out = false;
+  int fail_it = -1;
   for (int it = 0; it < ntiles; ++it) {
-    const int buf = it & 1;
+    const int buf = FP8 ? (it & 1) : it % kKvStages;
     const int kt0 = k0 + it * kAttnKeys;
     const float* ksc = nullptr;
     const float* vsc = nullptr;
@@ -245,13 +311,26 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
       ksc = reinterpret_cast<const float*>(raw0 + buf * RB + 2 * kAttnKeys * HD);
       vsc = ksc + kAttnKeys;
     } else {
-      if (it + 1 < ntiles) {
-        load_kv(buf ^ 1, kt0 + kAttnKeys);
-        cp_wait<1>();
-      } else {
-        cp_wait<0>();
+      // the first kKvStages tiles went out in the prologue; tile it + kKvStages - 1 goes to the
+      // stage of tile it - 1, which the barrier at the end of the previous step released
+      const int nxt = it + kKvStages - 1;
+      if (it >= 1 && nxt < ntiles && !timed_out) load_kv(nxt % kKvStages, k0 + nxt * kAttnKeys);
+      if (!timed_out && !mbar_wait(&kv_full[buf], (uint32_t)(it / kKvStages) & 1u, a.err)) {
+        timed_out = true;
+        fail_it = it;
       }
-      __syncthreads();
+      if (kt0 + kAttnKeys > k1) {
+        // the tile's rows past k1 hold other positions or heads (any bits): P is 0 there, so V
+        // must be finite; zero those rows (generic writes after the TMA's, ordered by the wait)
+        const int r0 = k1 - kt0;
+        for (int i = threadIdx.x; i < (kAttnKeys - r0) * CH; i += 128) {
+          const int r = r0 + i / CH, ch = i % CH;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(sV[buf] + chunk_off<HD>(r, ch)), "r"(0u)
+                       : "memory");
+        }
+        fence_async_shared();  // before any later TMA write of this buffer
+        __syncthreads();
+      }
     }
     const int kb = FP8 ? 0 : buf;  // bf16 tile of this step
 
@@ -367,6 +446,13 @@ __global__ void __launch_bounds__(128) k_bd_attention(AttnArgs a) {
       }
     }
     __syncthreads();  // buffer `buf` is refilled two iterations later
+  }
+  if constexpr (!FP8) {
+    // after a timeout no TMA may still be writing this CTA's shared memory when it leaves:
+    // thread 0 had issued tiles up to fail_it + kKvStages - 1 at most
+    if (threadIdx.x == 0 && fail_it >= 0)
+      for (int j = fail_it; j < ntiles && j < fail_it + kKvStages; ++j)
+        mbar_wait(&kv_full[j % kKvStages], (uint32_t)(j / kKvStages) & 1u, a.err);
   }
 
   // row sums across the quad
@@ -515,8 +601,22 @@ template <int HD>
 static cudaError_t launch_hd(const AttnArgs& a, cudaStream_t s) {
   const int G = a.Hq / a.Hkv;
   dim3 grid((a.T * G + kAttnRows - 1) / kAttnRows, a.Hkv, a.max_splits);
-  cudaError_t e = a.ks ? launch_k(k_bd_attention<HD, true>, grid, dim3(128), AttnSmem<HD, true>::kBytes, s, a)
-                       : launch_k(k_bd_attention<HD, false>, grid, dim3(128), AttnSmem<HD, false>::kBytes, s, a);
+  // bf16 cache: K and V of the layer as [Hkv * max_ctx][HD] for the TMA (boxes of 64 keys x
+  // min(HD, 64) features); the FP8 cache is staged by cp.async (the maps are not used)
+  CUtensorMap tk, tv;
+  memset(&tk, 0, sizeof(tk));
+  memset(&tv, 0, sizeof(tv));
+  if (!a.ks) {
+    char msg[160];
+    const uint64_t rows = (uint64_t)a.Hkv * a.max_ctx;
+    const uint32_t bi = HD < 64 ? HD : 64;
+    const int sw = HD < 64 ? 64 : 128;
+    if (!encode_tmap_2d_swizzle(&tk, a.kc, HD, rows, HD * 2, bi, kAttnKeys, sw, msg, sizeof(msg)) ||
+        !encode_tmap_2d_swizzle(&tv, a.vc, HD, rows, HD * 2, bi, kAttnKeys, sw, msg, sizeof(msg)))
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = a.ks ? launch_k(k_bd_attention<HD, true>, grid, dim3(128), AttnSmem<HD, true>::kBytes, s, tk, tv, a)
+                       : launch_k(k_bd_attention<HD, false>, grid, dim3(128), AttnSmem<HD, false>::kBytes, s, tk, tv, a);
   if (e != cudaSuccess) return e;
   if (a.max_splits > 1) e = launch_k(k_attn_combine, dim3(a.Hkv * a.T * G), dim3(128), 0, s, a);
   return e;

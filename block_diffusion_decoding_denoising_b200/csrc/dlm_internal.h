@@ -149,6 +149,9 @@ struct GemmPlan {
 // host helpers (dlm_gemm.cu)
 bool encode_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, char* err, size_t errlen);
+// The same with a 128-, 64- or 0-byte swizzle (bf16 elements, L2 promotion 256 B).
+bool encode_tmap_2d_swizzle(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                            uint32_t box_inner, uint32_t box_outer, int swizzle_bytes, char* err, size_t errlen);
 size_t gemm_partial_bytes(int T, int N, int K, int a_mode);
 // Plans y = x W^T.  `a0` is W (or Wg for A_PAIR, E for A_MNMAJOR), `a1` Wu for A_PAIR.
 // split: x holds high halves in rows [0, T) and low halves in rows [pad, pad + T),
