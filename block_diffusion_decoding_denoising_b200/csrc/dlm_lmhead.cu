@@ -496,19 +496,17 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
 // Merge of the clusters: for token t, M = max_c r_c, Z = sum_c Z_c e^(r_c - M), lse = M + ln Z,
 // maxprob = e^(max - lse), entropy = lse - A / Z, argmax from the lowest-index cluster holding
 // the max; s[t][f] = sum_c e^(r_c - M) s_c[f][t] / Z (given P: plain sum).
-// grid: d / 32 CTAs of 512 threads (16 warps x 32 features).  The per-token values are reduced
-// in two steps (16 cluster chunks, then the chunks in order); the s sums over the warps (each
-// a fixed set of clusters, the next cluster's 128 bytes loaded while the current one is
-// accumulated), then the warps in order.
+// grid: d / 16 CTAs of 512 threads.  The per-token values are reduced in two steps (16 cluster
+// chunks, then the chunks in order); then each warp takes one feature f (lane = token) and sums
+// its clusters in order, 128 contiguous bytes per cluster, eight clusters' loads in flight.
 constexpr int kLmfWarps = 16;
-constexpr int kLmfSmem = (kLmMaxClusters * 32 + kLmfWarps * 32 * 33 + 4 * kLmfWarps * 32) * 4;
+constexpr int kLmfSmem = (kLmMaxClusters * 32 + 4 * kLmfWarps * 32) * 4;
 __global__ void __launch_bounds__(kLmfWarps * 32) k_lmf_combine(LmfArgs a, dlm_row_stats stats, float* s) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ __align__(16) float sm_f[];
-  float(*w)[32] = reinterpret_cast<float(*)[32]>(sm_f);                         // [clusters][32]
-  float(*red)[32][33] = reinterpret_cast<float(*)[32][33]>(sm_f + kLmMaxClusters * 32);  // [warps][32][33]
-  float* cm = sm_f + kLmMaxClusters * 32 + kLmfWarps * 32 * 33;                 // [4][warps][32]
+  float(*w)[32] = reinterpret_cast<float(*)[32]>(sm_f);  // [clusters][32]
+  float* cm = sm_f + kLmMaxClusters * 32;                 // [4][warps][32]
   __shared__ float Mt[32], iZ[32];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   // 1. per token: thread (chunk = warp, token = lane) takes clusters chunk, chunk + 16, ...
@@ -572,47 +570,22 @@ __global__ void __launch_bounds__(kLmfWarps * 32) k_lmf_combine(LmfArgs a, dlm_r
     }
   }
   __syncthreads();
-  // 2. s: lane = feature blockIdx.x * 32 + lane, warp = clusters warp, warp + 16, ...
-  const int f = blockIdx.x * 32 + lane;
-  float acc[32];
+  // 2. s[t][f] = iZ[t] sum_c w[c][t] s_c[f][t] for f = this CTA's 16 features, one per warp
+  const int f = blockIdx.x * kLmfWarps + warp;
+  if (f >= a.d) return;
+  const float* src = a.part_s + (size_t)f * 32 + lane;
+  const size_t cs = (size_t)a.d * 32;  // one cluster's s block
+  float acc = 0.f;
+  int c = 0;
+  for (; c + 8 <= a.n_clu; c += 8) {
+    float x[8];
 #pragma unroll
-  for (int t = 0; t < 32; ++t) acc[t] = 0.f;
-  float4 cur[8], nxt[8];
-  int c = warp;
-  if (c < a.n_clu) {
-    const float4* src = reinterpret_cast<const float4*>(a.part_s + ((size_t)c * a.d + f) * 32);
+    for (int u = 0; u < 8; ++u) x[u] = __ldcg(src + (size_t)(c + u) * cs);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) cur[u] = __ldcg(src + u);
+    for (int u = 0; u < 8; ++u) acc += w[c + u][lane] * x[u];  // clusters in order
   }
-  for (; c < a.n_clu; c += kLmfWarps) {
-    const int cn = c + kLmfWarps;
-    if (cn < a.n_clu) {
-      const float4* src = reinterpret_cast<const float4*>(a.part_s + ((size_t)cn * a.d + f) * 32);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) nxt[u] = __ldcg(src + u);
-    }
-    const float4* wc = reinterpret_cast<const float4*>(&w[c][0]);  // broadcast reads
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float4 wv = wc[u];
-      acc[4 * u] += wv.x * cur[u].x;
-      acc[4 * u + 1] += wv.y * cur[u].y;
-      acc[4 * u + 2] += wv.z * cur[u].z;
-      acc[4 * u + 3] += wv.w * cur[u].w;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) cur[u] = nxt[u];
-  }
-#pragma unroll
-  for (int t = 0; t < 32; ++t) red[warp][lane][t] = acc[t];
-  __syncthreads();
-  for (int i = tid; i < 32 * 32; i += blockDim.x) {
-    const int t = i / 32, fl = i % 32;
-    if (t >= a.T) continue;
-    float v = 0.f;
-    for (int wv = 0; wv < kLmfWarps; ++wv) v += red[wv][fl][t];  // warps in order
-    s[(size_t)t * a.d + blockIdx.x * 32 + fl] = v * iZ[t];
-  }
+  for (; c < a.n_clu; ++c) acc += w[c][lane] * __ldcg(src + (size_t)c * cs);
+  if (lane < a.T) s[(size_t)lane * a.d + f] = acc * iZ[lane];
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1147,7 +1120,7 @@ cudaError_t lmhead_fused_launch(const void* x2, int x2_rows, int hi_row, int lo_
   cfg.numAttrs = g_pdl ? 2 : 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, k_lmhead_fused, tek, tem, tx, tp, a);
   if (e != cudaSuccess) return e;
-  return launch_k(k_lmf_combine, dim3(d / 32), dim3(kLmfWarps * 32), kLmfSmem, st, a, stats, s);
+  return launch_k(k_lmf_combine, dim3((d + kLmfWarps - 1) / kLmfWarps), dim3(kLmfWarps * 32), kLmfSmem, st, a, stats, s);
 }
 
 bool lmhead_fused_f4_supported(int T, int d) {
@@ -1220,7 +1193,7 @@ cudaError_t lmhead_fused_f4_launch(const dlm_nvfp4_matrix& E, const uint8_t* sfe
   cfg.numAttrs = g_pdl ? 2 : 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, k_lmhead_fused_f4, tec, tep, tes, txc, sfe_tiled, xscales, a);
   if (e != cudaSuccess) return e;
-  return launch_k(k_lmf_combine, dim3(d / 32), dim3(kLmfWarps * 32), kLmfSmem, st, a, stats, s);
+  return launch_k(k_lmf_combine, dim3((d + kLmfWarps - 1) / kLmfWarps), dim3(kLmfWarps * 32), kLmfSmem, st, a, stats, s);
 }
 
 }  // namespace dlm
