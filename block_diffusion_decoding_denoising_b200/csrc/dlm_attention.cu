@@ -498,7 +498,7 @@ k_bd_attention(const __grid_constant__ CUtensorMap tk, const __grid_constant__ C
 __global__ void __launch_bounds__(128) k_attn_combine(AttnArgs a) {
   pdl_trigger();
   pdl_wait();
-  __shared__ float wsp[64];
+  __shared__ float wsp[64], wl[64];
   __shared__ float red[4];
   __shared__ float den_s;
   const int G = a.Hq / a.Hkv;
@@ -522,11 +522,14 @@ __global__ void __launch_bounds__(128) k_attn_combine(AttnArgs a) {
   __syncthreads();
   const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
   const float w = (tid < nsplit && ls > 0.f) ? exp2f(ms - M) : 0.f;
-  if (tid < 64) wsp[tid] = w;
+  if (tid < 64) {
+    wsp[tid] = w;
+    wl[tid] = w * ls;  // the split's (m, l) were loaded by this thread above
+  }
   __syncthreads();
   if (tid == 0) {
     float den = 0.f;
-    for (int sp = 0; sp < nsplit; ++sp) den += wsp[sp] * a.part_ml[((size_t)sp * Rows + row) * 2 + 1];  // split order
+    for (int sp = 0; sp < nsplit; ++sp) den += wl[sp];  // split order
     den_s = den;
   }
   __syncthreads();
