@@ -524,12 +524,12 @@ __global__ void __launch_bounds__(128) k_attn_combine(AttnArgs a) {
   const float w = (tid < nsplit && ls > 0.f) ? exp2f(ms - M) : 0.f;
   if (tid < 64) {
     wsp[tid] = w;
-    wl[tid] = w * ls;  // the split's (m, l) were loaded by this thread above
+    wl[tid] = ls;  // the split's (m, l) were loaded by this thread above
   }
   __syncthreads();
   if (tid == 0) {
     float den = 0.f;
-    for (int sp = 0; sp < nsplit; ++sp) den += wl[sp];  // split order
+    for (int sp = 0; sp < nsplit; ++sp) den = fmaf(wsp[sp], wl[sp], den);  // split order
     den_s = den;
   }
   __syncthreads();

@@ -498,7 +498,7 @@ k_lmhead_fused(const __grid_constant__ CUtensorMap tek, const __grid_constant__ 
 // the max; s[t][f] = sum_c e^(r_c - M) s_c[f][t] / Z (given P: plain sum).
 // grid: d / 16 CTAs of 512 threads.  The per-token values are reduced in two steps (16 cluster
 // chunks, then the chunks in order); then each warp takes one feature f (lane = token) and sums
-// its clusters in order, 128 contiguous bytes per cluster, eight clusters' loads in flight.
+// its clusters the same way (128 contiguous bytes per cluster).
 constexpr int kLmfWarps = 16;
 constexpr int kLmfSmem = (kLmMaxClusters * 32 + 4 * kLmfWarps * 32) * 4;
 __global__ void __launch_bounds__(kLmfWarps * 32) k_lmf_combine(LmfArgs a, dlm_row_stats stats, float* s) {
@@ -571,21 +571,35 @@ __global__ void __launch_bounds__(kLmfWarps * 32) k_lmf_combine(LmfArgs a, dlm_r
   }
   __syncthreads();
   // 2. s[t][f] = iZ[t] sum_c w[c][t] s_c[f][t] for f = this CTA's 16 features, one per warp
+  //    (lane = token); the clusters are summed in 16 interleaved chunks (c = q, q + 16, ...)
+  //    whose sums are then added in chunk order, two chunks' loads in flight at a time
   const int f = blockIdx.x * kLmfWarps + warp;
   if (f >= a.d) return;
   const float* src = a.part_s + (size_t)f * 32 + lane;
   const size_t cs = (size_t)a.d * 32;  // one cluster's s block
-  float acc = 0.f;
-  int c = 0;
-  for (; c + 8 <= a.n_clu; c += 8) {
-    float x[8];
+  constexpr int kPer = (kLmMaxClusters + kLmfWarps - 1) / kLmfWarps;  // clusters per chunk
+  float v = 0.f;
+  for (int q = 0; q < kLmfWarps; q += 2) {
+    float x[2][kPer];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = __ldcg(src + (size_t)(c + u) * cs);
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int u = 0; u < 8; ++u) acc += w[c + u][lane] * x[u];  // clusters in order
+      for (int k = 0; k < kPer; ++k) {
+        const int c = q + h + k * kLmfWarps;
+        x[h][k] = c < a.n_clu ? __ldcg(src + (size_t)c * cs) : 0.f;
+      }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int c = q + h + k * kLmfWarps;
+        if (c < a.n_clu) acc = fmaf(w[c][lane], x[h][k], acc);
+      }
+      v += acc;
+    }
   }
-  for (; c < a.n_clu; ++c) acc += w[c][lane] * __ldcg(src + (size_t)c * cs);
-  if (lane < a.T) s[(size_t)lane * a.d + f] = acc * iZ[lane];
+  if (lane < a.T) s[(size_t)lane * a.d + f] = v * iZ[lane];
 }
 
 // ------------------------------------------------------------------------------------------
