@@ -687,7 +687,8 @@ def lmhead_case(args):
 def moe_case(args):
     """Routed-expert MLP sub-block with NVFP4 experts (dlm_moe_mlp_nvfp4) on a synthetic layer
     at the 4B-class width: d 2560, 64 experts of F 512, top-4, 32 rows, random router and
-    expert weights (quantized on the device), L2 flushed before every call.  Algorithmic
+    expert weights (quantized on the device), L2 flushed before every call, timed as a CUDA
+    graph of the call (and as eager calls, which add the host's work per call).  Algorithmic
     bytes: every expert's gate, up and down codes and scales (all are streamed) plus the
     router (bf16)."""
     import ctypes as C
@@ -710,7 +711,19 @@ def moe_case(args):
         fn()
     torch.cuda.synchronize()
     flush = _l2_flusher(dev)
-    t = _timed_calls(fn, max(args.steps, 5), flush)
+    t_eager = _timed_calls(fn, max(args.steps, 5), flush)
+    # the call's kernels replayed from a CUDA graph: device time without the host's per-call
+    # work (tensor-map encoding, eight launches) between them, as in a graph-launched decode
+    timing = "CUDA graph of one call"
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            fn()
+        torch.cuda.synchronize()
+        t = _timed_calls(graph.replay, max(args.steps, 5), flush)
+    except RuntimeError as e:  # capture refused: report the eager calls
+        timing = "eager calls (graph capture failed: %s)" % str(e).splitlines()[0][:80]
+        t = t_eager
     _, idx, _ = m(h)
     active = int(torch.unique(idx).numel())
     hbm, _, kind = peaks()
@@ -719,7 +732,8 @@ def moe_case(args):
     print(json.dumps({"case": "moe", "workload": "routed-expert MLP, NVFP4 experts: d %d, %d experts of F %d, top-%d, "
                       "%d rows" % (d, E, F, k, T), "us_per_call": t * 1e6, "algorithmic_bytes": nbytes,
                       "GBs": gbs, "frac": gbs / hbm, "peak": hbm, "peak_kind": kind, "experts_chosen": active,
-                      "l2": "flushed (256 MB written) before every call",
+                      "l2": "flushed (256 MB written) before every call", "timing": timing,
+                      "us_per_call_eager": t_eager * 1e6,
                       "note": "per call: routing, activation quantizers, two FP4 GEMMs and their finishers"}),
           flush=True)
 
