@@ -426,11 +426,16 @@ dlm_status act_quant(Runner& r, int T, const __nv_bfloat16* x, long lo, int K) {
   return DLM_OK;
 }
 
-// Finishes the tiles of a partial-sums GEMM with `epi` (one CTA per tile and 32 tokens).
+// Finishes the tiles of a partial-sums GEMM with `epi` (one CTA per tile and 32 tokens; the
+// plain store one CTA per tile and token).
 dlm_status finish_tiles(Runner& r, const GemmOut& y, int N, const EpiArgs& epi) {
   dlm_ctx* ctx = r.ctx;
   FinishArgs a{y, epi, N};
-  void (*k)(FinishArgs) = epi.op == EPI_QKV ? k_finish_qkv : (epi.op == EPI_SILU ? k_finish_silu : k_finish_store);
+  if (epi.op != EPI_QKV && epi.op != EPI_SILU) {  // one thread per feature and token
+    CU_LAUNCH(launch_k(k_finish_store, dim3(y.n_tiles, y.T), dim3(kTileM), 0, r.s, a));
+    return DLM_OK;
+  }
+  void (*k)(FinishArgs) = epi.op == EPI_QKV ? k_finish_qkv : k_finish_silu;
   CU_LAUNCH(launch_k(k, dim3(y.n_tiles, (y.T + 31) / 32), dim3(256), 0, r.s, a));
   return DLM_OK;
 }
@@ -1623,7 +1628,7 @@ dlm_status dlm_moe_mlp_nvfp4(const float* d_h_in, float* d_h_out, int T, int d, 
   eo.ld = d;
   eo.add = d_h_in;
   FinishArgs fo{p.out, eo, d};
-  CU_LAUNCH(launch_k(k_finish_store, dim3(p.out.n_tiles, (T + 31) / 32), dim3(256), 0, s, fo));
+  CU_LAUNCH(launch_k(k_finish_store, dim3(p.out.n_tiles, T), dim3(kTileM), 0, s, fo));
   return DLM_OK;
 }
 
@@ -1672,7 +1677,7 @@ dlm_status dlm_gemm_nvfp4(const float* d_x, const dlm_nvfp4_matrix* w, float* d_
     e.out = d_y;
     e.ld = N;
     FinishArgs fa{p.out, e, N};
-    CU_LAUNCH(launch_k(k_finish_store, dim3(p.out.n_tiles, (T + 31) / 32), dim3(256), 0, s, fa));
+    CU_LAUNCH(launch_k(k_finish_store, dim3(p.out.n_tiles, T), dim3(kTileM), 0, s, fa));
   }
   return DLM_OK;
 }

@@ -214,7 +214,6 @@ __global__ void __launch_bounds__(256) k_finish_silu(FinishArgs a) {
       if (t0 + j < a.out.T) e.act_amax[(size_t)tile * a.out.T + t0 + j] = fmaxf(am2[tg][j][0], am2[tg][j][1]);
 }
 
-// out[t][n] = scale * y (scale 0 means 1), rows r and r + 64 of the tile per thread.
 // Routed-expert MLP front, in two kernels.
 // k_moe_logits, grid (T, ceil(E / 8)): CTA (t, c) normalises row t, x = h / sqrt(mean(h^2) + eps)
 // g (fp32; CTA (t, 0) also stores it), and its 8 warps take the router logits of experts
@@ -306,25 +305,32 @@ __global__ void __launch_bounds__(256) k_moe_topk(MoeRouteArgs a) {
     }
 }
 
-__global__ void __launch_bounds__(256) k_finish_store(FinishArgs a) {
+// out[t][n] = scale * y (scale 0 means 1) (+ add[t][n]): one thread per feature n of the tile
+// and token t (grid: tiles x T, 128 threads), its slots summed in slot order, eight loads in
+// flight.
+__global__ void __launch_bounds__(128) k_finish_store(FinishArgs a) {
   pdl_trigger();
   pdl_wait();
   const EpiArgs& e = a.epi;
-  const int tile = blockIdx.x, r = threadIdx.x % 64, tg = threadIdx.x / 64;
-  const int t0 = blockIdx.y * 32 + tg * kFinTok;
-  if (t0 >= a.out.T) return;
-  float va[kFinTok], vb[kFinTok];
-  finish_load_pair(a.out, tile, r, r + 64, t0, va, vb);
-  const float sc = e.scale != 0.f ? e.scale : 1.f;
-  const int na = tile * kTileM + r, nb = na + 64;
+  const GemmOut& o = a.out;
+  const int tile = blockIdx.x, t = blockIdx.y, row = threadIdx.x;
+  const int n = tile * kTileM + row;
+  if (t >= o.T || n >= a.N) return;
+  const size_t TP = (size_t)(o.T + 31) / 32 * 32, ss = TP * kTileM;
+  const int ns = tile_slots(o, tile);
+  const float* p = o.partial + ((size_t)tile * o.max_slots * TP + t) * kTileM + row;
+  float v = 0.f;
+  int sl = 0;
+  for (; sl + 8 <= ns; sl += 8) {
+    float x[8];
 #pragma unroll
-  for (int j = 0; j < kFinTok; ++j) {
-    if (t0 + j < a.out.T) {
-      const size_t ia = (size_t)(t0 + j) * e.ld + na, ib = (size_t)(t0 + j) * e.ld + nb;
-      if (na < a.N) e.out[ia] = ((e.scale != 0.f) ? va[j] * sc : va[j]) + (e.add ? e.add[ia] : 0.f);
-      if (nb < a.N) e.out[ib] = ((e.scale != 0.f) ? vb[j] * sc : vb[j]) + (e.add ? e.add[ib] : 0.f);
-    }
+    for (int u = 0; u < 8; ++u) x[u] = __ldcg(p + (size_t)(sl + u) * ss);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v += x[u];
   }
+  for (; sl < ns; ++sl) v += __ldcg(p + (size_t)sl * ss);
+  const size_t i = (size_t)t * e.ld + n;
+  e.out[i] = ((e.scale != 0.f) ? v * e.scale : v) + (e.add ? e.add[i] : 0.f);
 }
 
 // Residual update and RMSNorm of one token row, spread over a cluster of kRnCluster CTAs:
