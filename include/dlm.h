@@ -110,7 +110,9 @@ typedef struct dlm_weights {
   const void* final_norm; /* bf16 [d] */
   const dlm_layer_weights* layers; /* host array [n_layers]; copied by dlm_ctx_create */
   dlm_nvfp4_matrix q_embed; /* NVFP4 E when weight_fmt == NVFP4: the LM head streams it; the
-                               embedding rows and P E use its dequantised values */
+                               embedding rows and P E use its dequantised values, read from the
+                               codes (the workspace holds a bf16 copy, V x d x 2 bytes, only
+                               where the LM head runs unfused: B > 32 or d % 512 != 0) */
 } dlm_weights;
 
 /* Per-row statistics of one round, device arrays of length B. */
